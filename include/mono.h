@@ -1,0 +1,205 @@
+/*
+ * mono.h -- C-ABI of the B200 (sm_100a) Monodratic mixer library.
+ *
+ * The library computes the forward pass of the stateless
+ * [batch, sequence, width] -> attention-delta mixer described on the
+ * aitechinspire.com Monodratic article ("Snapshot: key facts from the
+ * report"): Q/K/V projection with RoPE, learned product-hash routing of
+ * source blocks through bounded causal posting lists, exact causal softmax
+ * over the selected token set, and the output projection.  Normalisation,
+ * residuals and feed-forward layers stay with the host model.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - All tensors are contiguous and row-major.  Device pointers point to
+ *   global memory of the current CUDA device; `stream` is a cudaStream_t
+ *   (NULL = the legacy default stream).
+ * - Storage type: x, weights, Q, K, V, O and delta use cfg.dtype
+ *   (MONO_F32 = IEEE binary32, MONO_BF16 = bfloat16).  Codebooks and the
+ *   block summaries are always fp32; ids are int32.
+ * - Layouts:
+ *     x, delta        [B, S, W]
+ *     Wq, Wk, Wv      [H*d, W]   out_features x in_features: q = x Wq^T,
+ *                                head h owns rows h*d .. h*d+d-1
+ *     Wo              [W, H*d]   delta = O Wo^T
+ *     codebooks       [H, M, C, d/M] fp32
+ *     Q, K, V         [B, H, S, d]   (Q and K after RoPE)
+ *     sel             [B, H, S, R] int32, ascending block ids, -1 padding
+ *     O               [B, S, H*d]    head h in columns h*d .. h*d+d-1
+ *     forced          [B, H, S] int32 block id per query-head, -1 = none
+ * - Ownership: the caller allocates every device buffer, including the
+ *   workspace whose size mono_plan reports.  The library never allocates
+ *   device memory and keeps no state between calls; a plan is immutable
+ *   host data.
+ * - Every device pointer must be 16-byte aligned and the workspace
+ *   256-byte aligned (MONO_ERR_ALIGN otherwise).
+ * - Calls are asynchronous on `stream`.  Argument errors are reported by
+ *   the return code before anything is launched.  Errors that only the
+ *   device can see are recorded in a device error word in the workspace and
+ *   reported by mono_stats (MONO_ERR_DEVICE).  Nothing crosses the C
+ *   boundary by exception.
+ * - A call with B == 0 or S == 0 is valid and launches nothing.
+ */
+#ifndef MONO_H
+#define MONO_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MONO_VERSION 1
+
+enum mono_dtype { MONO_F32 = 0, MONO_BF16 = 1 };
+
+enum mono_status {
+    MONO_OK = 0,
+    MONO_ERR_INVALID = 1,     /* parameters violate the method's definition (e.g. S % Bs != 0, R > E, T > C^M) */
+    MONO_ERR_UNSUPPORTED = 2, /* valid, but outside what this build implements (e.g. d not in {64, 128}) */
+    MONO_ERR_NULL = 3,        /* a required pointer is NULL */
+    MONO_ERR_WORKSPACE = 4,   /* workspace pointer missing */
+    MONO_ERR_CUDA = 5,        /* a CUDA runtime call or kernel launch failed */
+    MONO_ERR_DEVICE = 6,      /* a kernel recorded an error in the device error word */
+    MONO_ERR_ALIGN = 7        /* a pointer is not suitably aligned */
+};
+
+/* Plan options (mono_config.flags). */
+enum mono_flags {
+    /* Run the plain query-major kernels (SIMT projections and attention)
+     * even where the tensor-core kernels apply.  Same results within the
+     * stated tolerances; used as the correctness baseline. */
+    MONO_FLAG_SIMPLE_KERNELS = 1
+};
+
+/* Shape and method parameters.  Symbols follow the pages' description:
+ * B batch, S sequence, W width, H heads, d head dim, Bs block size,
+ * L guaranteed local blocks, R remote blocks kept, E eligible candidates
+ * reranked, M subspaces, C codes per subspace (C^M product addresses),
+ * T probed addresses, cap posting-list capacity. */
+typedef struct mono_config {
+    int B, S, W, H, d;
+    int Bs, L, R, E, M, C, T, cap;
+    double rope_theta;
+    int dtype; /* enum mono_dtype */
+    int flags; /* enum mono_flags */
+} mono_config;
+
+typedef struct mono_plan_s mono_plan_t;
+
+/* Routing statistics of the last mono_route / mono_forward on a workspace
+ * (the quantities the pages ask to log: selected remote blocks per query
+ * and posting overflow counts). */
+typedef struct mono_stats {
+    int64_t overflow_total;    /* blocks dropped from full posting lists, all (b, h) */
+    int32_t overflow_max_bh;   /* largest per-(b, h) overflow */
+    int32_t device_error;      /* 0, or the first device error code recorded */
+    int64_t queries_lt_R;      /* query-heads that received fewer than R remote blocks */
+    int64_t remote_selected;   /* total remote blocks selected */
+    double mean_remote;        /* remote_selected / (B*H*S) */
+    int64_t forced_ignored;    /* forced ids that were not eligible */
+} mono_stats_t;
+
+/* Workspace regions that mono_workspace_region can locate (debug/export). */
+enum mono_ws_region {
+    MONO_WS_KBAR = 0,      /* [B,H,nb,d] fp32 block summaries */
+    MONO_WS_ADDR = 1,      /* [B,H,nb] int32 product address of each block */
+    MONO_WS_POST_IDS = 2,  /* [B,H,nb] int32 block ids sorted by (address, id) */
+    MONO_WS_POST_ADDR = 3, /* [B,H,nb] int32 address of each sorted entry */
+    MONO_WS_POST_RANK = 4, /* [B,H,nb] int32 position within its address; kept iff < cap */
+    MONO_WS_OVERFLOW = 5,  /* [B,H] int32 dropped blocks */
+    MONO_WS_Q = 6,         /* [B,H,S,d] dtype, used by mono_forward */
+    MONO_WS_K = 7,
+    MONO_WS_V = 8,
+    MONO_WS_SEL = 9,       /* [B,H,S,R] int32, used by mono_forward */
+    MONO_WS_O = 10,        /* [B,S,H*d] dtype, used by mono_forward */
+    MONO_WS_NREGIONS = 11
+};
+
+/* Validate `cfg` and build an immutable host-side plan.  Writes the
+ * workspace size in bytes the plan's calls need.  No device work.
+ * Returns MONO_OK, MONO_ERR_NULL, MONO_ERR_INVALID or MONO_ERR_UNSUPPORTED. */
+int mono_plan(const mono_config *cfg, mono_plan_t **plan, size_t *workspace_bytes);
+
+/* Free a plan (NULL is ignored). */
+void mono_plan_destroy(mono_plan_t *plan);
+
+/* Byte offset and size of a workspace region (see enum mono_ws_region). */
+int mono_workspace_region(const mono_plan_t *plan, int region, size_t *offset, size_t *bytes);
+
+/* Q/K/V projection + RoPE (aitechinspire.com article, Snapshot: after RoPE,
+ * source blocks are assigned to posting lists).  q = x Wq^T etc., no bias;
+ * RoPE rotates interleaved pairs (2i, 2i+1) of Q and K by t*theta^(-2i/d).
+ * Inputs x, Wq, Wk, Wv; outputs Q, K, V.  Uses the workspace for the
+ * rotation tables. */
+int mono_project(const mono_plan_t *plan, const void *x, const void *Wq, const void *Wk,
+                 const void *Wv, void *Q, void *K, void *V, void *workspace, void *stream);
+
+/* Learned product-hash routing ("Monodratic Routes Sparse Attention with
+ * Learned Product Hashes", Key Points; remio.ai article section on
+ * retrieval decisions): block summaries kbar (mean post-RoPE key), product
+ * address by per-subspace dot-product argmax, bounded causal posting lists
+ * (earliest cap blocks kept, the rest dropped and counted), per-query probe
+ * of the top-T product addresses, union of their lists filtered to blocks
+ * j <= t/Bs - L and capped at E, rerank by q.kbar keeping the top R.
+ * Integer decisions use fp32 with the fixed accumulation order of the
+ * specification, so results are deterministic.
+ * Inputs Q, K, codebooks; optional `forced` (NULL = none): an eligible
+ * forced block replaces the lowest-ranked selection (or is appended) so the
+ * count stays <= R.  Output sel.  Summaries, addresses, posting lists and
+ * overflow counts are left in the workspace (mono_workspace_region). */
+int mono_route(const mono_plan_t *plan, const void *Q, const void *K, const float *codebooks,
+               const int32_t *forced, int32_t *sel, void *workspace, void *stream);
+
+/* The three stages of mono_route, callable one at a time (same kernels,
+ * same results); each reads what the previous one left in the workspace.
+ *  - mono_route_summaries: block summaries kbar and product addresses (needs K).
+ *  - mono_route_lists:     bounded causal posting lists and overflow counts.
+ *  - mono_route_queries:   probe, union, causal filter, E cap, rerank -> sel
+ *                          (needs Q); also resets and fills the statistics.
+ * mono_route_summaries resets the device error word. */
+int mono_route_summaries(const mono_plan_t *plan, const void *K, const float *codebooks, void *workspace,
+                         void *stream);
+int mono_route_lists(const mono_plan_t *plan, void *workspace, void *stream);
+int mono_route_queries(const mono_plan_t *plan, const void *Q, const float *codebooks, const int32_t *forced,
+                       int32_t *sel, void *workspace, void *stream);
+
+/* Exact causal softmax over the selected token set (aitechinspire.com
+ * article, Snapshot): for query t of block bq, the tokens of the blocks in
+ * sel[t] plus the tokens s in [max(0, bq-L+1)*Bs, t], scale 1/sqrt(d),
+ * softmax in fp32 with fp32 accumulation.  Inputs Q, K, V, sel; output O.
+ * sel entries must be -1 or a block id <= t/Bs - L (out-of-range ids are
+ * skipped and recorded in the device error word). */
+int mono_attend(const mono_plan_t *plan, const void *Q, const void *K, const void *V,
+                const int32_t *sel, void *O, void *workspace, void *stream);
+
+/* Output projection delta = O Wo^T. */
+int mono_out_project(const mono_plan_t *plan, const void *O, const void *Wo, void *delta,
+                     void *workspace, void *stream);
+
+/* The whole mixer: mono_project, mono_route, mono_attend and
+ * mono_out_project on workspace-resident Q, K, V, sel and O. */
+int mono_forward(const mono_plan_t *plan, const void *x, const void *Wq, const void *Wk,
+                 const void *Wv, const void *Wo, const float *codebooks, const int32_t *forced,
+                 void *delta, void *workspace, void *stream);
+
+/* Synchronise `stream` and read the routing statistics and the device error
+ * word of the last mono_route / mono_forward on `workspace`.  Returns
+ * MONO_ERR_DEVICE if a kernel recorded an error. */
+int mono_stats(const mono_plan_t *plan, const void *workspace, void *stream, mono_stats_t *out);
+
+/* Static description of a status code. */
+const char *mono_strerror(int status);
+
+/* MONO_VERSION of the built library. */
+int mono_version(void);
+
+/* Number of CUDA kernels this library has launched in this process (all
+ * devices and streams).  Host-side counter; no device work. */
+unsigned long long mono_kernel_launches(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MONO_H */

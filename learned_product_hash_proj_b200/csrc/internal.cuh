@@ -1,0 +1,98 @@
+// internal.cuh -- plan, workspace layout and device helpers shared by the
+// kernels of the mixer library (not part of the public C-ABI).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "mono.h"
+
+namespace mono {
+
+constexpr int kMaxD = 128;
+constexpr int kMaxM = 8;
+constexpr int kMaxC = 64;
+constexpr int kMaxT = 32;
+constexpr int kMaxE = 32;
+constexpr int kMaxR = 16;
+constexpr int kMaxNb = 8192;
+constexpr int kRopeLo = 64;  // positions per low rotation table
+
+// Device error codes (first one recorded wins; see mono_stats).
+enum DevErr : unsigned {
+    kDevErrBadSel = 1,       // attention got a sel id outside [0, t/Bs - L]
+    kDevErrCandOverflow = 2, // probe candidate list exceeded its bound (never expected)
+    kDevErrTimeout = 3,      // a bounded wait ran out
+    kDevErrBadAddr = 4,      // an address outside [0, C^M)
+};
+
+// Counters at the start of the counter region (uint64 each).
+enum Counter { kCntQueriesLtR = 0, kCntRemoteSel = 1, kCntForcedIgnored = 2, kCntErr = 3, kCntN = 8 };
+
+enum Region {
+    kRegKbar = MONO_WS_KBAR,
+    kRegAddr = MONO_WS_ADDR,
+    kRegPostIds = MONO_WS_POST_IDS,
+    kRegPostAddr = MONO_WS_POST_ADDR,
+    kRegPostRank = MONO_WS_POST_RANK,
+    kRegOverflow = MONO_WS_OVERFLOW,
+    kRegQ = MONO_WS_Q,
+    kRegK = MONO_WS_K,
+    kRegV = MONO_WS_V,
+    kRegSel = MONO_WS_SEL,
+    kRegO = MONO_WS_O,
+    kRegCounters = MONO_WS_NREGIONS,
+    kRegRope,
+    kRegPairCount,   // [B,H,nb] int32 queries selecting each block (fast attention)
+    kRegPairStart,   // [B,H,nb+1] int32 exclusive scan of the counts
+    kRegPairFill,    // [B,H,nb] int32 fill cursors
+    kRegPairs,       // [B*H*S*R] int32 (t*R + r) grouped by block
+    kRegPartO,       // [B*H*S*R, d] bf16 remote partial outputs
+    kRegPartML,      // [B*H*S*R] float2 (max, sum) of remote partials
+    kRegN
+};
+
+struct Plan {
+    mono_config cfg;
+    int nb;        // S / Bs
+    long long A;   // C^M
+    int es;        // bytes per stored element (4 or 2)
+    bool fast;     // tensor-core kernels apply
+    size_t off[kRegN];
+    size_t bytes[kRegN];
+    size_t ws_bytes;
+};
+
+template <typename T> __device__ __forceinline__ float to_f(T v);
+template <> __device__ __forceinline__ float to_f<float>(float v) { return v; }
+template <> __device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 v) { return __bfloat162float(v); }
+
+template <typename T> __device__ __forceinline__ T from_f(float v);
+template <> __device__ __forceinline__ float from_f<float>(float v) { return v; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float v) { return __float2bfloat16_rn(v); }
+
+__device__ __forceinline__ void record_error(unsigned long long *counters, unsigned code) {
+    atomicCAS(&counters[kCntErr], 0ull, (unsigned long long)code);
+}
+
+inline char *ws_ptr(const Plan &p, void *ws, int region) { return (char *)ws + p.off[region]; }
+
+// Host-side count of kernel launches issued by this library (mono_kernel_launches).
+void count_launches(int n);
+
+// ---------------------------------------------------------------------------
+// kernel launchers (each returns cudaGetLastError() of its launch)
+// ---------------------------------------------------------------------------
+cudaError_t launch_rope_tables(const Plan &p, void *ws, cudaStream_t s);
+cudaError_t launch_project_simt(const Plan &p, const void *x, const void *Wq, const void *Wk, const void *Wv,
+                                void *Q, void *K, void *V, const void *ws, cudaStream_t s);
+cudaError_t launch_out_project_simt(const Plan &p, const void *O, const void *Wo, void *delta, cudaStream_t s);
+cudaError_t launch_summaries(const Plan &p, const void *K, const float *cb, void *ws, cudaStream_t s);
+cudaError_t launch_lists(const Plan &p, void *ws, cudaStream_t s);
+cudaError_t launch_queries(const Plan &p, const void *Q, const float *cb, const int32_t *forced, int32_t *sel,
+                           void *ws, cudaStream_t s);
+cudaError_t launch_attend_simt(const Plan &p, const void *Q, const void *K, const void *V, const int32_t *sel,
+                               void *O, void *ws, cudaStream_t s);
+
+}  // namespace mono

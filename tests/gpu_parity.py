@@ -1,0 +1,185 @@
+"""Stage-wise parity of the CUDA library against the oracle (helpers).
+
+Every stage of the GPU pass is checked against the oracle on the GPU's own
+stored inputs of that stage, so that rounding in one stage does not leak into
+the next one's comparison:
+
+* projection + RoPE : oracle fp64 on x, rounded once to the storage type
+* summaries, addresses, posting lists, overflow : bit-exact (fp32 decisions in
+  the order the specification fixes)
+* selected blocks   : bit-exact
+* attention         : oracle fp64 on the GPU's Q/K/V and sel
+* output projection : oracle fp64 on the GPU's O
+
+Tolerances: fp32 storage -> max abs error 1e-5; bf16 storage -> max abs error
+2e-2 x RMS of the reference.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle
+from learned_product_hash_proj_b200 import mono, synth
+
+TOL_F32_ABS = 1e-5
+TOL_BF16_REL_RMS = 2e-2
+
+
+def to_dev(a: np.ndarray, dtype: str, device="cuda") -> torch.Tensor:
+    t = torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32))
+    return (t.to(torch.bfloat16) if dtype == "bf16" else t).to(device).contiguous()
+
+
+def to_np(t: torch.Tensor) -> np.ndarray:
+    return t.detach().float().cpu().numpy() if t.dtype != torch.int32 else t.detach().cpu().numpy()
+
+
+def assert_close(got, ref, dtype: str, what: str):
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    err = np.abs(got - ref).max() if got.size else 0.0
+    if dtype == "f32":
+        assert err <= TOL_F32_ABS, f"{what}: max abs err {err:.3e} > {TOL_F32_ABS}"
+        return err
+    rms = float(np.sqrt(np.mean(ref * ref))) if ref.size else 0.0
+    assert err <= TOL_BF16_REL_RMS * rms, f"{what}: max abs err {err:.3e} > 2e-2 x RMS {rms:.3e}"
+    return err / max(rms, 1e-300)
+
+
+def sample_tokens(cfg, n: int, rng) -> np.ndarray:
+    """Flat token rows b*S + t: edges plus a uniform sample."""
+    total = cfg.B * cfg.S
+    edge = [0, cfg.S - 1, total - 1, cfg.Bs, cfg.Bs * cfg.L, min(total - 1, cfg.Bs * (cfg.L + 1) - 1)]
+    rows = np.unique(np.concatenate([np.array(edge), rng.integers(0, total, size=n)]))
+    return rows[(rows >= 0) & (rows < total)].astype(np.int64)
+
+
+def sample_queries(cfg, n: int, rng) -> np.ndarray:
+    """Flat query-heads (b*H + h)*S + t, sorted (the oracle rebuilds lists per (b, h))."""
+    total = cfg.B * cfg.H * cfg.S
+    edge = [0, cfg.S - 1, total - 1, cfg.Bs * cfg.L, cfg.Bs * (cfg.L + 1) - 1]
+    q = np.unique(np.concatenate([np.array(edge), rng.integers(0, total, size=n)]))
+    return np.sort(q[(q >= 0) & (q < total)]).astype(np.int64)
+
+
+class Run:
+    """Inputs of one workload on the device plus the GPU results of each stage."""
+
+    def __init__(self, cfg, seed=0, flags=0, forced_frac=None, inputs=None):
+        self.cfg = cfg
+        self.inp = inputs if inputs is not None else synth.make_inputs(cfg, seed)
+        self.forced = None if forced_frac is None else synth.make_forced(cfg, seed, forced_frac)
+        self.plan = mono.Plan(cfg, flags=flags)
+        dt = cfg.dtype
+        self.dev = {k: to_dev(v, dt) for k, v in self.inp.items() if k != "codebooks"}
+        self.dev["codebooks"] = torch.from_numpy(self.inp["codebooks"]).cuda().contiguous()
+        self.forced_dev = None if self.forced is None else torch.from_numpy(self.forced).cuda().contiguous()
+        self.ws = self.plan.workspace()
+        B, H, S, d, R, W = cfg.B, cfg.H, cfg.S, cfg.d, cfg.R, cfg.W
+        tdt = self.plan.dtype
+        self.Q = torch.empty((B, H, S, d), dtype=tdt, device="cuda")
+        self.K = torch.empty_like(self.Q)
+        self.V = torch.empty_like(self.Q)
+        self.sel = torch.empty((B, H, S, R), dtype=torch.int32, device="cuda")
+        self.O = torch.empty((B, S, H * d), dtype=tdt, device="cuda")
+        self.delta = torch.empty((B, S, W), dtype=tdt, device="cuda")
+
+    def run_stages(self):
+        d = self.dev
+        mono.project(self.plan, d["x"], d["Wq"], d["Wk"], d["Wv"], self.Q, self.K, self.V, self.ws)
+        mono.route(self.plan, self.Q, self.K, d["codebooks"], self.sel, self.ws, forced=self.forced_dev)
+        self.route_ws = {k: to_np(self.plan.region(self.ws, k)).copy()
+                         for k in ("kbar", "addr", "post_ids", "post_addr", "post_rank", "overflow")}
+        self.stats = mono.stats(self.plan, self.ws)
+        mono.attend(self.plan, self.Q, self.K, self.V, self.sel, self.O, self.ws)
+        mono.out_project(self.plan, self.O, d["Wo"], self.delta, self.ws)
+        torch.cuda.synchronize()
+        return self
+
+    def run_forward(self) -> torch.Tensor:
+        d = self.dev
+        out = torch.empty_like(self.delta)
+        ws = self.plan.workspace()
+        mono.forward(self.plan, d["x"], d["Wq"], d["Wk"], d["Wv"], d["Wo"], d["codebooks"], out, ws,
+                     forced=self.forced_dev)
+        torch.cuda.synchronize()
+        self.forward_stats = mono.stats(self.plan, ws)
+        return out
+
+
+def check_projection(run: Run, rows=None):
+    cfg = run.cfg
+    inp = run.inp
+    Q, K, V = oracle.project(cfg, inp["x"], inp["Wq"], inp["Wk"], inp["Wv"], rows=rows)
+    errs = []
+    for name, ref, got in (("Q", Q, run.Q), ("K", K, run.K), ("V", V, run.V)):
+        g = to_np(got)
+        if rows is not None:
+            b, t = rows // cfg.S, rows % cfg.S
+            g = g[b, :, t, :]                      # [n, H, d]
+        errs.append(assert_close(g, oracle.round_storage(ref, cfg.dtype), cfg.dtype, f"projection {name}"))
+    return max(errs)
+
+
+def check_routing(run: Run, qidx=None):
+    """Bit-exact summaries, addresses, posting lists, overflow and sel."""
+    cfg = run.cfg
+    Kg = to_np(run.K)
+    Qg = to_np(run.Q)
+    kbar, addr, amargin = oracle.summary_assign(cfg, Kg, run.inp["codebooks"])
+    ws = run.route_ws
+    np.testing.assert_array_equal(ws["kbar"].view(np.uint32), kbar.view(np.uint32), err_msg="kbar bits")
+    np.testing.assert_array_equal(ws["addr"], addr, err_msg="addresses")
+    ids, saddr, rank, ov = oracle.posting(cfg, addr)
+    np.testing.assert_array_equal(ws["post_ids"], ids, err_msg="posting ids")
+    np.testing.assert_array_equal(ws["post_addr"], saddr, err_msg="posting addresses")
+    np.testing.assert_array_equal(ws["post_rank"], rank, err_msg="posting ranks")
+    np.testing.assert_array_equal(ws["overflow"].astype(np.int64), ov, err_msg="overflow")
+    assert run.stats["overflow_total"] == int(ov.sum())
+    sel, ncand, pm, rm, ign = oracle.route_queries(cfg, Qg, kbar, run.inp["codebooks"], addr, forced=run.forced,
+                                                   qidx=qidx)
+    gsel = to_np(run.sel).reshape(cfg.B * cfg.H * cfg.S, cfg.R)
+    if qidx is None:
+        np.testing.assert_array_equal(gsel.reshape(sel.shape), sel, err_msg="sel")
+        n_valid = (sel >= 0).sum()
+        assert run.stats["remote_selected"] == int(n_valid)
+        assert run.stats["queries_lt_R"] == int(((sel >= 0).sum(axis=-1) < cfg.R).sum())
+        if run.forced is not None:
+            assert run.stats["forced_ignored"] == ign
+    else:
+        np.testing.assert_array_equal(gsel[qidx], sel, err_msg="sel (sampled queries)")
+    small = int((rm < 1e-4).sum())
+    n = cfg.B * cfg.H * cfg.S if qidx is None else len(qidx)
+    return dict(overflow=int(ov.sum()), queries=n, small_margin=small)
+
+
+def check_attention(run: Run, qidx=None):
+    cfg = run.cfg
+    Og = to_np(run.O)                                      # [B, S, H*d]
+    Oh = Og.reshape(cfg.B, cfg.S, cfg.H, cfg.d).transpose(0, 2, 1, 3)   # [B, H, S, d]
+    if qidx is None:
+        Qg, Kg, Vg = (to_np(a).astype(np.float64) for a in (run.Q, run.K, run.V))
+        ref = oracle.attend(cfg, Qg, Kg, Vg, to_np(run.sel))
+        return assert_close(Oh, ref, cfg.dtype, "attention")
+    # sampled: one (b, h) slice at a time keeps host memory small at full size
+    one = cfg.with_(B=1, H=1)
+    refs, gots = [], []
+    bh_of = qidx // cfg.S
+    for bh in np.unique(bh_of):
+        b, h = divmod(int(bh), cfg.H)
+        ts = (qidx[bh_of == bh] % cfg.S).astype(np.int64)
+        sl = [to_np(a[b:b + 1, h:h + 1]).astype(np.float64) for a in (run.Q, run.K, run.V)]
+        sel = to_np(run.sel[b:b + 1, h:h + 1])
+        refs.append(oracle.attend(one, *sl, sel, qidx=ts))
+        gots.append(Oh[b, h, ts])
+    return assert_close(np.concatenate(gots), np.concatenate(refs), cfg.dtype, "attention (sampled)")
+
+
+def check_out_projection(run: Run, rows=None):
+    cfg = run.cfg
+    Og = to_np(run.O).astype(np.float64)
+    ref = oracle.out_project(cfg, Og, run.inp["Wo"], rows=rows)
+    got = to_np(run.delta)
+    got = got.reshape(-1, cfg.W)[rows] if rows is not None else got
+    return assert_close(got, oracle.round_storage(ref, cfg.dtype), cfg.dtype, "output projection")
