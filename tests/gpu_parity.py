@@ -12,7 +12,8 @@ the next one's comparison:
 * output projection : oracle fp64 on the GPU's O
 
 Tolerances: fp32 storage -> max abs error 1e-5; bf16 storage -> max abs error
-2e-2 x RMS of the reference.
+2e-2 x RMS of the reference, on top of the bf16 storage rounding of each
+output element (at most 2^-8 of its magnitude).
 """
 from __future__ import annotations
 
@@ -35,16 +36,27 @@ def to_np(t: torch.Tensor) -> np.ndarray:
     return t.detach().float().cpu().numpy() if t.dtype != torch.int32 else t.detach().cpu().numpy()
 
 
+BF16_UNIT_ROUNDOFF = 2.0 ** -8   # storing a value in bf16 moves it by at most this fraction of itself
+
+
 def assert_close(got, ref, dtype: str, what: str):
+    """fp32: max |got - ref| <= 1e-5.  bf16: max (|got - ref| - 2^-8 |ref|) <= 2e-2 x RMS(ref).
+
+    `ref` is the unrounded fp64 reference.  A bf16 output carries up to half an
+    ulp (<= 2^-8 of its magnitude) of storage rounding that no kernel can avoid,
+    so that term is allowed on top of the 2e-2 x RMS computation tolerance.
+    """
     got = np.asarray(got, np.float64)
     ref = np.asarray(ref, np.float64)
-    err = np.abs(got - ref).max() if got.size else 0.0
     if dtype == "f32":
+        err = np.abs(got - ref).max() if got.size else 0.0
         assert err <= TOL_F32_ABS, f"{what}: max abs err {err:.3e} > {TOL_F32_ABS}"
         return err
     rms = float(np.sqrt(np.mean(ref * ref))) if ref.size else 0.0
-    assert err <= TOL_BF16_REL_RMS * rms, f"{what}: max abs err {err:.3e} > 2e-2 x RMS {rms:.3e}"
-    return err / max(rms, 1e-300)
+    excess = (np.abs(got - ref) - BF16_UNIT_ROUNDOFF * np.abs(ref)).max() if got.size else 0.0
+    assert excess <= TOL_BF16_REL_RMS * rms, \
+        f"{what}: max (|err| - 2^-8|ref|) {excess:.3e} > 2e-2 x RMS {rms:.3e}"
+    return excess / max(rms, 1e-300)
 
 
 def sample_tokens(cfg, n: int, rng) -> np.ndarray:
@@ -118,7 +130,7 @@ def check_projection(run: Run, rows=None):
         if rows is not None:
             b, t = rows // cfg.S, rows % cfg.S
             g = g[b, :, t, :]                      # [n, H, d]
-        errs.append(assert_close(g, oracle.round_storage(ref, cfg.dtype), cfg.dtype, f"projection {name}"))
+        errs.append(assert_close(g, ref, cfg.dtype, f"projection {name}"))
     return max(errs)
 
 
@@ -182,4 +194,4 @@ def check_out_projection(run: Run, rows=None):
     ref = oracle.out_project(cfg, Og, run.inp["Wo"], rows=rows)
     got = to_np(run.delta)
     got = got.reshape(-1, cfg.W)[rows] if rows is not None else got
-    return assert_close(got, oracle.round_storage(ref, cfg.dtype), cfg.dtype, "output projection")
+    return assert_close(got, ref, cfg.dtype, "output projection")
