@@ -62,13 +62,15 @@ void layout(Plan *p) {
     bytes[kRegCounters] = kCntN * 8;
     const size_t nhi = (S + kRopeLo - 1) / kRopeLo;
     bytes[kRegRope] = (nhi + kRopeLo) * (d / 2) * 8;
-    if (p->fast) {
+    if (p->fast && R > 0) {
         bytes[kRegPairCount] = B * H * nb * 4;
-        bytes[kRegPairStart] = B * H * (nb + 1) * 4;
+        bytes[kRegPairStart] = B * H * nb * 4;
         bytes[kRegPairFill] = B * H * nb * 4;
         bytes[kRegPairs] = B * H * S * R * 4;
         bytes[kRegPartO] = B * H * S * R * d * 2;
         bytes[kRegPartML] = B * H * S * R * 8;
+        bytes[kRegWork] = (size_t)p->max_work * 8;
+        bytes[kRegNWork] = 4;
     }
     size_t off = 0;
     for (int r = 0; r < kRegN; ++r) {
@@ -137,7 +139,13 @@ int mono_plan(const mono_config *cfg, mono_plan_t **plan, size_t *workspace_byte
     p.A = 1;
     for (int m = 0; m < cfg->M; ++m) p.A *= cfg->C;
     p.es = cfg->dtype == MONO_BF16 ? 2 : 4;
-    p.fast = false;
+    p.fast = attend_tc_supported(*cfg) && !(cfg->flags & MONO_FLAG_SIMPLE_KERNELS);
+    {
+        const long long pairs = (long long)cfg->B * cfg->H * cfg->S * cfg->R;
+        const long long mw = (long long)cfg->B * cfg->H * p.nb + (pairs + 127) / 128;
+        if (p.fast && cfg->R > 0 && mw > (1ll << 31) - 1) { free(ps); return MONO_ERR_UNSUPPORTED; }
+        p.max_work = (int)(mw < (1ll << 31) - 1 ? mw : 0);
+    }
     layout(&p);
     *plan = ps;
     if (workspace_bytes) *workspace_bytes = p.ws_bytes;
@@ -218,7 +226,9 @@ int mono_attend(const mono_plan_t *plan, const void *Q, const void *K, const voi
     if (empty(&p)) return MONO_OK;
     if ((st = check_ptrs({Q, K, V, O}))) return st;
     if (p.cfg.R > 0 && (st = check_ptrs({sel}))) return st;
-    return cuda_status(launch_attend_simt(p, Q, K, V, sel, O, workspace, (cudaStream_t)stream));
+    cudaStream_t s = (cudaStream_t)stream;
+    if (p.fast) return cuda_status(launch_attend_tc(p, Q, K, V, sel, O, workspace, s));
+    return cuda_status(launch_attend_simt(p, Q, K, V, sel, O, workspace, s));
 }
 
 int mono_out_project(const mono_plan_t *plan, const void *O, const void *Wo, void *delta, void *workspace,

@@ -50,6 +50,8 @@ enum Region {
     kRegPairs,       // [B*H*S*R] int32 (t*R + r) grouped by block
     kRegPartO,       // [B*H*S*R, d] bf16 remote partial outputs
     kRegPartML,      // [B*H*S*R] float2 (max, sum) of remote partials
+    kRegWork,        // [max_work] int2 (bucket, chunk) work items of the remote kernel
+    kRegNWork,       // int32 number of work items
     kRegN
 };
 
@@ -58,7 +60,8 @@ struct Plan {
     int nb;        // S / Bs
     long long A;   // C^M
     int es;        // bytes per stored element (4 or 2)
-    bool fast;     // tensor-core kernels apply
+    bool fast;     // tensor-core attention applies
+    int max_work;  // upper bound on remote work items
     size_t off[kRegN];
     size_t bytes[kRegN];
     size_t ws_bytes;
@@ -94,5 +97,8 @@ cudaError_t launch_queries(const Plan &p, const void *Q, const float *cb, const 
                            void *ws, cudaStream_t s);
 cudaError_t launch_attend_simt(const Plan &p, const void *Q, const void *K, const void *V, const int32_t *sel,
                                void *O, void *ws, cudaStream_t s);
+bool attend_tc_supported(const mono_config &c);
+cudaError_t launch_attend_tc(const Plan &p, const void *Q, const void *K, const void *V, const int32_t *sel, void *O,
+                             void *ws, cudaStream_t s);
 
 }  // namespace mono

@@ -67,6 +67,178 @@ __global__ void __launch_bounds__(128) k_summary_assign(const T *__restrict__ K,
 }
 
 // ---------------------------------------------------------------------------
+// (A2, A3) the same summaries with one warp per block: each lane owns D/32
+// adjacent columns and walks the block's rows in ascending t, so every row
+// read is one coalesced 128/256-byte load.  A CTA takes 4 consecutive blocks
+// of one (b, h) and keeps that head's codebook in shared memory.
+// grid (ceil(nb/4), H, B), 128 threads.
+// ---------------------------------------------------------------------------
+template <typename T, int D>
+__global__ void __launch_bounds__(128) k_summary_assign_w(const T *__restrict__ K, const float *__restrict__ cb,
+                                                          float *__restrict__ kbar, int32_t *__restrict__ addr, int S,
+                                                          int Bs, int M, int C, int H) {
+    constexpr int PER = D / 32;  // columns per lane
+    extern __shared__ float sm[];
+    float *s_cb = sm;                         // [C*D]
+    float *s_kb = s_cb + C * D;               // [4][D]
+    float *s_sc = s_kb + 4 * D;               // [4][M*C]
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int h = blockIdx.y, b = blockIdx.z;
+    const int nb = S / Bs;
+    const size_t bh = (size_t)b * H + h;
+    for (int i = threadIdx.x; i < C * D; i += blockDim.x) s_cb[i] = cb[(size_t)h * C * D + i];
+    const int j = blockIdx.x * 4 + warp;
+    float acc[PER];
+#pragma unroll
+    for (int e = 0; e < PER; ++e) acc[e] = 0.0f;
+    if (j < nb) {
+        const T *Kb = K + (bh * S + (size_t)j * Bs) * D + lane * PER;
+#pragma unroll 8
+        for (int t = 0; t < Bs; ++t) {
+            float x[PER];
+            if constexpr (sizeof(T) == 2) {
+                if constexpr (PER == 2) {
+                    float2 f = __bfloat1622float2(*(const __nv_bfloat162 *)(Kb + (size_t)t * D));
+                    x[0] = f.x; x[1] = f.y;
+                } else {
+                    uint2 u = __ldg((const uint2 *)(Kb + (size_t)t * D));
+                    float2 f0 = __bfloat1622float2(*(const __nv_bfloat162 *)&u.x);
+                    float2 f1 = __bfloat1622float2(*(const __nv_bfloat162 *)&u.y);
+                    x[0] = f0.x; x[1] = f0.y; x[2] = f1.x; x[3] = f1.y;
+                }
+            } else {
+#pragma unroll
+                for (int e = 0; e < PER; ++e) x[e] = __ldg(Kb + (size_t)t * D + e);
+            }
+#pragma unroll
+            for (int e = 0; e < PER; ++e) acc[e] = __fadd_rn(acc[e], x[e]);
+        }
+#pragma unroll
+        for (int e = 0; e < PER; ++e) {
+            const float v = __fdiv_rn(acc[e], (float)Bs);
+            s_kb[warp * D + lane * PER + e] = v;
+            kbar[(bh * nb + j) * D + lane * PER + e] = v;
+        }
+    }
+    __syncthreads();
+    if (j >= nb) return;
+    const int dm = D / M;
+    for (int mc = lane; mc < M * C; mc += 32) {
+        const int m = mc / C;
+        const float *w = s_cb + mc * dm;
+        const float *kv = s_kb + warp * D + m * dm;
+        float a = 0.0f;
+        for (int i = 0; i < dm; ++i) a = __fmaf_rn(kv[i], w[i], a);
+        s_sc[warp * M * C + mc] = a;
+    }
+    __syncwarp();
+    if (lane == 0) {
+        long long ad = 0;
+        const float *sc = s_sc + warp * M * C;
+        for (int m = 0; m < M; ++m) {
+            float best = sc[m * C];
+            int bc = 0;
+            for (int c = 1; c < C; ++c)
+                if (sc[m * C + c] > best) { best = sc[m * C + c]; bc = c; }
+            ad = ad * C + bc;
+        }
+        addr[bh * nb + j] = (int32_t)ad;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// (A4) posting lists by counting, for address spaces that fit in shared
+// memory (C^M <= kDenseA).  One warp walks the blocks in ascending id, 32 at a
+// time: __match_any_sync groups equal addresses, so each block's rank among
+// the earlier blocks of its address is the running count plus its position
+// in the group.  A scan of the counts over the addresses then gives each
+// block its slot in the (address, id) order.  Deterministic, no atomics.
+// grid (H, B), 1024 threads.
+// ---------------------------------------------------------------------------
+constexpr int kDenseA = 4096;
+
+__global__ void __launch_bounds__(1024) k_posting_dense(const int32_t *__restrict__ addr, int32_t *__restrict__ ids,
+                                                        int32_t *__restrict__ saddr, int32_t *__restrict__ rank,
+                                                        int32_t *__restrict__ overflow, int nb, int cap, int H, int A) {
+    __shared__ int s_cnt[kDenseA];
+    __shared__ int s_part[32];
+    __shared__ int s_ov[32];
+    extern __shared__ int32_t s_dyn[];
+    int32_t *s_addr = s_dyn;          // [nb]
+    int32_t *s_rank = s_dyn + nb;     // [nb]
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const size_t bh = (size_t)blockIdx.y * H + blockIdx.x;
+    for (int a = tid; a < A; a += blockDim.x) s_cnt[a] = 0;
+    for (int j = tid; j < nb; j += blockDim.x) s_addr[j] = addr[bh * nb + j];
+    __syncthreads();
+    if (warp == 0) {
+        for (int j0 = 0; j0 < nb; j0 += 32) {
+            const int j = j0 + lane;
+            const bool in = j < nb;
+            const int a = in ? s_addr[j] : -1 - lane;       // distinct dummies never match a real address
+            const unsigned peers = __match_any_sync(0xffffffffu, a);
+            const int base = in ? s_cnt[a] : 0;
+            const int pos = __popc(peers & ((1u << lane) - 1));
+            __syncwarp();
+            if (in) {
+                s_rank[j] = base + pos;
+                if (pos == 0) s_cnt[a] = base + __popc(peers);
+            }
+            __syncwarp();
+        }
+    }
+    __syncthreads();
+    // exclusive scan of s_cnt over the A addresses (each thread a contiguous run)
+    const int per = (A + blockDim.x - 1) / blockDim.x;
+    const int a0 = tid * per;
+    int run = 0;
+    for (int a = a0; a < min(A, a0 + per); ++a) run += s_cnt[a];
+    int x = run;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) s_part[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+        int w = lane < (int)(blockDim.x >> 5) ? s_part[lane] : 0;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            int y = __shfl_up_sync(0xffffffffu, w, o);
+            if (lane >= o) w += y;
+        }
+        s_part[lane] = w;
+    }
+    __syncthreads();
+    int off = (warp ? s_part[warp - 1] : 0) + x - run;
+    for (int a = a0; a < min(A, a0 + per); ++a) {
+        const int c = s_cnt[a];
+        s_cnt[a] = off;   // now the start of address a
+        off += c;
+    }
+    __syncthreads();
+    int dropped = 0;
+    for (int j = tid; j < nb; j += blockDim.x) {
+        const int a = s_addr[j], r = s_rank[j];
+        const int pos = s_cnt[a] + r;
+        ids[bh * nb + pos] = j;
+        saddr[bh * nb + pos] = a;
+        rank[bh * nb + pos] = r;
+        dropped += r >= cap;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) dropped += __shfl_xor_sync(0xffffffffu, dropped, o);
+    if (lane == 0) s_ov[warp] = dropped;
+    __syncthreads();
+    if (tid == 0) {
+        int tot = 0;
+        for (int w = 0; w < (int)(blockDim.x >> 5); ++w) tot += s_ov[w];
+        overflow[bh] = tot;
+    }
+}
+
+// ---------------------------------------------------------------------------
 // (A4) posting lists in canonical form: ids sorted by (address, id), the
 // address of each entry and its rank among the blocks of that address.  The
 // lists keep the earliest `cap` blocks of each address (rank < cap); the
@@ -357,6 +529,235 @@ __global__ void __launch_bounds__(128) k_probe_rerank(const T *__restrict__ Q, c
     }
 }
 
+// ---------------------------------------------------------------------------
+// (A5-A7) the same computation for M = 2 with every size fixed at compile
+// time, so all per-query state stays in registers.  The subspace-0 scores
+// also go to shared memory (one column per thread) so that the final stage can
+// walk the surviving codes by index.  Same pruning rule and arithmetic order
+// as k_probe_rerank.
+// ---------------------------------------------------------------------------
+template <int T_>
+struct RegTop {  // top-T_ by (value desc, index asc); fully unrolled
+    float v[T_];
+    int a[T_];
+    __device__ __forceinline__ void init() {
+#pragma unroll
+        for (int k = 0; k < T_; ++k) { v[k] = -INFINITY; a[k] = 0x7fffffff; }
+    }
+    __device__ __forceinline__ static bool before(float v1, int a1, float v2, int a2) {
+        return v1 > v2 || (v1 == v2 && a1 < a2);
+    }
+    __device__ __forceinline__ void push(float val, int ad) {
+        if (!before(val, ad, v[T_ - 1], a[T_ - 1])) return;
+        v[T_ - 1] = val;
+        a[T_ - 1] = ad;
+#pragma unroll
+        for (int k = T_ - 1; k > 0; --k) {
+            if (before(v[k], a[k], v[k - 1], a[k - 1])) {
+                float tv = v[k]; v[k] = v[k - 1]; v[k - 1] = tv;
+                int ta = a[k]; a[k] = a[k - 1]; a[k - 1] = ta;
+            }
+        }
+    }
+};
+
+template <typename T, int D, int C, int TP, int E, int R>
+__global__ void __launch_bounds__(128) k_probe_m2(const T *__restrict__ Q, const float *__restrict__ kbar,
+                                                  const float *__restrict__ cb, const int32_t *__restrict__ post_ids,
+                                                  const int32_t *__restrict__ post_addr,
+                                                  const int32_t *__restrict__ forced, int32_t *__restrict__ sel,
+                                                  unsigned long long *__restrict__ counters, int S, int H, int Bs,
+                                                  int L, int cap) {
+    constexpr int M = 2, DM = D / 2;
+    static_assert(C <= 32 && TP <= C * C && R >= 1, "shape");
+    extern __shared__ float smem[];
+    const int nb = S / Bs;
+    float *s_cb = smem;                               // [2*C*DM] = C*D floats
+    float *s_s0 = s_cb + C * D;                       // [C][128] subspace-0 scores per thread
+    int32_t *s_addr = (int32_t *)(s_s0 + C * 128);    // [nb]
+    int32_t *s_ids = s_addr + nb;                     // [nb]
+    const int h = blockIdx.y, b = blockIdx.z;
+    const size_t bh = (size_t)b * H + h;
+    for (int i = threadIdx.x; i < C * D; i += blockDim.x) s_cb[i] = cb[(size_t)h * C * D + i];
+    for (int i = threadIdx.x; i < nb; i += blockDim.x) {
+        s_addr[i] = post_addr[bh * nb + i];
+        s_ids[i] = post_ids[bh * nb + i];
+    }
+    __syncthreads();
+
+    const int tid = threadIdx.x;
+    const int t = blockIdx.x * blockDim.x + tid;
+    int n_sel = 0, lt_r = 0, ign = 0;
+    if (t < S) {
+        float q[D];
+        const T *qp = Q + (bh * S + t) * D;
+        if constexpr (sizeof(T) == 2) {
+#pragma unroll
+            for (int c = 0; c < D / 8; ++c) {
+                uint4 u = __ldg((const uint4 *)(qp + 8 * c));
+                const __nv_bfloat162 *h2 = (const __nv_bfloat162 *)&u;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    float2 f = __bfloat1622float2(h2[e]);
+                    q[8 * c + 2 * e] = f.x;
+                    q[8 * c + 2 * e + 1] = f.y;
+                }
+            }
+        } else {
+#pragma unroll
+            for (int c = 0; c < D / 4; ++c) {
+                float4 f = __ldg((const float4 *)(qp + 4 * c));
+                q[4 * c] = f.x; q[4 * c + 1] = f.y; q[4 * c + 2] = f.z; q[4 * c + 3] = f.w;
+            }
+        }
+        // subspace scores (fma chains in ascending element order)
+        float s0[C], s1[C];
+        float mx0 = 0.f, mx1 = 0.f;
+#pragma unroll
+        for (int c = 0; c < C; ++c) {
+            const float4 *w0 = (const float4 *)(s_cb + (0 * C + c) * DM);
+            const float4 *w1 = (const float4 *)(s_cb + (1 * C + c) * DM);
+            float a0 = 0.0f, a1 = 0.0f;
+#pragma unroll
+            for (int i4 = 0; i4 < DM / 4; ++i4) {
+                const float4 x = w0[i4], y = w1[i4];
+                a0 = __fmaf_rn(q[4 * i4 + 0], x.x, a0);
+                a0 = __fmaf_rn(q[4 * i4 + 1], x.y, a0);
+                a0 = __fmaf_rn(q[4 * i4 + 2], x.z, a0);
+                a0 = __fmaf_rn(q[4 * i4 + 3], x.w, a0);
+                a1 = __fmaf_rn(q[DM + 4 * i4 + 0], y.x, a1);
+                a1 = __fmaf_rn(q[DM + 4 * i4 + 1], y.y, a1);
+                a1 = __fmaf_rn(q[DM + 4 * i4 + 2], y.z, a1);
+                a1 = __fmaf_rn(q[DM + 4 * i4 + 3], y.w, a1);
+            }
+            s0[c] = a0;
+            s1[c] = a1;
+            s_s0[c * 128 + tid] = a0;
+            mx0 = fmaxf(mx0, fabsf(a0));
+            mx1 = fmaxf(mx1, fabsf(a1));
+        }
+        int e2;
+        frexpf(2.f * (mx0 + mx1) + 1e-30f, &e2);
+        const float delta = 3.0f * ldexpf(1.f, e2 - 24);   // (M+1) ulp(2G)
+
+        // stage 0: the subspace-0 codes that can still lead to a top-T address
+        RegTop<(TP < C ? TP : C)> u0;
+        constexpr int T0 = TP < C ? TP : C;
+        u0.init();
+#pragma unroll
+        for (int c = 0; c < C; ++c) u0.push(s0[c], c);
+        unsigned cand = 0;
+        if (TP >= C) {
+            cand = C == 32 ? 0xffffffffu : ((1u << C) - 1);
+        } else {
+            const float thr = u0.v[T0 - 1] - delta;
+            const float last_v = u0.v[T0 - 1];
+            const int last_a = u0.a[T0 - 1];
+#pragma unroll
+            for (int c = 0; c < C; ++c) {
+                const float v = s0[c];
+                if (!(v >= thr)) continue;
+                const bool held = !RegTop<T0>::before(last_v, last_a, v, c);
+                bool dom = true;
+                const float hi = v + delta;
+#pragma unroll
+                for (int k = 0; k < T0; ++k) dom = dom && (u0.v[k] > hi || (u0.v[k] >= v && u0.a[k] < c));
+                if (held || !dom) cand |= 1u << c;
+            }
+        }
+        // final stage: every completion of the surviving codes, ranked exactly
+        RegTop<TP> top;
+        top.init();
+        while (cand) {
+            const int c0 = __ffs(cand) - 1;
+            cand &= cand - 1;
+            const float v0 = s_s0[c0 * 128 + tid];
+#pragma unroll
+            for (int c1 = 0; c1 < C; ++c1) top.push(__fadd_rn(v0, s1[c1]), c0 * C + c1);
+        }
+
+        // union of the probed lists, causal filter, E cap; rerank on the fly
+        const int bq = t / Bs;
+        const int lim = bq - L;
+        RegTop<R> rk;
+        rk.init();
+        int nc = 0;
+#pragma unroll 1
+        for (int r = 0; r < TP && nc < E; ++r) {
+            const int a = top.a[r];
+            int lo = 0, hi = nb;
+            while (lo < hi) {
+                const int mid = (lo + hi) >> 1;
+                if (s_addr[mid] < a) lo = mid + 1;
+                else hi = mid;
+            }
+            for (int k = lo; k < nb && s_addr[k] == a && k - lo < cap && nc < E; ++k) {
+                const int j = s_ids[k];
+                if (j > lim) break;
+                ++nc;
+                const float4 *kr = (const float4 *)(kbar + (bh * nb + j) * D);
+                float acc = 0.0f;
+#pragma unroll
+                for (int i4 = 0; i4 < D / 4; ++i4) {
+                    const float4 x = __ldg(kr + i4);
+                    acc = __fmaf_rn(q[4 * i4 + 0], x.x, acc);
+                    acc = __fmaf_rn(q[4 * i4 + 1], x.y, acc);
+                    acc = __fmaf_rn(q[4 * i4 + 2], x.z, acc);
+                    acc = __fmaf_rn(q[4 * i4 + 3], x.w, acc);
+                }
+                rk.push(acc, j);
+            }
+        }
+        int ra[R];
+        int nr = nc < R ? nc : R;
+#pragma unroll
+        for (int k = 0; k < R; ++k) ra[k] = rk.a[k];
+        if (forced) {
+            const int f = forced[bh * S + t];
+            if (f >= 0) {
+                if (f <= lim) {
+                    bool present = false;
+#pragma unroll
+                    for (int k = 0; k < R; ++k) present |= (k < nr) && ra[k] == f;
+                    if (!present) {
+                        const int slot = nr < R ? nr : R - 1;
+#pragma unroll
+                        for (int k = 0; k < R; ++k)
+                            if (k == slot) ra[k] = f;
+                        if (nr < R) ++nr;
+                    }
+                } else {
+                    ign = 1;
+                }
+            }
+        }
+        // ascending ids, -1 padding
+#pragma unroll
+        for (int k = 0; k < R; ++k)
+            if (k >= nr) ra[k] = 0x7fffffff;
+#pragma unroll
+        for (int x = 0; x < R; ++x)
+#pragma unroll
+            for (int y = 0; y + 1 < R - x; ++y)
+                if (ra[y] > ra[y + 1]) { int tmp = ra[y]; ra[y] = ra[y + 1]; ra[y + 1] = tmp; }
+        int32_t *out = sel + (bh * S + t) * R;
+#pragma unroll
+        for (int k = 0; k < R; ++k) out[k] = k < nr ? ra[k] : -1;
+        n_sel = nr;
+        lt_r = nr < R;
+    }
+    for (int o = 16; o > 0; o >>= 1) {
+        n_sel += __shfl_xor_sync(0xffffffffu, n_sel, o);
+        lt_r += __shfl_xor_sync(0xffffffffu, lt_r, o);
+        ign += __shfl_xor_sync(0xffffffffu, ign, o);
+    }
+    if ((threadIdx.x & 31) == 0) {
+        if (lt_r) atomicAdd(&counters[kCntQueriesLtR], (unsigned long long)lt_r);
+        if (n_sel) atomicAdd(&counters[kCntRemoteSel], (unsigned long long)n_sel);
+        if (ign) atomicAdd(&counters[kCntForcedIgnored], (unsigned long long)ign);
+    }
+}
+
 cudaError_t launch_summaries(const Plan &p, const void *K, const float *cb, void *ws, cudaStream_t s) {
     const mono_config &c = p.cfg;
     float *kbar = (float *)ws_ptr(p, ws, kRegKbar);
@@ -364,12 +765,24 @@ cudaError_t launch_summaries(const Plan &p, const void *K, const float *cb, void
     unsigned long long *cnt = (unsigned long long *)ws_ptr(p, ws, kRegCounters);
     cudaError_t e = cudaMemsetAsync(cnt, 0, kCntN * 8, s);
     if (e != cudaSuccess) return e;
-    dim3 g1(p.nb, c.H, c.B);
-    if (c.dtype == MONO_BF16)
-        k_summary_assign<__nv_bfloat16><<<g1, 128, 0, s>>>((const __nv_bfloat16 *)K, cb, kbar, addr, c.S, c.d, c.Bs,
-                                                           c.M, c.C, c.H);
-    else
-        k_summary_assign<float><<<g1, 128, 0, s>>>((const float *)K, cb, kbar, addr, c.S, c.d, c.Bs, c.M, c.C, c.H);
+    const size_t smem = ((size_t)c.C * c.d + 4 * (size_t)c.d + 4 * (size_t)c.M * c.C) * 4;
+    dim3 g1((p.nb + 3) / 4, c.H, c.B);
+#define MONO_SUMW(TT, DD)                                                                                         \
+    do {                                                                                                          \
+        auto kern = k_summary_assign_w<TT, DD>;                                                                   \
+        if (smem > 48 * 1024 &&                                                                                   \
+            (e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess) \
+            return e;                                                                                             \
+        kern<<<g1, 128, smem, s>>>((const TT *)K, cb, kbar, addr, c.S, c.Bs, c.M, c.C, c.H);                    \
+    } while (0)
+    if (c.dtype == MONO_BF16) {
+        if (c.d == 64) MONO_SUMW(__nv_bfloat16, 64);
+        else MONO_SUMW(__nv_bfloat16, 128);
+    } else {
+        if (c.d == 64) MONO_SUMW(float, 64);
+        else MONO_SUMW(float, 128);
+    }
+#undef MONO_SUMW
     count_launches(1);
     return cudaGetLastError();
 }
@@ -377,10 +790,13 @@ cudaError_t launch_summaries(const Plan &p, const void *K, const float *cb, void
 cudaError_t launch_lists(const Plan &p, void *ws, cudaStream_t s) {
     const mono_config &c = p.cfg;
     dim3 g2(c.H, c.B);
-    k_posting_build<<<g2, 1024, p.nb * sizeof(int32_t), s>>>(
-        (const int32_t *)ws_ptr(p, ws, kRegAddr), (int32_t *)ws_ptr(p, ws, kRegPostIds),
-        (int32_t *)ws_ptr(p, ws, kRegPostAddr), (int32_t *)ws_ptr(p, ws, kRegPostRank),
-        (int32_t *)ws_ptr(p, ws, kRegOverflow), p.nb, c.cap, c.H);
+    const int32_t *addr = (const int32_t *)ws_ptr(p, ws, kRegAddr);
+    int32_t *ids = (int32_t *)ws_ptr(p, ws, kRegPostIds), *saddr = (int32_t *)ws_ptr(p, ws, kRegPostAddr);
+    int32_t *rank = (int32_t *)ws_ptr(p, ws, kRegPostRank), *ov = (int32_t *)ws_ptr(p, ws, kRegOverflow);
+    if (p.A <= kDenseA)
+        k_posting_dense<<<g2, 1024, (size_t)p.nb * 8, s>>>(addr, ids, saddr, rank, ov, p.nb, c.cap, c.H, (int)p.A);
+    else
+        k_posting_build<<<g2, 1024, p.nb * sizeof(int32_t), s>>>(addr, ids, saddr, rank, ov, p.nb, c.cap, c.H);
     count_launches(1);
     return cudaGetLastError();
 }
@@ -395,9 +811,29 @@ cudaError_t launch_queries(const Plan &p, const void *Q, const float *cb, const 
     const float *kbar = (const float *)ws_ptr(p, ws, kRegKbar);
     const int32_t *ids = (const int32_t *)ws_ptr(p, ws, kRegPostIds);
     const int32_t *saddr = (const int32_t *)ws_ptr(p, ws, kRegPostAddr);
-    const size_t smem = (size_t)c.C * c.d * 4 + (size_t)p.nb * 8;
     dim3 g3((c.S + 127) / 128, c.H, c.B);
     const bool bf = c.dtype == MONO_BF16;
+    // compile-time shapes of the configured workloads; any other shape takes the general kernel
+#define MONO_M2(TT, DD, CC, TPP, EE, RR)                                                                          \
+    if (c.M == 2 && c.d == DD && c.C == CC && c.T == TPP && c.E == EE && c.R == RR) {                           \
+        const size_t sm2 = (size_t)CC * DD * 4 + (size_t)CC * 128 * 4 + (size_t)p.nb * 8;                       \
+        auto kern = k_probe_m2<TT, DD, CC, TPP, EE, RR>;                                                        \
+        if (sm2 > 48 * 1024 &&                                                                                   \
+            (e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm2)) != cudaSuccess) \
+            return e;                                                                                            \
+        kern<<<g3, 128, sm2, s>>>((const TT *)Q, kbar, cb, ids, saddr, forced, sel, cnt, c.S, c.H, c.Bs, c.L, c.cap); \
+        count_launches(1);                                                                                       \
+        return cudaGetLastError();                                                                               \
+    }
+    if (bf) {
+        MONO_M2(__nv_bfloat16, 64, 16, 4, 5, 2)
+        MONO_M2(__nv_bfloat16, 128, 32, 8, 8, 4)
+    } else {
+        MONO_M2(float, 64, 16, 4, 5, 2)
+        MONO_M2(float, 64, 8, 4, 5, 2)
+    }
+#undef MONO_M2
+    const size_t smem = (size_t)c.C * c.d * 4 + (size_t)p.nb * 8;
 #define MONO_LAUNCH_PR(TT, DD)                                                                                     \
     do {                                                                                                           \
         auto kern = k_probe_rerank<TT, DD>;                                                                        \

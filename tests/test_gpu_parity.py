@@ -117,6 +117,40 @@ def test_empty_batch_is_a_no_op():
 
 
 # ---------------------------------------------------------------------------
+# tensor-core attention path (bf16, Bs in {64, 128}): shapes, raggedness, budgets
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("d,Bs,L,R,S", [
+    (64, 64, 2, 2, 832),      # 13 blocks: last query tile half full
+    (128, 64, 2, 4, 1024),
+    (64, 128, 2, 2, 1408),    # 11 blocks of 128
+    (128, 128, 1, 3, 768),
+    (64, 64, 3, 2, 960),      # widest local range: 256 keys
+    (64, 64, 1, 2, 640),
+])
+def test_tensor_core_attention_shapes(d, Bs, L, R, S):
+    cfg = small(d=d, Bs=Bs, L=L, R=R, E=max(5, R), S=S, H=2, C=8, cap=6, dtype="bf16")
+    full_check(Run(cfg, seed=10 + d + Bs + L))
+
+
+def test_tensor_core_attention_edge_cases():
+    full_check(Run(small(S=640, Bs=64, R=0, E=0, dtype="bf16"), seed=20))           # local only
+    full_check(Run(small(S=640, Bs=64, x="zeros", dtype="bf16"), seed=21))          # all ties
+    run = Run(small(S=1024, Bs=64, dtype="bf16", cap=8), seed=22, forced_frac=0.5)  # forced blocks
+    full_check(run)
+
+
+def test_simple_and_tensor_core_paths_agree():
+    from learned_product_hash_proj_b200 import mono
+    cfg = small(S=1024, Bs=64, C=16, cap=8, dtype="bf16")
+    fast = Run(cfg, seed=23).run_stages()
+    simple = Run(cfg, seed=23, flags=mono.MONO_FLAG_SIMPLE_KERNELS).run_stages()
+    assert torch.equal(fast.sel, simple.sel)
+    a, b = fast.O.float(), simple.O.float()
+    rms = b.pow(2).mean().sqrt().item()
+    assert ((a - b).abs() - 2.0 ** -7 * b.abs()).max().item() <= 2e-2 * rms
+
+
+# ---------------------------------------------------------------------------
 # full-size workloads: integer tables in full, sampled outputs
 # ---------------------------------------------------------------------------
 def sampled_check(name, n_rows=96, n_queries=1500, seed=0):
