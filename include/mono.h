@@ -67,9 +67,11 @@ enum mono_status {
 
 /* Plan options (mono_config.flags). */
 enum mono_flags {
-    /* Run the plain query-major kernels (SIMT projections and attention)
+    /* Run the plain kernels (SIMT projections, query-major SIMT attention)
      * even where the tensor-core kernels apply.  Same results within the
-     * stated tolerances; used as the correctness baseline. */
+     * stated tolerances; used as the correctness baseline.  The tensor-core
+     * kernels apply to bf16 storage with: projections W % 128 == 0 and
+     * H*d % 128 == 0; attention Bs in {64, 128} and 128 + (L-1)*Bs <= 256. */
     MONO_FLAG_SIMPLE_KERNELS = 1
 };
 

@@ -69,8 +69,8 @@ void layout(Plan *p) {
         bytes[kRegPairs] = B * H * S * R * 4;
         bytes[kRegPartO] = B * H * S * R * d * 2;
         bytes[kRegPartML] = B * H * S * R * 8;
-        bytes[kRegWork] = (size_t)p->max_work * 8;
-        bytes[kRegNWork] = 4;
+        bytes[kRegWork] = B * H * (size_t)p->max_work * 8;
+        bytes[kRegNWork] = B * H * 4;
     }
     size_t off = 0;
     for (int r = 0; r < kRegN; ++r) {
@@ -101,10 +101,6 @@ int check_ptrs(std::initializer_list<const void *> ptrs) {
 }
 
 }  // namespace
-
-struct mono_plan_s {
-    Plan p;
-};
 
 extern "C" {
 
@@ -140,9 +136,10 @@ int mono_plan(const mono_config *cfg, mono_plan_t **plan, size_t *workspace_byte
     for (int m = 0; m < cfg->M; ++m) p.A *= cfg->C;
     p.es = cfg->dtype == MONO_BF16 ? 2 : 4;
     p.fast = attend_tc_supported(*cfg) && !(cfg->flags & MONO_FLAG_SIMPLE_KERNELS);
+    p.gemm_tc = gemm_tc_supported(*cfg) && !(cfg->flags & MONO_FLAG_SIMPLE_KERNELS);
     {
-        const long long pairs = (long long)cfg->B * cfg->H * cfg->S * cfg->R;
-        const long long mw = (long long)cfg->B * cfg->H * p.nb + (pairs + 127) / 128;
+        // remote work items per (b, h): one per bucket at most, plus one per 128 pairs
+        const long long mw = (long long)p.nb + ((long long)cfg->S * cfg->R + 127) / 128;
         if (p.fast && cfg->R > 0 && mw > (1ll << 31) - 1) { free(ps); return MONO_ERR_UNSUPPORTED; }
         p.max_work = (int)(mw < (1ll << 31) - 1 ? mw : 0);
     }
@@ -171,6 +168,7 @@ int mono_project(const mono_plan_t *plan, const void *x, const void *Wq, const v
     if ((st = check_ptrs({x, Wq, Wk, Wv, Q, K, V}))) return st;
     cudaStream_t s = (cudaStream_t)stream;
     if ((st = cuda_status(launch_rope_tables(p, workspace, s)))) return st;
+    if (p.gemm_tc) return cuda_status(launch_project_tc(p, x, Wq, Wk, Wv, Q, K, V, workspace, s));
     return cuda_status(launch_project_simt(p, x, Wq, Wk, Wv, Q, K, V, workspace, s));
 }
 
@@ -238,6 +236,7 @@ int mono_out_project(const mono_plan_t *plan, const void *O, const void *Wo, voi
     const Plan &p = plan->p;
     if (empty(&p)) return MONO_OK;
     if ((st = check_ptrs({O, Wo, delta}))) return st;
+    if (p.gemm_tc) return cuda_status(launch_out_project_tc(p, O, Wo, delta, workspace, (cudaStream_t)stream));
     return cuda_status(launch_out_project_simt(p, O, Wo, delta, (cudaStream_t)stream));
 }
 

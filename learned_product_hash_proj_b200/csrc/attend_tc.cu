@@ -28,36 +28,52 @@ using bf16 = __nv_bfloat16;
 __device__ __forceinline__ bool sel_valid(int j, int t, int Bs, int L) { return j >= 0 && j <= t / Bs - L; }
 
 // ---------------------------------------------------------------------------
-// pair buckets
+// pair buckets.  Every (b, h) owns a segment of S*R pair slots and of
+// wcap = nb + ceil(S*R/kChunk) work items, so the buckets of different heads
+// never interact.  Each CTA of the count and fill kernels takes kQTile
+// consecutive queries of one (b, h) and aggregates them in shared memory:
+// one global atomic per distinct block per CTA instead of one per pair.
 // ---------------------------------------------------------------------------
-__global__ void k_pair_count(const int32_t *__restrict__ sel, int32_t *__restrict__ cnt, long long n_qh, int S,
-                             int R, int nb, int Bs, int L, unsigned long long *__restrict__ counters) {
-    const long long q = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-    if (q >= n_qh) return;
-    const long long bh = q / S;
-    const int t = (int)(q % S);
-    for (int r = 0; r < R; ++r) {
-        const int j = sel[q * R + r];
-        if (sel_valid(j, t, Bs, L)) atomicAdd(&cnt[bh * nb + j], 1);
-        else if (j >= 0) record_error(counters, kDevErrBadSel);
-    }
+constexpr int kChunk = 128;   // queries per remote work item
+constexpr int kQTile = 1024;  // queries per CTA of the count and fill kernels
+
+// grid (ceil(S/kQTile), B*H), 256 threads, smem nb ints
+__global__ void __launch_bounds__(256) k_pair_count(const int32_t *__restrict__ sel, int32_t *__restrict__ cnt,
+                                                    int S, int R, int nb, int Bs, int L,
+                                                    unsigned long long *__restrict__ counters) {
+    extern __shared__ int s_h[];
+    const long long bh = blockIdx.y;
+    for (int j = threadIdx.x; j < nb; j += blockDim.x) s_h[j] = 0;
+    __syncthreads();
+    const int t0 = blockIdx.x * kQTile, t1 = min(S, t0 + kQTile);
+    bool bad = false;
+    for (int t = t0 + threadIdx.x; t < t1; t += blockDim.x)
+        for (int r = 0; r < R; ++r) {
+            const int j = sel[((size_t)bh * S + t) * R + r];
+            if (sel_valid(j, t, Bs, L)) atomicAdd(&s_h[j], 1);
+            else bad |= j >= 0;
+        }
+    if (bad) record_error(counters, kDevErrBadSel);
+    __syncthreads();
+    for (int j = threadIdx.x; j < nb; j += blockDim.x)
+        if (s_h[j]) atomicAdd(&cnt[bh * nb + j], s_h[j]);
 }
 
-// exclusive scan of the bucket sizes over every (b, h, j), the fill cursors
-// reset, and one work item per chunk of <= kChunk queries of a bucket.
-constexpr int kChunk = 128;
-
+// exclusive scan of one (b, h)'s bucket sizes, fill cursors reset, and one
+// work item per chunk of <= kChunk queries.  grid B*H, 1024 threads.
 __global__ void __launch_bounds__(1024) k_pair_scan(const int32_t *__restrict__ cnt, int32_t *__restrict__ start,
                                                     int32_t *__restrict__ fill, int2 *__restrict__ work,
-                                                    int32_t *__restrict__ nwork, int n) {
+                                                    int32_t *__restrict__ nwork, int nb, int wcap) {
     __shared__ int s_w[32], s_c[32];
     __shared__ int carry_p, carry_c;
+    const long long bh = blockIdx.x;
     if (threadIdx.x == 0) { carry_p = 0; carry_c = 0; }
     __syncthreads();
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    for (int base = 0; base < n; base += blockDim.x) {
-        const int i = base + threadIdx.x;
-        const int c = i < n ? cnt[i] : 0;
+    const int nw = blockDim.x >> 5;
+    for (int base = 0; base < nb; base += blockDim.x) {
+        const int j = base + threadIdx.x;
+        const int c = j < nb ? cnt[bh * nb + j] : 0;
         const int ch = (c + kChunk - 1) / kChunk;
         int xp = c, xc = ch;  // inclusive warp scans
 #pragma unroll
@@ -68,7 +84,7 @@ __global__ void __launch_bounds__(1024) k_pair_scan(const int32_t *__restrict__ 
         if (lane == 31) { s_w[warp] = xp; s_c[warp] = xc; }
         __syncthreads();
         if (warp == 0) {
-            int wp = lane < (int)(blockDim.x >> 5) ? s_w[lane] : 0, wc = lane < (int)(blockDim.x >> 5) ? s_c[lane] : 0;
+            int wp = lane < nw ? s_w[lane] : 0, wc = lane < nw ? s_c[lane] : 0;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
                 int yp = __shfl_up_sync(0xffffffffu, wp, o), yc = __shfl_up_sync(0xffffffffu, wc, o);
@@ -80,34 +96,51 @@ __global__ void __launch_bounds__(1024) k_pair_scan(const int32_t *__restrict__ 
         __syncthreads();
         const int off_p = carry_p + (warp ? s_w[warp - 1] : 0) + xp - c;
         const int off_c = carry_c + (warp ? s_c[warp - 1] : 0) + xc - ch;
-        if (i < n) {
-            start[i] = off_p;
-            fill[i] = 0;
-            for (int k = 0; k < ch; ++k) work[off_c + k] = make_int2(i, k);
+        if (j < nb) {
+            start[bh * nb + j] = off_p;
+            fill[bh * nb + j] = 0;
+            for (int k = 0; k < ch; ++k) work[bh * wcap + off_c + k] = make_int2(j, k);
         }
         __syncthreads();
         if (threadIdx.x == 0) {
-            carry_p += s_w[(blockDim.x >> 5) - 1];
-            carry_c += s_c[(blockDim.x >> 5) - 1];
+            carry_p += s_w[nw - 1];
+            carry_c += s_c[nw - 1];
         }
         __syncthreads();
     }
-    if (threadIdx.x == 0) *nwork = carry_c;
+    if (threadIdx.x == 0) nwork[bh] = carry_c;
 }
 
-__global__ void k_pair_fill(const int32_t *__restrict__ sel, const int32_t *__restrict__ start,
-                            int32_t *__restrict__ fill, int32_t *__restrict__ pairs, long long n_qh, int S, int R,
-                            int nb, int Bs, int L) {
-    const long long q = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-    if (q >= n_qh) return;
-    const long long bh = q / S;
-    const int t = (int)(q % S);
-    for (int r = 0; r < R; ++r) {
-        const int j = sel[q * R + r];
-        if (!sel_valid(j, t, Bs, L)) continue;
-        const long long b = bh * nb + j;
-        const int slot = atomicAdd(&fill[b], 1);
-        pairs[start[b] + slot] = t * R + r;
+// grid (ceil(S/kQTile), B*H), 256 threads, smem 2*nb ints
+__global__ void __launch_bounds__(256) k_pair_fill(const int32_t *__restrict__ sel, const int32_t *__restrict__ start,
+                                                   int32_t *__restrict__ fill, int32_t *__restrict__ pairs, int S,
+                                                   int R, int nb, int Bs, int L) {
+    extern __shared__ int s_h[];
+    int *s_base = s_h + nb;
+    const long long bh = blockIdx.y;
+    for (int j = threadIdx.x; j < nb; j += blockDim.x) s_h[j] = 0;
+    __syncthreads();
+    const int t0 = blockIdx.x * kQTile, t1 = min(S, t0 + kQTile);
+    constexpr int kPer = (kQTile / 256) * kMaxR;   // pairs one thread can hold
+    int my_j[kPer], my_rank[kPer], my_val[kPer];
+    int n = 0;
+    for (int t = t0 + threadIdx.x; t < t1; t += blockDim.x)
+        for (int r = 0; r < R; ++r) {
+            const int j = sel[((size_t)bh * S + t) * R + r];
+            if (!sel_valid(j, t, Bs, L)) continue;
+            my_j[n] = j;
+            my_rank[n] = atomicAdd(&s_h[j], 1);
+            my_val[n] = t * R + r;
+            ++n;
+        }
+    __syncthreads();
+    for (int j = threadIdx.x; j < nb; j += blockDim.x)
+        if (s_h[j]) s_base[j] = atomicAdd(&fill[bh * nb + j], s_h[j]);
+    __syncthreads();
+    int32_t *seg = pairs + (size_t)bh * S * R;
+    for (int k = 0; k < n; ++k) {
+        const int j = my_j[k];
+        seg[start[bh * nb + j] + s_base[j] + my_rank[k]] = my_val[k];
     }
 }
 
@@ -116,14 +149,15 @@ __global__ void k_pair_fill(const int32_t *__restrict__ sel, const int32_t *__re
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ uint4 ldg16(const void *p) { return __ldg((const uint4 *)p); }
 
-// rows [0, nrows) of a [*, D] bf16 matrix -> K-major tile (kdim = D); rows >= valid are zero
+// rows [0, nrows) of a [*, D] bf16 matrix -> K-major tile (kdim = D); rows >= valid are zero.
+// Asynchronous: every copy is in flight at once; complete with cp_async_wait_all.
 template <int D>
 __device__ __forceinline__ void load_rows(uint8_t *tile, const bf16 *src, int nrows, int valid, int tid, int nthr) {
     for (int idx = tid; idx < nrows * (D / 8); idx += nthr) {
         const int row = idx / (D / 8), c = idx % (D / 8);
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (row < valid) v = ldg16(src + (size_t)row * D + 8 * c);
-        *(uint4 *)(tile + tc::kmajor_chunk(row, c, D)) = v;
+        const bool ok = row < valid;
+        tc::cp_async16(tile + tc::kmajor_chunk(row, c, D), ok ? (const void *)(src + (size_t)row * D + 8 * c) : src,
+                       ok);
     }
 }
 
@@ -133,9 +167,9 @@ template <int D>
 __device__ __forceinline__ void load_v(uint8_t *tile, const bf16 *src, int nkeys, int valid, int tid, int nthr) {
     for (int idx = tid; idx < nkeys * (D / 8); idx += nthr) {
         const int key = idx / (D / 8), c = idx % (D / 8);
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (key < valid) v = ldg16(src + (size_t)key * D + 8 * c);
-        *(uint4 *)(tile + tc::mnmajor_chunk(key, c, nkeys)) = v;
+        const bool ok = key < valid;
+        tc::cp_async16(tile + tc::mnmajor_chunk(key, c, nkeys),
+                       ok ? (const void *)(src + (size_t)key * D + 8 * c) : src, ok);
     }
 }
 
@@ -158,24 +192,29 @@ __global__ void __launch_bounds__(128) k_remote_tc(const bf16 *__restrict__ Q, c
                                                    const int2 *__restrict__ work, const int32_t *__restrict__ nwork,
                                                    bf16 *__restrict__ part_o, float2 *__restrict__ part_ml,
                                                    unsigned long long *__restrict__ counters, int S, int R, int nb,
-                                                   float scale_log2) {
-    constexpr int NCOLS = (BS + D) <= 128 ? 128 : 256;   // S: [0, BS), O: [BS, BS + D)
+                                                   int wcap, float scale_log2) {
+    // TMEM: S in columns [0, BS); O overwrites them once every thread has turned S into P
+    constexpr int NCOLS = (BS > D ? BS : D) <= 64 ? 64 : 128;
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ uint64_t mbar;
     __shared__ uint32_t tmem_base;
+    const long long bh = blockIdx.y;
     const int item = blockIdx.x;
-    if (item >= *nwork || timed_out(counters)) return;
+    if (item >= nwork[bh] || timed_out(counters)) return;
     const int tid = threadIdx.x, warp = tid >> 5;
-    const int2 w = work[item];
-    const long long bh = w.x / nb;
-    const int j = w.x % nb;
-    const int p0 = start[w.x] + w.y * kChunk;
-    const int n = min(kChunk, cnt[w.x] - w.y * kChunk);
+    const int2 w = work[bh * wcap + item];
+    const int j = w.x;
+    const size_t bj = (size_t)bh * nb + j;
+    const int p0 = start[bj] + w.y * kChunk;
+    const int n = min(kChunk, cnt[bj] - w.y * kChunk);
+    pairs += (size_t)bh * S * R;
 
+    // P reuses Q's space when it fits: Q is only read by the first MMA, which has completed when P is written
+    constexpr int QB = 128 * D * 2, KB = BS * D * 2, VB = BS * D * 2, PB = 128 * BS * 2;
     uint8_t *sQ = smem;                       // [128 x D]
-    uint8_t *sK = sQ + 128 * D * 2;           // [BS x D]
-    uint8_t *sVt = sK + BS * D * 2;           // V_j, MN-major [BS keys x D]
-    uint8_t *sP = sVt + D * BS * 2;           // [128 x BS]
+    uint8_t *sK = sQ + QB;                    // [BS x D]
+    uint8_t *sVt = sK + KB;                   // V_j, MN-major [BS keys x D]
+    uint8_t *sP = PB <= QB ? sQ : sVt + VB;   // [128 x BS]
 
     if (warp == 0) {
         tc::tmem_alloc(&tmem_base, NCOLS);
@@ -192,15 +231,12 @@ __global__ void __launch_bounds__(128) k_remote_tc(const bf16 *__restrict__ Q, c
     {
         const bf16 *qrow = Q + ((size_t)bh * S + t) * D;
 #pragma unroll
-        for (int c = 0; c < D / 8; ++c) {
-            uint4 v = make_uint4(0, 0, 0, 0);
-            if (tid < n) v = ldg16(qrow + 8 * c);
-            *(uint4 *)(sQ + tc::kmajor_chunk(tid, c, D)) = v;
-        }
+        for (int c = 0; c < D / 8; ++c) tc::cp_async16(sQ + tc::kmajor_chunk(tid, c, D), qrow + 8 * c, tid < n);
     }
     const size_t kv0 = ((size_t)bh * S + (size_t)j * BS) * D;
     load_rows<D>(sK, K + kv0, BS, BS, tid, 128);
     load_v<D>(sVt, V + kv0, BS, BS, tid, 128);
+    tc::cp_async_wait_all();
     tc::fence_smem_to_async();
     tc::fence_before_sync();
     __syncthreads();
@@ -255,7 +291,7 @@ __global__ void __launch_bounds__(128) k_remote_tc(const bf16 *__restrict__ Q, c
         const uint32_t ap = tc::smem_u32(sP), bv = tc::smem_u32(sVt);
 #pragma unroll
         for (int k = 0; k < BS / 16; ++k)
-            tc::mma_bf16(tmem + BS, tc::desc_kmajor(ap + 256 * k, BS), tc::desc_mnmajor(bv + 256 * k, BS), id, k > 0);
+            tc::mma_bf16(tmem, tc::desc_kmajor(ap + 256 * k, BS), tc::desc_mnmajor(bv + 256 * k, BS), id, k > 0);
         tc::commit(&mbar);
     }
     if (ok) ok = tc::mbar_wait(&mbar, 1);
@@ -267,7 +303,7 @@ __global__ void __launch_bounds__(128) k_remote_tc(const bf16 *__restrict__ Q, c
     const float inv = 1.f / l;
 #pragma unroll
     for (int c0 = 0; c0 < D; c0 += 32) {
-        tc::tmem_ld32(trow + BS + c0, v);
+        tc::tmem_ld32(trow + c0, v);
         if (tid < n && ok) {
             uint4 *dst = (uint4 *)(part_o + slot * D + c0);
 #pragma unroll
@@ -325,6 +361,24 @@ __global__ void __launch_bounds__(128) k_local_merge_tc(const bf16 *__restrict__
     load_rows<D>(sQ, Qb + (size_t)t0 * D, 128, nq, tid, 128);
     load_rows<D>(sK, Kb + (size_t)kstart * D, NK, nk, tid, 128);
     load_v<D>(sVt, Vb + (size_t)kstart * D, NK, nk, tid, 128);
+    // this query's remote selections and their (max, sum); the partial rows are
+    // prefetched to L2 so that the merge at the end does not wait on DRAM
+    const int t = t0 + tid;
+    const bool live = tid < nq;
+    int jr[kMaxR];
+    float2 ml[kMaxR];
+    for (int r = 0; r < R; ++r) {
+        jr[r] = -1;
+        if (!live) continue;
+        const size_t pq = ((size_t)bh * S + t) * R + r;
+        const int j = sel[pq];
+        if (sel_valid(j, t, BS, L)) {
+            jr[r] = j;
+            ml[r] = part_ml[pq];
+            for (int c = 0; c < D * 2; c += 128) tc::prefetch_l2((const uint8_t *)(part_o + pq * D) + c);
+        }
+    }
+    tc::cp_async_wait_all();
     tc::fence_smem_to_async();
     tc::fence_before_sync();
     __syncthreads();
@@ -342,40 +396,56 @@ __global__ void __launch_bounds__(128) k_local_merge_tc(const bf16 *__restrict__
     bool ok = tc::mbar_wait(&mbar, 0);
     tc::fence_after_sync();
 
-    // masked softmax of row t over keys s in [lo(t), t]
-    const int t = t0 + tid;
+    // masked softmax of row t over keys s in [lo(t), t].  In column terms the
+    // valid keys are [vlo, vhi]; 32-column chunks entirely inside need no
+    // per-element mask and chunks entirely outside need no exponential.
     const int lo = max(0, t / BS - L + 1) * BS;
+    const int vlo = lo - kstart, vhi = t - kstart;
     float v[32];
     float m = -INFINITY;
-#pragma unroll
+#pragma unroll 1
     for (int c0 = 0; c0 < NK; c0 += 32) {
         tc::tmem_ld32(trow + c0, v);
+        if (c0 + 31 < vlo || c0 > vhi) continue;
+        if (c0 >= vlo && c0 + 31 <= vhi) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            const int s = kstart + c0 + i;
-            if (s >= lo && s <= t) m = fmaxf(m, v[i]);
+            for (int i = 0; i < 32; ++i) m = fmaxf(m, v[i]);
+        } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+                if (c0 + i >= vlo && c0 + i <= vhi) m = fmaxf(m, v[i]);
         }
     }
     const float m2 = (m == -INFINITY) ? 0.f : m * scale_log2;
     float l = 0.f;
-    // P must not overwrite Q/K before every thread has finished reading S? Q/K are only read by MMA 1,
-    // which has completed (mbarrier), so P can reuse their space.
-#pragma unroll
+    // P may reuse the space of Q and K: they are only read by the first MMA,
+    // which has completed (mbarrier) before any thread gets here.
+#pragma unroll 1
     for (int c0 = 0; c0 < NK; c0 += 32) {
         tc::tmem_ld32(trow + c0, v);
+        uint32_t pk[16];
+        if (c0 + 31 < vlo || c0 > vhi) {
 #pragma unroll
-        for (int q8 = 0; q8 < 4; ++q8) {
-            uint32_t pk[4];
+            for (int u = 0; u < 16; ++u) pk[u] = 0u;
+        } else {
+            const bool full = c0 >= vlo && c0 + 31 <= vhi;
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int s = kstart + c0 + 8 * q8 + 2 * u;
-                const float a = (s >= lo && s <= t) ? exp2f(fmaf(v[8 * q8 + 2 * u], scale_log2, -m2)) : 0.f;
-                const float bb = (s + 1 >= lo && s + 1 <= t) ? exp2f(fmaf(v[8 * q8 + 2 * u + 1], scale_log2, -m2)) : 0.f;
+            for (int u = 0; u < 16; ++u) {
+                const int i = 2 * u;
+                float a = exp2f(fmaf(v[i], scale_log2, -m2));
+                float bb = exp2f(fmaf(v[i + 1], scale_log2, -m2));
+                if (!full) {
+                    a = (c0 + i >= vlo && c0 + i <= vhi) ? a : 0.f;
+                    bb = (c0 + i + 1 >= vlo && c0 + i + 1 <= vhi) ? bb : 0.f;
+                }
                 l += a + bb;
                 pk[u] = pack2(a, bb);
             }
-            *(uint4 *)(sP + tc::kmajor_chunk(tid, (c0 >> 3) + q8, NK)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
         }
+#pragma unroll
+        for (int q8 = 0; q8 < 4; ++q8)
+            *(uint4 *)(sP + tc::kmajor_chunk(tid, (c0 >> 3) + q8, NK)) =
+                make_uint4(pk[4 * q8], pk[4 * q8 + 1], pk[4 * q8 + 2], pk[4 * q8 + 3]);
     }
     tc::fence_smem_to_async();
     tc::fence_before_sync();
@@ -395,19 +465,8 @@ __global__ void __launch_bounds__(128) k_local_merge_tc(const bf16 *__restrict__
 
     // merge with the remote partials: out = (O_loc + sum_r l_r 2^(m_r - M) o_r 2^(m_loc... )) / ...
     float mm = m2;
-    int jr[kMaxR];
-    float2 ml[kMaxR];
-    const bool live = tid < nq;
-    for (int r = 0; r < R; ++r) {
-        jr[r] = -1;
-        if (!live) continue;
-        const int j = sel[((size_t)bh * S + t) * R + r];
-        if (sel_valid(j, t, BS, L)) {
-            jr[r] = j;
-            ml[r] = part_ml[((size_t)bh * S + t) * R + r];
-            mm = fmaxf(mm, ml[r].x);
-        }
-    }
+    for (int r = 0; r < R; ++r)
+        if (jr[r] >= 0) mm = fmaxf(mm, ml[r].x);
     const float wl = exp2f(m2 - mm);
     float den = l * wl;
     float wr[kMaxR];
@@ -466,7 +525,6 @@ static cudaError_t launch_tc_shape(const Plan &p, const bf16 *Q, const bf16 *K, 
     const mono_config &c = p.cfg;
     unsigned long long *cnt_err = (unsigned long long *)ws_ptr(p, ws, kRegCounters);
     const float scale_log2 = (float)(1.4426950408889634 / sqrt((double)c.d));
-    const long long n_qh = (long long)c.B * c.H * c.S;
     const int nbh = c.B * c.H * p.nb;
     cudaError_t e;
     if (c.R > 0) {
@@ -477,17 +535,26 @@ static cudaError_t launch_tc_shape(const Plan &p, const bf16 *Q, const bf16 *K, 
         int2 *work = (int2 *)ws_ptr(p, ws, kRegWork);
         int32_t *nwork = (int32_t *)ws_ptr(p, ws, kRegNWork);
         if ((e = cudaMemsetAsync(pc, 0, (size_t)nbh * 4, s)) != cudaSuccess) return e;
-        const int thr = 256;
-        const unsigned blocks = (unsigned)((n_qh + thr - 1) / thr);
-        k_pair_count<<<blocks, thr, 0, s>>>(sel, pc, n_qh, c.S, c.R, p.nb, c.Bs, c.L, cnt_err);
-        k_pair_scan<<<1, 1024, 0, s>>>(pc, ps, pf, work, nwork, nbh);
-        k_pair_fill<<<blocks, thr, 0, s>>>(sel, ps, pf, pairs, n_qh, c.S, c.R, p.nb, c.Bs, c.L);
-        const size_t smem = (size_t)(128 * D + BS * D + D * BS + 128 * BS) * 2;
+        const int nbhh = c.B * c.H;
+        const int wcap = p.max_work;  // work items per (b, h)
+        dim3 gq((c.S + kQTile - 1) / kQTile, nbhh);
+        const size_t hs = (size_t)p.nb * 4;
+        if (2 * hs > 48 * 1024) {
+            if ((e = cudaFuncSetAttribute(k_pair_count, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)hs)) ||
+                (e = cudaFuncSetAttribute(k_pair_fill, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)(2 * hs))))
+                return e;
+        }
+        k_pair_count<<<gq, 256, hs, s>>>(sel, pc, c.S, c.R, p.nb, c.Bs, c.L, cnt_err);
+        k_pair_scan<<<nbhh, 1024, 0, s>>>(pc, ps, pf, work, nwork, p.nb, wcap);
+        k_pair_fill<<<gq, 256, 2 * hs, s>>>(sel, ps, pf, pairs, c.S, c.R, p.nb, c.Bs, c.L);
+        const size_t pbytes = (size_t)128 * BS * 2, qbytes = (size_t)128 * D * 2;
+        const size_t smem = qbytes + (size_t)2 * BS * D * 2 + (pbytes <= qbytes ? 0 : pbytes);
         auto kr = k_remote_tc<D, BS>;
         if ((e = cudaFuncSetAttribute(kr, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
             return e;
-        kr<<<p.max_work, 128, smem, s>>>(Q, K, V, pairs, ps, pc, work, nwork, (bf16 *)ws_ptr(p, ws, kRegPartO),
-                                         (float2 *)ws_ptr(p, ws, kRegPartML), cnt_err, c.S, c.R, p.nb, scale_log2);
+        dim3 gr(wcap, nbhh);
+        kr<<<gr, 128, smem, s>>>(Q, K, V, pairs, ps, pc, work, nwork, (bf16 *)ws_ptr(p, ws, kRegPartO),
+                                 (float2 *)ws_ptr(p, ws, kRegPartML), cnt_err, c.S, c.R, p.nb, wcap, scale_log2);
         count_launches(4);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }

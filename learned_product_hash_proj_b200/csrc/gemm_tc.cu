@@ -1,0 +1,271 @@
+// gemm_tc.cu -- the projections on the tcgen05 tensor cores (bf16 storage,
+// fp32 accumulation): Q/K/V = x W^T with RoPE on Q and K fused into the
+// epilogue, and delta = O Wo^T.
+//
+// One CTA computes a 128 x 128 output tile:
+//   warp 0 (one lane)  TMA producer: A and B tiles (64-wide K slices, 128-byte
+//                      swizzle) into a STAGES-deep ring, completion counted on
+//                      the stage's "full" mbarrier;
+//   warp 1 (one lane)  MMA issuer: 4 x tcgen05.mma (K = 16 each) per slice into
+//                      a 128 x 128 fp32 accumulator in TMEM, then
+//                      tcgen05.commit frees the stage ("empty" mbarrier);
+//   warps 2..5         epilogue: TMEM -> registers (32 columns at a time),
+//                      RoPE on interleaved pairs, bf16, scatter to [B,H,S,d]
+//                      or row-major [M, N].
+// Every wait is bounded; on expiry the kernel records an error and finishes.
+// TMA loads have no cluster multicast; each CTA loads its own tiles.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "internal.cuh"
+#include "tc.cuh"
+
+namespace mono {
+
+using bf16 = __nv_bfloat16;
+
+namespace {
+
+constexpr int BM = 128, BN = 128, BK = 64, STAGES = 3;  // 97 KB: two CTAs per SM
+constexpr int A_BYTES = BM * BK * 2, B_BYTES = BN * BK * 2;
+constexpr int SMEM_BYTES = STAGES * (A_BYTES + B_BYTES) + 1024;  // + alignment slack
+
+enum { kEpiRope = 0, kEpiHeads = 1, kEpiPlain = 2 };
+
+struct TmaMaps {
+    CUtensorMap a;
+    CUtensorMap b[3];
+};
+
+struct Epi {
+    bf16 *out[3];
+    int mode[3];
+    int M, N;          // rows, columns of each output
+    int S, H, d;
+    const float2 *rope_hi, *rope_lo;
+    unsigned long long *counters;
+};
+
+__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y, uint64_t *mbar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+            tc::smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(tc::smem_u32(mbar))
+        : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t *mbar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(tc::smem_u32(mbar)), "r"(bytes)
+                 : "memory");
+}
+
+// K-major, 128-byte swizzle: 8-row x 128-byte atoms, 1024 bytes apart.
+__device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr & 0x3FFFF) >> 4);
+    d |= (uint64_t)1 << 16;             // leading byte offset: unused for swizzled K-major
+    d |= (uint64_t)(1024 >> 4) << 32;   // stride byte offset: next 8-row atom
+    d |= (uint64_t)1 << 46;             // sm_100 descriptor version
+    d |= (uint64_t)2 << 61;             // SWIZZLE_128B
+    return d;
+}
+
+__device__ __forceinline__ uint32_t pack2(float a, float b) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    return *(uint32_t *)&h;
+}
+
+__global__ void __launch_bounds__(192, 2) k_gemm_tc(const __grid_constant__ TmaMaps maps, const Epi epi, int K) {
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ uint64_t full[STAGES], empty[STAGES], accf;
+    __shared__ uint32_t tmem_base;
+    __shared__ int fail;
+    uint8_t *base = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int z = blockIdx.z;
+    const int m0 = blockIdx.y * BM, n0 = blockIdx.x * BN;
+    const int nk = K / BK;
+    if (tid == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            tc::mbar_init(&full[s], 1);
+            tc::mbar_init(&empty[s], 1);
+        }
+        tc::mbar_init(&accf, 1);
+        tc::fence_mbar_init();
+        fail = 0;
+    }
+    if (warp == 1) {
+        tc::tmem_alloc(&tmem_base, BN);
+        tc::tmem_relinquish();
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = tmem_base;
+
+    if (warp == 0 && lane == 0) {
+        // producer
+        for (int k = 0; k < nk; ++k) {
+            const int s = k % STAGES;
+            const uint32_t ph = (k / STAGES) & 1;
+            if (k >= STAGES && !tc::mbar_wait(&empty[s], ph ^ 1)) { fail = 1; break; }
+            uint8_t *sa = base + s * A_BYTES;
+            uint8_t *sb = base + STAGES * A_BYTES + s * B_BYTES;
+            mbar_expect_tx(&full[s], A_BYTES + B_BYTES);
+            tma_load_2d(sa, &maps.a, k * BK, m0, &full[s]);
+            tma_load_2d(sb, &maps.b[z], k * BK, n0, &full[s]);
+        }
+    } else if (warp == 1 && lane == 0) {
+        // MMA issuer
+        const uint32_t id = tc::idesc_bf16(BM, BN);
+        bool ok = true;
+        for (int k = 0; k < nk; ++k) {
+            const int s = k % STAGES;
+            const uint32_t ph = (k / STAGES) & 1;
+            if (!tc::mbar_wait(&full[s], ph)) { ok = false; fail = 1; break; }
+            tc::fence_after_sync();
+            const uint32_t sa = tc::smem_u32(base + s * A_BYTES);
+            const uint32_t sb = tc::smem_u32(base + STAGES * A_BYTES + s * B_BYTES);
+#pragma unroll
+            for (int kk = 0; kk < BK / 16; ++kk)
+                tc::mma_bf16(tmem, desc_sw128(sa + 32 * kk), desc_sw128(sb + 32 * kk), id, (k | kk) != 0);
+            tc::commit(&empty[s]);
+        }
+        if (ok) tc::commit(&accf);
+    } else if (warp >= 2) {
+        // epilogue: warp w reads TMEM lanes 32*(w%4) .. +31 = tile rows
+        const int q = warp & 3;
+        const int row = q * 32 + lane;
+        const int m = m0 + row;
+        const bool ok = tc::mbar_wait(&accf, 0, 1u << 20);
+        tc::fence_after_sync();
+        const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16);
+        const int mode = epi.mode[z];
+        bf16 *out = epi.out[z];
+        const int half = epi.d / 2;
+        for (int c0 = 0; c0 < BN; c0 += 32) {
+            float v[32];
+            tc::tmem_ld32(trow + c0, v);
+            if (!ok || m >= epi.M) continue;
+            const int n = n0 + c0;
+            bf16 *dst;
+            if (mode == kEpiPlain) {
+                dst = out + (size_t)m * epi.N + n;
+            } else {
+                const int b = m / epi.S, t = m % epi.S;
+                const int h = n / epi.d, i0 = n % epi.d;
+                if (mode == kEpiRope) {
+                    const float2 *hi = epi.rope_hi + (size_t)(t / kRopeLo) * half + i0 / 2;
+                    const float2 *lo = epi.rope_lo + (size_t)(t % kRopeLo) * half + i0 / 2;
+#pragma unroll
+                    for (int pr = 0; pr < 16; ++pr) {
+                        const float2 a = __ldg(hi + pr), bb = __ldg(lo + pr);
+                        const float c = a.x * bb.x - a.y * bb.y, sn = a.y * bb.x + a.x * bb.y;
+                        const float x0 = v[2 * pr], x1 = v[2 * pr + 1];
+                        v[2 * pr] = x0 * c - x1 * sn;
+                        v[2 * pr + 1] = x0 * sn + x1 * c;
+                    }
+                }
+                dst = out + (((size_t)b * epi.H + h) * epi.S + t) * epi.d + i0;
+            }
+            uint4 *d4 = (uint4 *)dst;
+#pragma unroll
+            for (int q8 = 0; q8 < 4; ++q8)
+                d4[q8] = make_uint4(pack2(v[8 * q8], v[8 * q8 + 1]), pack2(v[8 * q8 + 2], v[8 * q8 + 3]),
+                                    pack2(v[8 * q8 + 4], v[8 * q8 + 5]), pack2(v[8 * q8 + 6], v[8 * q8 + 7]));
+        }
+        if (!ok && lane == 0) fail = 1;
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    if (tid == 0 && fail) record_error(epi.counters, kDevErrTimeout);
+    if (warp == 1) tc::tmem_dealloc(tmem, BN);
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+bool get_encode() {
+    std::call_once(g_encode_once, [] {
+        void *fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_encode = (PFN_cuTensorMapEncodeTiled_v12000)fn;
+    });
+    return g_encode != nullptr;
+}
+
+// rows x K bf16 row-major matrix, box 64 (K) x box_rows, 128-byte swizzle
+bool make_map(CUtensorMap *map, const void *ptr, long long rows, int K, int box_rows) {
+    cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+    cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+cudaError_t launch(const TmaMaps &maps, const Epi &epi, int nz, int K, cudaStream_t s) {
+    static bool attr_set = false;
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(k_gemm_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    dim3 grid(epi.N / BN, (epi.M + BM - 1) / BM, nz);
+    k_gemm_tc<<<grid, 192, SMEM_BYTES, s>>>(maps, epi, K);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+bool gemm_tc_supported(const mono_config &c) {
+    return c.dtype == MONO_BF16 && c.W % BK == 0 && (c.H * c.d) % BN == 0 && c.W % BN == 0 &&
+           (c.H * c.d) % BK == 0 && (long long)c.B * c.S < (1ll << 31);
+}
+
+cudaError_t launch_project_tc(const Plan &p, const void *x, const void *Wq, const void *Wk, const void *Wv, void *Q,
+                              void *K, void *V, const void *ws, cudaStream_t s) {
+    const mono_config &c = p.cfg;
+    if (!get_encode()) return cudaErrorNotSupported;
+    TmaMaps maps;
+    const long long M = (long long)c.B * c.S;
+    const int N = c.H * c.d;
+    if (!make_map(&maps.a, x, M, c.W, BM) || !make_map(&maps.b[0], Wq, N, c.W, BN) ||
+        !make_map(&maps.b[1], Wk, N, c.W, BN) || !make_map(&maps.b[2], Wv, N, c.W, BN))
+        return cudaErrorInvalidValue;
+    Epi epi{};
+    epi.out[0] = (bf16 *)Q; epi.out[1] = (bf16 *)K; epi.out[2] = (bf16 *)V;
+    epi.mode[0] = kEpiRope; epi.mode[1] = kEpiRope; epi.mode[2] = kEpiHeads;
+    epi.M = (int)M; epi.N = N; epi.S = c.S; epi.H = c.H; epi.d = c.d;
+    const int half = c.d / 2, nhi = (c.S + kRopeLo - 1) / kRopeLo;
+    epi.rope_hi = (const float2 *)ws_ptr(p, (void *)ws, kRegRope);
+    epi.rope_lo = epi.rope_hi + (size_t)nhi * half;
+    epi.counters = (unsigned long long *)ws_ptr(p, (void *)ws, kRegCounters);
+    return launch(maps, epi, 3, c.W, s);
+}
+
+cudaError_t launch_out_project_tc(const Plan &p, const void *O, const void *Wo, void *delta, void *ws, cudaStream_t s) {
+    const mono_config &c = p.cfg;
+    if (!get_encode()) return cudaErrorNotSupported;
+    TmaMaps maps;
+    const long long M = (long long)c.B * c.S;
+    const int Kd = c.H * c.d;
+    if (!make_map(&maps.a, O, M, Kd, BM) || !make_map(&maps.b[0], Wo, c.W, Kd, BN)) return cudaErrorInvalidValue;
+    maps.b[1] = maps.b[0];
+    maps.b[2] = maps.b[0];
+    Epi epi{};
+    epi.out[0] = (bf16 *)delta;
+    epi.mode[0] = kEpiPlain;
+    epi.M = (int)M; epi.N = c.W; epi.S = c.S; epi.H = c.H; epi.d = c.d;
+    epi.counters = (unsigned long long *)ws_ptr(p, ws, kRegCounters);
+    return launch(maps, epi, 1, Kd, s);
+}
+
+}  // namespace mono

@@ -50,8 +50,8 @@ enum Region {
     kRegPairs,       // [B*H*S*R] int32 (t*R + r) grouped by block
     kRegPartO,       // [B*H*S*R, d] bf16 remote partial outputs
     kRegPartML,      // [B*H*S*R] float2 (max, sum) of remote partials
-    kRegWork,        // [max_work] int2 (bucket, chunk) work items of the remote kernel
-    kRegNWork,       // int32 number of work items
+    kRegWork,        // [B*H, max_work] int2 (block, chunk) work items of the remote kernel
+    kRegNWork,       // [B*H] int32 number of work items
     kRegN
 };
 
@@ -61,7 +61,8 @@ struct Plan {
     long long A;   // C^M
     int es;        // bytes per stored element (4 or 2)
     bool fast;     // tensor-core attention applies
-    int max_work;  // upper bound on remote work items
+    bool gemm_tc;  // tensor-core projections apply
+    int max_work;  // upper bound on remote work items per (b, h)
     size_t off[kRegN];
     size_t bytes[kRegN];
     size_t ws_bytes;
@@ -98,7 +99,16 @@ cudaError_t launch_queries(const Plan &p, const void *Q, const float *cb, const 
 cudaError_t launch_attend_simt(const Plan &p, const void *Q, const void *K, const void *V, const int32_t *sel,
                                void *O, void *ws, cudaStream_t s);
 bool attend_tc_supported(const mono_config &c);
+bool gemm_tc_supported(const mono_config &c);
+cudaError_t launch_project_tc(const Plan &p, const void *x, const void *Wq, const void *Wk, const void *Wv, void *Q,
+                              void *K, void *V, const void *ws, cudaStream_t s);
+cudaError_t launch_out_project_tc(const Plan &p, const void *O, const void *Wo, void *delta, void *ws, cudaStream_t s);
 cudaError_t launch_attend_tc(const Plan &p, const void *Q, const void *K, const void *V, const int32_t *sel, void *O,
                              void *ws, cudaStream_t s);
 
 }  // namespace mono
+
+// the opaque plan handle of the C-ABI
+struct mono_plan_s {
+    mono::Plan p;
+};

@@ -17,6 +17,7 @@
 // The explicit __fadd_rn / __fmaf_rn / __fdiv_rn intrinsics keep the compiler
 // from contracting or reordering that arithmetic.
 #include "internal.cuh"
+#include "tc.cuh"
 
 namespace mono {
 
@@ -78,40 +79,33 @@ __global__ void __launch_bounds__(128) k_summary_assign_w(const T *__restrict__ 
                                                           float *__restrict__ kbar, int32_t *__restrict__ addr, int S,
                                                           int Bs, int M, int C, int H) {
     constexpr int PER = D / 32;  // columns per lane
-    extern __shared__ float sm[];
-    float *s_cb = sm;                         // [C*D]
-    float *s_kb = s_cb + C * D;               // [4][D]
-    float *s_sc = s_kb + 4 * D;               // [4][M*C]
+    extern __shared__ __align__(16) float sm[];
+    float *s_cb = sm;                              // [C*D]
+    float *s_kb = s_cb + C * D;                    // [4][D]
+    float *s_sc = s_kb + 4 * D;                    // [4][M*C]
+    T *s_rows = (T *)(s_sc + 4 * M * C);           // [4][Bs*D] staged block rows
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int h = blockIdx.y, b = blockIdx.z;
     const int nb = S / Bs;
     const size_t bh = (size_t)b * H + h;
-    for (int i = threadIdx.x; i < C * D; i += blockDim.x) s_cb[i] = cb[(size_t)h * C * D + i];
     const int j = blockIdx.x * 4 + warp;
-    float acc[PER];
-#pragma unroll
-    for (int e = 0; e < PER; ++e) acc[e] = 0.0f;
+    // every copy of this warp's block in flight at once
+    const int chunks = Bs * D * (int)sizeof(T) / 16;
+    T *rows = s_rows + (size_t)warp * Bs * D;
     if (j < nb) {
-        const T *Kb = K + (bh * S + (size_t)j * Bs) * D + lane * PER;
-#pragma unroll 8
+        const uint8_t *src = (const uint8_t *)(K + (bh * S + (size_t)j * Bs) * D);
+        for (int c = lane; c < chunks; c += 32) tc::cp_async16((uint8_t *)rows + 16 * c, src + 16 * c, true);
+    }
+    for (int i = threadIdx.x; i < C * D; i += blockDim.x) s_cb[i] = cb[(size_t)h * C * D + i];
+    tc::cp_async_wait_all();
+    __syncwarp();
+    if (j < nb) {
+        float acc[PER];
+#pragma unroll
+        for (int e = 0; e < PER; ++e) acc[e] = 0.0f;
         for (int t = 0; t < Bs; ++t) {
-            float x[PER];
-            if constexpr (sizeof(T) == 2) {
-                if constexpr (PER == 2) {
-                    float2 f = __bfloat1622float2(*(const __nv_bfloat162 *)(Kb + (size_t)t * D));
-                    x[0] = f.x; x[1] = f.y;
-                } else {
-                    uint2 u = __ldg((const uint2 *)(Kb + (size_t)t * D));
-                    float2 f0 = __bfloat1622float2(*(const __nv_bfloat162 *)&u.x);
-                    float2 f1 = __bfloat1622float2(*(const __nv_bfloat162 *)&u.y);
-                    x[0] = f0.x; x[1] = f0.y; x[2] = f1.x; x[3] = f1.y;
-                }
-            } else {
 #pragma unroll
-                for (int e = 0; e < PER; ++e) x[e] = __ldg(Kb + (size_t)t * D + e);
-            }
-#pragma unroll
-            for (int e = 0; e < PER; ++e) acc[e] = __fadd_rn(acc[e], x[e]);
+            for (int e = 0; e < PER; ++e) acc[e] = __fadd_rn(acc[e], to_f(rows[(size_t)t * D + lane * PER + e]));
         }
 #pragma unroll
         for (int e = 0; e < PER; ++e) {
@@ -610,31 +604,34 @@ __global__ void __launch_bounds__(128) k_probe_m2(const T *__restrict__ Q, const
                 q[4 * c] = f.x; q[4 * c + 1] = f.y; q[4 * c + 2] = f.z; q[4 * c + 3] = f.w;
             }
         }
-        // subspace scores (fma chains in ascending element order)
+        // subspace scores: 2C independent fma chains, each in ascending element
+        // order, advanced together four elements at a time (same results as one
+        // chain after another, with 2C-way instruction-level parallelism)
         float s0[C], s1[C];
+#pragma unroll
+        for (int c = 0; c < C; ++c) { s0[c] = 0.0f; s1[c] = 0.0f; }
+#pragma unroll
+        for (int i4 = 0; i4 < DM / 4; ++i4) {
+#pragma unroll
+            for (int c = 0; c < C; ++c) {
+                const float4 x = ((const float4 *)(s_cb + (0 * C + c) * DM))[i4];
+                const float4 y = ((const float4 *)(s_cb + (1 * C + c) * DM))[i4];
+                s0[c] = __fmaf_rn(q[4 * i4 + 0], x.x, s0[c]);
+                s0[c] = __fmaf_rn(q[4 * i4 + 1], x.y, s0[c]);
+                s0[c] = __fmaf_rn(q[4 * i4 + 2], x.z, s0[c]);
+                s0[c] = __fmaf_rn(q[4 * i4 + 3], x.w, s0[c]);
+                s1[c] = __fmaf_rn(q[DM + 4 * i4 + 0], y.x, s1[c]);
+                s1[c] = __fmaf_rn(q[DM + 4 * i4 + 1], y.y, s1[c]);
+                s1[c] = __fmaf_rn(q[DM + 4 * i4 + 2], y.z, s1[c]);
+                s1[c] = __fmaf_rn(q[DM + 4 * i4 + 3], y.w, s1[c]);
+            }
+        }
         float mx0 = 0.f, mx1 = 0.f;
 #pragma unroll
         for (int c = 0; c < C; ++c) {
-            const float4 *w0 = (const float4 *)(s_cb + (0 * C + c) * DM);
-            const float4 *w1 = (const float4 *)(s_cb + (1 * C + c) * DM);
-            float a0 = 0.0f, a1 = 0.0f;
-#pragma unroll
-            for (int i4 = 0; i4 < DM / 4; ++i4) {
-                const float4 x = w0[i4], y = w1[i4];
-                a0 = __fmaf_rn(q[4 * i4 + 0], x.x, a0);
-                a0 = __fmaf_rn(q[4 * i4 + 1], x.y, a0);
-                a0 = __fmaf_rn(q[4 * i4 + 2], x.z, a0);
-                a0 = __fmaf_rn(q[4 * i4 + 3], x.w, a0);
-                a1 = __fmaf_rn(q[DM + 4 * i4 + 0], y.x, a1);
-                a1 = __fmaf_rn(q[DM + 4 * i4 + 1], y.y, a1);
-                a1 = __fmaf_rn(q[DM + 4 * i4 + 2], y.z, a1);
-                a1 = __fmaf_rn(q[DM + 4 * i4 + 3], y.w, a1);
-            }
-            s0[c] = a0;
-            s1[c] = a1;
-            s_s0[c * 128 + tid] = a0;
-            mx0 = fmaxf(mx0, fabsf(a0));
-            mx1 = fmaxf(mx1, fabsf(a1));
+            s_s0[c * 128 + tid] = s0[c];
+            mx0 = fmaxf(mx0, fabsf(s0[c]));
+            mx1 = fmaxf(mx1, fabsf(s1[c]));
         }
         int e2;
         frexpf(2.f * (mx0 + mx1) + 1e-30f, &e2);
@@ -682,8 +679,9 @@ __global__ void __launch_bounds__(128) k_probe_m2(const T *__restrict__ Q, const
         RegTop<R> rk;
         rk.init();
         int nc = 0;
-#pragma unroll 1
-        for (int r = 0; r < TP && nc < E; ++r) {
+#pragma unroll
+        for (int r = 0; r < TP; ++r) {
+            if (nc >= E) break;
             const int a = top.a[r];
             int lo = 0, hi = nb;
             while (lo < hi) {
@@ -765,7 +763,8 @@ cudaError_t launch_summaries(const Plan &p, const void *K, const float *cb, void
     unsigned long long *cnt = (unsigned long long *)ws_ptr(p, ws, kRegCounters);
     cudaError_t e = cudaMemsetAsync(cnt, 0, kCntN * 8, s);
     if (e != cudaSuccess) return e;
-    const size_t smem = ((size_t)c.C * c.d + 4 * (size_t)c.d + 4 * (size_t)c.M * c.C) * 4;
+    const size_t smem = ((size_t)c.C * c.d + 4 * (size_t)c.d + 4 * (size_t)c.M * c.C) * 4 +
+                        4 * (size_t)c.Bs * c.d * p.es;
     dim3 g1((p.nb + 3) / 4, c.H, c.B);
 #define MONO_SUMW(TT, DD)                                                                                         \
     do {                                                                                                          \

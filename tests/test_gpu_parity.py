@@ -139,6 +139,13 @@ def test_tensor_core_attention_edge_cases():
     full_check(run)
 
 
+@pytest.mark.parametrize("B,S,W,H,d", [(1, 832, 256, 2, 64), (2, 640, 384, 1, 128), (1, 1024, 128, 4, 64)])
+def test_tensor_core_projections(B, S, W, H, d):
+    # ragged token count (B*S not a multiple of the 128-row tile), several K and N
+    cfg = small(B=B, S=S, W=W, H=H, d=d, Bs=64, C=8, cap=6, dtype="bf16")
+    full_check(Run(cfg, seed=30 + W))
+
+
 def test_simple_and_tensor_core_paths_agree():
     from learned_product_hash_proj_b200 import mono
     cfg = small(S=1024, Bs=64, C=16, cap=8, dtype="bf16")
