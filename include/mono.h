@@ -62,7 +62,8 @@ enum mono_status {
     MONO_ERR_WORKSPACE = 4,   /* workspace pointer missing */
     MONO_ERR_CUDA = 5,        /* a CUDA runtime call or kernel launch failed */
     MONO_ERR_DEVICE = 6,      /* a kernel recorded an error in the device error word */
-    MONO_ERR_ALIGN = 7        /* a pointer is not suitably aligned */
+    MONO_ERR_ALIGN = 7,       /* a pointer is not suitably aligned */
+    MONO_ERR_SCRATCH = 8      /* the problem needs more than mono_route_static's fixed scratch array */
 };
 
 /* Plan options (mono_config.flags). */
@@ -166,6 +167,29 @@ int mono_route_summaries(const mono_plan_t *plan, const void *K, const float *co
 int mono_route_lists(const mono_plan_t *plan, void *workspace, void *stream);
 int mono_route_queries(const mono_plan_t *plan, const void *Q, const float *codebooks, const int32_t *forced,
                        int32_t *sel, void *workspace, void *stream);
+
+/* mono_route without a workspace, for callers that cannot allocate device
+ * memory (a plugin whose host framework owns every device allocation, or a
+ * serving loop that forbids cudaMalloc after start-up).  There is no
+ * counterpart on the pages: this is a deployment convenience of this library.
+ * Same kernels and same results as mono_route; inputs Q, K, codebooks,
+ * optional forced; output sel.  The routing tables live in one array of
+ * mono_route_static_capacity() bytes (16 MiB) that the library places in the
+ * global memory of every GPU it is loaded on, for the life of the process.
+ * The tables need B*H*nb*(d + 16) + B*H*4 bytes plus alignment; a larger
+ * problem returns MONO_ERR_SCRATCH before anything is launched.
+ * The first call on a device looks the array's device address up
+ * (cudaGetSymbolAddress, with that device current) and caches it, so make
+ * the first call on each device before any stream capture.  All calls on a
+ * device share the array: calls that overlap on the GPU (other streams or
+ * threads) race and must be serialised by the caller.  Each call clears the
+ * statistics counters it uses and overwrites the tables.  No memory is
+ * allocated by this entry point. */
+int mono_route_static(const mono_plan_t *plan, const void *Q, const void *K, const float *codebooks,
+                      const int32_t *forced, int32_t *sel, void *stream);
+
+/* Size in bytes of the fixed array behind mono_route_static. */
+size_t mono_route_static_capacity(void);
 
 /* Exact causal softmax over the selected token set (aitechinspire.com
  * article, Snapshot): for query t of block bq, the tokens of the blocks in

@@ -118,6 +118,7 @@ const char *mono_strerror(int s) {
         case MONO_ERR_CUDA: return "a CUDA call or kernel launch failed";
         case MONO_ERR_DEVICE: return "a kernel recorded a device error";
         case MONO_ERR_ALIGN: return "a pointer is not suitably aligned";
+        case MONO_ERR_SCRATCH: return "problem too large for the fixed scratch array of mono_route_static";
         default: return "unknown status";
     }
 }

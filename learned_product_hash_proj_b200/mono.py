@@ -24,13 +24,14 @@ _lib = ctypes.CDLL(LIB_PATH)
 MONO_F32, MONO_BF16 = 0, 1
 MONO_FLAG_SIMPLE_KERNELS = 1
 STATUS = {0: "MONO_OK", 1: "MONO_ERR_INVALID", 2: "MONO_ERR_UNSUPPORTED", 3: "MONO_ERR_NULL",
-          4: "MONO_ERR_WORKSPACE", 5: "MONO_ERR_CUDA", 6: "MONO_ERR_DEVICE", 7: "MONO_ERR_ALIGN"}
+          4: "MONO_ERR_WORKSPACE", 5: "MONO_ERR_CUDA", 6: "MONO_ERR_DEVICE", 7: "MONO_ERR_ALIGN", 8: "MONO_ERR_SCRATCH"}
 REGIONS = {"kbar": 0, "addr": 1, "post_ids": 2, "post_addr": 3, "post_rank": 4, "overflow": 5, "Q": 6, "K": 7,
            "V": 8, "sel": 9, "O": 10}
 
 EXPORTS = ("mono_plan", "mono_plan_destroy", "mono_workspace_region", "mono_project", "mono_route",
            "mono_route_summaries", "mono_route_lists", "mono_route_queries", "mono_attend",
-           "mono_out_project", "mono_forward", "mono_stats", "mono_strerror", "mono_version", "mono_kernel_launches")
+           "mono_out_project", "mono_forward", "mono_stats", "mono_strerror", "mono_version", "mono_kernel_launches",
+           "mono_route_static", "mono_route_static_capacity")
 
 
 class MonoError(RuntimeError):
@@ -73,6 +74,10 @@ _lib.mono_stats.argtypes = [_P, _P, _P, ctypes.POINTER(Stats)]
 _lib.mono_strerror.argtypes = [ctypes.c_int]
 _lib.mono_strerror.restype = ctypes.c_char_p
 _lib.mono_version.argtypes = []
+_lib.mono_route_static.argtypes = [_P] * 7
+_lib.mono_route_static.restype = ctypes.c_int
+_lib.mono_route_static_capacity.argtypes = []
+_lib.mono_route_static_capacity.restype = ctypes.c_size_t
 _lib.mono_kernel_launches.argtypes = []
 _lib.mono_kernel_launches.restype = ctypes.c_ulonglong
 for _f in ("mono_plan", "mono_workspace_region", "mono_project", "mono_route", "mono_route_summaries",
@@ -206,6 +211,21 @@ def route_queries(plan: Plan, Q, codebooks, sel, ws, forced=None, stream=None):
                                    _ptr(forced, "forced", (c.B, c.H, c.S), torch.int32, optional=True),
                                    _ptr(sel, "sel", (c.B, c.H, c.S, c.R), torch.int32), _ptr(ws, "workspace"),
                                    _stream(stream)), "mono_route_queries")
+
+
+def route_static(plan: Plan, Q, K, codebooks, sel, forced=None, stream=None):
+    """mono_route without a workspace, for callers that cannot allocate device memory.
+
+    The routing tables live in a fixed array owned by the library (see
+    mono_route_static in include/mono.h); calls that overlap on the GPU race.
+    """
+    c, dt = plan.cfg, plan.dtype
+    qkv = (c.B, c.H, c.S, c.d)
+    _check(_lib.mono_route_static(plan.handle, _ptr(Q, "Q", qkv, dt), _ptr(K, "K", qkv, dt),
+                                  _ptr(codebooks, "codebooks", (c.H, c.M, c.C, c.d // c.M), torch.float32),
+                                  _ptr(forced, "forced", (c.B, c.H, c.S), torch.int32, optional=True),
+                                  _ptr(sel, "sel", (c.B, c.H, c.S, c.R), torch.int32), _stream(stream)),
+           "mono_route_static")
 
 
 def attend(plan: Plan, Q, K, V, sel, O, ws, stream=None):
