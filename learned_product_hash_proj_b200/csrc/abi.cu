@@ -69,7 +69,7 @@ void layout(Plan *p) {
         bytes[kRegPairs] = B * H * S * R * 4;
         bytes[kRegPartO] = B * H * S * R * d * 2;
         bytes[kRegPartML] = B * H * S * R * 8;
-        bytes[kRegWork] = B * H * (size_t)p->max_work * 8;
+        bytes[kRegWork] = B * H * (size_t)p->max_work * 16;
         bytes[kRegNWork] = B * H * 4;
     }
     size_t off = 0;

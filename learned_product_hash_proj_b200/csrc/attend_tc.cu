@@ -18,6 +18,8 @@
 //     masked tile gives S and O.  The same CTA then reads the R remote
 //     partials of each query and merges them.
 // Scores are kept in the log2 domain: s2 = <q,k> * log2(e)/sqrt(d).
+#include <algorithm>
+
 #include "internal.cuh"
 #include "tc.cuh"
 
@@ -35,6 +37,8 @@ __device__ __forceinline__ bool sel_valid(int j, int t, int Bs, int L) { return 
 // one global atomic per distinct block per CTA instead of one per pair.
 // ---------------------------------------------------------------------------
 constexpr int kChunk = 128;   // queries per remote work item
+constexpr size_t kL2GroupBytes = 88u << 20;  // partials + Q/K/V of one launch group, under the 126 MB L2
+constexpr int kMaxGroup = 256;               // (b, h) slices per launch group
 constexpr int kQTile = 1024;  // queries per CTA of the count and fill kernels
 
 // grid (ceil(S/kQTile), B*H), 256 threads, smem nb ints
@@ -60,9 +64,10 @@ __global__ void __launch_bounds__(256) k_pair_count(const int32_t *__restrict__ 
 }
 
 // exclusive scan of one (b, h)'s bucket sizes, fill cursors reset, and one
-// work item per chunk of <= kChunk queries.  grid B*H, 1024 threads.
+// work item {block, first pair, pair count, 0} per chunk of <= kChunk
+// queries.  grid B*H, 1024 threads.
 __global__ void __launch_bounds__(1024) k_pair_scan(const int32_t *__restrict__ cnt, int32_t *__restrict__ start,
-                                                    int32_t *__restrict__ fill, int2 *__restrict__ work,
+                                                    int32_t *__restrict__ fill, int4 *__restrict__ work,
                                                     int32_t *__restrict__ nwork, int nb, int wcap) {
     __shared__ int s_w[32], s_c[32];
     __shared__ int carry_p, carry_c;
@@ -99,7 +104,8 @@ __global__ void __launch_bounds__(1024) k_pair_scan(const int32_t *__restrict__ 
         if (j < nb) {
             start[bh * nb + j] = off_p;
             fill[bh * nb + j] = 0;
-            for (int k = 0; k < ch; ++k) work[bh * wcap + off_c + k] = make_int2(j, k);
+            for (int k = 0; k < ch; ++k)
+                work[bh * wcap + off_c + k] = make_int4(j, off_p + k * kChunk, min(kChunk, c - k * kChunk), 0);
         }
         __syncthreads();
         if (threadIdx.x == 0) {
@@ -151,25 +157,26 @@ __device__ __forceinline__ uint4 ldg16(const void *p) { return __ldg((const uint
 
 // rows [0, nrows) of a [*, D] bf16 matrix -> K-major tile (kdim = D); rows >= valid are zero.
 // Asynchronous: every copy is in flight at once; complete with cp_async_wait_all.
+// Thread idx copies chunk c of row 8g + r8 with (r8, c, g) = (idx % 8, idx / 8 % (D/8), idx / D):
+// its destination kmajor_chunk(row, c, D) is exactly 16 * idx, so a warp writes 512 contiguous bytes.
 template <int D>
 __device__ __forceinline__ void load_rows(uint8_t *tile, const bf16 *src, int nrows, int valid, int tid, int nthr) {
     for (int idx = tid; idx < nrows * (D / 8); idx += nthr) {
-        const int row = idx / (D / 8), c = idx % (D / 8);
+        const int row = (idx / D) * 8 + (idx & 7), c = (idx >> 3) % (D / 8);
         const bool ok = row < valid;
-        tc::cp_async16(tile + tc::kmajor_chunk(row, c, D), ok ? (const void *)(src + (size_t)row * D + 8 * c) : src,
-                       ok);
+        tc::cp_async16(tile + 16 * idx, ok ? (const void *)(src + (size_t)row * D + 8 * c) : src, ok);
     }
 }
 
 // rows [0, nkeys) of V ([*, D]) -> MN-major tile for the B operand of O = P V
 // (K = keys, N = dims); rows >= valid are zero.  Whole 16-byte chunks, no transpose.
+// Thread idx copies chunk c = idx / nkeys of key idx % nkeys: destination mnmajor_chunk = 16 * idx.
 template <int D>
 __device__ __forceinline__ void load_v(uint8_t *tile, const bf16 *src, int nkeys, int valid, int tid, int nthr) {
     for (int idx = tid; idx < nkeys * (D / 8); idx += nthr) {
-        const int key = idx / (D / 8), c = idx % (D / 8);
+        const int key = idx % nkeys, c = idx / nkeys;
         const bool ok = key < valid;
-        tc::cp_async16(tile + tc::mnmajor_chunk(key, c, nkeys),
-                       ok ? (const void *)(src + (size_t)key * D + 8 * c) : src, ok);
+        tc::cp_async16(tile + 16 * idx, ok ? (const void *)(src + (size_t)key * D + 8 * c) : src, ok);
     }
 }
 
@@ -183,169 +190,263 @@ __device__ __forceinline__ bool timed_out(const unsigned long long *counters) {
 }
 
 // ---------------------------------------------------------------------------
-// remote partials: one CTA per (b, h, block j, chunk of <= 128 queries)
+// remote partials: persistent CTAs of 256 threads walk the work items
+// {block j, first pair, pair count} of a group of (b, h) slices with a
+// two-stage pipeline: while item k is computed, the tiles of item k+1 are in
+// flight (cp.async) and the descriptor and pair ids of item k+2 are being
+// loaded.  Per item: S = Q_sel K_j^T and O = P V_j on tcgen05 (TMEM, 64 or
+// 128 columns reused by every item), softmax in fp32, one partial per pair.
+// As in the local kernel, warps q and q+4 share TMEM lane quarter q and split
+// the columns.
 // ---------------------------------------------------------------------------
+struct RemoteItem {
+    long long bh;
+    int j, p0, n;
+};
+
 template <int D, int BS>
-__global__ void __launch_bounds__(128) k_remote_tc(const bf16 *__restrict__ Q, const bf16 *__restrict__ K,
+__global__ void __launch_bounds__(256) k_remote_tc(const bf16 *__restrict__ Q, const bf16 *__restrict__ K,
                                                    const bf16 *__restrict__ V, const int32_t *__restrict__ pairs,
-                                                   const int32_t *__restrict__ start, const int32_t *__restrict__ cnt,
-                                                   const int2 *__restrict__ work, const int32_t *__restrict__ nwork,
+                                                   const int4 *__restrict__ work, const int32_t *__restrict__ nwork,
                                                    bf16 *__restrict__ part_o, float2 *__restrict__ part_ml,
-                                                   unsigned long long *__restrict__ counters, int S, int R, int nb,
-                                                   int wcap, float scale_log2) {
+                                                   unsigned long long *__restrict__ counters, int S, int R, int wcap,
+                                                   float scale_log2, int bh0, int ng) {
     // TMEM: S in columns [0, BS); O overwrites them once every thread has turned S into P
     constexpr int NCOLS = (BS > D ? BS : D) <= 64 ? 64 : 128;
+    constexpr int HALF = BS / 2, DH = D / 2;
+    static_assert(HALF % 32 == 0 && DH % 32 == 0, "tile shape");
+    constexpr int QB = 128 * D * 2, KB = BS * D * 2, VB = BS * D * 2, PB = 128 * BS * 2;
+    constexpr int STAGE = QB + KB + VB;
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ uint64_t mbar;
     __shared__ uint32_t tmem_base;
-    const long long bh = blockIdx.y;
-    const int item = blockIdx.x;
-    if (item >= nwork[bh] || timed_out(counters)) return;
-    const int tid = threadIdx.x, warp = tid >> 5;
-    const int2 w = work[bh * wcap + item];
-    const int j = w.x;
-    const size_t bj = (size_t)bh * nb + j;
-    const int p0 = start[bj] + w.y * kChunk;
-    const int n = min(kChunk, cnt[bj] - w.y * kChunk);
-    pairs += (size_t)bh * S * R;
+    __shared__ float s_red[2][128];
+    __shared__ int s_pref[kMaxGroup + 1];
+    if (timed_out(counters)) return;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quarter = warp & 3, half = warp >> 2;
+    const int row = quarter * 32 + lane;
 
-    // P reuses Q's space when it fits: Q is only read by the first MMA, which has completed when P is written
-    constexpr int QB = 128 * D * 2, KB = BS * D * 2, VB = BS * D * 2, PB = 128 * BS * 2;
-    uint8_t *sQ = smem;                       // [128 x D]
-    uint8_t *sK = sQ + QB;                    // [BS x D]
-    uint8_t *sVt = sK + KB;                   // V_j, MN-major [BS keys x D]
-    uint8_t *sP = PB <= QB ? sQ : sVt + VB;   // [128 x BS]
-
+    if (tid == 0) {
+        int acc = 0;
+        for (int g = 0; g < ng; ++g) { s_pref[g] = acc; acc += nwork[bh0 + g]; }
+        s_pref[ng] = acc;
+        tc::mbar_init(&mbar, 1);
+        tc::fence_mbar_init();
+    }
     if (warp == 0) {
         tc::tmem_alloc(&tmem_base, NCOLS);
         tc::tmem_relinquish();
     }
-    if (tid == 0) {
-        tc::mbar_init(&mbar, 1);
-        tc::fence_mbar_init();
-    }
-    // gather the selecting queries' rows, and block j's keys and values
-    int pr = 0;
-    if (tid < n) pr = pairs[p0 + tid];
-    const int t = pr / R;
-    {
-        const bf16 *qrow = Q + ((size_t)bh * S + t) * D;
-#pragma unroll
-        for (int c = 0; c < D / 8; ++c) tc::cp_async16(sQ + tc::kmajor_chunk(tid, c, D), qrow + 8 * c, tid < n);
-    }
-    const size_t kv0 = ((size_t)bh * S + (size_t)j * BS) * D;
-    load_rows<D>(sK, K + kv0, BS, BS, tid, 128);
-    load_v<D>(sVt, V + kv0, BS, BS, tid, 128);
-    tc::cp_async_wait_all();
-    tc::fence_smem_to_async();
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tmem = tmem_base;
-    const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
+    const uint32_t trow = tmem + ((uint32_t)(quarter * 32) << 16);
+    const int total = s_pref[ng];
+    const int G = gridDim.x;
 
-    if (tid == 0) {
-        const uint32_t id = tc::idesc_bf16(128, BS);
-        const uint32_t aq = tc::smem_u32(sQ), bk = tc::smem_u32(sK);
+    auto descr = [&](int f) {
+        int lo = 0, hi = ng;  // last g with s_pref[g] <= f
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (s_pref[mid] <= f) lo = mid;
+            else hi = mid;
+        }
+        const long long bh = bh0 + lo;
+        const int4 w = work[bh * wcap + (f - s_pref[lo])];
+        RemoteItem it;
+        it.bh = bh; it.j = w.x; it.p0 = w.y; it.n = w.z;
+        return it;
+    };
+    auto pair_of = [&](const RemoteItem &it) { return row < it.n ? pairs[it.bh * S * R + it.p0 + row] : 0; };
+    auto issue = [&](int stage, const RemoteItem &it, int pr) {
+        uint8_t *sQ = smem + stage * STAGE, *sK = sQ + QB, *sV = sK + KB;
+        const bf16 *qrow = Q + ((size_t)it.bh * S + pr / R) * D;
 #pragma unroll
-        for (int k = 0; k < D / 16; ++k)
-            tc::mma_bf16(tmem, tc::desc_kmajor(aq + 256 * k, D), tc::desc_kmajor(bk + 256 * k, D), id, k > 0);
-        tc::commit(&mbar);
-    }
-    bool ok = tc::mbar_wait(&mbar, 0);
-    tc::fence_after_sync();
+        for (int c = half * (D / 16); c < (half + 1) * (D / 16); ++c)
+            tc::cp_async16(sQ + tc::kmajor_chunk(row, c, D), qrow + 8 * c, row < it.n);
+        const size_t kv0 = ((size_t)it.bh * S + (size_t)it.j * BS) * D;
+        load_rows<D>(sK, K + kv0, BS, BS, tid, 256);
+        load_v<D>(sV, V + kv0, BS, BS, tid, 256);
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    };
 
-    // softmax of this thread's row over the block's BS keys
-    float v[32];
-    float m = -INFINITY;
+    int f = blockIdx.x;
+    bool ok = true;
+    if (f < total) {
+        RemoteItem it0 = descr(f);
+        int pr0 = pair_of(it0);
+        issue(0, it0, pr0);
+        int f1 = f + G;
+        bool have1 = f1 < total;
+        RemoteItem it1{};
+        int pr1 = 0;
+        if (have1) { it1 = descr(f1); pr1 = pair_of(it1); }
+        for (int k = 0; ok; ++k) {
+            const int stage = k & 1;
+            if (have1) issue(stage ^ 1, it1, pr1);
+            const int f2 = f1 + G;
+            const bool have2 = have1 && f2 < total;
+            RemoteItem it2{};
+            if (have2) it2 = descr(f2);
+            if (have1) asm volatile("cp.async.wait_group 1;" ::: "memory");
+            else asm volatile("cp.async.wait_group 0;" ::: "memory");
+            tc::fence_smem_to_async();
+            tc::fence_before_sync();
+            __syncthreads();
+            tc::fence_after_sync();
+            const int pr2 = have2 ? pair_of(it2) : 0;   // consumed next iteration
+
+            uint8_t *sQ = smem + stage * STAGE, *sK = sQ + QB, *sV = sK + KB;
+            uint8_t *sP = PB <= QB ? sQ : smem + 2 * STAGE;
+            if (tid == 0) {
+                const uint32_t id = tc::idesc_bf16(128, BS);
+                const uint32_t aq = tc::smem_u32(sQ), bk = tc::smem_u32(sK);
 #pragma unroll
-    for (int c0 = 0; c0 < BS; c0 += 32) {
-        tc::tmem_ld32(trow + c0, v);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) m = fmaxf(m, v[i]);
-    }
-    const float m2 = m * scale_log2;
-    float l = 0.f;
-#pragma unroll
-    for (int c0 = 0; c0 < BS; c0 += 32) {
-        tc::tmem_ld32(trow + c0, v);
-#pragma unroll
-        for (int q8 = 0; q8 < 4; ++q8) {
-            uint32_t pk[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const float a = exp2f(fmaf(v[8 * q8 + 2 * u], scale_log2, -m2));
-                const float b = exp2f(fmaf(v[8 * q8 + 2 * u + 1], scale_log2, -m2));
-                l += a + b;
-                pk[u] = pack2(a, b);
+                for (int kk = 0; kk < D / 16; ++kk)
+                    tc::mma_bf16(tmem, tc::desc_kmajor(aq + 256 * kk, D), tc::desc_kmajor(bk + 256 * kk, D), id, kk > 0);
+                tc::commit(&mbar);
             }
-            *(uint4 *)(sP + tc::kmajor_chunk(tid, (c0 >> 3) + q8, BS)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-        }
-    }
-    tc::fence_smem_to_async();
-    tc::fence_before_sync();
-    __syncthreads();
-    tc::fence_after_sync();
-    if (tid == 0 && ok) {
-        const uint32_t id = tc::idesc_bf16(128, D, true);
-        const uint32_t ap = tc::smem_u32(sP), bv = tc::smem_u32(sVt);
+            ok = __syncthreads_and(tc::mbar_wait(&mbar, 0));   // CTA-uniform: the loop below has barriers
+            tc::fence_after_sync();
+            float v[32];
+            float m = -INFINITY;
 #pragma unroll
-        for (int k = 0; k < BS / 16; ++k)
-            tc::mma_bf16(tmem, tc::desc_kmajor(ap + 256 * k, BS), tc::desc_mnmajor(bv + 256 * k, BS), id, k > 0);
-        tc::commit(&mbar);
+            for (int c0 = half * HALF; c0 < half * HALF + HALF; c0 += 32) {
+                tc::tmem_ld32(trow + c0, v);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) m = fmaxf(m, v[i]);
+            }
+            s_red[half][row] = m;
+            __syncthreads();
+            m = fmaxf(s_red[0][row], s_red[1][row]);
+            const float m2 = m * scale_log2;
+            float l = 0.f;
+#pragma unroll
+            for (int c0 = half * HALF; c0 < half * HALF + HALF; c0 += 32) {
+                tc::tmem_ld32(trow + c0, v);
+#pragma unroll
+                for (int q8 = 0; q8 < 4; ++q8) {
+                    uint32_t pk[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const float a = exp2f(fmaf(v[8 * q8 + 2 * u], scale_log2, -m2));
+                        const float bb = exp2f(fmaf(v[8 * q8 + 2 * u + 1], scale_log2, -m2));
+                        l += a + bb;
+                        pk[u] = pack2(a, bb);
+                    }
+                    *(uint4 *)(sP + tc::kmajor_chunk(row, (c0 >> 3) + q8, BS)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                }
+            }
+            __syncthreads();  // every thread has read the maxima
+            s_red[half][row] = l;
+            tc::fence_smem_to_async();
+            tc::fence_before_sync();
+            __syncthreads();
+            tc::fence_after_sync();
+            l = s_red[0][row] + s_red[1][row];
+            if (tid == 0 && ok) {
+                const uint32_t id = tc::idesc_bf16(128, D, true);
+                const uint32_t ap = tc::smem_u32(sP), bv = tc::smem_u32(sV);
+#pragma unroll
+                for (int kk = 0; kk < BS / 16; ++kk)
+                    tc::mma_bf16(tmem, tc::desc_kmajor(ap + 256 * kk, BS), tc::desc_mnmajor(bv + 256 * kk, BS), id,
+                                 kk > 0);
+                tc::commit(&mbar);
+            }
+            ok = __syncthreads_and(ok && tc::mbar_wait(&mbar, 1));
+            tc::fence_after_sync();
+            const bool live = row < it0.n;
+            const size_t slot = (size_t)it0.bh * S * R + pr0;
+            const float inv = 1.f / l;
+#pragma unroll
+            for (int c0 = half * DH; c0 < half * DH + DH; c0 += 32) {
+                tc::tmem_ld32(trow + c0, v);
+                if (live && ok) {
+                    uint4 *dst = (uint4 *)(part_o + slot * D + c0);
+#pragma unroll
+                    for (int q8 = 0; q8 < 4; ++q8)
+                        dst[q8] = make_uint4(pack2(v[8 * q8] * inv, v[8 * q8 + 1] * inv),
+                                             pack2(v[8 * q8 + 2] * inv, v[8 * q8 + 3] * inv),
+                                             pack2(v[8 * q8 + 4] * inv, v[8 * q8 + 5] * inv),
+                                             pack2(v[8 * q8 + 6] * inv, v[8 * q8 + 7] * inv));
+                }
+            }
+            if (live && ok && half == 0) part_ml[slot] = make_float2(m2, l);
+            tc::fence_before_sync();
+            __syncthreads();  // the stage's tiles and TMEM are free again
+            tc::fence_after_sync();
+            if (!have1) break;
+            it0 = it1; pr0 = pr1;
+            it1 = it2; pr1 = pr2;
+            have1 = have2; f1 = f2;
+        }
+        asm volatile("cp.async.wait_group 0;" ::: "memory");
     }
-    if (ok) ok = tc::mbar_wait(&mbar, 1);
-    tc::fence_after_sync();
     if (!ok && tid == 0) record_error(counters, kDevErrTimeout);
-
-    // partial output of this (query, block) pair
-    const size_t slot = (size_t)bh * S * R + pr;
-    const float inv = 1.f / l;
-#pragma unroll
-    for (int c0 = 0; c0 < D; c0 += 32) {
-        tc::tmem_ld32(trow + c0, v);
-        if (tid < n && ok) {
-            uint4 *dst = (uint4 *)(part_o + slot * D + c0);
-#pragma unroll
-            for (int q8 = 0; q8 < 4; ++q8)
-                dst[q8] = make_uint4(pack2(v[8 * q8] * inv, v[8 * q8 + 1] * inv), pack2(v[8 * q8 + 2] * inv, v[8 * q8 + 3] * inv),
-                                     pack2(v[8 * q8 + 4] * inv, v[8 * q8 + 5] * inv), pack2(v[8 * q8 + 6] * inv, v[8 * q8 + 7] * inv));
-        }
-    }
-    if (tid < n && ok) part_ml[slot] = make_float2(m2, l);
     tc::fence_before_sync();
     __syncthreads();
     if (warp == 0) tc::tmem_dealloc(tmem, NCOLS);
 }
 
 // ---------------------------------------------------------------------------
-// local part + merge: one CTA per (b, h, tile of 128 queries)
+// local part + merge: persistent CTAs of 256 threads walk the 128-query tiles
+// of a group of (b, h) slices with a two-stage pipeline (the Q/K/V tiles of
+// tile k+1 are in flight while tile k is computed).  Per tile: S over the
+// tile's local key range (<= 256 keys) and O = P V on tcgen05, the masked
+// softmax in fp32, and the exact merge with the tile's remote partials.  TMEM
+// lane quarter q (rows 32q .. 32q+31) is read by warps q and q+4, each taking
+// half of the columns; their partial row max and sum meet in shared memory.
 // ---------------------------------------------------------------------------
-template <int D, int BS, int NK>
-__global__ void __launch_bounds__(128) k_local_merge_tc(const bf16 *__restrict__ Q, const bf16 *__restrict__ K,
+// Shared-memory plan of the local kernel: ST stages of {Q, K, V} tiles; P over
+// the current stage's Q/K once S is computed (else a region of its own); a
+// 1 KB row-exchange buffer in stage space that P leaves free (else past the
+// end).  Two stages when they fit, else one (no prefetch).
+__host__ __device__ constexpr int local_p_offset(int ST, int STAGE, int QB, int KB, int PB, int stage) {
+    return PB <= QB + KB ? stage * STAGE : ST * STAGE;
+}
+__host__ __device__ constexpr int local_red_offset(int ST, int STAGE, int QB, int KB, int PB, int stage) {
+    return PB > QB + KB ? stage * STAGE : (PB + 1024 <= QB + KB ? stage * STAGE + PB : ST * STAGE + 1024 * stage);
+}
+__host__ __device__ constexpr size_t local_bytes(int ST, int STAGE, int QB, int KB, int PB) {
+    return (size_t)ST * STAGE + (PB > QB + KB ? PB : 0) + (PB <= QB + KB && PB + 1024 > QB + KB ? 1024 * ST : 0);
+}
+template <int D, int NK>
+constexpr int local_stages() {
+    constexpr int QB = 128 * D * 2, KB = NK * D * 2, VB = D * NK * 2, PB = 128 * NK * 2, STAGE = QB + KB + VB;
+    // one stage: two single-buffered CTAs per SM hide each other's load latency
+    // better than one double-buffered CTA (measured at the headline shape)
+    return local_bytes(2, STAGE, QB, KB, PB) <= 110 * 1024 ? 2 : 1;
+}
+template <int D, int NK>
+constexpr size_t local_smem() {
+    constexpr int QB = 128 * D * 2, KB = NK * D * 2, VB = D * NK * 2, PB = 128 * NK * 2, STAGE = QB + KB + VB;
+    return local_bytes(local_stages<D, NK>(), STAGE, QB, KB, PB);
+}
+
+template <int D, int BS, int NK, int RMAX>
+__global__ void __launch_bounds__(256) k_local_merge_tc(const bf16 *__restrict__ Q, const bf16 *__restrict__ K,
                                                         const bf16 *__restrict__ V, const int32_t *__restrict__ sel,
                                                         const bf16 *__restrict__ part_o,
                                                         const float2 *__restrict__ part_ml, bf16 *__restrict__ O,
                                                         unsigned long long *__restrict__ counters, int S, int H, int R,
-                                                        int L, float scale_log2) {
+                                                        int L, float scale_log2, int bh0, int ng) {
     constexpr int NCOLS = NK <= 128 ? 128 : 256;  // S: [0, NK); O reuses [0, D) after the softmax
-    static_assert(NK <= 256 && NK % 32 == 0 && D <= NK, "tile shape");
+    constexpr int HALF = NK / 2, DH = D / 2;
+    static_assert(NK <= 256 && HALF % 32 == 0 && DH % 32 == 0 && D <= NK, "tile shape");
+    constexpr int QB = 128 * D * 2, KB = NK * D * 2, VB = D * NK * 2, PB = 128 * NK * 2, STAGE = QB + KB + VB;
+    constexpr int ST = local_stages<D, NK>();
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ uint64_t mbar;
     __shared__ uint32_t tmem_base;
     if (timed_out(counters)) return;
-    const int tid = threadIdx.x, warp = tid >> 5;
-    const int h = blockIdx.y, b = blockIdx.z;
-    const long long bh = (long long)b * H + h;
-    const int t0 = blockIdx.x * 128;
-    const int nq = min(128, S - t0);
-    const int kstart = max(0, t0 / BS - L + 1) * BS;
-    const int kend = min(S, t0 + 128);
-    const int nk = kend - kstart;
-
-    constexpr int QB = 128 * D * 2, KB = NK * D * 2, VB = D * NK * 2, PB = 128 * NK * 2;
-    uint8_t *sQ = smem, *sK = smem + QB, *sVt = smem + QB + KB;
-    uint8_t *sP = (PB <= QB + KB) ? smem : smem + QB + KB + VB;  // P reuses Q/K once S is computed
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quarter = warp & 3, half = warp >> 2;
+    const int row = quarter * 32 + lane;
+    const int ntiles = (S + 127) / 128;
+    const int total = ng * ntiles;
+    const int G = gridDim.x;
 
     if (warp == 0) {
         tc::tmem_alloc(&tmem_base, NCOLS);
@@ -355,158 +456,224 @@ __global__ void __launch_bounds__(128) k_local_merge_tc(const bf16 *__restrict__
         tc::mbar_init(&mbar, 1);
         tc::fence_mbar_init();
     }
-    const bf16 *Qb = Q + ((size_t)bh * S) * D;
-    const bf16 *Kb = K + ((size_t)bh * S) * D;
-    const bf16 *Vb = V + ((size_t)bh * S) * D;
-    load_rows<D>(sQ, Qb + (size_t)t0 * D, 128, nq, tid, 128);
-    load_rows<D>(sK, Kb + (size_t)kstart * D, NK, nk, tid, 128);
-    load_v<D>(sVt, Vb + (size_t)kstart * D, NK, nk, tid, 128);
-    // this query's remote selections and their (max, sum); the partial rows are
-    // prefetched to L2 so that the merge at the end does not wait on DRAM
-    const int t = t0 + tid;
-    const bool live = tid < nq;
-    int jr[kMaxR];
-    float2 ml[kMaxR];
-    for (int r = 0; r < R; ++r) {
-        jr[r] = -1;
-        if (!live) continue;
-        const size_t pq = ((size_t)bh * S + t) * R + r;
-        const int j = sel[pq];
-        if (sel_valid(j, t, BS, L)) {
-            jr[r] = j;
-            ml[r] = part_ml[pq];
-            for (int c = 0; c < D * 2; c += 128) tc::prefetch_l2((const uint8_t *)(part_o + pq * D) + c);
-        }
-    }
-    tc::cp_async_wait_all();
-    tc::fence_smem_to_async();
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tmem = tmem_base;
-    const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
-    if (tid == 0) {
-        const uint32_t id = tc::idesc_bf16(128, NK);
-        const uint32_t aq = tc::smem_u32(sQ), bk = tc::smem_u32(sK);
-#pragma unroll
-        for (int k = 0; k < D / 16; ++k)
-            tc::mma_bf16(tmem, tc::desc_kmajor(aq + 256 * k, D), tc::desc_kmajor(bk + 256 * k, D), id, k > 0);
-        tc::commit(&mbar);
-    }
-    bool ok = tc::mbar_wait(&mbar, 0);
-    tc::fence_after_sync();
+    const uint32_t trow = tmem + ((uint32_t)(quarter * 32) << 16);
 
-    // masked softmax of row t over keys s in [lo(t), t].  In column terms the
-    // valid keys are [vlo, vhi]; 32-column chunks entirely inside need no
-    // per-element mask and chunks entirely outside need no exponential.
-    const int lo = max(0, t / BS - L + 1) * BS;
-    const int vlo = lo - kstart, vhi = t - kstart;
-    float v[32];
-    float m = -INFINITY;
-#pragma unroll 1
-    for (int c0 = 0; c0 < NK; c0 += 32) {
-        tc::tmem_ld32(trow + c0, v);
-        if (c0 + 31 < vlo || c0 > vhi) continue;
-        if (c0 >= vlo && c0 + 31 <= vhi) {
+    auto issue = [&](int stage, int f) {
+        const long long bh = bh0 + f / ntiles;
+        const int t0 = (f % ntiles) * 128;
+        const int nq = min(128, S - t0);
+        const int kstart = max(0, t0 / BS - L + 1) * BS;
+        const int nk = min(S, t0 + 128) - kstart;
+        uint8_t *sQ = smem + stage * STAGE, *sK = sQ + QB, *sV = sK + KB;
+        const size_t base = (size_t)bh * S;
+        load_rows<D>(sQ, Q + (base + t0) * D, 128, nq, tid, 256);
+        load_rows<D>(sK, K + (base + kstart) * D, NK, nk, tid, 256);
+        load_v<D>(sV, V + (base + kstart) * D, NK, nk, tid, 256);
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+
+    bool ok = true;
+    int f = blockIdx.x;
+    // this row's selections of the next tile, loaded one tile ahead
+    // (R <= RMAX; arrays indexed by compile-time slot so they stay in registers)
+    constexpr int kPre = DH <= 32 ? (RMAX < 2 ? RMAX : 2) : 0;  // slots whose partial rows go to registers early
+    int selv[RMAX];
+    auto load_sel = [&](int ff) {
+        const long long bbh = bh0 + ff / ntiles;
+        const int tt = (ff % ntiles) * 128 + row;
 #pragma unroll
-            for (int i = 0; i < 32; ++i) m = fmaxf(m, v[i]);
-        } else {
-#pragma unroll
-            for (int i = 0; i < 32; ++i)
-                if (c0 + i >= vlo && c0 + i <= vhi) m = fmaxf(m, v[i]);
-        }
+        for (int r = 0; r < RMAX; ++r) selv[r] = (r < R && tt < S) ? sel[((size_t)bbh * S + tt) * R + r] : -1;
+    };
+    if (f < total) {
+        issue(0, f);
+        load_sel(f);
     }
-    const float m2 = (m == -INFINITY) ? 0.f : m * scale_log2;
-    float l = 0.f;
-    // P may reuse the space of Q and K: they are only read by the first MMA,
-    // which has completed (mbarrier) before any thread gets here.
-#pragma unroll 1
-    for (int c0 = 0; c0 < NK; c0 += 32) {
-        tc::tmem_ld32(trow + c0, v);
-        uint32_t pk[16];
-        if (c0 + 31 < vlo || c0 > vhi) {
+    for (int k = 0; f < total && ok; ++k, f += G) {
+        const int stage = ST == 2 ? (k & 1) : 0;
+        const bool have1 = f + G < total;
+        if (ST == 2 && have1) issue(stage ^ 1, f + G);
+        // this tile's geometry; this row's remote selections, their (max, sum)
+        // and partial rows are requested now and used by the merge at the end
+        const long long bh = bh0 + f / ntiles;
+        const int b = (int)(bh / H), h = (int)(bh % H);
+        const int t0 = (f % ntiles) * 128;
+        const int nq = min(128, S - t0);
+        const int kstart = max(0, t0 / BS - L + 1) * BS;
+        const int t = t0 + row;
+        const bool live = row < nq;
+        int jr[RMAX];
+        float2 ml[RMAX];
+        uint4 pre[kPre > 0 ? kPre : 1][DH / 8];
 #pragma unroll
-            for (int u = 0; u < 16; ++u) pk[u] = 0u;
-        } else {
-            const bool full = c0 >= vlo && c0 + 31 <= vhi;
+        for (int r = 0; r < RMAX; ++r) {
+            jr[r] = -1;
+            ml[r] = make_float2(0.f, 0.f);
+            if (r >= R || !live || !sel_valid(selv[r], t, BS, L)) continue;
+            const size_t pq = ((size_t)bh * S + t) * R + r;
+            jr[r] = selv[r];
+            ml[r] = part_ml[pq];
+            if (r < kPre) {
 #pragma unroll
-            for (int u = 0; u < 16; ++u) {
-                const int i = 2 * u;
-                float a = exp2f(fmaf(v[i], scale_log2, -m2));
-                float bb = exp2f(fmaf(v[i + 1], scale_log2, -m2));
-                if (!full) {
-                    a = (c0 + i >= vlo && c0 + i <= vhi) ? a : 0.f;
-                    bb = (c0 + i + 1 >= vlo && c0 + i + 1 <= vhi) ? bb : 0.f;
-                }
-                l += a + bb;
-                pk[u] = pack2(a, bb);
+                for (int q8 = 0; q8 < DH / 8; ++q8)
+                    pre[r < kPre ? r : 0][q8] = __ldg((const uint4 *)(part_o + pq * D + half * DH) + q8);
+            } else {
+                tc::prefetch_l2(part_o + pq * D + half * DH);
             }
         }
+        if (have1) load_sel(f + G);
+        if (ST == 2 && have1) asm volatile("cp.async.wait_group 1;" ::: "memory");
+        else asm volatile("cp.async.wait_group 0;" ::: "memory");
+        tc::fence_smem_to_async();
+        tc::fence_before_sync();
+        __syncthreads();
+        tc::fence_after_sync();
+        uint8_t *sQ = smem + stage * STAGE, *sK = sQ + QB, *sV = sK + KB;
+        uint8_t *sP = smem + local_p_offset(ST, STAGE, QB, KB, PB, stage);
+        float(*s_red)[128] = (float(*)[128])(smem + local_red_offset(ST, STAGE, QB, KB, PB, stage));
+        if (tid == 0) {
+            const uint32_t id = tc::idesc_bf16(128, NK);
+            const uint32_t aq = tc::smem_u32(sQ), bk = tc::smem_u32(sK);
 #pragma unroll
-        for (int q8 = 0; q8 < 4; ++q8)
-            *(uint4 *)(sP + tc::kmajor_chunk(tid, (c0 >> 3) + q8, NK)) =
-                make_uint4(pk[4 * q8], pk[4 * q8 + 1], pk[4 * q8 + 2], pk[4 * q8 + 3]);
-    }
-    tc::fence_smem_to_async();
-    tc::fence_before_sync();
-    __syncthreads();
-    tc::fence_after_sync();
-    if (tid == 0 && ok) {
-        const uint32_t id = tc::idesc_bf16(128, D, true);
-        const uint32_t ap = tc::smem_u32(sP), bv = tc::smem_u32(sVt);
-#pragma unroll
-        for (int k = 0; k < NK / 16; ++k)
-            tc::mma_bf16(tmem, tc::desc_kmajor(ap + 256 * k, NK), tc::desc_mnmajor(bv + 256 * k, NK), id, k > 0);
-        tc::commit(&mbar);
-    }
-    if (ok) ok = tc::mbar_wait(&mbar, 1);
-    tc::fence_after_sync();
-    if (!ok && tid == 0) record_error(counters, kDevErrTimeout);
-
-    // merge with the remote partials: out = (O_loc + sum_r l_r 2^(m_r - M) o_r 2^(m_loc... )) / ...
-    float mm = m2;
-    for (int r = 0; r < R; ++r)
-        if (jr[r] >= 0) mm = fmaxf(mm, ml[r].x);
-    const float wl = exp2f(m2 - mm);
-    float den = l * wl;
-    float wr[kMaxR];
-    for (int r = 0; r < R; ++r) {
-        wr[r] = 0.f;
-        if (jr[r] >= 0) {
-            wr[r] = ml[r].y * exp2f(ml[r].x - mm);
-            den += wr[r];
+            for (int kk = 0; kk < D / 16; ++kk)
+                tc::mma_bf16(tmem, tc::desc_kmajor(aq + 256 * kk, D), tc::desc_kmajor(bk + 256 * kk, D), id, kk > 0);
+            tc::commit(&mbar);
         }
-    }
-    const float inv = 1.f / den;
-    bf16 *orow = O + (((size_t)b * S + t) * H + h) * D;
+        ok = __syncthreads_and(tc::mbar_wait(&mbar, 0));
+        tc::fence_after_sync();
+
+        // masked softmax of row t over keys s in [lo(t), t]; in column terms
+        // [vlo, vhi].  32-column chunks entirely inside need no per-element
+        // mask, chunks entirely outside no exponential.
+        const int lo = max(0, t / BS - L + 1) * BS;
+        const int vlo = lo - kstart, vhi = t - kstart;
+        const int cbeg = half * HALF;
+        float v[32];
+        float m = -INFINITY;
+#pragma unroll 1
+        for (int c0 = cbeg; c0 < cbeg + HALF; c0 += 32) {
+            tc::tmem_ld32(trow + c0, v);
+            if (c0 + 31 < vlo || c0 > vhi) continue;
+            if (c0 >= vlo && c0 + 31 <= vhi) {
 #pragma unroll
-    for (int c0 = 0; c0 < D; c0 += 32) {
-        tc::tmem_ld32(trow + c0, v);
-        if (live && ok) {
+                for (int i = 0; i < 32; ++i) m = fmaxf(m, v[i]);
+            } else {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] *= wl;
-            for (int r = 0; r < R; ++r) {
-                if (jr[r] < 0) continue;
-                const uint4 *src = (const uint4 *)(part_o + (((size_t)bh * S + t) * R + r) * D + c0);
+                for (int i = 0; i < 32; ++i)
+                    if (c0 + i >= vlo && c0 + i <= vhi) m = fmaxf(m, v[i]);
+            }
+        }
+        s_red[half][row] = m;
+        __syncthreads();
+        m = fmaxf(s_red[0][row], s_red[1][row]);
+        const float m2 = (m == -INFINITY) ? 0.f : m * scale_log2;
+        float l = 0.f;
+#pragma unroll 1
+        for (int c0 = cbeg; c0 < cbeg + HALF; c0 += 32) {
+            tc::tmem_ld32(trow + c0, v);
+            uint32_t pk[16];
+            if (c0 + 31 < vlo || c0 > vhi) {
 #pragma unroll
-                for (int q8 = 0; q8 < 4; ++q8) {
-                    uint4 u4 = __ldg(src + q8);
-                    const __nv_bfloat162 *h2 = (const __nv_bfloat162 *)&u4;
+                for (int u = 0; u < 16; ++u) pk[u] = 0u;
+            } else {
+                const bool full = c0 >= vlo && c0 + 31 <= vhi;
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        float2 f = __bfloat1622float2(h2[e]);
-                        v[8 * q8 + 2 * e] = fmaf(wr[r], f.x, v[8 * q8 + 2 * e]);
-                        v[8 * q8 + 2 * e + 1] = fmaf(wr[r], f.y, v[8 * q8 + 2 * e + 1]);
+                for (int u = 0; u < 16; ++u) {
+                    const int i = 2 * u;
+                    float a = exp2f(fmaf(v[i], scale_log2, -m2));
+                    float bb = exp2f(fmaf(v[i + 1], scale_log2, -m2));
+                    if (!full) {
+                        a = (c0 + i >= vlo && c0 + i <= vhi) ? a : 0.f;
+                        bb = (c0 + i + 1 >= vlo && c0 + i + 1 <= vhi) ? bb : 0.f;
                     }
+                    l += a + bb;
+                    pk[u] = pack2(a, bb);
                 }
             }
-            uint4 *dst = (uint4 *)(orow + c0);
 #pragma unroll
             for (int q8 = 0; q8 < 4; ++q8)
-                dst[q8] = make_uint4(pack2(v[8 * q8] * inv, v[8 * q8 + 1] * inv), pack2(v[8 * q8 + 2] * inv, v[8 * q8 + 3] * inv),
-                                     pack2(v[8 * q8 + 4] * inv, v[8 * q8 + 5] * inv), pack2(v[8 * q8 + 6] * inv, v[8 * q8 + 7] * inv));
+                *(uint4 *)(sP + tc::kmajor_chunk(row, (c0 >> 3) + q8, NK)) =
+                    make_uint4(pk[4 * q8], pk[4 * q8 + 1], pk[4 * q8 + 2], pk[4 * q8 + 3]);
         }
+        __syncthreads();  // every thread has read the maxima
+        s_red[half][row] = l;
+        tc::fence_smem_to_async();
+        tc::fence_before_sync();
+        __syncthreads();
+        tc::fence_after_sync();
+        l = s_red[0][row] + s_red[1][row];
+        if (tid == 0 && ok) {
+            const uint32_t id = tc::idesc_bf16(128, D, true);
+            const uint32_t ap = tc::smem_u32(sP), bv = tc::smem_u32(sV);
+#pragma unroll
+            for (int kk = 0; kk < NK / 16; ++kk)
+                tc::mma_bf16(tmem, tc::desc_kmajor(ap + 256 * kk, NK), tc::desc_mnmajor(bv + 256 * kk, NK), id, kk > 0);
+            tc::commit(&mbar);
+        }
+        ok = __syncthreads_and(ok && tc::mbar_wait(&mbar, 1));
+        tc::fence_after_sync();
+
+        // merge with the remote partials (max/sum rescaling), this thread's half of the columns
+        float mm = m2;
+#pragma unroll
+        for (int r = 0; r < RMAX; ++r)
+            if (jr[r] >= 0) mm = fmaxf(mm, ml[r].x);
+        const float wl = exp2f(m2 - mm);
+        float den = l * wl;
+        float wr[RMAX];
+#pragma unroll
+        for (int r = 0; r < RMAX; ++r) {
+            wr[r] = 0.f;
+            if (jr[r] >= 0) {
+                wr[r] = ml[r].y * exp2f(ml[r].x - mm);
+                den += wr[r];
+            }
+        }
+        const float inv = 1.f / den;
+        bf16 *orow = O + (((size_t)b * S + t) * H + h) * D;
+#pragma unroll
+        for (int c0 = half * DH; c0 < half * DH + DH; c0 += 32) {
+            tc::tmem_ld32(trow + c0, v);
+            if (live && ok) {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) v[i] *= wl;
+#pragma unroll
+                for (int r = 0; r < RMAX; ++r) {
+                    if (jr[r] < 0) continue;
+                    const uint4 *src = (const uint4 *)(part_o + (((size_t)bh * S + t) * R + r) * D + c0);
+#pragma unroll
+                    for (int q8 = 0; q8 < 4; ++q8) {
+                        uint4 u4;
+                        if (kPre > 0 && r < kPre) u4 = pre[r < kPre ? r : 0][((c0 - half * DH) >> 3) + q8];
+                        else u4 = __ldg(src + q8);
+                        const __nv_bfloat162 *h2 = (const __nv_bfloat162 *)&u4;
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            float2 fv = __bfloat1622float2(h2[e]);
+                            v[8 * q8 + 2 * e] = fmaf(wr[r], fv.x, v[8 * q8 + 2 * e]);
+                            v[8 * q8 + 2 * e + 1] = fmaf(wr[r], fv.y, v[8 * q8 + 2 * e + 1]);
+                        }
+                    }
+                }
+                uint4 *dst = (uint4 *)(orow + c0);
+#pragma unroll
+                for (int q8 = 0; q8 < 4; ++q8)
+                    dst[q8] = make_uint4(pack2(v[8 * q8] * inv, v[8 * q8 + 1] * inv),
+                                         pack2(v[8 * q8 + 2] * inv, v[8 * q8 + 3] * inv),
+                                         pack2(v[8 * q8 + 4] * inv, v[8 * q8 + 5] * inv),
+                                         pack2(v[8 * q8 + 6] * inv, v[8 * q8 + 7] * inv));
+            }
+        }
+        tc::fence_before_sync();
+        __syncthreads();  // the stage's tiles, P and TMEM are free again
+        tc::fence_after_sync();
+        if (ST == 1 && have1) issue(0, f + G);
     }
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
+    if (!ok && tid == 0) record_error(counters, kDevErrTimeout);
     tc::fence_before_sync();
     __syncthreads();
     if (warp == 0) tc::tmem_dealloc(tmem, NCOLS);
@@ -519,7 +686,36 @@ bool attend_tc_supported(const mono_config &c) {
     return nk <= 256;
 }
 
-template <int D, int BS, int NK>
+// CTAs that are resident at once on the current device (SMs x CTAs per SM), for
+// persistent kernels.  CTAs per SM = the tightest of the thread, register and
+// shared-memory limits of an SM (2048 threads, 64K registers, 228 KB of
+// shared memory with 1 KB reserved per CTA).
+template <typename F>
+static cudaError_t persistent_grid(F kernel, int threads, size_t smem, int *out) {
+    int dev = 0, sms = 0;
+    cudaError_t e;
+    if ((e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                  cudaSharedmemCarveoutMaxShared)) != cudaSuccess)
+        return e;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    cudaFuncAttributes fa;
+    if ((e = cudaFuncGetAttributes(&fa, kernel)) != cudaSuccess) return e;
+    const int regs_per_warp = ((fa.numRegs * 32 + 255) / 256) * 256;
+    const int by_threads = 2048 / threads;
+    const int by_regs = 65536 / (regs_per_warp * (threads / 32));
+    const int by_smem = (int)((228 * 1024) / (smem + fa.sharedSizeBytes + 1024));
+    *out = sms * std::max(1, std::min(by_threads, std::min(by_regs, by_smem)));
+    return cudaSuccess;
+}
+
+template <int D, int BS>
+constexpr size_t remote_smem() {
+    constexpr size_t QB = 128 * D * 2, KB = BS * D * 2, PB = 128 * BS * 2;
+    return 2 * (QB + 2 * KB) + (PB <= QB ? 0 : PB);
+}
+
+template <int D, int BS, int NK, int RMAX>
 static cudaError_t launch_tc_shape(const Plan &p, const bf16 *Q, const bf16 *K, const bf16 *V, const int32_t *sel,
                                    bf16 *O, void *ws, cudaStream_t s) {
     const mono_config &c = p.cfg;
@@ -532,7 +728,7 @@ static cudaError_t launch_tc_shape(const Plan &p, const bf16 *Q, const bf16 *K, 
         int32_t *ps = (int32_t *)ws_ptr(p, ws, kRegPairStart);
         int32_t *pf = (int32_t *)ws_ptr(p, ws, kRegPairFill);
         int32_t *pairs = (int32_t *)ws_ptr(p, ws, kRegPairs);
-        int2 *work = (int2 *)ws_ptr(p, ws, kRegWork);
+        int4 *work = (int4 *)ws_ptr(p, ws, kRegWork);
         int32_t *nwork = (int32_t *)ws_ptr(p, ws, kRegNWork);
         if ((e = cudaMemsetAsync(pc, 0, (size_t)nbh * 4, s)) != cudaSuccess) return e;
         const int nbhh = c.B * c.H;
@@ -547,26 +743,43 @@ static cudaError_t launch_tc_shape(const Plan &p, const bf16 *Q, const bf16 *K, 
         k_pair_count<<<gq, 256, hs, s>>>(sel, pc, c.S, c.R, p.nb, c.Bs, c.L, cnt_err);
         k_pair_scan<<<nbhh, 1024, 0, s>>>(pc, ps, pf, work, nwork, p.nb, wcap);
         k_pair_fill<<<gq, 256, 2 * hs, s>>>(sel, ps, pf, pairs, c.S, c.R, p.nb, c.Bs, c.L);
-        const size_t pbytes = (size_t)128 * BS * 2, qbytes = (size_t)128 * D * 2;
-        const size_t smem = qbytes + (size_t)2 * BS * D * 2 + (pbytes <= qbytes ? 0 : pbytes);
-        auto kr = k_remote_tc<D, BS>;
-        if ((e = cudaFuncSetAttribute(kr, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
+        if ((e = cudaFuncSetAttribute(k_remote_tc<D, BS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)remote_smem<D, BS>())) != cudaSuccess)
             return e;
-        dim3 gr(wcap, nbhh);
-        kr<<<gr, 128, smem, s>>>(Q, K, V, pairs, ps, pc, work, nwork, (bf16 *)ws_ptr(p, ws, kRegPartO),
-                                 (float2 *)ws_ptr(p, ws, kRegPartML), cnt_err, c.S, c.R, p.nb, wcap, scale_log2);
-        count_launches(4);
+        count_launches(3);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
-    constexpr int QB = 128 * D * 2, KB = NK * D * 2, VB = D * NK * 2, PB = 128 * NK * 2;
-    const size_t smem = (size_t)QB + KB + VB + ((PB <= QB + KB) ? 0 : PB);
-    auto kl = k_local_merge_tc<D, BS, NK>;
+    const size_t smem = local_smem<D, NK>();
+    auto kl = k_local_merge_tc<D, BS, NK, RMAX>;
     if ((e = cudaFuncSetAttribute(kl, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess) return e;
-    dim3 grid((c.S + 127) / 128, c.H, c.B);
-    kl<<<grid, 128, smem, s>>>(Q, K, V, sel, (const bf16 *)ws_ptr(p, ws, kRegPartO),
-                               (const float2 *)ws_ptr(p, ws, kRegPartML), O, cnt_err, c.S, c.H, c.R, c.L, scale_log2);
-    count_launches(1);
-    return cudaGetLastError();
+    int local_ctas = 0;
+    if ((e = persistent_grid(kl, 256, smem, &local_ctas)) != cudaSuccess) return e;
+    // Remote then local, one group of (b, h) slices at a time: a group's partials
+    // (and its Q/K/V) are written by the remote kernel and read back by the
+    // local kernel right after, while they are still resident in L2.
+    int remote_ctas = 0;
+    if (c.R > 0 && (e = persistent_grid(k_remote_tc<D, BS>, 256, remote_smem<D, BS>(), &remote_ctas)) != cudaSuccess)
+        return e;
+    const int nbhh = c.B * c.H;
+    const size_t part_per_bh = (size_t)c.S * c.R * (2 * D + 8) + (size_t)3 * c.S * D * 2;
+    const int group = c.R > 0 ? (int)std::min<size_t>(kMaxGroup, std::max<size_t>(1, kL2GroupBytes / part_per_bh))
+                              : nbhh;
+    for (int g0 = 0; g0 < nbhh; g0 += group) {
+        const int ng = std::min(group, nbhh - g0);
+        if (c.R > 0) {
+            k_remote_tc<D, BS><<<remote_ctas, 256, remote_smem<D, BS>(), s>>>(
+                Q, K, V, (const int32_t *)ws_ptr(p, ws, kRegPairs), (const int4 *)ws_ptr(p, ws, kRegWork),
+                (const int32_t *)ws_ptr(p, ws, kRegNWork), (bf16 *)ws_ptr(p, ws, kRegPartO),
+                (float2 *)ws_ptr(p, ws, kRegPartML), cnt_err, c.S, c.R, p.max_work, scale_log2, g0, ng);
+            count_launches(1);
+        }
+        kl<<<local_ctas, 256, smem, s>>>(Q, K, V, sel, (const bf16 *)ws_ptr(p, ws, kRegPartO),
+                                         (const float2 *)ws_ptr(p, ws, kRegPartML), O, cnt_err, c.S, c.H, c.R, c.L,
+                                         scale_log2, g0, ng);
+        count_launches(1);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    return cudaSuccess;
 }
 
 cudaError_t launch_attend_tc(const Plan &p, const void *Q, const void *K, const void *V, const int32_t *sel, void *O,
@@ -576,7 +789,12 @@ cudaError_t launch_attend_tc(const Plan &p, const void *Q, const void *K, const 
     bf16 *o = (bf16 *)O;
     const int nk = 128 + (c.L - 1) * c.Bs;
     // NK = the local key range rounded up to a multiple of 32 (MMA N <= 256)
-#define MONO_TC(DD, BB, NN) return launch_tc_shape<DD, BB, NN>(p, q, k, v, sel, o, ws, s)
+#define MONO_TC(DD, BB, NN)                                                                                     \
+    do {                                                                                                        \
+        if (c.R <= 2) return launch_tc_shape<DD, BB, NN, 2>(p, q, k, v, sel, o, ws, s);                         \
+        if (c.R <= 4) return launch_tc_shape<DD, BB, NN, 4>(p, q, k, v, sel, o, ws, s);                         \
+        return launch_tc_shape<DD, BB, NN, kMaxR>(p, q, k, v, sel, o, ws, s);                                   \
+    } while (0)
     if (c.d == 64 && c.Bs == 64) {
         if (nk <= 128) MONO_TC(64, 64, 128);
         if (nk <= 192) MONO_TC(64, 64, 192);

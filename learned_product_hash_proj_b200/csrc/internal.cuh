@@ -50,7 +50,7 @@ enum Region {
     kRegPairs,       // [B*H*S*R] int32 (t*R + r) grouped by block
     kRegPartO,       // [B*H*S*R, d] bf16 remote partial outputs
     kRegPartML,      // [B*H*S*R] float2 (max, sum) of remote partials
-    kRegWork,        // [B*H, max_work] int2 (block, chunk) work items of the remote kernel
+    kRegWork,        // [B*H, max_work] int4 (block, first pair, pair count, 0) work items of the remote kernel
     kRegNWork,       // [B*H] int32 number of work items
     kRegN
 };

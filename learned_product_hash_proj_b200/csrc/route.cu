@@ -80,10 +80,11 @@ __global__ void __launch_bounds__(128) k_summary_assign_w(const T *__restrict__ 
                                                           int Bs, int M, int C, int H) {
     constexpr int PER = D / 32;  // columns per lane
     extern __shared__ __align__(16) float sm[];
-    float *s_cb = sm;                              // [C*D]
-    float *s_kb = s_cb + C * D;                    // [4][D]
+    const int dmp = D / M + 1;                     // padded codeword stride: lane mc reads bank (mc + i) % 32
+    float *s_cb = sm;                              // [M*C][dmp]
+    float *s_kb = s_cb + M * C * dmp;              // [4][D]
     float *s_sc = s_kb + 4 * D;                    // [4][M*C]
-    T *s_rows = (T *)(s_sc + 4 * M * C);           // [4][Bs*D] staged block rows
+    T *s_rows = (T *)(((uintptr_t)(s_sc + 4 * M * C) + 15) & ~(uintptr_t)15);  // [4][Bs*D] staged rows
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int h = blockIdx.y, b = blockIdx.z;
     const int nb = S / Bs;
@@ -96,7 +97,7 @@ __global__ void __launch_bounds__(128) k_summary_assign_w(const T *__restrict__ 
         const uint8_t *src = (const uint8_t *)(K + (bh * S + (size_t)j * Bs) * D);
         for (int c = lane; c < chunks; c += 32) tc::cp_async16((uint8_t *)rows + 16 * c, src + 16 * c, true);
     }
-    for (int i = threadIdx.x; i < C * D; i += blockDim.x) s_cb[i] = cb[(size_t)h * C * D + i];
+    for (int i = threadIdx.x; i < C * D; i += blockDim.x) s_cb[(i / (D / M)) * dmp + i % (D / M)] = cb[(size_t)h * C * D + i];
     tc::cp_async_wait_all();
     __syncwarp();
     if (j < nb) {
@@ -119,7 +120,7 @@ __global__ void __launch_bounds__(128) k_summary_assign_w(const T *__restrict__ 
     const int dm = D / M;
     for (int mc = lane; mc < M * C; mc += 32) {
         const int m = mc / C;
-        const float *w = s_cb + mc * dm;
+        const float *w = s_cb + mc * dmp;
         const float *kv = s_kb + warp * D + m * dm;
         float a = 0.0f;
         for (int i = 0; i < dm; ++i) a = __fmaf_rn(kv[i], w[i], a);
@@ -555,6 +556,50 @@ struct RegTop {  // top-T_ by (value desc, index asc); fully unrolled
     }
 };
 
+// Bit mask of the codes of one subspace that are not dominated by T0 others:
+// U = the top T0 by (score desc, code asc), found by T0 passes of an
+// ascending argmax (the first maximum wins a tie), plus every code within
+// delta of U's last score that some member of U does not dominate.
+template <int C, int T0>
+__device__ __forceinline__ unsigned survivors(const float (&s)[C], float delta) {
+    if constexpr (T0 >= C) {
+        return C == 32 ? 0xffffffffu : ((1u << C) - 1);
+    } else {
+        float uv[T0];
+        int ui[T0];
+        unsigned taken = 0;
+#pragma unroll
+        for (int k = 0; k < T0; ++k) {
+            float best = -INFINITY;
+            int bi = 0;
+            bool any = false;
+#pragma unroll
+            for (int c = 0; c < C; ++c) {
+                const bool free = !((taken >> c) & 1u);
+                const bool better = free && (!any || s[c] > best);
+                best = better ? s[c] : best;
+                bi = better ? c : bi;
+                any = any || free;
+            }
+            uv[k] = best;
+            ui[k] = bi;
+            taken |= 1u << bi;
+        }
+        const float thr = uv[T0 - 1] - delta;
+        unsigned keep = taken;
+#pragma unroll
+        for (int c = 0; c < C; ++c) {
+            if (((taken >> c) & 1u) || !(s[c] >= thr)) continue;
+            const float hi = s[c] + delta;
+            bool dom = true;
+#pragma unroll
+            for (int k = 0; k < T0; ++k) dom = dom && (uv[k] > hi || (uv[k] >= s[c] && ui[k] < c));
+            if (!dom) keep |= 1u << c;
+        }
+        return keep;
+    }
+}
+
 template <typename T, int D, int C, int TP, int E, int R>
 __global__ void __launch_bounds__(128) k_probe_m2(const T *__restrict__ Q, const float *__restrict__ kbar,
                                                   const float *__restrict__ cb, const int32_t *__restrict__ post_ids,
@@ -567,8 +612,8 @@ __global__ void __launch_bounds__(128) k_probe_m2(const T *__restrict__ Q, const
     extern __shared__ float smem[];
     const int nb = S / Bs;
     float *s_cb = smem;                               // [2*C*DM] = C*D floats
-    float *s_s0 = s_cb + C * D;                       // [C][128] subspace-0 scores per thread
-    int32_t *s_addr = (int32_t *)(s_s0 + C * 128);    // [nb]
+    float *s_s0 = s_cb + C * D;                       // [2C][128] subspace scores per thread
+    int32_t *s_addr = (int32_t *)(s_s0 + 2 * C * 128); // [nb]
     int32_t *s_ids = s_addr + nb;                     // [nb]
     const int h = blockIdx.y, b = blockIdx.z;
     const size_t bh = (size_t)b * H + h;
@@ -630,6 +675,7 @@ __global__ void __launch_bounds__(128) k_probe_m2(const T *__restrict__ Q, const
 #pragma unroll
         for (int c = 0; c < C; ++c) {
             s_s0[c * 128 + tid] = s0[c];
+            s_s0[(C + c) * 128 + tid] = s1[c];
             mx0 = fmaxf(mx0, fabsf(s0[c]));
             mx1 = fmaxf(mx1, fabsf(s1[c]));
         }
@@ -637,40 +683,22 @@ __global__ void __launch_bounds__(128) k_probe_m2(const T *__restrict__ Q, const
         frexpf(2.f * (mx0 + mx1) + 1e-30f, &e2);
         const float delta = 3.0f * ldexpf(1.f, e2 - 24);   // (M+1) ulp(2G)
 
-        // stage 0: the subspace-0 codes that can still lead to a top-T address
-        RegTop<(TP < C ? TP : C)> u0;
-        constexpr int T0 = TP < C ? TP : C;
-        u0.init();
-#pragma unroll
-        for (int c = 0; c < C; ++c) u0.push(s0[c], c);
-        unsigned cand = 0;
-        if (TP >= C) {
-            cand = C == 32 ? 0xffffffffu : ((1u << C) - 1);
-        } else {
-            const float thr = u0.v[T0 - 1] - delta;
-            const float last_v = u0.v[T0 - 1];
-            const int last_a = u0.a[T0 - 1];
-#pragma unroll
-            for (int c = 0; c < C; ++c) {
-                const float v = s0[c];
-                if (!(v >= thr)) continue;
-                const bool held = !RegTop<T0>::before(last_v, last_a, v, c);
-                bool dom = true;
-                const float hi = v + delta;
-#pragma unroll
-                for (int k = 0; k < T0; ++k) dom = dom && (u0.v[k] > hi || (u0.v[k] >= v && u0.a[k] < c));
-                if (held || !dom) cand |= 1u << c;
-            }
-        }
-        // final stage: every completion of the surviving codes, ranked exactly
+        // Each subspace keeps the codes that are not dominated by T others (see
+        // the pruning rule above): for subspace 0 as address prefixes, for
+        // subspace 1 as suffixes of any surviving prefix (for a fixed prefix the
+        // completions rank by s1 with ties to the lower code, which is the
+        // same rule).  The final top T lies in cand0 x cand1.
+        const unsigned cand0 = survivors<C, (TP < C ? TP : C)>(s0, delta);
+        const unsigned cand1 = survivors<C, (TP < C ? TP : C)>(s1, delta);
         RegTop<TP> top;
         top.init();
-        while (cand) {
-            const int c0 = __ffs(cand) - 1;
-            cand &= cand - 1;
+        for (unsigned m0 = cand0; m0; m0 &= m0 - 1) {
+            const int c0 = __ffs(m0) - 1;
             const float v0 = s_s0[c0 * 128 + tid];
-#pragma unroll
-            for (int c1 = 0; c1 < C; ++c1) top.push(__fadd_rn(v0, s1[c1]), c0 * C + c1);
+            for (unsigned m1 = cand1; m1; m1 &= m1 - 1) {
+                const int c1 = __ffs(m1) - 1;
+                top.push(__fadd_rn(v0, s_s0[(C + c1) * 128 + tid]), c0 * C + c1);
+            }
         }
 
         // union of the probed lists, causal filter, E cap; rerank on the fly
@@ -763,8 +791,8 @@ cudaError_t launch_summaries(const Plan &p, const void *K, const float *cb, void
     unsigned long long *cnt = (unsigned long long *)ws_ptr(p, ws, kRegCounters);
     cudaError_t e = cudaMemsetAsync(cnt, 0, kCntN * 8, s);
     if (e != cudaSuccess) return e;
-    const size_t smem = ((size_t)c.C * c.d + 4 * (size_t)c.d + 4 * (size_t)c.M * c.C) * 4 +
-                        4 * (size_t)c.Bs * c.d * p.es;
+    const size_t smem = ((size_t)c.M * c.C * (c.d / c.M + 1) + 4 * (size_t)c.d + 4 * (size_t)c.M * c.C) * 4 +
+                        4 * (size_t)c.Bs * c.d * p.es + 16;
     dim3 g1((p.nb + 3) / 4, c.H, c.B);
 #define MONO_SUMW(TT, DD)                                                                                         \
     do {                                                                                                          \
@@ -815,7 +843,7 @@ cudaError_t launch_queries(const Plan &p, const void *Q, const float *cb, const 
     // compile-time shapes of the configured workloads; any other shape takes the general kernel
 #define MONO_M2(TT, DD, CC, TPP, EE, RR)                                                                          \
     if (c.M == 2 && c.d == DD && c.C == CC && c.T == TPP && c.E == EE && c.R == RR) {                           \
-        const size_t sm2 = (size_t)CC * DD * 4 + (size_t)CC * 128 * 4 + (size_t)p.nb * 8;                       \
+        const size_t sm2 = (size_t)CC * DD * 4 + (size_t)2 * CC * 128 * 4 + (size_t)p.nb * 8;                   \
         auto kern = k_probe_m2<TT, DD, CC, TPP, EE, RR>;                                                        \
         if (sm2 > 48 * 1024 &&                                                                                   \
             (e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm2)) != cudaSuccess) \
