@@ -227,11 +227,14 @@ def run_ours(args):
     tokens = world * B * S
     value = tokens / (ra / 1e3)
 
-    # roofline: dominant kernel of the route+attend window, plus the window itself
+    # roofline: the dominant kernel of the route+attend window (among the stages
+    # that are one kernel each, so its event time is that kernel's time), plus the
+    # window itself.  "attend" is five kernels (buckets, remote, local) and is
+    # reported as a stage.
     hbm, bf16_tf, peak_kind = peaks()
     ab = algorithmic_bytes(cfg)
-    route_kernels = ("summaries", "lists", "queries", "attend")
-    dom = max(route_kernels, key=lambda n: stage[n])
+    single_kernel_stages = {"summaries": "k_summary_assign_w", "lists": "k_posting_dense", "queries": "k_probe_m2"}
+    dom = max(single_kernel_stages, key=lambda n: stage[n])
     achieved = ab[dom] / (stage[dom] / 1e3) / 1e9
     window_gbs = ab["route_attend"] / (ra / 1e3) / 1e9
     traffic = load_traffic(dom, cfg)
@@ -278,7 +281,8 @@ def run_ours(args):
                        "replicas": "one independent replica per GPU (no data-path collective)"},
             "route_attend_ms": ra, "forward_tokens_per_s": tokens / (fwd / 1e3),
             "stage_ms": stage,
-            "roofline": {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": hbm, "unit": "GB/s",
+            "roofline": {"bound": "hbm", "kernel": single_kernel_stages[dom], "stage": dom, "achieved": achieved,
+                         "peak": hbm, "unit": "GB/s",
                          "frac": achieved / hbm, "traffic": traffic, "algorithmic_bytes": ab[dom],
                          "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)"},
             "route_attend_roofline": {"bound": "hbm", "achieved": window_gbs, "peak": hbm, "unit": "GB/s",
@@ -300,14 +304,15 @@ def run_ours(args):
     dist.finalize()
 
 
-def load_traffic(kernel: str, cfg):
-    """dram read+write bytes per launch of `kernel` from the committed ncu summary, if it matches this build."""
+def load_traffic(stage: str, cfg):
+    """DRAM read+write bytes per launch of the stage's kernel, from the committed ncu summary
+    (profiles/traffic.json), or None when the summary does not cover this workload."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
             t = json.load(f)
-        e = t.get(cfg.name, {}).get(kernel)
-        return e if e is None else float(e)
+        e = t.get(cfg.name, {}).get(stage)
+        return None if e is None else float(e["bytes_per_launch"])
     except Exception:
         return None
 

@@ -600,27 +600,145 @@ __device__ __forceinline__ unsigned survivors(const float (&s)[C], float delta) 
     }
 }
 
+// The top T0 codes of one subspace by (score desc, code asc), in that order:
+// T0 passes of a tree argmax over the codes not yet taken, in which the right
+// operand wins only when strictly greater, so that the lowest code wins a tie.
+// Taken codes are masked with -inf; the scores are finite for finite inputs.
+template <int C, int T0>
+__device__ __forceinline__ void top_codes(const float (&s)[C], float (&uv)[T0], int (&ui)[T0]) {
+    static_assert((C & (C - 1)) == 0 && C >= 2, "C a power of two");
+    float w[C];
+#pragma unroll
+    for (int c = 0; c < C; ++c) w[c] = s[c];
+#pragma unroll
+    for (int k = 0; k < T0; ++k) {
+        float tv[C / 2];
+        int ti[C / 2];
+#pragma unroll
+        for (int p = 0; p < C / 2; ++p) {
+            const bool r = w[2 * p + 1] > w[2 * p];
+            tv[p] = r ? w[2 * p + 1] : w[2 * p];
+            ti[p] = r ? 2 * p + 1 : 2 * p;
+        }
+#pragma unroll
+        for (int n = C / 4; n >= 1; n >>= 1) {
+#pragma unroll
+            for (int p = 0; p < n; ++p) {
+                const bool r = tv[2 * p + 1] > tv[2 * p];
+                tv[p] = r ? tv[2 * p + 1] : tv[2 * p];
+                ti[p] = r ? ti[2 * p + 1] : ti[2 * p];
+            }
+        }
+        uv[k] = tv[0];
+        ui[k] = ti[0];
+        if (k + 1 < T0) {
+#pragma unroll
+            for (int c = 0; c < C; ++c) w[c] = (c == ti[0]) ? -INFINITY : w[c];
+        }
+    }
+}
+
+// Codes outside U = {ui} within delta of U's last score: candidates for the
+// near-tie rule below (a bit mask; almost always empty).
+template <int C, int T0>
+__device__ __forceinline__ unsigned near_codes(const float (&s)[C], const float (&uv)[T0], unsigned taken, float delta) {
+    const float thr = uv[T0 - 1] - delta;
+    unsigned m = 0;
+#pragma unroll
+    for (int c = 0; c < C; ++c) m |= (s[c] >= thr ? 1u : 0u) << c;
+    return m & ~taken;
+}
+
+// Of the near codes, those that some member of U does not dominate (the
+// pruning rule: u dominates p if s_u > s_p + delta, or s_u >= s_p and u < p).
+template <int T0>
+__device__ __forceinline__ unsigned undominated(unsigned near, const float *col, int stride, const float (&uv)[T0],
+                                                const int (&ui)[T0], float delta) {
+    unsigned keep = 0;
+    for (unsigned m = near; m; m &= m - 1) {
+        const int c = __ffs(m) - 1;
+        const float sc = col[c * stride], hi = sc + delta;
+        bool dom = true;
+#pragma unroll
+        for (int k = 0; k < T0; ++k) dom = dom && (uv[k] > hi || (uv[k] >= sc && ui[k] < c));
+        if (!dom) keep |= 1u << c;
+    }
+    return keep;
+}
+
+// Scores of one subspace: s[c] = q_m . codeword_{m,c}, one fma chain per code
+// in ascending element order (the chains advance together, eight elements at
+// a time, which changes nothing in any chain).  q is read from global memory
+// in pieces so that it never occupies registers as a whole.
+template <typename T, int DM, int C>
+__device__ __forceinline__ void sub_scores(const T *__restrict__ qm, const float *cbm, float (&s)[C]) {
+#pragma unroll
+    for (int c = 0; c < C; ++c) s[c] = 0.0f;
+#pragma unroll
+    for (int i8 = 0; i8 < DM / 8; ++i8) {
+        float qv[8];
+        if constexpr (sizeof(T) == 2) {
+            const uint4 u = __ldg((const uint4 *)(qm + 8 * i8));
+            const __nv_bfloat162 *h2 = (const __nv_bfloat162 *)&u;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 f = __bfloat1622float2(h2[e]);
+                qv[2 * e] = f.x;
+                qv[2 * e + 1] = f.y;
+            }
+        } else {
+            const float4 a = __ldg((const float4 *)(qm + 8 * i8)), b = __ldg((const float4 *)(qm + 8 * i8 + 4));
+            qv[0] = a.x; qv[1] = a.y; qv[2] = a.z; qv[3] = a.w;
+            qv[4] = b.x; qv[5] = b.y; qv[6] = b.z; qv[7] = b.w;
+        }
+#pragma unroll
+        for (int c = 0; c < C; ++c) {
+            const float4 x = ((const float4 *)(cbm + c * DM + 8 * i8))[0];
+            const float4 y = ((const float4 *)(cbm + c * DM + 8 * i8))[1];
+            float a = s[c];
+            a = __fmaf_rn(qv[0], x.x, a);
+            a = __fmaf_rn(qv[1], x.y, a);
+            a = __fmaf_rn(qv[2], x.z, a);
+            a = __fmaf_rn(qv[3], x.w, a);
+            a = __fmaf_rn(qv[4], y.x, a);
+            a = __fmaf_rn(qv[5], y.y, a);
+            a = __fmaf_rn(qv[6], y.z, a);
+            a = __fmaf_rn(qv[7], y.w, a);
+            s[c] = a;
+        }
+    }
+}
+
 template <typename T, int D, int C, int TP, int E, int R>
-__global__ void __launch_bounds__(128) k_probe_m2(const T *__restrict__ Q, const float *__restrict__ kbar,
-                                                  const float *__restrict__ cb, const int32_t *__restrict__ post_ids,
-                                                  const int32_t *__restrict__ post_addr,
-                                                  const int32_t *__restrict__ forced, int32_t *__restrict__ sel,
-                                                  unsigned long long *__restrict__ counters, int S, int H, int Bs,
-                                                  int L, int cap) {
-    constexpr int M = 2, DM = D / 2;
-    static_assert(C <= 32 && TP <= C * C && R >= 1, "shape");
+__global__ void __launch_bounds__(128, C <= 16 ? 5 : 3) k_probe_m2(const T *__restrict__ Q, const float *__restrict__ kbar,
+                                                     const float *__restrict__ cb, const int32_t *__restrict__ post_ids,
+                                                     const int32_t *__restrict__ post_addr,
+                                                     const int32_t *__restrict__ forced, int32_t *__restrict__ sel,
+                                                     unsigned long long *__restrict__ counters, int S, int H, int Bs,
+                                                     int L, int cap) {
+    constexpr int DM = D / 2, A = C * C;
+    static_assert(C <= 32 && TP <= C * C && R >= 1 && E >= 1, "shape");
     extern __shared__ float smem[];
     const int nb = S / Bs;
-    float *s_cb = smem;                               // [2*C*DM] = C*D floats
-    float *s_s0 = s_cb + C * D;                       // [2C][128] subspace scores per thread
-    int32_t *s_addr = (int32_t *)(s_s0 + 2 * C * 128); // [nb]
-    int32_t *s_ids = s_addr + nb;                     // [nb]
+    float *s_cb = smem;                                  // [2*C*DM] = C*D floats
+    float *s_sc = s_cb + C * D;                          // [2C][128] subspace scores, one column per thread
+    int32_t *s_first = (int32_t *)(s_sc + 2 * C * 128);  // [A] first position of each address, -1 if none
+    int32_t *s_addr = s_first + A;                       // [nb]
+    int32_t *s_ids = s_addr + nb;                        // [nb]
     const int h = blockIdx.y, b = blockIdx.z;
     const size_t bh = (size_t)b * H + h;
     for (int i = threadIdx.x; i < C * D; i += blockDim.x) s_cb[i] = cb[(size_t)h * C * D + i];
+    for (int i = threadIdx.x; i < A; i += blockDim.x) s_first[i] = -1;
     for (int i = threadIdx.x; i < nb; i += blockDim.x) {
         s_addr[i] = post_addr[bh * nb + i];
         s_ids[i] = post_ids[bh * nb + i];
+    }
+    __syncthreads();
+    // the posting arrays are sorted by address: each address's entries start
+    // where the address differs from the previous entry's
+    for (int i = threadIdx.x; i < nb; i += blockDim.x) {
+        const int a = s_addr[i];
+        if ((unsigned)a < (unsigned)A && (i == 0 || s_addr[i - 1] != a)) s_first[a] = i;
     }
     __syncthreads();
 
@@ -628,112 +746,151 @@ __global__ void __launch_bounds__(128) k_probe_m2(const T *__restrict__ Q, const
     const int t = blockIdx.x * blockDim.x + tid;
     int n_sel = 0, lt_r = 0, ign = 0;
     if (t < S) {
-        float q[D];
         const T *qp = Q + (bh * S + t) * D;
-        if constexpr (sizeof(T) == 2) {
-#pragma unroll
-            for (int c = 0; c < D / 8; ++c) {
-                uint4 u = __ldg((const uint4 *)(qp + 8 * c));
-                const __nv_bfloat162 *h2 = (const __nv_bfloat162 *)&u;
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    float2 f = __bfloat1622float2(h2[e]);
-                    q[8 * c + 2 * e] = f.x;
-                    q[8 * c + 2 * e + 1] = f.y;
-                }
-            }
-        } else {
-#pragma unroll
-            for (int c = 0; c < D / 4; ++c) {
-                float4 f = __ldg((const float4 *)(qp + 4 * c));
-                q[4 * c] = f.x; q[4 * c + 1] = f.y; q[4 * c + 2] = f.z; q[4 * c + 3] = f.w;
-            }
-        }
-        // subspace scores: 2C independent fma chains, each in ascending element
-        // order, advanced together four elements at a time (same results as one
-        // chain after another, with 2C-way instruction-level parallelism)
+        // subspace scores; both also go to shared memory for the rare paths,
+        // which walk codes by index
         float s0[C], s1[C];
-#pragma unroll
-        for (int c = 0; c < C; ++c) { s0[c] = 0.0f; s1[c] = 0.0f; }
-#pragma unroll
-        for (int i4 = 0; i4 < DM / 4; ++i4) {
-#pragma unroll
-            for (int c = 0; c < C; ++c) {
-                const float4 x = ((const float4 *)(s_cb + (0 * C + c) * DM))[i4];
-                const float4 y = ((const float4 *)(s_cb + (1 * C + c) * DM))[i4];
-                s0[c] = __fmaf_rn(q[4 * i4 + 0], x.x, s0[c]);
-                s0[c] = __fmaf_rn(q[4 * i4 + 1], x.y, s0[c]);
-                s0[c] = __fmaf_rn(q[4 * i4 + 2], x.z, s0[c]);
-                s0[c] = __fmaf_rn(q[4 * i4 + 3], x.w, s0[c]);
-                s1[c] = __fmaf_rn(q[DM + 4 * i4 + 0], y.x, s1[c]);
-                s1[c] = __fmaf_rn(q[DM + 4 * i4 + 1], y.y, s1[c]);
-                s1[c] = __fmaf_rn(q[DM + 4 * i4 + 2], y.z, s1[c]);
-                s1[c] = __fmaf_rn(q[DM + 4 * i4 + 3], y.w, s1[c]);
-            }
-        }
+        sub_scores<T, DM, C>(qp, s_cb, s0);
+        sub_scores<T, DM, C>(qp + DM, s_cb + C * DM, s1);
         float mx0 = 0.f, mx1 = 0.f;
 #pragma unroll
         for (int c = 0; c < C; ++c) {
-            s_s0[c * 128 + tid] = s0[c];
-            s_s0[(C + c) * 128 + tid] = s1[c];
+            s_sc[c * 128 + tid] = s0[c];
+            s_sc[(C + c) * 128 + tid] = s1[c];
             mx0 = fmaxf(mx0, fabsf(s0[c]));
             mx1 = fmaxf(mx1, fabsf(s1[c]));
         }
+        const bool finite = mx0 + mx1 <= 1.0e38f;
         int e2;
         frexpf(2.f * (mx0 + mx1) + 1e-30f, &e2);
         const float delta = 3.0f * ldexpf(1.f, e2 - 24);   // (M+1) ulp(2G)
 
-        // Each subspace keeps the codes that are not dominated by T others (see
-        // the pruning rule above): for subspace 0 as address prefixes, for
-        // subspace 1 as suffixes of any surviving prefix (for a fixed prefix the
-        // completions rank by s1 with ties to the lower code, which is the
-        // same rule).  The final top T lies in cand0 x cand1.
-        const unsigned cand0 = survivors<C, (TP < C ? TP : C)>(s0, delta);
-        const unsigned cand1 = survivors<C, (TP < C ? TP : C)>(s1, delta);
+        // Each subspace keeps U, its top T0 codes, and the near codes that
+        // some member of U does not dominate (the pruning rule above): for
+        // subspace 0 as address prefixes, for subspace 1 as suffixes of any
+        // surviving prefix (for a fixed prefix the completions rank by s1 with
+        // ties to the lower code, which is the same rule).  The final top T
+        // lies in cand0 x cand1.
+        constexpr int T0 = TP < C ? TP : C;
+        constexpr unsigned kAll = C == 32 ? 0xffffffffu : ((1u << C) - 1);
+        float uv0[T0], uv1[T0];
+        int ui0[T0], ui1[T0];
+        top_codes<C, T0>(s0, uv0, ui0);
+        top_codes<C, T0>(s1, uv1, ui1);
+        unsigned tk0 = 0, tk1 = 0;
+#pragma unroll
+        for (int k = 0; k < T0; ++k) { tk0 |= 1u << ui0[k]; tk1 |= 1u << ui1[k]; }
+        const unsigned nr0 = near_codes<C, T0>(s0, uv0, tk0, delta), nr1 = near_codes<C, T0>(s1, uv1, tk1, delta);
+        unsigned cand0 = tk0, cand1 = tk1;
+        if (!finite) {
+            cand0 = kAll;
+            cand1 = kAll;
+        } else if (nr0 | nr1) {
+            cand0 |= undominated<T0>(nr0, s_sc + tid, 128, uv0, ui0, delta);
+            cand1 |= undominated<T0>(nr1, s_sc + C * 128 + tid, 128, uv1, ui1, delta);
+        }
         RegTop<TP> top;
         top.init();
-        for (unsigned m0 = cand0; m0; m0 &= m0 - 1) {
-            const int c0 = __ffs(m0) - 1;
-            const float v0 = s_s0[c0 * 128 + tid];
-            for (unsigned m1 = cand1; m1; m1 &= m1 - 1) {
-                const int c1 = __ffs(m1) - 1;
-                top.push(__fadd_rn(v0, s_s0[(C + c1) * 128 + tid]), c0 * C + c1);
+        bool done = false;
+        if (cand0 == tk0 && cand1 == tk1) {
+            // U0 and U1 are sorted by score and fl(a + b) is monotone in a and
+            // b, so pair (i, j) of the ranks is preceded by the (i+1)(j+1)-1
+            // pairs (i' <= i, j' <= j) with scores at least as high: only pairs
+            // with (i+1)(j+1) <= T can be in the top T, unless an excluded pair
+            // reaches the T-th score (ties), which sends the query to the
+            // general walk below.
+            float vout = -INFINITY;
+#pragma unroll
+            for (int i = 0; i < T0; ++i)
+#pragma unroll
+                for (int j = 0; j < T0; ++j) {
+                    const float v = __fadd_rn(uv0[i], uv1[j]);
+                    if ((i + 1) * (j + 1) <= TP) top.push(v, ui0[i] * C + ui1[j]);
+                    else vout = fmaxf(vout, v);
+                }
+            done = vout < top.v[TP - 1];
+        }
+        if (!done) {
+            top.init();
+            for (unsigned m0 = cand0; m0; m0 &= m0 - 1) {
+                const int c0 = __ffs(m0) - 1;
+                const float v0 = s_sc[c0 * 128 + tid];
+                for (unsigned m1 = cand1; m1; m1 &= m1 - 1) {
+                    const int c1 = __ffs(m1) - 1;
+                    top.push(__fadd_rn(v0, s_sc[(C + c1) * 128 + tid]), c0 * C + c1);
+                }
             }
         }
 
-        // union of the probed lists, causal filter, E cap; rerank on the fly
+        // union of the probed lists in probe order, causal filter, E cap ...
         const int bq = t / Bs;
         const int lim = bq - L;
-        RegTop<R> rk;
-        rk.init();
+        int cid[E];
+#pragma unroll
+        for (int e = 0; e < E; ++e) cid[e] = 0;
         int nc = 0;
 #pragma unroll
         for (int r = 0; r < TP; ++r) {
-            if (nc >= E) break;
             const int a = top.a[r];
-            int lo = 0, hi = nb;
-            while (lo < hi) {
-                const int mid = (lo + hi) >> 1;
-                if (s_addr[mid] < a) lo = mid + 1;
-                else hi = mid;
-            }
-            for (int k = lo; k < nb && s_addr[k] == a && k - lo < cap && nc < E; ++k) {
+            int k = (nc < E && (unsigned)a < (unsigned)A) ? s_first[a] : -1;
+            if (k < 0) continue;
+            const int kend = min(nb, k + cap);
+            for (; k < kend && nc < E; ++k) {
+                if (s_addr[k] != a) break;
                 const int j = s_ids[k];
                 if (j > lim) break;
-                ++nc;
-                const float4 *kr = (const float4 *)(kbar + (bh * nb + j) * D);
-                float acc = 0.0f;
 #pragma unroll
-                for (int i4 = 0; i4 < D / 4; ++i4) {
-                    const float4 x = __ldg(kr + i4);
-                    acc = __fmaf_rn(q[4 * i4 + 0], x.x, acc);
-                    acc = __fmaf_rn(q[4 * i4 + 1], x.y, acc);
-                    acc = __fmaf_rn(q[4 * i4 + 2], x.z, acc);
-                    acc = __fmaf_rn(q[4 * i4 + 3], x.w, acc);
-                }
-                rk.push(acc, j);
+                for (int e = 0; e < E; ++e)
+                    if (e == nc) cid[e] = j;
+                ++nc;
             }
         }
+        // ... and the rerank q . kbar_j of the (at most E) candidates, their
+        // fma chains advancing together in ascending element order
+        float acc[E];
+#pragma unroll
+        for (int e = 0; e < E; ++e) acc[e] = 0.0f;
+        const float *kb = kbar + bh * nb * D;
+#pragma unroll 2
+        for (int i8 = 0; i8 < D / 8; ++i8) {
+            float qv[8];
+            if constexpr (sizeof(T) == 2) {
+                const uint4 u = __ldg((const uint4 *)(qp + 8 * i8));
+                const __nv_bfloat162 *h2 = (const __nv_bfloat162 *)&u;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 f = __bfloat1622float2(h2[e]);
+                    qv[2 * e] = f.x;
+                    qv[2 * e + 1] = f.y;
+                }
+            } else {
+                const float4 a = __ldg((const float4 *)(qp + 8 * i8)), b2 = __ldg((const float4 *)(qp + 8 * i8 + 4));
+                qv[0] = a.x; qv[1] = a.y; qv[2] = a.z; qv[3] = a.w;
+                qv[4] = b2.x; qv[5] = b2.y; qv[6] = b2.z; qv[7] = b2.w;
+            }
+#pragma unroll
+            for (int e = 0; e < E; ++e) {
+                if (e < nc) {
+                    const float4 *kr = (const float4 *)(kb + (size_t)cid[e] * D + 8 * i8);
+                    const float4 x = __ldg(kr), y = __ldg(kr + 1);
+                    float a = acc[e];
+                    a = __fmaf_rn(qv[0], x.x, a);
+                    a = __fmaf_rn(qv[1], x.y, a);
+                    a = __fmaf_rn(qv[2], x.z, a);
+                    a = __fmaf_rn(qv[3], x.w, a);
+                    a = __fmaf_rn(qv[4], y.x, a);
+                    a = __fmaf_rn(qv[5], y.y, a);
+                    a = __fmaf_rn(qv[6], y.z, a);
+                    a = __fmaf_rn(qv[7], y.w, a);
+                    acc[e] = a;
+                }
+            }
+        }
+        RegTop<R> rk;
+        rk.init();
+#pragma unroll
+        for (int e = 0; e < E; ++e)
+            if (e < nc) rk.push(acc[e], cid[e]);
         int ra[R];
         int nr = nc < R ? nc : R;
 #pragma unroll
@@ -843,7 +1000,7 @@ cudaError_t launch_queries(const Plan &p, const void *Q, const float *cb, const 
     // compile-time shapes of the configured workloads; any other shape takes the general kernel
 #define MONO_M2(TT, DD, CC, TPP, EE, RR)                                                                          \
     if (c.M == 2 && c.d == DD && c.C == CC && c.T == TPP && c.E == EE && c.R == RR) {                           \
-        const size_t sm2 = (size_t)CC * DD * 4 + (size_t)2 * CC * 128 * 4 + (size_t)p.nb * 8;                   \
+        const size_t sm2 = (size_t)CC * DD * 4 + (size_t)2 * CC * 128 * 4 + (size_t)CC * CC * 4 + (size_t)p.nb * 8;                   \
         auto kern = k_probe_m2<TT, DD, CC, TPP, EE, RR>;                                                        \
         if (sm2 > 48 * 1024 &&                                                                                   \
             (e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm2)) != cudaSuccess) \
