@@ -97,7 +97,10 @@ typedef struct mono_plan_s mono_plan_t;
 typedef struct mono_stats {
     int64_t overflow_total;    /* blocks dropped from full posting lists, all (b, h) */
     int32_t overflow_max_bh;   /* largest per-(b, h) overflow */
-    int32_t device_error;      /* 0, or the first device error code recorded */
+    int32_t device_error;      /* 0, or the first device error code recorded: 1 a sel id outside
+                                  [0, t/Bs - L], 2 probe candidate bound exceeded, 3 a bounded
+                                  wait ran out, 4 an address outside [0, C^M), 5 shared memory
+                                  not 1024-byte aligned */
     int64_t queries_lt_R;      /* query-heads that received fewer than R remote blocks */
     int64_t remote_selected;   /* total remote blocks selected */
     double mean_remote;        /* remote_selected / (B*H*S) */

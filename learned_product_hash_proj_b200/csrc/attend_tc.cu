@@ -18,6 +18,9 @@
 //     masked tile gives S and O.  The same CTA then reads the R remote
 //     partials of each query and merges them.
 // Scores are kept in the log2 domain: s2 = <q,k> * log2(e)/sqrt(d).
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include <algorithm>
 
 #include "internal.cuh"
@@ -155,31 +158,6 @@ __global__ void __launch_bounds__(256) k_pair_fill(const int32_t *__restrict__ s
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ uint4 ldg16(const void *p) { return __ldg((const uint4 *)p); }
 
-// rows [0, nrows) of a [*, D] bf16 matrix -> K-major tile (kdim = D); rows >= valid are zero.
-// Asynchronous: every copy is in flight at once; complete with cp_async_wait_all.
-// Thread idx copies chunk c of row 8g + r8 with (r8, c, g) = (idx % 8, idx / 8 % (D/8), idx / D):
-// its destination kmajor_chunk(row, c, D) is exactly 16 * idx, so a warp writes 512 contiguous bytes.
-template <int D>
-__device__ __forceinline__ void load_rows(uint8_t *tile, const bf16 *src, int nrows, int valid, int tid, int nthr) {
-    for (int idx = tid; idx < nrows * (D / 8); idx += nthr) {
-        const int row = (idx / D) * 8 + (idx & 7), c = (idx >> 3) % (D / 8);
-        const bool ok = row < valid;
-        tc::cp_async16(tile + 16 * idx, ok ? (const void *)(src + (size_t)row * D + 8 * c) : src, ok);
-    }
-}
-
-// rows [0, nkeys) of V ([*, D]) -> MN-major tile for the B operand of O = P V
-// (K = keys, N = dims); rows >= valid are zero.  Whole 16-byte chunks, no transpose.
-// Thread idx copies chunk c = idx / nkeys of key idx % nkeys: destination mnmajor_chunk = 16 * idx.
-template <int D>
-__device__ __forceinline__ void load_v(uint8_t *tile, const bf16 *src, int nkeys, int valid, int tid, int nthr) {
-    for (int idx = tid; idx < nkeys * (D / 8); idx += nthr) {
-        const int key = idx % nkeys, c = idx / nkeys;
-        const bool ok = key < valid;
-        tc::cp_async16(tile + 16 * idx, ok ? (const void *)(src + (size_t)key * D + 8 * c) : src, ok);
-    }
-}
-
 __device__ __forceinline__ uint32_t pack2(float a, float b) {
     __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
     return *(uint32_t *)&h;
@@ -193,36 +171,60 @@ __device__ __forceinline__ bool timed_out(const unsigned long long *counters) {
 // remote partials: persistent CTAs of 256 threads walk the work items
 // {block j, first pair, pair count} of a group of (b, h) slices with a
 // two-stage pipeline: while item k is computed, the tiles of item k+1 are in
-// flight (cp.async) and the descriptor and pair ids of item k+2 are being
-// loaded.  Per item: S = Q_sel K_j^T and O = P V_j on tcgen05 (TMEM, 64 or
-// 128 columns reused by every item), softmax in fp32, one partial per pair.
-// As in the local kernel, warps q and q+4 share TMEM lane quarter q and split
-// the columns.
+// flight and the descriptor and pair ids of item k+2 are being loaded.  K_j
+// and V_j arrive by TMA (128-byte swizzle, one thread issues them); the
+// gathered query rows by cp.async.  Per item: S = Q_sel K_j^T and O = P V_j on
+// tcgen05 (TMEM, 64 or 128 columns reused by every item), softmax in fp32,
+// one partial per pair.  As in the local kernel, warps q and q+4 share TMEM
+// lane quarter q and split the columns.
 // ---------------------------------------------------------------------------
 struct RemoteItem {
     long long bh;
     int j, p0, n;
 };
 
+// Q, K and V as [B*H, S, D] bf16 for TMA: 64-column (128-byte) boxes, 128-byte swizzle
+struct AttnMaps {
+    CUtensorMap q, k, v;
+};
+
+// dynamic shared memory of the remote kernel: two stages of {Q, K, V}, P (over
+// the stage's Q when it fits there), then the small state
 template <int D, int BS>
-__global__ void __launch_bounds__(256) k_remote_tc(const bf16 *__restrict__ Q, const bf16 *__restrict__ K,
-                                                   const bf16 *__restrict__ V, const int32_t *__restrict__ pairs,
-                                                   const int4 *__restrict__ work, const int32_t *__restrict__ nwork,
-                                                   bf16 *__restrict__ part_o, float2 *__restrict__ part_ml,
+struct RemoteSmem {
+    static constexpr int QB = 128 * D * 2, KB = BS * D * 2, VB = BS * D * 2, PB = 128 * BS * 2;
+    static constexpr int STAGE = QB + KB + VB;
+    static constexpr int P_OFF = PB <= QB ? -1 : 2 * STAGE;       // -1: P over the stage's Q
+    static constexpr int RED_OFF = 2 * STAGE + (PB <= QB ? 0 : PB);  // float [2][128]
+    static constexpr int PREF_OFF = RED_OFF + 1024;                // int [kMaxGroup + 1]
+    static constexpr int BAR_OFF = PREF_OFF + ((kMaxGroup + 1) * 4 + 15) / 16 * 16;  // 3 mbarriers + TMEM base
+    static constexpr int BYTES = BAR_OFF + 32;
+};
+
+template <int D, int BS>
+__global__ void __launch_bounds__(256) k_remote_tc(const __grid_constant__ AttnMaps maps, const bf16 *__restrict__ Q,
+                                                   const int32_t *__restrict__ pairs, const int4 *__restrict__ work,
+                                                   const int32_t *__restrict__ nwork, bf16 *__restrict__ part_o,
+                                                   float2 *__restrict__ part_ml,
                                                    unsigned long long *__restrict__ counters, int S, int R, int wcap,
                                                    float scale_log2, int bh0, int ng) {
     // TMEM: S in columns [0, BS); O overwrites them once every thread has turned S into P
     constexpr int NCOLS = (BS > D ? BS : D) <= 64 ? 64 : 128;
     constexpr int HALF = BS / 2, DH = D / 2;
-    static_assert(HALF % 32 == 0 && DH % 32 == 0, "tile shape");
-    constexpr int QB = 128 * D * 2, KB = BS * D * 2, VB = BS * D * 2, PB = 128 * BS * 2;
-    constexpr int STAGE = QB + KB + VB;
-    extern __shared__ __align__(128) uint8_t smem[];
-    __shared__ uint64_t mbar;
-    __shared__ uint32_t tmem_base;
-    __shared__ float s_red[2][128];
-    __shared__ int s_pref[kMaxGroup + 1];
+    static_assert(HALF % 32 == 0 && DH % 32 == 0 && D % 64 == 0, "tile shape");
+    using L = RemoteSmem<D, BS>;
+    constexpr int QB = L::QB, KB = L::KB, STAGE = L::STAGE;
+    extern __shared__ __align__(1024) uint8_t smem[];
+    float(*s_red)[128] = (float(*)[128])(smem + L::RED_OFF);
+    int *s_pref = (int *)(smem + L::PREF_OFF);
+    uint64_t *bar_kv = (uint64_t *)(smem + L::BAR_OFF);  // [2]: K/V of each stage landed
+    uint64_t *mbar = bar_kv + 2;                          // MMA completion
+    uint32_t *tmem_base = (uint32_t *)(mbar + 1);
     if (timed_out(counters)) return;
+    if (tc::smem_u32(smem) & 1023) {  // uniform; TMA's 128-byte swizzle needs 1024-byte aligned tiles
+        if (threadIdx.x == 0) record_error(counters, kDevErrSmemAlign);
+        return;
+    }
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int quarter = warp & 3, half = warp >> 2;
     const int row = quarter * 32 + lane;
@@ -231,17 +233,19 @@ __global__ void __launch_bounds__(256) k_remote_tc(const bf16 *__restrict__ Q, c
         int acc = 0;
         for (int g = 0; g < ng; ++g) { s_pref[g] = acc; acc += nwork[bh0 + g]; }
         s_pref[ng] = acc;
-        tc::mbar_init(&mbar, 1);
+        tc::mbar_init(&bar_kv[0], 1);
+        tc::mbar_init(&bar_kv[1], 1);
+        tc::mbar_init(mbar, 1);
         tc::fence_mbar_init();
     }
     if (warp == 0) {
-        tc::tmem_alloc(&tmem_base, NCOLS);
+        tc::tmem_alloc(tmem_base, NCOLS);
         tc::tmem_relinquish();
     }
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
-    const uint32_t tmem = tmem_base;
+    const uint32_t tmem = *tmem_base;
     const uint32_t trow = tmem + ((uint32_t)(quarter * 32) << 16);
     const int total = s_pref[ng];
     const int G = gridDim.x;
@@ -260,24 +264,35 @@ __global__ void __launch_bounds__(256) k_remote_tc(const bf16 *__restrict__ Q, c
         return it;
     };
     auto pair_of = [&](const RemoteItem &it) { return row < it.n ? pairs[it.bh * S * R + it.p0 + row] : 0; };
+    // the stage's tiles: K_j and V_j by TMA onto bar_kv[stage] (thread 0), the
+    // selected query rows by cp.async (every thread, one group)
     auto issue = [&](int stage, const RemoteItem &it, int pr) {
         uint8_t *sQ = smem + stage * STAGE, *sK = sQ + QB, *sV = sK + KB;
+        if (tid == 0) {
+            tc::mbar_expect_tx(&bar_kv[stage], 2 * KB);
+#pragma unroll
+            for (int a = 0; a < D / 64; ++a) {
+                tc::tma_load_3d(sK + a * (BS * 128), &maps.k, 64 * a, it.j * BS, (int)it.bh, &bar_kv[stage]);
+                tc::tma_load_3d(sV + a * (BS * 128), &maps.v, 64 * a, it.j * BS, (int)it.bh, &bar_kv[stage]);
+            }
+        }
         const bf16 *qrow = Q + ((size_t)it.bh * S + pr / R) * D;
 #pragma unroll
         for (int c = half * (D / 16); c < (half + 1) * (D / 16); ++c)
             tc::cp_async16(sQ + tc::kmajor_chunk(row, c, D), qrow + 8 * c, row < it.n);
-        const size_t kv0 = ((size_t)it.bh * S + (size_t)it.j * BS) * D;
-        load_rows<D>(sK, K + kv0, BS, BS, tid, 256);
-        load_v<D>(sV, V + kv0, BS, BS, tid, 256);
         asm volatile("cp.async.commit_group;" ::: "memory");
     };
 
     int f = blockIdx.x;
     bool ok = true;
+    // per stage: parity of the K/V loads issued and not yet seen complete, or -1
+    // (thread 0 issues and waits; before leaving it waits for what is left)
+    int pend[2] = {-1, -1};
     if (f < total) {
         RemoteItem it0 = descr(f);
         int pr0 = pair_of(it0);
         issue(0, it0, pr0);
+        pend[0] = 0;
         int f1 = f + G;
         bool have1 = f1 < total;
         RemoteItem it1{};
@@ -285,7 +300,12 @@ __global__ void __launch_bounds__(256) k_remote_tc(const bf16 *__restrict__ Q, c
         if (have1) { it1 = descr(f1); pr1 = pair_of(it1); }
         for (int k = 0; ok; ++k) {
             const int stage = k & 1;
-            if (have1) issue(stage ^ 1, it1, pr1);
+            const uint32_t kv_parity = (k >> 1) & 1;  // completions of bar_kv[stage] so far, mod 2
+            if (have1) {
+                issue(stage ^ 1, it1, pr1);
+                if (stage) pend[0] = ((k + 1) >> 1) & 1;
+                else pend[1] = ((k + 1) >> 1) & 1;
+            }
             const int f2 = f1 + G;
             const bool have2 = have1 && f2 < total;
             RemoteItem it2{};
@@ -293,22 +313,29 @@ __global__ void __launch_bounds__(256) k_remote_tc(const bf16 *__restrict__ Q, c
             if (have1) asm volatile("cp.async.wait_group 1;" ::: "memory");
             else asm volatile("cp.async.wait_group 0;" ::: "memory");
             tc::fence_smem_to_async();
+            const bool landed = tid != 0 || tc::mbar_wait(&bar_kv[stage], kv_parity);
+            if (landed) {
+                if (stage) pend[1] = -1;
+                else pend[0] = -1;
+            }
             tc::fence_before_sync();
-            __syncthreads();
+            ok = __syncthreads_and(landed);
             tc::fence_after_sync();
+            if (!ok) break;
             const int pr2 = have2 ? pair_of(it2) : 0;   // consumed next iteration
 
             uint8_t *sQ = smem + stage * STAGE, *sK = sQ + QB, *sV = sK + KB;
-            uint8_t *sP = PB <= QB ? sQ : smem + 2 * STAGE;
+            uint8_t *sP = L::P_OFF < 0 ? sQ : smem + L::P_OFF;
             if (tid == 0) {
                 const uint32_t id = tc::idesc_bf16(128, BS);
                 const uint32_t aq = tc::smem_u32(sQ), bk = tc::smem_u32(sK);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk)
-                    tc::mma_bf16(tmem, tc::desc_kmajor(aq + 256 * kk, D), tc::desc_kmajor(bk + 256 * kk, D), id, kk > 0);
-                tc::commit(&mbar);
+                    tc::mma_bf16(tmem, tc::desc_kmajor(aq + 256 * kk, D),
+                                 tc::desc_sw128(bk + (kk >> 2) * (BS * 128) + (kk & 3) * 32), id, kk > 0);
+                tc::commit(mbar);
             }
-            ok = __syncthreads_and(tc::mbar_wait(&mbar, 0));   // CTA-uniform: the loop below has barriers
+            ok = __syncthreads_and(tc::mbar_wait(mbar, 0));   // CTA-uniform: the code below has barriers
             tc::fence_after_sync();
             float v[32];
             float m = -INFINITY;
@@ -351,11 +378,11 @@ __global__ void __launch_bounds__(256) k_remote_tc(const bf16 *__restrict__ Q, c
                 const uint32_t ap = tc::smem_u32(sP), bv = tc::smem_u32(sV);
 #pragma unroll
                 for (int kk = 0; kk < BS / 16; ++kk)
-                    tc::mma_bf16(tmem, tc::desc_kmajor(ap + 256 * kk, BS), tc::desc_mnmajor(bv + 256 * kk, BS), id,
-                                 kk > 0);
-                tc::commit(&mbar);
+                    tc::mma_bf16(tmem, tc::desc_kmajor(ap + 256 * kk, BS), tc::desc_sw128_mn(bv + 2048 * kk, BS * 128),
+                                 id, kk > 0);
+                tc::commit(mbar);
             }
-            ok = __syncthreads_and(ok && tc::mbar_wait(&mbar, 1));
+            ok = __syncthreads_and(ok && tc::mbar_wait(mbar, 1));
             tc::fence_after_sync();
             const bool live = row < it0.n;
             const size_t slot = (size_t)it0.bh * S * R + pr0;
@@ -383,6 +410,11 @@ __global__ void __launch_bounds__(256) k_remote_tc(const bf16 *__restrict__ Q, c
             have1 = have2; f1 = f2;
         }
         asm volatile("cp.async.wait_group 0;" ::: "memory");
+        // leave no TMA write in flight into this CTA's shared memory
+        if (tid == 0) {
+            if (pend[0] >= 0 && !tc::mbar_wait(&bar_kv[0], (uint32_t)pend[0])) ok = false;
+            if (pend[1] >= 0 && !tc::mbar_wait(&bar_kv[1], (uint32_t)pend[1])) ok = false;
+        }
     }
     if (!ok && tid == 0) record_error(counters, kDevErrTimeout);
     tc::fence_before_sync();
@@ -392,55 +424,49 @@ __global__ void __launch_bounds__(256) k_remote_tc(const bf16 *__restrict__ Q, c
 
 // ---------------------------------------------------------------------------
 // local part + merge: persistent CTAs of 256 threads walk the 128-query tiles
-// of a group of (b, h) slices with a two-stage pipeline (the Q/K/V tiles of
-// tile k+1 are in flight while tile k is computed).  Per tile: S over the
-// tile's local key range (<= 256 keys) and O = P V on tcgen05, the masked
-// softmax in fp32, and the exact merge with the tile's remote partials.  TMEM
-// lane quarter q (rows 32q .. 32q+31) is read by warps q and q+4, each taking
-// half of the columns; their partial row max and sum meet in shared memory.
+// of a group of (b, h) slices.  Per tile: S over the tile's local key range
+// (<= 256 keys) and O = P V on tcgen05, the masked softmax in fp32, and the
+// exact merge with the tile's remote partials.  The Q, K and V tiles arrive
+// by TMA (128-byte swizzle; one thread issues them): the next tile's Q as
+// soon as this tile's S has been computed, its K and V once O has.  TMEM lane
+// quarter q (rows 32q .. 32q+31) is read by warps q and q+4, each taking half
+// of the columns; their partial row max and sum meet in shared memory (in the
+// K tile, which is free between the two MMAs).
 // ---------------------------------------------------------------------------
-// Shared-memory plan of the local kernel: ST stages of {Q, K, V} tiles; P over
-// the current stage's Q/K once S is computed (else a region of its own); a
-// 1 KB row-exchange buffer in stage space that P leaves free (else past the
-// end).  Two stages when they fit, else one (no prefetch).
-__host__ __device__ constexpr int local_p_offset(int ST, int STAGE, int QB, int KB, int PB, int stage) {
-    return PB <= QB + KB ? stage * STAGE : ST * STAGE;
-}
-__host__ __device__ constexpr int local_red_offset(int ST, int STAGE, int QB, int KB, int PB, int stage) {
-    return PB > QB + KB ? stage * STAGE : (PB + 1024 <= QB + KB ? stage * STAGE + PB : ST * STAGE + 1024 * stage);
-}
-__host__ __device__ constexpr size_t local_bytes(int ST, int STAGE, int QB, int KB, int PB) {
-    return (size_t)ST * STAGE + (PB > QB + KB ? PB : 0) + (PB <= QB + KB && PB + 1024 > QB + KB ? 1024 * ST : 0);
-}
 template <int D, int NK>
-constexpr int local_stages() {
-    constexpr int QB = 128 * D * 2, KB = NK * D * 2, VB = D * NK * 2, PB = 128 * NK * 2, STAGE = QB + KB + VB;
-    // one stage: two single-buffered CTAs per SM hide each other's load latency
-    // better than one double-buffered CTA (measured at the headline shape)
-    return local_bytes(2, STAGE, QB, KB, PB) <= 110 * 1024 ? 2 : 1;
-}
+struct LocalSmem {
+    static constexpr int QB = 128 * D * 2, KB = NK * D * 2, VB = NK * D * 2, PB = 128 * NK * 2;
+    static constexpr int Q_OFF = 0, K_OFF = QB, V_OFF = QB + KB, P_OFF = QB + KB + VB;
+    static constexpr int BAR_OFF = P_OFF + PB;  // 3 mbarriers + TMEM base
+    static constexpr int BYTES = BAR_OFF + 32;
+};
 template <int D, int NK>
 constexpr size_t local_smem() {
-    constexpr int QB = 128 * D * 2, KB = NK * D * 2, VB = D * NK * 2, PB = 128 * NK * 2, STAGE = QB + KB + VB;
-    return local_bytes(local_stages<D, NK>(), STAGE, QB, KB, PB);
+    return LocalSmem<D, NK>::BYTES;
 }
 
 template <int D, int BS, int NK, int RMAX>
-__global__ void __launch_bounds__(256) k_local_merge_tc(const bf16 *__restrict__ Q, const bf16 *__restrict__ K,
-                                                        const bf16 *__restrict__ V, const int32_t *__restrict__ sel,
+__global__ void __launch_bounds__(256) k_local_merge_tc(const __grid_constant__ AttnMaps maps,
+                                                        const int32_t *__restrict__ sel,
                                                         const bf16 *__restrict__ part_o,
                                                         const float2 *__restrict__ part_ml, bf16 *__restrict__ O,
                                                         unsigned long long *__restrict__ counters, int S, int H, int R,
                                                         int L, float scale_log2, int bh0, int ng) {
     constexpr int NCOLS = NK <= 128 ? 128 : 256;  // S: [0, NK); O reuses [0, D) after the softmax
     constexpr int HALF = NK / 2, DH = D / 2;
-    static_assert(NK <= 256 && HALF % 32 == 0 && DH % 32 == 0 && D <= NK, "tile shape");
-    constexpr int QB = 128 * D * 2, KB = NK * D * 2, VB = D * NK * 2, PB = 128 * NK * 2, STAGE = QB + KB + VB;
-    constexpr int ST = local_stages<D, NK>();
-    extern __shared__ __align__(128) uint8_t smem[];
-    __shared__ uint64_t mbar;
-    __shared__ uint32_t tmem_base;
+    static_assert(NK <= 256 && HALF % 32 == 0 && DH % 32 == 0 && D <= NK && D % 64 == 0, "tile shape");
+    using Lay = LocalSmem<D, NK>;
+    constexpr int QB = Lay::QB, KB = Lay::KB;
+    extern __shared__ __align__(1024) uint8_t smem[];
+    uint8_t *sQ = smem + Lay::Q_OFF, *sK = smem + Lay::K_OFF, *sV = smem + Lay::V_OFF, *sP = smem + Lay::P_OFF;
+    float(*s_red)[128] = (float(*)[128])sK;
+    uint64_t *bar_q = (uint64_t *)(smem + Lay::BAR_OFF), *bar_kv = bar_q + 1, *mbar = bar_q + 2;
+    uint32_t *tmem_base = (uint32_t *)(bar_q + 3);
     if (timed_out(counters)) return;
+    if (tc::smem_u32(smem) & 1023) {  // uniform; TMA's 128-byte swizzle needs 1024-byte aligned tiles
+        if (threadIdx.x == 0) record_error(counters, kDevErrSmemAlign);
+        return;
+    }
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int quarter = warp & 3, half = warp >> 2;
     const int row = quarter * 32 + lane;
@@ -449,31 +475,38 @@ __global__ void __launch_bounds__(256) k_local_merge_tc(const bf16 *__restrict__
     const int G = gridDim.x;
 
     if (warp == 0) {
-        tc::tmem_alloc(&tmem_base, NCOLS);
+        tc::tmem_alloc(tmem_base, NCOLS);
         tc::tmem_relinquish();
     }
     if (tid == 0) {
-        tc::mbar_init(&mbar, 1);
+        tc::mbar_init(bar_q, 1);
+        tc::mbar_init(bar_kv, 1);
+        tc::mbar_init(mbar, 1);
         tc::fence_mbar_init();
     }
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
-    const uint32_t tmem = tmem_base;
+    const uint32_t tmem = *tmem_base;
     const uint32_t trow = tmem + ((uint32_t)(quarter * 32) << 16);
 
-    auto issue = [&](int stage, int f) {
-        const long long bh = bh0 + f / ntiles;
-        const int t0 = (f % ntiles) * 128;
-        const int nq = min(128, S - t0);
+    // TMA of tile f's Q tile / K and V tiles (thread 0).  Rows past the end of
+    // the (b, h) slice read as zero.
+    auto issue_q = [&](int f) {
+        const int bh = bh0 + f / ntiles, t0 = (f % ntiles) * 128;
+        tc::mbar_expect_tx(bar_q, QB);
+#pragma unroll
+        for (int a = 0; a < D / 64; ++a) tc::tma_load_3d(sQ + a * (128 * 128), &maps.q, 64 * a, t0, bh, bar_q);
+    };
+    auto issue_kv = [&](int f) {
+        const int bh = bh0 + f / ntiles, t0 = (f % ntiles) * 128;
         const int kstart = max(0, t0 / BS - L + 1) * BS;
-        const int nk = min(S, t0 + 128) - kstart;
-        uint8_t *sQ = smem + stage * STAGE, *sK = sQ + QB, *sV = sK + KB;
-        const size_t base = (size_t)bh * S;
-        load_rows<D>(sQ, Q + (base + t0) * D, 128, nq, tid, 256);
-        load_rows<D>(sK, K + (base + kstart) * D, NK, nk, tid, 256);
-        load_v<D>(sV, V + (base + kstart) * D, NK, nk, tid, 256);
-        asm volatile("cp.async.commit_group;" ::: "memory");
+        tc::mbar_expect_tx(bar_kv, 2 * KB);
+#pragma unroll
+        for (int a = 0; a < D / 64; ++a) {
+            tc::tma_load_3d(sK + a * (NK * 128), &maps.k, 64 * a, kstart, bh, bar_kv);
+            tc::tma_load_3d(sV + a * (NK * 128), &maps.v, 64 * a, kstart, bh, bar_kv);
+        }
     };
 
     bool ok = true;
@@ -488,14 +521,19 @@ __global__ void __launch_bounds__(256) k_local_merge_tc(const bf16 *__restrict__
 #pragma unroll
         for (int r = 0; r < RMAX; ++r) selv[r] = (r < R && tt < S) ? sel[((size_t)bbh * S + tt) * R + r] : -1;
     };
+    // thread 0: the tile count k of the Q and of the K/V loads issued and not
+    // yet seen complete, or -1 (waited for before leaving)
+    int pend_q = -1, pend_kv = -1;
     if (f < total) {
-        issue(0, f);
+        if (tid == 0) {
+            issue_q(f);
+            issue_kv(f);
+            pend_q = pend_kv = 0;
+        }
         load_sel(f);
     }
     for (int k = 0; f < total && ok; ++k, f += G) {
-        const int stage = ST == 2 ? (k & 1) : 0;
         const bool have1 = f + G < total;
-        if (ST == 2 && have1) issue(stage ^ 1, f + G);
         // this tile's geometry; this row's remote selections, their (max, sum)
         // and partial rows are requested now and used by the merge at the end
         const long long bh = bh0 + f / ntiles;
@@ -525,25 +563,34 @@ __global__ void __launch_bounds__(256) k_local_merge_tc(const bf16 *__restrict__
             }
         }
         if (have1) load_sel(f + G);
-        if (ST == 2 && have1) asm volatile("cp.async.wait_group 1;" ::: "memory");
-        else asm volatile("cp.async.wait_group 0;" ::: "memory");
-        tc::fence_smem_to_async();
+        bool landed = true;
+        if (tid == 0) {
+            const uint32_t par = k & 1;  // each barrier completes once per tile
+            const bool lq = tc::mbar_wait(bar_q, par);
+            if (lq) pend_q = -1;
+            const bool lkv = lq && tc::mbar_wait(bar_kv, par);
+            if (lkv) pend_kv = -1;
+            landed = lq && lkv;
+        }
         tc::fence_before_sync();
-        __syncthreads();
+        ok = __syncthreads_and(landed);
         tc::fence_after_sync();
-        uint8_t *sQ = smem + stage * STAGE, *sK = sQ + QB, *sV = sK + KB;
-        uint8_t *sP = smem + local_p_offset(ST, STAGE, QB, KB, PB, stage);
-        float(*s_red)[128] = (float(*)[128])(smem + local_red_offset(ST, STAGE, QB, KB, PB, stage));
+        if (!ok) break;
         if (tid == 0) {
             const uint32_t id = tc::idesc_bf16(128, NK);
             const uint32_t aq = tc::smem_u32(sQ), bk = tc::smem_u32(sK);
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk)
-                tc::mma_bf16(tmem, tc::desc_kmajor(aq + 256 * kk, D), tc::desc_kmajor(bk + 256 * kk, D), id, kk > 0);
-            tc::commit(&mbar);
+                tc::mma_bf16(tmem, tc::desc_sw128(aq + (kk >> 2) * (128 * 128) + (kk & 3) * 32),
+                             tc::desc_sw128(bk + (kk >> 2) * (NK * 128) + (kk & 3) * 32), id, kk > 0);
+            tc::commit(mbar);
         }
-        ok = __syncthreads_and(tc::mbar_wait(&mbar, 0));
+        ok = __syncthreads_and(tc::mbar_wait(mbar, 0));
         tc::fence_after_sync();
+        if (tid == 0 && have1 && ok) {
+            issue_q(f + G);  // S is computed: the Q tile is free
+            pend_q = k + 1;
+        }
 
         // masked softmax of row t over keys s in [lo(t), t]; in column terms
         // [vlo, vhi].  32-column chunks entirely inside need no per-element
@@ -610,11 +657,17 @@ __global__ void __launch_bounds__(256) k_local_merge_tc(const bf16 *__restrict__
             const uint32_t ap = tc::smem_u32(sP), bv = tc::smem_u32(sV);
 #pragma unroll
             for (int kk = 0; kk < NK / 16; ++kk)
-                tc::mma_bf16(tmem, tc::desc_kmajor(ap + 256 * kk, NK), tc::desc_mnmajor(bv + 256 * kk, NK), id, kk > 0);
-            tc::commit(&mbar);
+                tc::mma_bf16(tmem, tc::desc_kmajor(ap + 256 * kk, NK), tc::desc_sw128_mn(bv + 2048 * kk, NK * 128),
+                             id, kk > 0);
+            tc::commit(mbar);
         }
-        ok = __syncthreads_and(ok && tc::mbar_wait(&mbar, 1));
+        ok = __syncthreads_and(ok && tc::mbar_wait(mbar, 1));
         tc::fence_after_sync();
+        if (tid == 0 && have1 && ok) {
+            tc::fence_smem_to_async();  // the row exchange in the K tile is read; TMA may overwrite it
+            issue_kv(f + G);            // O is computed: the K and V tiles are free
+            pend_kv = k + 1;
+        }
 
         // merge with the remote partials (max/sum rescaling), this thread's half of the columns
         float mm = m2;
@@ -668,11 +721,14 @@ __global__ void __launch_bounds__(256) k_local_merge_tc(const bf16 *__restrict__
             }
         }
         tc::fence_before_sync();
-        __syncthreads();  // the stage's tiles, P and TMEM are free again
+        __syncthreads();  // P and TMEM are free again
         tc::fence_after_sync();
-        if (ST == 1 && have1) issue(0, f + G);
     }
-    asm volatile("cp.async.wait_group 0;" ::: "memory");
+    // leave no TMA write in flight into this CTA's shared memory
+    if (tid == 0) {
+        if (pend_q >= 0 && !tc::mbar_wait(bar_q, pend_q & 1)) ok = false;
+        if (pend_kv >= 0 && !tc::mbar_wait(bar_kv, pend_kv & 1)) ok = false;
+    }
     if (!ok && tid == 0) record_error(counters, kDevErrTimeout);
     tc::fence_before_sync();
     __syncthreads();
@@ -709,10 +765,17 @@ static cudaError_t persistent_grid(F kernel, int threads, size_t smem, int *out)
     return cudaSuccess;
 }
 
-template <int D, int BS>
-constexpr size_t remote_smem() {
-    constexpr size_t QB = 128 * D * 2, KB = BS * D * 2, PB = 128 * BS * 2;
-    return 2 * (QB + 2 * KB) + (PB <= QB ? 0 : PB);
+// [B*H, S, D] bf16 tensor, boxes of 64 columns x box_rows rows x 1 slice, 128-byte swizzle
+static bool make_map_3d(CUtensorMap *map, const void *ptr, int D, int S, int BH, int box_rows) {
+    auto enc = (PFN_cuTensorMapEncodeTiled_v12000)tensor_map_encoder();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)S, (cuuint64_t)BH};
+    cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)S * D * 2};
+    cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 template <int D, int BS, int NK, int RMAX>
@@ -723,6 +786,12 @@ static cudaError_t launch_tc_shape(const Plan &p, const bf16 *Q, const bf16 *K, 
     const float scale_log2 = (float)(1.4426950408889634 / sqrt((double)c.d));
     const int nbh = c.B * c.H * p.nb;
     cudaError_t e;
+    AttnMaps lmaps, rmaps;
+    if (!make_map_3d(&lmaps.q, Q, D, c.S, c.B * c.H, 128) || !make_map_3d(&lmaps.k, K, D, c.S, c.B * c.H, NK) ||
+        !make_map_3d(&lmaps.v, V, D, c.S, c.B * c.H, NK) || !make_map_3d(&rmaps.q, Q, D, c.S, c.B * c.H, 128) ||
+        !make_map_3d(&rmaps.k, K, D, c.S, c.B * c.H, BS) || !make_map_3d(&rmaps.v, V, D, c.S, c.B * c.H, BS))
+        return cudaErrorInvalidValue;
+    constexpr size_t rsmem = RemoteSmem<D, BS>::BYTES;
     if (c.R > 0) {
         int32_t *pc = (int32_t *)ws_ptr(p, ws, kRegPairCount);
         int32_t *ps = (int32_t *)ws_ptr(p, ws, kRegPairStart);
@@ -743,8 +812,8 @@ static cudaError_t launch_tc_shape(const Plan &p, const bf16 *Q, const bf16 *K, 
         k_pair_count<<<gq, 256, hs, s>>>(sel, pc, c.S, c.R, p.nb, c.Bs, c.L, cnt_err);
         k_pair_scan<<<nbhh, 1024, 0, s>>>(pc, ps, pf, work, nwork, p.nb, wcap);
         k_pair_fill<<<gq, 256, 2 * hs, s>>>(sel, ps, pf, pairs, c.S, c.R, p.nb, c.Bs, c.L);
-        if ((e = cudaFuncSetAttribute(k_remote_tc<D, BS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      (int)remote_smem<D, BS>())) != cudaSuccess)
+        if ((e = cudaFuncSetAttribute(k_remote_tc<D, BS>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rsmem)) !=
+            cudaSuccess)
             return e;
         count_launches(3);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -758,7 +827,7 @@ static cudaError_t launch_tc_shape(const Plan &p, const bf16 *Q, const bf16 *K, 
     // (and its Q/K/V) are written by the remote kernel and read back by the
     // local kernel right after, while they are still resident in L2.
     int remote_ctas = 0;
-    if (c.R > 0 && (e = persistent_grid(k_remote_tc<D, BS>, 256, remote_smem<D, BS>(), &remote_ctas)) != cudaSuccess)
+    if (c.R > 0 && (e = persistent_grid(k_remote_tc<D, BS>, 256, rsmem, &remote_ctas)) != cudaSuccess)
         return e;
     const int nbhh = c.B * c.H;
     const size_t part_per_bh = (size_t)c.S * c.R * (2 * D + 8) + (size_t)3 * c.S * D * 2;
@@ -767,13 +836,13 @@ static cudaError_t launch_tc_shape(const Plan &p, const bf16 *Q, const bf16 *K, 
     for (int g0 = 0; g0 < nbhh; g0 += group) {
         const int ng = std::min(group, nbhh - g0);
         if (c.R > 0) {
-            k_remote_tc<D, BS><<<remote_ctas, 256, remote_smem<D, BS>(), s>>>(
-                Q, K, V, (const int32_t *)ws_ptr(p, ws, kRegPairs), (const int4 *)ws_ptr(p, ws, kRegWork),
+            k_remote_tc<D, BS><<<remote_ctas, 256, rsmem, s>>>(
+                rmaps, Q, (const int32_t *)ws_ptr(p, ws, kRegPairs), (const int4 *)ws_ptr(p, ws, kRegWork),
                 (const int32_t *)ws_ptr(p, ws, kRegNWork), (bf16 *)ws_ptr(p, ws, kRegPartO),
                 (float2 *)ws_ptr(p, ws, kRegPartML), cnt_err, c.S, c.R, p.max_work, scale_log2, g0, ng);
             count_launches(1);
         }
-        kl<<<local_ctas, 256, smem, s>>>(Q, K, V, sel, (const bf16 *)ws_ptr(p, ws, kRegPartO),
+        kl<<<local_ctas, 256, smem, s>>>(lmaps, sel, (const bf16 *)ws_ptr(p, ws, kRegPartO),
                                          (const float2 *)ws_ptr(p, ws, kRegPartML), O, cnt_err, c.S, c.H, c.R, c.L,
                                          scale_log2, g0, ng);
         count_launches(1);

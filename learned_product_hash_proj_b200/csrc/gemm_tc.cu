@@ -56,21 +56,8 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, i
         : "memory");
 }
 
-__device__ __forceinline__ void mbar_expect_tx(uint64_t *mbar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(tc::smem_u32(mbar)), "r"(bytes)
-                 : "memory");
-}
-
-// K-major, 128-byte swizzle: 8-row x 128-byte atoms, 1024 bytes apart.
-__device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr) {
-    uint64_t d = 0;
-    d |= (uint64_t)((saddr & 0x3FFFF) >> 4);
-    d |= (uint64_t)1 << 16;             // leading byte offset: unused for swizzled K-major
-    d |= (uint64_t)(1024 >> 4) << 32;   // stride byte offset: next 8-row atom
-    d |= (uint64_t)1 << 46;             // sm_100 descriptor version
-    d |= (uint64_t)2 << 61;             // SWIZZLE_128B
-    return d;
-}
+using tc::desc_sw128;
+using tc::mbar_expect_tx;
 
 __device__ __forceinline__ uint32_t pack2(float a, float b) {
     __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
@@ -185,16 +172,9 @@ __global__ void __launch_bounds__(192, 2) k_gemm_tc(const __grid_constant__ TmaM
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
-std::once_flag g_encode_once;
 
 bool get_encode() {
-    std::call_once(g_encode_once, [] {
-        void *fn = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            g_encode = (PFN_cuTensorMapEncodeTiled_v12000)fn;
-    });
+    g_encode = (PFN_cuTensorMapEncodeTiled_v12000)tensor_map_encoder();
     return g_encode != nullptr;
 }
 
@@ -209,6 +189,23 @@ bool make_map(CUtensorMap *map, const void *ptr, long long rows, int K, int box_
                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
+
+}  // namespace
+
+void *tensor_map_encoder() {
+    static std::once_flag once;
+    static void *fn = nullptr;
+    std::call_once(once, [] {
+        void *f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = f;
+    });
+    return fn;
+}
+
+namespace {
 
 cudaError_t launch(const TmaMaps &maps, const Epi &epi, int nz, int K, cudaStream_t s) {
     static bool attr_set = false;

@@ -25,6 +25,7 @@ enum DevErr : unsigned {
     kDevErrCandOverflow = 2, // probe candidate list exceeded its bound (never expected)
     kDevErrTimeout = 3,      // a bounded wait ran out
     kDevErrBadAddr = 4,      // an address outside [0, C^M)
+    kDevErrSmemAlign = 5,    // dynamic shared memory not 1024-byte aligned (TMA tiles need it)
 };
 
 // Counters at the start of the counter region (uint64 each).
@@ -99,6 +100,8 @@ cudaError_t launch_queries(const Plan &p, const void *Q, const float *cb, const 
 cudaError_t launch_attend_simt(const Plan &p, const void *Q, const void *K, const void *V, const int32_t *sel,
                                void *O, void *ws, cudaStream_t s);
 bool attend_tc_supported(const mono_config &c);
+// cuTensorMapEncodeTiled from the driver (a PFN_cuTensorMapEncodeTiled_v12000), or null
+void *tensor_map_encoder();
 bool gemm_tc_supported(const mono_config &c);
 cudaError_t launch_project_tc(const Plan &p, const void *x, const void *Wq, const void *Wk, const void *Wv, void *Q,
                               void *K, void *V, const void *ws, cudaStream_t s);
