@@ -651,13 +651,14 @@ __device__ __forceinline__ unsigned near_codes(const float (&s)[C], const float 
 
 // Of the near codes, those that some member of U does not dominate (the
 // pruning rule: u dominates p if s_u > s_p + delta, or s_u >= s_p and u < p).
-template <int T0>
-__device__ __forceinline__ unsigned undominated(unsigned near, const float *col, int stride, const float (&uv)[T0],
+template <int C, int T0>
+__device__ __forceinline__ unsigned undominated(unsigned near, const float (&s)[C], const float (&uv)[T0],
                                                 const int (&ui)[T0], float delta) {
     unsigned keep = 0;
-    for (unsigned m = near; m; m &= m - 1) {
-        const int c = __ffs(m) - 1;
-        const float sc = col[c * stride], hi = sc + delta;
+#pragma unroll
+    for (int c = 0; c < C; ++c) {
+        if (!((near >> c) & 1u)) continue;
+        const float sc = s[c], hi = sc + delta;
         bool dom = true;
 #pragma unroll
         for (int k = 0; k < T0; ++k) dom = dom && (uv[k] > hi || (uv[k] >= sc && ui[k] < c));
@@ -666,31 +667,37 @@ __device__ __forceinline__ unsigned undominated(unsigned near, const float *col,
     return keep;
 }
 
+// eight consecutive elements of a query row in shared memory, as fp32
+template <typename T>
+__device__ __forceinline__ void q8(const T *qm, float (&qv)[8]) {
+    if constexpr (sizeof(T) == 2) {
+        const uint4 u = *(const uint4 *)qm;
+        const __nv_bfloat162 *h2 = (const __nv_bfloat162 *)&u;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float2 f = __bfloat1622float2(h2[e]);
+            qv[2 * e] = f.x;
+            qv[2 * e + 1] = f.y;
+        }
+    } else {
+        const float4 a = ((const float4 *)qm)[0], b = ((const float4 *)qm)[1];
+        qv[0] = a.x; qv[1] = a.y; qv[2] = a.z; qv[3] = a.w;
+        qv[4] = b.x; qv[5] = b.y; qv[6] = b.z; qv[7] = b.w;
+    }
+}
+
 // Scores of one subspace: s[c] = q_m . codeword_{m,c}, one fma chain per code
 // in ascending element order (the chains advance together, eight elements at
-// a time, which changes nothing in any chain).  q is read from global memory
-// in pieces so that it never occupies registers as a whole.
+// a time, which changes nothing in any chain).  q_m is read from the query
+// tile in shared memory in pieces, so it never occupies registers as a whole.
 template <typename T, int DM, int C>
-__device__ __forceinline__ void sub_scores(const T *__restrict__ qm, const float *cbm, float (&s)[C]) {
+__device__ __forceinline__ void sub_scores(const T *qm, const float *cbm, float (&s)[C]) {
 #pragma unroll
     for (int c = 0; c < C; ++c) s[c] = 0.0f;
 #pragma unroll
     for (int i8 = 0; i8 < DM / 8; ++i8) {
         float qv[8];
-        if constexpr (sizeof(T) == 2) {
-            const uint4 u = __ldg((const uint4 *)(qm + 8 * i8));
-            const __nv_bfloat162 *h2 = (const __nv_bfloat162 *)&u;
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float2 f = __bfloat1622float2(h2[e]);
-                qv[2 * e] = f.x;
-                qv[2 * e + 1] = f.y;
-            }
-        } else {
-            const float4 a = __ldg((const float4 *)(qm + 8 * i8)), b = __ldg((const float4 *)(qm + 8 * i8 + 4));
-            qv[0] = a.x; qv[1] = a.y; qv[2] = a.z; qv[3] = a.w;
-            qv[4] = b.x; qv[5] = b.y; qv[6] = b.z; qv[7] = b.w;
-        }
+        q8<T>(qm + 8 * i8, qv);
 #pragma unroll
         for (int c = 0; c < C; ++c) {
             const float4 x = ((const float4 *)(cbm + c * DM + 8 * i8))[0];
@@ -709,6 +716,18 @@ __device__ __forceinline__ void sub_scores(const T *__restrict__ qm, const float
     }
 }
 
+// Row pitch (bytes) of the query tile in shared memory: the row plus 16 bytes,
+// so that the 16-byte reads of one warp (one row per lane) hit every bank once
+// per eight lanes.
+template <typename T, int D>
+constexpr int probe_q_pitch() {
+    return D * (int)sizeof(T) + 16;
+}
+template <typename T, int D, int C>
+constexpr size_t probe_m2_smem(int nb) {
+    return (size_t)C * D * 4 + (size_t)C * C * 4 + (size_t)128 * probe_q_pitch<T, D>() + (size_t)nb * 8;
+}
+
 template <typename T, int D, int C, int TP, int E, int R>
 __global__ void __launch_bounds__(128, C <= 16 ? 5 : 3) k_probe_m2(const T *__restrict__ Q, const float *__restrict__ kbar,
                                                      const float *__restrict__ cb, const int32_t *__restrict__ post_ids,
@@ -716,47 +735,65 @@ __global__ void __launch_bounds__(128, C <= 16 ? 5 : 3) k_probe_m2(const T *__re
                                                      const int32_t *__restrict__ forced, int32_t *__restrict__ sel,
                                                      unsigned long long *__restrict__ counters, int S, int H, int Bs,
                                                      int L, int cap) {
-    constexpr int DM = D / 2, A = C * C;
-    static_assert(C <= 32 && TP <= C * C && R >= 1 && E >= 1, "shape");
-    extern __shared__ float smem[];
+    constexpr int DM = D / 2, A = C * C, QP = probe_q_pitch<T, D>();
+    static_assert(C <= 32 && TP <= C * C && R >= 1 && E >= 1 && QP % 16 == 0, "shape");
+    extern __shared__ __align__(16) float smem[];
     const int nb = S / Bs;
     float *s_cb = smem;                                  // [2*C*DM] = C*D floats
-    float *s_sc = s_cb + C * D;                          // [2C][128] subspace scores, one column per thread
-    int32_t *s_first = (int32_t *)(s_sc + 2 * C * 128);  // [A] first position of each address, -1 if none
-    int32_t *s_addr = s_first + A;                       // [nb]
+    int32_t *s_first = (int32_t *)(s_cb + C * D);        // [A] first position of each address, -1 if none
+    uint8_t *s_q = (uint8_t *)(s_first + A);             // [128] query rows, pitch QP
+    int32_t *s_addr = (int32_t *)(s_q + 128 * QP);       // [nb]
     int32_t *s_ids = s_addr + nb;                        // [nb]
     const int h = blockIdx.y, b = blockIdx.z;
     const size_t bh = (size_t)b * H + h;
-    for (int i = threadIdx.x; i < C * D; i += blockDim.x) s_cb[i] = cb[(size_t)h * C * D + i];
-    for (int i = threadIdx.x; i < A; i += blockDim.x) s_first[i] = -1;
-    for (int i = threadIdx.x; i < nb; i += blockDim.x) {
-        s_addr[i] = post_addr[bh * nb + i];
-        s_ids[i] = post_ids[bh * nb + i];
+    const int tid = threadIdx.x;
+    const int t_lo = blockIdx.x * blockDim.x;
+    // Everything this CTA reads more than once goes to shared memory in one
+    // batch of asynchronous copies: its 128 query rows (contiguous in Q; rows
+    // past S as zero), the head's codebooks and the (b, h) posting arrays.
+    {
+        constexpr int CH = D * (int)sizeof(T) / 16;  // 16-byte chunks per query row
+        const uint8_t *src = (const uint8_t *)(Q + (bh * S + t_lo) * D);
+        for (int i = tid; i < 128 * CH; i += blockDim.x) {
+            const int r = i / CH, c = i % CH;
+            const bool ok = t_lo + r < S;
+            tc::cp_async16(s_q + r * QP + 16 * c, ok ? (const void *)(src + (size_t)r * (D * sizeof(T)) + 16 * c) : Q, ok);
+        }
+        const float *cbh = cb + (size_t)h * C * D;
+        for (int i = tid; i < C * D / 4; i += blockDim.x) tc::cp_async16(s_cb + 4 * i, cbh + 4 * i, true);
+        if ((nb & 3) == 0) {  // 16-byte aligned rows of the posting arrays
+            for (int i = tid; i < nb / 4; i += blockDim.x) {
+                tc::cp_async16(s_addr + 4 * i, post_addr + bh * nb + 4 * i, true);
+                tc::cp_async16(s_ids + 4 * i, post_ids + bh * nb + 4 * i, true);
+            }
+        } else {
+            for (int i = tid; i < nb; i += blockDim.x) {
+                s_addr[i] = post_addr[bh * nb + i];
+                s_ids[i] = post_ids[bh * nb + i];
+            }
+        }
     }
+    for (int i = tid; i < A; i += blockDim.x) s_first[i] = -1;
+    tc::cp_async_wait_all();
     __syncthreads();
     // the posting arrays are sorted by address: each address's entries start
     // where the address differs from the previous entry's
-    for (int i = threadIdx.x; i < nb; i += blockDim.x) {
+    for (int i = tid; i < nb; i += blockDim.x) {
         const int a = s_addr[i];
         if ((unsigned)a < (unsigned)A && (i == 0 || s_addr[i - 1] != a)) s_first[a] = i;
     }
     __syncthreads();
 
-    const int tid = threadIdx.x;
-    const int t = blockIdx.x * blockDim.x + tid;
+    const int t = t_lo + tid;
     int n_sel = 0, lt_r = 0, ign = 0;
     if (t < S) {
-        const T *qp = Q + (bh * S + t) * D;
-        // subspace scores; both also go to shared memory for the rare paths,
-        // which walk codes by index
+        const T *qp = (const T *)(s_q + tid * QP);
         float s0[C], s1[C];
         sub_scores<T, DM, C>(qp, s_cb, s0);
         sub_scores<T, DM, C>(qp + DM, s_cb + C * DM, s1);
         float mx0 = 0.f, mx1 = 0.f;
 #pragma unroll
         for (int c = 0; c < C; ++c) {
-            s_sc[c * 128 + tid] = s0[c];
-            s_sc[(C + c) * 128 + tid] = s1[c];
             mx0 = fmaxf(mx0, fabsf(s0[c]));
             mx1 = fmaxf(mx1, fabsf(s1[c]));
         }
@@ -786,8 +823,8 @@ __global__ void __launch_bounds__(128, C <= 16 ? 5 : 3) k_probe_m2(const T *__re
             cand0 = kAll;
             cand1 = kAll;
         } else if (nr0 | nr1) {
-            cand0 |= undominated<T0>(nr0, s_sc + tid, 128, uv0, ui0, delta);
-            cand1 |= undominated<T0>(nr1, s_sc + C * 128 + tid, 128, uv1, ui1, delta);
+            cand0 |= undominated<C, T0>(nr0, s0, uv0, ui0, delta);
+            cand1 |= undominated<C, T0>(nr1, s1, uv1, ui1, delta);
         }
         RegTop<TP> top;
         top.init();
@@ -811,13 +848,18 @@ __global__ void __launch_bounds__(128, C <= 16 ? 5 : 3) k_probe_m2(const T *__re
             done = vout < top.v[TP - 1];
         }
         if (!done) {
+            // general walk over cand0 x cand1 (rare: near ties); the scores are
+            // recomputed into arrays that can be indexed by code
+            float l0[C], l1[C];
+            sub_scores<T, DM, C>(qp, s_cb, l0);
+            sub_scores<T, DM, C>(qp + DM, s_cb + C * DM, l1);
             top.init();
             for (unsigned m0 = cand0; m0; m0 &= m0 - 1) {
                 const int c0 = __ffs(m0) - 1;
-                const float v0 = s_sc[c0 * 128 + tid];
+                const float v0 = l0[c0];
                 for (unsigned m1 = cand1; m1; m1 &= m1 - 1) {
                     const int c1 = __ffs(m1) - 1;
-                    top.push(__fadd_rn(v0, s_sc[(C + c1) * 128 + tid]), c0 * C + c1);
+                    top.push(__fadd_rn(v0, l1[c1]), c0 * C + c1);
                 }
             }
         }
@@ -843,6 +885,10 @@ __global__ void __launch_bounds__(128, C <= 16 ? 5 : 3) k_probe_m2(const T *__re
                 for (int e = 0; e < E; ++e)
                     if (e == nc) cid[e] = j;
                 ++nc;
+                // the rerank reads this row soon: start bringing it into L1 now
+                const float *kr = kbar + (bh * nb + j) * D;
+#pragma unroll
+                for (int o = 0; o < D; o += 32) asm volatile("prefetch.global.L1 [%0];" ::"l"(kr + o));
             }
         }
         // ... and the rerank q . kbar_j of the (at most E) candidates, their
@@ -854,20 +900,7 @@ __global__ void __launch_bounds__(128, C <= 16 ? 5 : 3) k_probe_m2(const T *__re
 #pragma unroll 2
         for (int i8 = 0; i8 < D / 8; ++i8) {
             float qv[8];
-            if constexpr (sizeof(T) == 2) {
-                const uint4 u = __ldg((const uint4 *)(qp + 8 * i8));
-                const __nv_bfloat162 *h2 = (const __nv_bfloat162 *)&u;
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float2 f = __bfloat1622float2(h2[e]);
-                    qv[2 * e] = f.x;
-                    qv[2 * e + 1] = f.y;
-                }
-            } else {
-                const float4 a = __ldg((const float4 *)(qp + 8 * i8)), b2 = __ldg((const float4 *)(qp + 8 * i8 + 4));
-                qv[0] = a.x; qv[1] = a.y; qv[2] = a.z; qv[3] = a.w;
-                qv[4] = b2.x; qv[5] = b2.y; qv[6] = b2.z; qv[7] = b2.w;
-            }
+            q8<T>(qp + 8 * i8, qv);
 #pragma unroll
             for (int e = 0; e < E; ++e) {
                 if (e < nc) {
@@ -1000,7 +1033,7 @@ cudaError_t launch_queries(const Plan &p, const void *Q, const float *cb, const 
     // compile-time shapes of the configured workloads; any other shape takes the general kernel
 #define MONO_M2(TT, DD, CC, TPP, EE, RR)                                                                          \
     if (c.M == 2 && c.d == DD && c.C == CC && c.T == TPP && c.E == EE && c.R == RR) {                           \
-        const size_t sm2 = (size_t)CC * DD * 4 + (size_t)2 * CC * 128 * 4 + (size_t)CC * CC * 4 + (size_t)p.nb * 8;                   \
+        const size_t sm2 = probe_m2_smem<TT, DD, CC>(p.nb);                                                     \
         auto kern = k_probe_m2<TT, DD, CC, TPP, EE, RR>;                                                        \
         if (sm2 > 48 * 1024 &&                                                                                   \
             (e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm2)) != cudaSuccess) \
