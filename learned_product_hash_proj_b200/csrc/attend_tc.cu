@@ -322,7 +322,6 @@ __global__ void __launch_bounds__(256) k_remote_tc(const __grid_constant__ AttnM
             ok = __syncthreads_and(landed);
             tc::fence_after_sync();
             if (!ok) break;
-            const int pr2 = have2 ? pair_of(it2) : 0;   // consumed next iteration
 
             uint8_t *sQ = smem + stage * STAGE, *sK = sQ + QB, *sV = sK + KB;
             uint8_t *sP = L::P_OFF < 0 ? sQ : smem + L::P_OFF;
@@ -373,6 +372,8 @@ __global__ void __launch_bounds__(256) k_remote_tc(const __grid_constant__ AttnM
             __syncthreads();
             tc::fence_after_sync();
             l = s_red[0][row] + s_red[1][row];
+            // pair ids of item k+2 (its descriptor load has landed by now), consumed next iteration
+            const int pr2 = have2 ? pair_of(it2) : 0;
             if (tid == 0 && ok) {
                 const uint32_t id = tc::idesc_bf16(128, D, true);
                 const uint32_t ap = tc::smem_u32(sP), bv = tc::smem_u32(sV);
@@ -736,6 +737,331 @@ __global__ void __launch_bounds__(256) k_local_merge_tc(const __grid_constant__ 
 }
 
 // ---------------------------------------------------------------------------
+// local part + merge, warp-specialised: one persistent CTA of 320 threads per
+// SM walks the 128-query tiles of a group of (b, h) slices.
+//   warp 0 (one lane)  TMA producer: the Q, K and V tiles of each tile into an
+//                      NST-deep ring of stages ("full" / "empty" mbarriers);
+//   warp 1 (one lane)  MMA issuer: S = Q K^T of tile i+1 is issued before
+//                      O = P V of tile i, so that the tensor core works on
+//                      one tile while the softmax runs on the other;
+//   warps 2-5, 6-9     two softmax groups that take alternate tiles, one
+//                      thread per query row: the masked softmax of S in fp32,
+//                      P (bf16) written back over S in tensor memory and
+//                      read from there by the P V MMA, then the merge with the
+//                      remote partials and the output row.
+// Tensor memory: 512 columns, 256 per group (S and P from column 0, O from
+// column 256 - D).  Every wait is bounded; a role that gives up sets a shared
+// abort flag that ends the others' waits, and the producer and the MMA issuer
+// wait for their own copies and MMAs in flight before the CTA exits.
+// ---------------------------------------------------------------------------
+template <int D, int NK>
+struct LocalWs {
+    static constexpr int QB = 128 * D * 2, KB = NK * D * 2, STAGE = QB + 2 * KB;
+    static constexpr int NST = (200 * 1024) / STAGE > 4 ? 4 : (200 * 1024) / STAGE;
+    static constexpr int O_COL = 256 - D;
+    static constexpr int BAR_OFF = NST * STAGE;
+    // mbarriers: full[NST], empty[NST], s_full[2], p_full[2], o_full[2], t_free[2], drain; then TMEM base, abort
+    static constexpr int NBAR = 2 * NST + 9;
+    static constexpr int BYTES = BAR_OFF + NBAR * 8 + 16;
+    static constexpr bool supported = NST >= 2 && NK + D <= 256 && D % 64 == 0 && NK % 32 == 0;
+};
+
+template <int D, int BS, int NK, int RMAX>
+__global__ void __launch_bounds__(320, 1) k_local_ws(const __grid_constant__ AttnMaps maps,
+                                                     const int32_t *__restrict__ sel, const bf16 *__restrict__ part_o,
+                                                     const float2 *__restrict__ part_ml, bf16 *__restrict__ O,
+                                                     unsigned long long *__restrict__ counters, int S, int H, int R,
+                                                     int L, float scale_log2, int bh0, int ng) {
+    using Lay = LocalWs<D, NK>;
+    static_assert(Lay::supported, "tile shape");
+    constexpr int QB = Lay::QB, KB = Lay::KB, STAGE = Lay::STAGE, NST = Lay::NST;
+    extern __shared__ __align__(1024) uint8_t smem[];
+    uint64_t *bars = (uint64_t *)(smem + Lay::BAR_OFF);
+    uint64_t *full = bars, *empty = bars + NST, *s_full = bars + 2 * NST, *p_full = s_full + 2, *o_full = s_full + 4,
+             *t_free = s_full + 6, *drain = s_full + 8;
+    uint32_t *tmem_base = (uint32_t *)(bars + Lay::NBAR);
+    volatile int *abort_flag = (volatile int *)(tmem_base + 1);
+    if (timed_out(counters)) return;
+    if (tc::smem_u32(smem) & 1023) {
+        if (threadIdx.x == 0) record_error(counters, kDevErrSmemAlign);
+        return;
+    }
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int ntiles = (S + 127) / 128;
+    const int total = ng * ntiles;
+    const int G = gridDim.x;
+    const int n = blockIdx.x < total ? (total - 1 - blockIdx.x) / G + 1 : 0;  // tiles of this CTA
+    auto tile_of = [&](int i) { return blockIdx.x + i * G; };
+
+    if (tid == 0) {
+        for (int s = 0; s < NST; ++s) {
+            tc::mbar_init(&full[s], 1);
+            tc::mbar_init(&empty[s], 1);
+        }
+        for (int g = 0; g < 2; ++g) {
+            tc::mbar_init(&s_full[g], 1);
+            tc::mbar_init(&p_full[g], 4);
+            tc::mbar_init(&o_full[g], 1);
+            tc::mbar_init(&t_free[g], 4);
+        }
+        tc::mbar_init(drain, 1);
+        *abort_flag = 0;
+        tc::fence_mbar_init();
+    }
+    if (warp == 1) {
+        tc::tmem_alloc(tmem_base, 512);
+        tc::tmem_relinquish();
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = *tmem_base;
+    bool ok = true;
+    auto fail = [&]() {
+        ok = false;
+        *abort_flag = 1;
+    };
+
+    if (warp == 0) {
+        // ---------------- TMA producer ----------------
+        if (lane == 0) {
+            int last_v[4] = {-1, -1, -1, -1};  // per stage: use count of its latest issue
+            for (int i = 0; i < n && ok; ++i) {
+                const int s = i % NST, v = i / NST;
+                if (v > 0 && !tc::mbar_wait_or_abort(&empty[s], (v - 1) & 1, abort_flag)) { fail(); break; }
+                const int f = tile_of(i);
+                const int bh = bh0 + f / ntiles, t0 = (f % ntiles) * 128;
+                const int kstart = max(0, t0 / BS - L + 1) * BS;
+                uint8_t *sQ = smem + s * STAGE, *sK = sQ + QB, *sV = sK + KB;
+                tc::mbar_expect_tx(&full[s], QB + 2 * KB);
+#pragma unroll
+                for (int a = 0; a < D / 64; ++a) {
+                    tc::tma_load_3d(sQ + a * (128 * 128), &maps.q, 64 * a, t0, bh, &full[s]);
+                    tc::tma_load_3d(sK + a * (NK * 128), &maps.k, 64 * a, kstart, bh, &full[s]);
+                    tc::tma_load_3d(sV + a * (NK * 128), &maps.v, 64 * a, kstart, bh, &full[s]);
+                }
+                last_v[s] = v;
+            }
+            // every copy issued has landed before the CTA may exit
+            for (int s = 0; s < NST; ++s)
+                if (last_v[s] >= 0 && !tc::mbar_wait(&full[s], last_v[s] & 1)) ok = false;
+        }
+    } else if (warp == 1) {
+        // ---------------- MMA issuer ----------------
+        if (lane == 0) {
+            const uint32_t id1 = tc::idesc_bf16(128, NK), id2 = tc::idesc_bf16(128, D, true);
+            auto mma1 = [&](int i) -> bool {
+                const int s = i % NST, v = i / NST, g = i & 1, u = i >> 1;
+                if (!tc::mbar_wait_or_abort(&full[s], v & 1, abort_flag)) return false;
+                if (u > 0 && !tc::mbar_wait_or_abort(&t_free[g], (u - 1) & 1, abort_flag)) return false;
+                tc::fence_after_sync();
+                const uint32_t aq = tc::smem_u32(smem + s * STAGE), bk = aq + QB;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk)
+                    tc::mma_bf16(tmem + g * 256, tc::desc_sw128(aq + (kk >> 2) * (128 * 128) + (kk & 3) * 32),
+                                 tc::desc_sw128(bk + (kk >> 2) * (NK * 128) + (kk & 3) * 32), id1, kk > 0);
+                tc::commit(&s_full[g]);
+                return true;
+            };
+            auto mma2 = [&](int i) -> bool {
+                const int s = i % NST, g = i & 1, u = i >> 1;
+                if (!tc::mbar_wait_or_abort(&p_full[g], u & 1, abort_flag)) return false;
+                tc::fence_after_sync();
+                const uint32_t bv = tc::smem_u32(smem + s * STAGE) + QB + KB;
+#pragma unroll
+                for (int kk = 0; kk < NK / 16; ++kk)
+                    tc::mma_bf16_ts(tmem + g * 256 + Lay::O_COL, tmem + g * 256 + 8 * kk,
+                                    tc::desc_sw128_mn(bv + 2048 * kk, NK * 128), id2, kk > 0);
+                tc::commit(&o_full[g]);
+                tc::commit(&empty[s]);
+                return true;
+            };
+            if (n > 0 && !mma1(0)) fail();
+            for (int i = 0; i < n && ok; ++i) {
+                if (i + 1 < n && !mma1(i + 1)) { fail(); break; }
+                if (!mma2(i)) { fail(); break; }
+            }
+            // every MMA issued has completed before the CTA may exit
+            tc::commit(drain);
+            if (!tc::mbar_wait(drain, 0)) ok = false;
+        }
+    } else {
+        // ---------------- softmax groups ----------------
+        const int g = (warp - 2) >> 2, quarter = warp & 3;
+        const int row = quarter * 32 + lane;
+        const uint32_t tS = tmem + g * 256 + ((uint32_t)(quarter * 32) << 16);
+        const uint32_t tO = tS + Lay::O_COL;
+        // remote partial rows held in registers from the tile's start (two of 64 or one of 128 values)
+        constexpr int kPre = D == 64 ? (RMAX < 2 ? RMAX : 2) : (RMAX < 1 ? RMAX : 1);
+        // this row's selections for the group's next tile, loaded one tile ahead
+        int selv[RMAX];
+        auto load_sel = [&](int i) {
+            const int f = tile_of(i);
+            const long long bh = bh0 + f / ntiles;
+            const int t = (f % ntiles) * 128 + row;
+#pragma unroll
+            for (int r = 0; r < RMAX; ++r) selv[r] = (r < R && t < S) ? sel[((size_t)bh * S + t) * R + r] : -1;
+        };
+        if (g < n) load_sel(g);
+        for (int i = g; i < n && ok; i += 2) {
+            const int u = i >> 1;
+            const int f = tile_of(i);
+            const long long bh = bh0 + f / ntiles;
+            const int b = (int)(bh / H), h = (int)(bh % H);
+            const int t0 = (f % ntiles) * 128;
+            const int kstart = max(0, t0 / BS - L + 1) * BS;
+            const int t = t0 + row;
+            const bool live = t < S;
+            // this row's remote selections, their (max, sum) and partial rows, requested now
+            int jr[RMAX];
+            float2 ml[RMAX];
+            uint4 pre[kPre > 0 ? kPre : 1][D / 8];
+#pragma unroll
+            for (int r = 0; r < RMAX; ++r) {
+                jr[r] = -1;
+                ml[r] = make_float2(0.f, 0.f);
+                const int j = selv[r];
+                if (!sel_valid(j, t, BS, L)) continue;
+                const size_t pq = ((size_t)bh * S + t) * R + r;
+                jr[r] = j;
+                ml[r] = part_ml[pq];
+                if (r < kPre) {
+#pragma unroll
+                    for (int q8 = 0; q8 < D / 8; ++q8)
+                        pre[r < kPre ? r : 0][q8] = __ldg((const uint4 *)(part_o + pq * D) + q8);
+                } else {
+                    tc::prefetch_l2(part_o + pq * D);
+                }
+            }
+            if (i + 2 < n) load_sel(i + 2);
+            // (the decision to go on is warp-uniform: the TMEM accesses below are warp-collective)
+            if (!__all_sync(0xffffffffu, tc::mbar_wait_or_abort(&s_full[g], u & 1, abort_flag))) { fail(); break; }
+            tc::fence_after_sync();
+
+            // masked softmax of row t over keys [lo(t), t]: columns [vlo, vhi]
+            const int lo = max(0, t / BS - L + 1) * BS;
+            const int vlo = lo - kstart, vhi = t - kstart;
+            float v[32];
+            float m = -INFINITY;
+            // (tcgen05.ld / st are warp-collective: every lane issues them, whatever its row needs)
+#pragma unroll 1
+            for (int c0 = 0; c0 < NK; c0 += 32) {
+                __syncwarp();
+                tc::tmem_ld32(tS + c0, v);
+                if (c0 + 31 < vlo || c0 > vhi) continue;
+                if (c0 >= vlo && c0 + 31 <= vhi) {
+#pragma unroll
+                    for (int k = 0; k < 32; ++k) m = fmaxf(m, v[k]);
+                } else {
+#pragma unroll
+                    for (int k = 0; k < 32; ++k)
+                        if (c0 + k >= vlo && c0 + k <= vhi) m = fmaxf(m, v[k]);
+                }
+            }
+            const float m2 = (m == -INFINITY) ? 0.f : m * scale_log2;
+            float l = 0.f;
+#pragma unroll 1
+            for (int c0 = 0; c0 < NK; c0 += 32) {
+                __syncwarp();
+                tc::tmem_ld32(tS + c0, v);
+                uint32_t pk[16];
+                if (c0 + 31 < vlo || c0 > vhi) {
+#pragma unroll
+                    for (int k = 0; k < 16; ++k) pk[k] = 0u;
+                } else {
+                    const bool full_chunk = c0 >= vlo && c0 + 31 <= vhi;
+#pragma unroll
+                    for (int k = 0; k < 16; ++k) {
+                        float a = exp2f(fmaf(v[2 * k], scale_log2, -m2));
+                        float bb = exp2f(fmaf(v[2 * k + 1], scale_log2, -m2));
+                        if (!full_chunk) {
+                            a = (c0 + 2 * k >= vlo && c0 + 2 * k <= vhi) ? a : 0.f;
+                            bb = (c0 + 2 * k + 1 >= vlo && c0 + 2 * k + 1 <= vhi) ? bb : 0.f;
+                        }
+                        l += a + bb;
+                        pk[k] = pack2(a, bb);
+                    }
+                }
+                // P over the columns of S already read (column c0/2 .. c0/2 + 15 of this row)
+                __syncwarp();
+                tc::tmem_st16(tS + (c0 >> 1), pk);
+            }
+            __syncwarp();
+            tc::tmem_st_wait();
+            tc::fence_before_sync();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&p_full[g]);
+
+            // merge with the remote partials (max/sum rescaling)
+            float mm = m2;
+#pragma unroll
+            for (int r = 0; r < RMAX; ++r)
+                if (jr[r] >= 0) mm = fmaxf(mm, ml[r].x);
+            const float wl = exp2f(m2 - mm);
+            float den = l * wl;
+            float wr[RMAX];
+#pragma unroll
+            for (int r = 0; r < RMAX; ++r) {
+                wr[r] = 0.f;
+                if (jr[r] >= 0) {
+                    wr[r] = ml[r].y * exp2f(ml[r].x - mm);
+                    den += wr[r];
+                }
+            }
+            const float inv = 1.f / den;
+            if (!__all_sync(0xffffffffu, tc::mbar_wait_or_abort(&o_full[g], u & 1, abort_flag))) { fail(); break; }
+            tc::fence_after_sync();
+            bf16 *orow = O + (((size_t)b * S + t) * H + h) * D;
+#pragma unroll
+            for (int c0 = 0; c0 < D; c0 += 32) {
+                __syncwarp();
+                tc::tmem_ld32(tO + c0, v);
+                if (live) {
+#pragma unroll
+                    for (int k = 0; k < 32; ++k) v[k] *= wl;
+#pragma unroll
+                    for (int r = 0; r < RMAX; ++r) {
+                        if (jr[r] < 0) continue;
+                        const uint4 *src = (const uint4 *)(part_o + (((size_t)bh * S + t) * R + r) * D + c0);
+#pragma unroll
+                        for (int q8 = 0; q8 < 4; ++q8) {
+                            uint4 u4;
+                            if (kPre > 0 && r < kPre) u4 = pre[r < kPre ? r : 0][(c0 >> 3) + q8];
+                            else u4 = __ldg(src + q8);
+                            const __nv_bfloat162 *h2 = (const __nv_bfloat162 *)&u4;
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const float2 fv = __bfloat1622float2(h2[e]);
+                                v[8 * q8 + 2 * e] = fmaf(wr[r], fv.x, v[8 * q8 + 2 * e]);
+                                v[8 * q8 + 2 * e + 1] = fmaf(wr[r], fv.y, v[8 * q8 + 2 * e + 1]);
+                            }
+                        }
+                    }
+                    uint4 *dst = (uint4 *)(orow + c0);
+#pragma unroll
+                    for (int q8 = 0; q8 < 4; ++q8)
+                        dst[q8] = make_uint4(pack2(v[8 * q8] * inv, v[8 * q8 + 1] * inv),
+                                             pack2(v[8 * q8 + 2] * inv, v[8 * q8 + 3] * inv),
+                                             pack2(v[8 * q8 + 4] * inv, v[8 * q8 + 5] * inv),
+                                             pack2(v[8 * q8 + 6] * inv, v[8 * q8 + 7] * inv));
+                }
+            }
+            tc::fence_before_sync();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&t_free[g]);
+        }
+    }
+    if (!ok) record_error(counters, kDevErrTimeout);
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    if (warp == 1) {
+        __syncwarp();
+        tc::tmem_dealloc(tmem, 512);
+    }
+}
+
+// ---------------------------------------------------------------------------
 bool attend_tc_supported(const mono_config &c) {
     if (c.dtype != MONO_BF16 || (c.d != 64 && c.d != 128) || (c.Bs != 64 && c.Bs != 128)) return false;
     const int nk = 128 + (c.L - 1) * c.Bs;
@@ -818,11 +1144,25 @@ static cudaError_t launch_tc_shape(const Plan &p, const bf16 *Q, const bf16 *K, 
         count_launches(3);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
-    const size_t smem = local_smem<D, NK>();
+    // the local part: the warp-specialised kernel where its stages and tensor
+    // memory fit, else the single-stage one
+    constexpr bool ws_local = LocalWs<D, NK>::supported;
+    const size_t smem = ws_local ? (size_t)LocalWs<D, NK>::BYTES : local_smem<D, NK>();
     auto kl = k_local_merge_tc<D, BS, NK, RMAX>;
-    if ((e = cudaFuncSetAttribute(kl, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess) return e;
     int local_ctas = 0;
-    if ((e = persistent_grid(kl, 256, smem, &local_ctas)) != cudaSuccess) return e;
+    if constexpr (ws_local) {
+        if ((e = cudaFuncSetAttribute(k_local_ws<D, BS, NK, RMAX>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)smem)) != cudaSuccess)
+            return e;
+        int dev = 0;
+        if ((e = cudaGetDevice(&dev)) != cudaSuccess ||
+            (e = cudaDeviceGetAttribute(&local_ctas, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+            return e;
+    } else {
+        if ((e = cudaFuncSetAttribute(kl, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
+            return e;
+        if ((e = persistent_grid(kl, 256, smem, &local_ctas)) != cudaSuccess) return e;
+    }
     // Remote then local, one group of (b, h) slices at a time: a group's partials
     // (and its Q/K/V) are written by the remote kernel and read back by the
     // local kernel right after, while they are still resident in L2.
@@ -842,9 +1182,16 @@ static cudaError_t launch_tc_shape(const Plan &p, const bf16 *Q, const bf16 *K, 
                 (float2 *)ws_ptr(p, ws, kRegPartML), cnt_err, c.S, c.R, p.max_work, scale_log2, g0, ng);
             count_launches(1);
         }
-        kl<<<local_ctas, 256, smem, s>>>(lmaps, sel, (const bf16 *)ws_ptr(p, ws, kRegPartO),
-                                         (const float2 *)ws_ptr(p, ws, kRegPartML), O, cnt_err, c.S, c.H, c.R, c.L,
-                                         scale_log2, g0, ng);
+        if constexpr (ws_local) {
+            const int tiles = ng * ((c.S + 127) / 128);
+            k_local_ws<D, BS, NK, RMAX><<<std::min(local_ctas, tiles), 320, smem, s>>>(
+                lmaps, sel, (const bf16 *)ws_ptr(p, ws, kRegPartO), (const float2 *)ws_ptr(p, ws, kRegPartML), O,
+                cnt_err, c.S, c.H, c.R, c.L, scale_log2, g0, ng);
+        } else {
+            kl<<<local_ctas, 256, smem, s>>>(lmaps, sel, (const bf16 *)ws_ptr(p, ws, kRegPartO),
+                                             (const float2 *)ws_ptr(p, ws, kRegPartML), O, cnt_err, c.S, c.H, c.R,
+                                             c.L, scale_log2, g0, ng);
+        }
         count_launches(1);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
