@@ -69,75 +69,114 @@ __global__ void __launch_bounds__(128) k_summary_assign(const T *__restrict__ K,
 
 // ---------------------------------------------------------------------------
 // (A2, A3) the same summaries with one warp per block: each lane owns D/32
-// adjacent columns and walks the block's rows in ascending t, so every row
-// read is one coalesced 128/256-byte load.  A CTA takes 4 consecutive blocks
-// of one (b, h) and keeps that head's codebook in shared memory.
-// grid (ceil(nb/4), H, B), 128 threads.
+// adjacent columns and walks the block's rows in ascending t, reading its
+// columns of a row as one 32- or 64-bit word.  A CTA takes 4 x bpw
+// consecutive blocks of one (b, h) (each warp bpw of them, all rows in flight
+// at once) and keeps that head's codebook in shared memory, transposed so that
+// lane mc reads codeword mc without bank conflicts.
+// grid (ceil(nb / (4 bpw)), H, B), 128 threads.
 // ---------------------------------------------------------------------------
+inline size_t summary_smem(int M, int C, int Bs, int D, int es, int bpw) {
+    return ((size_t)M * C * (D / M) + 4 * (size_t)D + 4 * (size_t)M * C) * 4 + 16 + (size_t)4 * bpw * Bs * D * es;
+}
+
 template <typename T, int D>
 __global__ void __launch_bounds__(128) k_summary_assign_w(const T *__restrict__ K, const float *__restrict__ cb,
                                                           float *__restrict__ kbar, int32_t *__restrict__ addr, int S,
-                                                          int Bs, int M, int C, int H) {
+                                                          int Bs, int M, int C, int H, int bpw) {
     constexpr int PER = D / 32;  // columns per lane
+    static_assert(PER == 2 || PER == 4, "D = 64 or 128");
     extern __shared__ __align__(16) float sm[];
-    const int dmp = D / M + 1;                     // padded codeword stride: lane mc reads bank (mc + i) % 32
-    float *s_cb = sm;                              // [M*C][dmp]
-    float *s_kb = s_cb + M * C * dmp;              // [4][D]
-    float *s_sc = s_kb + 4 * D;                    // [4][M*C]
-    T *s_rows = (T *)(((uintptr_t)(s_sc + 4 * M * C) + 15) & ~(uintptr_t)15);  // [4][Bs*D] staged rows
+    const int MC = M * C, dm = D / M;
+    float *s_cbT = sm;                              // [dm][M*C]: element i of codeword mc at i * MC + mc
+    float *s_kb = s_cbT + MC * dm;                  // [4][D]
+    float *s_sc = s_kb + 4 * D;                     // [4][M*C]
+    T *s_rows = (T *)(((uintptr_t)(s_sc + 4 * MC) + 15) & ~(uintptr_t)15);  // [4][bpw][Bs*D] staged rows
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int h = blockIdx.y, b = blockIdx.z;
     const int nb = S / Bs;
     const size_t bh = (size_t)b * H + h;
-    const int j = blockIdx.x * 4 + warp;
-    // every copy of this warp's block in flight at once
+    const int j0 = (blockIdx.x * 4 + warp) * bpw;
+    // every row copy of this warp's blocks in flight at once
     const int chunks = Bs * D * (int)sizeof(T) / 16;
-    T *rows = s_rows + (size_t)warp * Bs * D;
-    if (j < nb) {
-        const uint8_t *src = (const uint8_t *)(K + (bh * S + (size_t)j * Bs) * D);
-        for (int c = lane; c < chunks; c += 32) tc::cp_async16((uint8_t *)rows + 16 * c, src + 16 * c, true);
+    T *rows = s_rows + (size_t)warp * bpw * Bs * D;
+    for (int q = 0; q < bpw; ++q) {
+        if (j0 + q < nb) {
+            const uint8_t *src = (const uint8_t *)(K + (bh * S + (size_t)(j0 + q) * Bs) * D);
+            uint8_t *dst = (uint8_t *)(rows + (size_t)q * Bs * D);
+            for (int c = lane; c < chunks; c += 32) tc::cp_async16(dst + 16 * c, src + 16 * c, true);
+        }
     }
-    for (int i = threadIdx.x; i < C * D; i += blockDim.x) s_cb[(i / (D / M)) * dmp + i % (D / M)] = cb[(size_t)h * C * D + i];
+    // the head's codebook (C*D floats, [M][C][dm]), transposed, with independent 16-byte loads
+    {
+        const float4 *src = (const float4 *)(cb + (size_t)h * C * D);
+        for (int i4 = threadIdx.x; i4 < C * D / 4; i4 += blockDim.x) {
+            const float4 f = __ldg(src + i4);
+            const int mc = (4 * i4) / dm, i = (4 * i4) % dm;  // dm is a multiple of 4
+            s_cbT[(i + 0) * MC + mc] = f.x;
+            s_cbT[(i + 1) * MC + mc] = f.y;
+            s_cbT[(i + 2) * MC + mc] = f.z;
+            s_cbT[(i + 3) * MC + mc] = f.w;
+        }
+    }
     tc::cp_async_wait_all();
-    __syncwarp();
-    if (j < nb) {
-        float acc[PER];
-#pragma unroll
-        for (int e = 0; e < PER; ++e) acc[e] = 0.0f;
-        for (int t = 0; t < Bs; ++t) {
-#pragma unroll
-            for (int e = 0; e < PER; ++e) acc[e] = __fadd_rn(acc[e], to_f(rows[(size_t)t * D + lane * PER + e]));
-        }
-#pragma unroll
-        for (int e = 0; e < PER; ++e) {
-            const float v = __fdiv_rn(acc[e], (float)Bs);
-            s_kb[warp * D + lane * PER + e] = v;
-            kbar[(bh * nb + j) * D + lane * PER + e] = v;
-        }
-    }
     __syncthreads();
-    if (j >= nb) return;
-    const int dm = D / M;
-    for (int mc = lane; mc < M * C; mc += 32) {
-        const int m = mc / C;
-        const float *w = s_cb + mc * dmp;
-        const float *kv = s_kb + warp * D + m * dm;
-        float a = 0.0f;
-        for (int i = 0; i < dm; ++i) a = __fmaf_rn(kv[i], w[i], a);
-        s_sc[warp * M * C + mc] = a;
-    }
-    __syncwarp();
-    if (lane == 0) {
-        long long ad = 0;
-        const float *sc = s_sc + warp * M * C;
-        for (int m = 0; m < M; ++m) {
-            float best = sc[m * C];
-            int bc = 0;
-            for (int c = 1; c < C; ++c)
-                if (sc[m * C + c] > best) { best = sc[m * C + c]; bc = c; }
-            ad = ad * C + bc;
+    for (int q = 0; q < bpw; ++q) {
+        const int j = j0 + q;
+        if (j < nb) {
+            const T *rq = rows + (size_t)q * Bs * D;
+            float acc[PER];
+#pragma unroll
+            for (int e = 0; e < PER; ++e) acc[e] = 0.0f;
+            for (int t = 0; t < Bs; ++t) {
+                float v[PER];
+                if constexpr (sizeof(T) == 2) {
+                    if constexpr (PER == 2) {
+                        const float2 f = __bfloat1622float2(*(const __nv_bfloat162 *)(rq + (size_t)t * D + 2 * lane));
+                        v[0] = f.x; v[1] = f.y;
+                    } else {
+                        const uint2 u = *(const uint2 *)(rq + (size_t)t * D + 4 * lane);
+                        const float2 f0 = __bfloat1622float2(*(const __nv_bfloat162 *)&u.x);
+                        const float2 f1 = __bfloat1622float2(*(const __nv_bfloat162 *)&u.y);
+                        v[0] = f0.x; v[1] = f0.y; v[2] = f1.x; v[3] = f1.y;
+                    }
+                } else {
+#pragma unroll
+                    for (int e = 0; e < PER; ++e) v[e] = rq[(size_t)t * D + lane * PER + e];
+                }
+#pragma unroll
+                for (int e = 0; e < PER; ++e) acc[e] = __fadd_rn(acc[e], v[e]);
+            }
+#pragma unroll
+            for (int e = 0; e < PER; ++e) {
+                const float v = __fdiv_rn(acc[e], (float)Bs);
+                s_kb[warp * D + lane * PER + e] = v;
+                kbar[(bh * nb + j) * D + lane * PER + e] = v;
+            }
         }
-        addr[bh * nb + j] = (int32_t)ad;
+        __syncwarp();
+        if (j < nb) {
+            for (int mc = lane; mc < MC; mc += 32) {
+                const int m = mc / C;
+                const float *kv = s_kb + warp * D + m * dm;
+                float a = 0.0f;
+                for (int i = 0; i < dm; ++i) a = __fmaf_rn(kv[i], s_cbT[i * MC + mc], a);
+                s_sc[warp * MC + mc] = a;
+            }
+        }
+        __syncwarp();
+        // one lane per subspace: the first maximum wins (ascending c); lane 0 combines
+        int bc = 0;
+        if (j < nb && lane < M) {
+            const float *sc = s_sc + warp * MC + lane * C;
+            float best = sc[0];
+            for (int c = 1; c < C; ++c)
+                if (sc[c] > best) { best = sc[c]; bc = c; }
+        }
+        long long ad = 0;
+        for (int m = 0; m < M; ++m) ad = ad * C + __shfl_sync(0xffffffffu, bc, m);
+        if (j < nb && lane == 0) addr[bh * nb + j] = (int32_t)ad;
+        __syncwarp();
     }
 }
 
@@ -981,16 +1020,29 @@ cudaError_t launch_summaries(const Plan &p, const void *K, const float *cb, void
     unsigned long long *cnt = (unsigned long long *)ws_ptr(p, ws, kRegCounters);
     cudaError_t e = cudaMemsetAsync(cnt, 0, kCntN * 8, s);
     if (e != cudaSuccess) return e;
-    const size_t smem = ((size_t)c.M * c.C * (c.d / c.M + 1) + 4 * (size_t)c.d + 4 * (size_t)c.M * c.C) * 4 +
-                        4 * (size_t)c.Bs * c.d * p.es + 16;
-    dim3 g1((p.nb + 3) / 4, c.H, c.B);
+    // two blocks per warp when their rows fit in 64 KB per CTA, else one; blocks
+    // too large to stage take the plain kernel (one CTA per block)
+    const size_t block_bytes = (size_t)c.Bs * c.d * p.es;
+    const int bpw = 4 * 2 * block_bytes <= 64 * 1024 ? 2 : 1;
+    const size_t smem = summary_smem(c.M, c.C, c.Bs, c.d, (int)p.es, bpw);
+    if (smem > 160 * 1024) {
+        dim3 g0(p.nb, c.H, c.B);
+        if (c.dtype == MONO_BF16)
+            k_summary_assign<__nv_bfloat16><<<g0, 128, 0, s>>>((const __nv_bfloat16 *)K, cb, kbar, addr, c.S, c.d,
+                                                               c.Bs, c.M, c.C, c.H);
+        else
+            k_summary_assign<float><<<g0, 128, 0, s>>>((const float *)K, cb, kbar, addr, c.S, c.d, c.Bs, c.M, c.C, c.H);
+        count_launches(1);
+        return cudaGetLastError();
+    }
+    dim3 g1((p.nb + 4 * bpw - 1) / (4 * bpw), c.H, c.B);
 #define MONO_SUMW(TT, DD)                                                                                         \
     do {                                                                                                          \
         auto kern = k_summary_assign_w<TT, DD>;                                                                   \
         if (smem > 48 * 1024 &&                                                                                   \
             (e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess) \
             return e;                                                                                             \
-        kern<<<g1, 128, smem, s>>>((const TT *)K, cb, kbar, addr, c.S, c.Bs, c.M, c.C, c.H);                    \
+        kern<<<g1, 128, smem, s>>>((const TT *)K, cb, kbar, addr, c.S, c.Bs, c.M, c.C, c.H, bpw);               \
     } while (0)
     if (c.dtype == MONO_BF16) {
         if (c.d == 64) MONO_SUMW(__nv_bfloat16, 64);
