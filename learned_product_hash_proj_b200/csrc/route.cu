@@ -764,7 +764,7 @@ constexpr int probe_q_pitch() {
 }
 template <typename T, int D, int C>
 constexpr size_t probe_m2_smem(int nb) {
-    return (size_t)C * D * 4 + (size_t)C * C * 4 + (size_t)128 * probe_q_pitch<T, D>() + (size_t)nb * 8;
+    return (size_t)C * D * 4 + (size_t)C * C * 8 + (size_t)128 * probe_q_pitch<T, D>() + (size_t)nb * 8;
 }
 
 template <typename T, int D, int C, int TP, int E, int R>
@@ -779,8 +779,8 @@ __global__ void __launch_bounds__(128, C <= 16 ? 5 : 3) k_probe_m2(const T *__re
     extern __shared__ __align__(16) float smem[];
     const int nb = S / Bs;
     float *s_cb = smem;                                  // [2*C*DM] = C*D floats
-    int32_t *s_first = (int32_t *)(s_cb + C * D);        // [A] first position of each address, -1 if none
-    uint8_t *s_q = (uint8_t *)(s_first + A);             // [128] query rows, pitch QP
+    int2 *s_rng = (int2 *)(s_cb + C * D);                // [A] positions [first, end) of each address's entries
+    uint8_t *s_q = (uint8_t *)(s_rng + A);               // [128] query rows, pitch QP
     int32_t *s_addr = (int32_t *)(s_q + 128 * QP);       // [nb]
     int32_t *s_ids = s_addr + nb;                        // [nb]
     const int h = blockIdx.y, b = blockIdx.z;
@@ -812,14 +812,17 @@ __global__ void __launch_bounds__(128, C <= 16 ? 5 : 3) k_probe_m2(const T *__re
             }
         }
     }
-    for (int i = tid; i < A; i += blockDim.x) s_first[i] = -1;
+    for (int i = tid; i < A; i += blockDim.x) s_rng[i] = make_int2(0, 0);
     tc::cp_async_wait_all();
     __syncthreads();
     // the posting arrays are sorted by address: each address's entries start
-    // where the address differs from the previous entry's
+    // where the address differs from the previous entry's and end where it
+    // differs from the next one's
     for (int i = tid; i < nb; i += blockDim.x) {
         const int a = s_addr[i];
-        if ((unsigned)a < (unsigned)A && (i == 0 || s_addr[i - 1] != a)) s_first[a] = i;
+        if ((unsigned)a >= (unsigned)A) continue;
+        if (i == 0 || s_addr[i - 1] != a) s_rng[a].x = i;
+        if (i == nb - 1 || s_addr[i + 1] != a) s_rng[a].y = i + 1;
     }
     __syncthreads();
 
@@ -910,24 +913,22 @@ __global__ void __launch_bounds__(128, C <= 16 ? 5 : 3) k_probe_m2(const T *__re
 #pragma unroll
         for (int e = 0; e < E; ++e) cid[e] = 0;
         int nc = 0;
+        int2 rg[TP];  // every probed list's range, looked up at once
 #pragma unroll
         for (int r = 0; r < TP; ++r) {
             const int a = top.a[r];
-            int k = (nc < E && (unsigned)a < (unsigned)A) ? s_first[a] : -1;
-            if (k < 0) continue;
-            const int kend = min(nb, k + cap);
-            for (; k < kend && nc < E; ++k) {
-                if (s_addr[k] != a) break;
+            rg[r] = (unsigned)a < (unsigned)A ? s_rng[a] : make_int2(0, 0);
+        }
+#pragma unroll
+        for (int r = 0; r < TP; ++r) {
+            const int kend = min(rg[r].y, rg[r].x + cap);
+            for (int k = rg[r].x; k < kend && nc < E; ++k) {
                 const int j = s_ids[k];
                 if (j > lim) break;
 #pragma unroll
                 for (int e = 0; e < E; ++e)
                     if (e == nc) cid[e] = j;
                 ++nc;
-                // the rerank reads this row soon: start bringing it into L1 now
-                const float *kr = kbar + (bh * nb + j) * D;
-#pragma unroll
-                for (int o = 0; o < D; o += 32) asm volatile("prefetch.global.L1 [%0];" ::"l"(kr + o));
             }
         }
         // ... and the rerank q . kbar_j of the (at most E) candidates, their
