@@ -213,6 +213,78 @@ int mono_forward(const mono_plan_t *plan, const void *x, const void *Wq, const v
                  const void *Wv, const void *Wo, const float *codebooks, const int32_t *forced,
                  void *delta, void *workspace, void *stream);
 
+/* ------------------------------------------------------------------------
+ * Decode: one new token per sequence against caller-owned caches.
+ *
+ * The pages describe the batch forward only.  Every stage of it is causal
+ * (the posting lists keep the earliest `cap` blocks of each address, so a
+ * list at position t holds exactly the blocks a streaming build would hold),
+ * hence step t of the decode computes row t of mono_forward on the first t+1
+ * tokens: same projection, same routing decisions on the same Q/K values,
+ * same selected token set.  The incremental parts are the append of a block
+ * that position t completes to its posting list, and a single-query
+ * route + attend over the cache.
+ *
+ * The cache is one caller-allocated device buffer of mono_decode_cache_bytes
+ * bytes, for the plan's B, H and S (S = the largest context).  Its regions
+ * (enum mono_dec_region, located by mono_decode_cache_region):
+ * ------------------------------------------------------------------------ */
+enum mono_dec_region {
+    MONO_DEC_K = 0,        /* [B,H,S,d] dtype post-RoPE keys (the layout of mono_project's K) */
+    MONO_DEC_V = 1,        /* [B,H,S,d] dtype values */
+    MONO_DEC_KBAR = 2,     /* [B,H,nb,d] fp32 summaries of completed blocks */
+    MONO_DEC_ADDR = 3,     /* [B,H,nb] int32 product address of completed blocks */
+    MONO_DEC_COUNT = 4,    /* [B,H,A] int32 blocks that reached each address (kept: the first cap) */
+    MONO_DEC_HEAD = 5,     /* [B,H,A] int32 first kept block of each address, -1 if none */
+    MONO_DEC_TAIL = 6,     /* [B,H,A] int32 last kept block of each address */
+    MONO_DEC_NEXT = 7,     /* [B,H,nb] int32 next kept block of the same address, -1 at the end */
+    MONO_DEC_OVERFLOW = 8, /* [B,H] int32 blocks dropped from full lists */
+    MONO_DEC_Q = 9,        /* [B,H,d] dtype this step's post-RoPE query */
+    MONO_DEC_SEL = 10,     /* [B,H,R] int32 this step's remote blocks, ascending, -1 padded */
+    MONO_DEC_O = 11,       /* [B,H*d] dtype this step's attention output */
+    MONO_DEC_NREGIONS = 12
+};
+
+/* Size of the decode cache.  MONO_ERR_UNSUPPORTED if C^M > 4096. */
+int mono_decode_cache_bytes(const mono_plan_t *plan, size_t *bytes);
+
+/* Byte offset and size of a decode-cache region. */
+int mono_decode_cache_region(const mono_plan_t *plan, int region, size_t *offset, size_t *bytes);
+
+/* Start from a context of t0 tokens (0 <= t0 <= S) whose keys and values the
+ * caller has already written to the cache's K and V regions for positions
+ * < t0 (e.g. copied from mono_project's K and V): computes the summaries and
+ * addresses of the t0/Bs completed blocks (same arithmetic as
+ * mono_route_summaries) and builds their posting lists in ascending block
+ * order.  t0 = 0 empties the lists. */
+int mono_decode_prefill(const mono_plan_t *plan, int t0, const float *codebooks, void *cache, void *stream);
+
+/* One decode step at position t (steps in order t0, t0+1, ...; t < S).
+ * x_t [B,W] and delta_t [B,W] (dtype); weights as for mono_project and
+ * mono_out_project; forced_t [B,H] int32 or NULL (-1 = none), with the
+ * meaning it has in mono_route.  The stages, callable one at a time:
+ *  - mono_decode_project: q, k, v of x_t with RoPE at position t; q to the
+ *    cache's Q region, k and v appended to K and V at position t;
+ *  - mono_decode_route:   if t completes block j = t/Bs (t % Bs == Bs-1), its
+ *    summary and address and the append to its posting list (or the
+ *    overflow count); then the routing of the cache's Q: probe of the top-T
+ *    product addresses, union in probe order, blocks j <= t/Bs - L, E cap,
+ *    rerank by q.kbar, forced block -> the cache's SEL region;
+ *  - mono_decode_attend:  exact softmax of the cache's Q over the tokens of
+ *    the SEL blocks and the local tokens [max(0, t/Bs-L+1)*Bs, t] -> the
+ *    cache's O region (fp32 scores and accumulation);
+ *  - mono_decode_step:    the three, then delta_t = O Wo^T.
+ * Routing decisions use the fp32 order of mono_route, so for equal Q and K
+ * values the selections equal mono_route's row t. */
+int mono_decode_project(const mono_plan_t *plan, int t, const void *x_t, const void *Wq, const void *Wk,
+                        const void *Wv, void *cache, void *stream);
+int mono_decode_route(const mono_plan_t *plan, int t, const float *codebooks, const int32_t *forced_t, void *cache,
+                      void *stream);
+int mono_decode_attend(const mono_plan_t *plan, int t, void *cache, void *stream);
+int mono_decode_step(const mono_plan_t *plan, int t, const void *x_t, const void *Wq, const void *Wk,
+                     const void *Wv, const void *Wo, const float *codebooks, const int32_t *forced_t,
+                     void *delta_t, void *cache, void *stream);
+
 /* Synchronise `stream` and read the routing statistics and the device error
  * word of the last mono_route / mono_forward on `workspace`.  Returns
  * MONO_ERR_DEVICE if a kernel recorded an error. */

@@ -1,0 +1,638 @@
+// decode.cu -- one new token per sequence against caller-owned caches.
+//
+// Every stage of the mixer is causal, so decode step t computes row t of the
+// batch forward on the first t+1 tokens ("Monodratic Routes Sparse Attention
+// with Learned Product Hashes", Key Points: bounded causal posting lists; the
+// remio.ai article, section on retrieval decisions: lists keep the earliest
+// blocks of each address up to their capacity).  What is incremental:
+//   * the key and value of position t are appended to the cache;
+//   * when t completes block j, its summary kbar_j (mean of its post-RoPE
+//     keys), its product address and its append to that address's posting
+//     list (kept while the list holds fewer than cap blocks, else counted as
+//     overflow).  A list is a chain head -> next -> ... in ascending block id;
+//   * the query is routed against the lists: top-T product addresses by the
+//     summed subspace scores, union of their lists in probe order, causal
+//     filter j <= t/Bs - L, E cap, rerank by q.kbar, top R;
+//   * exact softmax over the tokens of the selected blocks plus the local
+//     tokens [max(0, t/Bs - L + 1) * Bs, t].
+// Routing decisions use the fp32 order of the batch kernels: dot products as
+// fma chains in ascending element order from +0, block sums in ascending t,
+// grid scores summed in ascending subspace order, ties to the lowest code,
+// address and block id.  For one query the exact top T is found by scoring
+// every one of the C^M addresses (C^M <= 4096).
+#include <cuda_runtime.h>
+
+#include <math.h>
+
+#include "internal.cuh"
+#include "mono.h"
+
+namespace mono {
+namespace {
+
+constexpr int kDecMaxA = 4096;
+
+struct DecLayout {
+    size_t off[MONO_DEC_NREGIONS];
+    size_t bytes[MONO_DEC_NREGIONS];
+    size_t total;
+};
+
+DecLayout dec_layout(const Plan &p) {
+    const mono_config &c = p.cfg;
+    const size_t B = c.B, H = c.H, S = c.S, d = c.d, nb = p.nb, A = (size_t)p.A, es = p.es;
+    const size_t R = c.R > 0 ? c.R : 1;
+    DecLayout L{};
+    size_t sz[MONO_DEC_NREGIONS] = {};
+    sz[MONO_DEC_K] = B * H * S * d * es;
+    sz[MONO_DEC_V] = B * H * S * d * es;
+    sz[MONO_DEC_KBAR] = B * H * nb * d * 4;
+    sz[MONO_DEC_ADDR] = B * H * nb * 4;
+    sz[MONO_DEC_COUNT] = B * H * A * 4;
+    sz[MONO_DEC_HEAD] = B * H * A * 4;
+    sz[MONO_DEC_TAIL] = B * H * A * 4;
+    sz[MONO_DEC_NEXT] = B * H * nb * 4;
+    sz[MONO_DEC_OVERFLOW] = B * H * 4;
+    sz[MONO_DEC_Q] = B * H * d * es;
+    sz[MONO_DEC_SEL] = B * H * R * 4;
+    sz[MONO_DEC_O] = B * H * d * es;
+    size_t o = 0;
+    for (int r = 0; r < MONO_DEC_NREGIONS; ++r) {
+        L.off[r] = o;
+        L.bytes[r] = sz[r];
+        o += (sz[r] + 255) / 256 * 256;
+    }
+    L.total = o;
+    return L;
+}
+
+struct DecPtrs {
+    void *K, *V, *Q, *O;
+    float *kbar;
+    int32_t *addr, *count, *head, *tail, *next, *overflow, *sel;
+};
+
+DecPtrs dec_ptrs(const DecLayout &L, void *cache) {
+    char *c = (char *)cache;
+    DecPtrs P;
+    P.K = c + L.off[MONO_DEC_K];
+    P.V = c + L.off[MONO_DEC_V];
+    P.Q = c + L.off[MONO_DEC_Q];
+    P.O = c + L.off[MONO_DEC_O];
+    P.kbar = (float *)(c + L.off[MONO_DEC_KBAR]);
+    P.addr = (int32_t *)(c + L.off[MONO_DEC_ADDR]);
+    P.count = (int32_t *)(c + L.off[MONO_DEC_COUNT]);
+    P.head = (int32_t *)(c + L.off[MONO_DEC_HEAD]);
+    P.tail = (int32_t *)(c + L.off[MONO_DEC_TAIL]);
+    P.next = (int32_t *)(c + L.off[MONO_DEC_NEXT]);
+    P.overflow = (int32_t *)(c + L.off[MONO_DEC_OVERFLOW]);
+    P.sel = (int32_t *)(c + L.off[MONO_DEC_SEL]);
+    return P;
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+// ---------------------------------------------------------------------------
+// projection of one token per sequence: one warp per interleaved output pair
+// (2i, 2i+1) of one head of one of Q, K, V, for all B sequences; lanes split
+// the W inputs, fp32 accumulation; RoPE on Q and K at position t (angles in
+// fp64); q to the Q region, k and v to the caches at position t.
+// grid ceil(3 H d/2 / 8), 256 threads.
+// ---------------------------------------------------------------------------
+template <typename T>
+__global__ void __launch_bounds__(256) k_dec_project(const T *__restrict__ x, const T *__restrict__ Wq,
+                                                     const T *__restrict__ Wk, const T *__restrict__ Wv, T *__restrict__ q,
+                                                     T *__restrict__ Kc, T *__restrict__ Vc, int t, int B, int W, int H,
+                                                     int d, int S, double theta) {
+    const int lane = threadIdx.x & 31;
+    const int gw = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    const int pairs = H * d / 2;
+    if (gw >= 3 * pairs) return;
+    const int which = gw / pairs, pr = gw % pairs;  // 0 q, 1 k, 2 v
+    const int h = (2 * pr) / d, i = pr % (d / 2);
+    const int n0 = h * d + 2 * i;
+    const T *Wm = which == 0 ? Wq : (which == 1 ? Wk : Wv);
+    const T *w0 = Wm + (size_t)n0 * W, *w1 = w0 + W;
+    double c = 1.0, s = 0.0;
+    if (which < 2) {
+        const double ang = (double)t * pow(theta, -2.0 * (double)i / (double)d);
+        c = cos(ang);
+        s = sin(ang);
+    }
+    for (int b = 0; b < B; ++b) {
+        const T *xb = x + (size_t)b * W;
+        float a0 = 0.f, a1 = 0.f;
+        for (int k = lane; k < W; k += 32) {
+            const float xv = to_f(xb[k]);
+            a0 = fmaf(xv, to_f(w0[k]), a0);
+            a1 = fmaf(xv, to_f(w1[k]), a1);
+        }
+        a0 = warp_sum(a0);
+        a1 = warp_sum(a1);
+        if (lane == 0) {
+            float r0 = a0, r1 = a1;
+            if (which < 2) {
+                r0 = (float)((double)a0 * c - (double)a1 * s);
+                r1 = (float)((double)a0 * s + (double)a1 * c);
+            }
+            T *dst;
+            if (which == 0) dst = q + ((size_t)b * H + h) * d + 2 * i;
+            else dst = (which == 1 ? Kc : Vc) + (((size_t)b * H + h) * S + t) * d + 2 * i;
+            dst[0] = from_f<T>(r0);
+            dst[1] = from_f<T>(r1);
+        }
+    }
+}
+
+// summary and address of block j of (b, h): lane owns columns lane, lane+32, ...
+// Same arithmetic as the batch summaries.  Returns the address (all lanes).
+template <typename T>
+__device__ int dec_summary(const T *Kc, const float *cb, float *kbar, int32_t *addr, size_t bh, int h, int j, int S,
+                           int Bs, int d, int M, int C, int nb, float *s_kb, float *s_sc) {
+    const int lane = threadIdx.x & 31;
+    const T *rows = Kc + (bh * S + (size_t)j * Bs) * d;
+    for (int i = lane; i < d; i += 32) {
+        float acc = 0.0f;
+        for (int tt = 0; tt < Bs; ++tt) acc = __fadd_rn(acc, to_f(rows[(size_t)tt * d + i]));
+        const float v = __fdiv_rn(acc, (float)Bs);
+        s_kb[i] = v;
+        kbar[(bh * nb + j) * d + i] = v;
+    }
+    __syncwarp();
+    const int dm = d / M;
+    for (int mc = lane; mc < M * C; mc += 32) {
+        const int m = mc / C;
+        const float *w = cb + ((size_t)h * M * C + mc) * dm;
+        float a = 0.0f;
+        for (int i = 0; i < dm; ++i) a = __fmaf_rn(s_kb[m * dm + i], w[i], a);
+        s_sc[mc] = a;
+    }
+    __syncwarp();
+    int ad = 0;
+    if (lane == 0) {
+        long long a = 0;
+        for (int m = 0; m < M; ++m) {
+            float best = s_sc[m * C];
+            int bc = 0;
+            for (int c2 = 1; c2 < C; ++c2)
+                if (s_sc[m * C + c2] > best) { best = s_sc[m * C + c2]; bc = c2; }
+            a = a * C + bc;
+        }
+        ad = (int)a;
+        addr[bh * nb + j] = ad;
+    }
+    __syncwarp();
+    return __shfl_sync(0xffffffffu, ad, 0);
+}
+
+// append block j to the list of address a (one thread).  A tail outside
+// [0, nb) -- a cache that mono_decode_prefill never initialised -- starts the
+// list afresh instead of writing out of bounds.
+__device__ __forceinline__ void dec_append(int32_t *count, int32_t *head, int32_t *tail, int32_t *next,
+                                           int32_t *overflow, size_t bh, long long A, int nb, int a, int j, int cap) {
+    const size_t ba = bh * A + a;
+    int cnt = count[ba];
+    if (cnt < 0 || (cnt > 0 && cnt < cap && (unsigned)tail[ba] >= (unsigned)nb)) cnt = 0;
+    if (cnt < cap) {
+        if (cnt == 0) head[ba] = j;
+        else next[bh * nb + tail[ba]] = j;
+        tail[ba] = j;
+        next[bh * nb + j] = -1;
+    } else {
+        overflow[bh] += 1;
+    }
+    count[ba] = cnt + 1;
+}
+
+// block completed at position t (one warp per (b, h)); grid (H, B), 32 threads
+template <typename T>
+__global__ void __launch_bounds__(32) k_dec_block(const T *__restrict__ Kc, const float *__restrict__ cb, DecPtrs P, int t,
+                                                  int S, int Bs, int d, int M, int C, int H, int nb, long long A,
+                                                  int cap) {
+    __shared__ float s_kb[kMaxD];
+    __shared__ float s_sc[kMaxM * kMaxC];
+    const int h = blockIdx.x, b = blockIdx.y;
+    const size_t bh = (size_t)b * H + h;
+    const int j = t / Bs;
+    const int a = dec_summary<T>(Kc, cb, P.kbar, P.addr, bh, h, j, S, Bs, d, M, C, nb, s_kb, s_sc);
+    if (threadIdx.x == 0) dec_append(P.count, P.head, P.tail, P.next, P.overflow, bh, A, nb, a, j, cap);
+}
+
+// prefill: summaries of blocks [0, nb0); grid (nb0, H, B), 32 threads
+template <typename T>
+__global__ void __launch_bounds__(32) k_dec_prefill_summaries(const T *__restrict__ Kc, const float *__restrict__ cb,
+                                                              DecPtrs P, int S, int Bs, int d, int M, int C, int H,
+                                                              int nb) {
+    __shared__ float s_kb[kMaxD];
+    __shared__ float s_sc[kMaxM * kMaxC];
+    const int j = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const size_t bh = (size_t)b * H + h;
+    dec_summary<T>(Kc, cb, P.kbar, P.addr, bh, h, j, S, Bs, d, M, C, nb, s_kb, s_sc);
+}
+
+// prefill: empty lists, then blocks [0, nb0) appended in ascending order; grid (H, B), 32 threads
+__global__ void __launch_bounds__(32) k_dec_prefill_lists(DecPtrs P, int nb0, int H, int nb, long long A, int cap) {
+    const int h = blockIdx.x, b = blockIdx.y;
+    const size_t bh = (size_t)b * H + h;
+    for (long long a = threadIdx.x; a < A; a += 32) {
+        P.count[bh * A + a] = 0;
+        P.head[bh * A + a] = -1;
+        P.tail[bh * A + a] = -1;
+    }
+    for (int j = threadIdx.x; j < nb; j += 32) P.next[bh * nb + j] = -1;
+    __syncwarp();
+    if (threadIdx.x == 0) {
+        P.overflow[bh] = 0;
+        for (int j = 0; j < nb0; ++j)
+            dec_append(P.count, P.head, P.tail, P.next, P.overflow, bh, A, nb, P.addr[bh * nb + j], j, cap);
+    }
+}
+
+__device__ __forceinline__ bool before(float v1, int a1, float v2, int a2) {
+    return v1 > v2 || (v1 == v2 && a1 < a2);
+}
+
+// ---------------------------------------------------------------------------
+// routing of the step's query, one warp per (b, h); grid (H, B), 32 threads
+// ---------------------------------------------------------------------------
+template <typename T>
+__global__ void __launch_bounds__(32) k_dec_route(const T *__restrict__ q, const float *__restrict__ cb,
+                                                  const int32_t *__restrict__ forced, DecPtrs P, int t, int Bs, int L,
+                                                  int R, int E, int M, int C, int TP, int cap, int H, int d, int nb,
+                                                  long long A) {
+    __shared__ float s_q[kMaxD];
+    __shared__ float s_sc[kMaxM * kMaxC];
+    __shared__ int s_top[kMaxT];
+    __shared__ int s_cand[kMaxE];
+    __shared__ float s_score[kMaxE];
+    const int lane = threadIdx.x;
+    const int h = blockIdx.x, b = blockIdx.y;
+    const size_t bh = (size_t)b * H + h;
+    for (int i = lane; i < d; i += 32) s_q[i] = to_f(q[bh * d + i]);
+    __syncwarp();
+    // subspace scores: fma chains in ascending element order from +0
+    const int dm = d / M;
+    for (int mc = lane; mc < M * C; mc += 32) {
+        const int m = mc / C;
+        const float *w = cb + ((size_t)h * M * C + mc) * dm;
+        float a = 0.0f;
+        for (int i = 0; i < dm; ++i) a = __fmaf_rn(s_q[m * dm + i], w[i], a);
+        s_sc[mc] = a;
+    }
+    __syncwarp();
+    // every address scored (subspace 0 most significant, summed in ascending
+    // subspace order); each lane keeps its top TP by (score desc, address asc)
+    float lv[kMaxT];
+    int la[kMaxT];
+    for (int k = 0; k < TP; ++k) { lv[k] = -INFINITY; la[k] = 0x7fffffff; }
+    for (long long ad = lane; ad < A; ad += 32) {
+        long long rest = ad, radix = A / C;
+        float v = 0.0f;
+        for (int m = 0; m < M; ++m) {
+            const int cm = (int)(rest / radix);
+            rest -= (long long)cm * radix;
+            radix /= C;
+            v = m == 0 ? s_sc[cm] : __fadd_rn(v, s_sc[m * C + cm]);
+        }
+        const int a32 = (int)ad;
+        if (!before(v, a32, lv[TP - 1], la[TP - 1])) continue;
+        int k = TP - 1;
+        while (k > 0 && before(v, a32, lv[k - 1], la[k - 1])) {
+            lv[k] = lv[k - 1];
+            la[k] = la[k - 1];
+            --k;
+        }
+        lv[k] = v;
+        la[k] = a32;
+    }
+    // merge: TP rounds of a warp argmax over the lanes' heads
+    int ptr = 0;
+    for (int r = 0; r < TP; ++r) {
+        float bv = ptr < TP ? lv[ptr] : -INFINITY;
+        int ba = ptr < TP ? la[ptr] : 0x7fffffff;
+        int bl = lane;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+            const int oa = __shfl_xor_sync(0xffffffffu, ba, o);
+            const int ol = __shfl_xor_sync(0xffffffffu, bl, o);
+            if (before(ov, oa, bv, ba)) { bv = ov; ba = oa; bl = ol; }
+        }
+        if (lane == 0) s_top[r] = ba;
+        if (lane == bl) ++ptr;
+    }
+    __syncwarp();
+    // union of the probed lists in probe order, causal filter, E cap
+    const int lim = t / Bs - L;
+    int nc = 0;
+    if (lane == 0) {
+        for (int r = 0; r < TP && nc < E; ++r) {
+            const int a = s_top[r];
+            if (a < 0 || (long long)a >= A || P.count[bh * A + a] <= 0) continue;
+            // at most cap kept entries; an id outside [0, nb) ends the walk
+            int steps = 0;
+            for (int j = P.head[bh * A + a]; (unsigned)j < (unsigned)nb && nc < E && steps < cap;
+                 j = P.next[bh * nb + j], ++steps) {
+                if (j > lim) break;  // ascending ids: the rest are later still
+                s_cand[nc++] = j;
+            }
+        }
+    }
+    nc = __shfl_sync(0xffffffffu, nc, 0);
+    __syncwarp();
+    // rerank: q . kbar_j, one candidate per lane
+    if (lane < nc) {
+        const float *kb = P.kbar + (bh * nb + s_cand[lane]) * d;
+        float a = 0.0f;
+        for (int i = 0; i < d; ++i) a = __fmaf_rn(s_q[i], kb[i], a);
+        s_score[lane] = a;
+    }
+    __syncwarp();
+    if (lane == 0) {
+        // top R by (score desc, id asc), in rank order
+        int ra[kMaxR];
+        int nr = 0;
+        bool used[kMaxE] = {};
+        for (; nr < R && nr < nc; ++nr) {
+            int bi = -1;
+            for (int e = 0; e < nc; ++e)
+                if (!used[e] && (bi < 0 || before(s_score[e], s_cand[e], s_score[bi], s_cand[bi]))) bi = e;
+            used[bi] = true;
+            ra[nr] = s_cand[bi];
+        }
+        if (forced) {
+            const int f = forced[bh];
+            if (f >= 0 && f <= lim) {
+                bool present = false;
+                for (int k = 0; k < nr; ++k) present |= ra[k] == f;
+                if (!present && R > 0) {
+                    if (nr < R) ra[nr++] = f;
+                    else ra[R - 1] = f;
+                }
+            }
+        }
+        // ascending ids, -1 padding
+        for (int x = 0; x < nr; ++x)
+            for (int y = 0; y + 1 < nr - x; ++y)
+                if (ra[y] > ra[y + 1]) { const int tmp = ra[y]; ra[y] = ra[y + 1]; ra[y + 1] = tmp; }
+        for (int k = 0; k < R; ++k) P.sel[bh * R + k] = k < nr ? ra[k] : -1;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// attention of the step's query: 4 warps split the keys, each with an online
+// softmax (lanes own d/32 dimensions), merged at the end; fp32 throughout.
+// grid (H, B), 128 threads
+// ---------------------------------------------------------------------------
+template <typename T>
+__global__ void __launch_bounds__(128) k_dec_attend(const T *__restrict__ q, const T *__restrict__ Kc,
+                                                    const T *__restrict__ Vc, const int32_t *__restrict__ sel,
+                                                    T *__restrict__ O, int t, int S, int Bs, int L, int R, int H, int d,
+                                                    float scale) {
+    constexpr int kPer = kMaxD / 32;
+    __shared__ float s_m[4], s_l[4];
+    __shared__ float s_acc[4][kMaxD];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int h = blockIdx.x, b = blockIdx.y;
+    const size_t bh = (size_t)b * H + h;
+    const int per = d / 32;
+    float qv[kPer];
+    for (int e = 0; e < per; ++e) qv[e] = to_f(q[bh * d + lane * per + e]);
+    const int bq = t / Bs, lim = bq - L;
+    int js[kMaxR];  // the selected remote blocks; ids outside [0, t/Bs - L] are skipped
+    int nr = 0;
+    for (int r = 0; r < R; ++r) {
+        const int j = sel[bh * R + r];
+        if (j >= 0 && j <= lim) js[nr++] = j;
+    }
+    const int lo = max(0, bq - L + 1) * Bs;
+    const int nkeys = nr * Bs + (t - lo + 1);
+    float m = -INFINITY, l = 0.f, acc[kPer];
+    for (int e = 0; e < per; ++e) acc[e] = 0.f;
+    for (int idx = warp; idx < nkeys; idx += 4) {
+        const int key = idx < nr * Bs ? js[idx / Bs] * Bs + idx % Bs : lo + (idx - nr * Bs);
+        const T *kr = Kc + (bh * S + key) * d + lane * per;
+        float part = 0.f;
+        for (int e = 0; e < per; ++e) part = fmaf(qv[e], to_f(kr[e]), part);
+        const float s = warp_sum(part) * scale;
+        const float mn = fmaxf(m, s);
+        const float corr = expf(m - mn), p = expf(s - mn);
+        l = l * corr + p;
+        const T *vr = Vc + (bh * S + key) * d + lane * per;
+        for (int e = 0; e < per; ++e) acc[e] = fmaf(p, to_f(vr[e]), acc[e] * corr);
+        m = mn;
+    }
+    if (lane == 0) {
+        s_m[warp] = m;
+        s_l[warp] = l;
+    }
+    for (int e = 0; e < per; ++e) s_acc[warp][lane * per + e] = acc[e];
+    __syncthreads();
+    if (warp == 0) {
+        float mm = -INFINITY;
+        for (int w = 0; w < 4; ++w) mm = fmaxf(mm, s_m[w]);
+        float den = 0.f, o[kPer];
+        for (int e = 0; e < per; ++e) o[e] = 0.f;
+        for (int w = 0; w < 4; ++w) {
+            if (s_m[w] == -INFINITY) continue;  // a warp without keys
+            const float f = expf(s_m[w] - mm);
+            den += s_l[w] * f;
+            for (int e = 0; e < per; ++e) o[e] += s_acc[w][lane * per + e] * f;
+        }
+        for (int e = 0; e < per; ++e) O[(size_t)b * H * d + (size_t)h * d + lane * per + e] = from_f<T>(o[e] / den);
+    }
+}
+
+// delta_t [B, W] = o [B, H d] Wo^T (Wo [W, H d]); one warp per output column
+template <typename T>
+__global__ void __launch_bounds__(256) k_dec_out(const T *__restrict__ o, const T *__restrict__ Wo,
+                                                 T *__restrict__ delta, int B, int W, int N) {
+    const int lane = threadIdx.x & 31;
+    const int w = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (w >= W) return;
+    const T *wr = Wo + (size_t)w * N;
+    for (int b = 0; b < B; ++b) {
+        const T *ob = o + (size_t)b * N;
+        float a = 0.f;
+        for (int k = lane; k < N; k += 32) a = fmaf(to_f(ob[k]), to_f(wr[k]), a);
+        a = warp_sum(a);
+        if (lane == 0) delta[(size_t)b * W + w] = from_f<T>(a);
+    }
+}
+
+int dec_check(const mono_plan_t *plan, const void *cache) {
+    if (!plan) return MONO_ERR_NULL;
+    if (!cache) return MONO_ERR_WORKSPACE;
+    if (((uintptr_t)cache & 255) != 0) return MONO_ERR_ALIGN;
+    if (plan->p.A > kDecMaxA) return MONO_ERR_UNSUPPORTED;
+    return MONO_OK;
+}
+
+int dec_status(cudaError_t e) { return e == cudaSuccess ? MONO_OK : MONO_ERR_CUDA; }
+
+bool dec_empty(const Plan &p) { return p.cfg.B == 0 || p.cfg.S == 0; }
+
+}  // namespace
+}  // namespace mono
+
+using namespace mono;
+
+extern "C" {
+
+int mono_decode_cache_bytes(const mono_plan_t *plan, size_t *bytes) {
+    if (!plan || !bytes) return MONO_ERR_NULL;
+    if (plan->p.A > kDecMaxA) return MONO_ERR_UNSUPPORTED;
+    *bytes = dec_layout(plan->p).total;
+    return MONO_OK;
+}
+
+int mono_decode_cache_region(const mono_plan_t *plan, int region, size_t *offset, size_t *bytes) {
+    if (!plan || !offset || !bytes) return MONO_ERR_NULL;
+    if (region < 0 || region >= MONO_DEC_NREGIONS) return MONO_ERR_INVALID;
+    const DecLayout L = dec_layout(plan->p);
+    *offset = L.off[region];
+    *bytes = L.bytes[region];
+    return MONO_OK;
+}
+
+int mono_decode_prefill(const mono_plan_t *plan, int t0, const float *codebooks, void *cache, void *stream) {
+    int st = dec_check(plan, cache);
+    if (st) return st;
+    const Plan &p = plan->p;
+    const mono_config &c = p.cfg;
+    if (t0 < 0 || t0 > c.S) return MONO_ERR_INVALID;
+    if (dec_empty(p)) return MONO_OK;
+    if (!codebooks) return MONO_ERR_NULL;
+    const DecLayout L = dec_layout(p);
+    const DecPtrs P = dec_ptrs(L, cache);
+    cudaStream_t s = (cudaStream_t)stream;
+    const int nb0 = t0 / c.Bs;
+    if (nb0 > 0) {
+        dim3 g(nb0, c.H, c.B);
+        if (c.dtype == MONO_BF16)
+            k_dec_prefill_summaries<__nv_bfloat16><<<g, 32, 0, s>>>((const __nv_bfloat16 *)P.K, codebooks, P, c.S, c.Bs,
+                                                                   c.d, c.M, c.C, c.H, p.nb);
+        else
+            k_dec_prefill_summaries<float><<<g, 32, 0, s>>>((const float *)P.K, codebooks, P, c.S, c.Bs, c.d, c.M, c.C,
+                                                            c.H, p.nb);
+        count_launches(1);
+    }
+    k_dec_prefill_lists<<<dim3(c.H, c.B), 32, 0, s>>>(P, nb0, c.H, p.nb, p.A, c.cap);
+    count_launches(1);
+    return dec_status(cudaGetLastError());
+}
+
+int mono_decode_project(const mono_plan_t *plan, int t, const void *x_t, const void *Wq, const void *Wk,
+                        const void *Wv, void *cache, void *stream) {
+    int st = dec_check(plan, cache);
+    if (st) return st;
+    const Plan &p = plan->p;
+    const mono_config &c = p.cfg;
+    if (t < 0 || t >= c.S) return MONO_ERR_INVALID;
+    if (dec_empty(p)) return MONO_OK;
+    if (!x_t || !Wq || !Wk || !Wv) return MONO_ERR_NULL;
+    const DecPtrs P = dec_ptrs(dec_layout(p), cache);
+    const int warps = 3 * c.H * c.d / 2;
+    const int grid = (warps + 7) / 8;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (c.dtype == MONO_BF16)
+        k_dec_project<__nv_bfloat16><<<grid, 256, 0, s>>>(
+            (const __nv_bfloat16 *)x_t, (const __nv_bfloat16 *)Wq, (const __nv_bfloat16 *)Wk,
+            (const __nv_bfloat16 *)Wv, (__nv_bfloat16 *)P.Q, (__nv_bfloat16 *)P.K, (__nv_bfloat16 *)P.V, t, c.B, c.W,
+            c.H, c.d, c.S, c.rope_theta);
+    else
+        k_dec_project<float><<<grid, 256, 0, s>>>((const float *)x_t, (const float *)Wq, (const float *)Wk,
+                                                  (const float *)Wv, (float *)P.Q, (float *)P.K, (float *)P.V, t, c.B,
+                                                  c.W, c.H, c.d, c.S, c.rope_theta);
+    count_launches(1);
+    return dec_status(cudaGetLastError());
+}
+
+int mono_decode_route(const mono_plan_t *plan, int t, const float *codebooks, const int32_t *forced_t, void *cache,
+                      void *stream) {
+    int st = dec_check(plan, cache);
+    if (st) return st;
+    const Plan &p = plan->p;
+    const mono_config &c = p.cfg;
+    if (t < 0 || t >= c.S) return MONO_ERR_INVALID;
+    if (dec_empty(p)) return MONO_OK;
+    if (!codebooks) return MONO_ERR_NULL;
+    if (forced_t && ((uintptr_t)forced_t & 3)) return MONO_ERR_ALIGN;
+    const DecPtrs P = dec_ptrs(dec_layout(p), cache);
+    cudaStream_t s = (cudaStream_t)stream;
+    const dim3 g(c.H, c.B);
+    const bool bf = c.dtype == MONO_BF16;
+    if (t % c.Bs == c.Bs - 1) {  // position t completes block t / Bs
+        if (bf)
+            k_dec_block<__nv_bfloat16><<<g, 32, 0, s>>>((const __nv_bfloat16 *)P.K, codebooks, P, t, c.S, c.Bs, c.d,
+                                                        c.M, c.C, c.H, p.nb, p.A, c.cap);
+        else
+            k_dec_block<float><<<g, 32, 0, s>>>((const float *)P.K, codebooks, P, t, c.S, c.Bs, c.d, c.M, c.C, c.H,
+                                                p.nb, p.A, c.cap);
+        count_launches(1);
+    }
+    if (c.R > 0) {
+        if (bf)
+            k_dec_route<__nv_bfloat16><<<g, 32, 0, s>>>((const __nv_bfloat16 *)P.Q, codebooks, forced_t, P, t, c.Bs,
+                                                        c.L, c.R, c.E, c.M, c.C, c.T, c.cap, c.H, c.d, p.nb, p.A);
+        else
+            k_dec_route<float><<<g, 32, 0, s>>>((const float *)P.Q, codebooks, forced_t, P, t, c.Bs, c.L, c.R, c.E,
+                                                c.M, c.C, c.T, c.cap, c.H, c.d, p.nb, p.A);
+        count_launches(1);
+    }
+    return dec_status(cudaGetLastError());
+}
+
+int mono_decode_attend(const mono_plan_t *plan, int t, void *cache, void *stream) {
+    int st = dec_check(plan, cache);
+    if (st) return st;
+    const Plan &p = plan->p;
+    const mono_config &c = p.cfg;
+    if (t < 0 || t >= c.S) return MONO_ERR_INVALID;
+    if (dec_empty(p)) return MONO_OK;
+    const DecPtrs P = dec_ptrs(dec_layout(p), cache);
+    const float scale = (float)(1.0 / sqrt((double)c.d));
+    const dim3 g(c.H, c.B);
+    cudaStream_t s = (cudaStream_t)stream;
+    if (c.dtype == MONO_BF16)
+        k_dec_attend<__nv_bfloat16><<<g, 128, 0, s>>>((const __nv_bfloat16 *)P.Q, (const __nv_bfloat16 *)P.K,
+                                                      (const __nv_bfloat16 *)P.V, P.sel, (__nv_bfloat16 *)P.O, t, c.S,
+                                                      c.Bs, c.L, c.R, c.H, c.d, scale);
+    else
+        k_dec_attend<float><<<g, 128, 0, s>>>((const float *)P.Q, (const float *)P.K, (const float *)P.V, P.sel,
+                                              (float *)P.O, t, c.S, c.Bs, c.L, c.R, c.H, c.d, scale);
+    count_launches(1);
+    return dec_status(cudaGetLastError());
+}
+
+int mono_decode_step(const mono_plan_t *plan, int t, const void *x_t, const void *Wq, const void *Wk, const void *Wv,
+                     const void *Wo, const float *codebooks, const int32_t *forced_t, void *delta_t, void *cache,
+                     void *stream) {
+    int st = dec_check(plan, cache);
+    if (st) return st;
+    const Plan &p = plan->p;
+    const mono_config &c = p.cfg;
+    if (t < 0 || t >= c.S) return MONO_ERR_INVALID;
+    if (dec_empty(p)) return MONO_OK;
+    if (!Wo || !delta_t) return MONO_ERR_NULL;
+    if ((st = mono_decode_project(plan, t, x_t, Wq, Wk, Wv, cache, stream))) return st;
+    if ((st = mono_decode_route(plan, t, codebooks, forced_t, cache, stream))) return st;
+    if ((st = mono_decode_attend(plan, t, cache, stream))) return st;
+    const DecPtrs P = dec_ptrs(dec_layout(p), cache);
+    cudaStream_t s = (cudaStream_t)stream;
+    const int grid = (c.W + 7) / 8;
+    if (c.dtype == MONO_BF16)
+        k_dec_out<__nv_bfloat16><<<grid, 256, 0, s>>>((const __nv_bfloat16 *)P.O, (const __nv_bfloat16 *)Wo,
+                                                      (__nv_bfloat16 *)delta_t, c.B, c.W, c.H * c.d);
+    else
+        k_dec_out<float><<<grid, 256, 0, s>>>((const float *)P.O, (const float *)Wo, (float *)delta_t, c.B, c.W,
+                                              c.H * c.d);
+    count_launches(1);
+    return dec_status(cudaGetLastError());
+}
+
+}  // extern "C"

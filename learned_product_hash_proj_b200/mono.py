@@ -27,11 +27,15 @@ STATUS = {0: "MONO_OK", 1: "MONO_ERR_INVALID", 2: "MONO_ERR_UNSUPPORTED", 3: "MO
           4: "MONO_ERR_WORKSPACE", 5: "MONO_ERR_CUDA", 6: "MONO_ERR_DEVICE", 7: "MONO_ERR_ALIGN", 8: "MONO_ERR_SCRATCH"}
 REGIONS = {"kbar": 0, "addr": 1, "post_ids": 2, "post_addr": 3, "post_rank": 4, "overflow": 5, "Q": 6, "K": 7,
            "V": 8, "sel": 9, "O": 10}
+DEC_REGIONS = {"K": 0, "V": 1, "kbar": 2, "addr": 3, "count": 4, "head": 5, "tail": 6, "next": 7, "overflow": 8,
+               "q": 9, "sel": 10, "o": 11}
 
 EXPORTS = ("mono_plan", "mono_plan_destroy", "mono_workspace_region", "mono_project", "mono_route",
            "mono_route_summaries", "mono_route_lists", "mono_route_queries", "mono_attend",
            "mono_out_project", "mono_forward", "mono_stats", "mono_strerror", "mono_version", "mono_kernel_launches",
-           "mono_route_static", "mono_route_static_capacity")
+           "mono_route_static", "mono_route_static_capacity", "mono_decode_cache_bytes",
+           "mono_decode_cache_region", "mono_decode_prefill", "mono_decode_project", "mono_decode_route",
+           "mono_decode_attend", "mono_decode_step")
 
 
 class MonoError(RuntimeError):
@@ -78,11 +82,21 @@ _lib.mono_route_static.argtypes = [_P] * 7
 _lib.mono_route_static.restype = ctypes.c_int
 _lib.mono_route_static_capacity.argtypes = []
 _lib.mono_route_static_capacity.restype = ctypes.c_size_t
+_lib.mono_decode_cache_bytes.argtypes = [_P, ctypes.POINTER(ctypes.c_size_t)]
+_lib.mono_decode_cache_region.argtypes = [_P, ctypes.c_int, ctypes.POINTER(ctypes.c_size_t),
+                                          ctypes.POINTER(ctypes.c_size_t)]
+_lib.mono_decode_prefill.argtypes = [_P, ctypes.c_int, _P, _P, _P]
+_lib.mono_decode_project.argtypes = [_P, ctypes.c_int] + [_P] * 6
+_lib.mono_decode_route.argtypes = [_P, ctypes.c_int] + [_P] * 4
+_lib.mono_decode_attend.argtypes = [_P, ctypes.c_int, _P, _P]
+_lib.mono_decode_step.argtypes = [_P, ctypes.c_int] + [_P] * 10
 _lib.mono_kernel_launches.argtypes = []
 _lib.mono_kernel_launches.restype = ctypes.c_ulonglong
 for _f in ("mono_plan", "mono_workspace_region", "mono_project", "mono_route", "mono_route_summaries",
            "mono_route_lists", "mono_route_queries", "mono_attend", "mono_out_project",
-           "mono_forward", "mono_stats", "mono_version"):
+           "mono_forward", "mono_stats", "mono_version", "mono_decode_cache_bytes", "mono_decode_cache_region",
+           "mono_decode_prefill", "mono_decode_project", "mono_decode_route", "mono_decode_attend",
+           "mono_decode_step"):
     getattr(_lib, _f).restype = ctypes.c_int
 
 
@@ -264,6 +278,74 @@ def stats(plan: Plan, ws, stream=None, check: bool = True) -> dict:
     d = st.as_dict()
     d["status"] = rc
     return d
+
+
+# ---------------------------------------------------------------------------
+# decode: one new token per sequence against a caller-owned cache
+# ---------------------------------------------------------------------------
+def decode_cache(plan: Plan, device="cuda") -> torch.Tensor:
+    """A caller-owned decode cache (uint8) of the size mono_decode_cache_bytes gives."""
+    n = ctypes.c_size_t()
+    _check(_lib.mono_decode_cache_bytes(plan.handle, ctypes.byref(n)), "mono_decode_cache_bytes")
+    return torch.zeros(max(int(n.value), 256), dtype=torch.uint8, device=device)
+
+
+def decode_region(plan: Plan, cache: torch.Tensor, name: str) -> torch.Tensor:
+    """A typed view of a decode-cache region (see mono_dec_region)."""
+    off, nbytes = ctypes.c_size_t(), ctypes.c_size_t()
+    _check(_lib.mono_decode_cache_region(plan.handle, DEC_REGIONS[name], ctypes.byref(off), ctypes.byref(nbytes)),
+           "mono_decode_cache_region")
+    c = plan.cfg
+    nb, A = c.S // c.Bs, c.C ** c.M
+    shapes = {"K": ((c.B, c.H, c.S, c.d), plan.dtype), "V": ((c.B, c.H, c.S, c.d), plan.dtype),
+              "kbar": ((c.B, c.H, nb, c.d), torch.float32), "addr": ((c.B, c.H, nb), torch.int32),
+              "count": ((c.B, c.H, A), torch.int32), "head": ((c.B, c.H, A), torch.int32),
+              "tail": ((c.B, c.H, A), torch.int32), "next": ((c.B, c.H, nb), torch.int32),
+              "overflow": ((c.B, c.H), torch.int32), "q": ((c.B, c.H, c.d), plan.dtype),
+              "sel": ((c.B, c.H, max(c.R, 1)), torch.int32), "o": ((c.B, c.H * c.d), plan.dtype)}
+    shape, dt = shapes[name]
+    raw = cache[off.value:off.value + nbytes.value]
+    return raw.view(dt).view(shape)
+
+
+def decode_prefill(plan: Plan, t0: int, codebooks, cache, stream=None):
+    c = plan.cfg
+    _check(_lib.mono_decode_prefill(plan.handle, int(t0),
+                                    _ptr(codebooks, "codebooks", (c.H, c.M, c.C, c.d // c.M), torch.float32),
+                                    _ptr(cache, "cache"), _stream(stream)), "mono_decode_prefill")
+
+
+def decode_project(plan: Plan, t: int, x_t, Wq, Wk, Wv, cache, stream=None):
+    c, dt = plan.cfg, plan.dtype
+    hd = c.H * c.d
+    _check(_lib.mono_decode_project(plan.handle, int(t), _ptr(x_t, "x_t", (c.B, c.W), dt),
+                                    _ptr(Wq, "Wq", (hd, c.W), dt), _ptr(Wk, "Wk", (hd, c.W), dt),
+                                    _ptr(Wv, "Wv", (hd, c.W), dt), _ptr(cache, "cache"), _stream(stream)),
+           "mono_decode_project")
+
+
+def decode_route(plan: Plan, t: int, codebooks, cache, forced_t=None, stream=None):
+    c = plan.cfg
+    _check(_lib.mono_decode_route(plan.handle, int(t),
+                                  _ptr(codebooks, "codebooks", (c.H, c.M, c.C, c.d // c.M), torch.float32),
+                                  _ptr(forced_t, "forced_t", (c.B, c.H), torch.int32, optional=True),
+                                  _ptr(cache, "cache"), _stream(stream)), "mono_decode_route")
+
+
+def decode_attend(plan: Plan, t: int, cache, stream=None):
+    _check(_lib.mono_decode_attend(plan.handle, int(t), _ptr(cache, "cache"), _stream(stream)), "mono_decode_attend")
+
+
+def decode_step(plan: Plan, t: int, x_t, Wq, Wk, Wv, Wo, codebooks, delta_t, cache, forced_t=None, stream=None):
+    c, dt = plan.cfg, plan.dtype
+    hd = c.H * c.d
+    _check(_lib.mono_decode_step(plan.handle, int(t), _ptr(x_t, "x_t", (c.B, c.W), dt),
+                                 _ptr(Wq, "Wq", (hd, c.W), dt), _ptr(Wk, "Wk", (hd, c.W), dt),
+                                 _ptr(Wv, "Wv", (hd, c.W), dt), _ptr(Wo, "Wo", (c.W, hd), dt),
+                                 _ptr(codebooks, "codebooks", (c.H, c.M, c.C, c.d // c.M), torch.float32),
+                                 _ptr(forced_t, "forced_t", (c.B, c.H), torch.int32, optional=True),
+                                 _ptr(delta_t, "delta_t", (c.B, c.W), dt), _ptr(cache, "cache"), _stream(stream)),
+           "mono_decode_step")
 
 
 def version() -> int:

@@ -112,3 +112,33 @@ def test_empty_inputs_launch_nothing(mono):
 def test_status_strings(mono):
     for code in mono.STATUS:
         assert mono.lib().mono_strerror(code)
+
+
+def test_decode_cache_layout_and_argument_checks(mono):
+    lib = mono.lib()
+    cfg = synth.config("pr1")
+    p = mono.Plan(cfg)
+    n = ctypes.c_size_t()
+    assert lib.mono_decode_cache_bytes(p.handle, ctypes.byref(n)) == 0 and n.value > 0
+    spans = []
+    for r in range(len(mono.DEC_REGIONS)):
+        off, nb = ctypes.c_size_t(), ctypes.c_size_t()
+        assert lib.mono_decode_cache_region(p.handle, r, ctypes.byref(off), ctypes.byref(nb)) == 0
+        assert off.value % 256 == 0 and off.value + nb.value <= n.value
+        spans.append((off.value, off.value + nb.value))
+    spans.sort()
+    assert all(a[1] <= b[0] for a, b in zip(spans, spans[1:]))
+    off, nb = ctypes.c_size_t(), ctypes.c_size_t()
+    assert lib.mono_decode_cache_region(p.handle, len(mono.DEC_REGIONS), ctypes.byref(off), ctypes.byref(nb)) == 1
+    fake = ctypes.c_void_p(1 << 20)            # never dereferenced: validation fails first
+    odd = ctypes.c_void_p((1 << 20) + 16)      # not 256-byte aligned
+    N = None
+    assert lib.mono_decode_step(None, 0, fake, fake, fake, fake, fake, fake, N, fake, fake, N) == 3  # NULL plan
+    assert lib.mono_decode_step(p.handle, 0, fake, fake, fake, fake, fake, fake, N, fake, N, N) == 4  # no cache
+    assert lib.mono_decode_route(p.handle, 0, fake, N, odd, N) == 7                                  # cache %256
+    assert lib.mono_decode_attend(p.handle, cfg.S, fake, N) == 1                                     # t >= S
+    assert lib.mono_decode_project(p.handle, -1, fake, fake, fake, fake, fake, N) == 1               # t < 0
+    assert lib.mono_decode_prefill(p.handle, cfg.S + 1, fake, fake, N) == 1                          # t0 > S
+    # the decode path scores every address of a query: C^M <= 4096
+    big = mono.Plan(synth.config("stress"))
+    assert lib.mono_decode_cache_bytes(big.handle, ctypes.byref(n)) == 2
