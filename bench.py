@@ -2,7 +2,7 @@
 """Benchmark of the Monodratic mixer on B200: route+attend tokens/s at S=32768.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload scale32k] [--no-sweep] [--no-cpu-baseline]
+                    [--workload scale32k] [--no-sweep] [--no-cpu-baseline] [--no-decode]
 
 A step is one pass of the whole hot path over one batch: projection + RoPE,
 block summaries + addresses, posting lists, probe/rerank, selected-set
@@ -260,6 +260,8 @@ def run_ours(args):
     torch.cuda.synchronize()
     e2e_ms = dist.reduce_max([mean([a.elapsed_time(b) for a, b in e2e_ev])], device=dev)[0]
 
+    decode = measure_decode(plan, cfg, K, V, inp, tdt, dev, stream, hbm) if not args.no_decode else None
+
     sweep = None
     if not args.no_sweep and world == 1 and args.workload == "scale32k":
         sweep = s_sweep(args, dev)
@@ -296,12 +298,79 @@ def run_ours(args):
                         "queries_lt_R": st["queries_lt_R"]},
             "timed_region_wall_s": wall,
         }
+        if decode:
+            out["decode"] = decode
         if sweep:
             out["s_sweep"] = sweep
         if cpu:
             out["cpu_baseline"] = cpu
         print(json.dumps(out), flush=True)
     dist.finalize()
+
+
+def measure_decode(plan, cfg, K, V, inp, tdt, dev, stream, hbm, n_steps=128):
+    """Decode latency at the end of the context: the cache holds the step's K and V,
+    prefilled to S - n_steps; n_steps timed decode steps (B sequences each) follow.
+    One warm-up pass over the same positions, then the lists are rebuilt.  Timed
+    twice: each step through the API from Python (eager), and the same n_steps
+    captured once into a CUDA graph and replayed (device time without the host's
+    per-call overhead)."""
+    import torch
+
+    from learned_product_hash_proj_b200 import mono
+    S, B = cfg.S, cfg.B
+    t0 = S - n_steps
+    cache = mono.decode_cache(plan, device=dev)
+    mono.decode_region(plan, cache, "K").copy_(K)
+    mono.decode_region(plan, cache, "V").copy_(V)
+    to = lambda a: torch.from_numpy(a).to(tdt).to(dev).contiguous()
+    Wq, Wk, Wv, Wo = (to(inp[k]) for k in ("Wq", "Wk", "Wv", "Wo"))
+    cb = torch.from_numpy(inp["codebooks"]).to(dev).contiguous()
+    xs = [to(inp["x"][:, t, :]) for t in range(t0, S)]
+    delta_t = torch.empty((B, cfg.W), dtype=tdt, device=dev)
+
+    def run():
+        mono.decode_prefill(plan, t0, cb, cache, stream)
+        for i, t in enumerate(range(t0, S)):
+            mono.decode_step(plan, t, xs[i], Wq, Wk, Wv, Wo, cb, delta_t, cache, stream=stream)
+
+    run()
+    torch.cuda.synchronize()
+    mono.decode_prefill(plan, t0, cb, cache, stream)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    ev[0].record(stream)
+    for i, t in enumerate(range(t0, S)):
+        mono.decode_step(plan, t, xs[i], Wq, Wk, Wv, Wo, cb, delta_t, cache, stream=stream)
+    ev[1].record(stream)
+    torch.cuda.synchronize()
+    ms_eager = ev[0].elapsed_time(ev[1]) / n_steps
+    # the same steps as one CUDA graph (captured on torch's capture stream)
+    g = torch.cuda.CUDAGraph()
+    mono.decode_prefill(plan, t0, cb, cache, stream)
+    torch.cuda.synchronize()
+    with torch.cuda.graph(g):
+        for i, t in enumerate(range(t0, S)):
+            mono.decode_step(plan, t, xs[i], Wq, Wk, Wv, Wo, cb, delta_t, cache)
+    mono.decode_prefill(plan, t0, cb, cache, stream)
+    torch.cuda.synchronize()
+    ev[0].record(stream)
+    g.replay()
+    ev[1].record(stream)
+    torch.cuda.synchronize()
+    ms = ev[0].elapsed_time(ev[1]) / n_steps
+    del g
+    es = 2 if cfg.dtype == "bf16" else 4
+    # bytes a step must read: the four weight matrices, and per (b, h) the K and V
+    # rows of its R remote and L local blocks plus E kbar rows
+    per_step = 4 * cfg.H * cfg.d * cfg.W * es + B * cfg.H * (
+        (cfg.R + cfg.L) * cfg.Bs * cfg.d * es * 2 + cfg.E * cfg.d * 4)
+    gbs = per_step / (ms / 1e3) / 1e9
+    return {"tokens_per_s": B / (ms / 1e3), "ms_per_token": ms, "ms_per_token_eager": ms_eager, "batch": B,
+            "context": t0, "steps": n_steps,
+            "api": "mono_decode_step (5 kernels per step, 6 when a block completes); ms_per_token from a CUDA "
+                   "graph of the steps, ms_per_token_eager from one Python call per step",
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
+                         "algorithmic_bytes": per_step}}
 
 
 def load_traffic(stage: str, cfg):
@@ -443,6 +512,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="scale32k")
+    ap.add_argument("--no-decode", action="store_true", help="skip the decode latency measurement")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -24,8 +24,11 @@
 
 #include <math.h>
 
+#include <initializer_list>
+
 #include "internal.cuh"
 #include "mono.h"
+#include "tc.cuh"
 
 namespace mono {
 namespace {
@@ -90,6 +93,21 @@ DecPtrs dec_ptrs(const DecLayout &L, void *cache) {
     return P;
 }
 
+// dot product of two rows of n elements, lanes taking 16-byte chunks (n * sizeof(T)
+// a multiple of 16 and both rows 16-byte aligned); fp32 accumulation, warp-reduced
+template <typename T>
+__device__ __forceinline__ float row_dot_part(const T *a, const T *b, int n, int lane) {
+    constexpr int V = 16 / sizeof(T);
+    float acc = 0.f;
+    for (int k = lane * V; k < n; k += 32 * V) {
+        const uint4 ua = *(const uint4 *)(a + k), ub = *(const uint4 *)(b + k);
+        const T *ta = (const T *)&ua, *tb = (const T *)&ub;
+#pragma unroll
+        for (int e = 0; e < V; ++e) acc = fmaf(to_f(ta[e]), to_f(tb[e]), acc);
+    }
+    return acc;
+}
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
@@ -125,14 +143,8 @@ __global__ void __launch_bounds__(256) k_dec_project(const T *__restrict__ x, co
     }
     for (int b = 0; b < B; ++b) {
         const T *xb = x + (size_t)b * W;
-        float a0 = 0.f, a1 = 0.f;
-        for (int k = lane; k < W; k += 32) {
-            const float xv = to_f(xb[k]);
-            a0 = fmaf(xv, to_f(w0[k]), a0);
-            a1 = fmaf(xv, to_f(w1[k]), a1);
-        }
-        a0 = warp_sum(a0);
-        a1 = warp_sum(a1);
+        const float a0 = warp_sum(row_dot_part(xb, w0, W, lane));
+        const float a1 = warp_sum(row_dot_part(xb, w1, W, lane));
         if (lane == 0) {
             float r0 = a0, r1 = a1;
             if (which < 2) {
@@ -157,6 +169,7 @@ __device__ int dec_summary(const T *Kc, const float *cb, float *kbar, int32_t *a
     const T *rows = Kc + (bh * S + (size_t)j * Bs) * d;
     for (int i = lane; i < d; i += 32) {
         float acc = 0.0f;
+#pragma unroll 8
         for (int tt = 0; tt < Bs; ++tt) acc = __fadd_rn(acc, to_f(rows[(size_t)tt * d + i]));
         const float v = __fdiv_rn(acc, (float)Bs);
         s_kb[i] = v;
@@ -257,28 +270,36 @@ __device__ __forceinline__ bool before(float v1, int a1, float v2, int a2) {
 }
 
 // ---------------------------------------------------------------------------
-// routing of the step's query, one warp per (b, h); grid (H, B), 32 threads
+// routing of the step's query, one warp per (b, h); grid (H, B), 32 threads,
+// dynamic shared memory C * d floats (the head's codebooks)
 // ---------------------------------------------------------------------------
 template <typename T>
 __global__ void __launch_bounds__(32) k_dec_route(const T *__restrict__ q, const float *__restrict__ cb,
                                                   const int32_t *__restrict__ forced, DecPtrs P, int t, int Bs, int L,
                                                   int R, int E, int M, int C, int TP, int cap, int H, int d, int nb,
                                                   long long A) {
+    extern __shared__ __align__(16) float s_cb[];  // [M][C][dm] of head h
     __shared__ float s_q[kMaxD];
     __shared__ float s_sc[kMaxM * kMaxC];
     __shared__ int s_top[kMaxT];
+    __shared__ int s_head[kMaxT], s_cnt[kMaxT];
     __shared__ int s_cand[kMaxE];
     __shared__ float s_score[kMaxE];
+    __shared__ __align__(16) float s_kb[kMaxE > 8 ? 8 : kMaxE][kMaxD];  // candidate kbar rows, 8 at a time
     const int lane = threadIdx.x;
     const int h = blockIdx.x, b = blockIdx.y;
     const size_t bh = (size_t)b * H + h;
     for (int i = lane; i < d; i += 32) s_q[i] = to_f(q[bh * d + i]);
+    {
+        const float4 *src = (const float4 *)(cb + (size_t)h * C * d);
+        for (int i = lane; i < C * d / 4; i += 32) ((float4 *)s_cb)[i] = __ldg(src + i);
+    }
     __syncwarp();
     // subspace scores: fma chains in ascending element order from +0
     const int dm = d / M;
     for (int mc = lane; mc < M * C; mc += 32) {
         const int m = mc / C;
-        const float *w = cb + ((size_t)h * M * C + mc) * dm;
+        const float *w = s_cb + mc * dm;
         float a = 0.0f;
         for (int i = 0; i < dm; ++i) a = __fmaf_rn(s_q[m * dm + i], w[i], a);
         s_sc[mc] = a;
@@ -289,16 +310,16 @@ __global__ void __launch_bounds__(32) k_dec_route(const T *__restrict__ q, const
     float lv[kMaxT];
     int la[kMaxT];
     for (int k = 0; k < TP; ++k) { lv[k] = -INFINITY; la[k] = 0x7fffffff; }
-    for (long long ad = lane; ad < A; ad += 32) {
-        long long rest = ad, radix = A / C;
+    const int A32 = (int)A;  // <= 4096 on this path
+    for (int a32 = lane; a32 < A32; a32 += 32) {
+        int rest = a32, radix = A32 / C;
         float v = 0.0f;
         for (int m = 0; m < M; ++m) {
-            const int cm = (int)(rest / radix);
-            rest -= (long long)cm * radix;
+            const int cm = rest / radix;
+            rest -= cm * radix;
             radix /= C;
             v = m == 0 ? s_sc[cm] : __fadd_rn(v, s_sc[m * C + cm]);
         }
-        const int a32 = (int)ad;
         if (!before(v, a32, lv[TP - 1], la[TP - 1])) continue;
         int k = TP - 1;
         while (k > 0 && before(v, a32, lv[k - 1], la[k - 1])) {
@@ -326,16 +347,23 @@ __global__ void __launch_bounds__(32) k_dec_route(const T *__restrict__ q, const
         if (lane == bl) ++ptr;
     }
     __syncwarp();
+    // the probed lists' heads and counts, fetched at once
+    if (lane < TP) {
+        const int a = s_top[lane];
+        const bool ok = a >= 0 && (long long)a < A;
+        s_cnt[lane] = ok ? P.count[bh * A + a] : 0;
+        s_head[lane] = ok ? P.head[bh * A + a] : -1;
+    }
+    __syncwarp();
     // union of the probed lists in probe order, causal filter, E cap
     const int lim = t / Bs - L;
     int nc = 0;
     if (lane == 0) {
         for (int r = 0; r < TP && nc < E; ++r) {
-            const int a = s_top[r];
-            if (a < 0 || (long long)a >= A || P.count[bh * A + a] <= 0) continue;
+            if (s_cnt[r] <= 0) continue;
             // at most cap kept entries; an id outside [0, nb) ends the walk
             int steps = 0;
-            for (int j = P.head[bh * A + a]; (unsigned)j < (unsigned)nb && nc < E && steps < cap;
+            for (int j = s_head[r]; (unsigned)j < (unsigned)nb && nc < E && steps < cap;
                  j = P.next[bh * nb + j], ++steps) {
                 if (j > lim) break;  // ascending ids: the rest are later still
                 s_cand[nc++] = j;
@@ -344,14 +372,21 @@ __global__ void __launch_bounds__(32) k_dec_route(const T *__restrict__ q, const
     }
     nc = __shfl_sync(0xffffffffu, nc, 0);
     __syncwarp();
-    // rerank: q . kbar_j, one candidate per lane
-    if (lane < nc) {
-        const float *kb = P.kbar + (bh * nb + s_cand[lane]) * d;
-        float a = 0.0f;
-        for (int i = 0; i < d; ++i) a = __fmaf_rn(s_q[i], kb[i], a);
-        s_score[lane] = a;
+    // rerank: q . kbar_j, one candidate per lane, from rows staged 8 at a time
+    for (int e0 = 0; e0 < nc; e0 += 8) {
+        const int ne = min(8, nc - e0);
+        for (int i = lane; i < ne * d / 4; i += 32) {
+            const int e = i / (d / 4), c4 = i % (d / 4);
+            ((float4 *)s_kb[e])[c4] = __ldg((const float4 *)(P.kbar + (bh * nb + s_cand[e0 + e]) * d) + c4);
+        }
+        __syncwarp();
+        if (lane < ne) {
+            float a = 0.0f;
+            for (int i = 0; i < d; ++i) a = __fmaf_rn(s_q[i], s_kb[lane][i], a);
+            s_score[e0 + lane] = a;
+        }
+        __syncwarp();
     }
-    __syncwarp();
     if (lane == 0) {
         // top R by (score desc, id asc), in rank order
         int ra[kMaxR];
@@ -384,47 +419,88 @@ __global__ void __launch_bounds__(32) k_dec_route(const T *__restrict__ q, const
 }
 
 // ---------------------------------------------------------------------------
-// attention of the step's query: 4 warps split the keys, each with an online
-// softmax (lanes own d/32 dimensions), merged at the end; fp32 throughout.
-// grid (H, B), 128 threads
+// attention of the step's query: the key list (R remote blocks, then the local
+// tokens) is walked in chunks of CH keys whose K and V rows are copied to
+// shared memory (cp.async, two buffers: chunk c+1 in flight while chunk c is
+// used; at the usual sizes one chunk holds every key, so all rows are in
+// flight at once).  8 warps split a chunk's keys, each with an online softmax
+// (lanes own d/32 dimensions); the warps merge at the end.  fp32 throughout.
+// grid (H, B), 256 threads, dynamic shared memory 2 * CH * d * sizeof(T) * 2.
 // ---------------------------------------------------------------------------
 template <typename T>
-__global__ void __launch_bounds__(128) k_dec_attend(const T *__restrict__ q, const T *__restrict__ Kc,
+constexpr int dec_chunk(int d) {
+    return (48 * 1024) / (d * (int)sizeof(T));  // keys per buffer: 96 KB of K and V rows
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256) k_dec_attend(const T *__restrict__ q, const T *__restrict__ Kc,
                                                     const T *__restrict__ Vc, const int32_t *__restrict__ sel,
                                                     T *__restrict__ O, int t, int S, int Bs, int L, int R, int H, int d,
                                                     float scale) {
-    constexpr int kPer = kMaxD / 32;
-    __shared__ float s_m[4], s_l[4];
-    __shared__ float s_acc[4][kMaxD];
+    constexpr int kPer = kMaxD / 32, NW = 8;
+    extern __shared__ __align__(16) uint8_t dsm[];
+    __shared__ float s_m[NW], s_l[NW];
+    __shared__ float s_acc[NW][kMaxD];
+    __shared__ int s_js[kMaxR];
+    __shared__ int s_nr;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int h = blockIdx.x, b = blockIdx.y;
     const size_t bh = (size_t)b * H + h;
     const int per = d / 32;
-    float qv[kPer];
-    for (int e = 0; e < per; ++e) qv[e] = to_f(q[bh * d + lane * per + e]);
+    const int CH = dec_chunk<T>(d);
+    const int rowb = d * (int)sizeof(T);      // bytes of one K or V row
+    T *bufK[2] = {(T *)dsm, (T *)(dsm + 2 * CH * rowb)};
+    T *bufV[2] = {(T *)(dsm + CH * rowb), (T *)(dsm + 3 * CH * rowb)};
     const int bq = t / Bs, lim = bq - L;
-    int js[kMaxR];  // the selected remote blocks; ids outside [0, t/Bs - L] are skipped
-    int nr = 0;
-    for (int r = 0; r < R; ++r) {
-        const int j = sel[bh * R + r];
-        if (j >= 0 && j <= lim) js[nr++] = j;
+    if (threadIdx.x == 0) {  // the selected remote blocks; ids outside [0, t/Bs - L] are skipped
+        int nr = 0;
+        for (int r = 0; r < R; ++r) {
+            const int j = sel[bh * R + r];
+            if (j >= 0 && j <= lim) s_js[nr++] = j;
+        }
+        s_nr = nr;
     }
+    __syncthreads();
+    const int nr = s_nr;
     const int lo = max(0, bq - L + 1) * Bs;
     const int nkeys = nr * Bs + (t - lo + 1);
+    auto key_of = [&](int idx) { return idx < nr * Bs ? s_js[idx / Bs] * Bs + idx % Bs : lo + (idx - nr * Bs); };
+    auto stage = [&](int buf, int c0) {  // rows of keys [c0, c0 + CH) into buffer buf
+        const int n = min(CH, nkeys - c0), chunks = rowb / 16;
+        for (int i = threadIdx.x; i < n * chunks; i += blockDim.x) {
+            const int k = i / chunks, c = i % chunks;
+            const size_t row = bh * S + key_of(c0 + k);
+            tc::cp_async16((uint8_t *)bufK[buf] + k * rowb + 16 * c, (const uint8_t *)(Kc + row * d) + 16 * c, true);
+            tc::cp_async16((uint8_t *)bufV[buf] + k * rowb + 16 * c, (const uint8_t *)(Vc + row * d) + 16 * c, true);
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+    float qv[kPer];
+    for (int e = 0; e < per; ++e) qv[e] = to_f(q[bh * d + lane * per + e]);
     float m = -INFINITY, l = 0.f, acc[kPer];
     for (int e = 0; e < per; ++e) acc[e] = 0.f;
-    for (int idx = warp; idx < nkeys; idx += 4) {
-        const int key = idx < nr * Bs ? js[idx / Bs] * Bs + idx % Bs : lo + (idx - nr * Bs);
-        const T *kr = Kc + (bh * S + key) * d + lane * per;
-        float part = 0.f;
-        for (int e = 0; e < per; ++e) part = fmaf(qv[e], to_f(kr[e]), part);
-        const float s = warp_sum(part) * scale;
-        const float mn = fmaxf(m, s);
-        const float corr = expf(m - mn), p = expf(s - mn);
-        l = l * corr + p;
-        const T *vr = Vc + (bh * S + key) * d + lane * per;
-        for (int e = 0; e < per; ++e) acc[e] = fmaf(p, to_f(vr[e]), acc[e] * corr);
-        m = mn;
+    stage(0, 0);
+    for (int c0 = 0, cb = 0; c0 < nkeys; c0 += CH, cb ^= 1) {
+        if (c0 + CH < nkeys) {
+            stage(cb ^ 1, c0 + CH);
+            asm volatile("cp.async.wait_group 1;" ::: "memory");
+        } else {
+            asm volatile("cp.async.wait_group 0;" ::: "memory");
+        }
+        __syncthreads();
+        const int n = min(CH, nkeys - c0);
+        for (int k = warp; k < n; k += NW) {
+            const T *kr = bufK[cb] + k * d + lane * per, *vr = bufV[cb] + k * d + lane * per;
+            float part = 0.f;
+            for (int e = 0; e < per; ++e) part = fmaf(qv[e], to_f(kr[e]), part);
+            const float s = warp_sum(part) * scale;
+            const float mn = fmaxf(m, s);
+            const float corr = expf(m - mn), p = expf(s - mn);
+            l = l * corr + p;
+            for (int e = 0; e < per; ++e) acc[e] = fmaf(p, to_f(vr[e]), acc[e] * corr);
+            m = mn;
+        }
+        __syncthreads();  // buffer cb is refilled two chunks later
     }
     if (lane == 0) {
         s_m[warp] = m;
@@ -434,10 +510,10 @@ __global__ void __launch_bounds__(128) k_dec_attend(const T *__restrict__ q, con
     __syncthreads();
     if (warp == 0) {
         float mm = -INFINITY;
-        for (int w = 0; w < 4; ++w) mm = fmaxf(mm, s_m[w]);
+        for (int w = 0; w < NW; ++w) mm = fmaxf(mm, s_m[w]);
         float den = 0.f, o[kPer];
         for (int e = 0; e < per; ++e) o[e] = 0.f;
-        for (int w = 0; w < 4; ++w) {
+        for (int w = 0; w < NW; ++w) {
             if (s_m[w] == -INFINITY) continue;  // a warp without keys
             const float f = expf(s_m[w] - mm);
             den += s_l[w] * f;
@@ -457,9 +533,7 @@ __global__ void __launch_bounds__(256) k_dec_out(const T *__restrict__ o, const 
     const T *wr = Wo + (size_t)w * N;
     for (int b = 0; b < B; ++b) {
         const T *ob = o + (size_t)b * N;
-        float a = 0.f;
-        for (int k = lane; k < N; k += 32) a = fmaf(to_f(ob[k]), to_f(wr[k]), a);
-        a = warp_sum(a);
+        const float a = warp_sum(row_dot_part(ob, wr, N, lane));
         if (lane == 0) delta[(size_t)b * W + w] = from_f<T>(a);
     }
 }
@@ -475,6 +549,15 @@ int dec_check(const mono_plan_t *plan, const void *cache) {
 int dec_status(cudaError_t e) { return e == cudaSuccess ? MONO_OK : MONO_ERR_CUDA; }
 
 bool dec_empty(const Plan &p) { return p.cfg.B == 0 || p.cfg.S == 0; }
+
+// the row vectors are read in 16-byte chunks
+int dec_ptrs16(std::initializer_list<const void *> ptrs) {
+    for (const void *q : ptrs) {
+        if (!q) return MONO_ERR_NULL;
+        if ((uintptr_t)q & 15) return MONO_ERR_ALIGN;
+    }
+    return MONO_OK;
+}
 
 }  // namespace
 }  // namespace mono
@@ -534,7 +617,7 @@ int mono_decode_project(const mono_plan_t *plan, int t, const void *x_t, const v
     const mono_config &c = p.cfg;
     if (t < 0 || t >= c.S) return MONO_ERR_INVALID;
     if (dec_empty(p)) return MONO_OK;
-    if (!x_t || !Wq || !Wk || !Wv) return MONO_ERR_NULL;
+    if ((st = dec_ptrs16({x_t, Wq, Wk, Wv}))) return st;
     const DecPtrs P = dec_ptrs(dec_layout(p), cache);
     const int warps = 3 * c.H * c.d / 2;
     const int grid = (warps + 7) / 8;
@@ -576,12 +659,22 @@ int mono_decode_route(const mono_plan_t *plan, int t, const float *codebooks, co
         count_launches(1);
     }
     if (c.R > 0) {
-        if (bf)
-            k_dec_route<__nv_bfloat16><<<g, 32, 0, s>>>((const __nv_bfloat16 *)P.Q, codebooks, forced_t, P, t, c.Bs,
-                                                        c.L, c.R, c.E, c.M, c.C, c.T, c.cap, c.H, c.d, p.nb, p.A);
-        else
-            k_dec_route<float><<<g, 32, 0, s>>>((const float *)P.Q, codebooks, forced_t, P, t, c.Bs, c.L, c.R, c.E,
-                                                c.M, c.C, c.T, c.cap, c.H, c.d, p.nb, p.A);
+        const size_t sm = (size_t)c.C * c.d * 4;
+        cudaError_t e;
+        if (bf) {
+            if (sm > 48 * 1024 && (e = cudaFuncSetAttribute(k_dec_route<__nv_bfloat16>,
+                                                            cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm)))
+                return dec_status(e);
+            k_dec_route<__nv_bfloat16><<<g, 32, sm, s>>>((const __nv_bfloat16 *)P.Q, codebooks, forced_t, P, t,
+                                                         c.Bs, c.L, c.R, c.E, c.M, c.C, c.T, c.cap, c.H, c.d, p.nb,
+                                                         p.A);
+        } else {
+            if (sm > 48 * 1024 &&
+                (e = cudaFuncSetAttribute(k_dec_route<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm)))
+                return dec_status(e);
+            k_dec_route<float><<<g, 32, sm, s>>>((const float *)P.Q, codebooks, forced_t, P, t, c.Bs, c.L, c.R, c.E,
+                                                 c.M, c.C, c.T, c.cap, c.H, c.d, p.nb, p.A);
+        }
         count_launches(1);
     }
     return dec_status(cudaGetLastError());
@@ -598,13 +691,22 @@ int mono_decode_attend(const mono_plan_t *plan, int t, void *cache, void *stream
     const float scale = (float)(1.0 / sqrt((double)c.d));
     const dim3 g(c.H, c.B);
     cudaStream_t s = (cudaStream_t)stream;
-    if (c.dtype == MONO_BF16)
-        k_dec_attend<__nv_bfloat16><<<g, 128, 0, s>>>((const __nv_bfloat16 *)P.Q, (const __nv_bfloat16 *)P.K,
-                                                      (const __nv_bfloat16 *)P.V, P.sel, (__nv_bfloat16 *)P.O, t, c.S,
-                                                      c.Bs, c.L, c.R, c.H, c.d, scale);
-    else
-        k_dec_attend<float><<<g, 128, 0, s>>>((const float *)P.Q, (const float *)P.K, (const float *)P.V, P.sel,
-                                              (float *)P.O, t, c.S, c.Bs, c.L, c.R, c.H, c.d, scale);
+    cudaError_t e;
+    if (c.dtype == MONO_BF16) {
+        const size_t sm = (size_t)4 * dec_chunk<__nv_bfloat16>(c.d) * c.d * 2;
+        if ((e = cudaFuncSetAttribute(k_dec_attend<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)sm)))
+            return dec_status(e);
+        k_dec_attend<__nv_bfloat16><<<g, 256, sm, s>>>((const __nv_bfloat16 *)P.Q, (const __nv_bfloat16 *)P.K,
+                                                       (const __nv_bfloat16 *)P.V, P.sel, (__nv_bfloat16 *)P.O, t, c.S,
+                                                       c.Bs, c.L, c.R, c.H, c.d, scale);
+    } else {
+        const size_t sm = (size_t)4 * dec_chunk<float>(c.d) * c.d * 4;
+        if ((e = cudaFuncSetAttribute(k_dec_attend<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm)))
+            return dec_status(e);
+        k_dec_attend<float><<<g, 256, sm, s>>>((const float *)P.Q, (const float *)P.K, (const float *)P.V, P.sel,
+                                               (float *)P.O, t, c.S, c.Bs, c.L, c.R, c.H, c.d, scale);
+    }
     count_launches(1);
     return dec_status(cudaGetLastError());
 }
@@ -618,7 +720,7 @@ int mono_decode_step(const mono_plan_t *plan, int t, const void *x_t, const void
     const mono_config &c = p.cfg;
     if (t < 0 || t >= c.S) return MONO_ERR_INVALID;
     if (dec_empty(p)) return MONO_OK;
-    if (!Wo || !delta_t) return MONO_ERR_NULL;
+    if ((st = dec_ptrs16({x_t, Wq, Wk, Wv, Wo, delta_t}))) return st;
     if ((st = mono_decode_project(plan, t, x_t, Wq, Wk, Wv, cache, stream))) return st;
     if ((st = mono_decode_route(plan, t, codebooks, forced_t, cache, stream))) return st;
     if ((st = mono_decode_attend(plan, t, cache, stream))) return st;
