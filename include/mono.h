@@ -285,6 +285,38 @@ int mono_decode_step(const mono_plan_t *plan, int t, const void *x_t, const void
                      const void *Wv, const void *Wo, const float *codebooks, const int32_t *forced_t,
                      void *delta_t, void *cache, void *stream);
 
+/* ------------------------------------------------------------------------
+ * Backward pass for a fixed selection.
+ *
+ * The routing (summaries, addresses, posting lists, probe, rerank) is
+ * piecewise constant in its inputs and has no gradient; the selection sel
+ * (e.g. from mono_route) is an input and the rest of the forward pass is
+ * differentiated: projection, RoPE, exact softmax over the selected token set
+ * of each query (the blocks of sel that lie in [0, t/Bs - L] plus the local
+ * tokens [max(0, t/Bs - L + 1) * Bs, t]), output projection.  Gradients are
+ * fp32 and accumulated in fp32; dK and dV of a block sum the queries that
+ * selected it in an unspecified order.  The backward workspace is a separate
+ * caller-allocated buffer of mono_backward_workspace_bytes bytes (256-byte
+ * aligned).
+ * ------------------------------------------------------------------------ */
+int mono_backward_workspace_bytes(const mono_plan_t *plan, size_t *bytes);
+
+/* Gradients of the selected-set attention O(Q, K, V; sel) given dO:
+ * Q, K, V [B,H,S,d] (dtype, post-RoPE, as mono_attend takes them), sel
+ * [B,H,S,R], dO [B,S,H*d] fp32 -> dQ, dK, dV [B,H,S,d] fp32 (with respect to
+ * the post-RoPE Q and K). */
+int mono_attend_backward(const mono_plan_t *plan, const void *Q, const void *K, const void *V, const int32_t *sel,
+                         const float *dO, float *dQ, float *dK, float *dV, void *bwd_workspace, void *stream);
+
+/* Gradients of the whole mixer for a fixed selection: inputs as mono_forward
+ * (x, Wq, Wk, Wv, Wo in dtype) plus sel [B,H,S,R] and ddelta [B,S,W] (dtype);
+ * outputs dx [B,S,W] and dWq, dWk, dWv [H*d,W], dWo [W,H*d], fp32.  The forward
+ * activations Q, K, V and O are recomputed into `workspace` (the forward
+ * workspace of the plan). */
+int mono_backward(const mono_plan_t *plan, const void *x, const void *Wq, const void *Wk, const void *Wv,
+                  const void *Wo, const int32_t *sel, const void *ddelta, float *dx, float *dWq, float *dWk,
+                  float *dWv, float *dWo, void *workspace, void *bwd_workspace, void *stream);
+
 /* Synchronise `stream` and read the routing statistics and the device error
  * word of the last mono_route / mono_forward on `workspace`.  Returns
  * MONO_ERR_DEVICE if a kernel recorded an error. */

@@ -1,0 +1,538 @@
+// backward.cu -- gradients of the mixer for a fixed selection.
+//
+// The routing (summaries, addresses, posting lists, probe, rerank) is
+// piecewise constant in its inputs and has no gradient, so the backward pass
+// takes the selection as an input and differentiates the rest of the forward
+// pass ("Monodratic Routes Sparse Attention with Learned Product Hashes", Key
+// Points; the aitechinspire.com article, Snapshot): projection without bias,
+// RoPE on q and k, exact softmax over the selected token set (the remote
+// blocks of sel plus the local tokens [max(0, t/Bs - L + 1) * Bs, t]), output
+// projection.  For one query t with probabilities P over its keys s:
+//     D_t = dO_t . O_t,   dS_ts = P_ts (dO_t . v_s - D_t),
+//     dQ_t = scale sum_s dS_ts k_s,   dK_s += scale dS_ts q_t,   dV_s += P_ts dO_t.
+// Kernels (fp32 arithmetic, gradients in fp32):
+//   k_bwd_dq     one warp per query-head: log-sum-exp and D from recomputed
+//                scores (the stored O is not needed), then dQ;
+//   k_bwd_count / k_bwd_scan / k_bwd_fill: per (b, h) and block j, the
+//                queries that selected j (lists in unspecified order);
+//   k_bwd_dkdv   one CTA per (b, h) and tile of up to 64 keys of one block:
+//                walks the block's local queries and its selecting queries,
+//                accumulating dK and dV of its keys in shared memory;
+//   k_bwd_rope   inverse rotation of dQ, dK and the token-major layout;
+//   k_gemm_any   the projection gradients (generic strided SIMT GEMM).
+#include <cuda_runtime.h>
+
+#include <math.h>
+
+#include <initializer_list>
+
+#include "internal.cuh"
+#include "mono.h"
+
+namespace mono {
+namespace {
+
+struct BwdLayout {
+    size_t lse, dsum, cnt, start, cursor, list, dO, dQ, dK, dV, dQp, dKp, dVp, total;
+};
+
+BwdLayout bwd_layout(const Plan &p) {
+    const mono_config &c = p.cfg;
+    const size_t B = c.B, H = c.H, S = c.S, d = c.d, nb = p.nb, R = c.R > 0 ? c.R : 1;
+    size_t o = 0;
+    auto take = [&](size_t bytes) {
+        const size_t at = o;
+        o += (bytes + 255) / 256 * 256;
+        return at;
+    };
+    BwdLayout L{};
+    L.lse = take(B * H * S * 4);
+    L.dsum = take(B * H * S * 4);
+    L.cnt = take(B * H * nb * 4);
+    L.start = take(B * H * nb * 4);
+    L.cursor = take(B * H * nb * 4);
+    L.list = take(B * H * S * R * 4);
+    L.dO = take(B * S * H * d * 4);
+    L.dQ = take(B * H * S * d * 4);
+    L.dK = take(B * H * S * d * 4);
+    L.dV = take(B * H * S * d * 4);
+    L.dQp = take(B * S * H * d * 4);
+    L.dKp = take(B * S * H * d * 4);
+    L.dVp = take(B * S * H * d * 4);
+    L.total = o;
+    return L;
+}
+
+__device__ __forceinline__ float bwd_warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+__device__ __forceinline__ bool bwd_sel_valid(int j, int t, int Bs, int L) { return j >= 0 && j <= t / Bs - L; }
+
+// ---------------------------------------------------------------------------
+// dQ, log-sum-exp and D of every query-head: one warp each, lanes own d/32
+// dimensions.  Pass 1 (online softmax over the selected keys) gives the
+// log-sum-exp and O in fp32, hence D = dO . O; pass 2 forms dS and dQ.
+// grid ceil(B H S / 8), 256 threads.
+// ---------------------------------------------------------------------------
+template <typename T>
+__global__ void __launch_bounds__(256) k_bwd_dq(const T *__restrict__ Q, const T *__restrict__ K,
+                                                const T *__restrict__ V, const int32_t *__restrict__ sel,
+                                                const float *__restrict__ dO, float *__restrict__ dQ,
+                                                float *__restrict__ lse_out, float *__restrict__ dsum_out, int B, int H,
+                                                int S, int d, int Bs, int L, int R, float scale) {
+    constexpr int kPer = kMaxD / 32;
+    const int lane = threadIdx.x & 31;
+    const long long w = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (w >= (long long)B * H * S) return;
+    const long long bh = w / S;
+    const int t = (int)(w % S);
+    const int b = (int)(bh / H), h = (int)(bh % H);
+    const int per = d / 32;
+    float q[kPer], g[kPer];
+    for (int e = 0; e < per; ++e) {
+        q[e] = to_f(Q[w * d + lane * per + e]);
+        g[e] = dO[(((size_t)b * S + t) * H + h) * d + lane * per + e];
+    }
+    int js[kMaxR];
+    int nr = 0;
+    for (int r = 0; r < R; ++r) {
+        const int j = sel[w * R + r];
+        if (bwd_sel_valid(j, t, Bs, L)) js[nr++] = j;
+    }
+    const int lo = max(0, t / Bs - L + 1) * Bs;
+    const int nkeys = nr * Bs + (t - lo + 1);
+    auto key_of = [&](int idx) { return idx < nr * Bs ? js[idx / Bs] * Bs + idx % Bs : lo + (idx - nr * Bs); };
+    const size_t base = (size_t)bh * S;
+    // pass 1: log-sum-exp and O
+    float m = -INFINITY, l = 0.f, o[kPer];
+    for (int e = 0; e < per; ++e) o[e] = 0.f;
+    for (int idx = 0; idx < nkeys; ++idx) {
+        const size_t row = (base + key_of(idx)) * d + lane * per;
+        float part = 0.f;
+        for (int e = 0; e < per; ++e) part = fmaf(q[e], to_f(K[row + e]), part);
+        const float s = bwd_warp_sum(part) * scale;
+        const float mn = fmaxf(m, s), corr = expf(m - mn), p = expf(s - mn);
+        l = l * corr + p;
+        for (int e = 0; e < per; ++e) o[e] = fmaf(p, to_f(V[row + e]), o[e] * corr);
+        m = mn;
+    }
+    const float lse = m + logf(l);
+    float dpart = 0.f;
+    for (int e = 0; e < per; ++e) dpart = fmaf(g[e], o[e] / l, dpart);
+    const float D = bwd_warp_sum(dpart);
+    // pass 2: dS and dQ
+    float dq[kPer];
+    for (int e = 0; e < per; ++e) dq[e] = 0.f;
+    for (int idx = 0; idx < nkeys; ++idx) {
+        const size_t row = (base + key_of(idx)) * d + lane * per;
+        float sp = 0.f, dp = 0.f;
+        for (int e = 0; e < per; ++e) {
+            sp = fmaf(q[e], to_f(K[row + e]), sp);
+            dp = fmaf(g[e], to_f(V[row + e]), dp);
+        }
+        const float s = bwd_warp_sum(sp) * scale;
+        const float p = expf(s - lse);
+        const float ds = p * (bwd_warp_sum(dp) - D);
+        for (int e = 0; e < per; ++e) dq[e] = fmaf(ds, to_f(K[row + e]), dq[e]);
+    }
+    for (int e = 0; e < per; ++e) dQ[w * d + lane * per + e] = dq[e] * scale;
+    if (lane == 0) {
+        lse_out[w] = lse;
+        dsum_out[w] = D;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// per (b, h) and block j, the queries that selected j: count, scan, fill
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) k_bwd_count(const int32_t *__restrict__ sel, int32_t *__restrict__ cnt,
+                                                   long long n, int S, int R, int nb, int Bs, int L) {
+    const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= n) return;
+    const long long w = i / R;
+    const int t = (int)(w % S);
+    const long long bh = w / S;
+    const int j = sel[i];
+    if (bwd_sel_valid(j, t, Bs, L)) atomicAdd(&cnt[bh * nb + j], 1);
+}
+
+// exclusive scan of the counts of one (b, h); grid B*H, 1024 threads
+__global__ void __launch_bounds__(1024) k_bwd_scan(const int32_t *__restrict__ cnt, int32_t *__restrict__ start,
+                                                   int32_t *__restrict__ cursor, int nb) {
+    __shared__ int s_part[32];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const size_t bh = blockIdx.x;
+    const int per = (nb + blockDim.x - 1) / blockDim.x;
+    const int j0 = tid * per;
+    int run = 0;
+    for (int j = j0; j < min(nb, j0 + per); ++j) run += cnt[bh * nb + j];
+    int x = run;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) s_part[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+        int v = lane < (int)(blockDim.x >> 5) ? s_part[lane] : 0;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, v, o);
+            if (lane >= o) v += y;
+        }
+        s_part[lane] = v;
+    }
+    __syncthreads();
+    int off = (warp ? s_part[warp - 1] : 0) + x - run;
+    for (int j = j0; j < min(nb, j0 + per); ++j) {
+        start[bh * nb + j] = off;
+        cursor[bh * nb + j] = off;
+        off += cnt[bh * nb + j];
+    }
+}
+
+__global__ void __launch_bounds__(256) k_bwd_fill(const int32_t *__restrict__ sel, int32_t *__restrict__ cursor,
+                                                  int32_t *__restrict__ list, long long n, int S, int R, int nb,
+                                                  int Bs, int L) {
+    const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= n) return;
+    const long long w = i / R;
+    const int t = (int)(w % S);
+    const long long bh = w / S;
+    const int j = sel[i];
+    if (!bwd_sel_valid(j, t, Bs, L)) return;
+    const int pos = atomicAdd(&cursor[bh * nb + j], 1);
+    list[bh * S * R + pos] = t;
+}
+
+// ---------------------------------------------------------------------------
+// dK and dV of a tile of up to 64 keys of block j of one (b, h): one thread
+// per key, the tile's K and V rows and the dK / dV accumulators in padded
+// shared memory (row stride d+1: conflict-free).  Queries come in groups of 8
+// (their q, dO, log-sum-exp and D staged in shared memory): first the local
+// ones (blocks j .. j+L-1; in block j itself only keys s <= t), then those
+// whose selection holds block j.
+// grid (ceil(Bs/64) * nb, H, B), 64 threads.
+// ---------------------------------------------------------------------------
+constexpr int kBwdKT = 64, kBwdQG = 8;
+
+inline size_t dkdv_smem(int d) {
+    return ((size_t)4 * kBwdKT * (d + 1) + (size_t)2 * kBwdQG * d + 3 * kBwdQG) * 4;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kBwdKT) k_bwd_dkdv(const T *__restrict__ Q, const T *__restrict__ K,
+                                                     const T *__restrict__ V, const float *__restrict__ dO,
+                                                     const float *__restrict__ lse, const float *__restrict__ dsum,
+                                                     const int32_t *__restrict__ cnt, const int32_t *__restrict__ start,
+                                                     const int32_t *__restrict__ list, float *__restrict__ dK,
+                                                     float *__restrict__ dV, int H, int S, int d, int Bs, int L, int R,
+                                                     int nb, float scale) {
+    extern __shared__ __align__(16) float bsm[];
+    const int dp1 = d + 1;
+    float *sk = bsm, *sv = sk + kBwdKT * dp1, *sdk = sv + kBwdKT * dp1, *sdv = sdk + kBwdKT * dp1;
+    float *sq = sdv + kBwdKT * dp1, *sg = sq + kBwdQG * d, *slse = sg + kBwdQG * d, *sD = slse + kBwdQG;
+    int *st = (int *)(sD + kBwdQG);
+    const int tpb = (Bs + kBwdKT - 1) / kBwdKT;
+    const int j = blockIdx.x / tpb, u = blockIdx.x % tpb;
+    const int h = blockIdx.y, b = blockIdx.z;
+    const size_t bh = (size_t)b * H + h;
+    const int k0 = j * Bs + u * kBwdKT;
+    const int nk = min(kBwdKT, Bs - u * kBwdKT);
+    const int tid = threadIdx.x;
+    for (int i = tid; i < kBwdKT * d; i += blockDim.x) {
+        const int s = i / d, e = i % d;
+        const bool in = s < nk;
+        sk[s * dp1 + e] = in ? to_f(K[(bh * S + k0 + s) * d + e]) : 0.f;
+        sv[s * dp1 + e] = in ? to_f(V[(bh * S + k0 + s) * d + e]) : 0.f;
+        sdk[s * dp1 + e] = 0.f;
+        sdv[s * dp1 + e] = 0.f;
+    }
+    const int t_loc0 = j * Bs, t_loc1 = min(S, (j + L) * Bs);  // local queries [t_loc0, t_loc1)
+    const int nloc = t_loc1 - t_loc0;
+    const int nrem = R > 0 ? cnt[bh * nb + j] : 0;
+    const int rem0 = R > 0 ? start[bh * nb + j] : 0;
+    const int nq = nloc + nrem;
+    const int key = k0 + tid;
+    for (int g0 = 0; g0 < nq; g0 += kBwdQG) {
+        const int ng = min(kBwdQG, nq - g0);
+        __syncthreads();  // the previous group is used up (and the tile is loaded)
+        for (int i = tid; i < ng * d; i += blockDim.x) {
+            const int qi = i / d, e = i % d;
+            const int n = g0 + qi;
+            const int t = n < nloc ? t_loc0 + n : list[bh * S * R + rem0 + (n - nloc)];
+            sq[qi * d + e] = to_f(Q[(bh * S + t) * d + e]);
+            sg[qi * d + e] = dO[(((size_t)b * S + t) * H + h) * d + e];
+            if (e == 0) {
+                st[qi] = t;
+                slse[qi] = lse[bh * S + t];
+                sD[qi] = dsum[bh * S + t];
+            }
+        }
+        __syncthreads();
+        if (tid < nk) {
+            for (int qi = 0; qi < ng; ++qi) {
+                const int t = st[qi];
+                if (g0 + qi < nloc && key > t) continue;  // causal inside the query's own block
+                const float *qq = sq + qi * d, *gg = sg + qi * d;
+                const float *kr = sk + tid * dp1, *vr = sv + tid * dp1;
+                float sp = 0.f, dp = 0.f;
+                for (int e = 0; e < d; ++e) {
+                    sp = fmaf(qq[e], kr[e], sp);
+                    dp = fmaf(gg[e], vr[e], dp);
+                }
+                const float p = expf(sp * scale - slse[qi]);
+                const float ds = p * (dp - sD[qi]) * scale;
+                float *dkr = sdk + tid * dp1, *dvr = sdv + tid * dp1;
+                for (int e = 0; e < d; ++e) {
+                    dvr[e] = fmaf(p, gg[e], dvr[e]);
+                    dkr[e] = fmaf(ds, qq[e], dkr[e]);
+                }
+            }
+        }
+    }
+    __syncthreads();
+    for (int i = tid; i < nk * d; i += blockDim.x) {
+        const int s = i / d, e = i % d;
+        dK[(bh * S + k0 + s) * d + e] = sdk[s * dp1 + e];
+        dV[(bh * S + k0 + s) * d + e] = sdv[s * dp1 + e];
+    }
+}
+
+// ---------------------------------------------------------------------------
+// gradients before RoPE, token-major: dQ and dK (post-RoPE, [B,H,S,d]) rotated
+// back by -t*theta^(-2i/d) (the transpose of the forward rotation), dV copied;
+// outputs [B*S, H*d].  One thread per (b, t, h, pair i); grid ceil(B S H d/2 / 256).
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) k_bwd_rope(const float *__restrict__ dQ, const float *__restrict__ dK,
+                                                  const float *__restrict__ dV, float *__restrict__ dQp,
+                                                  float *__restrict__ dKp, float *__restrict__ dVp, int B, int S, int H,
+                                                  int d, double theta) {
+    const long long n = (long long)B * S * H * (d / 2);
+    const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= n) return;
+    const int pr = (int)(i % (d / 2));
+    const int h = (int)((i / (d / 2)) % H);
+    const long long bt = i / ((long long)(d / 2) * H);
+    const int t = (int)(bt % S), b = (int)(bt / S);
+    const double ang = (double)t * pow(theta, -2.0 * (double)pr / (double)d);
+    const float c = (float)cos(ang), s = (float)sin(ang);
+    const size_t src = (((size_t)b * H + h) * S + t) * d + 2 * pr;
+    const size_t dst = ((size_t)bt * H + h) * d + 2 * pr;
+    const float q0 = dQ[src], q1 = dQ[src + 1], k0 = dK[src], k1 = dK[src + 1];
+    dQp[dst] = q0 * c + q1 * s;
+    dQp[dst + 1] = -q0 * s + q1 * c;
+    dKp[dst] = k0 * c + k1 * s;
+    dKp[dst + 1] = -k0 * s + k1 * c;
+    dVp[dst] = dV[src];
+    dVp[dst + 1] = dV[src + 1];
+}
+
+// ---------------------------------------------------------------------------
+// C[M,N] (fp32, row stride ldc) = beta*C + sum_k A(m,k) B(k,n), with
+// A(m,k) = A[m*am + k*ak] and B(k,n) = B[k*bk + n*bn] of types TA, TB
+// (fp32 accumulation).  64x64 tile per CTA, 16-deep k slices staged in shared
+// memory, 4x4 outputs per thread; the tile loads walk the operand's unit-stride
+// index across consecutive threads.  grid (ceil(N/64), ceil(M/64)), 256 threads.
+// ---------------------------------------------------------------------------
+template <typename TA, typename TB>
+__global__ void __launch_bounds__(256) k_gemm_any(int M, int N, int Kd, const TA *__restrict__ A, long long am,
+                                                  long long ak, const TB *__restrict__ Bm, long long bk, long long bn,
+                                                  float *__restrict__ C, long long ldc, float beta) {
+    __shared__ float sA[16][64 + 4];
+    __shared__ float sB[16][64 + 4];
+    const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+    const int m0 = blockIdx.y * 64, n0 = blockIdx.x * 64;
+    float acc[4][4] = {};
+    for (int k0 = 0; k0 < Kd; k0 += 16) {
+        for (int i = tid; i < 64 * 16; i += 256) {
+            int mm, kk;
+            if (ak == 1) { mm = i / 16; kk = i % 16; }
+            else { kk = i / 64; mm = i % 64; }
+            const int m = m0 + mm, k = k0 + kk;
+            sA[kk][mm] = (m < M && k < Kd) ? to_f(A[(long long)m * am + (long long)k * ak]) : 0.f;
+            int nn, kb;
+            if (bn == 1) { kb = i / 64; nn = i % 64; }
+            else { nn = i / 16; kb = i % 16; }
+            const int n = n0 + nn, k2 = k0 + kb;
+            sB[kb][nn] = (n < N && k2 < Kd) ? to_f(Bm[(long long)k2 * bk + (long long)n * bn]) : 0.f;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int kk = 0; kk < 16; ++kk) {
+            float a[4], bv[4];
+#pragma unroll
+            for (int r = 0; r < 4; ++r) a[r] = sA[kk][ty * 4 + r];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) bv[c] = sB[kk][tx * 4 + c];
+#pragma unroll
+            for (int r = 0; r < 4; ++r)
+#pragma unroll
+                for (int c = 0; c < 4; ++c) acc[r][c] = fmaf(a[r], bv[c], acc[r][c]);
+        }
+        __syncthreads();
+    }
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+        const int m = m0 + ty * 4 + r;
+        if (m >= M) continue;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            const int n = n0 + tx * 4 + c;
+            if (n >= N) continue;
+            float *dst = C + (long long)m * ldc + n;
+            *dst = beta == 0.f ? acc[r][c] : fmaf(beta, *dst, acc[r][c]);
+        }
+    }
+}
+
+template <typename TA, typename TB>
+cudaError_t gemm_any(int M, int N, int Kd, const TA *A, long long am, long long ak, const TB *Bm, long long bk,
+                     long long bn, float *C, long long ldc, float beta, cudaStream_t s) {
+    if (M == 0 || N == 0) return cudaSuccess;
+    dim3 g((N + 63) / 64, (M + 63) / 64);
+    k_gemm_any<TA, TB><<<g, 256, 0, s>>>(M, N, Kd, A, am, ak, Bm, bk, bn, C, ldc, beta);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t attend_backward(const Plan &p, const T *Q, const T *K, const T *V, const int32_t *sel, const float *dO,
+                            float *dQ, float *dK, float *dV, char *bws, cudaStream_t s) {
+    const mono_config &c = p.cfg;
+    const BwdLayout L = bwd_layout(p);
+    float *lse = (float *)(bws + L.lse), *dsum = (float *)(bws + L.dsum);
+    int32_t *cnt = (int32_t *)(bws + L.cnt), *start = (int32_t *)(bws + L.start);
+    int32_t *cursor = (int32_t *)(bws + L.cursor), *list = (int32_t *)(bws + L.list);
+    const float scale = (float)(1.0 / sqrt((double)c.d));
+    const long long nq = (long long)c.B * c.H * c.S;
+    cudaError_t e;
+    k_bwd_dq<T><<<(unsigned)((nq + 7) / 8), 256, 0, s>>>(Q, K, V, sel, dO, dQ, lse, dsum, c.B, c.H, c.S, c.d, c.Bs,
+                                                         c.L, c.R, scale);
+    count_launches(1);
+    if (c.R > 0) {
+        const long long n = nq * c.R;
+        if ((e = cudaMemsetAsync(cnt, 0, (size_t)c.B * c.H * p.nb * 4, s)) != cudaSuccess) return e;
+        k_bwd_count<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(sel, cnt, n, c.S, c.R, p.nb, c.Bs, c.L);
+        k_bwd_scan<<<c.B * c.H, 1024, 0, s>>>(cnt, start, cursor, p.nb);
+        k_bwd_fill<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(sel, cursor, list, n, c.S, c.R, p.nb, c.Bs, c.L);
+        count_launches(3);
+    }
+    const size_t sm = dkdv_smem(c.d);
+    if (sm > 48 * 1024 &&
+        (e = cudaFuncSetAttribute(k_bwd_dkdv<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm)) != cudaSuccess)
+        return e;
+    const int tpb = (c.Bs + kBwdKT - 1) / kBwdKT;
+    k_bwd_dkdv<T><<<dim3(tpb * p.nb, c.H, c.B), kBwdKT, sm, s>>>(Q, K, V, dO, lse, dsum, cnt, start, list, dK, dV, c.H,
+                                                                 c.S, c.d, c.Bs, c.L, c.R, p.nb, scale);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t backward_t(const Plan &p, const T *x, const T *Wq, const T *Wk, const T *Wv, const T *Wo,
+                       const int32_t *sel, const T *ddelta, float *dx, float *dWq, float *dWk, float *dWv, float *dWo,
+                       const T *Q, const T *K, const T *V, const T *O, char *bws, cudaStream_t s) {
+    const mono_config &c = p.cfg;
+    const BwdLayout L = bwd_layout(p);
+    float *dO = (float *)(bws + L.dO), *dQ = (float *)(bws + L.dQ), *dK = (float *)(bws + L.dK);
+    float *dV = (float *)(bws + L.dV), *dQp = (float *)(bws + L.dQp), *dKp = (float *)(bws + L.dKp);
+    float *dVp = (float *)(bws + L.dVp);
+    const int BS = c.B * c.S, Hd = c.H * c.d, W = c.W;
+    cudaError_t e;
+    // delta = O Wo^T:  dO = ddelta Wo,  dWo = ddelta^T O
+    if ((e = gemm_any<T, T>(BS, Hd, W, ddelta, W, 1, Wo, Hd, 1, dO, Hd, 0.f, s)) != cudaSuccess) return e;
+    if ((e = gemm_any<T, T>(W, Hd, BS, ddelta, 1, W, O, Hd, 1, dWo, Hd, 0.f, s)) != cudaSuccess) return e;
+    if ((e = attend_backward<T>(p, Q, K, V, sel, dO, dQ, dK, dV, bws, s)) != cudaSuccess) return e;
+    const long long npairs = (long long)BS * Hd / 2;
+    k_bwd_rope<<<(unsigned)((npairs + 255) / 256), 256, 0, s>>>(dQ, dK, dV, dQp, dKp, dVp, c.B, c.S, c.H, c.d,
+                                                                c.rope_theta);
+    count_launches(1);
+    // q = x Wq^T (per head, then RoPE):  dWq = dQp^T x,  dx = dQp Wq + dKp Wk + dVp Wv
+    if ((e = gemm_any<float, T>(Hd, W, BS, dQp, 1, Hd, x, W, 1, dWq, W, 0.f, s)) != cudaSuccess) return e;
+    if ((e = gemm_any<float, T>(Hd, W, BS, dKp, 1, Hd, x, W, 1, dWk, W, 0.f, s)) != cudaSuccess) return e;
+    if ((e = gemm_any<float, T>(Hd, W, BS, dVp, 1, Hd, x, W, 1, dWv, W, 0.f, s)) != cudaSuccess) return e;
+    if ((e = gemm_any<float, T>(BS, W, Hd, dQp, Hd, 1, Wq, W, 1, dx, W, 0.f, s)) != cudaSuccess) return e;
+    if ((e = gemm_any<float, T>(BS, W, Hd, dKp, Hd, 1, Wk, W, 1, dx, W, 1.f, s)) != cudaSuccess) return e;
+    return gemm_any<float, T>(BS, W, Hd, dVp, Hd, 1, Wv, W, 1, dx, W, 1.f, s);
+}
+
+int bwd_check(std::initializer_list<const void *> ptrs) {
+    for (const void *q : ptrs) {
+        if (!q) return MONO_ERR_NULL;
+        if ((uintptr_t)q & 15) return MONO_ERR_ALIGN;
+    }
+    return MONO_OK;
+}
+
+int bwd_status(cudaError_t e) { return e == cudaSuccess ? MONO_OK : MONO_ERR_CUDA; }
+
+}  // namespace
+}  // namespace mono
+
+using namespace mono;
+
+extern "C" {
+
+int mono_backward_workspace_bytes(const mono_plan_t *plan, size_t *bytes) {
+    if (!plan || !bytes) return MONO_ERR_NULL;
+    *bytes = bwd_layout(plan->p).total;
+    return MONO_OK;
+}
+
+int mono_attend_backward(const mono_plan_t *plan, const void *Q, const void *K, const void *V, const int32_t *sel,
+                         const float *dO, float *dQ, float *dK, float *dV, void *bwd_workspace, void *stream) {
+    if (!plan) return MONO_ERR_NULL;
+    if (!bwd_workspace) return MONO_ERR_WORKSPACE;
+    if ((uintptr_t)bwd_workspace & 255) return MONO_ERR_ALIGN;
+    const Plan &p = plan->p;
+    const mono_config &c = p.cfg;
+    if (c.B == 0 || c.S == 0) return MONO_OK;
+    int st = bwd_check({Q, K, V, dO, dQ, dK, dV});
+    if (st) return st;
+    if (c.R > 0 && (st = bwd_check({sel}))) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (c.dtype == MONO_BF16)
+        return bwd_status(attend_backward<__nv_bfloat16>(p, (const __nv_bfloat16 *)Q, (const __nv_bfloat16 *)K,
+                                                         (const __nv_bfloat16 *)V, sel, dO, dQ, dK, dV,
+                                                         (char *)bwd_workspace, s));
+    return bwd_status(attend_backward<float>(p, (const float *)Q, (const float *)K, (const float *)V, sel, dO, dQ, dK,
+                                             dV, (char *)bwd_workspace, s));
+}
+
+int mono_backward(const mono_plan_t *plan, const void *x, const void *Wq, const void *Wk, const void *Wv,
+                  const void *Wo, const int32_t *sel, const void *ddelta, float *dx, float *dWq, float *dWk,
+                  float *dWv, float *dWo, void *workspace, void *bwd_workspace, void *stream) {
+    if (!plan) return MONO_ERR_NULL;
+    if (!workspace || !bwd_workspace) return MONO_ERR_WORKSPACE;
+    if (((uintptr_t)workspace & 255) || ((uintptr_t)bwd_workspace & 255)) return MONO_ERR_ALIGN;
+    const Plan &p = plan->p;
+    const mono_config &c = p.cfg;
+    if (c.B == 0 || c.S == 0) return MONO_OK;
+    int st = bwd_check({x, Wq, Wk, Wv, Wo, ddelta, dx, dWq, dWk, dWv, dWo});
+    if (st) return st;
+    if (c.R > 0 && (st = bwd_check({sel}))) return st;
+    // the forward activations for this selection: Q, K, V and O in the workspace
+    void *Q = (char *)workspace + p.off[kRegQ], *K = (char *)workspace + p.off[kRegK];
+    void *V = (char *)workspace + p.off[kRegV], *O = (char *)workspace + p.off[kRegO];
+    if ((st = mono_project(plan, x, Wq, Wk, Wv, Q, K, V, workspace, stream))) return st;
+    if ((st = mono_attend(plan, Q, K, V, sel, O, workspace, stream))) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    char *bws = (char *)bwd_workspace;
+    if (c.dtype == MONO_BF16) {
+        using B16 = __nv_bfloat16;
+        return bwd_status(backward_t<B16>(p, (const B16 *)x, (const B16 *)Wq, (const B16 *)Wk, (const B16 *)Wv,
+                                          (const B16 *)Wo, sel, (const B16 *)ddelta, dx, dWq, dWk, dWv, dWo,
+                                          (const B16 *)Q, (const B16 *)K, (const B16 *)V, (const B16 *)O, bws, s));
+    }
+    return bwd_status(backward_t<float>(p, (const float *)x, (const float *)Wq, (const float *)Wk, (const float *)Wv,
+                                        (const float *)Wo, sel, (const float *)ddelta, dx, dWq, dWk, dWv, dWo,
+                                        (const float *)Q, (const float *)K, (const float *)V, (const float *)O, bws,
+                                        s));
+}
+
+}  // extern "C"

@@ -35,7 +35,8 @@ EXPORTS = ("mono_plan", "mono_plan_destroy", "mono_workspace_region", "mono_proj
            "mono_out_project", "mono_forward", "mono_stats", "mono_strerror", "mono_version", "mono_kernel_launches",
            "mono_route_static", "mono_route_static_capacity", "mono_decode_cache_bytes",
            "mono_decode_cache_region", "mono_decode_prefill", "mono_decode_project", "mono_decode_route",
-           "mono_decode_attend", "mono_decode_step")
+           "mono_decode_attend", "mono_decode_step", "mono_backward_workspace_bytes", "mono_attend_backward",
+           "mono_backward")
 
 
 class MonoError(RuntimeError):
@@ -90,13 +91,16 @@ _lib.mono_decode_project.argtypes = [_P, ctypes.c_int] + [_P] * 6
 _lib.mono_decode_route.argtypes = [_P, ctypes.c_int] + [_P] * 4
 _lib.mono_decode_attend.argtypes = [_P, ctypes.c_int, _P, _P]
 _lib.mono_decode_step.argtypes = [_P, ctypes.c_int] + [_P] * 10
+_lib.mono_backward_workspace_bytes.argtypes = [_P, ctypes.POINTER(ctypes.c_size_t)]
+_lib.mono_attend_backward.argtypes = [_P] * 11
+_lib.mono_backward.argtypes = [_P] * 16
 _lib.mono_kernel_launches.argtypes = []
 _lib.mono_kernel_launches.restype = ctypes.c_ulonglong
 for _f in ("mono_plan", "mono_workspace_region", "mono_project", "mono_route", "mono_route_summaries",
            "mono_route_lists", "mono_route_queries", "mono_attend", "mono_out_project",
            "mono_forward", "mono_stats", "mono_version", "mono_decode_cache_bytes", "mono_decode_cache_region",
            "mono_decode_prefill", "mono_decode_project", "mono_decode_route", "mono_decode_attend",
-           "mono_decode_step"):
+           "mono_decode_step", "mono_backward_workspace_bytes", "mono_attend_backward", "mono_backward"):
     getattr(_lib, _f).restype = ctypes.c_int
 
 
@@ -346,6 +350,40 @@ def decode_step(plan: Plan, t: int, x_t, Wq, Wk, Wv, Wo, codebooks, delta_t, cac
                                  _ptr(forced_t, "forced_t", (c.B, c.H), torch.int32, optional=True),
                                  _ptr(delta_t, "delta_t", (c.B, c.W), dt), _ptr(cache, "cache"), _stream(stream)),
            "mono_decode_step")
+
+
+# ---------------------------------------------------------------------------
+# backward pass for a fixed selection
+# ---------------------------------------------------------------------------
+def backward_workspace(plan: Plan, device="cuda") -> torch.Tensor:
+    """A caller-owned backward workspace of the size mono_backward_workspace_bytes gives."""
+    n = ctypes.c_size_t()
+    _check(_lib.mono_backward_workspace_bytes(plan.handle, ctypes.byref(n)), "mono_backward_workspace_bytes")
+    return torch.empty(max(int(n.value), 256), dtype=torch.uint8, device=device)
+
+
+def attend_backward(plan: Plan, Q, K, V, sel, dO, dQ, dK, dV, bws, stream=None):
+    c, dt = plan.cfg, plan.dtype
+    qkv = (c.B, c.H, c.S, c.d)
+    f32 = torch.float32
+    _check(_lib.mono_attend_backward(plan.handle, _ptr(Q, "Q", qkv, dt), _ptr(K, "K", qkv, dt), _ptr(V, "V", qkv, dt),
+                                     _ptr(sel, "sel", (c.B, c.H, c.S, c.R), torch.int32),
+                                     _ptr(dO, "dO", (c.B, c.S, c.H * c.d), f32), _ptr(dQ, "dQ", qkv, f32),
+                                     _ptr(dK, "dK", qkv, f32), _ptr(dV, "dV", qkv, f32),
+                                     _ptr(bws, "bwd_workspace"), _stream(stream)), "mono_attend_backward")
+
+
+def backward(plan: Plan, x, Wq, Wk, Wv, Wo, sel, ddelta, dx, dWq, dWk, dWv, dWo, ws, bws, stream=None):
+    c, dt = plan.cfg, plan.dtype
+    hd = c.H * c.d
+    f32 = torch.float32
+    _check(_lib.mono_backward(plan.handle, _ptr(x, "x", (c.B, c.S, c.W), dt), _ptr(Wq, "Wq", (hd, c.W), dt),
+                              _ptr(Wk, "Wk", (hd, c.W), dt), _ptr(Wv, "Wv", (hd, c.W), dt),
+                              _ptr(Wo, "Wo", (c.W, hd), dt), _ptr(sel, "sel", (c.B, c.H, c.S, c.R), torch.int32),
+                              _ptr(ddelta, "ddelta", (c.B, c.S, c.W), dt), _ptr(dx, "dx", (c.B, c.S, c.W), f32),
+                              _ptr(dWq, "dWq", (hd, c.W), f32), _ptr(dWk, "dWk", (hd, c.W), f32),
+                              _ptr(dWv, "dWv", (hd, c.W), f32), _ptr(dWo, "dWo", (c.W, hd), f32),
+                              _ptr(ws, "workspace"), _ptr(bws, "bwd_workspace"), _stream(stream)), "mono_backward")
 
 
 def version() -> int:

@@ -15,6 +15,10 @@ definition of the forward pass, with the gradients taken by autograd:
   Snapshot), scale 1/sqrt(d) -- written here as dense attention under that
   mask;
 * delta = O Wo^T.
+With storage="bf16" (or "f32") the activations are rounded to the storage type
+between stages, as the library and the C oracle's forward store them (Q and K
+after RoPE, V, O), and the rounding's derivative is taken as 1: the gradient
+of the computation as performed on its stored values.
 The routing (summaries, addresses, lists, probe, rerank) is piecewise
 constant in its inputs and has no gradient: the selection is an input.
 """
@@ -55,7 +59,15 @@ def selected_mask(cfg, sel: np.ndarray) -> torch.Tensor:
     return torch.from_numpy(mask)
 
 
-def forward(cfg, x, Wq, Wk, Wv, Wo, sel):
+def _stored(a: torch.Tensor, storage) -> torch.Tensor:
+    """a rounded to the storage type (round to nearest even), with derivative 1."""
+    if storage is None:
+        return a
+    r = a.to(torch.bfloat16 if storage == "bf16" else torch.float32).to(torch.float64)
+    return a + (r - a).detach()
+
+
+def forward(cfg, x, Wq, Wk, Wv, Wo, sel, storage=None):
     """delta [B, S, W] (float64 tensors in, float64 out), for a fixed selection sel [B, H, S, R]."""
     B, S, W, H, d = cfg.B, cfg.S, cfg.W, cfg.H, cfg.d
     theta = float(getattr(cfg, "theta", 10000.0))
@@ -63,19 +75,19 @@ def forward(cfg, x, Wq, Wk, Wv, Wo, sel):
     def heads(w):
         return (x @ w.T).reshape(B, S, H, d).permute(0, 2, 1, 3)             # [B, H, S, d]
 
-    Q, K, V = _rope(heads(Wq), theta), _rope(heads(Wk), theta), heads(Wv)
+    Q, K, V = (_stored(a, storage) for a in (_rope(heads(Wq), theta), _rope(heads(Wk), theta), heads(Wv)))
     scores = (Q @ K.transpose(-1, -2)) / np.sqrt(d)
     scores = scores.masked_fill(~selected_mask(cfg, sel), float("-inf"))
     P = torch.softmax(scores, dim=-1)
-    O = (P @ V).permute(0, 2, 1, 3).reshape(B, S, H * d)
+    O = _stored((P @ V).permute(0, 2, 1, 3).reshape(B, S, H * d), storage)
     return O @ Wo.T
 
 
-def gradients(cfg, x, Wq, Wk, Wv, Wo, sel, ddelta) -> dict:
+def gradients(cfg, x, Wq, Wk, Wv, Wo, sel, ddelta, storage=None) -> dict:
     """d(<delta, ddelta>) with respect to x, Wq, Wk, Wv, Wo (numpy float64 in and out)."""
     ts = {k: torch.tensor(np.asarray(v, np.float64), requires_grad=True)
           for k, v in (("x", x), ("Wq", Wq), ("Wk", Wk), ("Wv", Wv), ("Wo", Wo))}
-    delta = forward(cfg, ts["x"], ts["Wq"], ts["Wk"], ts["Wv"], ts["Wo"], np.asarray(sel))
+    delta = forward(cfg, ts["x"], ts["Wq"], ts["Wk"], ts["Wv"], ts["Wo"], np.asarray(sel), storage=storage)
     g = torch.autograd.grad(delta, list(ts.values()), grad_outputs=torch.tensor(np.asarray(ddelta, np.float64)))
     return {k: gi.numpy() for k, gi in zip(ts, g)}
 

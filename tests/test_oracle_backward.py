@@ -2,7 +2,8 @@
 
 * its forward equals the C oracle's fp64 stages (projection + RoPE, selected-set
   attention, output projection) on the same selection -- two independent
-  statements of the forward pass;
+  statements of the forward pass; with activations stored in fp32 or bf16
+  between stages it equals the C oracle's forward, which stores them the same way;
 * its gradients equal central finite differences (torch.autograd.gradcheck, fp64);
 * a closed form: with one-token blocks, one local block and no remote budget each
   query attends to itself only, so O = V and dV = dO, dQ = dK = 0.
@@ -38,6 +39,17 @@ def test_dense_forward_matches_the_c_oracle(R):
     t = {k: torch.tensor(np.asarray(inp[k], np.float64)) for k in ("x", "Wq", "Wk", "Wv", "Wo")}
     got = bwd.forward(cfg, t["x"], t["Wq"], t["Wk"], t["Wv"], t["Wo"], sel).numpy()
     np.testing.assert_allclose(got, ref, rtol=0, atol=1e-11)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_stored_forward_matches_the_c_oracle_forward(dtype):
+    # the C oracle's forward stores Q, K, V and O in the storage type between stages
+    cfg = tiny(dtype=dtype)
+    inp, sel = routed(cfg, seed=2)
+    ref = oracle.forward(cfg, inp)["delta"]
+    t = {k: torch.tensor(np.asarray(inp[k], np.float64)) for k in ("x", "Wq", "Wk", "Wv", "Wo")}
+    got = bwd.forward(cfg, t["x"], t["Wq"], t["Wk"], t["Wv"], t["Wo"], sel, storage=dtype).numpy()
+    np.testing.assert_allclose(got, ref, rtol=0, atol=1e-10)
 
 
 def test_gradients_match_finite_differences():
