@@ -3,6 +3,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload scale32k] [--no-sweep] [--no-cpu-baseline] [--no-decode]
+                    [--no-backward]
 
 A step is one pass of the whole hot path over one batch: projection + RoPE,
 block summaries + addresses, posting lists, probe/rerank, selected-set
@@ -261,6 +262,8 @@ def run_ours(args):
     e2e_ms = dist.reduce_max([mean([a.elapsed_time(b) for a, b in e2e_ev])], device=dev)[0]
 
     decode = measure_decode(plan, cfg, K, V, inp, tdt, dev, stream, hbm) if not args.no_decode else None
+    backward = measure_backward(plan, cfg, x, Wq, Wk, Wv, Wo, sel, ws, tdt, dev, stream) \
+        if not args.no_backward else None
 
     sweep = None
     if not args.no_sweep and world == 1 and args.workload == "scale32k":
@@ -300,6 +303,8 @@ def run_ours(args):
         }
         if decode:
             out["decode"] = decode
+        if backward:
+            out["backward"] = backward
         if sweep:
             out["s_sweep"] = sweep
         if cpu:
@@ -371,6 +376,49 @@ def measure_decode(plan, cfg, K, V, inp, tdt, dev, stream, hbm, n_steps=128):
                    "graph of the steps, ms_per_token_eager from one Python call per step",
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
                          "algorithmic_bytes": per_step}}
+
+
+# fp32 FMA peak from the unit counts: 148 SMs x 128 fp32 lanes x 2 flops x 1.965 GHz
+FP32_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+def measure_backward(plan, cfg, x, Wq, Wk, Wv, Wo, sel, ws, tdt, dev, stream, steps=3):
+    """mono_backward for the step's selection and a seeded upstream gradient: mean of `steps`
+    timed calls after one warm-up.  Algorithmic flops: the forward recompute (projection and
+    selected-set attention), the projection gradients (8 GEMMs of B*S x H*d x W) and the
+    attention gradients (per query and selected key: 2 dot products in the log-sum-exp pass,
+    3 in the dQ pass, 4 in the dK/dV pass, of d multiply-adds each)."""
+    import torch
+
+    from learned_product_hash_proj_b200 import mono
+    B, S, W, H, d = cfg.B, cfg.S, cfg.W, cfg.H, cfg.d
+    g = torch.Generator(device="cpu").manual_seed(11)
+    ddelta = torch.randn((B, S, W), generator=g).to(tdt).to(dev)
+    f32 = dict(dtype=torch.float32, device=dev)
+    dx = torch.empty((B, S, W), **f32)
+    dWq, dWk, dWv = (torch.empty((H * d, W), **f32) for _ in range(3))
+    dWo = torch.empty((W, H * d), **f32)
+    bws = mono.backward_workspace(plan, device=dev)
+    run = lambda: mono.backward(plan, x, Wq, Wk, Wv, Wo, sel, ddelta, dx, dWq, dWk, dWv, dWo, ws, bws, stream=stream)
+    run()
+    torch.cuda.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    ev[0].record(stream)
+    for _ in range(steps):
+        run()
+    ev[1].record(stream)
+    torch.cuda.synchronize()
+    ms = ev[0].elapsed_time(ev[1]) / steps
+    nsel = int((sel >= 0).sum().item())
+    keys = nsel * cfg.Bs + B * H * S * ((cfg.L - 1) * cfg.Bs + (cfg.Bs + 1) / 2)   # selected keys, all queries
+    gemm = 2.0 * B * S * H * d * W
+    flops = 3 * gemm + 2 * keys * 2 * d + 8 * gemm + (2 + 3 + 4) * keys * 2 * d
+    tf = flops / (ms / 1e3) / 1e12
+    return {"ms": ms, "tokens_per_s": B * S / (ms / 1e3),
+            "api": "mono_backward (forward recompute + gradients of x, Wq, Wk, Wv, Wo for a fixed selection)",
+            "roofline": {"bound": "alu", "achieved": tf, "peak": FP32_PEAK_TFLOPS, "unit": "TFLOP/s",
+                         "frac": tf / FP32_PEAK_TFLOPS, "algorithmic_flops": flops,
+                         "peak_source": "fp32 lanes x clock: 148 x 128 x 2 x 1.965 GHz"}}
 
 
 def load_traffic(stage: str, cfg):
@@ -513,6 +561,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="scale32k")
     ap.add_argument("--no-decode", action="store_true", help="skip the decode latency measurement")
+    ap.add_argument("--no-backward", action="store_true", help="skip the backward-pass measurement")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -19,7 +19,8 @@
 //                walks the block's local queries and its selecting queries,
 //                accumulating dK and dV of its keys in shared memory;
 //   k_bwd_rope   inverse rotation of dQ, dK and the token-major layout;
-//   k_gemm_any   the projection gradients (generic strided SIMT GEMM).
+//   k_gemm_any   the projection gradients (generic strided SIMT GEMM, split K
+//                with fp32 atomics where the output has few tiles).
 #include <cuda_runtime.h>
 
 #include <math.h>
@@ -77,20 +78,19 @@ __device__ __forceinline__ bool bwd_sel_valid(int j, int t, int Bs, int L) { ret
 // log-sum-exp and O in fp32, hence D = dO . O; pass 2 forms dS and dQ.
 // grid ceil(B H S / 8), 256 threads.
 // ---------------------------------------------------------------------------
-template <typename T>
+template <typename T, int DD>
 __global__ void __launch_bounds__(256) k_bwd_dq(const T *__restrict__ Q, const T *__restrict__ K,
                                                 const T *__restrict__ V, const int32_t *__restrict__ sel,
                                                 const float *__restrict__ dO, float *__restrict__ dQ,
                                                 float *__restrict__ lse_out, float *__restrict__ dsum_out, int B, int H,
-                                                int S, int d, int Bs, int L, int R, float scale) {
-    constexpr int kPer = kMaxD / 32;
+                                                int S, int Bs, int L, int R, float scale) {
+    constexpr int d = DD, kPer = DD / 32, per = kPer;
     const int lane = threadIdx.x & 31;
     const long long w = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     if (w >= (long long)B * H * S) return;
     const long long bh = w / S;
     const int t = (int)(w % S);
     const int b = (int)(bh / H), h = (int)(bh % H);
-    const int per = d / 32;
     float q[kPer], g[kPer];
     for (int e = 0; e < per; ++e) {
         q[e] = to_f(Q[w * d + lane * per + e]);
@@ -106,18 +106,43 @@ __global__ void __launch_bounds__(256) k_bwd_dq(const T *__restrict__ Q, const T
     const int nkeys = nr * Bs + (t - lo + 1);
     auto key_of = [&](int idx) { return idx < nr * Bs ? js[idx / Bs] * Bs + idx % Bs : lo + (idx - nr * Bs); };
     const size_t base = (size_t)bh * S;
+    // keys four at a time: their rows are loaded together and their warp sums interleave
+    constexpr int U = 4;
     // pass 1: log-sum-exp and O
     float m = -INFINITY, l = 0.f, o[kPer];
     for (int e = 0; e < per; ++e) o[e] = 0.f;
-    for (int idx = 0; idx < nkeys; ++idx) {
-        const size_t row = (base + key_of(idx)) * d + lane * per;
-        float part = 0.f;
-        for (int e = 0; e < per; ++e) part = fmaf(q[e], to_f(K[row + e]), part);
-        const float s = bwd_warp_sum(part) * scale;
-        const float mn = fmaxf(m, s), corr = expf(m - mn), p = expf(s - mn);
-        l = l * corr + p;
-        for (int e = 0; e < per; ++e) o[e] = fmaf(p, to_f(V[row + e]), o[e] * corr);
-        m = mn;
+    for (int idx = 0; idx < nkeys; idx += U) {
+        float kk[U][kPer], vv[U][kPer], sc[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const bool in = idx + u < nkeys;
+            const size_t row = (base + key_of(in ? idx + u : idx)) * d + lane * per;
+            for (int e = 0; e < per; ++e) {
+                kk[u][e] = to_f(K[row + e]);
+                vv[u][e] = to_f(V[row + e]);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            float part = 0.f;
+            for (int e = 0; e < per; ++e) part = fmaf(q[e], kk[u][e], part);
+            sc[u] = bwd_warp_sum(part) * scale;
+        }
+        float mx = m;
+#pragma unroll
+        for (int u = 0; u < U; ++u)
+            if (idx + u < nkeys) mx = fmaxf(mx, sc[u]);
+        const float corr = expf(m - mx);
+        l *= corr;
+        for (int e = 0; e < per; ++e) o[e] *= corr;
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            if (idx + u >= nkeys) continue;
+            const float p = expf(sc[u] - mx);
+            l += p;
+            for (int e = 0; e < per; ++e) o[e] = fmaf(p, vv[u][e], o[e]);
+        }
+        m = mx;
     }
     const float lse = m + logf(l);
     float dpart = 0.f;
@@ -126,17 +151,32 @@ __global__ void __launch_bounds__(256) k_bwd_dq(const T *__restrict__ Q, const T
     // pass 2: dS and dQ
     float dq[kPer];
     for (int e = 0; e < per; ++e) dq[e] = 0.f;
-    for (int idx = 0; idx < nkeys; ++idx) {
-        const size_t row = (base + key_of(idx)) * d + lane * per;
-        float sp = 0.f, dp = 0.f;
-        for (int e = 0; e < per; ++e) {
-            sp = fmaf(q[e], to_f(K[row + e]), sp);
-            dp = fmaf(g[e], to_f(V[row + e]), dp);
+    for (int idx = 0; idx < nkeys; idx += U) {
+        float kk[U][kPer], sp[U], dp[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const bool in = idx + u < nkeys;
+            const size_t row = (base + key_of(in ? idx + u : idx)) * d + lane * per;
+            float a = 0.f, c = 0.f;
+            for (int e = 0; e < per; ++e) {
+                kk[u][e] = to_f(K[row + e]);
+                a = fmaf(q[e], kk[u][e], a);
+                c = fmaf(g[e], to_f(V[row + e]), c);
+            }
+            sp[u] = a;
+            dp[u] = c;
         }
-        const float s = bwd_warp_sum(sp) * scale;
-        const float p = expf(s - lse);
-        const float ds = p * (bwd_warp_sum(dp) - D);
-        for (int e = 0; e < per; ++e) dq[e] = fmaf(ds, to_f(K[row + e]), dq[e]);
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            sp[u] = bwd_warp_sum(sp[u]);
+            dp[u] = bwd_warp_sum(dp[u]);
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            if (idx + u >= nkeys) continue;
+            const float ds = expf(sp[u] * scale - lse) * (dp[u] - D);
+            for (int e = 0; e < per; ++e) dq[e] = fmaf(ds, kk[u][e], dq[e]);
+        }
     }
     for (int e = 0; e < per; ++e) dQ[w * d + lane * per + e] = dq[e] * scale;
     if (lane == 0) {
@@ -333,69 +373,84 @@ __global__ void __launch_bounds__(256) k_bwd_rope(const float *__restrict__ dQ, 
 }
 
 // ---------------------------------------------------------------------------
-// C[M,N] (fp32, row stride ldc) = beta*C + sum_k A(m,k) B(k,n), with
+// C[M,N] (fp32, row stride ldc) (+)= sum_k A(m,k) B(k,n), with
 // A(m,k) = A[m*am + k*ak] and B(k,n) = B[k*bk + n*bn] of types TA, TB
-// (fp32 accumulation).  64x64 tile per CTA, 16-deep k slices staged in shared
-// memory, 4x4 outputs per thread; the tile loads walk the operand's unit-stride
-// index across consecutive threads.  grid (ceil(N/64), ceil(M/64)), 256 threads.
+// (fp32 accumulation).  128x128 tile per CTA, 8-deep k slices staged in shared
+// memory, 8x8 outputs per thread; the tile loads walk the operand's
+// unit-stride index across consecutive threads.  With split > 1 the CTA
+// (blockIdx.z) takes one of `split` k ranges and adds its partial sums to C
+// with fp32 atomics (C holds 0 or the sum to accumulate onto).
+// grid (ceil(N/128), ceil(M/128), split), 256 threads.
 // ---------------------------------------------------------------------------
 template <typename TA, typename TB>
 __global__ void __launch_bounds__(256) k_gemm_any(int M, int N, int Kd, const TA *__restrict__ A, long long am,
                                                   long long ak, const TB *__restrict__ Bm, long long bk, long long bn,
-                                                  float *__restrict__ C, long long ldc, float beta) {
-    __shared__ float sA[16][64 + 4];
-    __shared__ float sB[16][64 + 4];
+                                                  float *__restrict__ C, long long ldc, int kchunk, bool atomic) {
+    __shared__ __align__(16) float sA[8][128 + 4];
+    __shared__ __align__(16) float sB[8][128 + 4];
     const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
-    const int m0 = blockIdx.y * 64, n0 = blockIdx.x * 64;
-    float acc[4][4] = {};
-    for (int k0 = 0; k0 < Kd; k0 += 16) {
-        for (int i = tid; i < 64 * 16; i += 256) {
+    const int m0 = blockIdx.y * 128, n0 = blockIdx.x * 128;
+    const int kb = blockIdx.z * kchunk, ke = min(Kd, kb + kchunk);
+    float acc[8][8] = {};
+    for (int k0 = kb; k0 < ke; k0 += 8) {
+        for (int i = tid; i < 128 * 8; i += 256) {
             int mm, kk;
-            if (ak == 1) { mm = i / 16; kk = i % 16; }
-            else { kk = i / 64; mm = i % 64; }
+            if (ak == 1) { mm = i / 8; kk = i % 8; }
+            else { kk = i / 128; mm = i % 128; }
             const int m = m0 + mm, k = k0 + kk;
-            sA[kk][mm] = (m < M && k < Kd) ? to_f(A[(long long)m * am + (long long)k * ak]) : 0.f;
-            int nn, kb;
-            if (bn == 1) { kb = i / 64; nn = i % 64; }
-            else { nn = i / 16; kb = i % 16; }
-            const int n = n0 + nn, k2 = k0 + kb;
-            sB[kb][nn] = (n < N && k2 < Kd) ? to_f(Bm[(long long)k2 * bk + (long long)n * bn]) : 0.f;
+            sA[kk][mm] = (m < M && k < ke) ? to_f(A[(long long)m * am + (long long)k * ak]) : 0.f;
+            int nn, kq;
+            if (bn == 1) { kq = i / 128; nn = i % 128; }
+            else { nn = i / 8; kq = i % 8; }
+            const int n = n0 + nn, k2 = k0 + kq;
+            sB[kq][nn] = (n < N && k2 < ke) ? to_f(Bm[(long long)k2 * bk + (long long)n * bn]) : 0.f;
         }
         __syncthreads();
 #pragma unroll
-        for (int kk = 0; kk < 16; ++kk) {
-            float a[4], bv[4];
+        for (int kk = 0; kk < 8; ++kk) {
+            const float4 a0 = *(const float4 *)&sA[kk][ty * 8], a1 = *(const float4 *)&sA[kk][ty * 8 + 4];
+            const float4 b0 = *(const float4 *)&sB[kk][tx * 8], b1 = *(const float4 *)&sB[kk][tx * 8 + 4];
+            const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+            const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
-            for (int r = 0; r < 4; ++r) a[r] = sA[kk][ty * 4 + r];
+            for (int r = 0; r < 8; ++r)
 #pragma unroll
-            for (int c = 0; c < 4; ++c) bv[c] = sB[kk][tx * 4 + c];
-#pragma unroll
-            for (int r = 0; r < 4; ++r)
-#pragma unroll
-                for (int c = 0; c < 4; ++c) acc[r][c] = fmaf(a[r], bv[c], acc[r][c]);
+                for (int c = 0; c < 8; ++c) acc[r][c] = fmaf(a[r], bv[c], acc[r][c]);
         }
         __syncthreads();
     }
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
-        const int m = m0 + ty * 4 + r;
+    for (int r = 0; r < 8; ++r) {
+        const int m = m0 + ty * 8 + r;
         if (m >= M) continue;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            const int n = n0 + tx * 4 + c;
+        for (int c = 0; c < 8; ++c) {
+            const int n = n0 + tx * 8 + c;
             if (n >= N) continue;
             float *dst = C + (long long)m * ldc + n;
-            *dst = beta == 0.f ? acc[r][c] : fmaf(beta, *dst, acc[r][c]);
+            if (atomic) atomicAdd(dst, acc[r][c]);
+            else *dst = acc[r][c];
         }
     }
 }
 
+// beta 0: C = A B; beta 1: C += A B.  Output tiles fewer than twice the SMs split K.
 template <typename TA, typename TB>
 cudaError_t gemm_any(int M, int N, int Kd, const TA *A, long long am, long long ak, const TB *Bm, long long bk,
                      long long bn, float *C, long long ldc, float beta, cudaStream_t s) {
     if (M == 0 || N == 0) return cudaSuccess;
-    dim3 g((N + 63) / 64, (M + 63) / 64);
-    k_gemm_any<TA, TB><<<g, 256, 0, s>>>(M, N, Kd, A, am, ak, Bm, bk, bn, C, ldc, beta);
+    const int tiles = ((N + 127) / 128) * ((M + 127) / 128);
+    int split = 1;
+    while (split < 32 && tiles * split < 2 * 148 && Kd / (split * 2) >= 256) split *= 2;
+    const int kchunk = ((Kd + split - 1) / split + 7) / 8 * 8;
+    const bool atomic = split > 1 || beta != 0.f;
+    cudaError_t e;
+    if (atomic && beta == 0.f) {
+        if (ldc != N) return cudaErrorInvalidValue;  // callers pass dense C
+        if ((e = cudaMemsetAsync(C, 0, (size_t)M * N * sizeof(float), s)) != cudaSuccess) return e;
+    }
+    dim3 g((N + 127) / 128, (M + 127) / 128, split);
+    k_gemm_any<TA, TB><<<g, 256, 0, s>>>(M, N, Kd, A, am, ak, Bm, bk, bn, C, ldc, kchunk, atomic);
     count_launches(1);
     return cudaGetLastError();
 }
@@ -411,8 +466,12 @@ cudaError_t attend_backward(const Plan &p, const T *Q, const T *K, const T *V, c
     const float scale = (float)(1.0 / sqrt((double)c.d));
     const long long nq = (long long)c.B * c.H * c.S;
     cudaError_t e;
-    k_bwd_dq<T><<<(unsigned)((nq + 7) / 8), 256, 0, s>>>(Q, K, V, sel, dO, dQ, lse, dsum, c.B, c.H, c.S, c.d, c.Bs,
-                                                         c.L, c.R, scale);
+    if (c.d == 64)
+        k_bwd_dq<T, 64><<<(unsigned)((nq + 7) / 8), 256, 0, s>>>(Q, K, V, sel, dO, dQ, lse, dsum, c.B, c.H, c.S,
+                                                                 c.Bs, c.L, c.R, scale);
+    else
+        k_bwd_dq<T, 128><<<(unsigned)((nq + 7) / 8), 256, 0, s>>>(Q, K, V, sel, dO, dQ, lse, dsum, c.B, c.H, c.S,
+                                                                  c.Bs, c.L, c.R, scale);
     count_launches(1);
     if (c.R > 0) {
         const long long n = nq * c.R;
