@@ -17,7 +17,7 @@
 //                queries that selected j (lists in unspecified order);
 //   k_bwd_dkdv   one CTA per (b, h) and tile of up to 64 keys of one block:
 //                walks the block's local queries and its selecting queries,
-//                accumulating dK and dV of its keys in shared memory;
+//                accumulating dK and dV of its keys in registers;
 //   k_bwd_rope   inverse rotation of dQ, dK and the token-major layout;
 //   k_gemm_any   the projection gradients (generic strided SIMT GEMM, split K
 //                with fp32 atomics where the output has few tiles).
@@ -250,33 +250,29 @@ __global__ void __launch_bounds__(256) k_bwd_fill(const int32_t *__restrict__ se
 }
 
 // ---------------------------------------------------------------------------
-// dK and dV of a tile of up to 64 keys of block j of one (b, h): one thread
-// per key, the tile's K and V rows and the dK / dV accumulators in padded
-// shared memory (row stride d+1: conflict-free).  Queries come in groups of 8
-// (their q, dO, log-sum-exp and D staged in shared memory): first the local
-// ones (blocks j .. j+L-1; in block j itself only keys s <= t), then those
-// whose selection holds block j.
-// grid (ceil(Bs/64) * nb, H, B), 64 threads.
+// dK and dV of a tile of up to 64 keys of block j of one (b, h): D/16 threads
+// per key, each holding 16 dimensions of the key's K and V rows and of its dK
+// and dV accumulators in registers; a key's threads are consecutive lanes and
+// combine their partial dot products with xor shuffles.  Queries come in
+// groups of 8 (q, dO, log-sum-exp and D staged in shared memory, read as
+// broadcast float4): first the local ones (blocks j .. j+L-1; in block j
+// itself only keys s <= t, applied as a zero probability so that every lane
+// takes part in the shuffles), then those whose selection holds block j.
+// grid (ceil(Bs/64) * nb, H, B), 64 * D/16 threads.
 // ---------------------------------------------------------------------------
 constexpr int kBwdKT = 64, kBwdQG = 8;
 
-inline size_t dkdv_smem(int d) {
-    return ((size_t)4 * kBwdKT * (d + 1) + (size_t)2 * kBwdQG * d + 3 * kBwdQG) * 4;
-}
-
-template <typename T>
-__global__ void __launch_bounds__(kBwdKT) k_bwd_dkdv(const T *__restrict__ Q, const T *__restrict__ K,
-                                                     const T *__restrict__ V, const float *__restrict__ dO,
-                                                     const float *__restrict__ lse, const float *__restrict__ dsum,
-                                                     const int32_t *__restrict__ cnt, const int32_t *__restrict__ start,
-                                                     const int32_t *__restrict__ list, float *__restrict__ dK,
-                                                     float *__restrict__ dV, int H, int S, int d, int Bs, int L, int R,
-                                                     int nb, float scale) {
-    extern __shared__ __align__(16) float bsm[];
-    const int dp1 = d + 1;
-    float *sk = bsm, *sv = sk + kBwdKT * dp1, *sdk = sv + kBwdKT * dp1, *sdv = sdk + kBwdKT * dp1;
-    float *sq = sdv + kBwdKT * dp1, *sg = sq + kBwdQG * d, *slse = sg + kBwdQG * d, *sD = slse + kBwdQG;
-    int *st = (int *)(sD + kBwdQG);
+template <typename T, int DD>
+__global__ void __launch_bounds__(kBwdKT * DD / 16) k_bwd_dkdv(
+    const T *__restrict__ Q, const T *__restrict__ K, const T *__restrict__ V, const float *__restrict__ dO,
+    const float *__restrict__ lse, const float *__restrict__ dsum, const int32_t *__restrict__ cnt,
+    const int32_t *__restrict__ start, const int32_t *__restrict__ list, float *__restrict__ dK,
+    float *__restrict__ dV, int H, int S, int Bs, int L, int R, int nb, float scale) {
+    constexpr int TPK = DD / 16, NT = kBwdKT * TPK, E = 16;
+    __shared__ __align__(16) float sq[kBwdQG][DD];
+    __shared__ __align__(16) float sg[kBwdQG][DD];
+    __shared__ float slse[kBwdQG], sD[kBwdQG];
+    __shared__ int st[kBwdQG];
     const int tpb = (Bs + kBwdKT - 1) / kBwdKT;
     const int j = blockIdx.x / tpb, u = blockIdx.x % tpb;
     const int h = blockIdx.y, b = blockIdx.z;
@@ -284,29 +280,31 @@ __global__ void __launch_bounds__(kBwdKT) k_bwd_dkdv(const T *__restrict__ Q, co
     const int k0 = j * Bs + u * kBwdKT;
     const int nk = min(kBwdKT, Bs - u * kBwdKT);
     const int tid = threadIdx.x;
-    for (int i = tid; i < kBwdKT * d; i += blockDim.x) {
-        const int s = i / d, e = i % d;
-        const bool in = s < nk;
-        sk[s * dp1 + e] = in ? to_f(K[(bh * S + k0 + s) * d + e]) : 0.f;
-        sv[s * dp1 + e] = in ? to_f(V[(bh * S + k0 + s) * d + e]) : 0.f;
-        sdk[s * dp1 + e] = 0.f;
-        sdv[s * dp1 + e] = 0.f;
+    const int ks = tid / TPK, part = tid % TPK, e0 = part * E;
+    const bool live = ks < nk;
+    const int key = k0 + ks;
+    float kr[E], vr[E], dk[E], dv[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+        kr[e] = live ? to_f(K[(bh * S + key) * DD + e0 + e]) : 0.f;
+        vr[e] = live ? to_f(V[(bh * S + key) * DD + e0 + e]) : 0.f;
+        dk[e] = 0.f;
+        dv[e] = 0.f;
     }
     const int t_loc0 = j * Bs, t_loc1 = min(S, (j + L) * Bs);  // local queries [t_loc0, t_loc1)
     const int nloc = t_loc1 - t_loc0;
     const int nrem = R > 0 ? cnt[bh * nb + j] : 0;
     const int rem0 = R > 0 ? start[bh * nb + j] : 0;
     const int nq = nloc + nrem;
-    const int key = k0 + tid;
     for (int g0 = 0; g0 < nq; g0 += kBwdQG) {
         const int ng = min(kBwdQG, nq - g0);
-        __syncthreads();  // the previous group is used up (and the tile is loaded)
-        for (int i = tid; i < ng * d; i += blockDim.x) {
-            const int qi = i / d, e = i % d;
+        __syncthreads();  // the previous group is used up
+        for (int i = tid; i < ng * DD; i += NT) {
+            const int qi = i / DD, e = i % DD;
             const int n = g0 + qi;
             const int t = n < nloc ? t_loc0 + n : list[bh * S * R + rem0 + (n - nloc)];
-            sq[qi * d + e] = to_f(Q[(bh * S + t) * d + e]);
-            sg[qi * d + e] = dO[(((size_t)b * S + t) * H + h) * d + e];
+            sq[qi][e] = to_f(Q[(bh * S + t) * DD + e]);
+            sg[qi][e] = dO[(((size_t)b * S + t) * H + h) * DD + e];
             if (e == 0) {
                 st[qi] = t;
                 slse[qi] = lse[bh * S + t];
@@ -314,32 +312,42 @@ __global__ void __launch_bounds__(kBwdKT) k_bwd_dkdv(const T *__restrict__ Q, co
             }
         }
         __syncthreads();
-        if (tid < nk) {
-            for (int qi = 0; qi < ng; ++qi) {
-                const int t = st[qi];
-                if (g0 + qi < nloc && key > t) continue;  // causal inside the query's own block
-                const float *qq = sq + qi * d, *gg = sg + qi * d;
-                const float *kr = sk + tid * dp1, *vr = sv + tid * dp1;
-                float sp = 0.f, dp = 0.f;
-                for (int e = 0; e < d; ++e) {
-                    sp = fmaf(qq[e], kr[e], sp);
-                    dp = fmaf(gg[e], vr[e], dp);
-                }
-                const float p = expf(sp * scale - slse[qi]);
-                const float ds = p * (dp - sD[qi]) * scale;
-                float *dkr = sdk + tid * dp1, *dvr = sdv + tid * dp1;
-                for (int e = 0; e < d; ++e) {
-                    dvr[e] = fmaf(p, gg[e], dvr[e]);
-                    dkr[e] = fmaf(ds, qq[e], dkr[e]);
-                }
+        for (int qi = 0; qi < ng; ++qi) {
+            const float4 *q4 = (const float4 *)&sq[qi][e0], *g4 = (const float4 *)&sg[qi][e0];
+            float qv[E], gv[E];
+#pragma unroll
+            for (int c = 0; c < E / 4; ++c) {
+                const float4 a = q4[c], bb = g4[c];
+                qv[4 * c] = a.x; qv[4 * c + 1] = a.y; qv[4 * c + 2] = a.z; qv[4 * c + 3] = a.w;
+                gv[4 * c] = bb.x; gv[4 * c + 1] = bb.y; gv[4 * c + 2] = bb.z; gv[4 * c + 3] = bb.w;
+            }
+            float sp = 0.f, dp = 0.f;
+#pragma unroll
+            for (int e = 0; e < E; ++e) {
+                sp = fmaf(qv[e], kr[e], sp);
+                dp = fmaf(gv[e], vr[e], dp);
+            }
+#pragma unroll
+            for (int o = 1; o < TPK; o <<= 1) {
+                sp += __shfl_xor_sync(0xffffffffu, sp, o);
+                dp += __shfl_xor_sync(0xffffffffu, dp, o);
+            }
+            const bool masked = !live || (g0 + qi < nloc && key > st[qi]);  // causal inside the query's own block
+            const float p = masked ? 0.f : expf(sp * scale - slse[qi]);
+            const float ds = p * (dp - sD[qi]) * scale;
+#pragma unroll
+            for (int e = 0; e < E; ++e) {
+                dv[e] = fmaf(p, gv[e], dv[e]);
+                dk[e] = fmaf(ds, qv[e], dk[e]);
             }
         }
     }
-    __syncthreads();
-    for (int i = tid; i < nk * d; i += blockDim.x) {
-        const int s = i / d, e = i % d;
-        dK[(bh * S + k0 + s) * d + e] = sdk[s * dp1 + e];
-        dV[(bh * S + k0 + s) * d + e] = sdv[s * dp1 + e];
+    if (live) {
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+            dK[(bh * S + key) * DD + e0 + e] = dk[e];
+            dV[(bh * S + key) * DD + e0 + e] = dv[e];
+        }
     }
 }
 
@@ -481,13 +489,14 @@ cudaError_t attend_backward(const Plan &p, const T *Q, const T *K, const T *V, c
         k_bwd_fill<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(sel, cursor, list, n, c.S, c.R, p.nb, c.Bs, c.L);
         count_launches(3);
     }
-    const size_t sm = dkdv_smem(c.d);
-    if (sm > 48 * 1024 &&
-        (e = cudaFuncSetAttribute(k_bwd_dkdv<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm)) != cudaSuccess)
-        return e;
     const int tpb = (c.Bs + kBwdKT - 1) / kBwdKT;
-    k_bwd_dkdv<T><<<dim3(tpb * p.nb, c.H, c.B), kBwdKT, sm, s>>>(Q, K, V, dO, lse, dsum, cnt, start, list, dK, dV, c.H,
-                                                                 c.S, c.d, c.Bs, c.L, c.R, p.nb, scale);
+    const dim3 gk(tpb * p.nb, c.H, c.B);
+    if (c.d == 64)
+        k_bwd_dkdv<T, 64><<<gk, kBwdKT * 4, 0, s>>>(Q, K, V, dO, lse, dsum, cnt, start, list, dK, dV, c.H, c.S, c.Bs,
+                                                     c.L, c.R, p.nb, scale);
+    else
+        k_bwd_dkdv<T, 128><<<gk, kBwdKT * 8, 0, s>>>(Q, K, V, dO, lse, dsum, cnt, start, list, dK, dV, c.H, c.S, c.Bs,
+                                                      c.L, c.R, p.nb, scale);
     count_launches(1);
     return cudaGetLastError();
 }
