@@ -312,7 +312,12 @@ int mono_attend_backward(const mono_plan_t *plan, const void *Q, const void *K, 
  * (x, Wq, Wk, Wv, Wo in dtype) plus sel [B,H,S,R] and ddelta [B,S,W] (dtype);
  * outputs dx [B,S,W] and dWq, dWk, dWv [H*d,W], dWo [W,H*d], fp32.  The forward
  * activations Q, K, V and O are recomputed into `workspace` (the forward
- * workspace of the plan). */
+ * workspace of the plan).  With bf16 storage the five projection gradients
+ * run on the tensor cores with bf16 operands: the stored activations and
+ * weights and ddelta, which are bf16 already, and the fp32 gradients before
+ * the projections (dQ, dK after the inverse rotation, dV), each given as two
+ * bf16 terms hi + lo (16 significant bits); products accumulate in fp32.
+ * With fp32 storage every operand stays fp32. */
 int mono_backward(const mono_plan_t *plan, const void *x, const void *Wq, const void *Wk, const void *Wv,
                   const void *Wo, const int32_t *sel, const void *ddelta, float *dx, float *dWq, float *dWk,
                   float *dWv, float *dWo, void *workspace, void *bwd_workspace, void *stream);

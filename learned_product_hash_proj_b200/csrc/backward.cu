@@ -11,7 +11,7 @@
 //     D_t = dO_t . O_t,   dS_ts = P_ts (dO_t . v_s - D_t),
 //     dQ_t = scale sum_s dS_ts k_s,   dK_s += scale dS_ts q_t,   dV_s += P_ts dO_t.
 // Kernels (fp32 arithmetic, gradients in fp32):
-//   k_bwd_dq     one warp per query-head: log-sum-exp and D from recomputed
+//   k_bwd_dq     d/16 lanes per query-head: log-sum-exp and D from recomputed
 //                scores (the stored O is not needed), then dQ;
 //   k_bwd_count / k_bwd_scan / k_bwd_fill: per (b, h) and block j, the
 //                queries that selected j (lists in unspecified order);
@@ -19,8 +19,11 @@
 //                walks the block's local queries and its selecting queries,
 //                accumulating dK and dV of its keys in registers;
 //   k_bwd_rope   inverse rotation of dQ, dK and the token-major layout;
-//   k_gemm_any   the projection gradients (generic strided SIMT GEMM, split K
-//                with fp32 atomics where the output has few tiles).
+//   k_gemm_any   the projection gradients of fp32 storage (generic strided SIMT
+//                GEMM, split K with fp32 atomics where the output has few
+//                tiles); with bf16 storage they run on the tensor cores
+//                (k_gemm_grad_tc: bf16 operands -- the gradients before the
+//                projections rounded to bf16 -- with fp32 accumulation).
 #include <cuda_runtime.h>
 
 #include <math.h>
@@ -73,115 +76,186 @@ __device__ __forceinline__ float bwd_warp_sum(float v) {
 __device__ __forceinline__ bool bwd_sel_valid(int j, int t, int Bs, int L) { return j >= 0 && j <= t / Bs - L; }
 
 // ---------------------------------------------------------------------------
-// dQ, log-sum-exp and D of every query-head: one warp each, lanes own d/32
-// dimensions.  Pass 1 (online softmax over the selected keys) gives the
-// log-sum-exp and O in fp32, hence D = dO . O; pass 2 forms dS and dQ.
-// grid ceil(B H S / 8), 256 threads.
+// dQ, log-sum-exp and D of every query-head: D/16 consecutive lanes per query
+// (32/(D/16) queries of consecutive positions per warp), each lane holding 16
+// dimensions of q, dO and the accumulators in registers; a query's partial dot
+// products combine with xor shuffles.  Keys: the local ones [lo, t] first, then
+// the Bs keys of each valid remote block of sel.  The warp walks the largest
+// local count of its queries and every remote slot any of them holds; a key a
+// lane does not own counts with probability 0.  Pass 1 (online softmax) gives
+// the log-sum-exp and O in fp32, hence D = dO . O; pass 2 forms dS and dQ.
+// grid ceil(B H S * D/16 / 256), 256 threads.
 // ---------------------------------------------------------------------------
+constexpr int kDqE = 16;
+
+template <typename T> __device__ __forceinline__ void load16(const T *p, float *v);
+template <> __device__ __forceinline__ void load16<float>(const float *p, float *v) {
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        const float4 f = __ldg((const float4 *)p + c);
+        v[4 * c] = f.x; v[4 * c + 1] = f.y; v[4 * c + 2] = f.z; v[4 * c + 3] = f.w;
+    }
+}
+template <> __device__ __forceinline__ void load16<__nv_bfloat16>(const __nv_bfloat16 *p, float *v) {
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+        const uint4 r = __ldg((const uint4 *)p + c);
+        const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            v[8 * c + 2 * i] = __uint_as_float(w[i] << 16);
+            v[8 * c + 2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+        }
+    }
+}
+
+template <int TPQ>
+__device__ __forceinline__ float group_sum(float v) {
+#pragma unroll
+    for (int o = 1; o < TPQ; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
 template <typename T, int DD>
 __global__ void __launch_bounds__(256) k_bwd_dq(const T *__restrict__ Q, const T *__restrict__ K,
                                                 const T *__restrict__ V, const int32_t *__restrict__ sel,
                                                 const float *__restrict__ dO, float *__restrict__ dQ,
                                                 float *__restrict__ lse_out, float *__restrict__ dsum_out, int B, int H,
                                                 int S, int Bs, int L, int R, float scale) {
-    constexpr int d = DD, kPer = DD / 32, per = kPer;
-    const int lane = threadIdx.x & 31;
-    const long long w = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-    if (w >= (long long)B * H * S) return;
+    constexpr int TPQ = DD / kDqE, E = kDqE, U = 2;
+    const long long nq = (long long)B * H * S;
+    const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    const long long w0 = gid / TPQ;
+    const bool live = w0 < nq;
+    const long long w = live ? w0 : nq - 1;  // lanes past the end shadow the last query and store nothing
+    const int e0 = (int)(gid % TPQ) * E;
     const long long bh = w / S;
     const int t = (int)(w % S);
     const int b = (int)(bh / H), h = (int)(bh % H);
-    float q[kPer], g[kPer];
-    for (int e = 0; e < per; ++e) {
-        q[e] = to_f(Q[w * d + lane * per + e]);
-        g[e] = dO[(((size_t)b * S + t) * H + h) * d + lane * per + e];
-    }
-    int js[kMaxR];
-    int nr = 0;
-    for (int r = 0; r < R; ++r) {
-        const int j = sel[w * R + r];
-        if (bwd_sel_valid(j, t, Bs, L)) js[nr++] = j;
-    }
-    const int lo = max(0, t / Bs - L + 1) * Bs;
-    const int nkeys = nr * Bs + (t - lo + 1);
-    auto key_of = [&](int idx) { return idx < nr * Bs ? js[idx / Bs] * Bs + idx % Bs : lo + (idx - nr * Bs); };
     const size_t base = (size_t)bh * S;
-    // keys four at a time: their rows are loaded together and their warp sums interleave
-    constexpr int U = 4;
-    // pass 1: log-sum-exp and O
-    float m = -INFINITY, l = 0.f, o[kPer];
-    for (int e = 0; e < per; ++e) o[e] = 0.f;
-    for (int idx = 0; idx < nkeys; idx += U) {
-        float kk[U][kPer], vv[U][kPer], sc[U];
+    float q[E], g[E];
+    load16<T>(Q + w * DD + e0, q);
+    load16<float>(dO + (((size_t)b * S + t) * H + h) * DD + e0, g);
+    const int lo = max(0, t / Bs - L + 1) * Bs;
+    const int nloc = t - lo + 1;
+    int nloc_w = nloc;
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const bool in = idx + u < nkeys;
-            const size_t row = (base + key_of(in ? idx + u : idx)) * d + lane * per;
-            for (int e = 0; e < per; ++e) {
-                kk[u][e] = to_f(K[row + e]);
-                vv[u][e] = to_f(V[row + e]);
+    for (int o = 16; o > 0; o >>= 1) nloc_w = max(nloc_w, __shfl_xor_sync(0xffffffffu, nloc_w, o));
+
+    // one sweep over the query's keys; f(k row, v row, valid) per group of U keys
+    auto sweep = [&](auto &&f) {
+        for (int i = 0; i < nloc_w; i += U) {
+            const T *kr[U], *vr[U];
+            bool ok[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                ok[u] = i + u < nloc;
+                const size_t row = (base + (ok[u] ? lo + i + u : t)) * DD + e0;
+                kr[u] = K + row;
+                vr[u] = V + row;
+            }
+            f(kr, vr, ok);
+        }
+        for (int r = 0; r < R; ++r) {
+            const int j = sel[w * R + r];
+            const bool has = bwd_sel_valid(j, t, Bs, L);
+            if (!__any_sync(0xffffffffu, has)) continue;
+            for (int i = 0; i < Bs; i += U) {
+                const T *kr[U], *vr[U];
+                bool ok[U];
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    ok[u] = has && i + u < Bs;
+                    const size_t row = (base + (ok[u] ? (size_t)j * Bs + i + u : (size_t)t)) * DD + e0;
+                    kr[u] = K + row;
+                    vr[u] = V + row;
+                }
+                f(kr, vr, ok);
             }
         }
+    };
+
+    // pass 1: log-sum-exp and O (the first group holds key lo of every query: m is finite after it)
+    float m = -INFINITY, l = 0.f, o[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) o[e] = 0.f;
+    sweep([&](const T *const *kr, const T *const *vr, const bool *ok) {
+        float kk[U][E], sc[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) load16<T>(kr[u], kk[u]);
 #pragma unroll
         for (int u = 0; u < U; ++u) {
             float part = 0.f;
-            for (int e = 0; e < per; ++e) part = fmaf(q[e], kk[u][e], part);
-            sc[u] = bwd_warp_sum(part) * scale;
+#pragma unroll
+            for (int e = 0; e < E; ++e) part = fmaf(q[e], kk[u][e], part);
+            sc[u] = group_sum<TPQ>(part) * scale;
         }
         float mx = m;
 #pragma unroll
         for (int u = 0; u < U; ++u)
-            if (idx + u < nkeys) mx = fmaxf(mx, sc[u]);
+            if (ok[u]) mx = fmaxf(mx, sc[u]);
         const float corr = expf(m - mx);
         l *= corr;
-        for (int e = 0; e < per; ++e) o[e] *= corr;
+#pragma unroll
+        for (int e = 0; e < E; ++e) o[e] *= corr;
+        m = mx;
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-            if (idx + u >= nkeys) continue;
-            const float p = expf(sc[u] - mx);
+            const float p = ok[u] ? expf(sc[u] - mx) : 0.f;
+            float vv[E];
+            load16<T>(vr[u], vv);
             l += p;
-            for (int e = 0; e < per; ++e) o[e] = fmaf(p, vv[u][e], o[e]);
+#pragma unroll
+            for (int e = 0; e < E; ++e) o[e] = fmaf(p, vv[e], o[e]);
         }
-        m = mx;
-    }
+    });
     const float lse = m + logf(l);
     float dpart = 0.f;
-    for (int e = 0; e < per; ++e) dpart = fmaf(g[e], o[e] / l, dpart);
-    const float D = bwd_warp_sum(dpart);
+#pragma unroll
+    for (int e = 0; e < E; ++e) dpart = fmaf(g[e], o[e] / l, dpart);
+    const float D = group_sum<TPQ>(dpart);
+
     // pass 2: dS and dQ
-    float dq[kPer];
-    for (int e = 0; e < per; ++e) dq[e] = 0.f;
-    for (int idx = 0; idx < nkeys; idx += U) {
-        float kk[U][kPer], sp[U], dp[U];
+    float dq[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) dq[e] = 0.f;
+    sweep([&](const T *const *kr, const T *const *vr, const bool *ok) {
+        float kk[U][E], sp[U], dp[U];
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-            const bool in = idx + u < nkeys;
-            const size_t row = (base + key_of(in ? idx + u : idx)) * d + lane * per;
+            float vv[E];
+            load16<T>(kr[u], kk[u]);
+            load16<T>(vr[u], vv);
             float a = 0.f, c = 0.f;
-            for (int e = 0; e < per; ++e) {
-                kk[u][e] = to_f(K[row + e]);
+#pragma unroll
+            for (int e = 0; e < E; ++e) {
                 a = fmaf(q[e], kk[u][e], a);
-                c = fmaf(g[e], to_f(V[row + e]), c);
+                c = fmaf(g[e], vv[e], c);
             }
             sp[u] = a;
             dp[u] = c;
         }
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-            sp[u] = bwd_warp_sum(sp[u]);
-            dp[u] = bwd_warp_sum(dp[u]);
+            sp[u] = group_sum<TPQ>(sp[u]);
+            dp[u] = group_sum<TPQ>(dp[u]);
         }
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-            if (idx + u >= nkeys) continue;
-            const float ds = expf(sp[u] * scale - lse) * (dp[u] - D);
-            for (int e = 0; e < per; ++e) dq[e] = fmaf(ds, kk[u][e], dq[e]);
+            const float ds = ok[u] ? expf(sp[u] * scale - lse) * (dp[u] - D) : 0.f;
+#pragma unroll
+            for (int e = 0; e < E; ++e) dq[e] = fmaf(ds, kk[u][e], dq[e]);
         }
-    }
-    for (int e = 0; e < per; ++e) dQ[w * d + lane * per + e] = dq[e] * scale;
-    if (lane == 0) {
-        lse_out[w] = lse;
-        dsum_out[w] = D;
+    });
+    if (live) {
+        float4 *dst = (float4 *)(dQ + w * DD + e0);
+#pragma unroll
+        for (int c = 0; c < E / 4; ++c)
+            dst[c] = make_float4(dq[4 * c] * scale, dq[4 * c + 1] * scale, dq[4 * c + 2] * scale, dq[4 * c + 3] * scale);
+        if (e0 == 0) {
+            lse_out[w] = lse;
+            dsum_out[w] = D;
+        }
     }
 }
 
@@ -254,25 +328,28 @@ __global__ void __launch_bounds__(256) k_bwd_fill(const int32_t *__restrict__ se
 // per key, each holding 16 dimensions of the key's K and V rows and of its dK
 // and dV accumulators in registers; a key's threads are consecutive lanes and
 // combine their partial dot products with xor shuffles.  Queries come in
-// groups of 8 (q, dO, log-sum-exp and D staged in shared memory, read as
-// broadcast float4): first the local ones (blocks j .. j+L-1; in block j
-// itself only keys s <= t, applied as a zero probability so that every lane
-// takes part in the shuffles), then those whose selection holds block j.
+// groups of 16 (q, dO, log-sum-exp and D staged in shared memory, read as
+// broadcast float4; the next group's rows are fetched into registers while
+// the current one is computed, double-buffered): first the local ones (blocks
+// j .. j+L-1; in block j itself only keys s <= t, applied as a zero
+// probability so that every lane takes part in the shuffles), then those
+// whose selection holds block j.
 // grid (ceil(Bs/64) * nb, H, B), 64 * D/16 threads.
 // ---------------------------------------------------------------------------
-constexpr int kBwdKT = 64, kBwdQG = 8;
+constexpr int kBwdKT = 64, kBwdQG = 16;
 
 template <typename T, int DD>
-__global__ void __launch_bounds__(kBwdKT * DD / 16) k_bwd_dkdv(
+__global__ void __launch_bounds__(kBwdKT * DD / 16, DD == 64 ? 2 : 1) k_bwd_dkdv(
     const T *__restrict__ Q, const T *__restrict__ K, const T *__restrict__ V, const float *__restrict__ dO,
     const float *__restrict__ lse, const float *__restrict__ dsum, const int32_t *__restrict__ cnt,
     const int32_t *__restrict__ start, const int32_t *__restrict__ list, float *__restrict__ dK,
     float *__restrict__ dV, int H, int S, int Bs, int L, int R, int nb, float scale) {
     constexpr int TPK = DD / 16, NT = kBwdKT * TPK, E = 16;
-    __shared__ __align__(16) float sq[kBwdQG][DD];
-    __shared__ __align__(16) float sg[kBwdQG][DD];
-    __shared__ float slse[kBwdQG], sD[kBwdQG];
-    __shared__ int st[kBwdQG];
+    constexpr int PER = kBwdQG * DD / NT;  // staged elements per thread and array (one dimension, PER queries)
+    __shared__ __align__(16) float sq[2][kBwdQG][DD];
+    __shared__ __align__(16) float sg[2][kBwdQG][DD];
+    __shared__ float slse[2][kBwdQG], sD[2][kBwdQG];
+    __shared__ int st[2][kBwdQG];
     const int tpb = (Bs + kBwdKT - 1) / kBwdKT;
     const int j = blockIdx.x / tpb, u = blockIdx.x % tpb;
     const int h = blockIdx.y, b = blockIdx.z;
@@ -296,24 +373,50 @@ __global__ void __launch_bounds__(kBwdKT * DD / 16) k_bwd_dkdv(
     const int nrem = R > 0 ? cnt[bh * nb + j] : 0;
     const int rem0 = R > 0 ? start[bh * nb + j] : 0;
     const int nq = nloc + nrem;
-    for (int g0 = 0; g0 < nq; g0 += kBwdQG) {
-        const int ng = min(kBwdQG, nq - g0);
-        __syncthreads();  // the previous group is used up
-        for (int i = tid; i < ng * DD; i += NT) {
-            const int qi = i / DD, e = i % DD;
-            const int n = g0 + qi;
-            const int t = n < nloc ? t_loc0 + n : list[bh * S * R + rem0 + (n - nloc)];
-            sq[qi][e] = to_f(Q[(bh * S + t) * DD + e]);
-            sg[qi][e] = dO[(((size_t)b * S + t) * H + h) * DD + e];
-            if (e == 0) {
-                st[qi] = t;
-                slse[qi] = lse[bh * S + t];
-                sD[qi] = dsum[bh * S + t];
+    // thread tid stages dimension fe of queries fq0, fq0 + NT/DD, ... of a group
+    const int fe = tid % DD, fq0 = tid / DD;
+    float rq[PER], rg[PER], rl[PER], rd[PER];
+    int rt[PER];
+    auto fetch = [&](int g0) {
+#pragma unroll
+        for (int k = 0; k < PER; ++k) {
+            const int n = g0 + fq0 + k * (NT / DD);
+            const bool in = n < nq;
+            const int t = !in ? 0 : n < nloc ? t_loc0 + n : list[bh * S * R + rem0 + (n - nloc)];
+            rt[k] = t;
+            rq[k] = in ? to_f(Q[(bh * S + t) * DD + fe]) : 0.f;
+            rg[k] = in ? dO[(((size_t)b * S + t) * H + h) * DD + fe] : 0.f;
+            if (fe == 0) {
+                rl[k] = in ? lse[bh * S + t] : 0.f;
+                rd[k] = in ? dsum[bh * S + t] : 0.f;
             }
         }
-        __syncthreads();
+    };
+    auto stash = [&](int buf) {
+#pragma unroll
+        for (int k = 0; k < PER; ++k) {
+            const int qi = fq0 + k * (NT / DD);
+            sq[buf][qi][fe] = rq[k];
+            sg[buf][qi][fe] = rg[k];
+            if (fe == 0) {
+                st[buf][qi] = rt[k];
+                slse[buf][qi] = rl[k];
+                sD[buf][qi] = rd[k];
+            }
+        }
+    };
+    if (nq > 0) {
+        fetch(0);
+        stash(0);
+    }
+    __syncthreads();
+    int buf = 0;
+    for (int g0 = 0; g0 < nq; g0 += kBwdQG, buf ^= 1) {
+        const int ng = min(kBwdQG, nq - g0);
+        const bool more = g0 + kBwdQG < nq;
+        if (more) fetch(g0 + kBwdQG);  // in flight while this group is computed
         for (int qi = 0; qi < ng; ++qi) {
-            const float4 *q4 = (const float4 *)&sq[qi][e0], *g4 = (const float4 *)&sg[qi][e0];
+            const float4 *q4 = (const float4 *)&sq[buf][qi][e0], *g4 = (const float4 *)&sg[buf][qi][e0];
             float qv[E], gv[E];
 #pragma unroll
             for (int c = 0; c < E / 4; ++c) {
@@ -332,15 +435,17 @@ __global__ void __launch_bounds__(kBwdKT * DD / 16) k_bwd_dkdv(
                 sp += __shfl_xor_sync(0xffffffffu, sp, o);
                 dp += __shfl_xor_sync(0xffffffffu, dp, o);
             }
-            const bool masked = !live || (g0 + qi < nloc && key > st[qi]);  // causal inside the query's own block
-            const float p = masked ? 0.f : expf(sp * scale - slse[qi]);
-            const float ds = p * (dp - sD[qi]) * scale;
+            const bool masked = !live || (g0 + qi < nloc && key > st[buf][qi]);  // causal in the query's own block
+            const float p = masked ? 0.f : expf(sp * scale - slse[buf][qi]);
+            const float ds = p * (dp - sD[buf][qi]) * scale;
 #pragma unroll
             for (int e = 0; e < E; ++e) {
                 dv[e] = fmaf(p, gv[e], dv[e]);
                 dk[e] = fmaf(ds, qv[e], dk[e]);
             }
         }
+        if (more) stash(buf ^ 1);  // every thread finished reading buf ^ 1 before the last barrier
+        __syncthreads();
     }
     if (live) {
 #pragma unroll
@@ -354,11 +459,22 @@ __global__ void __launch_bounds__(kBwdKT * DD / 16) k_bwd_dkdv(
 // ---------------------------------------------------------------------------
 // gradients before RoPE, token-major: dQ and dK (post-RoPE, [B,H,S,d]) rotated
 // back by -t*theta^(-2i/d) (the transpose of the forward rotation), dV copied;
-// outputs [B*S, H*d].  One thread per (b, t, h, pair i); grid ceil(B S H d/2 / 256).
+// outputs [B*S, H*d] in fp32 or, for the tensor-core GEMMs, as two bf16 terms
+// hi = bf16(v), lo = bf16(v - hi) at out and out + B*S*H*d (their sum carries
+// 16 significant bits).  One thread per (b, t, h, pair i);
+// grid ceil(B S H d/2 / 256).
 // ---------------------------------------------------------------------------
+__device__ __forceinline__ void put_grad(float *out, size_t i, size_t, float v) { out[i] = v; }
+__device__ __forceinline__ void put_grad(__nv_bfloat16 *out, size_t i, size_t n, float v) {
+    const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+    out[i] = hi;
+    out[n + i] = __float2bfloat16_rn(v - __bfloat162float(hi));
+}
+
+template <typename TO>
 __global__ void __launch_bounds__(256) k_bwd_rope(const float *__restrict__ dQ, const float *__restrict__ dK,
-                                                  const float *__restrict__ dV, float *__restrict__ dQp,
-                                                  float *__restrict__ dKp, float *__restrict__ dVp, int B, int S, int H,
+                                                  const float *__restrict__ dV, TO *__restrict__ dQp,
+                                                  TO *__restrict__ dKp, TO *__restrict__ dVp, int B, int S, int H,
                                                   int d, double theta) {
     const long long n = (long long)B * S * H * (d / 2);
     const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
@@ -372,12 +488,13 @@ __global__ void __launch_bounds__(256) k_bwd_rope(const float *__restrict__ dQ, 
     const size_t src = (((size_t)b * H + h) * S + t) * d + 2 * pr;
     const size_t dst = ((size_t)bt * H + h) * d + 2 * pr;
     const float q0 = dQ[src], q1 = dQ[src + 1], k0 = dK[src], k1 = dK[src + 1];
-    dQp[dst] = q0 * c + q1 * s;
-    dQp[dst + 1] = -q0 * s + q1 * c;
-    dKp[dst] = k0 * c + k1 * s;
-    dKp[dst + 1] = -k0 * s + k1 * c;
-    dVp[dst] = dV[src];
-    dVp[dst + 1] = dV[src + 1];
+    const size_t nn = (size_t)n * 2;
+    put_grad(dQp, dst, nn, q0 * c + q1 * s);
+    put_grad(dQp, dst + 1, nn, -q0 * s + q1 * c);
+    put_grad(dKp, dst, nn, k0 * c + k1 * s);
+    put_grad(dKp, dst + 1, nn, -k0 * s + k1 * c);
+    put_grad(dVp, dst, nn, dV[src]);
+    put_grad(dVp, dst + 1, nn, dV[src + 1]);
 }
 
 // ---------------------------------------------------------------------------
@@ -474,12 +591,12 @@ cudaError_t attend_backward(const Plan &p, const T *Q, const T *K, const T *V, c
     const float scale = (float)(1.0 / sqrt((double)c.d));
     const long long nq = (long long)c.B * c.H * c.S;
     cudaError_t e;
+    const int tpq = c.d / kDqE;
+    const unsigned gq = (unsigned)((nq * tpq + 255) / 256);
     if (c.d == 64)
-        k_bwd_dq<T, 64><<<(unsigned)((nq + 7) / 8), 256, 0, s>>>(Q, K, V, sel, dO, dQ, lse, dsum, c.B, c.H, c.S,
-                                                                 c.Bs, c.L, c.R, scale);
+        k_bwd_dq<T, 64><<<gq, 256, 0, s>>>(Q, K, V, sel, dO, dQ, lse, dsum, c.B, c.H, c.S, c.Bs, c.L, c.R, scale);
     else
-        k_bwd_dq<T, 128><<<(unsigned)((nq + 7) / 8), 256, 0, s>>>(Q, K, V, sel, dO, dQ, lse, dsum, c.B, c.H, c.S,
-                                                                  c.Bs, c.L, c.R, scale);
+        k_bwd_dq<T, 128><<<gq, 256, 0, s>>>(Q, K, V, sel, dO, dQ, lse, dsum, c.B, c.H, c.S, c.Bs, c.L, c.R, scale);
     count_launches(1);
     if (c.R > 0) {
         const long long n = nq * c.R;
@@ -501,24 +618,59 @@ cudaError_t attend_backward(const Plan &p, const T *Q, const T *K, const T *V, c
     return cudaGetLastError();
 }
 
+// The projection gradients on the tensor cores (bf16 storage): the operands are
+// the stored bf16 activations and weights, the upstream gradient ddelta (all
+// exact in bf16) and the fp32 gradients before the projections, dQp, dKp, dVp,
+// each as its two-term bf16 split hi + lo (in its own workspace region), so the
+// products are those of fp32 operands to 16 significant bits; accumulation and
+// outputs fp32.
+bool grads_tc_supported(const mono_config &c) {
+    const int BS = c.B * c.S, Hd = c.H * c.d, W = c.W;
+    return c.dtype == MONO_BF16 && gemm_grad_tc_supported(BS, Hd, W, false, true) &&
+           gemm_grad_tc_supported(W, Hd, BS, true, true) && gemm_grad_tc_supported(Hd, W, BS, true, true) &&
+           gemm_grad_tc_supported(BS, W, Hd, false, true);
+}
+
 template <typename T>
 cudaError_t backward_t(const Plan &p, const T *x, const T *Wq, const T *Wk, const T *Wv, const T *Wo,
                        const int32_t *sel, const T *ddelta, float *dx, float *dWq, float *dWk, float *dWv, float *dWo,
-                       const T *Q, const T *K, const T *V, const T *O, char *bws, cudaStream_t s) {
+                       const T *Q, const T *K, const T *V, const T *O, char *bws, unsigned long long *counters,
+                       cudaStream_t s) {
     const mono_config &c = p.cfg;
     const BwdLayout L = bwd_layout(p);
     float *dO = (float *)(bws + L.dO), *dQ = (float *)(bws + L.dQ), *dK = (float *)(bws + L.dK);
-    float *dV = (float *)(bws + L.dV), *dQp = (float *)(bws + L.dQp), *dKp = (float *)(bws + L.dKp);
-    float *dVp = (float *)(bws + L.dVp);
+    float *dV = (float *)(bws + L.dV);
     const int BS = c.B * c.S, Hd = c.H * c.d, W = c.W;
+    const bool tc = grads_tc_supported(c);
+    const long long npairs = (long long)BS * Hd / 2;
+    const unsigned rope_grid = (unsigned)((npairs + 255) / 256);
     cudaError_t e;
+    if (tc) {
+        // delta = O Wo^T:  dO = ddelta Wo (Wo MN-major),  dWo = ddelta^T O (both MN-major)
+        const void *a0[1] = {ddelta}, *b0[1] = {Wo}, *b1[1] = {O};
+        float *c0[1] = {dO}, *c1[1] = {dWo};
+        if ((e = gemm_grad_tc(BS, Hd, W, 1, 1, a0, false, b0, true, c0, false, counters, s)) != cudaSuccess) return e;
+        if ((e = gemm_grad_tc(W, Hd, BS, 1, 1, a0, true, b1, true, c1, false, counters, s)) != cudaSuccess) return e;
+        if ((e = attend_backward<T>(p, Q, K, V, sel, dO, dQ, dK, dV, bws, s)) != cudaSuccess) return e;
+        using B16 = __nv_bfloat16;
+        B16 *hq = (B16 *)(bws + L.dQp), *hk = (B16 *)(bws + L.dKp), *hv = (B16 *)(bws + L.dVp);
+        k_bwd_rope<B16><<<rope_grid, 256, 0, s>>>(dQ, dK, dV, hq, hk, hv, c.B, c.S, c.H, c.d, c.rope_theta);
+        count_launches(1);
+        // q = x Wq^T (per head, then RoPE):  dWq = dQp^T x (both MN-major),  dx = dQp Wq + dKp Wk + dVp Wv,
+        // each dZp as hi + lo
+        const size_t n = (size_t)BS * Hd;
+        const void *ah[6] = {hq, hq + n, hk, hk + n, hv, hv + n};
+        const void *xs[6] = {x, x, x, x, x, x}, *ws[6] = {Wq, Wq, Wk, Wk, Wv, Wv};
+        float *cw[3] = {dWq, dWk, dWv}, *cx[1] = {dx};
+        if ((e = gemm_grad_tc(Hd, W, BS, 2, 3, ah, true, xs, true, cw, false, counters, s)) != cudaSuccess) return e;
+        return gemm_grad_tc(BS, W, Hd, 6, 1, ah, false, ws, true, cx, false, counters, s);
+    }
+    float *dQp = (float *)(bws + L.dQp), *dKp = (float *)(bws + L.dKp), *dVp = (float *)(bws + L.dVp);
     // delta = O Wo^T:  dO = ddelta Wo,  dWo = ddelta^T O
     if ((e = gemm_any<T, T>(BS, Hd, W, ddelta, W, 1, Wo, Hd, 1, dO, Hd, 0.f, s)) != cudaSuccess) return e;
     if ((e = gemm_any<T, T>(W, Hd, BS, ddelta, 1, W, O, Hd, 1, dWo, Hd, 0.f, s)) != cudaSuccess) return e;
     if ((e = attend_backward<T>(p, Q, K, V, sel, dO, dQ, dK, dV, bws, s)) != cudaSuccess) return e;
-    const long long npairs = (long long)BS * Hd / 2;
-    k_bwd_rope<<<(unsigned)((npairs + 255) / 256), 256, 0, s>>>(dQ, dK, dV, dQp, dKp, dVp, c.B, c.S, c.H, c.d,
-                                                                c.rope_theta);
+    k_bwd_rope<float><<<rope_grid, 256, 0, s>>>(dQ, dK, dV, dQp, dKp, dVp, c.B, c.S, c.H, c.d, c.rope_theta);
     count_launches(1);
     // q = x Wq^T (per head, then RoPE):  dWq = dQp^T x,  dx = dQp Wq + dKp Wk + dVp Wv
     if ((e = gemm_any<float, T>(Hd, W, BS, dQp, 1, Hd, x, W, 1, dWq, W, 0.f, s)) != cudaSuccess) return e;
@@ -591,16 +743,18 @@ int mono_backward(const mono_plan_t *plan, const void *x, const void *Wq, const 
     if ((st = mono_attend(plan, Q, K, V, sel, O, workspace, stream))) return st;
     cudaStream_t s = (cudaStream_t)stream;
     char *bws = (char *)bwd_workspace;
+    unsigned long long *counters = (unsigned long long *)ws_ptr(p, workspace, kRegCounters);
     if (c.dtype == MONO_BF16) {
         using B16 = __nv_bfloat16;
         return bwd_status(backward_t<B16>(p, (const B16 *)x, (const B16 *)Wq, (const B16 *)Wk, (const B16 *)Wv,
                                           (const B16 *)Wo, sel, (const B16 *)ddelta, dx, dWq, dWk, dWv, dWo,
-                                          (const B16 *)Q, (const B16 *)K, (const B16 *)V, (const B16 *)O, bws, s));
+                                          (const B16 *)Q, (const B16 *)K, (const B16 *)V, (const B16 *)O, bws, counters,
+                                          s));
     }
     return bwd_status(backward_t<float>(p, (const float *)x, (const float *)Wq, (const float *)Wk, (const float *)Wv,
                                         (const float *)Wo, sel, (const float *)ddelta, dx, dWq, dWk, dWv, dWo,
                                         (const float *)Q, (const float *)K, (const float *)V, (const float *)O, bws,
-                                        s));
+                                        counters, s));
 }
 
 }  // extern "C"

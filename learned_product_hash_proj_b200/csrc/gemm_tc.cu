@@ -265,4 +265,212 @@ cudaError_t launch_out_project_tc(const Plan &p, const void *O, const void *Wo, 
     return launch(maps, epi, 1, Kd, s);
 }
 
+// ---------------------------------------------------------------------------
+// The gradient GEMMs on the tensor cores: C_g[M,N] (fp32, row-major) (+)=
+// sum_src A_src(m,k) B_src(n,k) over bf16 operands, each stored K-major
+// ([M or N rows][K], a row contiguous in k) or MN-major ([K rows][M or N], a
+// row contiguous in m or n).  ngroups independent outputs (dWq, dWk, dWv),
+// each the sum of nsrc products over the same K (dx = dQp Wq + dKp Wk + dVp Wv;
+// an fp32 operand given as the two bf16 terms of its hi + lo split); the k
+// slices are split over blockIdx.z, partial sums added with fp32 atomics.  Same roles as k_gemm_tc; an MN-major tile is two 64-wide column
+// blocks of 64 K-rows each (128-byte swizzle), 8 KB apart.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr int kGradMaxOps = 6;
+
+struct GradMaps {
+    CUtensorMap a[kGradMaxOps];  // group-major: operand pair g * nsrc + src
+    CUtensorMap b[kGradMaxOps];
+};
+
+struct GradArgs {
+    float *out[3];
+    int M, N, K;     // of each product
+    int nsrc;        // products summed into each output
+    int ngroups;     // outputs
+    int split;       // k-slice ranges per output tile (blockIdx.z % split)
+    int a_mn, b_mn;  // operand major-ness
+    int atomic;      // add into C instead of storing
+    unsigned long long *counters;
+};
+
+__device__ __forceinline__ void load_operand(uint8_t *dst, const CUtensorMap *map, bool mn, int mn0, int k0,
+                                             uint64_t *bar) {
+    if (mn) {
+        tma_load_2d(dst, map, mn0, k0, bar);
+        tma_load_2d(dst + A_BYTES / 2, map, mn0 + 64, k0, bar);
+    } else {
+        tma_load_2d(dst, map, k0, mn0, bar);
+    }
+}
+
+__device__ __forceinline__ uint64_t operand_desc(uint32_t saddr, bool mn, int kk) {
+    return mn ? tc::desc_sw128_mn(saddr + 2048 * kk, A_BYTES / 2) : desc_sw128(saddr + 32 * kk);
+}
+
+__global__ void __launch_bounds__(192, 2) k_gemm_grad_tc(const __grid_constant__ GradMaps maps, const GradArgs g) {
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ uint64_t full[STAGES], empty[STAGES], accf;
+    __shared__ uint32_t tmem_base;
+    __shared__ int fail;
+    uint8_t *base = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int grp = blockIdx.z / g.split, part = blockIdx.z % g.split;
+    const int m0 = blockIdx.y * BM, n0 = blockIdx.x * BN;
+    const int kslices = (g.K + BK - 1) / BK;
+    const int total = kslices * g.nsrc;
+    const int per = (total + g.split - 1) / g.split;
+    const int kb = part * per;
+    const int nk = max(0, min(total, kb + per) - kb);
+    if (tid == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            tc::mbar_init(&full[s], 1);
+            tc::mbar_init(&empty[s], 1);
+        }
+        tc::mbar_init(&accf, 1);
+        tc::fence_mbar_init();
+        fail = 0;
+    }
+    if (warp == 1) {
+        tc::tmem_alloc(&tmem_base, BN);
+        tc::tmem_relinquish();
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = tmem_base;
+    const bool amn = g.a_mn != 0, bmn = g.b_mn != 0;
+
+    if (warp == 0 && lane == 0) {
+        for (int i = 0; i < nk; ++i) {
+            const int s = i % STAGES;
+            const uint32_t ph = (i / STAGES) & 1;
+            if (i >= STAGES && !tc::mbar_wait(&empty[s], ph ^ 1)) { fail = 1; break; }
+            const int sl = kb + i;
+            const int src = grp * g.nsrc + sl / kslices;
+            const int k0 = (sl % kslices) * BK;
+            uint8_t *sa = base + s * A_BYTES;
+            uint8_t *sb = base + STAGES * A_BYTES + s * B_BYTES;
+            mbar_expect_tx(&full[s], A_BYTES + B_BYTES);
+            load_operand(sa, &maps.a[src], amn, m0, k0, &full[s]);
+            load_operand(sb, &maps.b[src], bmn, n0, k0, &full[s]);
+        }
+    } else if (warp == 1 && lane == 0) {
+        const uint32_t id = tc::idesc_bf16(BM, BN, bmn, amn);
+        bool ok = true;
+        for (int i = 0; i < nk; ++i) {
+            const int s = i % STAGES;
+            const uint32_t ph = (i / STAGES) & 1;
+            if (!tc::mbar_wait(&full[s], ph)) { ok = false; fail = 1; break; }
+            tc::fence_after_sync();
+            const uint32_t sa = tc::smem_u32(base + s * A_BYTES);
+            const uint32_t sb = tc::smem_u32(base + STAGES * A_BYTES + s * B_BYTES);
+#pragma unroll
+            for (int kk = 0; kk < BK / 16; ++kk)
+                tc::mma_bf16(tmem, operand_desc(sa, amn, kk), operand_desc(sb, bmn, kk), id, (i | kk) != 0);
+            tc::commit(&empty[s]);
+        }
+        if (ok && nk > 0) tc::commit(&accf);
+    } else if (warp >= 2) {
+        // warp w reads TMEM lanes 32*(w%4) .. +31 = tile rows
+        const int q = warp & 3;
+        const int m = m0 + q * 32 + lane;
+        const bool ok = nk > 0 && tc::mbar_wait(&accf, 0, 1u << 20);
+        tc::fence_after_sync();
+        const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16);
+        float *out = g.out[grp];
+        for (int c0 = 0; c0 < BN; c0 += 32) {
+            float v[32];
+            tc::tmem_ld32(trow + c0, v);
+            if (!ok || m >= g.M) continue;
+            const int n = n0 + c0;
+            float *dst = out + (size_t)m * g.N + n;
+            if (n + 32 <= g.N) {
+#pragma unroll
+                for (int c4 = 0; c4 < 8; ++c4) {
+                    const float4 f = make_float4(v[4 * c4], v[4 * c4 + 1], v[4 * c4 + 2], v[4 * c4 + 3]);
+                    if (g.atomic) atomicAdd((float4 *)dst + c4, f);
+                    else ((float4 *)dst)[c4] = f;
+                }
+            } else {
+#pragma unroll
+                for (int c = 0; c < 32; ++c) {
+                    if (n + c >= g.N) break;
+                    if (g.atomic) atomicAdd(dst + c, v[c]);
+                    else dst[c] = v[c];
+                }
+            }
+        }
+        if (nk > 0 && !ok && lane == 0) fail = 1;
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    if (tid == 0 && fail) record_error(g.counters, kDevErrTimeout);
+    if (warp == 1) tc::tmem_dealloc(tmem, BN);
+}
+
+}  // namespace
+
+bool gemm_grad_tc_supported(int M, int N, int K, bool a_mn, bool b_mn) {
+    // TMA row strides are multiples of 16 bytes; fp32 rows of C hold whole float4s
+    return M > 0 && N > 0 && K > 0 && (a_mn ? M % 8 : K % 8) == 0 && (b_mn ? N % 8 : K % 8) == 0 && N % 4 == 0 &&
+           tensor_map_encoder() != nullptr;
+}
+
+cudaError_t gemm_grad_tc(int M, int N, int K, int nsrc, int ngroups, const void *const *A, bool a_mn,
+                         const void *const *B, bool b_mn, float *const *C, bool accumulate,
+                         unsigned long long *counters, cudaStream_t s) {
+    if (M == 0 || N == 0) return cudaSuccess;
+    if (nsrc < 1 || ngroups < 1 || ngroups > 3 || nsrc * ngroups > kGradMaxOps) return cudaErrorInvalidValue;
+    if (!gemm_grad_tc_supported(M, N, K, a_mn, b_mn) || !get_encode()) return cudaErrorNotSupported;
+    GradMaps maps;
+    const int nmaps = nsrc * ngroups;
+    for (int i = 0; i < nmaps; ++i) {
+        // K-major: [MN rows][K], box 64 x 128; MN-major: [K rows][MN], box 64 x 64 (two per tile)
+        const bool ok_a = a_mn ? make_map(&maps.a[i], A[i], K, M, 64) : make_map(&maps.a[i], A[i], M, K, BM);
+        const bool ok_b = b_mn ? make_map(&maps.b[i], B[i], K, N, 64) : make_map(&maps.b[i], B[i], N, K, BN);
+        if (!ok_a || !ok_b) return cudaErrorInvalidValue;
+    }
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int slots = 2 * sms;
+    const int tiles = ((N + BN - 1) / BN) * ((M + BM - 1) / BM) * ngroups;
+    const int total = ((K + BK - 1) / BK) * nsrc;
+    // split K where the tiles alone fill the GPU's CTA slots poorly: the split with the best last-wave fill
+    int split = 1;
+    double best = 0.0;
+    for (int sp = 1; sp <= 16 && total / sp >= 4; ++sp) {
+        const long long ctas = (long long)tiles * sp;
+        const double fill = (double)ctas / (double)(((ctas + slots - 1) / slots) * slots);
+        if (fill > best + 1e-9) {
+            best = fill;
+            split = sp;
+        }
+    }
+    const int per = (total + split - 1) / split;
+    split = (total + per - 1) / per;  // every k range non-empty
+    GradArgs g{};
+    for (int i = 0; i < 3; ++i) g.out[i] = C[i < ngroups ? i : 0];
+    g.M = M; g.N = N; g.K = K; g.nsrc = nsrc; g.ngroups = ngroups; g.split = split;
+    g.a_mn = a_mn; g.b_mn = b_mn;
+    g.atomic = split > 1 || accumulate;
+    g.counters = counters;
+    cudaError_t e;
+    if (split > 1 && !accumulate)
+        for (int i = 0; i < ngroups; ++i)
+            if ((e = cudaMemsetAsync(C[i], 0, (size_t)M * N * sizeof(float), s)) != cudaSuccess) return e;
+    static bool attr_set = false;
+    if (!attr_set) {
+        if ((e = cudaFuncSetAttribute(k_gemm_grad_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES)) !=
+            cudaSuccess)
+            return e;
+        attr_set = true;
+    }
+    dim3 grid((N + BN - 1) / BN, (M + BM - 1) / BM, ngroups * split);
+    k_gemm_grad_tc<<<grid, 192, SMEM_BYTES, s>>>(maps, g);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
 }  // namespace mono

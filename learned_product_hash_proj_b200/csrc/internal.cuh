@@ -106,6 +106,13 @@ bool gemm_tc_supported(const mono_config &c);
 cudaError_t launch_project_tc(const Plan &p, const void *x, const void *Wq, const void *Wk, const void *Wv, void *Q,
                               void *K, void *V, const void *ws, cudaStream_t s);
 cudaError_t launch_out_project_tc(const Plan &p, const void *O, const void *Wo, void *delta, void *ws, cudaStream_t s);
+// C_g[M,N] (fp32) (+)= sum_{src < nsrc} A_{g,src}(m,k) B_{g,src}(n,k) for g < ngroups (<= 3, nsrc * ngroups
+// <= 6; A and B hold the operands group-major), bf16 operands on the tensor cores; an operand is K-major
+// ([M|N rows][K]) or MN-major ([K rows][M|N]).  Pointers 16-byte aligned; row lengths multiples of 8 (supported() checks).
+bool gemm_grad_tc_supported(int M, int N, int K, bool a_mn, bool b_mn);
+cudaError_t gemm_grad_tc(int M, int N, int K, int nsrc, int ngroups, const void *const *A, bool a_mn,
+                         const void *const *B, bool b_mn, float *const *C, bool accumulate,
+                         unsigned long long *counters, cudaStream_t s);
 cudaError_t launch_attend_tc(const Plan &p, const void *Q, const void *K, const void *V, const int32_t *sel, void *O,
                              void *ws, cudaStream_t s);
 

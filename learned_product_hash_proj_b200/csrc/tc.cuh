@@ -63,12 +63,13 @@ __device__ __forceinline__ uint32_t mnmajor_chunk(int k, int c, int nk) {
     return (uint32_t)(c * (nk * 16) + (k >> 3) * 128 + (k & 7) * 16);
 }
 
-// instruction descriptor: kind::f16, A = B = bf16, D = f32, M x N; A K-major;
-// B K-major (b_mn = false) or MN-major (b_mn = true).
-__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool b_mn = false) {
+// instruction descriptor: kind::f16, A = B = bf16, D = f32, M x N; A and B
+// each K-major (false) or MN-major (true).
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool b_mn = false, bool a_mn = false) {
     return (1u << 4)                    // D format f32
            | (1u << 7)                  // A format bf16
            | (1u << 10)                 // B format bf16
+           | ((a_mn ? 1u : 0u) << 15)   // A major-ness
            | ((b_mn ? 1u : 0u) << 16)   // B major-ness
            | ((uint32_t)(N >> 3) << 17) //
            | ((uint32_t)(M >> 4) << 24);

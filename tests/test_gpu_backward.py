@@ -9,8 +9,11 @@
   max |err| <= 1e-4 x RMS(ref) for fp32.  For bf16 the forward attention forms
   O with bf16 probabilities on the tensor cores, which is what the batch
   tolerance for O (2e-2 x RMS) covers, and dWo = ddelta^T O inherits it: the
-  bf16 bound is that same 2e-2 x RMS (measured: dx, dWq, dWk, dWv within
-  2e-3 x RMS, dWo 2.4e-3 x RMS).
+  bf16 bound is that same 2e-2 x RMS.  The bf16 projection gradients run on
+  the tensor cores with the fp32 gradients before the projections split into
+  two bf16 terms (16 significant bits).  Rounding them to one bf16 term would
+  alone cost up to 2.2e-2 x RMS in dx at these sizes (a float64 emulation of
+  that rounding), which is why they are split.
 """
 import numpy as np
 import pytest
@@ -70,9 +73,18 @@ def test_attend_backward_matches_oracle(name):
         close(to_np(got), ref, 2e-4, f"attention {nm}")
 
 
-@pytest.mark.parametrize("dtype", ["f32", "bf16"])
-def test_backward_matches_oracle(dtype):
-    cfg = small(dtype=dtype)
+FULL_CASES = {
+    "f32": dict(),
+    "bf16": dict(dtype="bf16"),
+    # widths off the 128-wide tensor-core tiles: ragged tiles in every gradient GEMM, split K in dWq/dWk/dWv
+    "bf16_ragged": dict(dtype="bf16", S=320, W=192, H=3),
+}
+
+
+@pytest.mark.parametrize("name", list(FULL_CASES))
+def test_backward_matches_oracle(name):
+    cfg = small(**FULL_CASES[name])
+    dtype = cfg.dtype
     run = Run(cfg, seed=8).run_stages()
     plan, d = run.plan, run.dev
     rng = np.random.default_rng(9)
