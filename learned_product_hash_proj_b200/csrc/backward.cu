@@ -18,7 +18,8 @@
 //   k_bwd_dkdv   one CTA per (b, h) and tile of up to 64 keys of one block:
 //                walks the block's local queries and its selecting queries,
 //                accumulating dK and dV of its keys in registers;
-//   k_bwd_rope   inverse rotation of dQ, dK and the token-major layout;
+//   (dq, dk and dv leave these kernels either as [B,H,S,d] for the post-RoPE
+//   q and k, or rotated back and token-major for the projection gradients)
 //   k_gemm_any   the projection gradients of fp32 storage (generic strided SIMT
 //                GEMM, split K with fp32 atomics where the output has few
 //                tiles); with bf16 storage they run on the tensor cores
@@ -37,7 +38,7 @@ namespace mono {
 namespace {
 
 struct BwdLayout {
-    size_t lse, dsum, cnt, start, cursor, list, dO, dQ, dK, dV, dQp, dKp, dVp, total;
+    size_t lse, dsum, cnt, start, cursor, list, dO, dQp, dKp, dVp, total;
 };
 
 BwdLayout bwd_layout(const Plan &p) {
@@ -57,9 +58,6 @@ BwdLayout bwd_layout(const Plan &p) {
     L.cursor = take(B * H * nb * 4);
     L.list = take(B * H * S * R * 4);
     L.dO = take(B * S * H * d * 4);
-    L.dQ = take(B * H * S * d * 4);
-    L.dK = take(B * H * S * d * 4);
-    L.dV = take(B * H * S * d * 4);
     L.dQp = take(B * S * H * d * 4);
     L.dKp = take(B * S * H * d * 4);
     L.dVp = take(B * S * H * d * 4);
@@ -87,6 +85,71 @@ __device__ __forceinline__ bool bwd_sel_valid(int j, int t, int Bs, int L) { ret
 // grid ceil(B H S * D/16 / 256), 256 threads.
 // ---------------------------------------------------------------------------
 constexpr int kDqE = 16;
+
+// Where the attention gradients go: [B,H,S,d] fp32 with respect to the
+// post-RoPE q and k (mono_attend_backward), or with respect to the projection
+// outputs before RoPE -- dq and dk rotated back by the forward's angle of their
+// position (the transpose of its rotation, from its cos/sin tables), dv as is --
+// token-major [B*S, H*d], in fp32 or as two bf16 terms hi = bf16(v),
+// lo = bf16(v - hi) at out and out + B*S*H*d (their sum carries 16 significant
+// bits) for the tensor-core GEMMs.
+enum GradMode { kOutHeads = 0, kOutTokensF32 = 1, kOutTokensSplit = 2 };
+
+struct GradOut {
+    void *q, *k, *v;
+    const float2 *rope_hi, *rope_lo;  // token modes: the forward's tables (positions t / 64 and t % 64)
+    int mode;
+};
+
+__device__ __forceinline__ uint32_t bf16_pair(float a, float b) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    return *(uint32_t *)&h;
+}
+
+// the 16 gradient values v of dimensions e0 .. e0+15 of (b, h, position t)
+template <int DD>
+__device__ __forceinline__ void store_grad16(const GradOut &go, void *out, bool rotate, float *v, int b, int h, int t,
+                                             int e0, int B, int H, int S) {
+    if (go.mode == kOutHeads) {
+        float4 *dst = (float4 *)((float *)out + (((size_t)b * H + h) * S + t) * DD + e0);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) dst[c] = make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+        return;
+    }
+    if (rotate) {
+        const float2 *hi = go.rope_hi + (size_t)(t / kRopeLo) * (DD / 2) + e0 / 2;
+        const float2 *lo = go.rope_lo + (size_t)(t % kRopeLo) * (DD / 2) + e0 / 2;
+#pragma unroll
+        for (int pr = 0; pr < 8; ++pr) {
+            const float2 a = __ldg(hi + pr), bb = __ldg(lo + pr);
+            const float c = a.x * bb.x - a.y * bb.y, sn = a.y * bb.x + a.x * bb.y;
+            const float x0 = v[2 * pr], x1 = v[2 * pr + 1];
+            v[2 * pr] = x0 * c + x1 * sn;
+            v[2 * pr + 1] = -x0 * sn + x1 * c;
+        }
+    }
+    const size_t dst = (((size_t)b * S + t) * H + h) * DD + e0;
+    if (go.mode == kOutTokensF32) {
+        float4 *o4 = (float4 *)((float *)out + dst);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) o4[c] = make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+        return;
+    }
+    const size_t n = (size_t)B * S * H * DD;
+    uint32_t hw[8], lw[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const float h0 = __bfloat162float(__float2bfloat16_rn(v[2 * i]));
+        const float h1 = __bfloat162float(__float2bfloat16_rn(v[2 * i + 1]));
+        hw[i] = bf16_pair(h0, h1);
+        lw[i] = bf16_pair(v[2 * i] - h0, v[2 * i + 1] - h1);
+    }
+    uint4 *oh = (uint4 *)((__nv_bfloat16 *)out + dst), *ol = (uint4 *)((__nv_bfloat16 *)out + n + dst);
+    oh[0] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+    oh[1] = make_uint4(hw[4], hw[5], hw[6], hw[7]);
+    ol[0] = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+    ol[1] = make_uint4(lw[4], lw[5], lw[6], lw[7]);
+}
 
 template <typename T> __device__ __forceinline__ void load16(const T *p, float *v);
 template <> __device__ __forceinline__ void load16<float>(const float *p, float *v) {
@@ -119,7 +182,7 @@ __device__ __forceinline__ float group_sum(float v) {
 template <typename T, int DD>
 __global__ void __launch_bounds__(256) k_bwd_dq(const T *__restrict__ Q, const T *__restrict__ K,
                                                 const T *__restrict__ V, const int32_t *__restrict__ sel,
-                                                const float *__restrict__ dO, float *__restrict__ dQ,
+                                                const float *__restrict__ dO, const GradOut go,
                                                 float *__restrict__ lse_out, float *__restrict__ dsum_out, int B, int H,
                                                 int S, int Bs, int L, int R, float scale) {
     constexpr int TPQ = DD / kDqE, E = kDqE, U = 2;
@@ -185,10 +248,13 @@ __global__ void __launch_bounds__(256) k_bwd_dq(const T *__restrict__ Q, const T
         for (int u = 0; u < U; ++u) load16<T>(kr[u], kk[u]);
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-            float part = 0.f;
+            float part = 0.f, part2 = 0.f;
 #pragma unroll
-            for (int e = 0; e < E; ++e) part = fmaf(q[e], kk[u][e], part);
-            sc[u] = group_sum<TPQ>(part) * scale;
+            for (int e = 0; e < E / 2; ++e) {
+                part = fmaf(q[e], kk[u][e], part);
+                part2 = fmaf(q[e + E / 2], kk[u][e + E / 2], part2);
+            }
+            sc[u] = group_sum<TPQ>(part + part2) * scale;
         }
         float mx = m;
 #pragma unroll
@@ -226,14 +292,16 @@ __global__ void __launch_bounds__(256) k_bwd_dq(const T *__restrict__ Q, const T
             float vv[E];
             load16<T>(kr[u], kk[u]);
             load16<T>(vr[u], vv);
-            float a = 0.f, c = 0.f;
+            float a = 0.f, c = 0.f, a2 = 0.f, c2 = 0.f;
 #pragma unroll
-            for (int e = 0; e < E; ++e) {
+            for (int e = 0; e < E / 2; ++e) {
                 a = fmaf(q[e], kk[u][e], a);
                 c = fmaf(g[e], vv[e], c);
+                a2 = fmaf(q[e + E / 2], kk[u][e + E / 2], a2);
+                c2 = fmaf(g[e + E / 2], vv[e + E / 2], c2);
             }
-            sp[u] = a;
-            dp[u] = c;
+            sp[u] = a + a2;
+            dp[u] = c + c2;
         }
 #pragma unroll
         for (int u = 0; u < U; ++u) {
@@ -248,10 +316,9 @@ __global__ void __launch_bounds__(256) k_bwd_dq(const T *__restrict__ Q, const T
         }
     });
     if (live) {
-        float4 *dst = (float4 *)(dQ + w * DD + e0);
 #pragma unroll
-        for (int c = 0; c < E / 4; ++c)
-            dst[c] = make_float4(dq[4 * c] * scale, dq[4 * c + 1] * scale, dq[4 * c + 2] * scale, dq[4 * c + 3] * scale);
+        for (int e = 0; e < E; ++e) dq[e] *= scale;
+        store_grad16<DD>(go, go.q, true, dq, b, h, t, e0, B, H, S);
         if (e0 == 0) {
             lse_out[w] = lse;
             dsum_out[w] = D;
@@ -329,8 +396,10 @@ __global__ void __launch_bounds__(256) k_bwd_fill(const int32_t *__restrict__ se
 // and dV accumulators in registers; a key's threads are consecutive lanes and
 // combine their partial dot products with xor shuffles.  Queries come in
 // groups of 16 (q, dO, log-sum-exp and D staged in shared memory, read as
-// broadcast float4; the next group's rows are fetched into registers while
-// the current one is computed, double-buffered): first the local ones (blocks
+// broadcast float4; each 16-float segment of a row padded to 20 floats so
+// that the segments of a key's lanes sit in distinct banks; the next group's
+// rows are fetched into registers while the current one is computed,
+// double-buffered): first the local ones (blocks
 // j .. j+L-1; in block j itself only keys s <= t, applied as a zero
 // probability so that every lane takes part in the shuffles), then those
 // whose selection holds block j.
@@ -342,12 +411,13 @@ template <typename T, int DD>
 __global__ void __launch_bounds__(kBwdKT * DD / 16, DD == 64 ? 2 : 1) k_bwd_dkdv(
     const T *__restrict__ Q, const T *__restrict__ K, const T *__restrict__ V, const float *__restrict__ dO,
     const float *__restrict__ lse, const float *__restrict__ dsum, const int32_t *__restrict__ cnt,
-    const int32_t *__restrict__ start, const int32_t *__restrict__ list, float *__restrict__ dK,
-    float *__restrict__ dV, int H, int S, int Bs, int L, int R, int nb, float scale) {
+    const int32_t *__restrict__ start, const int32_t *__restrict__ list, const GradOut go, int B, int H, int S,
+    int Bs, int L, int R, int nb, float scale) {
     constexpr int TPK = DD / 16, NT = kBwdKT * TPK, E = 16;
     constexpr int PER = kBwdQG * DD / NT;  // staged elements per thread and array (one dimension, PER queries)
-    __shared__ __align__(16) float sq[2][kBwdQG][DD];
-    __shared__ __align__(16) float sg[2][kBwdQG][DD];
+    constexpr int SEG = 20, ROW = TPK * SEG;  // padded segment and row, in floats
+    __shared__ __align__(16) float sq[2][kBwdQG][ROW];
+    __shared__ __align__(16) float sg[2][kBwdQG][ROW];
     __shared__ float slse[2][kBwdQG], sD[2][kBwdQG];
     __shared__ int st[2][kBwdQG];
     const int tpb = (Bs + kBwdKT - 1) / kBwdKT;
@@ -373,8 +443,8 @@ __global__ void __launch_bounds__(kBwdKT * DD / 16, DD == 64 ? 2 : 1) k_bwd_dkdv
     const int nrem = R > 0 ? cnt[bh * nb + j] : 0;
     const int rem0 = R > 0 ? start[bh * nb + j] : 0;
     const int nq = nloc + nrem;
-    // thread tid stages dimension fe of queries fq0, fq0 + NT/DD, ... of a group
-    const int fe = tid % DD, fq0 = tid / DD;
+    // thread tid stages dimension fe of queries fq0, fq0 + NT/DD, ... of a group (at padded column fc)
+    const int fe = tid % DD, fq0 = tid / DD, fc = fe + (fe / E) * (SEG - E);
     float rq[PER], rg[PER], rl[PER], rd[PER];
     int rt[PER];
     auto fetch = [&](int g0) {
@@ -396,8 +466,8 @@ __global__ void __launch_bounds__(kBwdKT * DD / 16, DD == 64 ? 2 : 1) k_bwd_dkdv
 #pragma unroll
         for (int k = 0; k < PER; ++k) {
             const int qi = fq0 + k * (NT / DD);
-            sq[buf][qi][fe] = rq[k];
-            sg[buf][qi][fe] = rg[k];
+            sq[buf][qi][fc] = rq[k];
+            sg[buf][qi][fc] = rg[k];
             if (fe == 0) {
                 st[buf][qi] = rt[k];
                 slse[buf][qi] = rl[k];
@@ -416,7 +486,8 @@ __global__ void __launch_bounds__(kBwdKT * DD / 16, DD == 64 ? 2 : 1) k_bwd_dkdv
         const bool more = g0 + kBwdQG < nq;
         if (more) fetch(g0 + kBwdQG);  // in flight while this group is computed
         for (int qi = 0; qi < ng; ++qi) {
-            const float4 *q4 = (const float4 *)&sq[buf][qi][e0], *g4 = (const float4 *)&sg[buf][qi][e0];
+            const float4 *q4 = (const float4 *)&sq[buf][qi][part * SEG];
+            const float4 *g4 = (const float4 *)&sg[buf][qi][part * SEG];
             float qv[E], gv[E];
 #pragma unroll
             for (int c = 0; c < E / 4; ++c) {
@@ -424,12 +495,16 @@ __global__ void __launch_bounds__(kBwdKT * DD / 16, DD == 64 ? 2 : 1) k_bwd_dkdv
                 qv[4 * c] = a.x; qv[4 * c + 1] = a.y; qv[4 * c + 2] = a.z; qv[4 * c + 3] = a.w;
                 gv[4 * c] = bb.x; gv[4 * c + 1] = bb.y; gv[4 * c + 2] = bb.z; gv[4 * c + 3] = bb.w;
             }
-            float sp = 0.f, dp = 0.f;
+            float sp = 0.f, dp = 0.f, sp2 = 0.f, dp2 = 0.f;  // two chains each
 #pragma unroll
-            for (int e = 0; e < E; ++e) {
+            for (int e = 0; e < E / 2; ++e) {
                 sp = fmaf(qv[e], kr[e], sp);
                 dp = fmaf(gv[e], vr[e], dp);
+                sp2 = fmaf(qv[e + E / 2], kr[e + E / 2], sp2);
+                dp2 = fmaf(gv[e + E / 2], vr[e + E / 2], dp2);
             }
+            sp += sp2;
+            dp += dp2;
 #pragma unroll
             for (int o = 1; o < TPK; o <<= 1) {
                 sp += __shfl_xor_sync(0xffffffffu, sp, o);
@@ -448,53 +523,9 @@ __global__ void __launch_bounds__(kBwdKT * DD / 16, DD == 64 ? 2 : 1) k_bwd_dkdv
         __syncthreads();
     }
     if (live) {
-#pragma unroll
-        for (int e = 0; e < E; ++e) {
-            dK[(bh * S + key) * DD + e0 + e] = dk[e];
-            dV[(bh * S + key) * DD + e0 + e] = dv[e];
-        }
+        store_grad16<DD>(go, go.k, true, dk, b, h, key, e0, B, H, S);
+        store_grad16<DD>(go, go.v, false, dv, b, h, key, e0, B, H, S);
     }
-}
-
-// ---------------------------------------------------------------------------
-// gradients before RoPE, token-major: dQ and dK (post-RoPE, [B,H,S,d]) rotated
-// back by -t*theta^(-2i/d) (the transpose of the forward rotation), dV copied;
-// outputs [B*S, H*d] in fp32 or, for the tensor-core GEMMs, as two bf16 terms
-// hi = bf16(v), lo = bf16(v - hi) at out and out + B*S*H*d (their sum carries
-// 16 significant bits).  One thread per (b, t, h, pair i);
-// grid ceil(B S H d/2 / 256).
-// ---------------------------------------------------------------------------
-__device__ __forceinline__ void put_grad(float *out, size_t i, size_t, float v) { out[i] = v; }
-__device__ __forceinline__ void put_grad(__nv_bfloat16 *out, size_t i, size_t n, float v) {
-    const __nv_bfloat16 hi = __float2bfloat16_rn(v);
-    out[i] = hi;
-    out[n + i] = __float2bfloat16_rn(v - __bfloat162float(hi));
-}
-
-template <typename TO>
-__global__ void __launch_bounds__(256) k_bwd_rope(const float *__restrict__ dQ, const float *__restrict__ dK,
-                                                  const float *__restrict__ dV, TO *__restrict__ dQp,
-                                                  TO *__restrict__ dKp, TO *__restrict__ dVp, int B, int S, int H,
-                                                  int d, double theta) {
-    const long long n = (long long)B * S * H * (d / 2);
-    const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-    if (i >= n) return;
-    const int pr = (int)(i % (d / 2));
-    const int h = (int)((i / (d / 2)) % H);
-    const long long bt = i / ((long long)(d / 2) * H);
-    const int t = (int)(bt % S), b = (int)(bt / S);
-    const double ang = (double)t * pow(theta, -2.0 * (double)pr / (double)d);
-    const float c = (float)cos(ang), s = (float)sin(ang);
-    const size_t src = (((size_t)b * H + h) * S + t) * d + 2 * pr;
-    const size_t dst = ((size_t)bt * H + h) * d + 2 * pr;
-    const float q0 = dQ[src], q1 = dQ[src + 1], k0 = dK[src], k1 = dK[src + 1];
-    const size_t nn = (size_t)n * 2;
-    put_grad(dQp, dst, nn, q0 * c + q1 * s);
-    put_grad(dQp, dst + 1, nn, -q0 * s + q1 * c);
-    put_grad(dKp, dst, nn, k0 * c + k1 * s);
-    put_grad(dKp, dst + 1, nn, -k0 * s + k1 * c);
-    put_grad(dVp, dst, nn, dV[src]);
-    put_grad(dVp, dst + 1, nn, dV[src + 1]);
 }
 
 // ---------------------------------------------------------------------------
@@ -582,7 +613,7 @@ cudaError_t gemm_any(int M, int N, int Kd, const TA *A, long long am, long long 
 
 template <typename T>
 cudaError_t attend_backward(const Plan &p, const T *Q, const T *K, const T *V, const int32_t *sel, const float *dO,
-                            float *dQ, float *dK, float *dV, char *bws, cudaStream_t s) {
+                            const GradOut &go, char *bws, cudaStream_t s) {
     const mono_config &c = p.cfg;
     const BwdLayout L = bwd_layout(p);
     float *lse = (float *)(bws + L.lse), *dsum = (float *)(bws + L.dsum);
@@ -594,9 +625,9 @@ cudaError_t attend_backward(const Plan &p, const T *Q, const T *K, const T *V, c
     const int tpq = c.d / kDqE;
     const unsigned gq = (unsigned)((nq * tpq + 255) / 256);
     if (c.d == 64)
-        k_bwd_dq<T, 64><<<gq, 256, 0, s>>>(Q, K, V, sel, dO, dQ, lse, dsum, c.B, c.H, c.S, c.Bs, c.L, c.R, scale);
+        k_bwd_dq<T, 64><<<gq, 256, 0, s>>>(Q, K, V, sel, dO, go, lse, dsum, c.B, c.H, c.S, c.Bs, c.L, c.R, scale);
     else
-        k_bwd_dq<T, 128><<<gq, 256, 0, s>>>(Q, K, V, sel, dO, dQ, lse, dsum, c.B, c.H, c.S, c.Bs, c.L, c.R, scale);
+        k_bwd_dq<T, 128><<<gq, 256, 0, s>>>(Q, K, V, sel, dO, go, lse, dsum, c.B, c.H, c.S, c.Bs, c.L, c.R, scale);
     count_launches(1);
     if (c.R > 0) {
         const long long n = nq * c.R;
@@ -609,11 +640,11 @@ cudaError_t attend_backward(const Plan &p, const T *Q, const T *K, const T *V, c
     const int tpb = (c.Bs + kBwdKT - 1) / kBwdKT;
     const dim3 gk(tpb * p.nb, c.H, c.B);
     if (c.d == 64)
-        k_bwd_dkdv<T, 64><<<gk, kBwdKT * 4, 0, s>>>(Q, K, V, dO, lse, dsum, cnt, start, list, dK, dV, c.H, c.S, c.Bs,
-                                                     c.L, c.R, p.nb, scale);
+        k_bwd_dkdv<T, 64><<<gk, kBwdKT * 4, 0, s>>>(Q, K, V, dO, lse, dsum, cnt, start, list, go, c.B, c.H, c.S,
+                                                     c.Bs, c.L, c.R, p.nb, scale);
     else
-        k_bwd_dkdv<T, 128><<<gk, kBwdKT * 8, 0, s>>>(Q, K, V, dO, lse, dsum, cnt, start, list, dK, dV, c.H, c.S, c.Bs,
-                                                      c.L, c.R, p.nb, scale);
+        k_bwd_dkdv<T, 128><<<gk, kBwdKT * 8, 0, s>>>(Q, K, V, dO, lse, dsum, cnt, start, list, go, c.B, c.H, c.S,
+                                                      c.Bs, c.L, c.R, p.nb, scale);
     count_launches(1);
     return cudaGetLastError();
 }
@@ -634,16 +665,21 @@ bool grads_tc_supported(const mono_config &c) {
 template <typename T>
 cudaError_t backward_t(const Plan &p, const T *x, const T *Wq, const T *Wk, const T *Wv, const T *Wo,
                        const int32_t *sel, const T *ddelta, float *dx, float *dWq, float *dWk, float *dWv, float *dWo,
-                       const T *Q, const T *K, const T *V, const T *O, char *bws, unsigned long long *counters,
-                       cudaStream_t s) {
+                       const T *Q, const T *K, const T *V, const T *O, char *bws, void *ws, cudaStream_t s) {
     const mono_config &c = p.cfg;
     const BwdLayout L = bwd_layout(p);
-    float *dO = (float *)(bws + L.dO), *dQ = (float *)(bws + L.dQ), *dK = (float *)(bws + L.dK);
-    float *dV = (float *)(bws + L.dV);
+    unsigned long long *counters = (unsigned long long *)ws_ptr(p, ws, kRegCounters);
+    float *dO = (float *)(bws + L.dO);
     const int BS = c.B * c.S, Hd = c.H * c.d, W = c.W;
     const bool tc = grads_tc_supported(c);
-    const long long npairs = (long long)BS * Hd / 2;
-    const unsigned rope_grid = (unsigned)((npairs + 255) / 256);
+    // dQp, dKp, dVp: the attention gradients before RoPE, token-major, written by the attention kernels
+    GradOut go{};
+    go.q = bws + L.dQp;
+    go.k = bws + L.dKp;
+    go.v = bws + L.dVp;
+    go.rope_hi = (const float2 *)ws_ptr(p, ws, kRegRope);  // built by the projection of the forward recompute
+    go.rope_lo = go.rope_hi + (size_t)((c.S + kRopeLo - 1) / kRopeLo) * (c.d / 2);
+    go.mode = tc ? kOutTokensSplit : kOutTokensF32;
     cudaError_t e;
     if (tc) {
         // delta = O Wo^T:  dO = ddelta Wo (Wo MN-major),  dWo = ddelta^T O (both MN-major)
@@ -651,27 +687,23 @@ cudaError_t backward_t(const Plan &p, const T *x, const T *Wq, const T *Wk, cons
         float *c0[1] = {dO}, *c1[1] = {dWo};
         if ((e = gemm_grad_tc(BS, Hd, W, 1, 1, a0, false, b0, true, c0, false, counters, s)) != cudaSuccess) return e;
         if ((e = gemm_grad_tc(W, Hd, BS, 1, 1, a0, true, b1, true, c1, false, counters, s)) != cudaSuccess) return e;
-        if ((e = attend_backward<T>(p, Q, K, V, sel, dO, dQ, dK, dV, bws, s)) != cudaSuccess) return e;
-        using B16 = __nv_bfloat16;
-        B16 *hq = (B16 *)(bws + L.dQp), *hk = (B16 *)(bws + L.dKp), *hv = (B16 *)(bws + L.dVp);
-        k_bwd_rope<B16><<<rope_grid, 256, 0, s>>>(dQ, dK, dV, hq, hk, hv, c.B, c.S, c.H, c.d, c.rope_theta);
-        count_launches(1);
+        if ((e = attend_backward<T>(p, Q, K, V, sel, dO, go, bws, s)) != cudaSuccess) return e;
         // q = x Wq^T (per head, then RoPE):  dWq = dQp^T x (both MN-major),  dx = dQp Wq + dKp Wk + dVp Wv,
         // each dZp as hi + lo
+        using B16 = __nv_bfloat16;
+        const B16 *hq = (const B16 *)go.q, *hk = (const B16 *)go.k, *hv = (const B16 *)go.v;
         const size_t n = (size_t)BS * Hd;
         const void *ah[6] = {hq, hq + n, hk, hk + n, hv, hv + n};
-        const void *xs[6] = {x, x, x, x, x, x}, *ws[6] = {Wq, Wq, Wk, Wk, Wv, Wv};
+        const void *xs[6] = {x, x, x, x, x, x}, *wz[6] = {Wq, Wq, Wk, Wk, Wv, Wv};
         float *cw[3] = {dWq, dWk, dWv}, *cx[1] = {dx};
         if ((e = gemm_grad_tc(Hd, W, BS, 2, 3, ah, true, xs, true, cw, false, counters, s)) != cudaSuccess) return e;
-        return gemm_grad_tc(BS, W, Hd, 6, 1, ah, false, ws, true, cx, false, counters, s);
+        return gemm_grad_tc(BS, W, Hd, 6, 1, ah, false, wz, true, cx, false, counters, s);
     }
-    float *dQp = (float *)(bws + L.dQp), *dKp = (float *)(bws + L.dKp), *dVp = (float *)(bws + L.dVp);
+    const float *dQp = (const float *)go.q, *dKp = (const float *)go.k, *dVp = (const float *)go.v;
     // delta = O Wo^T:  dO = ddelta Wo,  dWo = ddelta^T O
     if ((e = gemm_any<T, T>(BS, Hd, W, ddelta, W, 1, Wo, Hd, 1, dO, Hd, 0.f, s)) != cudaSuccess) return e;
     if ((e = gemm_any<T, T>(W, Hd, BS, ddelta, 1, W, O, Hd, 1, dWo, Hd, 0.f, s)) != cudaSuccess) return e;
-    if ((e = attend_backward<T>(p, Q, K, V, sel, dO, dQ, dK, dV, bws, s)) != cudaSuccess) return e;
-    k_bwd_rope<float><<<rope_grid, 256, 0, s>>>(dQ, dK, dV, dQp, dKp, dVp, c.B, c.S, c.H, c.d, c.rope_theta);
-    count_launches(1);
+    if ((e = attend_backward<T>(p, Q, K, V, sel, dO, go, bws, s)) != cudaSuccess) return e;
     // q = x Wq^T (per head, then RoPE):  dWq = dQp^T x,  dx = dQp Wq + dKp Wk + dVp Wv
     if ((e = gemm_any<float, T>(Hd, W, BS, dQp, 1, Hd, x, W, 1, dWq, W, 0.f, s)) != cudaSuccess) return e;
     if ((e = gemm_any<float, T>(Hd, W, BS, dKp, 1, Hd, x, W, 1, dWk, W, 0.f, s)) != cudaSuccess) return e;
@@ -716,12 +748,17 @@ int mono_attend_backward(const mono_plan_t *plan, const void *Q, const void *K, 
     if (st) return st;
     if (c.R > 0 && (st = bwd_check({sel}))) return st;
     cudaStream_t s = (cudaStream_t)stream;
+    GradOut go{};
+    go.q = dQ;
+    go.k = dK;
+    go.v = dV;
+    go.mode = kOutHeads;
     if (c.dtype == MONO_BF16)
         return bwd_status(attend_backward<__nv_bfloat16>(p, (const __nv_bfloat16 *)Q, (const __nv_bfloat16 *)K,
-                                                         (const __nv_bfloat16 *)V, sel, dO, dQ, dK, dV,
-                                                         (char *)bwd_workspace, s));
-    return bwd_status(attend_backward<float>(p, (const float *)Q, (const float *)K, (const float *)V, sel, dO, dQ, dK,
-                                             dV, (char *)bwd_workspace, s));
+                                                         (const __nv_bfloat16 *)V, sel, dO, go, (char *)bwd_workspace,
+                                                         s));
+    return bwd_status(attend_backward<float>(p, (const float *)Q, (const float *)K, (const float *)V, sel, dO, go,
+                                             (char *)bwd_workspace, s));
 }
 
 int mono_backward(const mono_plan_t *plan, const void *x, const void *Wq, const void *Wk, const void *Wv,
@@ -743,18 +780,17 @@ int mono_backward(const mono_plan_t *plan, const void *x, const void *Wq, const 
     if ((st = mono_attend(plan, Q, K, V, sel, O, workspace, stream))) return st;
     cudaStream_t s = (cudaStream_t)stream;
     char *bws = (char *)bwd_workspace;
-    unsigned long long *counters = (unsigned long long *)ws_ptr(p, workspace, kRegCounters);
     if (c.dtype == MONO_BF16) {
         using B16 = __nv_bfloat16;
         return bwd_status(backward_t<B16>(p, (const B16 *)x, (const B16 *)Wq, (const B16 *)Wk, (const B16 *)Wv,
                                           (const B16 *)Wo, sel, (const B16 *)ddelta, dx, dWq, dWk, dWv, dWo,
-                                          (const B16 *)Q, (const B16 *)K, (const B16 *)V, (const B16 *)O, bws, counters,
+                                          (const B16 *)Q, (const B16 *)K, (const B16 *)V, (const B16 *)O, bws, workspace,
                                           s));
     }
     return bwd_status(backward_t<float>(p, (const float *)x, (const float *)Wq, (const float *)Wk, (const float *)Wv,
                                         (const float *)Wo, sel, (const float *)ddelta, dx, dWq, dWk, dWv, dWo,
                                         (const float *)Q, (const float *)K, (const float *)V, (const float *)O, bws,
-                                        counters, s));
+                                        workspace, s));
 }
 
 }  // extern "C"

@@ -437,15 +437,18 @@ cudaError_t gemm_grad_tc(int M, int N, int K, int nsrc, int ngroups, const void 
     const int slots = 2 * sms;
     const int tiles = ((N + BN - 1) / BN) * ((M + BM - 1) / BM) * ngroups;
     const int total = ((K + BK - 1) / BK) * nsrc;
-    // split K where the tiles alone fill the GPU's CTA slots poorly: the split with the best last-wave fill
+    // split K only where the tiles alone leave CTA slots idle (fewer tiles than slots): the smallest split
+    // whose wave fill is clearly (5 %) better than every smaller one's; each split re-adds the output once
     int split = 1;
-    double best = 0.0;
-    for (int sp = 1; sp <= 16 && total / sp >= 4; ++sp) {
-        const long long ctas = (long long)tiles * sp;
-        const double fill = (double)ctas / (double)(((ctas + slots - 1) / slots) * slots);
-        if (fill > best + 1e-9) {
-            best = fill;
-            split = sp;
+    if (tiles < slots) {
+        double best = (double)tiles / (double)slots;
+        for (int sp = 2; sp <= 16 && total / sp >= 4; ++sp) {
+            const long long ctas = (long long)tiles * sp;
+            const double fill = (double)ctas / (double)(((ctas + slots - 1) / slots) * slots);
+            if (fill > best * 1.05) {
+                best = fill;
+                split = sp;
+            }
         }
     }
     const int per = (total + split - 1) / split;
