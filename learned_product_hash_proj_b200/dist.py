@@ -1,10 +1,17 @@
-"""One process per GPU: rank discovery and the host-side aggregation of a
-multi-GPU measurement.
+"""One process per GPU: rank discovery, the host-side aggregation of a
+multi-GPU measurement, and the head-sharded mixer.
 
 The mixer's work shards with no exchange: every (batch, head) routes and
 attends on its own, so N GPUs run N independent replicas of a workload (each
 rank its own sequences) and the only collective is the reduction of the
 timings (the maximum over ranks) and of the token counts (the sum).
+
+Head sharding splits one workload instead: rank r of N runs the heads
+[r H/N, (r+1) H/N) -- their rows of Wq, Wk, Wv, their columns of Wo and their
+codebooks -- through the whole mixer.  Projection, routing (codebooks, posting
+lists and probes are per head) and attention of a head need nothing from the
+other heads; the output projection delta = sum_h O_h Wo_h^T leaves each rank a
+partial sum over its heads, and one all-reduce (sum) gives every rank delta.
 """
 from __future__ import annotations
 
@@ -61,6 +68,67 @@ def throughput(tokens_per_rank: list[float], seconds_per_rank: list[float], devi
     tot = reduce_sum([sum(tokens_per_rank)], device)[0]
     t = reduce_max([max(seconds_per_rank)], device)[0]
     return tot / t
+
+
+# --- head-sharded mixer ----------------------------------------------------
+
+
+def head_range(H: int, rank: int, world: int) -> tuple[int, int]:
+    """The heads [h0, h1) of `rank` when H heads are split evenly over `world` ranks."""
+    if world < 1 or not 0 <= rank < world:
+        raise ValueError(f"rank {rank} outside a world of {world}")
+    if H % world:
+        raise ValueError(f"{H} heads do not split evenly over {world} ranks")
+    per = H // world
+    return rank * per, (rank + 1) * per
+
+
+def shard_config(cfg, rank: int, world: int):
+    """The configuration one rank runs: the same workload with its H / world heads."""
+    h0, h1 = head_range(cfg.H, rank, world)
+    return cfg.with_(H=h1 - h0)
+
+
+def _contig(a):
+    return a.contiguous() if isinstance(a, torch.Tensor) else a.copy()
+
+
+def shard_weights(params: dict, cfg, rank: int, world: int) -> dict:
+    """Rank's slice of the mixer's parameters (numpy arrays or torch tensors, copied contiguous):
+    rows [h0 d, h1 d) of Wq, Wk, Wv ([H d, W]), the same columns of Wo ([W, H d]) and heads
+    [h0, h1) of the codebooks ([H, M, C, d/M]).  Other entries (x) are passed through."""
+    h0, h1 = head_range(cfg.H, rank, world)
+    r0, r1 = h0 * cfg.d, h1 * cfg.d
+    out = dict(params)
+    for k in ("Wq", "Wk", "Wv"):
+        out[k] = _contig(params[k][r0:r1])
+    out["Wo"] = _contig(params["Wo"][:, r0:r1])
+    out["codebooks"] = _contig(params["codebooks"][h0:h1])
+    return out
+
+
+def reduce_partial_delta(delta, group=None, stream=None):
+    """Sum the ranks' partial deltas in place: every rank ends with the whole delta.  The sum is
+    taken in delta's dtype (for bf16 storage each reduction step rounds to bf16).  With a CUDA
+    stream, the all-reduce is ordered after the work already queued on it."""
+    if not dist.is_initialized() or dist.get_world_size(group) == 1:
+        return delta
+    if stream is not None:
+        with torch.cuda.stream(stream):
+            dist.all_reduce(delta, op=dist.ReduceOp.SUM, group=group)
+    else:
+        dist.all_reduce(delta, op=dist.ReduceOp.SUM, group=group)
+    return delta
+
+
+def head_sharded_forward(plan, x, shard: dict, delta, ws, group=None, forced=None, stream=None):
+    """The mixer on this rank's heads (plan built from shard_config, shard from shard_weights, on
+    this rank's GPU), then the all-reduce of the partial delta: delta [B, S, W] is the whole
+    mixer's output on every rank.  forced, if given, holds this rank's heads."""
+    from . import mono
+    mono.forward(plan, x, shard["Wq"], shard["Wk"], shard["Wv"], shard["Wo"], shard["codebooks"], delta, ws,
+                 forced=forced, stream=stream)
+    return reduce_partial_delta(delta, group, stream)
 
 
 def finalize():
