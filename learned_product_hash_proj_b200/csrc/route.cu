@@ -71,13 +71,17 @@ __global__ void __launch_bounds__(128) k_summary_assign(const T *__restrict__ K,
 // (A2, A3) the same summaries with one warp per block: each lane owns D/32
 // adjacent columns and walks the block's rows in ascending t, reading its
 // columns of a row as one 32- or 64-bit word.  A CTA takes 4 x bpw
-// consecutive blocks of one (b, h) (each warp bpw of them, all rows in flight
-// at once) and keeps that head's codebook in shared memory, transposed so that
-// lane mc reads codeword mc without bank conflicts.
+// consecutive blocks of one (b, h), each warp bpw of them through a two-deep
+// ring: block q+1's rows stream in (cp.async) while block q is summed.  The
+// head's codebook sits in shared memory, transposed so that lane mc reads
+// codeword mc without bank conflicts.
 // grid (ceil(nb / (4 bpw)), H, B), 128 threads.
 // ---------------------------------------------------------------------------
-inline size_t summary_smem(int M, int C, int Bs, int D, int es, int bpw) {
-    return ((size_t)M * C * (D / M) + 4 * (size_t)D + 4 * (size_t)M * C) * 4 + 16 + (size_t)4 * bpw * Bs * D * es;
+constexpr int kSumRing = 2;  // staged blocks per warp
+
+inline size_t summary_smem(int M, int C, int Bs, int D, int es) {
+    return ((size_t)M * C * (D / M) + 4 * (size_t)D + 4 * (size_t)M * C) * 4 + 16 +
+           (size_t)4 * kSumRing * Bs * D * es;
 }
 
 template <typename T, int D>
@@ -97,16 +101,18 @@ __global__ void __launch_bounds__(128) k_summary_assign_w(const T *__restrict__ 
     const int nb = S / Bs;
     const size_t bh = (size_t)b * H + h;
     const int j0 = (blockIdx.x * 4 + warp) * bpw;
-    // every row copy of this warp's blocks in flight at once
+    // block q's rows into ring slot q % 2; one commit group per block (empty past the warp's last block)
     const int chunks = Bs * D * (int)sizeof(T) / 16;
-    T *rows = s_rows + (size_t)warp * bpw * Bs * D;
-    for (int q = 0; q < bpw; ++q) {
-        if (j0 + q < nb) {
+    T *rows = s_rows + (size_t)warp * kSumRing * Bs * D;
+    auto prefetch = [&](int q) {
+        if (q < bpw && j0 + q < nb) {
             const uint8_t *src = (const uint8_t *)(K + (bh * S + (size_t)(j0 + q) * Bs) * D);
-            uint8_t *dst = (uint8_t *)(rows + (size_t)q * Bs * D);
+            uint8_t *dst = (uint8_t *)(rows + (size_t)(q % kSumRing) * Bs * D);
             for (int c = lane; c < chunks; c += 32) tc::cp_async16(dst + 16 * c, src + 16 * c, true);
         }
-    }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+    prefetch(0);
     // the head's codebook (C*D floats, [M][C][dm]), transposed, with independent 16-byte loads
     {
         const float4 *src = (const float4 *)(cb + (size_t)h * C * D);
@@ -119,12 +125,14 @@ __global__ void __launch_bounds__(128) k_summary_assign_w(const T *__restrict__ 
             s_cbT[(i + 3) * MC + mc] = f.w;
         }
     }
-    tc::cp_async_wait_all();
-    __syncthreads();
+    __syncthreads();  // the codebook; block 0 may still be in flight
     for (int q = 0; q < bpw; ++q) {
         const int j = j0 + q;
+        prefetch(q + 1);  // into the slot block q - 1 used (released by the warp barrier ending that step)
+        asm volatile("cp.async.wait_group 1;" ::: "memory");  // block q has landed (this lane's copies)
+        __syncwarp();                                         // ... and every lane's
         if (j < nb) {
-            const T *rq = rows + (size_t)q * Bs * D;
+            const T *rq = rows + (size_t)(q % kSumRing) * Bs * D;
             float acc[PER];
 #pragma unroll
             for (int e = 0; e < PER; ++e) acc[e] = 0.0f;
@@ -1021,11 +1029,13 @@ cudaError_t launch_summaries(const Plan &p, const void *K, const float *cb, void
     unsigned long long *cnt = (unsigned long long *)ws_ptr(p, ws, kRegCounters);
     cudaError_t e = cudaMemsetAsync(cnt, 0, kCntN * 8, s);
     if (e != cudaSuccess) return e;
-    // two blocks per warp when their rows fit in 64 KB per CTA, else one; blocks
-    // too large to stage take the plain kernel (one CTA per block)
-    const size_t block_bytes = (size_t)c.Bs * c.d * p.es;
-    const int bpw = 4 * 2 * block_bytes <= 64 * 1024 ? 2 : 1;
-    const size_t smem = summary_smem(c.M, c.C, c.Bs, c.d, (int)p.es, bpw);
+    // blocks per warp: about one wave of 3 CTAs per SM over all blocks; blocks
+    // too large to stage twice per warp take the plain kernel (one CTA per block)
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const long long blocks = (long long)c.B * c.H * p.nb;
+    const int bpw = (int)std::min<long long>(16, std::max<long long>(1, (blocks + 12ll * sms - 1) / (12ll * sms)));
+    const size_t smem = summary_smem(c.M, c.C, c.Bs, c.d, (int)p.es);
     if (smem > 160 * 1024) {
         dim3 g0(p.nb, c.H, c.B);
         if (c.dtype == MONO_BF16)
