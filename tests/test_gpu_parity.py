@@ -132,6 +132,11 @@ def test_tensor_core_attention_shapes(d, Bs, L, R, S):
     full_check(Run(cfg, seed=10 + d + Bs + L))
 
 
+def test_tensor_core_attention_more_slices_than_one_launch_group():
+    # 2 x 130 = 260 (b, h) slices: the attention runs as a launch pair over 256 slices, then one over 4
+    full_check(Run(small(B=2, H=130, S=256, Bs=64, C=8, cap=3, dtype="bf16"), seed=23))
+
+
 def test_tensor_core_attention_edge_cases():
     full_check(Run(small(S=640, Bs=64, R=0, E=0, dtype="bf16"), seed=20))           # local only
     full_check(Run(small(S=640, Bs=64, x="zeros", dtype="bf16"), seed=21))          # all ties
