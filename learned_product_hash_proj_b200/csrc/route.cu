@@ -95,7 +95,7 @@ __global__ void __launch_bounds__(128) k_summary_assign_w(const T *__restrict__ 
     float *s_cbT = sm;                              // [dm][M*C]: element i of codeword mc at i * MC + mc
     float *s_kb = s_cbT + MC * dm;                  // [4][D]
     float *s_sc = s_kb + 4 * D;                     // [4][M*C]
-    T *s_rows = (T *)(((uintptr_t)(s_sc + 4 * MC) + 15) & ~(uintptr_t)15);  // [4][bpw][Bs*D] staged rows
+    T *s_rows = (T *)(((uintptr_t)(s_sc + 4 * MC) + 15) & ~(uintptr_t)15);  // [4][kSumRing][Bs*D] staged rows
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int h = blockIdx.y, b = blockIdx.z;
     const int nb = S / Bs;

@@ -142,3 +142,36 @@ def test_decode_cache_layout_and_argument_checks(mono):
     # the decode path scores every address of a query: C^M <= 4096
     big = mono.Plan(synth.config("stress"))
     assert lib.mono_decode_cache_bytes(big.handle, ctypes.byref(n)) == 2
+
+
+def test_backward_workspace_and_argument_checks(mono):
+    lib = mono.lib()
+    sizes = []
+    for S in (1024, 2048):
+        p = mono.Plan(synth.config("pr1", S=S))
+        n = ctypes.c_size_t()
+        assert lib.mono_backward_workspace_bytes(p.handle, ctypes.byref(n)) == 0
+        assert n.value % 256 == 0
+        sizes.append(n.value)
+    assert sizes[1] > sizes[0] > 0
+    assert lib.mono_backward_workspace_bytes(None, ctypes.byref(ctypes.c_size_t())) == 3
+    p = mono.Plan(synth.config("pr1"))
+    fake = ctypes.c_void_p(1 << 20)            # never dereferenced: validation fails first
+    odd16 = ctypes.c_void_p((1 << 20) + 8)     # not 16-byte aligned
+    odd256 = ctypes.c_void_p((1 << 20) + 16)   # not 256-byte aligned
+    N = None
+    f6 = [fake] * 6
+    # mono_backward(plan, x, Wq, Wk, Wv, Wo, sel, ddelta, dx, dWq, dWk, dWv, dWo, ws, bws, stream)
+    assert lib.mono_backward(None, *f6, fake, *[fake] * 5, fake, fake, N) == 3                 # NULL plan
+    assert lib.mono_backward(p.handle, *f6, fake, *[fake] * 5, N, fake, N) == 4                # no workspace
+    assert lib.mono_backward(p.handle, *f6, fake, *[fake] * 5, fake, N, N) == 4                # no bwd workspace
+    assert lib.mono_backward(p.handle, *f6, fake, *[fake] * 5, fake, odd256, N) == 7           # bws %256
+    assert lib.mono_backward(p.handle, *f6, fake, odd16, *[fake] * 4, fake, fake, N) == 7      # misaligned dx
+    assert lib.mono_backward(p.handle, fake, fake, fake, fake, fake, N, fake, *[fake] * 5, fake, fake, N) == 3  # sel
+    # mono_attend_backward(plan, Q, K, V, sel, dO, dQ, dK, dV, bws, stream)
+    assert lib.mono_attend_backward(p.handle, *[fake] * 8, N, N) == 4                           # no bwd workspace
+    assert lib.mono_attend_backward(p.handle, fake, fake, fake, fake, fake, N, fake, fake, fake, N) == 3  # NULL dQ
+    assert lib.mono_attend_backward(p.handle, fake, odd16, *[fake] * 6, fake, N) == 7         # misaligned K
+    # empty batch: nothing to do, nothing launched
+    pe = mono.Plan(synth.config("pr1", B=0))
+    assert lib.mono_backward(pe.handle, *f6, fake, *[fake] * 5, fake, fake, N) == 0
