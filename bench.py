@@ -69,7 +69,8 @@ def describe(cfg) -> str:
 
 
 # ---------------------------------------------------------------------------
-# algorithmic bytes (per call) of each stage; see DESIGN.md "Measurement"
+# algorithmic bytes (per call) of each stage: what the stage must read and
+# write at least once, each tensor counted once per call
 # ---------------------------------------------------------------------------
 def algorithmic_bytes(cfg) -> dict:
     es = 2 if cfg.dtype == "bf16" else 4
