@@ -208,12 +208,9 @@ void *tensor_map_encoder() {
 namespace {
 
 cudaError_t launch(const TmaMaps &maps, const Epi &epi, int nz, int K, cudaStream_t s) {
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(k_gemm_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    // set on every call: the attribute belongs to the current device, and a host call is cheap next to the GEMM
+    cudaError_t e = cudaFuncSetAttribute(k_gemm_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    if (e != cudaSuccess) return e;
     dim3 grid(epi.N / BN, (epi.M + BM - 1) / BM, nz);
     k_gemm_tc<<<grid, 192, SMEM_BYTES, s>>>(maps, epi, K);
     count_launches(1);
@@ -463,13 +460,9 @@ cudaError_t gemm_grad_tc(int M, int N, int K, int nsrc, int ngroups, const void 
     if (split > 1 && !accumulate)
         for (int i = 0; i < ngroups; ++i)
             if ((e = cudaMemsetAsync(C[i], 0, (size_t)M * N * sizeof(float), s)) != cudaSuccess) return e;
-    static bool attr_set = false;
-    if (!attr_set) {
-        if ((e = cudaFuncSetAttribute(k_gemm_grad_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES)) !=
-            cudaSuccess)
-            return e;
-        attr_set = true;
-    }
+    if ((e = cudaFuncSetAttribute(k_gemm_grad_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES)) !=
+        cudaSuccess)
+        return e;
     dim3 grid((N + BN - 1) / BN, (M + BM - 1) / BM, ngroups * split);
     k_gemm_grad_tc<<<grid, 192, SMEM_BYTES, s>>>(maps, g);
     count_launches(1);
