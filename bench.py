@@ -250,26 +250,49 @@ def run_ours(args):
     window_gbs = ab["route_attend"] / (ra / 1e3) / 1e9
     traffic = load_traffic(dom, cfg)
 
-    # end to end through the public API with host buffers: pinned x -> device, forward, delta -> host
+    # end to end through the public API with host buffers, as a serving loop runs it: step i's x goes from
+    # pinned host memory to the device on a copy stream while step i-1 computes, and step i-1's delta comes back
+    # on another while step i computes (device x and delta double-buffered; events order each buffer's reuse).
+    # Every step's copies and its L2 flush are inside the timed region, which spans the whole loop.
     x_host = torch.from_numpy(inp["x"]).to(tdt).pin_memory()
-    d_host = torch.empty(delta.shape, dtype=tdt).pin_memory()
-    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    d_host = [torch.empty(delta.shape, dtype=tdt).pin_memory() for _ in range(2)]
+    xb = [x, torch.empty_like(x)]
+    db = [torch.empty_like(delta) for _ in range(2)]
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev = lambda: torch.cuda.Event()
+    in_done, comp_done, out_done = [ev(), ev()], [ev(), ev()], [ev(), ev()]
 
-    def e2e_step(pair):
-        flush.zero_()
-        pair[0].record(stream)
-        x.copy_(x_host, non_blocking=True)
-        mono.forward(plan, x, Wq, Wk, Wv, Wo, cb, delta, ws, stream=stream)
-        d_host.copy_(delta, non_blocking=True)
-        pair[1].record(stream)
+    def e2e_run(n):
+        for i in range(n):
+            j = i % 2
+            with torch.cuda.stream(s_in):
+                if i >= 2:
+                    s_in.wait_event(comp_done[j])             # step i-2 no longer reads xb[j]
+                xb[j].copy_(x_host, non_blocking=True)
+                in_done[j].record(s_in)
+            stream.wait_event(in_done[j])
+            if i >= 2:
+                stream.wait_event(out_done[j])                # step i-2's delta has left db[j]
+            flush.zero_()
+            mono.forward(plan, xb[j], Wq, Wk, Wv, Wo, cb, db[j], ws, stream=stream)
+            comp_done[j].record(stream)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(comp_done[j])
+                d_host[j].copy_(db[j], non_blocking=True)
+                out_done[j].record(s_out)
 
-    for _ in range(max(1, min(args.warmup, 3))):
-        e2e_step((torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)))
+    e2e_run(max(2, min(args.warmup, 3)))
     torch.cuda.synchronize()
-    for k in range(args.steps):
-        e2e_step(e2e_ev[k])
+    e2e_t0, e2e_t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2e_t0.record(s_in)
+    stream.wait_event(e2e_t0)
+    e2e_run(args.steps)
+    e2e_t1.record(s_out)
     torch.cuda.synchronize()
-    e2e_ms = dist.reduce_max([mean([a.elapsed_time(b) for a, b in e2e_ev])], device=dev)[0]
+    # the pipeline delivered the staged pass's result (same inputs, deterministic kernels)
+    if not torch.equal(d_host[(args.steps - 1) % 2].to(dev), delta):
+        raise RuntimeError("end-to-end pipeline: delta differs from the staged pass")
+    e2e_ms = dist.reduce_max([e2e_t0.elapsed_time(e2e_t1) / args.steps], device=dev)[0]
 
     decode = measure_decode(plan, cfg, K, V, inp, tdt, dev, stream, hbm) if not args.no_decode else None
     backward = measure_backward(plan, cfg, x, Wq, Wk, Wv, Wo, sel, ws, tdt, dev, stream) \
@@ -304,7 +327,9 @@ def run_ours(args):
                                       "frac": window_gbs / hbm, "algorithmic_bytes": ab["route_attend"]},
             "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": UNIT, "api": "mono_forward",
                     "h2d_bytes_per_step": int(x_host.numel() * x_host.element_size()),
-                    "d2h_bytes_per_step": int(d_host.numel() * d_host.element_size()), "ms_per_step": e2e_ms},
+                    "d2h_bytes_per_step": int(d_host[0].numel() * d_host[0].element_size()), "ms_per_step": e2e_ms,
+                    "pipeline": "H2D of step i and D2H of step i-1 on two copy streams overlap step i's forward; "
+                                "timed from the first copy-in to the last copy-out, L2 flush per step included"},
             "gpu_launches": int(launches),
             "clocks": clocks,
             "routing": {"overflow_total": st["overflow_total"], "mean_remote": st["mean_remote"],
