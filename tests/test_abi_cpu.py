@@ -175,3 +175,25 @@ def test_backward_workspace_and_argument_checks(mono):
     # empty batch: nothing to do, nothing launched
     pe = mono.Plan(synth.config("pr1", B=0))
     assert lib.mono_backward(pe.handle, *f6, fake, *[fake] * 5, fake, fake, N) == 0
+
+
+def test_binding_refuses_host_tensors(mono):
+    # no CPU fallback anywhere in the product path: host tensors are an error, before the library is called
+    import torch
+    cfg = synth.config("pr1")
+    p = mono.Plan(cfg)
+    dt = p.dtype
+    hd = cfg.H * cfg.d
+    x = torch.zeros((cfg.B, cfg.S, cfg.W), dtype=dt)
+    W = torch.zeros((hd, cfg.W), dtype=dt)
+    Wo = torch.zeros((cfg.W, hd), dtype=dt)
+    cb = torch.zeros((cfg.H, cfg.M, cfg.C, cfg.d // cfg.M), dtype=torch.float32)
+    ws = torch.zeros(p.workspace_bytes, dtype=torch.uint8)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        mono.forward(p, x, W, W, W, Wo, cb, torch.zeros_like(x), ws)
+    sel = torch.zeros((cfg.B, cfg.H, cfg.S, cfg.R), dtype=torch.int32)
+    f32 = dict(dtype=torch.float32)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        mono.backward(p, x, W, W, W, Wo, sel, x, torch.zeros(x.shape, **f32), torch.zeros(W.shape, **f32),
+                      torch.zeros(W.shape, **f32), torch.zeros(W.shape, **f32), torch.zeros(Wo.shape, **f32), ws,
+                      torch.zeros(256, dtype=torch.uint8))
