@@ -244,11 +244,14 @@ def run_ours(args):
     # reported as a stage.
     hbm, bf16_tf, peak_kind = peaks()
     ab = algorithmic_bytes(cfg)
-    single_kernel_stages = {"summaries": "k_summary_assign_w", "lists": "k_posting_dense", "queries": "k_probe_m2"}
+    single_kernel_stages = {"summaries": "k_summary_assign_w",
+                            "lists": "k_posting_dense" if cfg.A <= 4096 else "k_posting_build",
+                            "queries": "k_probe_m2" if cfg.M == 2 else "k_probe_rerank"}
     dom = max(single_kernel_stages, key=lambda n: stage[n])
     achieved = ab[dom] / (stage[dom] / 1e3) / 1e9
     window_gbs = ab["route_attend"] / (ra / 1e3) / 1e9
     traffic = load_traffic(dom, cfg)
+    projections = projection_roofline(cfg, stage)
 
     # end to end through the public API with host buffers, as a serving loop runs it: step i's x goes from
     # pinned host memory to the device on a copy stream while step i-1 computes, and step i-1's delta comes back
@@ -325,6 +328,8 @@ def run_ours(args):
                          "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)"},
             "route_attend_roofline": {"bound": "hbm", "achieved": window_gbs, "peak": hbm, "unit": "GB/s",
                                       "frac": window_gbs / hbm, "algorithmic_bytes": ab["route_attend"]},
+            "projections": projections,
+            "proj_tensor_frac": projections["qkv"]["frac"],
             "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": UNIT, "api": "mono_forward",
                     "h2d_bytes_per_step": int(x_host.numel() * x_host.element_size()),
                     "d2h_bytes_per_step": int(d_host[0].numel() * d_host[0].element_size()), "ms_per_step": e2e_ms,
@@ -468,6 +473,42 @@ def measure_backward(plan, cfg, x, Wq, Wk, Wv, Wo, sel, ws, tdt, dev, stream, st
                                         "fp32 lanes x clock (148 x 128 x 2 x 1.965 GHz) for the rest"}}
 
 
+def projection_roofline(cfg, stage: dict) -> dict:
+    """Tensor-pipe fraction of the projection GEMMs (outside the route+attend metric): algorithmic flops
+    (2 M N K per GEMM: Q/K/V = 3 GEMMs of B*S x H*d x W, the output projection one of B*S x W x H*d) over the
+    stage's event time, against the measured sustained bf16 peak (the GEMMs run inside a long step)."""
+    tpeak, tsrc = bf16_sustained_peak()
+    gemm = 2.0 * cfg.B * cfg.S * cfg.H * cfg.d * cfg.W
+    out = {}
+    for name, st, fl in (("qkv", "project", 3 * gemm), ("out", "out_project", gemm)):
+        tf = fl / (stage[st] / 1e3) / 1e12
+        out[name] = {"bound": "tensor", "achieved": tf, "peak": tpeak, "unit": "TFLOP/s", "frac": tf / tpeak,
+                     "algorithmic_flops": fl, "ms": stage[st], "kernel": "k_gemm_tc" if cfg.dtype == "bf16"
+                     else "k_gemm_simt"}
+    out["peak_source"] = f"{tsrc} bf16_tflops_sustained (MEASURED_PEAKS.json)"
+    if cfg.dtype != "bf16":
+        out["note"] = "fp32 storage runs the SIMT GEMM; the bf16 tensor peak is a reference only"
+    return out
+
+
+def host_cpu() -> dict:
+    """The host's CPU model and how many cores this process may use (for the CPU-baseline record)."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    try:
+        usable = len(os.sched_getaffinity(0))
+    except AttributeError:
+        usable = os.cpu_count()
+    return {"cpu_model": model, "nproc": usable}
+
+
 def load_traffic(stage: str, cfg):
     """DRAM read+write bytes per launch of the stage's kernel, from the committed ncu summary
     (profiles/traffic.json), or None when the summary does not cover this workload."""
@@ -544,20 +585,29 @@ def oracle_route_attend(cfg, Q1, K1, V1, cb1, qidx=None):
 
 
 def cpu_baseline(cfg, inp, Q, K, V, n_heads: int = 4):
-    """The oracle's route+attend on the GPU's Q/K/V for `n_heads` full heads, extrapolated to all heads."""
+    """The oracle's route+attend on the GPU's Q/K/V for `n_heads` heads of batch 0, extrapolated to the whole
+    workload: each head's summaries and lists in full, and the route+attend of all its queries, or, where the
+    oracle's sort of the whole address grid per query makes that slow (C^M > 256), of a seeded sample of about
+    4e6 / C^M queries (at least 256), scaled by S / sample.  About 4-15 s of single-threaded work."""
     import oracle
     oracle.build()
-    tot = 0.0
     n_heads = min(n_heads, cfg.H)
+    n_q = cfg.S if cfg.A <= 256 else min(cfg.S, max(256, int(4e6 // cfg.A)))
+    qidx = None if n_q == cfg.S else np.sort(np.random.default_rng(5).choice(cfg.S, n_q, replace=False))
+    t_tab = t_q = 0.0
     for h in range(n_heads):
         sl = [t[0:1, h:h + 1].float().cpu().numpy() for t in (Q, K, V)]
         cb1 = np.ascontiguousarray(inp["codebooks"][h:h + 1])
-        a, b = oracle_route_attend(cfg, *sl, cb1)
-        tot += a + b
-    est = tot * (cfg.B * cfg.H) / n_heads
-    return {"value": cfg.B * cfg.S / est, "unit": UNIT, "cores": 1, "kind": "oracle",
-            "sample": f"route+attend of heads 0..{n_heads - 1} of {cfg.H} (batch 0, all {cfg.S} queries each) on "
-                      f"the GPU's Q/K/V, {tot:.1f} s single-threaded, extrapolated x{cfg.B * cfg.H / n_heads:g}"}
+        a, b = oracle_route_attend(cfg, *sl, cb1, qidx=None if qidx is None else qidx.astype(np.int64))
+        t_tab += a
+        t_q += b
+    per_slice = (t_tab + t_q * cfg.S / n_q) / n_heads
+    est = per_slice * cfg.B * cfg.H
+    q_txt = f"all {cfg.S} queries" if qidx is None else f"a seeded sample of {n_q} of its {cfg.S} queries"
+    return {"value": cfg.B * cfg.S / est, "unit": UNIT, "cores": 1, "kind": "oracle", **host_cpu(),
+            "sample": f"heads 0..{n_heads - 1} of {cfg.H} (batch 0): summaries and lists of each slice in full, "
+                      f"route+attend of {q_txt}, on the GPU's Q/K/V; {t_tab + t_q:.1f} s single-threaded, "
+                      f"extrapolated linearly to {cfg.B} x {cfg.H} slices x {cfg.S} queries"}
 
 
 def run_reference(args):
@@ -595,7 +645,8 @@ def run_reference(args):
            "ms_per_step": 1e3 * statistics.mean(a + b for a, b in per_step), "higher_is_better": True,
            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
            "config": {"workload": describe(cfg)},
-           "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
+           "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample,
+                            **host_cpu()},
            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(out), flush=True)
 

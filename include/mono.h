@@ -125,6 +125,13 @@ enum mono_ws_region {
 
 /* Validate `cfg` and build an immutable host-side plan.  Writes the
  * workspace size in bytes the plan's calls need.  No device work.
+ * The parameters are those of the mixer the aitechinspire.com article
+ * describes ("Snapshot: key facts from the report": blocks, bounded causal
+ * posting lists, probed product addresses, a fixed number R of remote
+ * blocks plus guaranteed local blocks); the validity rules are the method's
+ * definition (S a whole number of blocks, R <= E, T <= C^M, cap >= 1, ...).
+ * `cfg` is read, not kept.  `*plan` is owned by the caller (free it with
+ * mono_plan_destroy); it is NULL on any error.
  * Returns MONO_OK, MONO_ERR_NULL, MONO_ERR_INVALID or MONO_ERR_UNSUPPORTED. */
 int mono_plan(const mono_config *cfg, mono_plan_t **plan, size_t *workspace_bytes);
 
@@ -179,15 +186,18 @@ int mono_route_queries(const mono_plan_t *plan, const void *Q, const float *code
  * optional forced; output sel.  The routing tables live in one array of
  * mono_route_static_capacity() bytes (16 MiB) that the library places in the
  * global memory of every GPU it is loaded on, for the life of the process.
- * The tables need B*H*nb*(d + 16) + B*H*4 bytes plus alignment; a larger
- * problem returns MONO_ERR_SCRATCH before anything is launched.
+ * The tables need B*H*nb*(4*d + 16) + B*H*4 + 64 bytes, each of the seven
+ * regions rounded up to 256 bytes (kbar is fp32); a larger problem returns
+ * MONO_ERR_SCRATCH before anything is launched.
  * The first call on a device looks the array's device address up
  * (cudaGetSymbolAddress, with that device current) and caches it, so make
  * the first call on each device before any stream capture.  All calls on a
  * device share the array: calls that overlap on the GPU (other streams or
  * threads) race and must be serialised by the caller.  Each call clears the
- * statistics counters it uses and overwrites the tables.  No memory is
- * allocated by this entry point. */
+ * statistics counters it uses and overwrites the tables; mono_stats with a
+ * NULL workspace reads them back.  The cached address is not valid across
+ * cudaDeviceReset: do not call this entry point on a device after resetting
+ * it in the same process.  No memory is allocated by this entry point. */
 int mono_route_static(const mono_plan_t *plan, const void *Q, const void *K, const float *codebooks,
                       const int32_t *forced, int32_t *sel, void *stream);
 
@@ -203,12 +213,24 @@ size_t mono_route_static_capacity(void);
 int mono_attend(const mono_plan_t *plan, const void *Q, const void *K, const void *V,
                 const int32_t *sel, void *O, void *workspace, void *stream);
 
-/* Output projection delta = O Wo^T. */
+/* Output projection delta = O Wo^T: the last step of the stateless
+ * [batch, sequence, width] -> attention-delta mixer (aitechinspire.com
+ * article, "Snapshot: key facts from the report"; the host model adds the
+ * residual).  O [B,S,H*d] and Wo [W,H*d] in dtype; delta [B,S,W] in dtype,
+ * rounded once from the fp32 accumulation.  The workspace holds the device
+ * error word that a bounded wait of the tensor-core kernel may set. */
 int mono_out_project(const mono_plan_t *plan, const void *O, const void *Wo, void *delta,
                      void *workspace, void *stream);
 
-/* The whole mixer: mono_project, mono_route, mono_attend and
- * mono_out_project on workspace-resident Q, K, V, sel and O. */
+/* The whole mixer (aitechinspire.com article, "Snapshot: key facts from
+ * the report" and "What's the core idea?": after RoPE, blocks go to bounded
+ * causal posting lists; each query probes product addresses, reranks,
+ * selects R remote blocks, adds its guaranteed local blocks and runs exact
+ * causal softmax over those tokens; the stateless mixer returns an attention
+ * delta): mono_project, mono_route, mono_attend and mono_out_project on
+ * workspace-resident Q, K, V, sel and O.  Inputs x [B,S,W], weights,
+ * codebooks, optional forced; output delta [B,S,W].  The workspace keeps
+ * every intermediate (mono_workspace_region) for mono_stats and debugging. */
 int mono_forward(const mono_plan_t *plan, const void *x, const void *Wq, const void *Wk,
                  const void *Wv, const void *Wo, const float *codebooks, const int32_t *forced,
                  void *delta, void *workspace, void *stream);
@@ -323,8 +345,14 @@ int mono_backward(const mono_plan_t *plan, const void *x, const void *Wq, const 
                   float *dWv, float *dWo, void *workspace, void *bwd_workspace, void *stream);
 
 /* Synchronise `stream` and read the routing statistics and the device error
- * word of the last mono_route / mono_forward on `workspace`.  Returns
- * MONO_ERR_DEVICE if a kernel recorded an error. */
+ * word of the last mono_route / mono_forward on `workspace`: the quantities
+ * the aitechinspire.com article ("Practical notes for tinkerers") asks a user
+ * to log next to accuracy -- selected remote blocks per query and posting
+ * overflow counts.  With workspace == NULL the statistics and error word of
+ * the last mono_route_static call on the current device are read instead
+ * (from that entry point's fixed array, with the same plan).  `out` is
+ * caller-owned host memory.  Returns MONO_ERR_DEVICE if a kernel recorded an
+ * error. */
 int mono_stats(const mono_plan_t *plan, const void *workspace, void *stream, mono_stats_t *out);
 
 /* Static description of a status code. */

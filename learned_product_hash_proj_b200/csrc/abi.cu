@@ -260,10 +260,18 @@ int mono_forward(const mono_plan_t *plan, const void *x, const void *Wq, const v
 
 int mono_stats(const mono_plan_t *plan, const void *workspace, void *stream, mono_stats_t *out) {
     if (!plan || !out) return MONO_ERR_NULL;
-    if (!workspace) return MONO_ERR_WORKSPACE;
-    const Plan &p = plan->p;
     memset(out, 0, sizeof(*out));
-    if (empty(&p)) return MONO_OK;
+    if (empty(&plan->p)) return MONO_OK;
+    // NULL workspace: the tables mono_route_static left in its fixed array
+    Plan rp;
+    const bool from_static = workspace == nullptr;
+    if (from_static) {
+        void *base = nullptr;
+        const int st = route_static_tables(plan->p, &base, &rp);
+        if (st != MONO_OK) return st;
+        workspace = base;
+    }
+    const Plan &p = from_static ? rp : plan->p;
     cudaStream_t s = (cudaStream_t)stream;
     if (cudaStreamSynchronize(s) != cudaSuccess) return MONO_ERR_CUDA;
     unsigned long long cnt[kCntN];

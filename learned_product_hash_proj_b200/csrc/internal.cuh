@@ -113,6 +113,10 @@ bool gemm_grad_tc_supported(int M, int N, int K, bool a_mn, bool b_mn);
 cudaError_t gemm_grad_tc(int M, int N, int K, int nsrc, int ngroups, const void *const *A, bool a_mn,
                          const void *const *B, bool b_mn, float *const *C, bool accumulate,
                          unsigned long long *counters, cudaStream_t s);
+// The routing regions that mono_route_static uses for plan `p` (offsets in
+// rp->off relative to *base, the device address of its fixed array on the
+// current device); MONO_ERR_SCRATCH if they do not fit.
+int route_static_tables(const Plan &p, void **base, Plan *rp);
 cudaError_t launch_attend_tc(const Plan &p, const void *Q, const void *K, const void *V, const int32_t *sel, void *O,
                              void *ws, cudaStream_t s);
 

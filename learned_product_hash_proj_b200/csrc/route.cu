@@ -1073,10 +1073,24 @@ cudaError_t launch_lists(const Plan &p, void *ws, cudaStream_t s) {
     const int32_t *addr = (const int32_t *)ws_ptr(p, ws, kRegAddr);
     int32_t *ids = (int32_t *)ws_ptr(p, ws, kRegPostIds), *saddr = (int32_t *)ws_ptr(p, ws, kRegPostAddr);
     int32_t *rank = (int32_t *)ws_ptr(p, ws, kRegPostRank), *ov = (int32_t *)ws_ptr(p, ws, kRegOverflow);
-    if (p.A <= kDenseA)
-        k_posting_dense<<<g2, 1024, (size_t)p.nb * 8, s>>>(addr, ids, saddr, rank, ov, p.nb, c.cap, c.H, (int)p.A);
-    else
-        k_posting_build<<<g2, 1024, p.nb * sizeof(int32_t), s>>>(addr, ids, saddr, rank, ov, p.nb, c.cap, c.H);
+    // dynamic shared memory beyond the default 48 KB (with the kernels' static arrays) needs the opt-in
+    // attribute: up to 8192 blocks take 64 KB of addresses and ranks in the dense kernel
+    cudaError_t e = cudaSuccess;
+    if (p.A <= kDenseA) {
+        const size_t dyn = (size_t)p.nb * 8;
+        if (dyn + sizeof(int) * (kDenseA + 64) > 48 * 1024 &&
+            (e = cudaFuncSetAttribute(k_posting_dense, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn)) !=
+                cudaSuccess)
+            return e;
+        k_posting_dense<<<g2, 1024, dyn, s>>>(addr, ids, saddr, rank, ov, p.nb, c.cap, c.H, (int)p.A);
+    } else {
+        const size_t dyn = (size_t)p.nb * sizeof(int32_t);
+        if (dyn + sizeof(int) * 32 > 48 * 1024 &&
+            (e = cudaFuncSetAttribute(k_posting_build, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn)) !=
+                cudaSuccess)
+            return e;
+        k_posting_build<<<g2, 1024, dyn, s>>>(addr, ids, saddr, rank, ov, p.nb, c.cap, c.H);
+    }
     count_launches(1);
     return cudaGetLastError();
 }

@@ -18,7 +18,9 @@
 // before any stream capture begins.  Every call on a device shares the one
 // array and leaves its tables there: calls that overlap on the GPU (different
 // streams, or other threads) race with each other and must be serialised by
-// the caller.  The statistics counters are cleared by every call.
+// the caller.  The statistics counters are cleared by every call; mono_stats
+// with a NULL workspace reads them (and the overflow counts) back from here.
+// The cached address does not survive cudaDeviceReset.
 #include <mutex>
 
 #include "internal.cuh"
@@ -69,6 +71,12 @@ int scratch_address(void **out) {
 }
 
 }  // namespace
+
+int route_static_tables(const Plan &p, void **base, Plan *rp) {
+    if (route_layout(p, rp) > kStaticRouteScratchBytes) return MONO_ERR_SCRATCH;
+    return scratch_address(base);
+}
+
 }  // namespace mono
 
 using namespace mono;
@@ -86,9 +94,8 @@ int mono_route_static(const mono_plan_t *plan, const void *Q, const void *K, con
     if (((uintptr_t)Q | (uintptr_t)K | (uintptr_t)codebooks | (uintptr_t)sel) % 16) return MONO_ERR_ALIGN;
     if (forced && (uintptr_t)forced % 4) return MONO_ERR_ALIGN;
     Plan rp;
-    if (route_layout(p, &rp) > kStaticRouteScratchBytes) return MONO_ERR_SCRATCH;
     void *scratch = nullptr;
-    int st = scratch_address(&scratch);
+    int st = route_static_tables(p, &scratch, &rp);
     if (st != MONO_OK) return st;
     cudaStream_t s = (cudaStream_t)stream;
     if (launch_summaries(rp, K, codebooks, scratch, s) != cudaSuccess) return MONO_ERR_CUDA;

@@ -204,3 +204,39 @@ def test_skewed_batch_full_size():
     run, info = sampled_check("stress", n_rows=48, n_queries=400)
     assert info["overflow"] > 0
     assert run.stats["overflow_total"] == info["overflow"]
+
+
+# ---------------------------------------------------------------------------
+# the largest block count a plan accepts (8192 blocks): the posting kernels'
+# shared memory then passes the default 48 KB (dense kernel: 64 KB of
+# addresses and ranks).  Routing only, on seeded Q/K, against the oracle in full.
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("M,C,T", [(2, 8, 4), (4, 16, 16)])
+def test_routing_at_the_largest_block_count(M, C, T):
+    from learned_product_hash_proj_b200 import mono
+    cfg = synth.Config(B=1, S=8192 * 32, W=64, H=1, d=64, Bs=32, L=2, R=2, E=5, M=M, C=C, T=T, cap=1,
+                       dtype="bf16")
+    rng = np.random.default_rng(40 + M)
+    shape = (cfg.B, cfg.H, cfg.S, cfg.d)
+    Qn = synth.round_bf16(rng.standard_normal(shape, dtype=np.float32))
+    Kn = synth.round_bf16(rng.standard_normal(shape, dtype=np.float32) * 3.0)
+    cb = synth.make_codebooks(cfg, 40 + M)
+    plan = mono.Plan(cfg)
+    ws = plan.workspace()
+    Q, K = (torch.from_numpy(a).to(torch.bfloat16).cuda() for a in (Qn, Kn))
+    sel = torch.empty((cfg.B, cfg.H, cfg.S, cfg.R), dtype=torch.int32, device="cuda")
+    mono.route(plan, Q, K, torch.from_numpy(cb).cuda(), sel, ws)
+    torch.cuda.synchronize()
+    st = mono.stats(plan, ws)
+    kbar, addr, _ = oracle.summary_assign(cfg, Kn, cb)
+    np.testing.assert_array_equal(to_np(plan.region(ws, "addr")), addr, err_msg="addresses")
+    ids, saddr, rank, ov = oracle.posting(cfg, addr)
+    np.testing.assert_array_equal(to_np(plan.region(ws, "post_ids")), ids, err_msg="posting ids")
+    np.testing.assert_array_equal(to_np(plan.region(ws, "post_rank")), rank, err_msg="posting ranks")
+    np.testing.assert_array_equal(to_np(plan.region(ws, "overflow")).astype(np.int64), ov, err_msg="overflow")
+    assert st["overflow_total"] == int(ov.sum()) > 0
+    # every 7th query; the oracle sorts the whole grid per query, so the 65536-address grid gets 400
+    qidx = np.arange(0, cfg.S, 7, dtype=np.int64) if cfg.A <= 4096 else \
+        np.sort(rng.choice(cfg.S, 400, replace=False)).astype(np.int64)
+    osel, *_ = oracle.route_queries(cfg, Qn, kbar, cb, addr, qidx=qidx)
+    np.testing.assert_array_equal(to_np(sel).reshape(-1, cfg.R)[qidx], osel, err_msg="sel")

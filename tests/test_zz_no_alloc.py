@@ -8,7 +8,9 @@ caller workspace.  These tests call it through the C-ABI and check that it
 returns exactly what mono_route returns, on two calls in a row with different
 inputs (the array keeps the previous call's contents, so the second call
 checks that nothing stale leaks through), and that an oversize problem is
-refused before anything is launched.
+refused before anything is launched.  The statistics a static call leaves in
+the array (overflow counts, selection counters, device error word) are read
+back through mono_stats with no workspace and must equal mono_route's.
 
 This file is collected last so that a run stopping at the first failure has
 already run every other test; it also passes on its own in a fresh process.
@@ -70,6 +72,32 @@ def test_matches_mono_route_on_two_calls_in_a_row(mono, name):
         assert rc == 0, mono.STATUS.get(rc, rc)
         torch.cuda.synchronize()
         assert torch.equal(got, ref), f"seed {seed}: {(got != ref).sum().item()} selections differ"
+
+
+def test_stats_of_the_static_call_match_mono_stats(mono):
+    # Routing statistics and the device error word of a static call stay in the fixed array; mono_stats reads
+    # them back when it is given no workspace.  Every other block of K is zero, so those blocks share address 0
+    # and the lists overflow: the overflow totals must agree with mono_route's, and so must the other counters.
+    cfg = synth.Config(B=2, S=2048, W=128, H=3, d=64, Bs=32, L=2, R=2, E=5, M=2, C=8, T=4, cap=3, dtype="bf16")
+    plan = mono.Plan(cfg)
+    ws = plan.workspace()
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    Q, K, cb = _inputs(cfg, 3)
+    blk = (torch.arange(cfg.S, device="cuda") // cfg.Bs) % 2 == 0
+    K = (K * blk.view(1, 1, cfg.S, 1).to(K.dtype)).contiguous()
+    ref = torch.empty((cfg.B, cfg.H, cfg.S, cfg.R), dtype=torch.int32, device="cuda")
+    mono.route(plan, Q, K, cb, ref, ws)
+    want = mono.stats(plan, ws)
+    assert want["overflow_total"] > 0
+    got_sel = torch.full_like(ref, -7)
+    for _ in range(2):
+        rc = mono.lib().mono_route_static(plan.handle, _p(Q), _p(K), _p(cb), None, _p(got_sel), stream)
+        assert rc == 0, mono.STATUS.get(rc, rc)
+        st = mono.Stats()
+        rc = mono.lib().mono_stats(plan.handle, None, stream, ctypes.byref(st))
+        assert rc == 0, mono.STATUS.get(rc, rc)
+        assert torch.equal(got_sel, ref)
+        assert st.as_dict() == {k: want[k] for k in st.as_dict()}
 
 
 def test_rejects_problems_beyond_the_fixed_array(mono):
