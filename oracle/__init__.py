@@ -13,6 +13,9 @@ Stages (each cites its source in ``mono_oracle.c``):
 * :func:`summary_assign`  block-mean key summary and product address (fp32)
 * :func:`posting`         bounded causal posting lists, overflow count
 * :func:`route_queries`   probe, union, causal filter, E cap, rerank (fp32)
+* :func:`summary_assign64`, :func:`route_queries64`
+                          the same routing decisions in fp64 (with margins), the
+                          precision-independent reference for the fp32 ones
 * :func:`attend`          exact softmax over the selected token set (fp64)
 * :func:`out_project`     delta = O Wo^T (fp64)
 * :func:`forward`         all of the above with the stored-precision rounding
@@ -63,9 +66,11 @@ def _load():
             lib.orc_posting.argtypes = [ctypes.POINTER(_Cfg), P, P, P, P, P]
             lib.orc_route_queries.argtypes = [ctypes.POINTER(_Cfg), P, P, P, P, P, L, P, P, P, P, P, P]
             lib.orc_attend.argtypes = [ctypes.POINTER(_Cfg), P, P, P, P, L, P, P]
+            lib.orc_summary_assign64.argtypes = [ctypes.POINTER(_Cfg), P, P, P, P, P]
+            lib.orc_route_queries64.argtypes = [ctypes.POINTER(_Cfg), P, P, P, P, P, L, P, P, P, P, P, P]
             lib.orc_out_project.argtypes = [ctypes.POINTER(_Cfg), P, P, L, P, P]
             for f in ("orc_project", "orc_summary_assign", "orc_posting", "orc_route_queries", "orc_attend",
-                      "orc_out_project"):
+                      "orc_out_project", "orc_summary_assign64", "orc_route_queries64"):
                 getattr(lib, f).restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -148,6 +153,48 @@ def route_queries(cfg, Q, kbar, codebooks, addr, forced=None, qidx=None):
                                0 if qidx is None else len(qidx), _p(qidx), _p(sel), _p(ncand), _p(pm), _p(rm),
                                _p(ign))
     _check(rc, "route_queries")
+    if qidx is None:
+        sel = sel.reshape(cfg.B, cfg.H, cfg.S, cfg.R)
+        ncand = ncand.reshape(cfg.B, cfg.H, cfg.S)
+        pm = pm.reshape(cfg.B, cfg.H, cfg.S)
+        rm = rm.reshape(cfg.B, cfg.H, cfg.S)
+    return sel, ncand, pm, rm, int(ign[0])
+
+
+def summary_assign64(cfg, K, codebooks):
+    """fp64 routing: kbar [B,H,nb,d] fp64, addr [B,H,nb] int32, assign margin [B,H,nb] fp64."""
+    lib = _load()
+    K = _c(K, np.float64)
+    cb = _c(codebooks, np.float64)
+    nb = cfg.S // cfg.Bs
+    kbar = np.empty((cfg.B, cfg.H, nb, cfg.d), np.float64)
+    addr = np.empty((cfg.B, cfg.H, nb), np.int32)
+    margin = np.empty((cfg.B, cfg.H, nb), np.float64)
+    _check(lib.orc_summary_assign64(ctypes.byref(_cfg(cfg)), _p(K), _p(cb), _p(kbar), _p(addr), _p(margin)),
+           "summary_assign64")
+    return kbar, addr, margin
+
+
+def route_queries64(cfg, Q, kbar, codebooks, addr, forced=None, qidx=None):
+    """fp64 routing: sel, ncand, probe margin (smallest neighbour gap among grid ranks 1..T+1), rerank
+    margin (smallest neighbour gap among rerank ranks 1..R+1), forced_ignored.  Shapes as route_queries."""
+    lib = _load()
+    Q = _c(Q, np.float64)
+    kbar = _c(kbar, np.float64)
+    cb = _c(codebooks, np.float64)
+    addr = _c(addr, np.int32)
+    forced = _c(forced, np.int32)
+    qidx = _c(qidx, np.int64)
+    n = cfg.B * cfg.H * cfg.S if qidx is None else len(qidx)
+    sel = np.empty((n, max(cfg.R, 0)), np.int32)
+    ncand = np.empty(n, np.int32)
+    pm = np.empty(n, np.float64)
+    rm = np.empty(n, np.float64)
+    ign = np.zeros(1, np.int64)
+    rc = lib.orc_route_queries64(ctypes.byref(_cfg(cfg)), _p(Q), _p(kbar), _p(cb), _p(addr), _p(forced),
+                                 0 if qidx is None else len(qidx), _p(qidx), _p(sel), _p(ncand), _p(pm), _p(rm),
+                                 _p(ign))
+    _check(rc, "route_queries64")
     if qidx is None:
         sel = sel.reshape(cfg.B, cfg.H, cfg.S, cfg.R)
         ncand = ncand.reshape(cfg.B, cfg.H, cfg.S)

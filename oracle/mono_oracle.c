@@ -27,6 +27,11 @@
  *     products as a chain of fused multiply-adds starting from +0.0f in
  *     ascending element order.  Build with -ffp-contract=off so that no other
  *     contraction happens.
+ *   - A second statement of the routing (orc_summary_assign64,
+ *     orc_route_queries64) takes the same decisions in fp64 from the stored
+ *     Q, K and codebooks: the plain-precision reference against which the
+ *     fp32 decisions are measured (they may differ only where an fp64 margin
+ *     is within fp32 rounding of zero).
  *
  * Every function returns 0 on success and a negative value on bad arguments.
  */
@@ -445,5 +450,192 @@ int orc_out_project(const orc_cfg *c, const double *O, const double *Wo, long nr
             delta[r * W + o] = acc;
         }
     }
+    return 0;
+}
+
+
+/* ------------------------------------------------------------------------ */
+/* Routing in fp64: the same steps as orc_summary_assign and                */
+/* orc_route_queries ([P2] Snapshot; [P4]/[P5] product addresses, strict     */
+/* capacity, causality), with every score, sum and mean in double precision */
+/* on the stored inputs upcast exactly.  The plain reading of the method:    */
+/* the decision each step names, taken on the real-valued scores as closely */
+/* as fp64 allows, with the same tie rules (lowest code, lowest address,     */
+/* lowest block id).  Margins are reported so that a caller can tell which  */
+/* decisions fp32 rounding could flip.                                       */
+/*                                                                            */
+/* orc_summary_assign64: kbar[j] = (sum of the block's keys) / Bs in fp64;   */
+/* code c_m = argmax_c <kbar_m, cw[h,m,c]>; margin = min over m of          */
+/* best - second best (+inf when C = 1).                                     */
+/* ------------------------------------------------------------------------ */
+static double dot64(const double *a, const double *b, int n)
+{
+    double acc = 0.0;
+    for (int i = 0; i < n; ++i) acc += a[i] * b[i];
+    return acc;
+}
+
+int orc_summary_assign64(const orc_cfg *c, const double *K, const double *cb,
+                         double *kbar, int32_t *addr, double *margin)
+{
+    if (!cfg_ok(c) || !K || !cb || !kbar || !addr) return -1;
+    const int S = c->S, d = c->d, Bs = c->Bs, M = c->M, C = c->C, dm = d / M;
+    const int nb = S / Bs;
+    for (long bh = 0; bh < (long)c->B * c->H; ++bh) {
+        const int h = (int)(bh % c->H);
+        for (int j = 0; j < nb; ++j) {
+            double *kb = kbar + (bh * nb + j) * d;
+            for (int i = 0; i < d; ++i) {
+                double acc = 0.0;
+                for (int t = j * Bs; t < (j + 1) * Bs; ++t) acc += K[(bh * S + t) * d + i];
+                kb[i] = acc / (double)Bs;
+            }
+            long a = 0;
+            double mg = INFINITY;
+            for (int m = 0; m < M; ++m) {
+                const double *cwm = cb + ((long)(h * M + m) * C) * dm;
+                int best_c = 0;
+                double best = dot64(kb + m * dm, cwm, dm);
+                double second = -INFINITY;
+                for (int cc = 1; cc < C; ++cc) {
+                    double sc = dot64(kb + m * dm, cwm + (long)cc * dm, dm);
+                    if (sc > best) { second = best; best = sc; best_c = cc; }
+                    else if (sc > second) second = sc;
+                }
+                if (C > 1 && best - second < mg) mg = best - second;
+                a = a * C + best_c;
+            }
+            addr[bh * nb + j] = (int32_t)a;
+            if (margin) margin[bh * nb + j] = mg;
+        }
+    }
+    return 0;
+}
+
+/* orc_route_queries64: per query-head, subspace scores and the grid score   */
+/* of every address in fp64; probes = the first T under (g desc, a asc);     */
+/* union in probe order over the kept lists (rebuilt from addr), causal      */
+/* filter j <= bq - L, E cap; rerank <q, kbar_j> in fp64 under (score desc,  */
+/* j asc), first R; forced block as in orc_route_queries; ascending, -1 pad. */
+/* probe_margin[n] = the smallest gap between neighbours among grid ranks    */
+/* 1..T+1 (the probe set and its order, which the E cap reads);              */
+/* rerank_margin[n] = the smallest gap between neighbours among rerank       */
+/* ranks 1..R+1 of the candidates (+inf where there is no such pair).        */
+typedef struct { double g; int32_t a; } ga64_pair;
+
+static int cmp_ga64(const void *x, const void *y)
+{
+    const ga64_pair *p = (const ga64_pair *)x, *q = (const ga64_pair *)y;
+    if (p->g != q->g) return p->g > q->g ? -1 : 1;
+    return (p->a > q->a) - (p->a < q->a);
+}
+
+static double min_gap(const ga64_pair *v, int n)
+{
+    double mg = INFINITY;
+    for (int k = 0; k + 1 < n; ++k)
+        if (v[k].g - v[k + 1].g < mg) mg = v[k].g - v[k + 1].g;
+    return mg;
+}
+
+int orc_route_queries64(const orc_cfg *c, const double *Q, const double *kbar, const double *cb,
+                        const int32_t *addr, const int32_t *forced, long nq, const int64_t *qidx,
+                        int32_t *sel, int32_t *ncand, double *probe_margin, double *rerank_margin,
+                        int64_t *forced_ignored)
+{
+    if (!cfg_ok(c) || !Q || !kbar || !cb || !addr || !sel) return -1;
+    const int S = c->S, H = c->H, d = c->d, Bs = c->Bs, M = c->M, C = c->C, dm = d / M;
+    const int nb = S / Bs, T = c->T, R = c->R, E = c->E, L = c->L, cap = c->cap;
+    const long A = n_addr(c);
+    if (T > A || R > 64) return -1;
+    const long total = (long)c->B * H * S;
+    const long n = qidx ? nq : total;
+
+    double *s = (double *)malloc(sizeof(double) * (size_t)M * C);
+    ga64_pair *grid = (ga64_pair *)malloc(sizeof(ga64_pair) * (size_t)A);
+    int32_t *list = (int32_t *)malloc(sizeof(int32_t) * (size_t)A * cap);
+    int32_t *len = (int32_t *)malloc(sizeof(int32_t) * (size_t)A);
+    int32_t *cand = (int32_t *)malloc(sizeof(int32_t) * (size_t)(E > 0 ? E : 1));
+    ga64_pair *rr = (ga64_pair *)malloc(sizeof(ga64_pair) * (size_t)(E > 0 ? E : 1));
+    if (!s || !grid || !list || !len || !cand || !rr) {
+        free(s); free(grid); free(list); free(len); free(cand); free(rr);
+        return -3;
+    }
+    long cur_bh = -1;
+    int64_t ignored = 0;
+    int bad = 0;
+    for (long qi = 0; qi < n; ++qi) {
+        long flat = qidx ? (long)qidx[qi] : qi;
+        if (flat < 0 || flat >= total) { bad = 1; break; }
+        long bh = flat / S;
+        int t = (int)(flat % S), h = (int)(bh % H);
+        if (bh != cur_bh) {
+            memset(len, 0, sizeof(int32_t) * (size_t)A);
+            for (int j = 0; j < nb; ++j) {
+                int32_t a = addr[bh * nb + j];
+                if (a < 0 || a >= A) { bad = 1; break; }
+                if (len[a] < cap) list[(long)a * cap + len[a]++] = j;
+            }
+            if (bad) break;
+            cur_bh = bh;
+        }
+        const double *q = Q + flat * d;
+        const int bq = t / Bs;
+        for (int m = 0; m < M; ++m)
+            for (int cc = 0; cc < C; ++cc)
+                s[m * C + cc] = dot64(q + m * dm, cb + ((long)(h * M + m) * C + cc) * dm, dm);
+        for (long a = 0; a < A; ++a) {
+            long rem = a;
+            int code[16];
+            for (int m = M - 1; m >= 0; --m) { code[m] = (int)(rem % C); rem /= C; }
+            double g = 0.0;
+            for (int m = 0; m < M; ++m) g += s[m * C + code[m]];
+            grid[a].g = g;
+            grid[a].a = (int32_t)a;
+        }
+        qsort(grid, (size_t)A, sizeof(ga64_pair), cmp_ga64);
+        if (probe_margin) probe_margin[qi] = min_gap(grid, (int)(T < A ? T + 1 : A));
+        int nc = 0;
+        for (int r = 0; r < T && nc < E; ++r) {
+            int32_t a = grid[r].a;
+            for (int k = 0; k < len[a] && nc < E; ++k) {
+                int32_t j = list[(long)a * cap + k];
+                if (j <= bq - L) cand[nc++] = j;
+            }
+        }
+        if (ncand) ncand[qi] = nc;
+        for (int k = 0; k < nc; ++k) {
+            rr[k].g = dot64(q, kbar + (bh * nb + cand[k]) * (long)d, d);
+            rr[k].a = cand[k];
+        }
+        qsort(rr, (size_t)nc, sizeof(ga64_pair), cmp_ga64);
+        if (rerank_margin) rerank_margin[qi] = R > 0 ? min_gap(rr, nc < R + 1 ? nc : R + 1) : INFINITY;
+        int ns = nc < R ? nc : R;
+        int32_t chosen[64];
+        for (int k = 0; k < ns; ++k) chosen[k] = rr[k].a;
+        if (forced && R > 0) {
+            int32_t f = forced[flat];
+            if (f >= 0) {
+                if (f <= bq - L) {
+                    int present = 0;
+                    for (int k = 0; k < ns; ++k) present |= (chosen[k] == f);
+                    if (!present) {
+                        if (ns < R) chosen[ns++] = f;
+                        else chosen[R - 1] = f;
+                    }
+                } else {
+                    ignored++;
+                }
+            }
+        }
+        for (int x = 1; x < ns; ++x)
+            for (int y = x; y > 0 && chosen[y - 1] > chosen[y]; --y) {
+                int32_t tmp = chosen[y]; chosen[y] = chosen[y - 1]; chosen[y - 1] = tmp;
+            }
+        for (int k = 0; k < R; ++k) sel[qi * R + k] = k < ns ? chosen[k] : -1;
+    }
+    free(s); free(grid); free(list); free(len); free(cand); free(rr);
+    if (bad) return -2;
+    if (forced_ignored) *forced_ignored = ignored;
     return 0;
 }

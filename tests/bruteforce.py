@@ -93,3 +93,82 @@ def route_bh(Q_bh, K_bh, cw_h, cfg, forced_bh=None):
         chosen = sorted(chosen)
         sel.append(chosen + [-1] * (R - len(chosen)))
     return addr, lists, overflow, sel
+
+
+# ---------------------------------------------------------------------------
+# The same rules on exact rationals: every sum, mean and dot product is exact
+# (fractions.Fraction on the stored binary32 values), so each decision is the
+# one the real-valued scores make.  The fp64 routing of the oracle must agree
+# with it wherever no margin is within fp64 rounding of zero.
+# ---------------------------------------------------------------------------
+from fractions import Fraction  # noqa: E402
+
+
+def _fr(v):
+    return Fraction(float(v))
+
+
+def _dot_exact(a, b):
+    return sum((x * y for x, y in zip(a, b)), Fraction(0))
+
+
+def route_bh_exact(Q_bh, K_bh, cw_h, cfg, forced_bh=None):
+    """Route every query of one (batch, head) exactly.  Returns (addr, overflow, sel, assign margins,
+    probe margins, rerank margins) with the margins defined as in the oracle's fp64 routing: per block the
+    smallest best-minus-second code score over the subspaces; per query the smallest gap between neighbours
+    among grid ranks 1..T+1 and among rerank ranks 1..R+1."""
+    S, d = Q_bh.shape
+    Bs, M, C, T, R, E, L, cap = cfg.Bs, cfg.M, cfg.C, cfg.T, cfg.R, cfg.E, cfg.L, cfg.cap
+    nb, dm = S // Bs, d // M
+    K = [[_fr(v) for v in row] for row in K_bh]
+    Q = [[_fr(v) for v in row] for row in Q_bh]
+    cw = [[[_fr(v) for v in cw_h[m][c]] for c in range(C)] for m in range(M)]
+    kb = [[sum((K[t][i] for t in range(j * Bs, (j + 1) * Bs)), Fraction(0)) / Bs for i in range(d)]
+          for j in range(nb)]
+    addr, amargin = [], []
+    for j in range(nb):
+        a, mg = 0, None
+        for m in range(M):
+            sc = [_dot_exact(kb[j][m * dm:(m + 1) * dm], cw[m][c]) for c in range(C)]
+            order = sorted(range(C), key=lambda c: (-sc[c], c))
+            a = a * C + order[0]
+            if C > 1:
+                gap = sc[order[0]] - sc[order[1]]
+                mg = gap if mg is None else min(mg, gap)
+        addr.append(a)
+        amargin.append(mg)
+    lists, overflow = {}, 0
+    for j, a in enumerate(addr):
+        bucket = lists.setdefault(a, [])
+        if len(bucket) < cap:
+            bucket.append(j)
+        else:
+            overflow += 1
+    sel, pmargin, rmargin = [], [], []
+    for t in range(S):
+        q = Q[t]
+        sub = [[_dot_exact(q[m * dm:(m + 1) * dm], cw[m][c]) for c in range(C)] for m in range(M)]
+        scored = sorted(((-sum((sub[m][combo[m]] for m in range(M)), Fraction(0)), address(combo, C))
+                         for combo in itertools.product(range(C), repeat=M)))
+        top = scored[:T + 1]
+        pmargin.append(min((top[k + 1][0] - top[k][0] for k in range(len(top) - 1)), default=None))
+        bq = t // Bs
+        cands = []
+        for _, a in scored[:T]:
+            for j in lists.get(a, []):
+                if j <= bq - L and len(cands) < E:
+                    cands.append(j)
+        ranked = sorted(((-_dot_exact(q, kb[j]), j) for j in cands))
+        rk = ranked[:R + 1] if R > 0 else []
+        rmargin.append(min((rk[k + 1][0] - rk[k][0] for k in range(len(rk) - 1)), default=None))
+        chosen = [j for _, j in ranked[:R]]
+        if forced_bh is not None and R > 0:
+            f = int(forced_bh[t])
+            if 0 <= f <= bq - L and f not in chosen:
+                if len(chosen) < R:
+                    chosen.append(f)
+                else:
+                    chosen[-1] = f
+        chosen = sorted(chosen)
+        sel.append(chosen + [-1] * (R - len(chosen)))
+    return addr, overflow, sel, amargin, pmargin, rmargin

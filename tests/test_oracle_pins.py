@@ -15,7 +15,7 @@ import pytest
 import torch
 
 import oracle
-from bruteforce import route_bh
+from bruteforce import route_bh, route_bh_exact
 from fp32_exact import F, add32, dot_chain32, fma32, round_f32
 from learned_product_hash_proj_b200 import synth
 
@@ -183,6 +183,70 @@ def test_routing_matches_independent_bruteforce(seed, dup):
             assert addr[0, h].tolist() == b_addr
             assert ov[0, h] == b_ov
             np.testing.assert_array_equal(sel[0, h], np.array(b_sel, np.int32))
+
+
+def _fp64_route(cfg, Qs, Ks, cb, forced=None):
+    kbar, addr, am = oracle.summary_assign64(cfg, Ks, cb)
+    ids, saddr, rank, ov = oracle.posting(cfg, addr)
+    sel, ncand, pm, rm, ign = oracle.route_queries64(cfg, Qs, kbar, cb, addr, forced=forced)
+    return addr, ov, sel, am, pm, rm
+
+
+def _close_margin(got, want):
+    # the oracle's fp64 margins against exact rationals: equal up to fp64 rounding of the scores
+    if want is None:
+        assert got == np.inf
+    else:
+        assert abs(got - float(want)) <= 1e-12 * max(1.0, abs(float(want))) + 1e-13
+
+
+@pytest.mark.parametrize("seed,dup", [(6, False), (7, True), (9, False)])
+def test_fp64_routing_matches_exact_rational_bruteforce(seed, dup):
+    # The fp64 statement of the routing takes every decision (code argmax, top-T addresses, E cap, top-R
+    # rerank, forced replacement) as the exact real-valued scores do, with the same tie rules, and reports
+    # the margins of those decisions.  Pinned against an enumerator on exact rationals.
+    cfg = tiny(S=96, Bs=8, H=2, L=2, R=2, E=3, T=3, cap=2)
+    inp = synth.make_inputs(cfg, seed=seed)
+    if dup:   # exact ties between codewords: the lowest code must win in both
+        inp["codebooks"][:, 0, 2] = inp["codebooks"][:, 0, 0]
+        inp["codebooks"][:, 1, 1] = inp["codebooks"][:, 1, 3]
+    forced = synth.make_forced(cfg, seed=seed, frac=0.3)
+    Qs, Ks, Vs = stored_qkv(cfg, inp)
+    for use_forced in (None, forced):
+        addr, ov, sel, am, pm, rm = _fp64_route(cfg, Qs, Ks, inp["codebooks"], forced=use_forced)
+        for h in range(cfg.H):
+            e_addr, e_ov, e_sel, e_am, e_pm, e_rm = route_bh_exact(
+                Qs[0, h], Ks[0, h], inp["codebooks"][h], cfg, None if use_forced is None else use_forced[0, h])
+            assert addr[0, h].tolist() == e_addr
+            assert ov[0, h] == e_ov
+            np.testing.assert_array_equal(sel[0, h], np.array(e_sel, np.int32))
+            for got, want in zip(am[0, h], e_am):
+                _close_margin(got, want)
+            for got, want in zip(pm[0, h], e_pm):
+                _close_margin(got, want)
+            for got, want in zip(rm[0, h], e_rm):
+                _close_margin(got, want)
+
+
+def test_fp32_and_fp64_routing_agree_when_the_arithmetic_is_exact():
+    # Small-integer Q, K and codewords keep every sum and product exact in fp32 and fp64 alike (the block
+    # mean divides by Bs = 8, a power of two): the two statements must then give identical addresses and
+    # selections, ties included, and both must equal the exact enumerator.
+    cfg = tiny(S=96, Bs=8, H=2, L=2, R=2, E=3, T=3, cap=2)
+    rng = np.random.default_rng(12)
+    Q = rng.integers(-3, 4, size=(1, cfg.H, cfg.S, cfg.d)).astype(np.float32)
+    K = rng.integers(-3, 4, size=(1, cfg.H, cfg.S, cfg.d)).astype(np.float32)
+    cb = rng.integers(-2, 3, size=(cfg.H, cfg.M, cfg.C, cfg.d // cfg.M)).astype(np.float32)
+    kbar32, addr32, _ = oracle.summary_assign(cfg, K, cb)
+    sel32, *_ = oracle.route_queries(cfg, Q, kbar32, cb, addr32)
+    addr64, ov64, sel64, *_ = _fp64_route(cfg, Q, K, cb)
+    np.testing.assert_array_equal(addr32, addr64)
+    np.testing.assert_array_equal(sel32, sel64)
+    assert (sel64 >= 0).any()
+    for h in range(cfg.H):
+        e_addr, e_ov, e_sel, *_ = route_bh_exact(Q[0, h], K[0, h], cb[h], cfg)
+        assert addr64[0, h].tolist() == e_addr
+        np.testing.assert_array_equal(sel64[0, h], np.array(e_sel, np.int32))
 
 
 def test_selected_blocks_lie_before_the_local_window():
