@@ -260,6 +260,27 @@ static int cmp_ga(const void *x, const void *y)
     return (p->a > q->a) - (p->a < q->a);
 }
 
+/* The first k entries of v[0..n) under the order cmp, in that order: one scan
+ * that keeps the best k seen so far sorted by insertion.  The order is total
+ * (ties on the score go to the lower index), so this is exactly the first k
+ * of the fully sorted array.  Returns min(k, n). */
+static int first_k(const void *v, long n, int k, size_t size, int (*cmp)(const void *, const void *), void *best)
+{
+    int got = 0;
+    char *b = (char *)best;
+    for (long i = 0; i < n; ++i) {
+        const char *e = (const char *)v + (size_t)i * size;
+        if (got == k && cmp(e, b + (size_t)(k - 1) * size) >= 0) continue;
+        int pos = got < k ? got++ : k - 1;
+        while (pos > 0 && cmp(e, b + (size_t)(pos - 1) * size) < 0) {
+            memcpy(b + (size_t)pos * size, b + (size_t)(pos - 1) * size, size);
+            --pos;
+        }
+        memcpy(b + (size_t)pos * size, e, size);
+    }
+    return got;
+}
+
 int orc_route_queries(const orc_cfg *c, const float *Q, const float *kbar, const float *cb,
                       const int32_t *addr, const int32_t *forced, long nq, const int64_t *qidx,
                       int32_t *sel, int32_t *ncand, float *probe_margin, float *rerank_margin,
@@ -275,12 +296,13 @@ int orc_route_queries(const orc_cfg *c, const float *Q, const float *kbar, const
 
     float *s = (float *)malloc(sizeof(float) * (size_t)M * C);
     ga_pair *grid = (ga_pair *)malloc(sizeof(ga_pair) * (size_t)A);
+    ga_pair *top = (ga_pair *)malloc(sizeof(ga_pair) * (size_t)(T + 1));
     int32_t *list = (int32_t *)malloc(sizeof(int32_t) * (size_t)A * cap);
     int32_t *len = (int32_t *)malloc(sizeof(int32_t) * (size_t)A);
     int32_t *cand = (int32_t *)malloc(sizeof(int32_t) * (size_t)(E > 0 ? E : 1));
     ga_pair *rr = (ga_pair *)malloc(sizeof(ga_pair) * (size_t)(E > 0 ? E : 1));
-    if (!s || !grid || !list || !len || !cand || !rr) {
-        free(s); free(grid); free(list); free(len); free(cand); free(rr);
+    if (!s || !grid || !top || !list || !len || !cand || !rr) {
+        free(s); free(grid); free(top); free(list); free(len); free(cand); free(rr);
         return -3;
     }
     long cur_bh = -1;
@@ -315,12 +337,12 @@ int orc_route_queries(const orc_cfg *c, const float *Q, const float *kbar, const
             grid[a].g = g;
             grid[a].a = (int32_t)a;
         }
-        qsort(grid, (size_t)A, sizeof(ga_pair), cmp_ga);
-        if (probe_margin) probe_margin[qi] = (T < A) ? grid[T - 1].g - grid[T].g : INFINITY;
+        first_k(grid, A, T + 1, sizeof(ga_pair), cmp_ga, top);   /* = grid sorted, first T+1 */
+        if (probe_margin) probe_margin[qi] = (T < A) ? top[T - 1].g - top[T].g : INFINITY;
         /* 3. union of the probed lists, causal filter, E cap */
         int nc = 0;
         for (int r = 0; r < T && nc < E; ++r) {
-            int32_t a = grid[r].a;
+            int32_t a = top[r].a;
             for (int k = 0; k < len[a] && nc < E; ++k) {
                 int32_t j = list[(long)a * cap + k];
                 if (j <= bq - L) cand[nc++] = j;
@@ -360,7 +382,7 @@ int orc_route_queries(const orc_cfg *c, const float *Q, const float *kbar, const
             }
         for (int k = 0; k < R; ++k) sel[qi * R + k] = k < ns ? chosen[k] : -1;
     }
-    free(s); free(grid); free(list); free(len); free(cand); free(rr);
+    free(s); free(grid); free(top); free(list); free(len); free(cand); free(rr);
     if (ignored < 0) return -2;
     if (forced_ignored) *forced_ignored = ignored;
     return 0;
@@ -553,12 +575,13 @@ int orc_route_queries64(const orc_cfg *c, const double *Q, const double *kbar, c
 
     double *s = (double *)malloc(sizeof(double) * (size_t)M * C);
     ga64_pair *grid = (ga64_pair *)malloc(sizeof(ga64_pair) * (size_t)A);
+    ga64_pair *top = (ga64_pair *)malloc(sizeof(ga64_pair) * (size_t)(T + 1));
     int32_t *list = (int32_t *)malloc(sizeof(int32_t) * (size_t)A * cap);
     int32_t *len = (int32_t *)malloc(sizeof(int32_t) * (size_t)A);
     int32_t *cand = (int32_t *)malloc(sizeof(int32_t) * (size_t)(E > 0 ? E : 1));
     ga64_pair *rr = (ga64_pair *)malloc(sizeof(ga64_pair) * (size_t)(E > 0 ? E : 1));
-    if (!s || !grid || !list || !len || !cand || !rr) {
-        free(s); free(grid); free(list); free(len); free(cand); free(rr);
+    if (!s || !grid || !top || !list || !len || !cand || !rr) {
+        free(s); free(grid); free(top); free(list); free(len); free(cand); free(rr);
         return -3;
     }
     long cur_bh = -1;
@@ -593,11 +616,11 @@ int orc_route_queries64(const orc_cfg *c, const double *Q, const double *kbar, c
             grid[a].g = g;
             grid[a].a = (int32_t)a;
         }
-        qsort(grid, (size_t)A, sizeof(ga64_pair), cmp_ga64);
-        if (probe_margin) probe_margin[qi] = min_gap(grid, (int)(T < A ? T + 1 : A));
+        const int ntop = first_k(grid, A, T + 1, sizeof(ga64_pair), cmp_ga64, top);  /* = sorted, first T+1 */
+        if (probe_margin) probe_margin[qi] = min_gap(top, ntop);
         int nc = 0;
         for (int r = 0; r < T && nc < E; ++r) {
-            int32_t a = grid[r].a;
+            int32_t a = top[r].a;
             for (int k = 0; k < len[a] && nc < E; ++k) {
                 int32_t j = list[(long)a * cap + k];
                 if (j <= bq - L) cand[nc++] = j;
@@ -634,7 +657,7 @@ int orc_route_queries64(const orc_cfg *c, const double *Q, const double *kbar, c
             }
         for (int k = 0; k < R; ++k) sel[qi * R + k] = k < ns ? chosen[k] : -1;
     }
-    free(s); free(grid); free(list); free(len); free(cand); free(rr);
+    free(s); free(grid); free(top); free(list); free(len); free(cand); free(rr);
     if (bad) return -2;
     if (forced_ignored) *forced_ignored = ignored;
     return 0;
