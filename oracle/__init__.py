@@ -12,6 +12,8 @@ Stages (each cites its source in ``mono_oracle.c``):
 * :func:`project`         Q/K/V = x W^T, RoPE on Q and K (fp64)
 * :func:`summary_assign`  block-mean key summary and product address (fp32)
 * :func:`posting`         bounded causal posting lists, overflow count
+* :func:`posting_redirect` the same lists with redirect-on-overflow (next address
+                          in mixed-radix order with room)
 * :func:`route_queries`   probe, union, causal filter, E cap, rerank (fp32)
 * :func:`summary_assign64`, :func:`route_queries64`
                           the same routing decisions in fp64 (with margins), the
@@ -64,13 +66,14 @@ def _load():
             lib.orc_project.argtypes = [ctypes.POINTER(_Cfg), P, P, P, P, L, P, P, P, P]
             lib.orc_summary_assign.argtypes = [ctypes.POINTER(_Cfg), P, P, P, P, P]
             lib.orc_posting.argtypes = [ctypes.POINTER(_Cfg), P, P, P, P, P]
+            lib.orc_posting_redirect.argtypes = [ctypes.POINTER(_Cfg), P, P, P, P, P, P]
             lib.orc_route_queries.argtypes = [ctypes.POINTER(_Cfg), P, P, P, P, P, L, P, P, P, P, P, P]
             lib.orc_attend.argtypes = [ctypes.POINTER(_Cfg), P, P, P, P, L, P, P]
             lib.orc_summary_assign64.argtypes = [ctypes.POINTER(_Cfg), P, P, P, P, P]
             lib.orc_route_queries64.argtypes = [ctypes.POINTER(_Cfg), P, P, P, P, P, L, P, P, P, P, P, P]
             lib.orc_out_project.argtypes = [ctypes.POINTER(_Cfg), P, P, L, P, P]
             for f in ("orc_project", "orc_summary_assign", "orc_posting", "orc_route_queries", "orc_attend",
-                      "orc_out_project", "orc_summary_assign64", "orc_route_queries64"):
+                      "orc_out_project", "orc_summary_assign64", "orc_route_queries64", "orc_posting_redirect"):
                 getattr(lib, f).restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -132,6 +135,22 @@ def posting(cfg, addr):
     ov = np.empty((cfg.B, cfg.H), np.int64)
     _check(lib.orc_posting(ctypes.byref(_cfg(cfg)), _p(addr), _p(ids), _p(saddr), _p(rank), _p(ov)), "posting")
     return ids, saddr, rank, ov
+
+
+def posting_redirect(cfg, addr):
+    """Redirect-on-overflow lists: list address of each block [B,H,nb] (-1 = dropped), and the canonical
+    export over list addresses (dropped blocks last under C^M): ids, their list address, rank, overflow [B,H]."""
+    lib = _load()
+    addr = _c(addr, np.int32)
+    nb = cfg.S // cfg.Bs
+    la = np.empty((cfg.B, cfg.H, nb), np.int32)
+    ids = np.empty((cfg.B, cfg.H, nb), np.int32)
+    saddr = np.empty((cfg.B, cfg.H, nb), np.int32)
+    rank = np.empty((cfg.B, cfg.H, nb), np.int32)
+    ov = np.empty((cfg.B, cfg.H), np.int64)
+    _check(lib.orc_posting_redirect(ctypes.byref(_cfg(cfg)), _p(addr), _p(la), _p(ids), _p(saddr), _p(rank),
+                                    _p(ov)), "posting_redirect")
+    return la, ids, saddr, rank, ov
 
 
 def route_queries(cfg, Q, kbar, codebooks, addr, forced=None, qidx=None):

@@ -226,6 +226,58 @@ int orc_posting(const orc_cfg *c, const int32_t *addr, int32_t *ids, int32_t *so
 }
 
 /* ------------------------------------------------------------------------ */
+/* Bounded causal posting lists with redirect-on-overflow ([P4]/[P5]: a     */
+/* strict capacity bounds each list, and overflow handling may drop or      */
+/* redirect blocks; the pages give no redirect rule).  This library's        */
+/* reading: scanning blocks j = 0..nb-1 in order, block j goes to the list  */
+/* of its own address if that list holds fewer than cap blocks, else to the */
+/* first list with room among the next addresses in mixed-radix order,      */
+/* addr+1, addr+2, ... (mod C^M); only when every list is full is it        */
+/* dropped, and the (b,h) overflow counter incremented.  The lists stay     */
+/* causal: block j's placement depends on blocks 0..j only.                 */
+/* list_addr[j] = the address of the list holding block j, or -1 (dropped). */
+/* Export in canonical form as orc_posting, over the list addresses: ids    */
+/* sorted by (list address, j), the dropped blocks last under the address   */
+/* C^M (outside the grid); rank = position within the list address.         */
+/* ------------------------------------------------------------------------ */
+int orc_posting_redirect(const orc_cfg *c, const int32_t *addr, int32_t *list_addr, int32_t *ids,
+                         int32_t *sorted_addr, int32_t *rank, int64_t *overflow)
+{
+    if (!cfg_ok(c) || !addr || !list_addr) return -1;
+    const int nb = c->S / c->Bs;
+    const long A = n_addr(c);
+    aj_pair *tmp = (aj_pair *)malloc(sizeof(aj_pair) * (nb > 0 ? nb : 1));
+    int32_t *len = (int32_t *)calloc((size_t)A, sizeof(int32_t));
+    if (!tmp || !len) { free(tmp); free(len); return -3; }
+    for (long bh = 0; bh < (long)c->B * c->H; ++bh) {
+        const int32_t *ad = addr + bh * nb;
+        int32_t *la = list_addr + bh * nb;
+        int64_t ov = 0;
+        memset(len, 0, sizeof(int32_t) * (size_t)A);
+        for (int j = 0; j < nb; ++j) {
+            if (ad[j] < 0 || ad[j] >= A) { free(tmp); free(len); return -2; }
+            la[j] = -1;
+            for (long step = 0; step < A; ++step) {
+                const long a = (ad[j] + step) % A;
+                if (len[a] < c->cap) { len[a]++; la[j] = (int32_t)a; break; }
+            }
+            if (la[j] < 0) ov++;
+        }
+        if (overflow) overflow[bh] = ov;
+        for (int j = 0; j < nb; ++j) { tmp[j].a = la[j] >= 0 ? la[j] : (int32_t)A; tmp[j].j = j; }
+        qsort(tmp, (size_t)nb, sizeof(aj_pair), cmp_aj);
+        for (int k = 0; k < nb; ++k) {
+            if (ids) ids[bh * nb + k] = tmp[k].j;
+            if (sorted_addr) sorted_addr[bh * nb + k] = tmp[k].a;
+            if (rank) rank[bh * nb + k] = (k > 0 && tmp[k - 1].a == tmp[k].a) ? rank[bh * nb + k - 1] + 1 : 0;
+        }
+    }
+    free(tmp);
+    free(len);
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
 /* Per-query routing ([P2] Snapshot: each query probes product addresses,    */
 /* reranks returned candidates and selects a fixed number of remote source   */
 /* blocks; [P1] Key Points: two remote blocks out of five eligible;          */
@@ -244,7 +296,8 @@ int orc_posting(const orc_cfg *c, const int32_t *addr, int32_t *ids, int32_t *so
 /* if f is not selected it is appended when fewer than R blocks are          */
 /* selected, else it replaces the lowest-ranked selected block; with R = 0   */
 /* nothing is selected.  An ineligible forced id is ignored and counted.     */
-/* Lists are rebuilt here from addr by the plain append-if-room scan.        */
+/* Lists are rebuilt here from addr by the plain append-if-room scan; addr  */
+/* holds each block's list address, -1 for a block that no list holds.     */
 /* qidx: optional flat query-head indices ((b*H+h)*S + t), NULL = all.       */
 /* Outputs per listed query: sel [n,R], ncand [n] (eligible candidates       */
 /* after the E cap), probe_margin [n] = g(T-th) - g((T+1)-th) (or +inf),     */
@@ -317,6 +370,7 @@ int orc_route_queries(const orc_cfg *c, const float *Q, const float *kbar, const
             memset(len, 0, sizeof(int32_t) * (size_t)A);
             for (int j = 0; j < nb; ++j) {
                 int32_t a = addr[bh * nb + j];
+                if (a < 0) continue;  /* a block that no list holds (redirect mode: dropped) */
                 if (len[a] < cap) list[(long)a * cap + len[a]++] = j;
             }
             cur_bh = bh;
@@ -596,7 +650,8 @@ int orc_route_queries64(const orc_cfg *c, const double *Q, const double *kbar, c
             memset(len, 0, sizeof(int32_t) * (size_t)A);
             for (int j = 0; j < nb; ++j) {
                 int32_t a = addr[bh * nb + j];
-                if (a < 0 || a >= A) { bad = 1; break; }
+                if (a < 0) continue;  /* a block that no list holds (redirect mode: dropped) */
+                if (a >= A) { bad = 1; break; }
                 if (len[a] < cap) list[(long)a * cap + len[a]++] = j;
             }
             if (bad) break;

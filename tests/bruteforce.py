@@ -47,21 +47,39 @@ def address(codes, C):
     return a
 
 
-def route_bh(Q_bh, K_bh, cw_h, cfg, forced_bh=None):
+def redirect_lists(addr, A, cap):
+    """Redirect-on-overflow placement: block j goes to the first list with room among its own address and the
+    next ones in mixed-radix order (a, a+1, ... mod A); dropped only when every list is full."""
+    lists, overflow = {}, 0
+    for j, a in enumerate(addr):
+        for step in range(A):
+            b = (a + step) % A
+            if len(lists.get(b, [])) < cap:
+                lists.setdefault(b, []).append(j)
+                break
+        else:
+            overflow += 1
+    return lists, overflow
+
+
+def route_bh(Q_bh, K_bh, cw_h, cfg, forced_bh=None, redirect=False):
     """Route every query of one (batch, head).  Returns (addr, lists, overflow, sel)."""
     S, d = Q_bh.shape
     Bs, M, C, T, R, E, L, cap = cfg.Bs, cfg.M, cfg.C, cfg.T, cfg.R, cfg.E, cfg.L, cfg.cap
     nb = S // Bs
     kb = summaries(K_bh, Bs)
     addr = [address(codes_of(kb[j], cw_h, M, C), C) for j in range(nb)]
-    lists = {}
-    overflow = 0
-    for j, a in enumerate(addr):
-        bucket = lists.setdefault(a, [])
-        if len(bucket) < cap:
-            bucket.append(j)
-        else:
-            overflow += 1
+    if redirect:
+        lists, overflow = redirect_lists(addr, C ** M, cap)
+    else:
+        lists = {}
+        overflow = 0
+        for j, a in enumerate(addr):
+            bucket = lists.setdefault(a, [])
+            if len(bucket) < cap:
+                bucket.append(j)
+            else:
+                overflow += 1
     dm = d // M
     sel = []
     for t in range(S):

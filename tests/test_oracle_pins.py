@@ -15,7 +15,7 @@ import pytest
 import torch
 
 import oracle
-from bruteforce import route_bh, route_bh_exact
+from bruteforce import redirect_lists, route_bh, route_bh_exact
 from fp32_exact import F, add32, dot_chain32, fma32, round_f32
 from learned_product_hash_proj_b200 import synth
 
@@ -247,6 +247,84 @@ def test_fp32_and_fp64_routing_agree_when_the_arithmetic_is_exact():
         e_addr, e_ov, e_sel, *_ = route_bh_exact(Q[0, h], K[0, h], cb[h], cfg)
         assert addr64[0, h].tolist() == e_addr
         np.testing.assert_array_equal(sel64[0, h], np.array(e_sel, np.int32))
+
+
+# ---------------------------------------------------------------------------
+# redirect-on-overflow (remio.ai, zh/de, section on retrieval decisions: a strict capacity bounds each list and
+# overflow handling may drop or redirect blocks; the reading taken: the next address in mixed-radix order with room)
+# ---------------------------------------------------------------------------
+def _skewed_addr(rng, B, H, nb, A, hot=0.6):
+    a = rng.integers(0, A, size=(B, H, nb)).astype(np.int32)
+    a[rng.random((B, H, nb)) < hot] = rng.integers(0, 3)          # most blocks on one hot address
+    return a
+
+
+@pytest.mark.parametrize("C,cap,nb", [(4, 2, 40), (8, 3, 96), (3, 2, 18), (3, 2, 22)])
+def test_redirect_lists_match_bruteforce_and_keep_every_block_while_a_list_has_room(C, cap, nb):
+    A = C * C
+    cfg = tiny(S=nb * 8, Bs=8, H=2, M=2, C=C, T=3, cap=cap)
+    rng = np.random.default_rng(A + cap + nb)
+    addr = _skewed_addr(rng, 1, cfg.H, nb, A)
+    la, ids, saddr, rank, ov = oracle.posting_redirect(cfg, addr)
+    for h in range(cfg.H):
+        lists, b_ov = redirect_lists(addr[0, h].tolist(), A, cap)
+        assert ov[0, h] == b_ov
+        for a_, members in lists.items():
+            np.testing.assert_array_equal(np.nonzero(la[0, h] == a_)[0], members)
+        # no list above cap; a block is dropped only when every list is full at its time
+        kept = np.zeros(A, int)
+        for j in range(nb):
+            if la[0, h, j] < 0:
+                assert (kept >= cap).all()
+            else:
+                kept[la[0, h, j]] += 1
+        assert (kept <= cap).all() and kept.sum() + ov[0, h] == nb
+        # canonical export: sorted by (list address, id), the dropped last under A
+        key = np.where(la[0, h] >= 0, la[0, h], A)
+        order = np.lexsort((np.arange(nb), key))
+        np.testing.assert_array_equal(ids[0, h], order)
+        np.testing.assert_array_equal(saddr[0, h], key[order])
+    assert (ov > 0).any() == (nb > A * cap)
+
+
+def test_redirect_equals_drop_when_no_list_fills():
+    cfg = tiny(S=256, Bs=8, H=2, cap=32)                          # cap >= nb = 32: no list can fill
+    rng = np.random.default_rng(3)
+    addr = _skewed_addr(rng, 1, cfg.H, cfg.nb, cfg.A)
+    la, ids, saddr, rank, ov = oracle.posting_redirect(cfg, addr)
+    d_ids, d_saddr, d_rank, d_ov = oracle.posting(cfg, addr)
+    np.testing.assert_array_equal(la, addr)
+    for got, want in ((ids, d_ids), (saddr, d_saddr), (rank, d_rank), (ov, d_ov)):
+        np.testing.assert_array_equal(got, want)
+
+
+def test_redirect_lists_are_causal():
+    # the placement of blocks 0..j-1 does not depend on later blocks (a prefix of the sequence)
+    cfg = tiny(S=512, Bs=8, H=1, C=4, cap=2)
+    rng = np.random.default_rng(5)
+    addr = _skewed_addr(rng, 1, 1, cfg.nb, cfg.A, hot=0.8)
+    la = oracle.posting_redirect(cfg, addr)[0]
+    for cut in (8, 31, 50):
+        short = cfg.with_(S=cut * cfg.Bs)
+        np.testing.assert_array_equal(oracle.posting_redirect(short, addr[:, :, :cut])[0], la[:, :, :cut])
+
+
+@pytest.mark.parametrize("seed", [11, 12])
+def test_routing_over_redirected_lists_matches_bruteforce(seed):
+    # queries probe the redirected lists exactly as they probe dropped-mode lists
+    cfg = tiny(S=96, Bs=8, H=2, L=2, R=2, E=3, T=3, cap=1, C=2)
+    inp = synth.make_inputs(cfg, seed=seed)
+    Qs, Ks, Vs = stored_qkv(cfg, inp)
+    kbar, addr, _ = oracle.summary_assign(cfg, Ks, inp["codebooks"])
+    la, *_, ov = oracle.posting_redirect(cfg, addr)
+    sel, *_ = oracle.route_queries(cfg, Qs, kbar, inp["codebooks"], la)
+    redirected = 0
+    for h in range(cfg.H):
+        b_addr, b_lists, b_ov, b_sel = route_bh(Qs[0, h], Ks[0, h], inp["codebooks"][h], cfg, redirect=True)
+        assert ov[0, h] == b_ov
+        np.testing.assert_array_equal(sel[0, h], np.array(b_sel, np.int32))
+        redirected += int((la[0, h] != addr[0, h]).sum())
+    assert redirected > 0
 
 
 def test_selected_blocks_lie_before_the_local_window():
