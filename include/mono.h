@@ -73,7 +73,17 @@ enum mono_flags {
      * stated tolerances; used as the correctness baseline.  The tensor-core
      * kernels apply to bf16 storage with: projections W % 128 == 0 and
      * H*d % 128 == 0; attention Bs in {64, 128} and 128 + (L-1)*Bs <= 256. */
-    MONO_FLAG_SIMPLE_KERNELS = 1
+    MONO_FLAG_SIMPLE_KERNELS = 1,
+    /* Redirect-on-overflow instead of drop (remio.ai article, the section on
+     * retrieval decisions: a strict capacity bounds each list, and overflow
+     * handling may drop or redirect blocks; the pages give no rule).  A block
+     * whose own list is full goes to the first list with room among the next
+     * addresses in mixed-radix order (a+1, a+2, ... mod C^M); it is dropped,
+     * and counted in the overflow, only when every list is full.  The posting
+     * export lists blocks under the address of the list that holds them, the
+     * dropped ones last under the address C^M.  Needs C^M <= 65536; not
+     * available to the decode entry points (MONO_ERR_UNSUPPORTED). */
+    MONO_FLAG_REDIRECT = 2
 };
 
 /* Shape and method parameters.  Symbols follow the pages' description:
@@ -105,6 +115,8 @@ typedef struct mono_stats {
     int64_t remote_selected;   /* total remote blocks selected */
     double mean_remote;        /* remote_selected / (B*H*S) */
     int64_t forced_ignored;    /* forced ids that were not eligible */
+    int64_t probe_walks;       /* query-heads whose exact top-T left the probe's fast path for the general
+                                  walk (near ties); the first 4096 are listed in MONO_WS_WALK_LOG */
 } mono_stats_t;
 
 /* Workspace regions that mono_workspace_region can locate (debug/export). */
@@ -120,7 +132,9 @@ enum mono_ws_region {
     MONO_WS_V = 8,
     MONO_WS_SEL = 9,       /* [B,H,S,R] int32, used by mono_forward */
     MONO_WS_O = 10,        /* [B,S,H*d] dtype, used by mono_forward */
-    MONO_WS_NREGIONS = 11
+    MONO_WS_WALK_LOG = 11, /* [4096] int32: flat indices (b*H+h)*S+t of the first query-heads whose probe took the
+                              general walk (mono_stats.probe_walks of them; unspecified order) */
+    MONO_WS_NREGIONS = 12
 };
 
 /* Validate `cfg` and build an immutable host-side plan.  Writes the
@@ -213,6 +227,24 @@ size_t mono_route_static_capacity(void);
 int mono_attend(const mono_plan_t *plan, const void *Q, const void *K, const void *V,
                 const int32_t *sel, void *O, void *workspace, void *stream);
 
+/* The stages of mono_attend, callable one at a time (same kernels, same
+ * results): with the tensor-core kernels (bf16, see MONO_FLAG_SIMPLE_KERNELS)
+ *  - mono_attend_pairs:  the (query, remote block) pairs of sel grouped by
+ *                        block into work items, in the workspace;
+ *  - mono_attend_remote: one partial softmax (normalised output in bf16, its
+ *                        max and sum) per pair, block by block, in the
+ *                        workspace;
+ *  - mono_attend_local:  the local part of every query tile and the exact
+ *                        merge with its remote partials -> O.
+ * With the plain kernels the whole attention is one query-major kernel,
+ * which mono_attend_local runs; the other two do nothing.  Each stage reads
+ * what the previous one left in the workspace. */
+int mono_attend_pairs(const mono_plan_t *plan, const int32_t *sel, void *workspace, void *stream);
+int mono_attend_remote(const mono_plan_t *plan, const void *Q, const void *K, const void *V, void *workspace,
+                       void *stream);
+int mono_attend_local(const mono_plan_t *plan, const void *Q, const void *K, const void *V, const int32_t *sel,
+                      void *O, void *workspace, void *stream);
+
 /* Output projection delta = O Wo^T: the last step of the stateless
  * [batch, sequence, width] -> attention-delta mixer (aitechinspire.com
  * article, "Snapshot: key facts from the report"; the host model adds the
@@ -221,6 +253,30 @@ int mono_attend(const mono_plan_t *plan, const void *Q, const void *K, const voi
  * error word that a bounded wait of the tensor-core kernel may set. */
 int mono_out_project(const mono_plan_t *plan, const void *O, const void *Wo, void *delta,
                      void *workspace, void *stream);
+
+/* ------------------------------------------------------------------------
+ * Head-sharded mixer on several GPUs (one process per GPU): rank r of N runs
+ * a plan of H/N heads (its rows of Wq, Wk, Wv, its columns of Wo, its
+ * codebooks).  The mixer's output delta = sum over heads of O_h Wo_h^T (the
+ * output projection of the aitechinspire.com article's attention-delta
+ * mixer, "Snapshot: key facts from the report") is then a sum of the ranks'
+ * partials, taken as a reduce-scatter over token rows: the B*S rows are
+ * split into N equal chunks, chunk c owned by rank c.
+ *  - mono_out_project_scatter: the rank's output projection, its fp32 rows
+ *    written by the GEMM epilogue straight into the owners' staging buffers
+ *    (stage[c]: rank c's buffer, [N][B*S/N][W] fp32, this rank's partial at
+ *    slot `rank`; pointers of other GPUs' memory reachable by peer access,
+ *    e.g. symmetric memory over NVLink).  No partial is rounded to bf16.
+ *  - mono_stage_reduce: after every rank's scatter has completed (the caller
+ *    orders this, e.g. with a collective on the stream), the owner sums its N
+ *    staged partials in fp32 in ascending rank order and rounds once:
+ *    delta_chunk [B*S/N][W] bf16 = rows c*B*S/N .. of delta.
+ * bf16 storage with the tensor-core projections only (MONO_ERR_UNSUPPORTED
+ * otherwise); 1 <= N <= 8 with (B*S) % N == 0 (MONO_ERR_INVALID).
+ * ------------------------------------------------------------------------ */
+int mono_out_project_scatter(const mono_plan_t *plan, const void *O, const void *Wo, float *const *stage,
+                             int nranks, int rank, void *workspace, void *stream);
+int mono_stage_reduce(const mono_plan_t *plan, const float *stage, int nranks, void *delta_chunk, void *stream);
 
 /* The whole mixer (aitechinspire.com article, "Snapshot: key facts from
  * the report" and "What's the core idea?": after RoPE, blocks go to bounded

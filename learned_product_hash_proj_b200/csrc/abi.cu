@@ -41,6 +41,8 @@ int validate(const mono_config *c) {
     if (c->S / c->Bs > kMaxNb) return MONO_ERR_UNSUPPORTED;
     if (c->W % 64 != 0) return MONO_ERR_UNSUPPORTED;
     if ((long long)c->B * c->H * c->S * c->d > (1ll << 40)) return MONO_ERR_UNSUPPORTED;
+    if ((c->flags & MONO_FLAG_REDIRECT) && A > 65536.0L) return MONO_ERR_UNSUPPORTED;
+    if (c->flags & ~(MONO_FLAG_SIMPLE_KERNELS | MONO_FLAG_REDIRECT)) return MONO_ERR_INVALID;
     return MONO_OK;
 }
 
@@ -60,6 +62,7 @@ void layout(Plan *p) {
     bytes[kRegSel] = B * H * S * R * 4;
     bytes[kRegO] = B * S * H * d * es;
     bytes[kRegCounters] = kCntN * 8;
+    bytes[kRegWalkLog] = kWalkLogCap * 4;
     const size_t nhi = (S + kRopeLo - 1) / kRopeLo;
     bytes[kRegRope] = (nhi + kRopeLo) * (d / 2) * 8;
     if (p->fast && R > 0) {
@@ -230,6 +233,39 @@ int mono_attend(const mono_plan_t *plan, const void *Q, const void *K, const voi
     return cuda_status(launch_attend_simt(p, Q, K, V, sel, O, workspace, s));
 }
 
+static int attend_part(const mono_plan_t *plan, const void *Q, const void *K, const void *V, const int32_t *sel,
+                       void *O, void *workspace, void *stream, int parts) {
+    int st = check_common(plan, workspace);
+    if (st) return st;
+    const Plan &p = plan->p;
+    if (empty(&p)) return MONO_OK;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (!p.fast) {  // one query-major kernel does the whole attention: it runs as the local stage
+        if (!(parts & kAttendLocal)) return MONO_OK;
+        if ((st = check_ptrs({Q, K, V, O}))) return st;
+        if (p.cfg.R > 0 && (st = check_ptrs({sel}))) return st;
+        return cuda_status(launch_attend_simt(p, Q, K, V, sel, O, workspace, s));
+    }
+    if ((parts & (kAttendRemote | kAttendLocal)) && (st = check_ptrs({Q, K, V}))) return st;
+    if ((parts & kAttendLocal) && (st = check_ptrs({O}))) return st;
+    if (p.cfg.R > 0 && (parts & (kAttendPairs | kAttendLocal)) && (st = check_ptrs({sel}))) return st;
+    return cuda_status(launch_attend_tc(p, Q, K, V, sel, O, workspace, s, parts));
+}
+
+int mono_attend_pairs(const mono_plan_t *plan, const int32_t *sel, void *workspace, void *stream) {
+    return attend_part(plan, nullptr, nullptr, nullptr, sel, nullptr, workspace, stream, kAttendPairs);
+}
+
+int mono_attend_remote(const mono_plan_t *plan, const void *Q, const void *K, const void *V, void *workspace,
+                       void *stream) {
+    return attend_part(plan, Q, K, V, nullptr, nullptr, workspace, stream, kAttendRemote);
+}
+
+int mono_attend_local(const mono_plan_t *plan, const void *Q, const void *K, const void *V, const int32_t *sel,
+                      void *O, void *workspace, void *stream) {
+    return attend_part(plan, Q, K, V, sel, O, workspace, stream, kAttendLocal);
+}
+
 int mono_out_project(const mono_plan_t *plan, const void *O, const void *Wo, void *delta, void *workspace,
                      void *stream) {
     int st = check_common(plan, workspace);
@@ -239,6 +275,34 @@ int mono_out_project(const mono_plan_t *plan, const void *O, const void *Wo, voi
     if ((st = check_ptrs({O, Wo, delta}))) return st;
     if (p.gemm_tc) return cuda_status(launch_out_project_tc(p, O, Wo, delta, workspace, (cudaStream_t)stream));
     return cuda_status(launch_out_project_simt(p, O, Wo, delta, (cudaStream_t)stream));
+}
+
+int mono_out_project_scatter(const mono_plan_t *plan, const void *O, const void *Wo, float *const *stage,
+                             int nranks, int rank, void *workspace, void *stream) {
+    int st = check_common(plan, workspace);
+    if (st) return st;
+    const Plan &p = plan->p;
+    if (!stage) return MONO_ERR_NULL;
+    if (nranks < 1 || nranks > 8 || rank < 0 || rank >= nranks) return MONO_ERR_INVALID;
+    if (((long long)p.cfg.B * p.cfg.S) % nranks) return MONO_ERR_INVALID;
+    if (!p.gemm_tc) return MONO_ERR_UNSUPPORTED;
+    if (empty(&p)) return MONO_OK;
+    if ((st = check_ptrs({O, Wo}))) return st;
+    for (int r = 0; r < nranks; ++r)
+        if ((st = check_ptrs({stage[r]}))) return st;
+    return cuda_status(launch_out_project_stage(p, O, Wo, stage, nranks, rank, workspace, (cudaStream_t)stream));
+}
+
+int mono_stage_reduce(const mono_plan_t *plan, const float *stage, int nranks, void *delta_chunk, void *stream) {
+    if (!plan) return MONO_ERR_NULL;
+    const Plan &p = plan->p;
+    if (nranks < 1 || nranks > 8) return MONO_ERR_INVALID;
+    if (((long long)p.cfg.B * p.cfg.S) % nranks) return MONO_ERR_INVALID;
+    if (!p.gemm_tc) return MONO_ERR_UNSUPPORTED;
+    if (empty(&p)) return MONO_OK;
+    int st;
+    if ((st = check_ptrs({stage, delta_chunk}))) return st;
+    return cuda_status(launch_stage_reduce(p, stage, nranks, delta_chunk, (cudaStream_t)stream));
 }
 
 int mono_forward(const mono_plan_t *plan, const void *x, const void *Wq, const void *Wk, const void *Wv,
@@ -289,6 +353,7 @@ int mono_stats(const mono_plan_t *plan, const void *workspace, void *stream, mon
     out->queries_lt_R = (int64_t)cnt[kCntQueriesLtR];
     out->remote_selected = (int64_t)cnt[kCntRemoteSel];
     out->forced_ignored = (int64_t)cnt[kCntForcedIgnored];
+    out->probe_walks = (int64_t)cnt[kCntWalks];
     out->device_error = (int32_t)cnt[kCntErr];
     out->mean_remote = (double)out->remote_selected / ((double)p.cfg.B * p.cfg.H * p.cfg.S);
     return out->device_error ? MONO_ERR_DEVICE : MONO_OK;

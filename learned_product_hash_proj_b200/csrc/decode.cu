@@ -543,6 +543,7 @@ int dec_check(const mono_plan_t *plan, const void *cache) {
     if (!cache) return MONO_ERR_WORKSPACE;
     if (((uintptr_t)cache & 255) != 0) return MONO_ERR_ALIGN;
     if (plan->p.A > kDecMaxA) return MONO_ERR_UNSUPPORTED;
+    if (plan->p.cfg.flags & MONO_FLAG_REDIRECT) return MONO_ERR_UNSUPPORTED;  // the cache lists append in drop mode
     return MONO_OK;
 }
 
@@ -569,6 +570,7 @@ extern "C" {
 int mono_decode_cache_bytes(const mono_plan_t *plan, size_t *bytes) {
     if (!plan || !bytes) return MONO_ERR_NULL;
     if (plan->p.A > kDecMaxA) return MONO_ERR_UNSUPPORTED;
+    if (plan->p.cfg.flags & MONO_FLAG_REDIRECT) return MONO_ERR_UNSUPPORTED;
     *bytes = dec_layout(plan->p).total;
     return MONO_OK;
 }

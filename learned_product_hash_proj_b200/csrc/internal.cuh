@@ -28,8 +28,12 @@ enum DevErr : unsigned {
     kDevErrSmemAlign = 5,    // dynamic shared memory not 1024-byte aligned (TMA tiles need it)
 };
 
-// Counters at the start of the counter region (uint64 each).
-enum Counter { kCntQueriesLtR = 0, kCntRemoteSel = 1, kCntForcedIgnored = 2, kCntErr = 3, kCntN = 8 };
+// Counters at the start of the counter region (uint64 each).  kCntWalks counts
+// the query-heads whose probe left the fast path for the general walk (near
+// ties in the staged top-T, or a stage with too many surviving prefixes); the
+// first kWalkLogCap of them are logged by flat index in the walk-log region.
+enum Counter { kCntQueriesLtR = 0, kCntRemoteSel = 1, kCntForcedIgnored = 2, kCntErr = 3, kCntWalks = 4, kCntN = 8 };
+constexpr int kWalkLogCap = 4096;
 
 enum Region {
     kRegKbar = MONO_WS_KBAR,
@@ -43,6 +47,7 @@ enum Region {
     kRegV = MONO_WS_V,
     kRegSel = MONO_WS_SEL,
     kRegO = MONO_WS_O,
+    kRegWalkLog = MONO_WS_WALK_LOG,
     kRegCounters = MONO_WS_NREGIONS,
     kRegRope,
     kRegPairCount,   // [B,H,nb] int32 queries selecting each block (fast attention)
@@ -81,6 +86,12 @@ __device__ __forceinline__ void record_error(unsigned long long *counters, unsig
     atomicCAS(&counters[kCntErr], 0ull, (unsigned long long)code);
 }
 
+// Count a query-head that took the probe's general walk and log its flat index.
+__device__ __forceinline__ void log_walk(unsigned long long *counters, int32_t *walk_log, long long flat) {
+    const unsigned long long k = atomicAdd(&counters[kCntWalks], 1ull);
+    if (k < (unsigned long long)kWalkLogCap) walk_log[k] = (int32_t)flat;
+}
+
 inline char *ws_ptr(const Plan &p, void *ws, int region) { return (char *)ws + p.off[region]; }
 
 // Host-side count of kernel launches issued by this library (mono_kernel_launches).
@@ -106,6 +117,10 @@ bool gemm_tc_supported(const mono_config &c);
 cudaError_t launch_project_tc(const Plan &p, const void *x, const void *Wq, const void *Wk, const void *Wv, void *Q,
                               void *K, void *V, const void *ws, cudaStream_t s);
 cudaError_t launch_out_project_tc(const Plan &p, const void *O, const void *Wo, void *delta, void *ws, cudaStream_t s);
+// head-sharded output projection: fp32 rows scattered to the owners' staging buffers, then the owner's sum
+cudaError_t launch_out_project_stage(const Plan &p, const void *O, const void *Wo, float *const *stage, int nranks,
+                                     int rank, void *ws, cudaStream_t s);
+cudaError_t launch_stage_reduce(const Plan &p, const float *stage, int nranks, void *out, cudaStream_t s);
 // C_g[M,N] (fp32) (+)= sum_{src < nsrc} A_{g,src}(m,k) B_{g,src}(n,k) for g < ngroups (<= 3, nsrc * ngroups
 // <= 6; A and B hold the operands group-major), bf16 operands on the tensor cores; an operand is K-major
 // ([M|N rows][K]) or MN-major ([K rows][M|N]).  Pointers 16-byte aligned; row lengths multiples of 8 (supported() checks).
@@ -117,8 +132,10 @@ cudaError_t gemm_grad_tc(int M, int N, int K, int nsrc, int ngroups, const void 
 // rp->off relative to *base, the device address of its fixed array on the
 // current device); MONO_ERR_SCRATCH if they do not fit.
 int route_static_tables(const Plan &p, void **base, Plan *rp);
+// the stages of the tensor-core attention: pair buckets, remote partials, local part + merge
+enum AttendParts { kAttendPairs = 1, kAttendRemote = 2, kAttendLocal = 4, kAttendAll = 7 };
 cudaError_t launch_attend_tc(const Plan &p, const void *Q, const void *K, const void *V, const int32_t *sel, void *O,
-                             void *ws, cudaStream_t s);
+                             void *ws, cudaStream_t s, int parts = kAttendAll);
 
 }  // namespace mono
 

@@ -322,6 +322,110 @@ __global__ void __launch_bounds__(1024) k_posting_build(const int32_t *__restric
 }
 
 // ---------------------------------------------------------------------------
+// (A4, redirect-on-overflow) the lists of one (b, h) when a block whose own
+// list is full goes to the first list with room among the next addresses in
+// mixed-radix order (a+1, a+2, ... mod C^M), and is dropped (and counted) only
+// when every list is full.  The placement depends on the order of the blocks,
+// so one warp places them in ascending order: a count per address and a
+// bitmap of the full lists in shared memory; the search for a list with room
+// scans the bitmap 32 words (1024 addresses) per step.  Then every thread
+// takes part in the canonical export by comparison counting over the list
+// addresses, the dropped blocks last under the address C^M.
+// grid (H, B), 1024 threads; dynamic smem: bitmap [ceil(A/32)] u32, list
+// addresses [nb] int32, counts [A] u16 (A <= kRedirectMaxA).
+// ---------------------------------------------------------------------------
+constexpr int kRedirectMaxA = 65536;
+
+inline size_t redirect_smem(long long A, int nb) {
+    return (size_t)((A + 31) / 32) * 4 + (size_t)nb * 4 + (size_t)A * 2;
+}
+
+// first address in [p0, p1) whose list is not full, or -1 (all lanes of warp 0)
+__device__ __forceinline__ int first_free(const uint32_t *s_full, int p0, int p1, int lane) {
+    if (p0 >= p1) return -1;
+    const int wl = p0 >> 5, wh = (p1 - 1) >> 5;
+    for (int w0 = wl; w0 <= wh; w0 += 32) {
+        const int w = w0 + lane;
+        uint32_t freeb = 0;
+        if (w <= wh) {
+            freeb = ~s_full[w];
+            if (w == wl) freeb &= ~0u << (p0 & 31);
+            if (w == wh && (p1 & 31) != 0) freeb &= (1u << (p1 & 31)) - 1u;
+        }
+        const unsigned bal = __ballot_sync(0xffffffffu, freeb != 0);
+        if (bal) {
+            const int src = __ffs(bal) - 1;
+            const uint32_t fb = __shfl_sync(0xffffffffu, freeb, src);
+            return ((w0 + src) << 5) + __ffs(fb) - 1;
+        }
+    }
+    return -1;
+}
+
+__global__ void __launch_bounds__(1024) k_posting_redirect(const int32_t *__restrict__ addr, int32_t *__restrict__ ids,
+                                                           int32_t *__restrict__ saddr, int32_t *__restrict__ rank,
+                                                           int32_t *__restrict__ overflow, int nb, int cap, int H,
+                                                           int A) {
+    extern __shared__ uint32_t s_red[];
+    const int nw = (A + 31) / 32;
+    uint32_t *s_full = s_red;                          // [nw]: bit set = list full (and every bit past A)
+    int32_t *s_key = (int32_t *)(s_full + nw);         // [nb]: own address, then list address (A = dropped)
+    uint16_t *s_cnt = (uint16_t *)(s_key + nb);        // [A]
+    __shared__ int s_ov;
+    const int tid = threadIdx.x, lane = tid & 31;
+    const size_t bh = (size_t)blockIdx.y * H + blockIdx.x;
+    const int ecap = min(cap, nb + 1);                 // a list can never hold more than nb blocks
+    for (int i = tid; i < nw; i += blockDim.x)
+        s_full[i] = (i == nw - 1 && (A & 31)) ? ~((1u << (A & 31)) - 1u) : 0u;
+    for (int i = tid; i < A; i += blockDim.x) s_cnt[i] = 0;
+    for (int j = tid; j < nb; j += blockDim.x) s_key[j] = addr[bh * nb + j];
+    __syncthreads();
+    if (tid < 32) {
+        int ov = 0;
+        for (int j = 0; j < nb; ++j) {
+            const int a = s_key[j];
+            int dst = -1;
+            if ((unsigned)a < (unsigned)A) {
+                if (s_cnt[a] < ecap) dst = a;
+                else {
+                    dst = first_free(s_full, a + 1, A, lane);
+                    if (dst < 0) dst = first_free(s_full, 0, a, lane);
+                }
+            }
+            __syncwarp();
+            if (lane == 0) {
+                if (dst >= 0) {
+                    const int n = s_cnt[dst] + 1;
+                    s_cnt[dst] = (uint16_t)n;
+                    if (n >= ecap) s_full[dst >> 5] |= 1u << (dst & 31);
+                    s_key[j] = dst;
+                } else {
+                    s_key[j] = A;
+                }
+            }
+            ov += dst < 0;
+            __syncwarp();
+        }
+        if (lane == 0) s_ov = ov;
+    }
+    __syncthreads();
+    for (int j = tid; j < nb; j += blockDim.x) {
+        const int a = s_key[j];
+        int less = 0, before = 0;
+        for (int k = 0; k < nb; ++k) {
+            const int ak = s_key[k];
+            less += ak < a;
+            before += (ak == a) & (k < j);
+        }
+        const int pos = less + before;
+        ids[bh * nb + pos] = j;
+        saddr[bh * nb + pos] = a;
+        rank[bh * nb + pos] = before;
+    }
+    if (tid == 0) overflow[bh] = s_ov;
+}
+
+// ---------------------------------------------------------------------------
 // (A5-A7) per-query probe, union, causal filter, E cap and rerank.
 //
 // Probe: the top-T addresses of the product grid under (g desc, address asc),
@@ -386,7 +490,8 @@ __global__ void __launch_bounds__(128) k_probe_rerank(const T *__restrict__ Q, c
                                                       const float *__restrict__ cb, const int32_t *__restrict__ post_ids,
                                                       const int32_t *__restrict__ post_addr,
                                                       const int32_t *__restrict__ forced, int32_t *__restrict__ sel,
-                                                      unsigned long long *__restrict__ counters, int S, int H, int Bs,
+                                                      unsigned long long *__restrict__ counters,
+                                                      int32_t *__restrict__ walk_log, int S, int H, int Bs,
                                                       int L, int R, int E, int M, int C, int Tp, int cap) {
     extern __shared__ float smem[];
     const int nb = S / Bs;
@@ -467,6 +572,7 @@ __global__ void __launch_bounds__(128) k_probe_rerank(const T *__restrict__ Q, c
             np = nn;
         }
         if (fallback) {
+            log_walk(counters, walk_log, (long long)bh * S + t);
             top.init(Tp);
             long long A = 1;
             for (int m = 0; m < M; ++m) A *= C;
@@ -733,34 +839,71 @@ __device__ __forceinline__ void q8(const T *qm, float (&qv)[8]) {
     }
 }
 
-// Scores of one subspace: s[c] = q_m . codeword_{m,c}, one fma chain per code
-// in ascending element order (the chains advance together, eight elements at
-// a time, which changes nothing in any chain).  q_m is read from the query
-// tile in shared memory in pieces, so it never occupies registers as a whole.
-template <typename T, int DM, int C>
-__device__ __forceinline__ void sub_scores(const T *qm, const float *cbm, float (&s)[C]) {
+// ---------------------------------------------------------------------------
+// Paired fp32 arithmetic of sm_100: fma.rn.f32x2 performs two independent
+// IEEE fused multiply-adds, each rounded once to nearest-even, on the two
+// 32-bit halves of 64-bit registers.  One instruction advances two fma chains
+// by one step, with exactly the results of two __fmaf_rn calls.
+// ---------------------------------------------------------------------------
+typedef unsigned long long f2_t;
+
+__device__ __forceinline__ f2_t f2_dup(float v) {
+    f2_t r;
+    asm("mov.b64 %0, {%1, %1};" : "=l"(r) : "f"(v));
+    return r;
+}
+__device__ __forceinline__ void f2_split(f2_t v, float &lo, float &hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ f2_t f2_fma(f2_t a, f2_t b, f2_t c) {
+    f2_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+
+// Scores of one subspace for NQ queries: s[q][c] = q_m . codeword_{m,c}, one
+// fma chain per (query, code) in ascending element order from +0.  The
+// subspace's codebook is stored transposed in shared memory (element i of
+// codes 0..C-1 contiguous), so one 16-byte read gives element i of four codes
+// as two pairs, and one paired fma advances the chains of codes c and c+1 of
+// a query together; the NQ queries share the codebook reads.  q is read from
+// the query tile in shared memory eight elements at a time.  The chains run
+// interleaved, which changes nothing in any one of them.
+template <typename T, int DM, int C, int NQ>
+__device__ __forceinline__ void sub_scores_x2(const T *const (&qm)[NQ], const float *cbT, float (&s)[NQ][C]) {
+    static_assert(C % 4 == 0, "codes in groups of four");
+    f2_t acc[NQ][C / 2];
 #pragma unroll
-    for (int c = 0; c < C; ++c) s[c] = 0.0f;
+    for (int q = 0; q < NQ; ++q)
+#pragma unroll
+        for (int p = 0; p < C / 2; ++p) acc[q][p] = 0ull;  // (+0, +0)
 #pragma unroll
     for (int i8 = 0; i8 < DM / 8; ++i8) {
-        float qv[8];
-        q8<T>(qm + 8 * i8, qv);
+        float qv[NQ][8];
 #pragma unroll
-        for (int c = 0; c < C; ++c) {
-            const float4 x = ((const float4 *)(cbm + c * DM + 8 * i8))[0];
-            const float4 y = ((const float4 *)(cbm + c * DM + 8 * i8))[1];
-            float a = s[c];
-            a = __fmaf_rn(qv[0], x.x, a);
-            a = __fmaf_rn(qv[1], x.y, a);
-            a = __fmaf_rn(qv[2], x.z, a);
-            a = __fmaf_rn(qv[3], x.w, a);
-            a = __fmaf_rn(qv[4], y.x, a);
-            a = __fmaf_rn(qv[5], y.y, a);
-            a = __fmaf_rn(qv[6], y.z, a);
-            a = __fmaf_rn(qv[7], y.w, a);
-            s[c] = a;
+        for (int q = 0; q < NQ; ++q) q8<T>(qm[q] + 8 * i8, qv[q]);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const ulonglong2 *row = (const ulonglong2 *)(cbT + (8 * i8 + e) * C);
+            f2_t w[C / 2];
+#pragma unroll
+            for (int c4 = 0; c4 < C / 4; ++c4) {
+                const ulonglong2 v = row[c4];
+                w[2 * c4] = v.x;
+                w[2 * c4 + 1] = v.y;
+            }
+#pragma unroll
+            for (int q = 0; q < NQ; ++q) {
+                const f2_t qq = f2_dup(qv[q][e]);
+#pragma unroll
+                for (int p = 0; p < C / 2; ++p) acc[q][p] = f2_fma(qq, w[p], acc[q][p]);
+            }
         }
     }
+#pragma unroll
+    for (int q = 0; q < NQ; ++q)
+#pragma unroll
+        for (int p = 0; p < C / 2; ++p) f2_split(acc[q][p], s[q][2 * p], s[q][2 * p + 1]);
 }
 
 // Row pitch (bytes) of the query tile in shared memory: the row plus 16 bytes,
@@ -770,44 +913,229 @@ template <typename T, int D>
 constexpr int probe_q_pitch() {
     return D * (int)sizeof(T) + 16;
 }
+// queries per thread: two where both queries' subspace scores fit in registers
+template <int C>
+constexpr int probe_nq() {
+    return C <= 16 ? 2 : 1;
+}
 template <typename T, int D, int C>
 constexpr size_t probe_m2_smem(int nb) {
-    return (size_t)C * D * 4 + (size_t)C * C * 8 + (size_t)128 * probe_q_pitch<T, D>() + (size_t)nb * 8;
+    return (size_t)C * D * 4 + (size_t)C * C * 8 + (size_t)128 * probe_nq<C>() * probe_q_pitch<T, D>() +
+           (size_t)nb * 8;
 }
 
+// The probe, union, causal filter, E cap and rerank of one query-head t from
+// its subspace scores (see k_probe_m2).  Writes sel; returns the number of
+// remote blocks selected and sets *ign when a forced id was not eligible.
 template <typename T, int D, int C, int TP, int E, int R>
-__global__ void __launch_bounds__(128, C <= 16 ? 5 : 3) k_probe_m2(const T *__restrict__ Q, const float *__restrict__ kbar,
+__device__ __forceinline__ int route_query_m2(const float (&s0)[C], const float (&s1)[C], const T *qp,
+                                              const int2 *s_rng, const int32_t *s_ids, const float *kb,
+                                              const int32_t *forced, int32_t *out, int t, size_t bh, int S,
+                                              int Bs, int L, int cap, unsigned long long *counters,
+                                              int32_t *walk_log, int *ign) {
+    constexpr int A = C * C;
+    float mx0 = 0.f, mx1 = 0.f;
+#pragma unroll
+    for (int c = 0; c < C; ++c) {
+        mx0 = fmaxf(mx0, fabsf(s0[c]));
+        mx1 = fmaxf(mx1, fabsf(s1[c]));
+    }
+    const bool finite = mx0 + mx1 <= 1.0e38f;
+    int e2;
+    frexpf(2.f * (mx0 + mx1) + 1e-30f, &e2);
+    const float delta = 3.0f * ldexpf(1.f, e2 - 24);   // (M+1) ulp(2G)
+
+    // Each subspace keeps U, its top T0 codes, and the near codes that some
+    // member of U does not dominate (the pruning rule above): for subspace 0
+    // as address prefixes, for subspace 1 as suffixes of any surviving prefix
+    // (for a fixed prefix the completions rank by s1 with ties to the lower
+    // code, which is the same rule).  The final top T lies in cand0 x cand1.
+    constexpr int T0 = TP < C ? TP : C;
+    constexpr unsigned kAll = C == 32 ? 0xffffffffu : ((1u << C) - 1);
+    float uv0[T0], uv1[T0];
+    int ui0[T0], ui1[T0];
+    top_codes<C, T0>(s0, uv0, ui0);
+    top_codes<C, T0>(s1, uv1, ui1);
+    unsigned tk0 = 0, tk1 = 0;
+#pragma unroll
+    for (int k = 0; k < T0; ++k) { tk0 |= 1u << ui0[k]; tk1 |= 1u << ui1[k]; }
+    const unsigned nr0 = near_codes<C, T0>(s0, uv0, tk0, delta), nr1 = near_codes<C, T0>(s1, uv1, tk1, delta);
+    unsigned cand0 = tk0, cand1 = tk1;
+    if (!finite) {
+        cand0 = kAll;
+        cand1 = kAll;
+    } else if (nr0 | nr1) {
+        cand0 |= undominated<C, T0>(nr0, s0, uv0, ui0, delta);
+        cand1 |= undominated<C, T0>(nr1, s1, uv1, ui1, delta);
+    }
+    RegTop<TP> top;
+    top.init();
+    bool done = false;
+    if (cand0 == tk0 && cand1 == tk1) {
+        // U0 and U1 are sorted by score and fl(a + b) is monotone in a and
+        // b, so pair (i, j) of the ranks is preceded by the (i+1)(j+1)-1
+        // pairs (i' <= i, j' <= j) with scores at least as high: only pairs
+        // with (i+1)(j+1) <= T can be in the top T, unless an excluded pair
+        // reaches the T-th score (ties), which sends the query to the
+        // general walk below.
+        float vout = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < T0; ++i)
+#pragma unroll
+            for (int j = 0; j < T0; ++j) {
+                const float v = __fadd_rn(uv0[i], uv1[j]);
+                if ((i + 1) * (j + 1) <= TP) top.push(v, ui0[i] * C + ui1[j]);
+                else vout = fmaxf(vout, v);
+            }
+        done = vout < top.v[TP - 1];
+    }
+    if (!done) {
+        // general walk over cand0 x cand1 (rare: near ties), on copies of the
+        // scores that can be indexed by code
+        log_walk(counters, walk_log, (long long)bh * S + t);
+        float l0[C], l1[C];
+#pragma unroll
+        for (int c = 0; c < C; ++c) { l0[c] = s0[c]; l1[c] = s1[c]; }
+        top.init();
+        for (unsigned m0 = cand0; m0; m0 &= m0 - 1) {
+            const int c0 = __ffs(m0) - 1;
+            const float v0 = l0[c0];
+            for (unsigned m1 = cand1; m1; m1 &= m1 - 1) {
+                const int c1 = __ffs(m1) - 1;
+                top.push(__fadd_rn(v0, l1[c1]), c0 * C + c1);
+            }
+        }
+    }
+
+    // union of the probed lists in probe order, causal filter, E cap ...
+    const int bq = t / Bs;
+    const int lim = bq - L;
+    int cid[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) cid[e] = 0;
+    int nc = 0;
+    int2 rg[TP];  // every probed list's range, looked up at once
+#pragma unroll
+    for (int r = 0; r < TP; ++r) {
+        const int a = top.a[r];
+        rg[r] = (unsigned)a < (unsigned)A ? s_rng[a] : make_int2(0, 0);
+    }
+#pragma unroll
+    for (int r = 0; r < TP; ++r) {
+        const int kend = min(rg[r].y, rg[r].x + cap);
+        for (int k = rg[r].x; k < kend && nc < E; ++k) {
+            const int j = s_ids[k];
+            if (j > lim) break;
+#pragma unroll
+            for (int e = 0; e < E; ++e)
+                if (e == nc) cid[e] = j;
+            ++nc;
+        }
+    }
+    // ... and the rerank q . kbar_j of the (at most E) candidates, their
+    // fma chains advancing together in ascending element order
+    float acc[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) acc[e] = 0.0f;
+#pragma unroll 2
+    for (int i8 = 0; i8 < D / 8; ++i8) {
+        float qv[8];
+        q8<T>(qp + 8 * i8, qv);
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+            if (e < nc) {
+                const float4 *kr = (const float4 *)(kb + (size_t)cid[e] * D + 8 * i8);
+                const float4 x = __ldg(kr), y = __ldg(kr + 1);
+                float a = acc[e];
+                a = __fmaf_rn(qv[0], x.x, a);
+                a = __fmaf_rn(qv[1], x.y, a);
+                a = __fmaf_rn(qv[2], x.z, a);
+                a = __fmaf_rn(qv[3], x.w, a);
+                a = __fmaf_rn(qv[4], y.x, a);
+                a = __fmaf_rn(qv[5], y.y, a);
+                a = __fmaf_rn(qv[6], y.z, a);
+                a = __fmaf_rn(qv[7], y.w, a);
+                acc[e] = a;
+            }
+        }
+    }
+    RegTop<R> rk;
+    rk.init();
+#pragma unroll
+    for (int e = 0; e < E; ++e)
+        if (e < nc) rk.push(acc[e], cid[e]);
+    int ra[R];
+    int nr = nc < R ? nc : R;
+#pragma unroll
+    for (int k = 0; k < R; ++k) ra[k] = rk.a[k];
+    if (forced) {
+        const int f = forced[bh * S + t];
+        if (f >= 0) {
+            if (f <= lim) {
+                bool present = false;
+#pragma unroll
+                for (int k = 0; k < R; ++k) present |= (k < nr) && ra[k] == f;
+                if (!present) {
+                    const int slot = nr < R ? nr : R - 1;
+#pragma unroll
+                    for (int k = 0; k < R; ++k)
+                        if (k == slot) ra[k] = f;
+                    if (nr < R) ++nr;
+                }
+            } else {
+                *ign += 1;
+            }
+        }
+    }
+    // ascending ids, -1 padding
+#pragma unroll
+    for (int k = 0; k < R; ++k)
+        if (k >= nr) ra[k] = 0x7fffffff;
+#pragma unroll
+    for (int x = 0; x < R; ++x)
+#pragma unroll
+        for (int y = 0; y + 1 < R - x; ++y)
+            if (ra[y] > ra[y + 1]) { int tmp = ra[y]; ra[y] = ra[y + 1]; ra[y + 1] = tmp; }
+#pragma unroll
+    for (int k = 0; k < R; ++k) out[k] = k < nr ? ra[k] : -1;
+    return nr;
+}
+
+// M = 2 with every size fixed at compile time, so all per-query state stays
+// in registers.  A CTA takes 128 x NQ consecutive queries of one (b, h); its
+// thread tid the queries tid, tid + 128, ...  Everything the CTA reads more
+// than once goes to shared memory in one batch: the query rows, the head's
+// codebooks (transposed for the paired chains) and the (b, h) posting arrays.
+// Same pruning rule and arithmetic order as k_probe_rerank.
+template <typename T, int D, int C, int TP, int E, int R>
+__global__ void __launch_bounds__(128, C <= 16 ? 4 : 3) k_probe_m2(const T *__restrict__ Q, const float *__restrict__ kbar,
                                                      const float *__restrict__ cb, const int32_t *__restrict__ post_ids,
                                                      const int32_t *__restrict__ post_addr,
                                                      const int32_t *__restrict__ forced, int32_t *__restrict__ sel,
-                                                     unsigned long long *__restrict__ counters, int S, int H, int Bs,
+                                                     unsigned long long *__restrict__ counters,
+                                                     int32_t *__restrict__ walk_log, int S, int H, int Bs,
                                                      int L, int cap) {
-    constexpr int DM = D / 2, A = C * C, QP = probe_q_pitch<T, D>();
-    static_assert(C <= 32 && TP <= C * C && R >= 1 && E >= 1 && QP % 16 == 0, "shape");
+    constexpr int DM = D / 2, A = C * C, QP = probe_q_pitch<T, D>(), NQ = probe_nq<C>(), QT = 128 * NQ;
+    static_assert(C <= 32 && TP <= C * C && R >= 1 && E >= 1 && QP % 16 == 0 && DM % 8 == 0, "shape");
     extern __shared__ __align__(16) float smem[];
     const int nb = S / Bs;
-    float *s_cb = smem;                                  // [2*C*DM] = C*D floats
-    int2 *s_rng = (int2 *)(s_cb + C * D);                // [A] positions [first, end) of each address's entries
-    uint8_t *s_q = (uint8_t *)(s_rng + A);               // [128] query rows, pitch QP
-    int32_t *s_addr = (int32_t *)(s_q + 128 * QP);       // [nb]
+    float *s_cbT = smem;                                 // [2][DM][C]: element i of codeword (m, c) at (m DM + i) C + c
+    int2 *s_rng = (int2 *)(s_cbT + C * D);               // [A] positions [first, end) of each address's entries
+    uint8_t *s_q = (uint8_t *)(s_rng + A);               // [QT] query rows, pitch QP
+    int32_t *s_addr = (int32_t *)(s_q + QT * QP);        // [nb]
     int32_t *s_ids = s_addr + nb;                        // [nb]
     const int h = blockIdx.y, b = blockIdx.z;
     const size_t bh = (size_t)b * H + h;
     const int tid = threadIdx.x;
-    const int t_lo = blockIdx.x * blockDim.x;
-    // Everything this CTA reads more than once goes to shared memory in one
-    // batch of asynchronous copies: its 128 query rows (contiguous in Q; rows
-    // past S as zero), the head's codebooks and the (b, h) posting arrays.
+    const int t_lo = blockIdx.x * QT;
     {
         constexpr int CH = D * (int)sizeof(T) / 16;  // 16-byte chunks per query row
         const uint8_t *src = (const uint8_t *)(Q + (bh * S + t_lo) * D);
-        for (int i = tid; i < 128 * CH; i += blockDim.x) {
+        for (int i = tid; i < QT * CH; i += blockDim.x) {
             const int r = i / CH, c = i % CH;
             const bool ok = t_lo + r < S;
             tc::cp_async16(s_q + r * QP + 16 * c, ok ? (const void *)(src + (size_t)r * (D * sizeof(T)) + 16 * c) : Q, ok);
         }
-        const float *cbh = cb + (size_t)h * C * D;
-        for (int i = tid; i < C * D / 4; i += blockDim.x) tc::cp_async16(s_cb + 4 * i, cbh + 4 * i, true);
         if ((nb & 3) == 0) {  // 16-byte aligned rows of the posting arrays
             for (int i = tid; i < nb / 4; i += blockDim.x) {
                 tc::cp_async16(s_addr + 4 * i, post_addr + bh * nb + 4 * i, true);
@@ -818,6 +1146,19 @@ __global__ void __launch_bounds__(128, C <= 16 ? 5 : 3) k_probe_m2(const T *__re
                 s_addr[i] = post_addr[bh * nb + i];
                 s_ids[i] = post_ids[bh * nb + i];
             }
+        }
+    }
+    // the head's codebooks ([2][C][DM] floats), transposed, with independent 16-byte loads
+    {
+        const float4 *src = (const float4 *)(cb + (size_t)h * C * D);
+        for (int i4 = tid; i4 < C * D / 4; i4 += blockDim.x) {
+            const float4 f = __ldg(src + i4);
+            const int mc = (4 * i4) / DM, i = (4 * i4) % DM;  // DM is a multiple of 4
+            float *dst = s_cbT + ((mc / C) * DM + i) * C + mc % C;
+            dst[0] = f.x;
+            dst[C] = f.y;
+            dst[2 * C] = f.z;
+            dst[3 * C] = f.w;
         }
     }
     for (int i = tid; i < A; i += blockDim.x) s_rng[i] = make_int2(0, 0);
@@ -834,181 +1175,30 @@ __global__ void __launch_bounds__(128, C <= 16 ? 5 : 3) k_probe_m2(const T *__re
     }
     __syncthreads();
 
-    const int t = t_lo + tid;
+    // subspace scores of this thread's queries (rows past S are zeros and are not routed)
+    float s0[NQ][C], s1[NQ][C];
+    {
+        const T *qm0[NQ], *qm1[NQ];
+#pragma unroll
+        for (int q = 0; q < NQ; ++q) {
+            qm0[q] = (const T *)(s_q + (tid + 128 * q) * QP);
+            qm1[q] = qm0[q] + DM;
+        }
+        sub_scores_x2<T, DM, C, NQ>(qm0, s_cbT, s0);
+        sub_scores_x2<T, DM, C, NQ>(qm1, s_cbT + DM * C, s1);
+    }
     int n_sel = 0, lt_r = 0, ign = 0;
-    if (t < S) {
-        const T *qp = (const T *)(s_q + tid * QP);
-        float s0[C], s1[C];
-        sub_scores<T, DM, C>(qp, s_cb, s0);
-        sub_scores<T, DM, C>(qp + DM, s_cb + C * DM, s1);
-        float mx0 = 0.f, mx1 = 0.f;
+    const float *kb = kbar + bh * nb * D;
 #pragma unroll
-        for (int c = 0; c < C; ++c) {
-            mx0 = fmaxf(mx0, fabsf(s0[c]));
-            mx1 = fmaxf(mx1, fabsf(s1[c]));
+    for (int q = 0; q < NQ; ++q) {
+        const int t = t_lo + tid + 128 * q;
+        if (t < S) {
+            const int nr = route_query_m2<T, D, C, TP, E, R>(s0[q], s1[q], (const T *)(s_q + (tid + 128 * q) * QP),
+                                                             s_rng, s_ids, kb, forced, sel + (bh * S + t) * R, t, bh,
+                                                             S, Bs, L, cap, counters, walk_log, &ign);
+            n_sel += nr;
+            lt_r += nr < R;
         }
-        const bool finite = mx0 + mx1 <= 1.0e38f;
-        int e2;
-        frexpf(2.f * (mx0 + mx1) + 1e-30f, &e2);
-        const float delta = 3.0f * ldexpf(1.f, e2 - 24);   // (M+1) ulp(2G)
-
-        // Each subspace keeps U, its top T0 codes, and the near codes that
-        // some member of U does not dominate (the pruning rule above): for
-        // subspace 0 as address prefixes, for subspace 1 as suffixes of any
-        // surviving prefix (for a fixed prefix the completions rank by s1 with
-        // ties to the lower code, which is the same rule).  The final top T
-        // lies in cand0 x cand1.
-        constexpr int T0 = TP < C ? TP : C;
-        constexpr unsigned kAll = C == 32 ? 0xffffffffu : ((1u << C) - 1);
-        float uv0[T0], uv1[T0];
-        int ui0[T0], ui1[T0];
-        top_codes<C, T0>(s0, uv0, ui0);
-        top_codes<C, T0>(s1, uv1, ui1);
-        unsigned tk0 = 0, tk1 = 0;
-#pragma unroll
-        for (int k = 0; k < T0; ++k) { tk0 |= 1u << ui0[k]; tk1 |= 1u << ui1[k]; }
-        const unsigned nr0 = near_codes<C, T0>(s0, uv0, tk0, delta), nr1 = near_codes<C, T0>(s1, uv1, tk1, delta);
-        unsigned cand0 = tk0, cand1 = tk1;
-        if (!finite) {
-            cand0 = kAll;
-            cand1 = kAll;
-        } else if (nr0 | nr1) {
-            cand0 |= undominated<C, T0>(nr0, s0, uv0, ui0, delta);
-            cand1 |= undominated<C, T0>(nr1, s1, uv1, ui1, delta);
-        }
-        RegTop<TP> top;
-        top.init();
-        bool done = false;
-        if (cand0 == tk0 && cand1 == tk1) {
-            // U0 and U1 are sorted by score and fl(a + b) is monotone in a and
-            // b, so pair (i, j) of the ranks is preceded by the (i+1)(j+1)-1
-            // pairs (i' <= i, j' <= j) with scores at least as high: only pairs
-            // with (i+1)(j+1) <= T can be in the top T, unless an excluded pair
-            // reaches the T-th score (ties), which sends the query to the
-            // general walk below.
-            float vout = -INFINITY;
-#pragma unroll
-            for (int i = 0; i < T0; ++i)
-#pragma unroll
-                for (int j = 0; j < T0; ++j) {
-                    const float v = __fadd_rn(uv0[i], uv1[j]);
-                    if ((i + 1) * (j + 1) <= TP) top.push(v, ui0[i] * C + ui1[j]);
-                    else vout = fmaxf(vout, v);
-                }
-            done = vout < top.v[TP - 1];
-        }
-        if (!done) {
-            // general walk over cand0 x cand1 (rare: near ties); the scores are
-            // recomputed into arrays that can be indexed by code
-            float l0[C], l1[C];
-            sub_scores<T, DM, C>(qp, s_cb, l0);
-            sub_scores<T, DM, C>(qp + DM, s_cb + C * DM, l1);
-            top.init();
-            for (unsigned m0 = cand0; m0; m0 &= m0 - 1) {
-                const int c0 = __ffs(m0) - 1;
-                const float v0 = l0[c0];
-                for (unsigned m1 = cand1; m1; m1 &= m1 - 1) {
-                    const int c1 = __ffs(m1) - 1;
-                    top.push(__fadd_rn(v0, l1[c1]), c0 * C + c1);
-                }
-            }
-        }
-
-        // union of the probed lists in probe order, causal filter, E cap ...
-        const int bq = t / Bs;
-        const int lim = bq - L;
-        int cid[E];
-#pragma unroll
-        for (int e = 0; e < E; ++e) cid[e] = 0;
-        int nc = 0;
-        int2 rg[TP];  // every probed list's range, looked up at once
-#pragma unroll
-        for (int r = 0; r < TP; ++r) {
-            const int a = top.a[r];
-            rg[r] = (unsigned)a < (unsigned)A ? s_rng[a] : make_int2(0, 0);
-        }
-#pragma unroll
-        for (int r = 0; r < TP; ++r) {
-            const int kend = min(rg[r].y, rg[r].x + cap);
-            for (int k = rg[r].x; k < kend && nc < E; ++k) {
-                const int j = s_ids[k];
-                if (j > lim) break;
-#pragma unroll
-                for (int e = 0; e < E; ++e)
-                    if (e == nc) cid[e] = j;
-                ++nc;
-            }
-        }
-        // ... and the rerank q . kbar_j of the (at most E) candidates, their
-        // fma chains advancing together in ascending element order
-        float acc[E];
-#pragma unroll
-        for (int e = 0; e < E; ++e) acc[e] = 0.0f;
-        const float *kb = kbar + bh * nb * D;
-#pragma unroll 2
-        for (int i8 = 0; i8 < D / 8; ++i8) {
-            float qv[8];
-            q8<T>(qp + 8 * i8, qv);
-#pragma unroll
-            for (int e = 0; e < E; ++e) {
-                if (e < nc) {
-                    const float4 *kr = (const float4 *)(kb + (size_t)cid[e] * D + 8 * i8);
-                    const float4 x = __ldg(kr), y = __ldg(kr + 1);
-                    float a = acc[e];
-                    a = __fmaf_rn(qv[0], x.x, a);
-                    a = __fmaf_rn(qv[1], x.y, a);
-                    a = __fmaf_rn(qv[2], x.z, a);
-                    a = __fmaf_rn(qv[3], x.w, a);
-                    a = __fmaf_rn(qv[4], y.x, a);
-                    a = __fmaf_rn(qv[5], y.y, a);
-                    a = __fmaf_rn(qv[6], y.z, a);
-                    a = __fmaf_rn(qv[7], y.w, a);
-                    acc[e] = a;
-                }
-            }
-        }
-        RegTop<R> rk;
-        rk.init();
-#pragma unroll
-        for (int e = 0; e < E; ++e)
-            if (e < nc) rk.push(acc[e], cid[e]);
-        int ra[R];
-        int nr = nc < R ? nc : R;
-#pragma unroll
-        for (int k = 0; k < R; ++k) ra[k] = rk.a[k];
-        if (forced) {
-            const int f = forced[bh * S + t];
-            if (f >= 0) {
-                if (f <= lim) {
-                    bool present = false;
-#pragma unroll
-                    for (int k = 0; k < R; ++k) present |= (k < nr) && ra[k] == f;
-                    if (!present) {
-                        const int slot = nr < R ? nr : R - 1;
-#pragma unroll
-                        for (int k = 0; k < R; ++k)
-                            if (k == slot) ra[k] = f;
-                        if (nr < R) ++nr;
-                    }
-                } else {
-                    ign = 1;
-                }
-            }
-        }
-        // ascending ids, -1 padding
-#pragma unroll
-        for (int k = 0; k < R; ++k)
-            if (k >= nr) ra[k] = 0x7fffffff;
-#pragma unroll
-        for (int x = 0; x < R; ++x)
-#pragma unroll
-            for (int y = 0; y + 1 < R - x; ++y)
-                if (ra[y] > ra[y + 1]) { int tmp = ra[y]; ra[y] = ra[y + 1]; ra[y + 1] = tmp; }
-        int32_t *out = sel + (bh * S + t) * R;
-#pragma unroll
-        for (int k = 0; k < R; ++k) out[k] = k < nr ? ra[k] : -1;
-        n_sel = nr;
-        lt_r = nr < R;
     }
     for (int o = 16; o > 0; o >>= 1) {
         n_sel += __shfl_xor_sync(0xffffffffu, n_sel, o);
@@ -1076,7 +1266,14 @@ cudaError_t launch_lists(const Plan &p, void *ws, cudaStream_t s) {
     // dynamic shared memory beyond the default 48 KB (with the kernels' static arrays) needs the opt-in
     // attribute: up to 8192 blocks take 64 KB of addresses and ranks in the dense kernel
     cudaError_t e = cudaSuccess;
-    if (p.A <= kDenseA) {
+    if (c.flags & MONO_FLAG_REDIRECT) {
+        const size_t dyn = redirect_smem(p.A, p.nb);
+        if (dyn + 64 > 48 * 1024 &&
+            (e = cudaFuncSetAttribute(k_posting_redirect, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn)) !=
+                cudaSuccess)
+            return e;
+        k_posting_redirect<<<g2, 1024, dyn, s>>>(addr, ids, saddr, rank, ov, p.nb, c.cap, c.H, (int)p.A);
+    } else if (p.A <= kDenseA) {
         const size_t dyn = (size_t)p.nb * 8;
         if (dyn + sizeof(int) * (kDenseA + 64) > 48 * 1024 &&
             (e = cudaFuncSetAttribute(k_posting_dense, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn)) !=
@@ -1099,8 +1296,10 @@ cudaError_t launch_queries(const Plan &p, const void *Q, const float *cb, const 
                            void *ws, cudaStream_t s) {
     const mono_config &c = p.cfg;
     unsigned long long *cnt = (unsigned long long *)ws_ptr(p, ws, kRegCounters);
+    int32_t *walk_log = (int32_t *)ws_ptr(p, ws, kRegWalkLog);
     cudaError_t e = cudaMemsetAsync(cnt, 0, 3 * 8, s);  // statistics; the error word is kept
     if (e != cudaSuccess) return e;
+    if ((e = cudaMemsetAsync(cnt + kCntWalks, 0, 8, s)) != cudaSuccess) return e;
     if (c.R == 0) return cudaSuccess;  // nothing to select: sel has no entries
     const float *kbar = (const float *)ws_ptr(p, ws, kRegKbar);
     const int32_t *ids = (const int32_t *)ws_ptr(p, ws, kRegPostIds);
@@ -1115,7 +1314,9 @@ cudaError_t launch_queries(const Plan &p, const void *Q, const float *cb, const 
         if (sm2 > 48 * 1024 &&                                                                                   \
             (e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm2)) != cudaSuccess) \
             return e;                                                                                            \
-        kern<<<g3, 128, sm2, s>>>((const TT *)Q, kbar, cb, ids, saddr, forced, sel, cnt, c.S, c.H, c.Bs, c.L, c.cap); \
+        const dim3 gm2((c.S + 128 * probe_nq<CC>() - 1) / (128 * probe_nq<CC>()), c.H, c.B);                  \
+        kern<<<gm2, 128, sm2, s>>>((const TT *)Q, kbar, cb, ids, saddr, forced, sel, cnt, walk_log, c.S, c.H, c.Bs, c.L, \
+                                  c.cap);                                                                        \
         count_launches(1);                                                                                       \
         return cudaGetLastError();                                                                               \
     }
@@ -1135,7 +1336,8 @@ cudaError_t launch_queries(const Plan &p, const void *Q, const float *cb, const 
             e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);                \
             if (e != cudaSuccess) return e;                                                                        \
         }                                                                                                          \
-        kern<<<g3, 128, smem, s>>>((const TT *)Q, kbar, cb, ids, saddr, forced, sel, cnt, c.S, c.H, c.Bs, c.L,   \
+        kern<<<g3, 128, smem, s>>>((const TT *)Q, kbar, cb, ids, saddr, forced, sel, cnt, walk_log, c.S, c.H,    \
+                                   c.Bs, c.L,                                                                      \
                                    c.R, c.E, c.M, c.C, c.T, c.cap);                                                \
     } while (0)
     if (bf && c.d == 64) MONO_LAUNCH_PR(__nv_bfloat16, 64);

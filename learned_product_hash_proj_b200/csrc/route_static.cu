@@ -44,11 +44,12 @@ size_t route_layout(const Plan &p, Plan *rp) {
     const size_t bh = (size_t)c.B * c.H, nb = (size_t)p.nb;
     *rp = p;
     for (int r = 0; r < kRegN; ++r) { rp->off[r] = 0; rp->bytes[r] = 0; }
-    const int regions[] = {kRegKbar, kRegAddr, kRegPostIds, kRegPostAddr, kRegPostRank, kRegOverflow, kRegCounters};
+    const int regions[] = {kRegKbar, kRegAddr, kRegPostIds, kRegPostAddr, kRegPostRank, kRegOverflow, kRegCounters,
+                           kRegWalkLog};
     const size_t sizes[] = {bh * nb * c.d * 4, bh * nb * 4, bh * nb * 4, bh * nb * 4, bh * nb * 4, bh * 4,
-                            (size_t)kCntN * 8};
+                            (size_t)kCntN * 8, (size_t)kWalkLogCap * 4};
     size_t off = 0;
-    for (int i = 0; i < 7; ++i) {
+    for (int i = 0; i < 8; ++i) {
         rp->off[regions[i]] = off;
         rp->bytes[regions[i]] = sizes[i];
         off = align256(off + sizes[i]);

@@ -23,10 +23,12 @@ _lib = ctypes.CDLL(LIB_PATH)
 
 MONO_F32, MONO_BF16 = 0, 1
 MONO_FLAG_SIMPLE_KERNELS = 1
+MONO_FLAG_REDIRECT = 2
 STATUS = {0: "MONO_OK", 1: "MONO_ERR_INVALID", 2: "MONO_ERR_UNSUPPORTED", 3: "MONO_ERR_NULL",
           4: "MONO_ERR_WORKSPACE", 5: "MONO_ERR_CUDA", 6: "MONO_ERR_DEVICE", 7: "MONO_ERR_ALIGN", 8: "MONO_ERR_SCRATCH"}
 REGIONS = {"kbar": 0, "addr": 1, "post_ids": 2, "post_addr": 3, "post_rank": 4, "overflow": 5, "Q": 6, "K": 7,
-           "V": 8, "sel": 9, "O": 10}
+           "V": 8, "sel": 9, "O": 10, "walk_log": 11}
+WALK_LOG_CAP = 4096
 DEC_REGIONS = {"K": 0, "V": 1, "kbar": 2, "addr": 3, "count": 4, "head": 5, "tail": 6, "next": 7, "overflow": 8,
                "q": 9, "sel": 10, "o": 11}
 
@@ -36,7 +38,8 @@ EXPORTS = ("mono_plan", "mono_plan_destroy", "mono_workspace_region", "mono_proj
            "mono_route_static", "mono_route_static_capacity", "mono_decode_cache_bytes",
            "mono_decode_cache_region", "mono_decode_prefill", "mono_decode_project", "mono_decode_route",
            "mono_decode_attend", "mono_decode_step", "mono_backward_workspace_bytes", "mono_attend_backward",
-           "mono_backward")
+           "mono_backward", "mono_out_project_scatter", "mono_stage_reduce", "mono_attend_pairs",
+           "mono_attend_remote", "mono_attend_local")
 
 
 class MonoError(RuntimeError):
@@ -55,7 +58,7 @@ class Stats(ctypes.Structure):
     _fields_ = [("overflow_total", ctypes.c_int64), ("overflow_max_bh", ctypes.c_int32),
                 ("device_error", ctypes.c_int32), ("queries_lt_R", ctypes.c_int64),
                 ("remote_selected", ctypes.c_int64), ("mean_remote", ctypes.c_double),
-                ("forced_ignored", ctypes.c_int64)]
+                ("forced_ignored", ctypes.c_int64), ("probe_walks", ctypes.c_int64)]
 
     def as_dict(self) -> dict:
         return {k: getattr(self, k) for k, _ in self._fields_}
@@ -94,13 +97,21 @@ _lib.mono_decode_step.argtypes = [_P, ctypes.c_int] + [_P] * 10
 _lib.mono_backward_workspace_bytes.argtypes = [_P, ctypes.POINTER(ctypes.c_size_t)]
 _lib.mono_attend_backward.argtypes = [_P] * 11
 _lib.mono_backward.argtypes = [_P] * 16
+_lib.mono_out_project_scatter.argtypes = [_P, _P, _P, ctypes.POINTER(ctypes.c_void_p), ctypes.c_int, ctypes.c_int,
+                                          _P, _P]
+_lib.mono_stage_reduce.argtypes = [_P, _P, ctypes.c_int, _P, _P]
+_lib.mono_attend_pairs.argtypes = [_P] * 4
+_lib.mono_attend_remote.argtypes = [_P] * 6
+_lib.mono_attend_local.argtypes = [_P] * 8
 _lib.mono_kernel_launches.argtypes = []
 _lib.mono_kernel_launches.restype = ctypes.c_ulonglong
 for _f in ("mono_plan", "mono_workspace_region", "mono_project", "mono_route", "mono_route_summaries",
            "mono_route_lists", "mono_route_queries", "mono_attend", "mono_out_project",
            "mono_forward", "mono_stats", "mono_version", "mono_decode_cache_bytes", "mono_decode_cache_region",
            "mono_decode_prefill", "mono_decode_project", "mono_decode_route", "mono_decode_attend",
-           "mono_decode_step", "mono_backward_workspace_bytes", "mono_attend_backward", "mono_backward"):
+           "mono_decode_step", "mono_backward_workspace_bytes", "mono_attend_backward", "mono_backward",
+           "mono_out_project_scatter", "mono_stage_reduce", "mono_attend_pairs", "mono_attend_remote",
+           "mono_attend_local"):
     getattr(_lib, _f).restype = ctypes.c_int
 
 
@@ -164,7 +175,7 @@ class Plan:
                   "post_rank": ((c.B, c.H, nb), torch.int32), "overflow": ((c.B, c.H), torch.int32),
                   "Q": ((c.B, c.H, c.S, c.d), self.dtype), "K": ((c.B, c.H, c.S, c.d), self.dtype),
                   "V": ((c.B, c.H, c.S, c.d), self.dtype), "sel": ((c.B, c.H, c.S, c.R), torch.int32),
-                  "O": ((c.B, c.S, c.H * c.d), self.dtype)}
+                  "O": ((c.B, c.S, c.H * c.d), self.dtype), "walk_log": ((WALK_LOG_CAP,), torch.int32)}
         shape, dt = shapes[name]
         raw = ws[off.value:off.value + nbytes.value]
         return raw.view(dt).view(shape)
@@ -255,11 +266,61 @@ def attend(plan: Plan, Q, K, V, sel, O, ws, stream=None):
            "mono_attend")
 
 
+def attend_pairs(plan: Plan, sel, ws, stream=None):
+    c = plan.cfg
+    _check(_lib.mono_attend_pairs(plan.handle, _ptr(sel, "sel", (c.B, c.H, c.S, c.R), torch.int32,
+                                                    optional=c.R == 0),
+                                  _ptr(ws, "workspace"), _stream(stream)), "mono_attend_pairs")
+
+
+def attend_remote(plan: Plan, Q, K, V, ws, stream=None):
+    c, dt = plan.cfg, plan.dtype
+    qkv = (c.B, c.H, c.S, c.d)
+    _check(_lib.mono_attend_remote(plan.handle, _ptr(Q, "Q", qkv, dt), _ptr(K, "K", qkv, dt), _ptr(V, "V", qkv, dt),
+                                   _ptr(ws, "workspace"), _stream(stream)), "mono_attend_remote")
+
+
+def attend_local(plan: Plan, Q, K, V, sel, O, ws, stream=None):
+    c, dt = plan.cfg, plan.dtype
+    qkv = (c.B, c.H, c.S, c.d)
+    _check(_lib.mono_attend_local(plan.handle, _ptr(Q, "Q", qkv, dt), _ptr(K, "K", qkv, dt), _ptr(V, "V", qkv, dt),
+                                  _ptr(sel, "sel", (c.B, c.H, c.S, c.R), torch.int32, optional=c.R == 0),
+                                  _ptr(O, "O", (c.B, c.S, c.H * c.d), dt), _ptr(ws, "workspace"), _stream(stream)),
+           "mono_attend_local")
+
+
 def out_project(plan: Plan, O, Wo, delta, ws, stream=None):
     c, dt = plan.cfg, plan.dtype
     _check(_lib.mono_out_project(plan.handle, _ptr(O, "O", (c.B, c.S, c.H * c.d), dt),
                                  _ptr(Wo, "Wo", (c.W, c.H * c.d), dt), _ptr(delta, "delta", (c.B, c.S, c.W), dt),
                                  _ptr(ws, "workspace"), _stream(stream)), "mono_out_project")
+
+
+def out_project_scatter(plan: Plan, O, Wo, stages, rank: int, ws, stream=None):
+    """The head shard's output projection into the owners' staging buffers (mono_out_project_scatter).
+    `stages`: one entry per rank c -- rank c's fp32 staging buffer [N, B*S/N, W], as a CUDA tensor of this
+    device or as a raw device address (int) of peer-accessible memory."""
+    c, dt = plan.cfg, plan.dtype
+    n = len(stages)
+    ptrs = (ctypes.c_void_p * n)()
+    for r, st in enumerate(stages):
+        if isinstance(st, torch.Tensor):
+            ptrs[r] = _ptr(st, f"stage[{r}]", (n, c.B * c.S // n, c.W), torch.float32).value
+        else:
+            ptrs[r] = int(st)
+    _check(_lib.mono_out_project_scatter(plan.handle, _ptr(O, "O", (c.B, c.S, c.H * c.d), dt),
+                                         _ptr(Wo, "Wo", (c.W, c.H * c.d), dt), ptrs, ctypes.c_int(n),
+                                         ctypes.c_int(rank), _ptr(ws, "workspace"), _stream(stream)),
+           "mono_out_project_scatter")
+
+
+def stage_reduce(plan: Plan, stage, nranks: int, delta_chunk, stream=None):
+    """The owner's fixed-order fp32 sum of its staged partials, rounded once (mono_stage_reduce)."""
+    c, dt = plan.cfg, plan.dtype
+    rows = c.B * c.S // nranks
+    _check(_lib.mono_stage_reduce(plan.handle, _ptr(stage, "stage", (nranks, rows, c.W), torch.float32),
+                                  ctypes.c_int(nranks), _ptr(delta_chunk, "delta_chunk", (rows, c.W), dt),
+                                  _stream(stream)), "mono_stage_reduce")
 
 
 def forward(plan: Plan, x, Wq, Wk, Wv, Wo, codebooks, delta, ws, forced=None, stream=None):

@@ -12,3 +12,14 @@ for p in (_ROOT, os.path.dirname(os.path.abspath(__file__))):
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
     config.addinivalue_line("markers", "slow: long-running (full-size workloads)")
+
+
+def pytest_terminal_summary(terminalreporter):
+    """Print the routing counts the GPU parity tests recorded (queries checked per workload, selections that
+    differ from the fp64 oracle and the margins behind them)."""
+    mod = sys.modules.get("gpu_parity")
+    lines = getattr(mod, "ROUTING_LOG", None)
+    if lines:
+        terminalreporter.section("routing against the oracle (fp32 bit-exact, fp64 margin rule)")
+        for line in lines:
+            terminalreporter.write_line(line)

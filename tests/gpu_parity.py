@@ -14,8 +14,16 @@ the next one's comparison:
 Tolerances: fp32 storage -> max abs error 1e-5; bf16 storage -> max abs error
 2e-2 x RMS of the reference, on top of the bf16 storage rounding of each
 output element (at most 2^-8 of its magnitude).
+
+Routing is also measured against the oracle's fp64 statement of the same
+decisions (check_fp64_rule): a GPU address or selection may differ from the
+fp64 one only where a margin of a decision behind it is below 1e-4, and such
+queries must stay below 0.1 % of all queries.
 """
 from __future__ import annotations
+
+import concurrent.futures as cf
+import os
 
 import numpy as np
 import torch
@@ -75,11 +83,21 @@ def sample_queries(cfg, n: int, rng) -> np.ndarray:
     return np.sort(q[(q >= 0) & (q < total)]).astype(np.int64)
 
 
+def oracle_lists(cfg, addr, redirect: bool):
+    """The oracle's posting lists for block addresses `addr`: (the address of the list holding each block, or
+    -1 when dropped -- what the query routing reads), ids, list address, rank, overflow."""
+    if redirect:
+        return oracle.posting_redirect(cfg, addr)
+    ids, saddr, rank, ov = oracle.posting(cfg, addr)
+    return addr, ids, saddr, rank, ov
+
+
 class Run:
     """Inputs of one workload on the device plus the GPU results of each stage."""
 
     def __init__(self, cfg, seed=0, flags=0, forced_frac=None, inputs=None):
         self.cfg = cfg
+        self.redirect = bool(flags & mono.MONO_FLAG_REDIRECT)
         self.inp = inputs if inputs is not None else synth.make_inputs(cfg, seed)
         self.forced = None if forced_frac is None else synth.make_forced(cfg, seed, forced_frac)
         self.plan = mono.Plan(cfg, flags=flags)
@@ -102,7 +120,7 @@ class Run:
         mono.project(self.plan, d["x"], d["Wq"], d["Wk"], d["Wv"], self.Q, self.K, self.V, self.ws)
         mono.route(self.plan, self.Q, self.K, d["codebooks"], self.sel, self.ws, forced=self.forced_dev)
         self.route_ws = {k: to_np(self.plan.region(self.ws, k)).copy()
-                         for k in ("kbar", "addr", "post_ids", "post_addr", "post_rank", "overflow")}
+                         for k in ("kbar", "addr", "post_ids", "post_addr", "post_rank", "overflow", "walk_log")}
         self.stats = mono.stats(self.plan, self.ws)
         mono.attend(self.plan, self.Q, self.K, self.V, self.sel, self.O, self.ws)
         mono.out_project(self.plan, self.O, d["Wo"], self.delta, self.ws)
@@ -143,13 +161,13 @@ def check_routing(run: Run, qidx=None):
     ws = run.route_ws
     np.testing.assert_array_equal(ws["kbar"].view(np.uint32), kbar.view(np.uint32), err_msg="kbar bits")
     np.testing.assert_array_equal(ws["addr"], addr, err_msg="addresses")
-    ids, saddr, rank, ov = oracle.posting(cfg, addr)
+    laddr, ids, saddr, rank, ov = oracle_lists(cfg, addr, run.redirect)
     np.testing.assert_array_equal(ws["post_ids"], ids, err_msg="posting ids")
     np.testing.assert_array_equal(ws["post_addr"], saddr, err_msg="posting addresses")
     np.testing.assert_array_equal(ws["post_rank"], rank, err_msg="posting ranks")
     np.testing.assert_array_equal(ws["overflow"].astype(np.int64), ov, err_msg="overflow")
     assert run.stats["overflow_total"] == int(ov.sum())
-    sel, ncand, pm, rm, ign = oracle.route_queries(cfg, Qg, kbar, run.inp["codebooks"], addr, forced=run.forced,
+    sel, ncand, pm, rm, ign = oracle.route_queries(cfg, Qg, kbar, run.inp["codebooks"], laddr, forced=run.forced,
                                                    qidx=qidx)
     gsel = to_np(run.sel).reshape(cfg.B * cfg.H * cfg.S, cfg.R)
     if qidx is None:
@@ -195,3 +213,118 @@ def check_out_projection(run: Run, rows=None):
     got = to_np(run.delta)
     got = got.reshape(-1, cfg.W)[rows] if rows is not None else got
     return assert_close(got, ref, cfg.dtype, "output projection")
+
+
+# ---------------------------------------------------------------------------
+# routing of whole (b, h) slices against both statements of the oracle, in
+# threads (the oracle's C calls release the interpreter lock)
+# ---------------------------------------------------------------------------
+ROUTING_LOG: list[str] = []  # per workload: queries checked and counts against the fp64 oracle (printed at the end)
+FP64_MARGIN = 1e-4          # decisions closer than this may differ from the fp64 oracle ...
+FP64_MAX_SHARE = 1e-3       # ... on fewer than 0.1 % of the queries
+
+
+def _pool():
+    return cf.ThreadPoolExecutor(max_workers=max(1, min(64, os.cpu_count() or 1)))
+
+
+def oracle_route_slices(run, bhs, chunk: int = 2048):
+    """For each (b, h) in bhs: the oracle's fp32 and fp64 routing of every query of the slice on the GPU's
+    stored Q and K.  Returns {(b, h): dict(addr32, ov32, sel32, addr64, am64, sel64, pm64, rm64)}."""
+    cfg = run.cfg
+    one = cfg.with_(B=1, H=1)
+    cb = run.inp["codebooks"]
+    res, jobs = {}, []
+    with _pool() as ex:
+        for b, h in bhs:
+            Q1 = np.ascontiguousarray(to_np(run.Q[b:b + 1, h:h + 1]), np.float32)
+            K1 = np.ascontiguousarray(to_np(run.K[b:b + 1, h:h + 1]), np.float32)
+            Q64, K64 = Q1.astype(np.float64), K1.astype(np.float64)
+            cb1 = np.ascontiguousarray(cb[h:h + 1])
+            f1 = None if run.forced is None else np.ascontiguousarray(run.forced[b:b + 1, h:h + 1])
+            kbar32, addr32, _ = oracle.summary_assign(one, K1, cb1)
+            kbar64, addr64, am64 = oracle.summary_assign64(one, K64, cb1)
+            la32, _, _, _, ov32 = oracle_lists(one, addr32, run.redirect)
+            la64 = oracle_lists(one, addr64, run.redirect)[0]
+            r = dict(addr32=addr32[0, 0], ov32=int(ov32.sum()), addr64=addr64[0, 0], am64=am64[0, 0],
+                     sel32=np.empty((cfg.S, cfg.R), np.int32), sel64=np.empty((cfg.S, cfg.R), np.int32),
+                     pm64=np.empty(cfg.S), rm64=np.empty(cfg.S))
+            res[(b, h)] = r
+            for q0 in range(0, cfg.S, chunk):
+                qidx = np.arange(q0, min(cfg.S, q0 + chunk), dtype=np.int64)
+                jobs.append((r, qidx, 32, ex.submit(oracle.route_queries, one, Q1, kbar32, cb1, la32, f1, qidx)))
+                jobs.append((r, qidx, 64, ex.submit(oracle.route_queries64, one, Q64, kbar64, cb1, la64, f1, qidx)))
+        for r, qidx, mode, fut in jobs:
+            sel, _, pm, rm, _ = fut.result()
+            if mode == 32:
+                r["sel32"][qidx] = sel
+            else:
+                r["sel64"][qidx] = sel
+                r["pm64"][qidx] = pm
+                r["rm64"][qidx] = rm
+    return res
+
+
+def check_routing_slices(run, bhs):
+    """Every query of the given (b, h) slices: selections bit-exact against the fp32 oracle, and the fp64
+    margin rule.  Returns the counts for the report."""
+    cfg = run.cfg
+    res = oracle_route_slices(run, bhs)
+    gaddr = run.route_ws["addr"]
+    gov = run.route_ws["overflow"]
+    n_q = n_blocks = n_mis = n_flip = small_p = small_r = 0
+    for (b, h), r in res.items():
+        np.testing.assert_array_equal(gaddr[b, h], r["addr32"], err_msg=f"addresses of slice {(b, h)}")
+        assert int(gov[b, h]) == r["ov32"], f"overflow of slice {(b, h)}"
+        gsel = to_np(run.sel[b, h])
+        bad = np.nonzero((gsel != r["sel32"]).any(-1))[0]
+        assert bad.size == 0, f"slice {(b, h)}: {bad.size} queries differ from the fp32 oracle, first t={bad[:8]}"
+        flips = gaddr[b, h] != r["addr64"]
+        assert (r["am64"][flips] < FP64_MARGIN).all(), f"slice {(b, h)}: address flip at an fp64 margin >= 1e-4"
+        mis = (gsel != r["sel64"]).any(-1)
+        expl = (r["pm64"] < FP64_MARGIN) | (r["rm64"] < FP64_MARGIN) | bool(flips.any())
+        unexplained = np.nonzero(mis & ~expl)[0]
+        assert unexplained.size == 0, \
+            f"slice {(b, h)}: selections differ from the fp64 oracle at margins >= 1e-4, t={unexplained[:8]}"
+        n_q += cfg.S
+        n_blocks += cfg.nb
+        n_mis += int(mis.sum())
+        n_flip += int(flips.sum())
+        small_p += int((r["pm64"] < FP64_MARGIN).sum())
+        small_r += int((r["rm64"] < FP64_MARGIN).sum())
+    assert n_flip <= FP64_MAX_SHARE * n_blocks, f"{n_flip} of {n_blocks} addresses differ from the fp64 oracle"
+    assert n_mis < FP64_MAX_SHARE * n_q, f"{n_mis} of {n_q} selections differ from the fp64 oracle"
+    return dict(queries=n_q, fp32_mismatch=0, fp64_mismatch=n_mis, fp64_addr_flips=n_flip,
+                small_probe_margin=small_p, small_rerank_margin=small_r)
+
+
+def check_fp64_rule(run):
+    """All (b, h) slices of a workload: see check_routing_slices."""
+    cfg = run.cfg
+    return check_routing_slices(run, [(b, h) for b in range(cfg.B) for h in range(cfg.H)])
+
+
+def log_routing(run, info: dict, what: str = ""):
+    cfg = run.cfg
+    ROUTING_LOG.append(f"{cfg.name}{what} B={cfg.B} S={cfg.S} H={cfg.H} A={cfg.A} {cfg.dtype}: " +
+                       " ".join(f"{k}={v}" for k, v in info.items()))
+
+
+def check_walk_queries(run, checked_slices):
+    """The query-heads whose probe took the general walk (the kernel logs the first mono.WALK_LOG_CAP of them)
+    and that lie outside `checked_slices`: their selections against the fp32 oracle, bit for bit.  Returns
+    (walks counted, walks compared here)."""
+    cfg = run.cfg
+    n = int(run.stats["probe_walks"])
+    logged = np.sort(run.route_ws["walk_log"][:min(n, mono.WALK_LOG_CAP)].astype(np.int64))
+    assert ((logged >= 0) & (logged < cfg.B * cfg.H * cfg.S)).all()
+    done = {b * cfg.H + h for b, h in checked_slices}
+    rest = logged[[int(q // cfg.S) not in done for q in logged]]
+    if rest.size:
+        kbar, addr, _ = oracle.summary_assign(cfg, to_np(run.K), run.inp["codebooks"])
+        laddr = oracle_lists(cfg, addr, run.redirect)[0]
+        sel, *_ = oracle.route_queries(cfg, to_np(run.Q), kbar, run.inp["codebooks"], laddr, forced=run.forced,
+                                       qidx=rest)
+        gsel = to_np(run.sel).reshape(-1, cfg.R)[rest]
+        np.testing.assert_array_equal(gsel, sel, err_msg="sel of general-walk queries")
+    return n, int(rest.size)

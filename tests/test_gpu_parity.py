@@ -11,8 +11,9 @@ import pytest
 import torch
 
 import oracle
-from gpu_parity import (Run, check_attention, check_out_projection, check_projection, check_routing, sample_queries,
-                        sample_tokens, to_np)
+from gpu_parity import (Run, check_attention, check_fp64_rule, check_out_projection, check_projection, check_routing,
+                        check_routing_slices, check_walk_queries, log_routing, sample_queries, sample_tokens,
+                        to_np)
 from learned_product_hash_proj_b200 import synth
 
 pytestmark = pytest.mark.gpu
@@ -36,6 +37,8 @@ def full_check(run: Run):
     run.run_stages()
     check_projection(run)
     info = check_routing(run)
+    info.update(check_fp64_rule(run))
+    log_routing(run, info)
     check_attention(run)
     check_out_projection(run)
     delta_fwd = run.run_forward()
@@ -165,14 +168,22 @@ def test_simple_and_tensor_core_paths_agree():
 # ---------------------------------------------------------------------------
 # full-size workloads: integer tables in full, sampled outputs
 # ---------------------------------------------------------------------------
-def sampled_check(name, n_rows=96, n_queries=1500, seed=0):
+def sampled_check(name, n_rows=96, n_queries=1500, seed=0, slices=None, flags=0):
+    """Full-size workload: integer tables in full; every query of `slices` ((b, h) pairs, default all) routed
+    by both statements of the oracle (fp32 bit-exact, fp64 margin rule); sampled projection, attention and
+    output rows; causality and order of every selection."""
     cfg = synth.config(name)
-    run = Run(cfg, seed=seed).run_stages()
+    run = Run(cfg, seed=seed, flags=flags).run_stages()
     rng = np.random.default_rng(123)
     rows = sample_tokens(cfg, n_rows, rng)
     qidx = sample_queries(cfg, n_queries, rng)
     check_projection(run, rows=rows)
     info = check_routing(run, qidx=qidx)
+    if slices is None:
+        slices = [(b, h) for b in range(cfg.B) for h in range(cfg.H)]
+    info.update(check_routing_slices(run, slices))
+    info["probe_walks"], info["walks_outside_slices_checked"] = check_walk_queries(run, slices)
+    log_routing(run, info, f" ({len(slices)} of {cfg.B * cfg.H} slices, every query)")
     check_attention(run, qidx=qidx)
     check_out_projection(run, rows=rows)
     # properties that hold at any size, on every query
@@ -186,7 +197,7 @@ def sampled_check(name, n_rows=96, n_queries=1500, seed=0):
     return run, info
 
 
-@pytest.mark.parametrize("name", ["scale4k", "scale32k"])
+@pytest.mark.parametrize("name", ["scale4k", "scale8k", "scale16k", "scale32k"])
 def test_scale_workloads(name):
     run, info = sampled_check(name)
     assert info["overflow"] == 0 or name == "scale4k"
@@ -201,9 +212,34 @@ def test_long_context_full_size():
 
 
 def test_skewed_batch_full_size():
-    run, info = sampled_check("stress", n_rows=48, n_queries=400)
+    # the oracle sorts all 65536 addresses per query: four whole (b, h) slices, spread over the batch
+    run, info = sampled_check("stress", n_rows=48, n_queries=400, slices=[(0, 0), (5, 3), (10, 9), (15, 15)])
     assert info["overflow"] > 0
     assert run.stats["overflow_total"] == info["overflow"]
+
+
+# ---------------------------------------------------------------------------
+# redirect-on-overflow (plan flag): lists, overflow, selections, attention
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("dtype,C", [("f32", 8), ("bf16", 4), ("bf16", 3)])
+def test_redirect_on_overflow(dtype, C):
+    from learned_product_hash_proj_b200 import mono
+    # 33 blocks per (b, h) over C^2 addresses with cap 3: lists overflow; with C = 3 (27 slots) blocks drop too
+    run = Run(small(dtype=dtype, C=C, T=4, cap=3), seed=40 + C, forced_frac=0.3, flags=mono.MONO_FLAG_REDIRECT)
+    info = full_check(run)
+    # some blocks sit in a list other than their own address's (the export is checked in full by full_check)
+    ids, la, own = run.route_ws["post_ids"], run.route_ws["post_addr"], run.route_ws["addr"]
+    listed = la < run.cfg.A
+    assert (np.take_along_axis(own, ids, axis=-1)[listed] != la[listed]).any()
+    assert (info["overflow"] > 0) == (C == 3)
+
+
+def test_redirect_on_overflow_skewed_batch_full_size():
+    from learned_product_hash_proj_b200 import mono
+    # the batched skewed workload, whose drop-mode lists overflow: redirect keeps those blocks
+    run, info = sampled_check("stress", n_rows=48, n_queries=400, slices=[(0, 0), (7, 11), (15, 15)],
+                              flags=mono.MONO_FLAG_REDIRECT)
+    assert info["overflow"] == 0
 
 
 # ---------------------------------------------------------------------------
@@ -211,8 +247,9 @@ def test_skewed_batch_full_size():
 # shared memory then passes the default 48 KB (dense kernel: 64 KB of
 # addresses and ranks).  Routing only, on seeded Q/K, against the oracle in full.
 # ---------------------------------------------------------------------------
-@pytest.mark.parametrize("M,C,T", [(2, 8, 4), (4, 16, 16)])
-def test_routing_at_the_largest_block_count(M, C, T):
+@pytest.mark.parametrize("M,C,T,redirect", [(2, 8, 4, False), (4, 16, 16, False), (4, 16, 16, True)])
+def test_routing_at_the_largest_block_count(M, C, T, redirect):
+    from gpu_parity import oracle_lists
     from learned_product_hash_proj_b200 import mono
     cfg = synth.Config(B=1, S=8192 * 32, W=64, H=1, d=64, Bs=32, L=2, R=2, E=5, M=M, C=C, T=T, cap=1,
                        dtype="bf16")
@@ -221,7 +258,7 @@ def test_routing_at_the_largest_block_count(M, C, T):
     Qn = synth.round_bf16(rng.standard_normal(shape, dtype=np.float32))
     Kn = synth.round_bf16(rng.standard_normal(shape, dtype=np.float32) * 3.0)
     cb = synth.make_codebooks(cfg, 40 + M)
-    plan = mono.Plan(cfg)
+    plan = mono.Plan(cfg, flags=mono.MONO_FLAG_REDIRECT if redirect else 0)
     ws = plan.workspace()
     Q, K = (torch.from_numpy(a).to(torch.bfloat16).cuda() for a in (Qn, Kn))
     sel = torch.empty((cfg.B, cfg.H, cfg.S, cfg.R), dtype=torch.int32, device="cuda")
@@ -230,13 +267,29 @@ def test_routing_at_the_largest_block_count(M, C, T):
     st = mono.stats(plan, ws)
     kbar, addr, _ = oracle.summary_assign(cfg, Kn, cb)
     np.testing.assert_array_equal(to_np(plan.region(ws, "addr")), addr, err_msg="addresses")
-    ids, saddr, rank, ov = oracle.posting(cfg, addr)
+    laddr, ids, saddr, rank, ov = oracle_lists(cfg, addr, redirect)
     np.testing.assert_array_equal(to_np(plan.region(ws, "post_ids")), ids, err_msg="posting ids")
+    np.testing.assert_array_equal(to_np(plan.region(ws, "post_addr")), saddr, err_msg="posting addresses")
     np.testing.assert_array_equal(to_np(plan.region(ws, "post_rank")), rank, err_msg="posting ranks")
     np.testing.assert_array_equal(to_np(plan.region(ws, "overflow")).astype(np.int64), ov, err_msg="overflow")
-    assert st["overflow_total"] == int(ov.sum()) > 0
+    assert st["overflow_total"] == int(ov.sum())
+    assert (ov.sum() > 0) != redirect          # 8192 blocks fill 8192 of 65536 lists of one: nothing drops
     # every 7th query; the oracle sorts the whole grid per query, so the 65536-address grid gets 400
     qidx = np.arange(0, cfg.S, 7, dtype=np.int64) if cfg.A <= 4096 else \
         np.sort(rng.choice(cfg.S, 400, replace=False)).astype(np.int64)
-    osel, *_ = oracle.route_queries(cfg, Qn, kbar, cb, addr, qidx=qidx)
+    osel, *_ = oracle.route_queries(cfg, Qn, kbar, cb, laddr, qidx=qidx)
     np.testing.assert_array_equal(to_np(sel).reshape(-1, cfg.R)[qidx], osel, err_msg="sel")
+
+
+@pytest.mark.parametrize("dtype,H", [("bf16", 2), ("bf16", 130), ("f32", 2)])
+def test_attention_stages_one_at_a_time_equal_the_whole_call(dtype, H):
+    # mono_attend_pairs, _remote and _local in turn give mono_attend's output bit for bit (with 2 x 130 slices,
+    # more than one launch group of the remote and local kernels)
+    from learned_product_hash_proj_b200 import mono
+    run = Run(small(dtype=dtype, H=H, S=640 if H == 2 else 256, Bs=64, C=8, cap=4), seed=50).run_stages()
+    O2 = torch.full_like(run.O, float("nan"))
+    mono.attend_pairs(run.plan, run.sel, run.ws)
+    mono.attend_remote(run.plan, run.Q, run.K, run.V, run.ws)
+    mono.attend_local(run.plan, run.Q, run.K, run.V, run.sel, O2, run.ws)
+    torch.cuda.synchronize()
+    assert torch.equal(O2, run.O)
