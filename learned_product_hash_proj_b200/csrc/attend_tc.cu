@@ -423,6 +423,288 @@ __global__ void __launch_bounds__(256) k_remote_tc(const __grid_constant__ AttnM
 }
 
 // ---------------------------------------------------------------------------
+// remote partials, warp-specialised: one persistent CTA of 320 threads per SM
+// walks the work items {block j, first pair, pair count} of a group of (b, h)
+// slices through an NST-deep ring of stages.
+//   warp 0             producer: per item, the selecting queries' rows by
+//                      cp.async (every lane, 16-byte pieces, arriving on the
+//                      stage's "full" barrier as they land) and their pair
+//                      ids into the stage; K_j and V_j by TMA (lane 0);
+//   warp 1 (one lane)  MMA issuer: S = Q K_j^T of item i+1 is issued before
+//                      O = P V_j of item i, so that the tensor core works on
+//                      one item while the softmax runs on the other;
+//   warps 2-5, 6-9     two softmax groups that take alternate items, one
+//                      thread per query row: the softmax of S in fp32, P
+//                      (bf16) written back over S in tensor memory and read
+//                      from there by the P V MMA, then the normalised partial
+//                      (bf16) and its (max, sum) for the merge.
+// A stage is released ("empty") by the MMA issuer once both MMAs of its item
+// have completed and by the four warps of the group once they have read the
+// item's pair ids.  Tensor memory: 512 columns, 256 per group (S and P from
+// column 0, O from column 256 - D).  Every wait is bounded; a role that gives
+// up sets a shared abort flag that ends the others' waits, and the producer
+// and the MMA issuer wait for their own copies and MMAs in flight before the
+// CTA exits.
+// ---------------------------------------------------------------------------
+template <int D, int BS>
+struct RemoteWs {
+    static constexpr int QB = 128 * D * 2, KB = BS * D * 2, IDS = 128 * 4 + 16;
+    static constexpr int STAGE = QB + 2 * KB + 1024;  // Q, K, V, then pair ids and item (kept 1024-aligned)
+    static constexpr int NST = (200 * 1024) / STAGE > 6 ? 6 : (200 * 1024) / STAGE;
+    static constexpr int O_COL = 256 - D;
+    static constexpr int PREF_OFF = NST * STAGE;                                     // int [kMaxGroup + 1]
+    static constexpr int BAR_OFF = PREF_OFF + ((kMaxGroup + 1) * 4 + 15) / 16 * 16;
+    // mbarriers: full[NST], empty[NST], s_full[2], p_full[2], o_full[2], t_free[2], drain; then TMEM base, abort
+    static constexpr int NBAR = 2 * NST + 9;
+    static constexpr int BYTES = BAR_OFF + NBAR * 8 + 16;
+    static constexpr bool supported = NST >= 2 && BS + D <= 256 && D % 64 == 0 && BS % 32 == 0 && IDS <= 1024;
+};
+
+template <int D, int BS>
+__global__ void __launch_bounds__(320, 1) k_remote_ws(const __grid_constant__ AttnMaps maps, const bf16 *__restrict__ Q,
+                                                      const int32_t *__restrict__ pairs, const int4 *__restrict__ work,
+                                                      const int32_t *__restrict__ nwork, bf16 *__restrict__ part_o,
+                                                      float2 *__restrict__ part_ml,
+                                                      unsigned long long *__restrict__ counters, int S, int R,
+                                                      int wcap, float scale_log2, int bh0, int ng) {
+    using Lay = RemoteWs<D, BS>;
+    static_assert(Lay::supported, "tile shape");
+    constexpr int QB = Lay::QB, KB = Lay::KB, STAGE = Lay::STAGE, NST = Lay::NST;
+    constexpr int CH = D * 2 / 16;  // 16-byte pieces of a query row
+    extern __shared__ __align__(1024) uint8_t smem[];
+    int *s_pref = (int *)(smem + Lay::PREF_OFF);
+    uint64_t *bars = (uint64_t *)(smem + Lay::BAR_OFF);
+    uint64_t *full = bars, *empty = bars + NST, *s_full = bars + 2 * NST, *p_full = s_full + 2, *o_full = s_full + 4,
+             *t_free = s_full + 6, *drain = s_full + 8;
+    uint32_t *tmem_base = (uint32_t *)(bars + Lay::NBAR);
+    volatile int *abort_flag = (volatile int *)(tmem_base + 1);
+    if (timed_out(counters)) return;
+    if (tc::smem_u32(smem) & 1023) {
+        if (threadIdx.x == 0) record_error(counters, kDevErrSmemAlign);
+        return;
+    }
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    // a stage: Q rows (K-major, no swizzle), K_j and V_j (TMA, 128-byte swizzle), pair ids [128], item (bh, n)
+    auto stage_q = [&](int s) { return smem + s * STAGE; };
+    auto stage_ids = [&](int s) { return (int *)(smem + s * STAGE + QB + 2 * KB); };
+
+    if (tid == 0) {
+        int acc = 0;
+        for (int g = 0; g < ng; ++g) { s_pref[g] = acc; acc += nwork[bh0 + g]; }
+        s_pref[ng] = acc;
+        for (int s = 0; s < NST; ++s) {
+            tc::mbar_init(&full[s], 32 + 1);  // every producer lane's copies + the K/V transaction
+            tc::mbar_init(&empty[s], 1 + 4);  // the MMA issuer + the group's four warps
+        }
+        for (int g = 0; g < 2; ++g) {
+            tc::mbar_init(&s_full[g], 1);
+            tc::mbar_init(&p_full[g], 4);
+            tc::mbar_init(&o_full[g], 1);
+            tc::mbar_init(&t_free[g], 4);
+        }
+        tc::mbar_init(drain, 1);
+        *abort_flag = 0;
+        tc::fence_mbar_init();
+    }
+    if (warp == 1) {
+        tc::tmem_alloc(tmem_base, 512);
+        tc::tmem_relinquish();
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = *tmem_base;
+    const int total = s_pref[ng];
+    const int G = gridDim.x;
+    const int n = blockIdx.x < total ? (total - 1 - blockIdx.x) / G + 1 : 0;  // items of this CTA
+    bool ok = true;
+    auto fail = [&]() {
+        ok = false;
+        *abort_flag = 1;
+    };
+
+    if (warp == 0) {
+        // ---------------- producer (the whole warp) ----------------
+        int last_v[NST];
+#pragma unroll
+        for (int s = 0; s < NST; ++s) last_v[s] = -1;
+        for (int i = 0; i < n && ok; ++i) {
+            const int s = i % NST, v = i / NST;
+            if (v > 0 && !__all_sync(0xffffffffu, tc::mbar_wait_or_abort(&empty[s], (v - 1) & 1, abort_flag))) {
+                fail();
+                break;
+            }
+            // the item: slice lo with s_pref[lo] <= f < s_pref[lo + 1]
+            const int f = blockIdx.x + i * G;
+            int lo = 0, hi = ng;
+            while (hi - lo > 1) {
+                const int mid = (lo + hi) >> 1;
+                if (s_pref[mid] <= f) lo = mid;
+                else hi = mid;
+            }
+            const long long bh = bh0 + lo;
+            const int4 w = work[bh * wcap + (f - s_pref[lo])];
+            const int j = w.x, p0 = w.y, cnt = w.z;
+            uint8_t *sQ = stage_q(s), *sK = sQ + QB, *sV = sK + KB;
+            int *ids = stage_ids(s);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int row = lane + 32 * k;
+                const bool live = row < cnt;
+                const int pr = live ? pairs[bh * S * R + p0 + row] : -1;
+                ids[row] = pr;
+                const bf16 *qrow = Q + ((size_t)bh * S + (live ? pr / R : 0)) * D;
+#pragma unroll
+                for (int c = 0; c < CH; ++c) tc::cp_async16(sQ + tc::kmajor_chunk(row, c, D), qrow + 8 * c, live);
+            }
+            if (lane == 0) {
+                ids[128] = (int)(bh - bh0);
+                ids[129] = cnt;
+            }
+            asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(tc::smem_u32(&full[s]))
+                         : "memory");
+            __syncwarp();
+            if (lane == 0) {
+                tc::mbar_expect_tx(&full[s], 2 * KB);
+#pragma unroll
+                for (int a = 0; a < D / 64; ++a) {
+                    tc::tma_load_3d(sK + a * (BS * 128), &maps.k, 64 * a, j * BS, (int)bh, &full[s]);
+                    tc::tma_load_3d(sV + a * (BS * 128), &maps.v, 64 * a, j * BS, (int)bh, &full[s]);
+                }
+            }
+            last_v[s] = v;
+        }
+        // every copy issued has landed before the CTA may exit
+        asm volatile("cp.async.wait_all;" ::: "memory");
+        if (lane == 0)
+            for (int s = 0; s < NST; ++s)
+                if (last_v[s] >= 0 && !tc::mbar_wait(&full[s], last_v[s] & 1)) ok = false;
+    } else if (warp == 1) {
+        // ---------------- MMA issuer ----------------
+        if (lane == 0) {
+            const uint32_t id1 = tc::idesc_bf16(128, BS), id2 = tc::idesc_bf16(128, D, true);
+            auto mma1 = [&](int i) -> bool {
+                const int s = i % NST, v = i / NST, g = i & 1, u = i >> 1;
+                if (!tc::mbar_wait_or_abort(&full[s], v & 1, abort_flag)) return false;
+                if (u > 0 && !tc::mbar_wait_or_abort(&t_free[g], (u - 1) & 1, abort_flag)) return false;
+                tc::fence_smem_to_async();
+                tc::fence_after_sync();
+                const uint32_t aq = tc::smem_u32(stage_q(s)), bk = aq + QB;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk)
+                    tc::mma_bf16(tmem + g * 256, tc::desc_kmajor(aq + 256 * kk, D),
+                                 tc::desc_sw128(bk + (kk >> 2) * (BS * 128) + (kk & 3) * 32), id1, kk > 0);
+                tc::commit(&s_full[g]);
+                return true;
+            };
+            auto mma2 = [&](int i) -> bool {
+                const int s = i % NST, g = i & 1, u = i >> 1;
+                if (!tc::mbar_wait_or_abort(&p_full[g], u & 1, abort_flag)) return false;
+                tc::fence_after_sync();
+                const uint32_t bv = tc::smem_u32(stage_q(s)) + QB + KB;
+#pragma unroll
+                for (int kk = 0; kk < BS / 16; ++kk)
+                    tc::mma_bf16_ts(tmem + g * 256 + Lay::O_COL, tmem + g * 256 + 8 * kk,
+                                    tc::desc_sw128_mn(bv + 2048 * kk, BS * 128), id2, kk > 0);
+                tc::commit(&o_full[g]);
+                tc::commit(&empty[s]);
+                return true;
+            };
+            if (n > 0 && !mma1(0)) fail();
+            for (int i = 0; i < n && ok; ++i) {
+                if (i + 1 < n && !mma1(i + 1)) { fail(); break; }
+                if (!mma2(i)) { fail(); break; }
+            }
+            // every MMA issued has completed before the CTA may exit
+            tc::commit(drain);
+            if (!tc::mbar_wait(drain, 0)) ok = false;
+        }
+    } else {
+        // ---------------- softmax groups ----------------
+        const int g = (warp - 2) >> 2, quarter = warp & 3;
+        const int row = quarter * 32 + lane;
+        const uint32_t tS = tmem + g * 256 + ((uint32_t)(quarter * 32) << 16);
+        const uint32_t tO = tS + Lay::O_COL;
+        for (int i = g; i < n && ok; i += 2) {
+            const int s = i % NST, v = i / NST, u = i >> 1;
+            // (the decisions to go on are warp-uniform: the TMEM accesses below are warp-collective)
+            if (!__all_sync(0xffffffffu, tc::mbar_wait_or_abort(&full[s], v & 1, abort_flag))) { fail(); break; }
+            const int *ids = stage_ids(s);
+            const int pr = ids[row];
+            const long long bh = bh0 + ids[128];
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&empty[s]);  // this warp is done with the stage
+            if (!__all_sync(0xffffffffu, tc::mbar_wait_or_abort(&s_full[g], u & 1, abort_flag))) { fail(); break; }
+            tc::fence_after_sync();
+            // softmax of the row over the block's BS keys (all visible: the block lies before the query)
+            float vv[32];
+            float m = -INFINITY;
+#pragma unroll
+            for (int c0 = 0; c0 < BS; c0 += 32) {
+                __syncwarp();
+                tc::tmem_ld32(tS + c0, vv);
+#pragma unroll
+                for (int k = 0; k < 32; ++k) m = fmaxf(m, vv[k]);
+            }
+            const float m2 = m * scale_log2;
+            float l = 0.f;
+#pragma unroll
+            for (int c0 = 0; c0 < BS; c0 += 32) {
+                __syncwarp();
+                tc::tmem_ld32(tS + c0, vv);
+                uint32_t pk[16];
+#pragma unroll
+                for (int k = 0; k < 16; ++k) {
+                    const float a = exp2f(fmaf(vv[2 * k], scale_log2, -m2));
+                    const float bb = exp2f(fmaf(vv[2 * k + 1], scale_log2, -m2));
+                    l += a + bb;
+                    pk[k] = pack2(a, bb);
+                }
+                // P over the columns of S already read (column c0/2 .. c0/2 + 15 of this row)
+                __syncwarp();
+                tc::tmem_st16(tS + (c0 >> 1), pk);
+            }
+            __syncwarp();
+            tc::tmem_st_wait();
+            tc::fence_before_sync();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&p_full[g]);
+            const float inv = 1.f / l;
+            if (!__all_sync(0xffffffffu, tc::mbar_wait_or_abort(&o_full[g], u & 1, abort_flag))) { fail(); break; }
+            tc::fence_after_sync();
+            const bool live = pr >= 0;
+            const size_t slot = (size_t)bh * S * R + (live ? pr : 0);
+#pragma unroll
+            for (int c0 = 0; c0 < D; c0 += 32) {
+                __syncwarp();
+                tc::tmem_ld32(tO + c0, vv);
+                if (live) {
+                    uint4 *dst = (uint4 *)(part_o + slot * D + c0);
+#pragma unroll
+                    for (int q8 = 0; q8 < 4; ++q8)
+                        dst[q8] = make_uint4(pack2(vv[8 * q8] * inv, vv[8 * q8 + 1] * inv),
+                                             pack2(vv[8 * q8 + 2] * inv, vv[8 * q8 + 3] * inv),
+                                             pack2(vv[8 * q8 + 4] * inv, vv[8 * q8 + 5] * inv),
+                                             pack2(vv[8 * q8 + 6] * inv, vv[8 * q8 + 7] * inv));
+                }
+            }
+            if (live) part_ml[slot] = make_float2(m2, l);
+            tc::fence_before_sync();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&t_free[g]);
+        }
+    }
+    if (!ok) record_error(counters, kDevErrTimeout);
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    if (warp == 1) {
+        __syncwarp();
+        tc::tmem_dealloc(tmem, 512);
+    }
+}
+
+// ---------------------------------------------------------------------------
 // local part + merge: persistent CTAs of 256 threads walk the 128-query tiles
 // of a group of (b, h) slices.  Per tile: S over the tile's local key range
 // (<= 256 keys) and O = P V on tcgen05, the masked softmax in fp32, and the
@@ -1105,7 +1387,7 @@ static bool make_map_3d(CUtensorMap *map, const void *ptr, int D, int S, int BH,
 
 template <int D, int BS, int NK, int RMAX>
 static cudaError_t launch_tc_shape(const Plan &p, const bf16 *Q, const bf16 *K, const bf16 *V, const int32_t *sel,
-                                   bf16 *O, void *ws, cudaStream_t s) {
+                                   bf16 *O, void *ws, cudaStream_t s, int parts) {
     const mono_config &c = p.cfg;
     unsigned long long *cnt_err = (unsigned long long *)ws_ptr(p, ws, kRegCounters);
     const float scale_log2 = (float)(1.4426950408889634 / sqrt((double)c.d));
@@ -1117,7 +1399,9 @@ static cudaError_t launch_tc_shape(const Plan &p, const bf16 *Q, const bf16 *K, 
         !make_map_3d(&rmaps.k, K, D, c.S, c.B * c.H, BS) || !make_map_3d(&rmaps.v, V, D, c.S, c.B * c.H, BS))
         return cudaErrorInvalidValue;
     constexpr size_t rsmem = RemoteSmem<D, BS>::BYTES;
-    if (c.R > 0) {
+    // the warp-specialised remote kernel where its ring fits (every tensor-core shape), else the two-stage one
+    constexpr bool kRemoteWs = RemoteWs<D, BS>::supported;
+    if (c.R > 0 && (parts & kAttendPairs)) {
         int32_t *pc = (int32_t *)ws_ptr(p, ws, kRegPairCount);
         int32_t *ps = (int32_t *)ws_ptr(p, ws, kRegPairStart);
         int32_t *pf = (int32_t *)ws_ptr(p, ws, kRegPairFill);
@@ -1137,11 +1421,18 @@ static cudaError_t launch_tc_shape(const Plan &p, const bf16 *Q, const bf16 *K, 
         k_pair_count<<<gq, 256, hs, s>>>(sel, pc, c.S, c.R, p.nb, c.Bs, c.L, cnt_err);
         k_pair_scan<<<nbhh, 1024, 0, s>>>(pc, ps, pf, work, nwork, p.nb, wcap);
         k_pair_fill<<<gq, 256, 2 * hs, s>>>(sel, ps, pf, pairs, c.S, c.R, p.nb, c.Bs, c.L);
-        if ((e = cudaFuncSetAttribute(k_remote_tc<D, BS>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rsmem)) !=
-            cudaSuccess)
-            return e;
         count_launches(3);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    if (c.R > 0 && (parts & kAttendRemote)) {
+        if constexpr (kRemoteWs) {
+            if ((e = cudaFuncSetAttribute(k_remote_ws<D, BS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          (int)RemoteWs<D, BS>::BYTES)) != cudaSuccess)
+                return e;
+        } else if ((e = cudaFuncSetAttribute(k_remote_tc<D, BS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)rsmem)) != cudaSuccess) {
+            return e;
+        }
     }
     // the local part: the warp-specialised kernel where its stages and tensor
     // memory fit, else the single-stage one
@@ -1168,19 +1459,39 @@ static cudaError_t launch_tc_shape(const Plan &p, const bf16 *Q, const bf16 *K, 
     // (attention at S = 32768, 16 heads: 275 us in one group, 327 us in four):
     // fewer launch tails, and the remote kernel balances more work items.
     int remote_ctas = 0;
-    if (c.R > 0 && (e = persistent_grid(k_remote_tc<D, BS>, 256, rsmem, &remote_ctas)) != cudaSuccess)
-        return e;
+    if (c.R > 0) {
+        if constexpr (kRemoteWs) {
+            int dev = 0;
+            if ((e = cudaGetDevice(&dev)) != cudaSuccess ||
+                (e = cudaDeviceGetAttribute(&remote_ctas, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+                return e;
+        } else if ((e = persistent_grid(k_remote_tc<D, BS>, 256, rsmem, &remote_ctas)) != cudaSuccess) {
+            return e;
+        }
+    }
     const int nbhh = c.B * c.H;
     const int group = c.R > 0 ? std::min(kMaxGroup, nbhh) : nbhh;
+    // all stages at once: remote then local per group of slices; one stage at a time: over every group
+    const bool both = (parts & kAttendRemote) && (parts & kAttendLocal);
+    for (int pass = 0; pass < (both ? 1 : 2); ++pass)
     for (int g0 = 0; g0 < nbhh; g0 += group) {
         const int ng = std::min(group, nbhh - g0);
-        if (c.R > 0) {
-            k_remote_tc<D, BS><<<remote_ctas, 256, rsmem, s>>>(
-                rmaps, Q, (const int32_t *)ws_ptr(p, ws, kRegPairs), (const int4 *)ws_ptr(p, ws, kRegWork),
-                (const int32_t *)ws_ptr(p, ws, kRegNWork), (bf16 *)ws_ptr(p, ws, kRegPartO),
-                (float2 *)ws_ptr(p, ws, kRegPartML), cnt_err, c.S, c.R, p.max_work, scale_log2, g0, ng);
+        const bool do_remote = (parts & kAttendRemote) && (both || pass == 0);
+        const bool do_local = (parts & kAttendLocal) && (both || pass == 1);
+        if (c.R > 0 && do_remote) {
+            if constexpr (kRemoteWs)
+                k_remote_ws<D, BS><<<remote_ctas, 320, RemoteWs<D, BS>::BYTES, s>>>(
+                    rmaps, Q, (const int32_t *)ws_ptr(p, ws, kRegPairs), (const int4 *)ws_ptr(p, ws, kRegWork),
+                    (const int32_t *)ws_ptr(p, ws, kRegNWork), (bf16 *)ws_ptr(p, ws, kRegPartO),
+                    (float2 *)ws_ptr(p, ws, kRegPartML), cnt_err, c.S, c.R, p.max_work, scale_log2, g0, ng);
+            else
+                k_remote_tc<D, BS><<<remote_ctas, 256, rsmem, s>>>(
+                    rmaps, Q, (const int32_t *)ws_ptr(p, ws, kRegPairs), (const int4 *)ws_ptr(p, ws, kRegWork),
+                    (const int32_t *)ws_ptr(p, ws, kRegNWork), (bf16 *)ws_ptr(p, ws, kRegPartO),
+                    (float2 *)ws_ptr(p, ws, kRegPartML), cnt_err, c.S, c.R, p.max_work, scale_log2, g0, ng);
             count_launches(1);
         }
+        if (!do_local) continue;
         if constexpr (ws_local) {
             const int tiles = ng * ((c.S + 127) / 128);
             k_local_ws<D, BS, NK, RMAX><<<std::min(local_ctas, tiles), 320, smem, s>>>(
@@ -1198,7 +1509,7 @@ static cudaError_t launch_tc_shape(const Plan &p, const bf16 *Q, const bf16 *K, 
 }
 
 cudaError_t launch_attend_tc(const Plan &p, const void *Q, const void *K, const void *V, const int32_t *sel, void *O,
-                             void *ws, cudaStream_t s) {
+                             void *ws, cudaStream_t s, int parts) {
     const mono_config &c = p.cfg;
     const bf16 *q = (const bf16 *)Q, *k = (const bf16 *)K, *v = (const bf16 *)V;
     bf16 *o = (bf16 *)O;
@@ -1206,9 +1517,9 @@ cudaError_t launch_attend_tc(const Plan &p, const void *Q, const void *K, const 
     // NK = the local key range rounded up to a multiple of 32 (MMA N <= 256)
 #define MONO_TC(DD, BB, NN)                                                                                     \
     do {                                                                                                        \
-        if (c.R <= 2) return launch_tc_shape<DD, BB, NN, 2>(p, q, k, v, sel, o, ws, s);                         \
-        if (c.R <= 4) return launch_tc_shape<DD, BB, NN, 4>(p, q, k, v, sel, o, ws, s);                         \
-        return launch_tc_shape<DD, BB, NN, kMaxR>(p, q, k, v, sel, o, ws, s);                                   \
+        if (c.R <= 2) return launch_tc_shape<DD, BB, NN, 2>(p, q, k, v, sel, o, ws, s, parts);                  \
+        if (c.R <= 4) return launch_tc_shape<DD, BB, NN, 4>(p, q, k, v, sel, o, ws, s, parts);                  \
+        return launch_tc_shape<DD, BB, NN, kMaxR>(p, q, k, v, sel, o, ws, s, parts);                            \
     } while (0)
     if (c.d == 64 && c.Bs == 64) {
         if (nk <= 128) MONO_TC(64, 64, 128);

@@ -17,6 +17,7 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "internal.cuh"
@@ -32,7 +33,8 @@ constexpr int BM = 128, BN = 128, BK = 64, STAGES = 3;  // 97 KB: two CTAs per S
 constexpr int A_BYTES = BM * BK * 2, B_BYTES = BN * BK * 2;
 constexpr int SMEM_BYTES = STAGES * (A_BYTES + B_BYTES) + 1024;  // + alignment slack
 
-enum { kEpiRope = 0, kEpiHeads = 1, kEpiPlain = 2 };
+enum { kEpiRope = 0, kEpiHeads = 1, kEpiPlain = 2, kEpiStage = 3 };
+constexpr int kMaxRanks = 8;
 
 struct TmaMaps {
     CUtensorMap a;
@@ -46,6 +48,10 @@ struct Epi {
     int S, H, d;
     const float2 *rope_hi, *rope_lo;
     unsigned long long *counters;
+    // kEpiStage: row m of the fp32 result goes to stage[c] (c = m / rows_chunk, possibly another GPU's memory)
+    // at row rank * rows_chunk + m % rows_chunk
+    float *stage[kMaxRanks];
+    int rank, rows_chunk;
 };
 
 __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y, uint64_t *mbar) {
@@ -137,6 +143,14 @@ __global__ void __launch_bounds__(192, 2) k_gemm_tc(const __grid_constant__ TmaM
             tc::tmem_ld32(trow + c0, v);
             if (!ok || m >= epi.M) continue;
             const int n = n0 + c0;
+            if (mode == kEpiStage) {
+                const int c = m / epi.rows_chunk;
+                float4 *f4 = (float4 *)(epi.stage[c] + ((size_t)epi.rank * epi.rows_chunk + (m - c * epi.rows_chunk)) *
+                                                           epi.N + n);
+#pragma unroll
+                for (int q4 = 0; q4 < 8; ++q4) f4[q4] = make_float4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
+                continue;
+            }
             bf16 *dst;
             if (mode == kEpiPlain) {
                 dst = out + (size_t)m * epi.N + n;
@@ -465,6 +479,71 @@ cudaError_t gemm_grad_tc(int M, int N, int K, int nsrc, int ngroups, const void 
         return e;
     dim3 grid((N + BN - 1) / BN, (M + BM - 1) / BM, ngroups * split);
     k_gemm_grad_tc<<<grid, 192, SMEM_BYTES, s>>>(maps, g);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+}  // namespace mono
+
+namespace mono {
+
+// ---------------------------------------------------------------------------
+// Output projection of one head shard fused with the scatter half of a
+// reduce-scatter: the fp32 tile of rows [m0, m0 + 128) goes straight from the
+// epilogue to the staging buffer of the rank that owns each row (rows split
+// into nranks equal chunks), which may be another GPU's memory reached over
+// NVLink (plain stores).  The transfer of a tile overlaps the MMAs of the
+// next tiles; no partial is rounded to bf16.
+// ---------------------------------------------------------------------------
+cudaError_t launch_out_project_stage(const Plan &p, const void *O, const void *Wo, float *const *stage, int nranks,
+                                     int rank, void *ws, cudaStream_t s) {
+    const mono_config &c = p.cfg;
+    if (!get_encode()) return cudaErrorNotSupported;
+    if (nranks < 1 || nranks > kMaxRanks) return cudaErrorInvalidValue;
+    TmaMaps maps;
+    const long long M = (long long)c.B * c.S;
+    const int Kd = c.H * c.d;
+    if (!make_map(&maps.a, O, M, Kd, BM) || !make_map(&maps.b[0], Wo, c.W, Kd, BN)) return cudaErrorInvalidValue;
+    maps.b[1] = maps.b[0];
+    maps.b[2] = maps.b[0];
+    Epi epi{};
+    epi.mode[0] = kEpiStage;
+    epi.M = (int)M; epi.N = c.W; epi.S = c.S; epi.H = c.H; epi.d = c.d;
+    epi.counters = (unsigned long long *)ws_ptr(p, ws, kRegCounters);
+    for (int r = 0; r < nranks; ++r) epi.stage[r] = stage[r];
+    epi.rank = rank;
+    epi.rows_chunk = (int)(M / nranks);
+    return launch(maps, epi, 1, Kd, s);
+}
+
+// ---------------------------------------------------------------------------
+// The reduce half: this rank's chunk is the sum of the nranks partials staged
+// for it, added in fp32 in ascending rank order and rounded once to bf16.
+// stage [nranks][rows][W] fp32 (this GPU's buffer), out [rows][W] bf16.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) k_stage_reduce(const float4 *__restrict__ stage, uint2 *__restrict__ out,
+                                                      long long n4, int nranks) {
+    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (long long)gridDim.x * blockDim.x) {
+        float4 a = __ldg(stage + i);
+        for (int r = 1; r < nranks; ++r) {
+            const float4 b = __ldg(stage + (size_t)r * n4 + i);
+            a.x = __fadd_rn(a.x, b.x);
+            a.y = __fadd_rn(a.y, b.y);
+            a.z = __fadd_rn(a.z, b.z);
+            a.w = __fadd_rn(a.w, b.w);
+        }
+        out[i] = make_uint2(pack2(a.x, a.y), pack2(a.z, a.w));
+    }
+}
+
+cudaError_t launch_stage_reduce(const Plan &p, const float *stage, int nranks, void *out, cudaStream_t s) {
+    const mono_config &c = p.cfg;
+    const long long n4 = (long long)c.B * c.S / nranks * c.W / 4;
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const long long want = (n4 + 255) / 256;
+    const int grid = (int)std::max<long long>(1, std::min<long long>(want, 8ll * sms));
+    k_stage_reduce<<<grid, 256, 0, s>>>((const float4 *)stage, (uint2 *)out, n4, nranks);
     count_launches(1);
     return cudaGetLastError();
 }

@@ -12,6 +12,8 @@ codebooks -- through the whole mixer.  Projection, routing (codebooks, posting
 lists and probes are per head) and attention of a head need nothing from the
 other heads; the output projection delta = sum_h O_h Wo_h^T leaves each rank a
 partial sum over its heads, and one all-reduce (sum) gives every rank delta.
+head_sharded_forward_fused replaces that all-reduce by the output projection
+fused with a reduce-scatter over peer memory (fp32 partials, one rounding).
 """
 from __future__ import annotations
 
@@ -129,6 +131,72 @@ def head_sharded_forward(plan, x, shard: dict, delta, ws, group=None, forced=Non
     mono.forward(plan, x, shard["Wq"], shard["Wk"], shard["Wv"], shard["Wo"], shard["codebooks"], delta, ws,
                  forced=forced, stream=stream)
     return reduce_partial_delta(delta, group, stream)
+
+
+# --- head-sharded mixer, output projection fused with the reduce-scatter ----
+
+
+def stage_rows(cfg, world: int) -> int:
+    """Token rows per rank in the reduce-scatter of the head-sharded delta: B*S split into `world` chunks."""
+    rows = cfg.B * cfg.S
+    if world < 1 or rows % world:
+        raise ValueError(f"{rows} token rows do not split evenly over {world} ranks")
+    return rows // world
+
+
+def chunk_of(cfg, world: int, rank: int) -> slice:
+    """The rows [rank * rows, (rank + 1) * rows) of the flattened [B*S, W] delta that `rank` reduces."""
+    rows = stage_rows(cfg, world)
+    return slice(rank * rows, (rank + 1) * rows)
+
+
+def alloc_stage(cfg, world: int, device, symmetric: bool = False, group=None):
+    """This rank's staging buffer [world, rows, W] fp32 for the partials the ranks send it.  With
+    `symmetric`, the buffer comes from torch's symmetric memory and the return value also lists every rank's
+    buffer as a device address this GPU can store to (NVLink peer access); else only the local buffer."""
+    shape = (world, stage_rows(cfg, world), cfg.W)
+    if not symmetric:
+        return torch.empty(shape, dtype=torch.float32, device=device), None
+    import torch.distributed._symmetric_memory as symm_mem
+    buf = symm_mem.empty(shape, dtype=torch.float32, device=device)
+    hdl = symm_mem.rendezvous(buf, group if group is not None else dist.group.WORLD)
+    return buf, [int(p) for p in hdl.buffer_ptrs]
+
+
+def head_sharded_forward_fused(plan, x, shard: dict, delta, ws, stage, stage_ptrs, rank: int, world: int,
+                               group=None, forced=None, stream=None):
+    """The mixer on this rank's heads with the output projection fused into the reduce-scatter: the GEMM
+    epilogue stores each fp32 row of the partial delta into the staging buffer of the rank that owns the row
+    (stage_ptrs, every rank's buffer from alloc_stage(symmetric=True)); a collective on the stream then orders
+    every rank's stores before this rank sums the `world` partials of its rows in fp32, in rank order, and
+    rounds once; an all-gather gives every rank the whole delta [B, S, W]."""
+    from . import mono
+    cfg = plan.cfg
+    Q, K, V, sel, O = (plan.region(ws, k) for k in ("Q", "K", "V", "sel", "O"))
+    mono.project(plan, x, shard["Wq"], shard["Wk"], shard["Wv"], Q, K, V, ws, stream)
+    mono.route(plan, Q, K, shard["codebooks"], sel, ws, forced=forced, stream=stream)
+    mono.attend(plan, Q, K, V, sel, O, ws, stream)
+    mono.out_project_scatter(plan, O, shard["Wo"], stage_ptrs, rank, ws, stream)
+    flat = delta.view(-1, cfg.W)
+    chunk = torch.empty_like(flat[chunk_of(cfg, world, rank)])
+    ctx = torch.cuda.stream(stream) if stream is not None else _null()
+    with ctx:
+        if dist.is_initialized() and world > 1:
+            dist.all_reduce(torch.zeros(1, device=delta.device), group=group)   # every rank's stores are done
+        mono.stage_reduce(plan, stage, world, chunk, stream)
+        if dist.is_initialized() and world > 1:
+            dist.all_gather_into_tensor(flat, chunk, group=group)
+        else:
+            flat.copy_(chunk)
+    return delta
+
+
+class _null:
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *a):
+        return False
 
 
 def finalize():

@@ -92,3 +92,17 @@ def test_shard_slices_and_errors():
     import torch
     t = torch.ones(3)
     assert dist.reduce_partial_delta(t) is t and float(t.sum()) == 3.0
+
+
+def test_reduce_scatter_chunks_tile_the_rows():
+    # the row chunks of the fused output-projection reduce-scatter cover the B*S rows once, in rank order
+    from learned_product_hash_proj_b200 import dist as d
+    from learned_product_hash_proj_b200 import synth
+    cfg = synth.Config(B=2, S=96, W=16, H=4, d=8, Bs=8, L=1, R=2, E=3, M=2, C=4, T=3, cap=2, dtype="f32")
+    for world in (1, 2, 3, 4):
+        rows = d.stage_rows(cfg, world)
+        got = np.concatenate([np.arange(cfg.B * cfg.S)[d.chunk_of(cfg, world, r)] for r in range(world)])
+        np.testing.assert_array_equal(got, np.arange(cfg.B * cfg.S))
+        assert rows * world == cfg.B * cfg.S
+    with pytest.raises(ValueError):
+        d.stage_rows(cfg, 5)
