@@ -182,9 +182,12 @@ int mono_route(const mono_plan_t *plan, const void *Q, const void *K, const floa
 /* The three stages of mono_route, callable one at a time (same kernels,
  * same results); each reads what the previous one left in the workspace.
  *  - mono_route_summaries: block summaries kbar and product addresses (needs K).
- *  - mono_route_lists:     bounded causal posting lists and overflow counts.
+ *  - mono_route_lists:     bounded causal posting lists and overflow counts;
+ *                          resets the routing statistics.
  *  - mono_route_queries:   probe, union, causal filter, E cap, rerank -> sel
  *                          (needs Q); also resets and fills the statistics.
+ * Inside mono_route the probe is launched so that it may start while the
+ * lists kernel still runs; it waits for the lists before reading them.
  * mono_route_summaries resets the device error word. */
 int mono_route_summaries(const mono_plan_t *plan, const void *K, const float *codebooks, void *workspace,
                          void *stream);

@@ -41,7 +41,7 @@ int validate(const mono_config *c) {
     if (c->S / c->Bs > kMaxNb) return MONO_ERR_UNSUPPORTED;
     if (c->W % 64 != 0) return MONO_ERR_UNSUPPORTED;
     if ((long long)c->B * c->H * c->S * c->d > (1ll << 40)) return MONO_ERR_UNSUPPORTED;
-    if ((c->flags & MONO_FLAG_REDIRECT) && A > 65536.0L) return MONO_ERR_UNSUPPORTED;
+    if ((c->flags & MONO_FLAG_REDIRECT) && A > (long double)kRedirectMaxA) return MONO_ERR_UNSUPPORTED;
     if (c->flags & ~(MONO_FLAG_SIMPLE_KERNELS | MONO_FLAG_REDIRECT)) return MONO_ERR_INVALID;
     return MONO_OK;
 }
@@ -217,7 +217,8 @@ int mono_route(const mono_plan_t *plan, const void *Q, const void *K, const floa
     if (forced && !aligned(forced, 4)) return MONO_ERR_ALIGN;
     if ((st = mono_route_summaries(plan, K, codebooks, workspace, stream))) return st;
     if ((st = mono_route_lists(plan, workspace, stream))) return st;
-    return mono_route_queries(plan, Q, codebooks, forced, sel, workspace, stream);
+    // the lists launch cleared the statistics: the probe follows it directly (programmatic launch)
+    return cuda_status(launch_queries(p, Q, codebooks, forced, sel, workspace, (cudaStream_t)stream, false));
 }
 
 int mono_attend(const mono_plan_t *plan, const void *Q, const void *K, const void *V, const int32_t *sel, void *O,

@@ -32,8 +32,11 @@ enum DevErr : unsigned {
 // the query-heads whose probe left the fast path for the general walk (near
 // ties in the staged top-T, or a stage with too many surviving prefixes); the
 // first kWalkLogCap of them are logged by flat index in the walk-log region.
-enum Counter { kCntQueriesLtR = 0, kCntRemoteSel = 1, kCntForcedIgnored = 2, kCntErr = 3, kCntWalks = 4, kCntN = 8 };
+// The routing statistics are the first kCntStats counters (reset together), the error word after them.
+enum Counter { kCntQueriesLtR = 0, kCntRemoteSel = 1, kCntForcedIgnored = 2, kCntWalks = 3, kCntStats = 4, kCntErr = 4,
+               kCntN = 8 };
 constexpr int kWalkLogCap = 4096;
+constexpr int kRedirectMaxA = 65536;  // largest C^M of redirect-on-overflow lists (per-address counts in shared memory)
 
 enum Region {
     kRegKbar = MONO_WS_KBAR,
@@ -106,8 +109,10 @@ cudaError_t launch_project_simt(const Plan &p, const void *x, const void *Wq, co
 cudaError_t launch_out_project_simt(const Plan &p, const void *O, const void *Wo, void *delta, cudaStream_t s);
 cudaError_t launch_summaries(const Plan &p, const void *K, const float *cb, void *ws, cudaStream_t s);
 cudaError_t launch_lists(const Plan &p, void *ws, cudaStream_t s);
+// reset_stats: clear the routing statistics first (the lists launch has done it when the two run back to back,
+// which lets the probe start while the lists kernel still runs)
 cudaError_t launch_queries(const Plan &p, const void *Q, const float *cb, const int32_t *forced, int32_t *sel,
-                           void *ws, cudaStream_t s);
+                           void *ws, cudaStream_t s, bool reset_stats = true);
 cudaError_t launch_attend_simt(const Plan &p, const void *Q, const void *K, const void *V, const int32_t *sel,
                                void *O, void *ws, cudaStream_t s);
 bool attend_tc_supported(const mono_config &c);

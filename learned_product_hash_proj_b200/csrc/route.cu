@@ -21,6 +21,14 @@
 
 namespace mono {
 
+// Programmatic dependent launch between the posting lists and the probe: the
+// lists kernel lets the probe's CTAs start at once (they load their queries
+// and score the codebooks meanwhile), and the probe waits for the lists to be
+// complete and visible only before it reads them.  Without a programmatic
+// launch the wait returns at once.
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait_primary() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ---------------------------------------------------------------------------
 // (A2, A3) block summary kbar = mean of the Bs post-RoPE keys, and the product
 // address: per subspace m the code with the largest <kbar_m, cw[h,m,c]>.
@@ -202,6 +210,7 @@ constexpr int kDenseA = 4096;
 __global__ void __launch_bounds__(1024) k_posting_dense(const int32_t *__restrict__ addr, int32_t *__restrict__ ids,
                                                         int32_t *__restrict__ saddr, int32_t *__restrict__ rank,
                                                         int32_t *__restrict__ overflow, int nb, int cap, int H, int A) {
+    pdl_launch_dependents();
     __shared__ int s_cnt[kDenseA];
     __shared__ int s_part[32];
     __shared__ int s_ov[32];
@@ -291,6 +300,7 @@ __global__ void __launch_bounds__(1024) k_posting_dense(const int32_t *__restric
 __global__ void __launch_bounds__(1024) k_posting_build(const int32_t *__restrict__ addr, int32_t *__restrict__ ids,
                                                         int32_t *__restrict__ saddr, int32_t *__restrict__ rank,
                                                         int32_t *__restrict__ overflow, int nb, int cap, int H) {
+    pdl_launch_dependents();
     extern __shared__ int32_t s_addr[];
     __shared__ int s_ov[32];
     const size_t bh = (size_t)blockIdx.y * H + blockIdx.x;
@@ -334,8 +344,6 @@ __global__ void __launch_bounds__(1024) k_posting_build(const int32_t *__restric
 // grid (H, B), 1024 threads; dynamic smem: bitmap [ceil(A/32)] u32, list
 // addresses [nb] int32, counts [A] u16 (A <= kRedirectMaxA).
 // ---------------------------------------------------------------------------
-constexpr int kRedirectMaxA = 65536;
-
 inline size_t redirect_smem(long long A, int nb) {
     return (size_t)((A + 31) / 32) * 4 + (size_t)nb * 4 + (size_t)A * 2;
 }
@@ -366,6 +374,7 @@ __global__ void __launch_bounds__(1024) k_posting_redirect(const int32_t *__rest
                                                            int32_t *__restrict__ saddr, int32_t *__restrict__ rank,
                                                            int32_t *__restrict__ overflow, int nb, int cap, int H,
                                                            int A) {
+    pdl_launch_dependents();
     extern __shared__ uint32_t s_red[];
     const int nw = (A + 31) / 32;
     uint32_t *s_full = s_red;                          // [nw]: bit set = list full (and every bit past A)
@@ -493,6 +502,7 @@ __global__ void __launch_bounds__(128) k_probe_rerank(const T *__restrict__ Q, c
                                                       unsigned long long *__restrict__ counters,
                                                       int32_t *__restrict__ walk_log, int S, int H, int Bs,
                                                       int L, int R, int E, int M, int C, int Tp, int cap) {
+    pdl_wait_primary();  // the posting lists are complete
     extern __shared__ float smem[];
     const int nb = S / Bs;
     float *s_cb = smem;                                     // [M*C*dm] = C*D floats
@@ -1136,17 +1146,6 @@ __global__ void __launch_bounds__(128, C <= 16 ? 4 : 3) k_probe_m2(const T *__re
             const bool ok = t_lo + r < S;
             tc::cp_async16(s_q + r * QP + 16 * c, ok ? (const void *)(src + (size_t)r * (D * sizeof(T)) + 16 * c) : Q, ok);
         }
-        if ((nb & 3) == 0) {  // 16-byte aligned rows of the posting arrays
-            for (int i = tid; i < nb / 4; i += blockDim.x) {
-                tc::cp_async16(s_addr + 4 * i, post_addr + bh * nb + 4 * i, true);
-                tc::cp_async16(s_ids + 4 * i, post_ids + bh * nb + 4 * i, true);
-            }
-        } else {
-            for (int i = tid; i < nb; i += blockDim.x) {
-                s_addr[i] = post_addr[bh * nb + i];
-                s_ids[i] = post_ids[bh * nb + i];
-            }
-        }
     }
     // the head's codebooks ([2][C][DM] floats), transposed, with independent 16-byte loads
     {
@@ -1164,16 +1163,6 @@ __global__ void __launch_bounds__(128, C <= 16 ? 4 : 3) k_probe_m2(const T *__re
     for (int i = tid; i < A; i += blockDim.x) s_rng[i] = make_int2(0, 0);
     tc::cp_async_wait_all();
     __syncthreads();
-    // the posting arrays are sorted by address: each address's entries start
-    // where the address differs from the previous entry's and end where it
-    // differs from the next one's
-    for (int i = tid; i < nb; i += blockDim.x) {
-        const int a = s_addr[i];
-        if ((unsigned)a >= (unsigned)A) continue;
-        if (i == 0 || s_addr[i - 1] != a) s_rng[a].x = i;
-        if (i == nb - 1 || s_addr[i + 1] != a) s_rng[a].y = i + 1;
-    }
-    __syncthreads();
 
     // subspace scores of this thread's queries (rows past S are zeros and are not routed)
     float s0[NQ][C], s1[NQ][C];
@@ -1187,6 +1176,32 @@ __global__ void __launch_bounds__(128, C <= 16 ? 4 : 3) k_probe_m2(const T *__re
         sub_scores_x2<T, DM, C, NQ>(qm0, s_cbT, s0);
         sub_scores_x2<T, DM, C, NQ>(qm1, s_cbT + DM * C, s1);
     }
+
+    // the posting lists: complete once the lists kernel is (programmatic launch)
+    pdl_wait_primary();
+    if ((nb & 3) == 0) {  // 16-byte aligned rows of the posting arrays
+        for (int i = tid; i < nb / 4; i += blockDim.x) {
+            tc::cp_async16(s_addr + 4 * i, post_addr + bh * nb + 4 * i, true);
+            tc::cp_async16(s_ids + 4 * i, post_ids + bh * nb + 4 * i, true);
+        }
+    } else {
+        for (int i = tid; i < nb; i += blockDim.x) {
+            s_addr[i] = post_addr[bh * nb + i];
+            s_ids[i] = post_ids[bh * nb + i];
+        }
+    }
+    tc::cp_async_wait_all();
+    __syncthreads();
+    // the posting arrays are sorted by address: each address's entries start
+    // where the address differs from the previous entry's and end where it
+    // differs from the next one's
+    for (int i = tid; i < nb; i += blockDim.x) {
+        const int a = s_addr[i];
+        if ((unsigned)a >= (unsigned)A) continue;
+        if (i == 0 || s_addr[i - 1] != a) s_rng[a].x = i;
+        if (i == nb - 1 || s_addr[i + 1] != a) s_rng[a].y = i + 1;
+    }
+    __syncthreads();
     int n_sel = 0, lt_r = 0, ign = 0;
     const float *kb = kbar + bh * nb * D;
 #pragma unroll
@@ -1259,6 +1274,8 @@ cudaError_t launch_summaries(const Plan &p, const void *K, const float *cb, void
 
 cudaError_t launch_lists(const Plan &p, void *ws, cudaStream_t s) {
     const mono_config &c = p.cfg;
+    // the statistics the probe fills (so that the probe can follow this kernel directly)
+    if (cudaError_t e0 = cudaMemsetAsync(ws_ptr(p, ws, kRegCounters), 0, kCntStats * 8, s)) return e0;
     dim3 g2(c.H, c.B);
     const int32_t *addr = (const int32_t *)ws_ptr(p, ws, kRegAddr);
     int32_t *ids = (int32_t *)ws_ptr(p, ws, kRegPostIds), *saddr = (int32_t *)ws_ptr(p, ws, kRegPostAddr);
@@ -1292,14 +1309,32 @@ cudaError_t launch_lists(const Plan &p, void *ws, cudaStream_t s) {
     return cudaGetLastError();
 }
 
+// a probe kernel, launched so that it may start while the lists kernel before
+// it on the stream still runs (it waits for the lists itself: pdl_wait_primary)
+template <typename... KArgs, typename... Args>
+static cudaError_t launch_after_lists(void (*kern)(KArgs...), dim3 grid, size_t smem, cudaStream_t s,
+                                      Args... args) {
+    cudaLaunchConfig_t lc = {};
+    lc.gridDim = grid;
+    lc.blockDim = dim3(128);
+    lc.dynamicSmemBytes = smem;
+    lc.stream = s;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    lc.attrs = at;
+    lc.numAttrs = 1;
+    return cudaLaunchKernelEx(&lc, kern, (KArgs)args...);
+}
+
 cudaError_t launch_queries(const Plan &p, const void *Q, const float *cb, const int32_t *forced, int32_t *sel,
-                           void *ws, cudaStream_t s) {
+                           void *ws, cudaStream_t s, bool reset_stats) {
     const mono_config &c = p.cfg;
     unsigned long long *cnt = (unsigned long long *)ws_ptr(p, ws, kRegCounters);
     int32_t *walk_log = (int32_t *)ws_ptr(p, ws, kRegWalkLog);
-    cudaError_t e = cudaMemsetAsync(cnt, 0, 3 * 8, s);  // statistics; the error word is kept
-    if (e != cudaSuccess) return e;
-    if ((e = cudaMemsetAsync(cnt + kCntWalks, 0, 8, s)) != cudaSuccess) return e;
+    cudaError_t e = cudaSuccess;
+    if (reset_stats && (e = cudaMemsetAsync(cnt, 0, kCntStats * 8, s)) != cudaSuccess)  // the error word is kept
+        return e;
     if (c.R == 0) return cudaSuccess;  // nothing to select: sel has no entries
     const float *kbar = (const float *)ws_ptr(p, ws, kRegKbar);
     const int32_t *ids = (const int32_t *)ws_ptr(p, ws, kRegPostIds);
@@ -1315,8 +1350,9 @@ cudaError_t launch_queries(const Plan &p, const void *Q, const float *cb, const 
             (e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm2)) != cudaSuccess) \
             return e;                                                                                            \
         const dim3 gm2((c.S + 128 * probe_nq<CC>() - 1) / (128 * probe_nq<CC>()), c.H, c.B);                  \
-        kern<<<gm2, 128, sm2, s>>>((const TT *)Q, kbar, cb, ids, saddr, forced, sel, cnt, walk_log, c.S, c.H, c.Bs, c.L, \
-                                  c.cap);                                                                        \
+        if ((e = launch_after_lists(kern, gm2, sm2, s, (const TT *)Q, kbar, cb, ids, saddr, forced, sel, cnt,        \
+                                    walk_log, c.S, c.H, c.Bs, c.L, c.cap)) != cudaSuccess)                          \
+            return e;                                                                                            \
         count_launches(1);                                                                                       \
         return cudaGetLastError();                                                                               \
     }
@@ -1336,9 +1372,9 @@ cudaError_t launch_queries(const Plan &p, const void *Q, const float *cb, const 
             e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);                \
             if (e != cudaSuccess) return e;                                                                        \
         }                                                                                                          \
-        kern<<<g3, 128, smem, s>>>((const TT *)Q, kbar, cb, ids, saddr, forced, sel, cnt, walk_log, c.S, c.H,    \
-                                   c.Bs, c.L,                                                                      \
-                                   c.R, c.E, c.M, c.C, c.T, c.cap);                                                \
+        if ((e = launch_after_lists(kern, g3, smem, s, (const TT *)Q, kbar, cb, ids, saddr, forced, sel, cnt,        \
+                                    walk_log, c.S, c.H, c.Bs, c.L, c.R, c.E, c.M, c.C, c.T, c.cap)) != cudaSuccess)  \
+            return e;                                                                                              \
     } while (0)
     if (bf && c.d == 64) MONO_LAUNCH_PR(__nv_bfloat16, 64);
     else if (bf) MONO_LAUNCH_PR(__nv_bfloat16, 128);

@@ -101,7 +101,7 @@ int mono_route_static(const mono_plan_t *plan, const void *Q, const void *K, con
     cudaStream_t s = (cudaStream_t)stream;
     if (launch_summaries(rp, K, codebooks, scratch, s) != cudaSuccess) return MONO_ERR_CUDA;
     if (launch_lists(rp, scratch, s) != cudaSuccess) return MONO_ERR_CUDA;
-    if (launch_queries(rp, Q, codebooks, forced, sel, scratch, s) != cudaSuccess) return MONO_ERR_CUDA;
+    if (launch_queries(rp, Q, codebooks, forced, sel, scratch, s, false) != cudaSuccess) return MONO_ERR_CUDA;
     return MONO_OK;
 }
 
