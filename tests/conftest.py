@@ -15,11 +15,12 @@ def pytest_configure(config):
 
 
 def pytest_terminal_summary(terminalreporter):
-    """Print the routing counts the GPU parity tests recorded (queries checked per workload, selections that
-    differ from the fp64 oracle and the margins behind them)."""
+    """Print what the GPU parity tests recorded: per workload the queries whose routing was checked against the
+    oracle (fp32 bit-exact, fp64 margin rule) with the counts of differences and small margins; per gradient the
+    error ratio against its bound."""
     mod = sys.modules.get("gpu_parity")
-    lines = getattr(mod, "ROUTING_LOG", None)
+    lines = getattr(mod, "PARITY_LOG", None)
     if lines:
-        terminalreporter.section("routing against the oracle (fp32 bit-exact, fp64 margin rule)")
+        terminalreporter.section("parity against the oracle")
         for line in lines:
             terminalreporter.write_line(line)

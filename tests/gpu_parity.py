@@ -219,7 +219,7 @@ def check_out_projection(run: Run, rows=None):
 # routing of whole (b, h) slices against both statements of the oracle, in
 # threads (the oracle's C calls release the interpreter lock)
 # ---------------------------------------------------------------------------
-ROUTING_LOG: list[str] = []  # per workload: queries checked and counts against the fp64 oracle (printed at the end)
+PARITY_LOG: list[str] = []  # per workload: queries checked and counts against the fp64 oracle (printed at the end)
 FP64_MARGIN = 1e-4          # decisions closer than this may differ from the fp64 oracle ...
 FP64_MAX_SHARE = 1e-3       # ... on fewer than 0.1 % of the queries
 
@@ -306,7 +306,7 @@ def check_fp64_rule(run):
 
 def log_routing(run, info: dict, what: str = ""):
     cfg = run.cfg
-    ROUTING_LOG.append(f"{cfg.name}{what} B={cfg.B} S={cfg.S} H={cfg.H} A={cfg.A} {cfg.dtype}: " +
+    PARITY_LOG.append(f"{cfg.name}{what} B={cfg.B} S={cfg.S} H={cfg.H} A={cfg.A} {cfg.dtype}: " +
                        " ".join(f"{k}={v}" for k, v in info.items()))
 
 

@@ -54,6 +54,8 @@ def close(got, ref, rel, what):
     got, ref = np.asarray(got, np.float64), np.asarray(ref, np.float64)
     rms = float(np.sqrt(np.mean(ref * ref)))
     err = float(np.abs(got - ref).max())
+    import gpu_parity
+    gpu_parity.PARITY_LOG.append(f"backward {what}: max |err| / RMS = {err / max(rms, 1e-300):.3e} (bound {rel})")
     assert err <= rel * rms + 1e-7, f"{what}: max |err| {err:.3e} > {rel} x RMS {rms:.3e}"
 
 
@@ -78,6 +80,8 @@ FULL_CASES = {
     "bf16": dict(dtype="bf16"),
     # widths off the 128-wide tensor-core tiles: ragged tiles in every gradient GEMM, split K in dWq/dWk/dWv
     "bf16_ragged": dict(dtype="bf16", S=320, W=192, H=3),
+    # a longer sequence: 64 blocks of 64, selections reaching far back
+    "bf16_S4096": dict(dtype="bf16", B=1, S=4096, Bs=64, C=16, cap=8),
 }
 
 
