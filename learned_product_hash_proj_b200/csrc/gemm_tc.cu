@@ -70,6 +70,45 @@ __device__ __forceinline__ uint32_t pack2(float a, float b) {
     return *(uint32_t *)&h;
 }
 
+// 32 accumulator columns n .. n+31 of output row m: RoPE (kEpiRope) on
+// interleaved pairs, bf16, to [B,H,S,d] (kEpiRope, kEpiHeads) or row-major
+// [M, N] (kEpiPlain); fp32 to the owner's staging buffer (kEpiStage)
+__device__ __forceinline__ void epi_store(const Epi &epi, int mode, bf16 *out, int half, int m, int n, float (&v)[32]) {
+    if (mode == kEpiStage) {
+        const int c = m / epi.rows_chunk;
+        float4 *f4 = (float4 *)(epi.stage[c] + ((size_t)epi.rank * epi.rows_chunk + (m - c * epi.rows_chunk)) * epi.N +
+                                n);
+#pragma unroll
+        for (int q4 = 0; q4 < 8; ++q4) f4[q4] = make_float4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
+        return;
+    }
+    bf16 *dst;
+    if (mode == kEpiPlain) {
+        dst = out + (size_t)m * epi.N + n;
+    } else {
+        const int b = m / epi.S, t = m % epi.S;
+        const int h = n / epi.d, i0 = n % epi.d;
+        if (mode == kEpiRope) {
+            const float2 *hi = epi.rope_hi + (size_t)(t / kRopeLo) * half + i0 / 2;
+            const float2 *lo = epi.rope_lo + (size_t)(t % kRopeLo) * half + i0 / 2;
+#pragma unroll
+            for (int pr = 0; pr < 16; ++pr) {
+                const float2 a = __ldg(hi + pr), bb = __ldg(lo + pr);
+                const float c = a.x * bb.x - a.y * bb.y, sn = a.y * bb.x + a.x * bb.y;
+                const float x0 = v[2 * pr], x1 = v[2 * pr + 1];
+                v[2 * pr] = x0 * c - x1 * sn;
+                v[2 * pr + 1] = x0 * sn + x1 * c;
+            }
+        }
+        dst = out + (((size_t)b * epi.H + h) * epi.S + t) * epi.d + i0;
+    }
+    uint4 *d4 = (uint4 *)dst;
+#pragma unroll
+    for (int q8 = 0; q8 < 4; ++q8)
+        d4[q8] = make_uint4(pack2(v[8 * q8], v[8 * q8 + 1]), pack2(v[8 * q8 + 2], v[8 * q8 + 3]),
+                            pack2(v[8 * q8 + 4], v[8 * q8 + 5]), pack2(v[8 * q8 + 6], v[8 * q8 + 7]));
+}
+
 __global__ void __launch_bounds__(192, 2) k_gemm_tc(const __grid_constant__ TmaMaps maps, const Epi epi, int K) {
     extern __shared__ uint8_t smem_raw[];
     __shared__ uint64_t full[STAGES], empty[STAGES], accf;
@@ -142,40 +181,7 @@ __global__ void __launch_bounds__(192, 2) k_gemm_tc(const __grid_constant__ TmaM
             float v[32];
             tc::tmem_ld32(trow + c0, v);
             if (!ok || m >= epi.M) continue;
-            const int n = n0 + c0;
-            if (mode == kEpiStage) {
-                const int c = m / epi.rows_chunk;
-                float4 *f4 = (float4 *)(epi.stage[c] + ((size_t)epi.rank * epi.rows_chunk + (m - c * epi.rows_chunk)) *
-                                                           epi.N + n);
-#pragma unroll
-                for (int q4 = 0; q4 < 8; ++q4) f4[q4] = make_float4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
-                continue;
-            }
-            bf16 *dst;
-            if (mode == kEpiPlain) {
-                dst = out + (size_t)m * epi.N + n;
-            } else {
-                const int b = m / epi.S, t = m % epi.S;
-                const int h = n / epi.d, i0 = n % epi.d;
-                if (mode == kEpiRope) {
-                    const float2 *hi = epi.rope_hi + (size_t)(t / kRopeLo) * half + i0 / 2;
-                    const float2 *lo = epi.rope_lo + (size_t)(t % kRopeLo) * half + i0 / 2;
-#pragma unroll
-                    for (int pr = 0; pr < 16; ++pr) {
-                        const float2 a = __ldg(hi + pr), bb = __ldg(lo + pr);
-                        const float c = a.x * bb.x - a.y * bb.y, sn = a.y * bb.x + a.x * bb.y;
-                        const float x0 = v[2 * pr], x1 = v[2 * pr + 1];
-                        v[2 * pr] = x0 * c - x1 * sn;
-                        v[2 * pr + 1] = x0 * sn + x1 * c;
-                    }
-                }
-                dst = out + (((size_t)b * epi.H + h) * epi.S + t) * epi.d + i0;
-            }
-            uint4 *d4 = (uint4 *)dst;
-#pragma unroll
-            for (int q8 = 0; q8 < 4; ++q8)
-                d4[q8] = make_uint4(pack2(v[8 * q8], v[8 * q8 + 1]), pack2(v[8 * q8 + 2], v[8 * q8 + 3]),
-                                    pack2(v[8 * q8 + 4], v[8 * q8 + 5]), pack2(v[8 * q8 + 6], v[8 * q8 + 7]));
+            epi_store(epi, mode, out, half, m, n0 + c0, v);
         }
         if (!ok && lane == 0) fail = 1;
     }
@@ -183,6 +189,141 @@ __global__ void __launch_bounds__(192, 2) k_gemm_tc(const __grid_constant__ TmaM
     __syncthreads();
     if (tid == 0 && fail) record_error(epi.counters, kDevErrTimeout);
     if (warp == 1) tc::tmem_dealloc(tmem, BN);
+}
+
+// ---------------------------------------------------------------------------
+// The same product as a persistent kernel with 128 x 256 tiles: one CTA per SM
+// walks the tiles (the n tiles and outputs of one 128-row band of A first, so
+// that concurrent CTAs share A in L2).  The producer runs ahead across tile
+// boundaries through a 4-stage ring of 48 KB stages; the MMA issuer
+// alternates two 128 x 256 fp32 accumulators in TMEM (all 512 columns), so
+// the epilogue of tile i (four warps, TMEM -> registers -> RoPE -> bf16
+// stores) overlaps the MMAs of tile i+1.
+// ---------------------------------------------------------------------------
+constexpr int PBN = 256, PSTAGES = 4;
+constexpr int PB_BYTES = PBN * BK * 2;
+constexpr int PSMEM_BYTES = PSTAGES * (A_BYTES + PB_BYTES) + 1024;
+
+__global__ void __launch_bounds__(192, 1) k_gemm_tcp(const __grid_constant__ TmaMaps maps, const Epi epi, int K,
+                                                     int tiles_n, int tiles_m, int nz) {
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ uint64_t full[PSTAGES], empty[PSTAGES], accf[2], accfree[2], drain;
+    __shared__ uint32_t tmem_base;
+    __shared__ int fail;
+    uint8_t *base = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int nk = K / BK;
+    const int total = tiles_n * tiles_m * nz;
+    const int G = gridDim.x;
+    auto tile_of = [&](int t, int &m0, int &n0, int &z) {
+        const int per_m = tiles_n * nz;
+        m0 = (t / per_m) * BM;
+        const int r = t % per_m;
+        z = r / tiles_n;
+        n0 = (r % tiles_n) * PBN;
+    };
+    if (tid == 0) {
+        for (int s = 0; s < PSTAGES; ++s) {
+            tc::mbar_init(&full[s], 1);
+            tc::mbar_init(&empty[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            tc::mbar_init(&accf[a], 1);
+            tc::mbar_init(&accfree[a], 4);
+        }
+        tc::mbar_init(&drain, 1);
+        tc::fence_mbar_init();
+        fail = 0;
+    }
+    if (warp == 1) {
+        tc::tmem_alloc(&tmem_base, 2 * PBN);
+        tc::tmem_relinquish();
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = tmem_base;
+
+    if (warp == 0 && lane == 0) {
+        // producer: every k slice of every tile of this CTA, one ring
+        int kc = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < total && ok; t += G) {
+            int m0, n0, z;
+            tile_of(t, m0, n0, z);
+            for (int k = 0; k < nk; ++k, ++kc) {
+                const int s = kc % PSTAGES;
+                if (kc >= PSTAGES && !tc::mbar_wait(&empty[s], ((kc / PSTAGES) - 1) & 1)) { ok = false; break; }
+                uint8_t *sa = base + s * (A_BYTES + PB_BYTES);
+                uint8_t *sb = sa + A_BYTES;
+                mbar_expect_tx(&full[s], A_BYTES + PB_BYTES);
+                tma_load_2d(sa, &maps.a, k * BK, m0, &full[s]);
+                tma_load_2d(sb, &maps.b[z], k * BK, n0, &full[s]);
+            }
+        }
+        if (!ok) {
+            fail = 1;
+            // leave no copy in flight: the last load of each stage has landed
+            for (int j = kc - 1; j >= 0 && j >= kc - PSTAGES; --j) tc::mbar_wait(&full[j % PSTAGES], (j / PSTAGES) & 1);
+        }
+    } else if (warp == 1 && lane == 0) {
+        // MMA issuer: tile lt of this CTA into accumulator lt & 1
+        const uint32_t id = tc::idesc_bf16(BM, PBN);
+        int kc = 0, lt = 0;
+        for (int t = blockIdx.x; t < total && !fail; t += G, ++lt) {
+            const int a = lt & 1;
+            if (lt >= 2 && !tc::mbar_wait(&accfree[a], ((lt >> 1) - 1) & 1, 1u << 20)) { fail = 1; break; }
+            tc::fence_after_sync();
+            bool ok = true;
+            for (int k = 0; k < nk; ++k, ++kc) {
+                const int s = kc % PSTAGES;
+                if (!tc::mbar_wait(&full[s], (kc / PSTAGES) & 1)) { ok = false; break; }
+                tc::fence_after_sync();
+                const uint32_t sa = tc::smem_u32(base + s * (A_BYTES + PB_BYTES));
+                const uint32_t sb = sa + A_BYTES;
+#pragma unroll
+                for (int kk = 0; kk < BK / 16; ++kk)
+                    tc::mma_bf16(tmem + a * PBN, desc_sw128(sa + 32 * kk), desc_sw128(sb + 32 * kk), id,
+                                 (k | kk) != 0);
+                tc::commit(&empty[s]);
+            }
+            if (!ok) { fail = 1; break; }
+            tc::commit(&accf[a]);
+        }
+        // every MMA issued has completed before the CTA frees its tensor memory
+        tc::commit(&drain);
+        if (!tc::mbar_wait(&drain, 0, 1u << 20)) fail = 1;
+    } else if (warp >= 2) {
+        // epilogue: warp w reads TMEM lanes 32*(w%4) .. +31 = tile rows
+        const int q = warp & 3;
+        const int half = epi.d / 2;
+        int lt = 0;
+        for (int t = blockIdx.x; t < total; t += G, ++lt) {
+            int m0, n0, z;
+            tile_of(t, m0, n0, z);
+            const int a = lt & 1;
+            const bool ok = __all_sync(0xffffffffu, tc::mbar_wait(&accf[a], (lt >> 1) & 1, 1u << 20));
+            if (!ok) { if (lane == 0) fail = 1; break; }
+            tc::fence_after_sync();
+            const uint32_t trow = tmem + a * PBN + ((uint32_t)(q * 32) << 16);
+            const int m = m0 + q * 32 + lane;
+            const int mode = epi.mode[z];
+            bf16 *out = epi.out[z];
+            for (int c0 = 0; c0 < PBN; c0 += 32) {
+                float v[32];
+                __syncwarp();
+                tc::tmem_ld32(trow + c0, v);
+                if (m < epi.M) epi_store(epi, mode, out, half, m, n0 + c0, v);
+            }
+            tc::fence_before_sync();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&accfree[a]);
+        }
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    if (tid == 0 && fail) record_error(epi.counters, kDevErrTimeout);
+    if (warp == 1) tc::tmem_dealloc(tmem, 2 * PBN);
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
@@ -231,6 +372,21 @@ cudaError_t launch(const TmaMaps &maps, const Epi &epi, int nz, int K, cudaStrea
     return cudaGetLastError();
 }
 
+// the persistent 128 x 256 kernel; `maps.b` boxes 256 rows
+cudaError_t launch_persistent(const TmaMaps &maps, const Epi &epi, int nz, int K, cudaStream_t s) {
+    cudaError_t e = cudaFuncSetAttribute(k_gemm_tcp, cudaFuncAttributeMaxDynamicSharedMemorySize, PSMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    int dev = 0, sms = 148;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+        return e;
+    const int tn = epi.N / PBN, tm = (epi.M + BM - 1) / BM;
+    const int total = tn * tm * nz;
+    k_gemm_tcp<<<std::min(total, sms), 192, PSMEM_BYTES, s>>>(maps, epi, K, tn, tm, nz);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
 }  // namespace
 
 bool gemm_tc_supported(const mono_config &c) {
@@ -256,6 +412,12 @@ cudaError_t launch_project_tc(const Plan &p, const void *x, const void *Wq, cons
     epi.rope_hi = (const float2 *)ws_ptr(p, (void *)ws, kRegRope);
     epi.rope_lo = epi.rope_hi + (size_t)nhi * half;
     epi.counters = (unsigned long long *)ws_ptr(p, (void *)ws, kRegCounters);
+    if (N % PBN == 0) {
+        if (!make_map(&maps.b[0], Wq, N, c.W, PBN) || !make_map(&maps.b[1], Wk, N, c.W, PBN) ||
+            !make_map(&maps.b[2], Wv, N, c.W, PBN))
+            return cudaErrorInvalidValue;
+        return launch_persistent(maps, epi, 3, c.W, s);
+    }
     return launch(maps, epi, 3, c.W, s);
 }
 
@@ -273,6 +435,12 @@ cudaError_t launch_out_project_tc(const Plan &p, const void *O, const void *Wo, 
     epi.mode[0] = kEpiPlain;
     epi.M = (int)M; epi.N = c.W; epi.S = c.S; epi.H = c.H; epi.d = c.d;
     epi.counters = (unsigned long long *)ws_ptr(p, ws, kRegCounters);
+    if (c.W % PBN == 0) {
+        if (!make_map(&maps.b[0], Wo, c.W, Kd, PBN)) return cudaErrorInvalidValue;
+        maps.b[1] = maps.b[0];
+        maps.b[2] = maps.b[0];
+        return launch_persistent(maps, epi, 1, Kd, s);
+    }
     return launch(maps, epi, 1, Kd, s);
 }
 
