@@ -43,17 +43,41 @@ constexpr int kChunk = 128;   // queries per remote work item
 constexpr int kMaxGroup = 256;               // (b, h) slices per launch group
 constexpr int kQTile = 1024;  // queries per CTA of the count and fill kernels
 
-// grid (ceil(S/kQTile), B*H), 256 threads, smem nb ints
-__global__ void __launch_bounds__(256) k_pair_count(const int32_t *__restrict__ sel, int32_t *__restrict__ cnt,
-                                                    int S, int R, int nb, int Bs, int L,
-                                                    unsigned long long *__restrict__ counters) {
+// Programmatic dependent launch along the attention's kernels: each kernel
+// lets its successor's CTAs start at once, and each waits for its
+// predecessor's results only before reading them (without a programmatic
+// launch the wait returns at once).
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// One (b, h) slice per CTA: the number of queries selecting each block (a
+// shared-memory histogram of sel), its exclusive scan, the fill cursors reset,
+// and one work item {block, first pair, pair count, 0} per chunk of <= kChunk
+// queries.  Also clears the slice's done counter (and its launch group's
+// ticket) of the fused kernel.  Nothing has to be zeroed before it runs.
+// grid B*H, 1024 threads, smem nb ints.
+__global__ void __launch_bounds__(1024) k_pair_count_scan(const int32_t *__restrict__ sel, int32_t *__restrict__ start,
+                                                          int32_t *__restrict__ fill, int4 *__restrict__ work,
+                                                          int32_t *__restrict__ nwork, int *__restrict__ done,
+                                                          int *__restrict__ tickets, int S, int R, int nb, int Bs,
+                                                          int L, int wcap, int group,
+                                                          unsigned long long *__restrict__ counters) {
     extern __shared__ int s_h[];
-    const long long bh = blockIdx.y;
+    __shared__ int s_w[32], s_c[32];
+    __shared__ int carry_p, carry_c;
+    pdl_trigger();
+    const long long bh = blockIdx.x;
     for (int j = threadIdx.x; j < nb; j += blockDim.x) s_h[j] = 0;
+    if (threadIdx.x == 0) {
+        carry_p = 0;
+        carry_c = 0;
+        done[bh] = 0;
+        if (bh % group == 0) tickets[bh / group] = 0;
+    }
+    pdl_wait();  // sel is complete
     __syncthreads();
-    const int t0 = blockIdx.x * kQTile, t1 = min(S, t0 + kQTile);
     bool bad = false;
-    for (int t = t0 + threadIdx.x; t < t1; t += blockDim.x)
+    for (int t = threadIdx.x; t < S; t += blockDim.x)
         for (int r = 0; r < R; ++r) {
             const int j = sel[((size_t)bh * S + t) * R + r];
             if (sel_valid(j, t, Bs, L)) atomicAdd(&s_h[j], 1);
@@ -61,26 +85,11 @@ __global__ void __launch_bounds__(256) k_pair_count(const int32_t *__restrict__ 
         }
     if (bad) record_error(counters, kDevErrBadSel);
     __syncthreads();
-    for (int j = threadIdx.x; j < nb; j += blockDim.x)
-        if (s_h[j]) atomicAdd(&cnt[bh * nb + j], s_h[j]);
-}
-
-// exclusive scan of one (b, h)'s bucket sizes, fill cursors reset, and one
-// work item {block, first pair, pair count, 0} per chunk of <= kChunk
-// queries.  grid B*H, 1024 threads.
-__global__ void __launch_bounds__(1024) k_pair_scan(const int32_t *__restrict__ cnt, int32_t *__restrict__ start,
-                                                    int32_t *__restrict__ fill, int4 *__restrict__ work,
-                                                    int32_t *__restrict__ nwork, int nb, int wcap) {
-    __shared__ int s_w[32], s_c[32];
-    __shared__ int carry_p, carry_c;
-    const long long bh = blockIdx.x;
-    if (threadIdx.x == 0) { carry_p = 0; carry_c = 0; }
-    __syncthreads();
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int nw = blockDim.x >> 5;
     for (int base = 0; base < nb; base += blockDim.x) {
         const int j = base + threadIdx.x;
-        const int c = j < nb ? cnt[bh * nb + j] : 0;
+        const int c = j < nb ? s_h[j] : 0;
         const int ch = (c + kChunk - 1) / kChunk;
         int xp = c, xc = ch;  // inclusive warp scans
 #pragma unroll
@@ -125,8 +134,10 @@ __global__ void __launch_bounds__(256) k_pair_fill(const int32_t *__restrict__ s
                                                    int R, int nb, int Bs, int L) {
     extern __shared__ int s_h[];
     int *s_base = s_h + nb;
+    pdl_trigger();
     const long long bh = blockIdx.y;
     for (int j = threadIdx.x; j < nb; j += blockDim.x) s_h[j] = 0;
+    pdl_wait();  // the bucket starts and cleared cursors
     __syncthreads();
     const int t0 = blockIdx.x * kQTile, t1 = min(S, t0 + kQTile);
     constexpr int kPer = (kQTile / 256) * kMaxR;   // pairs one thread can hold
@@ -1428,6 +1439,7 @@ __global__ void __launch_bounds__(320, 1) k_attend_ws(const __grid_constant__ At
     const int ntiles = (S + 127) / 128;
     auto stage_q = [&](int s) { return smem + s * STAGE; };
     auto stage_rec = [&](int s) { return (int *)(smem + s * STAGE + QB + 2 * KVB); };  // [128] ids, kind, slice, n|t0
+    pdl_wait();  // the work items, pair ids, done counters and ticket are ready
 
     if (tid == 0) {
         int acc = 0;
@@ -1895,6 +1907,24 @@ static bool make_map_3d(CUtensorMap *map, const void *ptr, int D, int S, int BH,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// a kernel launched so that it may start while the kernel before it on the
+// stream still runs (it waits for its predecessor itself: pdl_wait)
+template <typename... KArgs, typename... Args>
+static cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                              Args... args) {
+    cudaLaunchConfig_t lc = {};
+    lc.gridDim = grid;
+    lc.blockDim = block;
+    lc.dynamicSmemBytes = smem;
+    lc.stream = s;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    lc.attrs = at;
+    lc.numAttrs = 1;
+    return cudaLaunchKernelEx(&lc, kern, (KArgs)args...);
+}
+
 template <int D, int BS, int NK, int RMAX>
 static cudaError_t launch_tc_shape(const Plan &p, const bf16 *Q, const bf16 *K, const bf16 *V, const int32_t *sel,
                                    bf16 *O, void *ws, cudaStream_t s, int parts) {
@@ -1912,27 +1942,29 @@ static cudaError_t launch_tc_shape(const Plan &p, const bf16 *Q, const bf16 *K, 
     // the warp-specialised remote kernel where its ring fits (every tensor-core shape), else the two-stage one
     constexpr bool kRemoteWs = RemoteWs<D, BS>::supported;
     if (c.R > 0 && (parts & kAttendPairs)) {
-        int32_t *pc = (int32_t *)ws_ptr(p, ws, kRegPairCount);
         int32_t *ps = (int32_t *)ws_ptr(p, ws, kRegPairStart);
         int32_t *pf = (int32_t *)ws_ptr(p, ws, kRegPairFill);
         int32_t *pairs = (int32_t *)ws_ptr(p, ws, kRegPairs);
         int4 *work = (int4 *)ws_ptr(p, ws, kRegWork);
         int32_t *nwork = (int32_t *)ws_ptr(p, ws, kRegNWork);
-        if ((e = cudaMemsetAsync(pc, 0, (size_t)nbh * 4, s)) != cudaSuccess) return e;
+        int *done = (int *)ws_ptr(p, ws, kRegDone);
         const int nbhh = c.B * c.H;
         const int wcap = p.max_work;  // work items per (b, h)
-        dim3 gq((c.S + kQTile - 1) / kQTile, nbhh);
+        const int grp = std::min(kMaxGroup, nbhh);
         const size_t hs = (size_t)p.nb * 4;
         if (2 * hs > 48 * 1024) {
-            if ((e = cudaFuncSetAttribute(k_pair_count, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)hs)) ||
+            if ((e = cudaFuncSetAttribute(k_pair_count_scan, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)hs)) ||
                 (e = cudaFuncSetAttribute(k_pair_fill, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)(2 * hs))))
                 return e;
         }
-        k_pair_count<<<gq, 256, hs, s>>>(sel, pc, c.S, c.R, p.nb, c.Bs, c.L, cnt_err);
-        k_pair_scan<<<nbhh, 1024, 0, s>>>(pc, ps, pf, work, nwork, p.nb, wcap);
-        k_pair_fill<<<gq, 256, 2 * hs, s>>>(sel, ps, pf, pairs, c.S, c.R, p.nb, c.Bs, c.L);
-        count_launches(3);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        if ((e = launch_pdl(k_pair_count_scan, dim3(nbhh), dim3(1024), hs, s, sel, ps, pf, work, nwork, done,
+                            done + nbhh, c.S, c.R, p.nb, c.Bs, c.L, wcap, grp, cnt_err)) != cudaSuccess)
+            return e;
+        dim3 gq((c.S + kQTile - 1) / kQTile, nbhh);
+        if ((e = launch_pdl(k_pair_fill, gq, dim3(256), 2 * hs, s, sel, (const int32_t *)ps, pf, pairs, c.S, c.R, p.nb,
+                            c.Bs, c.L)) != cudaSuccess)
+            return e;
+        count_launches(2);
     }
     if (c.R > 0 && (parts & kAttendRemote)) {
         if constexpr (kRemoteWs) {
@@ -1989,23 +2021,21 @@ static cudaError_t launch_tc_shape(const Plan &p, const bf16 *Q, const bf16 *K, 
             auto kf = k_attend_ws<D, BS, NK, RMAX>;
             if ((e = cudaFuncSetAttribute(kf, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fsmem)) != cudaSuccess)
                 return e;
-            int *done = (int *)ws_ptr(p, ws, kRegDone);  // [B*H] counts, then one ticket per launch group
-            const int ngroups = (nbhh + group - 1) / group;
-            if ((e = cudaMemsetAsync(done, 0, (size_t)(nbhh + ngroups) * 4, s)) != cudaSuccess) return e;
+            // [B*H] done counts, then one ticket per launch group: cleared by k_pair_count_scan
+            int *done = (int *)ws_ptr(p, ws, kRegDone);
             int dev = 0, sms = 0;
             if ((e = cudaGetDevice(&dev)) != cudaSuccess ||
                 (e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
                 return e;
             for (int g0 = 0; g0 < nbhh; g0 += group) {
                 const int ng = std::min(group, nbhh - g0);
-                kf<<<sms, 320, fsmem, s>>>(lmaps, rmaps, Q, sel, (const int32_t *)ws_ptr(p, ws, kRegPairs),
-                                           (const int4 *)ws_ptr(p, ws, kRegWork),
-                                           (const int32_t *)ws_ptr(p, ws, kRegNWork), (bf16 *)ws_ptr(p, ws, kRegPartO),
-                                           (float2 *)ws_ptr(p, ws, kRegPartML), done, done + nbhh + g0 / group, O,
-                                           cnt_err, c.S, c.H, c.R, c.L,
-                                           p.max_work, scale_log2, g0, ng);
+                if ((e = launch_pdl(kf, dim3(sms), dim3(320), fsmem, s, lmaps, rmaps, Q, sel,
+                                    (const int32_t *)ws_ptr(p, ws, kRegPairs), (const int4 *)ws_ptr(p, ws, kRegWork),
+                                    (const int32_t *)ws_ptr(p, ws, kRegNWork), (bf16 *)ws_ptr(p, ws, kRegPartO),
+                                    (float2 *)ws_ptr(p, ws, kRegPartML), done, done + nbhh + g0 / group, O, cnt_err,
+                                    c.S, c.H, c.R, c.L, p.max_work, scale_log2, g0, ng)) != cudaSuccess)
+                    return e;
                 count_launches(1);
-                if ((e = cudaGetLastError()) != cudaSuccess) return e;
             }
             return cudaSuccess;
         }

@@ -503,6 +503,7 @@ __global__ void __launch_bounds__(128) k_probe_rerank(const T *__restrict__ Q, c
                                                       int32_t *__restrict__ walk_log, int S, int H, int Bs,
                                                       int L, int R, int E, int M, int C, int Tp, int cap) {
     pdl_wait_primary();  // the posting lists are complete
+    pdl_launch_dependents();
     extern __shared__ float smem[];
     const int nb = S / Bs;
     float *s_cb = smem;                                     // [M*C*dm] = C*D floats
@@ -1128,6 +1129,7 @@ __global__ void __launch_bounds__(128, C <= 16 ? 4 : 3) k_probe_m2(const T *__re
     constexpr int DM = D / 2, A = C * C, QP = probe_q_pitch<T, D>(), NQ = probe_nq<C>(), QT = 128 * NQ;
     static_assert(C <= 32 && TP <= C * C && R >= 1 && E >= 1 && QP % 16 == 0 && DM % 8 == 0, "shape");
     extern __shared__ __align__(16) float smem[];
+    pdl_launch_dependents();  // the attention's first kernel may start; it waits for sel itself
     const int nb = S / Bs;
     float *s_cbT = smem;                                 // [2][DM][C]: element i of codeword (m, c) at (m DM + i) C + c
     int2 *s_rng = (int2 *)(s_cbT + C * D);               // [A] positions [first, end) of each address's entries
