@@ -66,6 +66,7 @@ void layout(Plan *p) {
     const size_t nhi = (S + kRopeLo - 1) / kRopeLo;
     bytes[kRegRope] = (nhi + kRopeLo) * (d / 2) * 8;
     if (p->fast && R > 0) {
+        bytes[kRegPairCount] = B * H * nb * 4;
         bytes[kRegPairStart] = B * H * nb * 4;
         bytes[kRegPairFill] = B * H * nb * 4;
         bytes[kRegPairs] = B * H * S * R * 4;

@@ -26,6 +26,17 @@
 #include "internal.cuh"
 #include "tc.cuh"
 
+// Which attention kernels mono_attend runs on the tensor cores (compile-time
+// choices between equivalent paths; the results are the same bit for bit):
+// the remote partials by the two-stage kernel instead of the warp-specialised
+// one, and the remote and local parts fused into one kernel.
+#ifndef MONO_REMOTE_TWO_STAGE
+#define MONO_REMOTE_TWO_STAGE 0
+#endif
+#ifndef MONO_ATTEND_FUSED
+#define MONO_ATTEND_FUSED 0
+#endif
+
 namespace mono {
 
 using bf16 = __nv_bfloat16;
@@ -50,34 +61,17 @@ constexpr int kQTile = 1024;  // queries per CTA of the count and fill kernels
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
-// One (b, h) slice per CTA: the number of queries selecting each block (a
-// shared-memory histogram of sel), its exclusive scan, the fill cursors reset,
-// and one work item {block, first pair, pair count, 0} per chunk of <= kChunk
-// queries.  Also clears the slice's done counter (and its launch group's
-// ticket) of the fused kernel.  Nothing has to be zeroed before it runs.
-// grid B*H, 1024 threads, smem nb ints.
-__global__ void __launch_bounds__(1024) k_pair_count_scan(const int32_t *__restrict__ sel, int32_t *__restrict__ start,
-                                                          int32_t *__restrict__ fill, int4 *__restrict__ work,
-                                                          int32_t *__restrict__ nwork, int *__restrict__ done,
-                                                          int *__restrict__ tickets, int S, int R, int nb, int Bs,
-                                                          int L, int wcap, int group,
-                                                          unsigned long long *__restrict__ counters) {
+// grid (ceil(S/kQTile), B*H), 256 threads, smem nb ints
+__global__ void __launch_bounds__(256) k_pair_count(const int32_t *__restrict__ sel, int32_t *__restrict__ cnt,
+                                                    int S, int R, int nb, int Bs, int L,
+                                                    unsigned long long *__restrict__ counters) {
     extern __shared__ int s_h[];
-    __shared__ int s_w[32], s_c[32];
-    __shared__ int carry_p, carry_c;
-    pdl_trigger();
-    const long long bh = blockIdx.x;
+    const long long bh = blockIdx.y;
     for (int j = threadIdx.x; j < nb; j += blockDim.x) s_h[j] = 0;
-    if (threadIdx.x == 0) {
-        carry_p = 0;
-        carry_c = 0;
-        done[bh] = 0;
-        if (bh % group == 0) tickets[bh / group] = 0;
-    }
-    pdl_wait();  // sel is complete
     __syncthreads();
+    const int t0 = blockIdx.x * kQTile, t1 = min(S, t0 + kQTile);
     bool bad = false;
-    for (int t = threadIdx.x; t < S; t += blockDim.x)
+    for (int t = t0 + threadIdx.x; t < t1; t += blockDim.x)
         for (int r = 0; r < R; ++r) {
             const int j = sel[((size_t)bh * S + t) * R + r];
             if (sel_valid(j, t, Bs, L)) atomicAdd(&s_h[j], 1);
@@ -85,11 +79,35 @@ __global__ void __launch_bounds__(1024) k_pair_count_scan(const int32_t *__restr
         }
     if (bad) record_error(counters, kDevErrBadSel);
     __syncthreads();
+    for (int j = threadIdx.x; j < nb; j += blockDim.x)
+        if (s_h[j]) atomicAdd(&cnt[bh * nb + j], s_h[j]);
+}
+
+// exclusive scan of one (b, h)'s bucket sizes, fill cursors reset, and one
+// work item {block, first pair, pair count, 0} per chunk of <= kChunk
+// queries; also clears the slice's done counter (and its launch group's
+// ticket) of the fused kernel.  grid B*H, 1024 threads.
+__global__ void __launch_bounds__(1024) k_pair_scan(const int32_t *__restrict__ cnt, int32_t *__restrict__ start,
+                                                    int32_t *__restrict__ fill, int4 *__restrict__ work,
+                                                    int32_t *__restrict__ nwork, int *__restrict__ done,
+                                                    int *__restrict__ tickets, int nb, int wcap, int group) {
+    __shared__ int s_w[32], s_c[32];
+    __shared__ int carry_p, carry_c;
+    pdl_trigger();
+    const long long bh = blockIdx.x;
+    if (threadIdx.x == 0) {
+        carry_p = 0;
+        carry_c = 0;
+        done[bh] = 0;
+        if (bh % group == 0) tickets[bh / group] = 0;
+    }
+    pdl_wait();  // the counts are complete
+    __syncthreads();
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int nw = blockDim.x >> 5;
     for (int base = 0; base < nb; base += blockDim.x) {
         const int j = base + threadIdx.x;
-        const int c = j < nb ? s_h[j] : 0;
+        const int c = j < nb ? cnt[bh * nb + j] : 0;
         const int ch = (c + kChunk - 1) / kChunk;
         int xp = c, xc = ch;  // inclusive warp scans
 #pragma unroll
@@ -434,25 +452,28 @@ __global__ void __launch_bounds__(256) k_remote_tc(const __grid_constant__ AttnM
 }
 
 // ---------------------------------------------------------------------------
-// remote partials, warp-specialised: one persistent CTA of 320 threads per SM
-// walks the work items {block j, first pair, pair count} of a group of (b, h)
-// slices through an NST-deep ring of stages.
+// remote partials, warp-specialised: one persistent CTA per SM walks the
+// work items {block j, first pair, pair count} of a group of (b, h) slices
+// through an NST-deep ring of stages.
 //   warp 0             producer: per item, the selecting queries' rows by
 //                      cp.async (every lane, 16-byte pieces, arriving on the
 //                      stage's "full" barrier as they land) and their pair
-//                      ids into the stage; K_j and V_j by TMA (lane 0);
-//   warp 1 (one lane)  MMA issuer: S = Q K_j^T of item i+1 is issued before
-//                      O = P V_j of item i, so that the tensor core works on
-//                      one item while the softmax runs on the other;
-//   warps 2-5, 6-9     two softmax groups that take alternate items, one
+//                      ids into the stage; K_j and V_j by TMA (lane 0).  The
+//                      work item and pair ids of the next items are read
+//                      one and two steps ahead;
+//   warp 1 (one lane)  MMA issuer: S = Q K_j^T of items i+1 .. i+NG-1 is
+//                      issued before O = P V_j of item i, so that every
+//                      softmax group has an item while the tensor core works;
+//   NG groups of 4     softmax groups that take items in turn (4 where the
+//   warps              tensor memory holds that many items, else 2), one
 //                      thread per query row: the softmax of S in fp32, P
 //                      (bf16) written back over S in tensor memory and read
 //                      from there by the P V MMA, then the normalised partial
 //                      (bf16) and its (max, sum) for the merge.
 // A stage is released ("empty") by the MMA issuer once both MMAs of its item
 // have completed and by the four warps of the group once they have read the
-// item's pair ids.  Tensor memory: 512 columns, 256 per group (S and P from
-// column 0, O from column 256 - D).  Every wait is bounded; a role that gives
+// item's pair ids.  Tensor memory: 512 columns, 512/NG per group (S and P
+// first, O in the last D columns).  Every wait is bounded; a role that gives
 // up sets a shared abort flag that ends the others' waits, and the producer
 // and the MMA issuer wait for their own copies and MMAs in flight before the
 // CTA exits.
@@ -462,31 +483,34 @@ struct RemoteWs {
     static constexpr int QB = 128 * D * 2, KB = BS * D * 2, IDS = 128 * 4 + 16;
     static constexpr int STAGE = QB + 2 * KB + 1024;  // Q, K, V, then pair ids and item (kept 1024-aligned)
     static constexpr int NST = (200 * 1024) / STAGE > 6 ? 6 : (200 * 1024) / STAGE;
-    static constexpr int O_COL = 256 - D;
+    // softmax groups: as many as the 512 tensor-memory columns hold (S/P and O of one item each)
+    static constexpr int NG = (BS + D <= 128) ? 4 : 2;
+    static constexpr int TG = 512 / NG;              // columns per group
+    static constexpr int O_COL = TG - D;
+    static constexpr int THREADS = 64 + NG * 128;
     static constexpr int PREF_OFF = NST * STAGE;                                     // int [kMaxGroup + 1]
     static constexpr int BAR_OFF = PREF_OFF + ((kMaxGroup + 1) * 4 + 15) / 16 * 16;
-    // mbarriers: full[NST], empty[NST], s_full[2], p_full[2], o_full[2], t_free[2], drain; then TMEM base, abort
-    static constexpr int NBAR = 2 * NST + 9;
+    // mbarriers: full[NST], empty[NST], s_full[NG], p_full[NG], o_full[NG], t_free[NG], drain; TMEM base, abort
+    static constexpr int NBAR = 2 * NST + 4 * NG + 1;
     static constexpr int BYTES = BAR_OFF + NBAR * 8 + 16;
-    static constexpr bool supported = NST >= 2 && BS + D <= 256 && D % 64 == 0 && BS % 32 == 0 && IDS <= 1024;
+    static constexpr bool supported = NST >= NG + 1 && BS + D <= TG && D % 64 == 0 && BS % 32 == 0 && IDS <= 1024;
 };
 
 template <int D, int BS>
-__global__ void __launch_bounds__(320, 1) k_remote_ws(const __grid_constant__ AttnMaps maps, const bf16 *__restrict__ Q,
-                                                      const int32_t *__restrict__ pairs, const int4 *__restrict__ work,
-                                                      const int32_t *__restrict__ nwork, bf16 *__restrict__ part_o,
-                                                      float2 *__restrict__ part_ml,
-                                                      unsigned long long *__restrict__ counters, int S, int R,
-                                                      int wcap, float scale_log2, int bh0, int ng) {
+__global__ void __launch_bounds__(RemoteWs<D, BS>::THREADS, 1)
+    k_remote_ws(const __grid_constant__ AttnMaps maps, const bf16 *__restrict__ Q, const int32_t *__restrict__ pairs,
+                const int4 *__restrict__ work, const int32_t *__restrict__ nwork, bf16 *__restrict__ part_o,
+                float2 *__restrict__ part_ml, unsigned long long *__restrict__ counters, int S, int R, int wcap,
+                float scale_log2, int bh0, int ng) {
     using Lay = RemoteWs<D, BS>;
     static_assert(Lay::supported, "tile shape");
-    constexpr int QB = Lay::QB, KB = Lay::KB, STAGE = Lay::STAGE, NST = Lay::NST;
+    constexpr int QB = Lay::QB, KB = Lay::KB, STAGE = Lay::STAGE, NST = Lay::NST, NG = Lay::NG, TG = Lay::TG;
     constexpr int CH = D * 2 / 16;  // 16-byte pieces of a query row
     extern __shared__ __align__(1024) uint8_t smem[];
     int *s_pref = (int *)(smem + Lay::PREF_OFF);
     uint64_t *bars = (uint64_t *)(smem + Lay::BAR_OFF);
-    uint64_t *full = bars, *empty = bars + NST, *s_full = bars + 2 * NST, *p_full = s_full + 2, *o_full = s_full + 4,
-             *t_free = s_full + 6, *drain = s_full + 8;
+    uint64_t *full = bars, *empty = bars + NST, *s_full = bars + 2 * NST, *p_full = s_full + NG,
+             *o_full = s_full + 2 * NG, *t_free = s_full + 3 * NG, *drain = s_full + 4 * NG;
     uint32_t *tmem_base = (uint32_t *)(bars + Lay::NBAR);
     volatile int *abort_flag = (volatile int *)(tmem_base + 1);
     if (timed_out(counters)) return;
@@ -507,7 +531,7 @@ __global__ void __launch_bounds__(320, 1) k_remote_ws(const __grid_constant__ At
             tc::mbar_init(&full[s], 32 + 1);  // every producer lane's copies + the K/V transaction
             tc::mbar_init(&empty[s], 1 + 4);  // the MMA issuer + the group's four warps
         }
-        for (int g = 0; g < 2; ++g) {
+        for (int g = 0; g < NG; ++g) {
             tc::mbar_init(&s_full[g], 1);
             tc::mbar_init(&p_full[g], 4);
             tc::mbar_init(&o_full[g], 1);
@@ -536,40 +560,58 @@ __global__ void __launch_bounds__(320, 1) k_remote_ws(const __grid_constant__ At
 
     if (warp == 0) {
         // ---------------- producer (the whole warp) ----------------
+        // Software-pipelined: while item i's copies are issued, the pair ids of item i+1 (whose work item was
+        // read one step earlier) and the work item of i+2 are in flight, so no step waits on a chain of loads.
+        auto slice_of = [&](int f, int &g) {
+            int lo = 0, hi = ng;  // last slice with s_pref[lo] <= f
+            while (hi - lo > 1) {
+                const int mid = (lo + hi) >> 1;
+                if (s_pref[mid] <= f) lo = mid;
+                else hi = mid;
+            }
+            g = lo;
+        };
+        auto load_item = [&](int i, int &g, int4 &w) {
+            const int f = blockIdx.x + i * G;
+            slice_of(f, g);
+            w = work[(size_t)(bh0 + g) * wcap + (f - s_pref[g])];
+        };
+        auto load_ids = [&](int g, const int4 &w, int (&pr)[4]) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int row = lane + 32 * k;
+                pr[k] = row < w.z ? pairs[(size_t)(bh0 + g) * S * R + w.y + row] : -1;
+            }
+        };
         int last_v[NST];
 #pragma unroll
         for (int s = 0; s < NST; ++s) last_v[s] = -1;
+        int g0 = 0, g1 = 0;
+        int4 w0 = make_int4(0, 0, 0, 0), w1 = w0;
+        int pr0[4] = {-1, -1, -1, -1};
+        if (n > 0) { load_item(0, g0, w0); load_ids(g0, w0, pr0); }
+        if (n > 1) load_item(1, g1, w1);
         for (int i = 0; i < n && ok; ++i) {
             const int s = i % NST, v = i / NST;
             if (v > 0 && !__all_sync(0xffffffffu, tc::mbar_wait_or_abort(&empty[s], (v - 1) & 1, abort_flag))) {
                 fail();
                 break;
             }
-            // the item: slice lo with s_pref[lo] <= f < s_pref[lo + 1]
-            const int f = blockIdx.x + i * G;
-            int lo = 0, hi = ng;
-            while (hi - lo > 1) {
-                const int mid = (lo + hi) >> 1;
-                if (s_pref[mid] <= f) lo = mid;
-                else hi = mid;
-            }
-            const long long bh = bh0 + lo;
-            const int4 w = work[bh * wcap + (f - s_pref[lo])];
-            const int j = w.x, p0 = w.y, cnt = w.z;
+            const long long bh = bh0 + g0;
+            const int j = w0.x, cnt = w0.z;
             uint8_t *sQ = stage_q(s), *sK = sQ + QB, *sV = sK + KB;
             int *ids = stage_ids(s);
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
                 const int row = lane + 32 * k;
                 const bool live = row < cnt;
-                const int pr = live ? pairs[bh * S * R + p0 + row] : -1;
-                ids[row] = pr;
-                const bf16 *qrow = Q + ((size_t)bh * S + (live ? pr / R : 0)) * D;
+                ids[row] = pr0[k];
+                const bf16 *qrow = Q + ((size_t)bh * S + (live ? pr0[k] / R : 0)) * D;
 #pragma unroll
                 for (int c = 0; c < CH; ++c) tc::cp_async16(sQ + tc::kmajor_chunk(row, c, D), qrow + 8 * c, live);
             }
             if (lane == 0) {
-                ids[128] = (int)(bh - bh0);
+                ids[128] = g0;
                 ids[129] = cnt;
             }
             asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(tc::smem_u32(&full[s]))
@@ -584,6 +626,16 @@ __global__ void __launch_bounds__(320, 1) k_remote_ws(const __grid_constant__ At
                 }
             }
             last_v[s] = v;
+            // the next items' loads, consumed in the next steps
+            int pr1[4] = {-1, -1, -1, -1};
+            if (i + 1 < n) load_ids(g1, w1, pr1);
+            int g2 = 0;
+            int4 w2 = make_int4(0, 0, 0, 0);
+            if (i + 2 < n) load_item(i + 2, g2, w2);
+            g0 = g1; w0 = w1;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) pr0[k] = pr1[k];
+            g1 = g2; w1 = w2;
         }
         // every copy issued has landed before the CTA may exit
         asm volatile("cp.async.wait_all;" ::: "memory");
@@ -595,7 +647,7 @@ __global__ void __launch_bounds__(320, 1) k_remote_ws(const __grid_constant__ At
         if (lane == 0) {
             const uint32_t id1 = tc::idesc_bf16(128, BS), id2 = tc::idesc_bf16(128, D, true);
             auto mma1 = [&](int i) -> bool {
-                const int s = i % NST, v = i / NST, g = i & 1, u = i >> 1;
+                const int s = i % NST, v = i / NST, g = i % NG, u = i / NG;
                 if (!tc::mbar_wait_or_abort(&full[s], v & 1, abort_flag)) return false;
                 if (u > 0 && !tc::mbar_wait_or_abort(&t_free[g], (u - 1) & 1, abort_flag)) return false;
                 tc::fence_smem_to_async();
@@ -603,27 +655,29 @@ __global__ void __launch_bounds__(320, 1) k_remote_ws(const __grid_constant__ At
                 const uint32_t aq = tc::smem_u32(stage_q(s)), bk = aq + QB;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk)
-                    tc::mma_bf16(tmem + g * 256, tc::desc_kmajor(aq + 256 * kk, D),
+                    tc::mma_bf16(tmem + g * TG, tc::desc_kmajor(aq + 256 * kk, D),
                                  tc::desc_sw128(bk + (kk >> 2) * (BS * 128) + (kk & 3) * 32), id1, kk > 0);
                 tc::commit(&s_full[g]);
                 return true;
             };
             auto mma2 = [&](int i) -> bool {
-                const int s = i % NST, g = i & 1, u = i >> 1;
+                const int s = i % NST, g = i % NG, u = i / NG;
                 if (!tc::mbar_wait_or_abort(&p_full[g], u & 1, abort_flag)) return false;
                 tc::fence_after_sync();
                 const uint32_t bv = tc::smem_u32(stage_q(s)) + QB + KB;
 #pragma unroll
                 for (int kk = 0; kk < BS / 16; ++kk)
-                    tc::mma_bf16_ts(tmem + g * 256 + Lay::O_COL, tmem + g * 256 + 8 * kk,
+                    tc::mma_bf16_ts(tmem + g * TG + Lay::O_COL, tmem + g * TG + 8 * kk,
                                     tc::desc_sw128_mn(bv + 2048 * kk, BS * 128), id2, kk > 0);
                 tc::commit(&o_full[g]);
                 tc::commit(&empty[s]);
                 return true;
             };
-            if (n > 0 && !mma1(0)) fail();
+            // S of the next NG-1 items is issued before O of this one, so every softmax group has work
+            for (int i = 0; i < NG - 1 && i < n && ok; ++i)
+                if (!mma1(i)) fail();
             for (int i = 0; i < n && ok; ++i) {
-                if (i + 1 < n && !mma1(i + 1)) { fail(); break; }
+                if (i + NG - 1 < n && !mma1(i + NG - 1)) { fail(); break; }
                 if (!mma2(i)) { fail(); break; }
             }
             // every MMA issued has completed before the CTA may exit
@@ -634,10 +688,10 @@ __global__ void __launch_bounds__(320, 1) k_remote_ws(const __grid_constant__ At
         // ---------------- softmax groups ----------------
         const int g = (warp - 2) >> 2, quarter = warp & 3;
         const int row = quarter * 32 + lane;
-        const uint32_t tS = tmem + g * 256 + ((uint32_t)(quarter * 32) << 16);
+        const uint32_t tS = tmem + g * TG + ((uint32_t)(quarter * 32) << 16);
         const uint32_t tO = tS + Lay::O_COL;
-        for (int i = g; i < n && ok; i += 2) {
-            const int s = i % NST, v = i / NST, u = i >> 1;
+        for (int i = g; i < n && ok; i += NG) {
+            const int s = i % NST, v = i / NST, u = i / NG;
             // (the decisions to go on are warp-uniform: the TMEM accesses below are warp-collective)
             if (!__all_sync(0xffffffffu, tc::mbar_wait_or_abort(&full[s], v & 1, abort_flag))) { fail(); break; }
             const int *ids = stage_ids(s);
@@ -1939,9 +1993,10 @@ static cudaError_t launch_tc_shape(const Plan &p, const bf16 *Q, const bf16 *K, 
         !make_map_3d(&rmaps.k, K, D, c.S, c.B * c.H, BS) || !make_map_3d(&rmaps.v, V, D, c.S, c.B * c.H, BS))
         return cudaErrorInvalidValue;
     constexpr size_t rsmem = RemoteSmem<D, BS>::BYTES;
-    // the warp-specialised remote kernel where its ring fits (every tensor-core shape), else the two-stage one
-    constexpr bool kRemoteWs = RemoteWs<D, BS>::supported;
+    // the warp-specialised remote kernel where its ring fits, else the two-stage one
+    constexpr bool kRemoteWs = RemoteWs<D, BS>::supported && !MONO_REMOTE_TWO_STAGE;
     if (c.R > 0 && (parts & kAttendPairs)) {
+        int32_t *pc = (int32_t *)ws_ptr(p, ws, kRegPairCount);
         int32_t *ps = (int32_t *)ws_ptr(p, ws, kRegPairStart);
         int32_t *pf = (int32_t *)ws_ptr(p, ws, kRegPairFill);
         int32_t *pairs = (int32_t *)ws_ptr(p, ws, kRegPairs);
@@ -1951,19 +2006,22 @@ static cudaError_t launch_tc_shape(const Plan &p, const bf16 *Q, const bf16 *K, 
         const int nbhh = c.B * c.H;
         const int wcap = p.max_work;  // work items per (b, h)
         const int grp = std::min(kMaxGroup, nbhh);
+        if ((e = cudaMemsetAsync(pc, 0, (size_t)nbh * 4, s)) != cudaSuccess) return e;
+        dim3 gq((c.S + kQTile - 1) / kQTile, nbhh);
         const size_t hs = (size_t)p.nb * 4;
         if (2 * hs > 48 * 1024) {
-            if ((e = cudaFuncSetAttribute(k_pair_count_scan, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)hs)) ||
+            if ((e = cudaFuncSetAttribute(k_pair_count, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)hs)) ||
                 (e = cudaFuncSetAttribute(k_pair_fill, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)(2 * hs))))
                 return e;
         }
-        if ((e = launch_pdl(k_pair_count_scan, dim3(nbhh), dim3(1024), hs, s, sel, ps, pf, work, nwork, done,
-                            done + nbhh, c.S, c.R, p.nb, c.Bs, c.L, wcap, grp, cnt_err)) != cudaSuccess)
+        k_pair_count<<<gq, 256, hs, s>>>(sel, pc, c.S, c.R, p.nb, c.Bs, c.L, cnt_err);
+        if ((e = launch_pdl(k_pair_scan, dim3(nbhh), dim3(1024), 0, s, (const int32_t *)pc, ps, pf, work, nwork, done,
+                            done + nbhh, p.nb, wcap, grp)) != cudaSuccess)
             return e;
-        dim3 gq((c.S + kQTile - 1) / kQTile, nbhh);
         if ((e = launch_pdl(k_pair_fill, gq, dim3(256), 2 * hs, s, sel, (const int32_t *)ps, pf, pairs, c.S, c.R, p.nb,
                             c.Bs, c.L)) != cudaSuccess)
             return e;
+        count_launches(1);
         count_launches(2);
     }
     if (c.R > 0 && (parts & kAttendRemote)) {
@@ -2013,15 +2071,15 @@ static cudaError_t launch_tc_shape(const Plan &p, const bf16 *Q, const bf16 *K, 
     }
     const int nbhh = c.B * c.H;
     const int group = c.R > 0 ? std::min(kMaxGroup, nbhh) : nbhh;
-    // all stages at once: the fused kernel per group of slices where it applies
-    constexpr bool kFused = AttendWs<D, BS, NK>::supported;
+    // all stages at once: the fused kernel per group of slices where it applies and is selected
+    constexpr bool kFused = AttendWs<D, BS, NK>::supported && MONO_ATTEND_FUSED;
     if constexpr (kFused) {
         if (c.R > 0 && (parts & kAttendRemote) && (parts & kAttendLocal)) {
             constexpr size_t fsmem = AttendWs<D, BS, NK>::BYTES;
             auto kf = k_attend_ws<D, BS, NK, RMAX>;
             if ((e = cudaFuncSetAttribute(kf, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fsmem)) != cudaSuccess)
                 return e;
-            // [B*H] done counts, then one ticket per launch group: cleared by k_pair_count_scan
+            // [B*H] done counts, then one ticket per launch group: cleared by k_pair_scan
             int *done = (int *)ws_ptr(p, ws, kRegDone);
             int dev = 0, sms = 0;
             if ((e = cudaGetDevice(&dev)) != cudaSuccess ||
@@ -2049,7 +2107,7 @@ static cudaError_t launch_tc_shape(const Plan &p, const bf16 *Q, const bf16 *K, 
         const bool do_local = (parts & kAttendLocal) && (both || pass == 1);
         if (c.R > 0 && do_remote) {
             if constexpr (kRemoteWs)
-                k_remote_ws<D, BS><<<remote_ctas, 320, RemoteWs<D, BS>::BYTES, s>>>(
+                k_remote_ws<D, BS><<<remote_ctas, RemoteWs<D, BS>::THREADS, RemoteWs<D, BS>::BYTES, s>>>(
                     rmaps, Q, (const int32_t *)ws_ptr(p, ws, kRegPairs), (const int4 *)ws_ptr(p, ws, kRegWork),
                     (const int32_t *)ws_ptr(p, ws, kRegNWork), (bf16 *)ws_ptr(p, ws, kRegPartO),
                     (float2 *)ws_ptr(p, ws, kRegPartML), cnt_err, c.S, c.R, p.max_work, scale_log2, g0, ng);

@@ -53,6 +53,7 @@ enum Region {
     kRegWalkLog = MONO_WS_WALK_LOG,
     kRegCounters = MONO_WS_NREGIONS,
     kRegRope,
+    kRegPairCount,   // [B,H,nb] int32 queries selecting each block (fast attention)
     kRegPairStart,   // [B,H,nb+1] int32 exclusive scan of the counts
     kRegPairFill,    // [B,H,nb] int32 fill cursors
     kRegPairs,       // [B*H*S*R] int32 (t*R + r) grouped by block
