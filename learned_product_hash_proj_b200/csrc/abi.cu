@@ -74,7 +74,6 @@ void layout(Plan *p) {
         bytes[kRegPartML] = B * H * S * R * 8;
         bytes[kRegWork] = B * H * (size_t)p->max_work * 16;
         bytes[kRegNWork] = B * H * 4;
-        bytes[kRegDone] = (B * H + (B * H + 255) / 256) * 4;  // counts + one ticket per launch group of 256
     }
     size_t off = 0;
     for (int r = 0; r < kRegN; ++r) {

@@ -26,17 +26,6 @@
 #include "internal.cuh"
 #include "tc.cuh"
 
-// Which attention kernels mono_attend runs on the tensor cores (compile-time
-// choices between equivalent paths; the results are the same bit for bit):
-// the remote partials by the two-stage kernel instead of the warp-specialised
-// one, and the remote and local parts fused into one kernel.
-#ifndef MONO_REMOTE_TWO_STAGE
-#define MONO_REMOTE_TWO_STAGE 0
-#endif
-#ifndef MONO_ATTEND_FUSED
-#define MONO_ATTEND_FUSED 0
-#endif
-
 namespace mono {
 
 using bf16 = __nv_bfloat16;
@@ -85,12 +74,10 @@ __global__ void __launch_bounds__(256) k_pair_count(const int32_t *__restrict__ 
 
 // exclusive scan of one (b, h)'s bucket sizes, fill cursors reset, and one
 // work item {block, first pair, pair count, 0} per chunk of <= kChunk
-// queries; also clears the slice's done counter (and its launch group's
-// ticket) of the fused kernel.  grid B*H, 1024 threads.
+// queries.  grid B*H, 1024 threads.
 __global__ void __launch_bounds__(1024) k_pair_scan(const int32_t *__restrict__ cnt, int32_t *__restrict__ start,
                                                     int32_t *__restrict__ fill, int4 *__restrict__ work,
-                                                    int32_t *__restrict__ nwork, int *__restrict__ done,
-                                                    int *__restrict__ tickets, int nb, int wcap, int group) {
+                                                    int32_t *__restrict__ nwork, int nb, int wcap) {
     __shared__ int s_w[32], s_c[32];
     __shared__ int carry_p, carry_c;
     pdl_trigger();
@@ -98,8 +85,6 @@ __global__ void __launch_bounds__(1024) k_pair_scan(const int32_t *__restrict__ 
     if (threadIdx.x == 0) {
         carry_p = 0;
         carry_c = 0;
-        done[bh] = 0;
-        if (bh % group == 0) tickets[bh / group] = 0;
     }
     pdl_wait();  // the counts are complete
     __syncthreads();
@@ -449,324 +434,6 @@ __global__ void __launch_bounds__(256) k_remote_tc(const __grid_constant__ AttnM
     tc::fence_before_sync();
     __syncthreads();
     if (warp == 0) tc::tmem_dealloc(tmem, NCOLS);
-}
-
-// ---------------------------------------------------------------------------
-// remote partials, warp-specialised: one persistent CTA per SM walks the
-// work items {block j, first pair, pair count} of a group of (b, h) slices
-// through an NST-deep ring of stages.
-//   warp 0             producer: per item, the selecting queries' rows by
-//                      cp.async (every lane, 16-byte pieces, arriving on the
-//                      stage's "full" barrier as they land) and their pair
-//                      ids into the stage; K_j and V_j by TMA (lane 0).  The
-//                      work item and pair ids of the next items are read
-//                      one and two steps ahead;
-//   warp 1 (one lane)  MMA issuer: S = Q K_j^T of items i+1 .. i+NG-1 is
-//                      issued before O = P V_j of item i, so that every
-//                      softmax group has an item while the tensor core works;
-//   NG groups of 4     softmax groups that take items in turn (4 where the
-//   warps              tensor memory holds that many items, else 2), one
-//                      thread per query row: the softmax of S in fp32, P
-//                      (bf16) written back over S in tensor memory and read
-//                      from there by the P V MMA, then the normalised partial
-//                      (bf16) and its (max, sum) for the merge.
-// A stage is released ("empty") by the MMA issuer once both MMAs of its item
-// have completed and by the four warps of the group once they have read the
-// item's pair ids.  Tensor memory: 512 columns, 512/NG per group (S and P
-// first, O in the last D columns).  Every wait is bounded; a role that gives
-// up sets a shared abort flag that ends the others' waits, and the producer
-// and the MMA issuer wait for their own copies and MMAs in flight before the
-// CTA exits.
-// ---------------------------------------------------------------------------
-template <int D, int BS>
-struct RemoteWs {
-    static constexpr int QB = 128 * D * 2, KB = BS * D * 2, IDS = 128 * 4 + 16;
-    static constexpr int STAGE = QB + 2 * KB + 1024;  // Q, K, V, then pair ids and item (kept 1024-aligned)
-    static constexpr int NST = (200 * 1024) / STAGE > 6 ? 6 : (200 * 1024) / STAGE;
-    // softmax groups: as many as the 512 tensor-memory columns hold (S/P and O of one item each)
-    static constexpr int NG = (BS + D <= 128) ? 4 : 2;
-    static constexpr int TG = 512 / NG;              // columns per group
-    static constexpr int O_COL = TG - D;
-    static constexpr int THREADS = 64 + NG * 128;
-    static constexpr int PREF_OFF = NST * STAGE;                                     // int [kMaxGroup + 1]
-    static constexpr int BAR_OFF = PREF_OFF + ((kMaxGroup + 1) * 4 + 15) / 16 * 16;
-    // mbarriers: full[NST], empty[NST], s_full[NG], p_full[NG], o_full[NG], t_free[NG], drain; TMEM base, abort
-    static constexpr int NBAR = 2 * NST + 4 * NG + 1;
-    static constexpr int BYTES = BAR_OFF + NBAR * 8 + 16;
-    static constexpr bool supported = NST >= NG + 1 && BS + D <= TG && D % 64 == 0 && BS % 32 == 0 && IDS <= 1024;
-};
-
-template <int D, int BS>
-__global__ void __launch_bounds__(RemoteWs<D, BS>::THREADS, 1)
-    k_remote_ws(const __grid_constant__ AttnMaps maps, const bf16 *__restrict__ Q, const int32_t *__restrict__ pairs,
-                const int4 *__restrict__ work, const int32_t *__restrict__ nwork, bf16 *__restrict__ part_o,
-                float2 *__restrict__ part_ml, unsigned long long *__restrict__ counters, int S, int R, int wcap,
-                float scale_log2, int bh0, int ng) {
-    using Lay = RemoteWs<D, BS>;
-    static_assert(Lay::supported, "tile shape");
-    constexpr int QB = Lay::QB, KB = Lay::KB, STAGE = Lay::STAGE, NST = Lay::NST, NG = Lay::NG, TG = Lay::TG;
-    constexpr int CH = D * 2 / 16;  // 16-byte pieces of a query row
-    extern __shared__ __align__(1024) uint8_t smem[];
-    int *s_pref = (int *)(smem + Lay::PREF_OFF);
-    uint64_t *bars = (uint64_t *)(smem + Lay::BAR_OFF);
-    uint64_t *full = bars, *empty = bars + NST, *s_full = bars + 2 * NST, *p_full = s_full + NG,
-             *o_full = s_full + 2 * NG, *t_free = s_full + 3 * NG, *drain = s_full + 4 * NG;
-    uint32_t *tmem_base = (uint32_t *)(bars + Lay::NBAR);
-    volatile int *abort_flag = (volatile int *)(tmem_base + 1);
-    if (timed_out(counters)) return;
-    if (tc::smem_u32(smem) & 1023) {
-        if (threadIdx.x == 0) record_error(counters, kDevErrSmemAlign);
-        return;
-    }
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    // a stage: Q rows (K-major, no swizzle), K_j and V_j (TMA, 128-byte swizzle), pair ids [128], item (bh, n)
-    auto stage_q = [&](int s) { return smem + s * STAGE; };
-    auto stage_ids = [&](int s) { return (int *)(smem + s * STAGE + QB + 2 * KB); };
-
-    if (tid == 0) {
-        int acc = 0;
-        for (int g = 0; g < ng; ++g) { s_pref[g] = acc; acc += nwork[bh0 + g]; }
-        s_pref[ng] = acc;
-        for (int s = 0; s < NST; ++s) {
-            tc::mbar_init(&full[s], 32 + 1);  // every producer lane's copies + the K/V transaction
-            tc::mbar_init(&empty[s], 1 + 4);  // the MMA issuer + the group's four warps
-        }
-        for (int g = 0; g < NG; ++g) {
-            tc::mbar_init(&s_full[g], 1);
-            tc::mbar_init(&p_full[g], 4);
-            tc::mbar_init(&o_full[g], 1);
-            tc::mbar_init(&t_free[g], 4);
-        }
-        tc::mbar_init(drain, 1);
-        *abort_flag = 0;
-        tc::fence_mbar_init();
-    }
-    if (warp == 1) {
-        tc::tmem_alloc(tmem_base, 512);
-        tc::tmem_relinquish();
-    }
-    tc::fence_before_sync();
-    __syncthreads();
-    tc::fence_after_sync();
-    const uint32_t tmem = *tmem_base;
-    const int total = s_pref[ng];
-    const int G = gridDim.x;
-    const int n = blockIdx.x < total ? (total - 1 - blockIdx.x) / G + 1 : 0;  // items of this CTA
-    bool ok = true;
-    auto fail = [&]() {
-        ok = false;
-        *abort_flag = 1;
-    };
-
-    if (warp == 0) {
-        // ---------------- producer (the whole warp) ----------------
-        // Software-pipelined: while item i's copies are issued, the pair ids of item i+1 (whose work item was
-        // read one step earlier) and the work item of i+2 are in flight, so no step waits on a chain of loads.
-        auto slice_of = [&](int f, int &g) {
-            int lo = 0, hi = ng;  // last slice with s_pref[lo] <= f
-            while (hi - lo > 1) {
-                const int mid = (lo + hi) >> 1;
-                if (s_pref[mid] <= f) lo = mid;
-                else hi = mid;
-            }
-            g = lo;
-        };
-        auto load_item = [&](int i, int &g, int4 &w) {
-            const int f = blockIdx.x + i * G;
-            slice_of(f, g);
-            w = work[(size_t)(bh0 + g) * wcap + (f - s_pref[g])];
-        };
-        auto load_ids = [&](int g, const int4 &w, int (&pr)[4]) {
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const int row = lane + 32 * k;
-                pr[k] = row < w.z ? pairs[(size_t)(bh0 + g) * S * R + w.y + row] : -1;
-            }
-        };
-        int last_v[NST];
-#pragma unroll
-        for (int s = 0; s < NST; ++s) last_v[s] = -1;
-        int g0 = 0, g1 = 0;
-        int4 w0 = make_int4(0, 0, 0, 0), w1 = w0;
-        int pr0[4] = {-1, -1, -1, -1};
-        if (n > 0) { load_item(0, g0, w0); load_ids(g0, w0, pr0); }
-        if (n > 1) load_item(1, g1, w1);
-        for (int i = 0; i < n && ok; ++i) {
-            const int s = i % NST, v = i / NST;
-            if (v > 0 && !__all_sync(0xffffffffu, tc::mbar_wait_or_abort(&empty[s], (v - 1) & 1, abort_flag))) {
-                fail();
-                break;
-            }
-            const long long bh = bh0 + g0;
-            const int j = w0.x, cnt = w0.z;
-            uint8_t *sQ = stage_q(s), *sK = sQ + QB, *sV = sK + KB;
-            int *ids = stage_ids(s);
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const int row = lane + 32 * k;
-                const bool live = row < cnt;
-                ids[row] = pr0[k];
-                const bf16 *qrow = Q + ((size_t)bh * S + (live ? pr0[k] / R : 0)) * D;
-#pragma unroll
-                for (int c = 0; c < CH; ++c) tc::cp_async16(sQ + tc::kmajor_chunk(row, c, D), qrow + 8 * c, live);
-            }
-            if (lane == 0) {
-                ids[128] = g0;
-                ids[129] = cnt;
-            }
-            asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(tc::smem_u32(&full[s]))
-                         : "memory");
-            __syncwarp();
-            if (lane == 0) {
-                tc::mbar_expect_tx(&full[s], 2 * KB);
-#pragma unroll
-                for (int a = 0; a < D / 64; ++a) {
-                    tc::tma_load_3d(sK + a * (BS * 128), &maps.k, 64 * a, j * BS, (int)bh, &full[s]);
-                    tc::tma_load_3d(sV + a * (BS * 128), &maps.v, 64 * a, j * BS, (int)bh, &full[s]);
-                }
-            }
-            last_v[s] = v;
-            // the next items' loads, consumed in the next steps
-            int pr1[4] = {-1, -1, -1, -1};
-            if (i + 1 < n) load_ids(g1, w1, pr1);
-            int g2 = 0;
-            int4 w2 = make_int4(0, 0, 0, 0);
-            if (i + 2 < n) load_item(i + 2, g2, w2);
-            g0 = g1; w0 = w1;
-#pragma unroll
-            for (int k = 0; k < 4; ++k) pr0[k] = pr1[k];
-            g1 = g2; w1 = w2;
-        }
-        // every copy issued has landed before the CTA may exit
-        asm volatile("cp.async.wait_all;" ::: "memory");
-        if (lane == 0)
-            for (int s = 0; s < NST; ++s)
-                if (last_v[s] >= 0 && !tc::mbar_wait(&full[s], last_v[s] & 1)) ok = false;
-    } else if (warp == 1) {
-        // ---------------- MMA issuer ----------------
-        if (lane == 0) {
-            const uint32_t id1 = tc::idesc_bf16(128, BS), id2 = tc::idesc_bf16(128, D, true);
-            auto mma1 = [&](int i) -> bool {
-                const int s = i % NST, v = i / NST, g = i % NG, u = i / NG;
-                if (!tc::mbar_wait_or_abort(&full[s], v & 1, abort_flag)) return false;
-                if (u > 0 && !tc::mbar_wait_or_abort(&t_free[g], (u - 1) & 1, abort_flag)) return false;
-                tc::fence_smem_to_async();
-                tc::fence_after_sync();
-                const uint32_t aq = tc::smem_u32(stage_q(s)), bk = aq + QB;
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk)
-                    tc::mma_bf16(tmem + g * TG, tc::desc_kmajor(aq + 256 * kk, D),
-                                 tc::desc_sw128(bk + (kk >> 2) * (BS * 128) + (kk & 3) * 32), id1, kk > 0);
-                tc::commit(&s_full[g]);
-                return true;
-            };
-            auto mma2 = [&](int i) -> bool {
-                const int s = i % NST, g = i % NG, u = i / NG;
-                if (!tc::mbar_wait_or_abort(&p_full[g], u & 1, abort_flag)) return false;
-                tc::fence_after_sync();
-                const uint32_t bv = tc::smem_u32(stage_q(s)) + QB + KB;
-#pragma unroll
-                for (int kk = 0; kk < BS / 16; ++kk)
-                    tc::mma_bf16_ts(tmem + g * TG + Lay::O_COL, tmem + g * TG + 8 * kk,
-                                    tc::desc_sw128_mn(bv + 2048 * kk, BS * 128), id2, kk > 0);
-                tc::commit(&o_full[g]);
-                tc::commit(&empty[s]);
-                return true;
-            };
-            // S of the next NG-1 items is issued before O of this one, so every softmax group has work
-            for (int i = 0; i < NG - 1 && i < n && ok; ++i)
-                if (!mma1(i)) fail();
-            for (int i = 0; i < n && ok; ++i) {
-                if (i + NG - 1 < n && !mma1(i + NG - 1)) { fail(); break; }
-                if (!mma2(i)) { fail(); break; }
-            }
-            // every MMA issued has completed before the CTA may exit
-            tc::commit(drain);
-            if (!tc::mbar_wait(drain, 0)) ok = false;
-        }
-    } else {
-        // ---------------- softmax groups ----------------
-        const int g = (warp - 2) >> 2, quarter = warp & 3;
-        const int row = quarter * 32 + lane;
-        const uint32_t tS = tmem + g * TG + ((uint32_t)(quarter * 32) << 16);
-        const uint32_t tO = tS + Lay::O_COL;
-        for (int i = g; i < n && ok; i += NG) {
-            const int s = i % NST, v = i / NST, u = i / NG;
-            // (the decisions to go on are warp-uniform: the TMEM accesses below are warp-collective)
-            if (!__all_sync(0xffffffffu, tc::mbar_wait_or_abort(&full[s], v & 1, abort_flag))) { fail(); break; }
-            const int *ids = stage_ids(s);
-            const int pr = ids[row];
-            const long long bh = bh0 + ids[128];
-            __syncwarp();
-            if (lane == 0) tc::mbar_arrive(&empty[s]);  // this warp is done with the stage
-            if (!__all_sync(0xffffffffu, tc::mbar_wait_or_abort(&s_full[g], u & 1, abort_flag))) { fail(); break; }
-            tc::fence_after_sync();
-            // softmax of the row over the block's BS keys (all visible: the block lies before the query)
-            float vv[32];
-            float m = -INFINITY;
-#pragma unroll
-            for (int c0 = 0; c0 < BS; c0 += 32) {
-                __syncwarp();
-                tc::tmem_ld32(tS + c0, vv);
-#pragma unroll
-                for (int k = 0; k < 32; ++k) m = fmaxf(m, vv[k]);
-            }
-            const float m2 = m * scale_log2;
-            float l = 0.f;
-#pragma unroll
-            for (int c0 = 0; c0 < BS; c0 += 32) {
-                __syncwarp();
-                tc::tmem_ld32(tS + c0, vv);
-                uint32_t pk[16];
-#pragma unroll
-                for (int k = 0; k < 16; ++k) {
-                    const float a = exp2f(fmaf(vv[2 * k], scale_log2, -m2));
-                    const float bb = exp2f(fmaf(vv[2 * k + 1], scale_log2, -m2));
-                    l += a + bb;
-                    pk[k] = pack2(a, bb);
-                }
-                // P over the columns of S already read (column c0/2 .. c0/2 + 15 of this row)
-                __syncwarp();
-                tc::tmem_st16(tS + (c0 >> 1), pk);
-            }
-            __syncwarp();
-            tc::tmem_st_wait();
-            tc::fence_before_sync();
-            __syncwarp();
-            if (lane == 0) tc::mbar_arrive(&p_full[g]);
-            const float inv = 1.f / l;
-            if (!__all_sync(0xffffffffu, tc::mbar_wait_or_abort(&o_full[g], u & 1, abort_flag))) { fail(); break; }
-            tc::fence_after_sync();
-            const bool live = pr >= 0;
-            const size_t slot = (size_t)bh * S * R + (live ? pr : 0);
-#pragma unroll
-            for (int c0 = 0; c0 < D; c0 += 32) {
-                __syncwarp();
-                tc::tmem_ld32(tO + c0, vv);
-                if (live) {
-                    uint4 *dst = (uint4 *)(part_o + slot * D + c0);
-#pragma unroll
-                    for (int q8 = 0; q8 < 4; ++q8)
-                        dst[q8] = make_uint4(pack2(vv[8 * q8] * inv, vv[8 * q8 + 1] * inv),
-                                             pack2(vv[8 * q8 + 2] * inv, vv[8 * q8 + 3] * inv),
-                                             pack2(vv[8 * q8 + 4] * inv, vv[8 * q8 + 5] * inv),
-                                             pack2(vv[8 * q8 + 6] * inv, vv[8 * q8 + 7] * inv));
-                }
-            }
-            if (live) part_ml[slot] = make_float2(m2, l);
-            tc::fence_before_sync();
-            __syncwarp();
-            if (lane == 0) tc::mbar_arrive(&t_free[g]);
-        }
-    }
-    if (!ok) record_error(counters, kDevErrTimeout);
-    tc::fence_before_sync();
-    __syncthreads();
-    tc::fence_after_sync();
-    if (warp == 1) {
-        __syncwarp();
-        tc::tmem_dealloc(tmem, 512);
-    }
 }
 
 // ---------------------------------------------------------------------------
@@ -1408,517 +1075,6 @@ __global__ void __launch_bounds__(320, 1) k_local_ws(const __grid_constant__ Att
 }
 
 // ---------------------------------------------------------------------------
-// The whole selected-set attention of a group of (b, h) slices in one
-// persistent warp-specialised kernel (one 320-thread CTA per SM), so that a
-// slice's remote partials are read back while they are still in L2 and no
-// launch tail separates the two parts.  The work list runs in phases: phase k
-// holds the remote items {block j, first pair, pair count} of slice k, then
-// the 128-query local tiles of slice k-1.  The producer of each CTA takes the
-// next item from a ticket counter, so items are taken in order by CTAs that
-// are running.  The roles are those of k_remote_ws and k_local_ws:
-//   warp 0             producer: a remote item's query rows by cp.async (every
-//                      lane) and K_j, V_j by TMA, or a local tile's Q tile and
-//                      K/V window by TMA (lane 0), into a ring of stages;
-//   warp 1 (one lane)  MMA issuer: S = Q K^T of item i+1 before O = P V of
-//                      item i (N = Bs keys for a remote item, NK for a tile);
-//   warps 2-5, 6-9     softmax groups on alternate items: a remote item's
-//                      softmax and partial, or a tile's masked softmax and its
-//                      merge with the partials of its queries' remote blocks.
-// A remote item's four warps each add 1 to the slice's done counter after
-// their partial rows are stored (and fenced); a local tile of slice g first
-// waits (bounded) until the counter reaches 4 x the slice's remote items.
-// Every item taken before a waiting tile is held by a running CTA and is a
-// remote item of an earlier or the same phase or a tile of an earlier slice,
-// so the waits end.  When the tickets run out the producer writes an end
-// record into the next two stages, one for each softmax group.
-// ---------------------------------------------------------------------------
-template <int D, int BS, int NK>
-struct AttendWs {
-    static constexpr int QB = 128 * D * 2, KVB = NK * D * 2;
-    static constexpr int STAGE = QB + 2 * KVB + 1024;  // Q, K, V, then the item's record (pair ids, kind, slice)
-    static constexpr int NST = (200 * 1024) / STAGE > 4 ? 4 : (200 * 1024) / STAGE;
-    static constexpr int O_COL = 256 - D;
-    static constexpr int PH_OFF = NST * STAGE;                                   // int [kMaxGroup + 2] phase starts
-    static constexpr int NR_OFF = PH_OFF + (kMaxGroup + 2) * 4;                  // int [kMaxGroup] remote items
-    static constexpr int BAR_OFF = (NR_OFF + kMaxGroup * 4 + 15) / 16 * 16;
-    static constexpr int NBAR = 2 * NST + 9;
-    static constexpr int BYTES = BAR_OFF + NBAR * 8 + 16;
-    static constexpr bool supported = NST >= 2 && NK + D <= 256 && BS <= NK && D % 64 == 0 && NK % 32 == 0 &&
-                                      BS % 32 == 0 && STAGE % 1024 == 0 && BYTES <= 227 * 1024;
-};
-
-__device__ __forceinline__ int ld_acquire(const int *p) {
-    int v;
-    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-__device__ __forceinline__ uint4 ld_cg16(const void *p) {
-    uint4 v;
-    asm volatile("ld.global.cg.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
-    return v;
-}
-__device__ __forceinline__ float2 ld_cg_f2(const float2 *p) {
-    float2 v;
-    asm volatile("ld.global.cg.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "l"(p));
-    return v;
-}
-
-template <int D, int BS, int NK, int RMAX>
-__global__ void __launch_bounds__(320, 1) k_attend_ws(const __grid_constant__ AttnMaps lm, const __grid_constant__ AttnMaps rm,
-                                                      const bf16 *__restrict__ Q, const int32_t *__restrict__ sel,
-                                                      const int32_t *__restrict__ pairs, const int4 *__restrict__ work,
-                                                      const int32_t *__restrict__ nwork, bf16 *part_o, float2 *part_ml,
-                                                      int *done, int *ticket, bf16 *__restrict__ O,
-                                                      unsigned long long *__restrict__ counters, int S, int H, int R,
-                                                      int L, int wcap, float scale_log2, int bh0, int ng) {
-    using Lay = AttendWs<D, BS, NK>;
-    static_assert(Lay::supported, "tile shape");
-    constexpr int QB = Lay::QB, KVB = Lay::KVB, STAGE = Lay::STAGE, NST = Lay::NST;
-    constexpr int RKB = BS * D * 2;  // a remote block's K (or V) tile
-    constexpr int CH = D * 2 / 16;
-    extern __shared__ __align__(1024) uint8_t smem[];
-    int *s_ph = (int *)(smem + Lay::PH_OFF);
-    int *s_nr = (int *)(smem + Lay::NR_OFF);
-    uint64_t *bars = (uint64_t *)(smem + Lay::BAR_OFF);
-    uint64_t *full = bars, *empty = bars + NST, *s_full = bars + 2 * NST, *p_full = s_full + 2, *o_full = s_full + 4,
-             *t_free = s_full + 6, *drain = s_full + 8;
-    uint32_t *tmem_base = (uint32_t *)(bars + Lay::NBAR);
-    volatile int *abort_flag = (volatile int *)(tmem_base + 1);
-    if (timed_out(counters)) return;
-    if (tc::smem_u32(smem) & 1023) {
-        if (threadIdx.x == 0) record_error(counters, kDevErrSmemAlign);
-        return;
-    }
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int ntiles = (S + 127) / 128;
-    auto stage_q = [&](int s) { return smem + s * STAGE; };
-    auto stage_rec = [&](int s) { return (int *)(smem + s * STAGE + QB + 2 * KVB); };  // [128] ids, kind, slice, n|t0
-    pdl_wait();  // the work items, pair ids, done counters and ticket are ready
-
-    if (tid == 0) {
-        int acc = 0;
-        for (int k = 0; k <= ng; ++k) {
-            s_ph[k] = acc;
-            if (k < ng) { s_nr[k] = nwork[bh0 + k]; acc += s_nr[k]; }
-            if (k >= 1) acc += ntiles;
-        }
-        s_ph[ng + 1] = acc;
-        for (int s = 0; s < NST; ++s) {
-            tc::mbar_init(&full[s], 32 + 1);  // every producer lane + the transaction
-            tc::mbar_init(&empty[s], 1 + 4);  // the MMA issuer + the group's four warps
-        }
-        for (int g = 0; g < 2; ++g) {
-            tc::mbar_init(&s_full[g], 1);
-            tc::mbar_init(&p_full[g], 4);
-            tc::mbar_init(&o_full[g], 1);
-            tc::mbar_init(&t_free[g], 4);
-        }
-        tc::mbar_init(drain, 1);
-        *abort_flag = 0;
-        tc::fence_mbar_init();
-    }
-    if (warp == 1) {
-        tc::tmem_alloc(tmem_base, 512);
-        tc::tmem_relinquish();
-    }
-    tc::fence_before_sync();
-    __syncthreads();
-    tc::fence_after_sync();
-    const uint32_t tmem = *tmem_base;
-    const int total = s_ph[ng + 1];
-    bool ok = true;
-    auto fail = [&]() {
-        ok = false;
-        *abort_flag = 1;
-    };
-    // item f: (remote?, slice within the group, index within the slice's remote items or tiles)
-    auto item_of = [&](int f, bool &remote, int &g, int &idx) {
-        int lo = 0, hi = ng + 1;  // last phase k with s_ph[k] <= f
-        while (hi - lo > 1) {
-            const int mid = (lo + hi) >> 1;
-            if (s_ph[mid] <= f) lo = mid;
-            else hi = mid;
-        }
-        const int u = f - s_ph[lo];
-        const int nr = lo < ng ? s_nr[lo] : 0;
-        remote = u < nr;
-        g = remote ? lo : lo - 1;
-        idx = remote ? u : u - nr;
-    };
-
-    if (warp == 0) {
-        // ---------------- producer (the whole warp) ----------------
-        int last_v[NST];
-#pragma unroll
-        for (int s = 0; s < NST; ++s) last_v[s] = -1;
-        int ends = 0;  // end records written (one per softmax group)
-        for (int i = 0; ends < 2 && ok; ++i) {
-            const int s = i % NST, v = i / NST;
-            if (v > 0 && !__all_sync(0xffffffffu, tc::mbar_wait_or_abort(&empty[s], (v - 1) & 1, abort_flag))) {
-                fail();
-                break;
-            }
-            int f = 0;
-            if (lane == 0 && ends == 0) f = atomicAdd(ticket, 1);
-            f = ends ? total : __shfl_sync(0xffffffffu, f, 0);
-            uint8_t *sQ = stage_q(s), *sK = sQ + QB, *sV = sK + KVB;
-            int *rec = stage_rec(s);
-            if (f >= total) {
-                // no item left: an end record for the softmax group of this slot
-                if (lane == 0) rec[128] = 2;
-                __syncwarp();
-                tc::mbar_arrive(&full[s]);
-                if (lane == 0) tc::mbar_arrive(&full[s]);
-                last_v[s] = v;
-                ++ends;
-                continue;
-            }
-            bool remote;
-            int g, idx;
-            item_of(f, remote, g, idx);
-            const int bh = bh0 + g;
-            if (remote) {
-                const int4 w = work[(size_t)bh * wcap + idx];
-                const int j = w.x, p0 = w.y, cnt = w.z;
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const int row = lane + 32 * k;
-                    const bool live = row < cnt;
-                    const int pr = live ? pairs[(size_t)bh * S * R + p0 + row] : -1;
-                    rec[row] = pr;
-                    const bf16 *qrow = Q + ((size_t)bh * S + (live ? pr / R : 0)) * D;
-#pragma unroll
-                    for (int c = 0; c < CH; ++c) tc::cp_async16(sQ + tc::kmajor_chunk(row, c, D), qrow + 8 * c, live);
-                }
-                if (lane == 0) { rec[128] = 1; rec[129] = g; rec[130] = cnt; }
-                asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(tc::smem_u32(&full[s]))
-                             : "memory");
-                __syncwarp();
-                if (lane == 0) {
-                    tc::mbar_expect_tx(&full[s], 2 * RKB);
-#pragma unroll
-                    for (int a = 0; a < D / 64; ++a) {
-                        tc::tma_load_3d(sK + a * (BS * 128), &rm.k, 64 * a, j * BS, bh, &full[s]);
-                        tc::tma_load_3d(sV + a * (BS * 128), &rm.v, 64 * a, j * BS, bh, &full[s]);
-                    }
-                }
-            } else {
-                const int t0 = idx * 128;
-                const int kstart = max(0, t0 / BS - L + 1) * BS;
-                if (lane == 0) { rec[128] = 0; rec[129] = g; rec[130] = t0; }
-                __syncwarp();
-                tc::mbar_arrive(&full[s]);
-                if (lane == 0) {
-                    tc::mbar_expect_tx(&full[s], QB + 2 * KVB);
-#pragma unroll
-                    for (int a = 0; a < D / 64; ++a) {
-                        tc::tma_load_3d(sQ + a * (128 * 128), &lm.q, 64 * a, t0, bh, &full[s]);
-                        tc::tma_load_3d(sK + a * (NK * 128), &lm.k, 64 * a, kstart, bh, &full[s]);
-                        tc::tma_load_3d(sV + a * (NK * 128), &lm.v, 64 * a, kstart, bh, &full[s]);
-                    }
-                }
-            }
-            last_v[s] = v;
-        }
-        asm volatile("cp.async.wait_all;" ::: "memory");
-        if (lane == 0)
-            for (int s = 0; s < NST; ++s)
-                if (last_v[s] >= 0 && !tc::mbar_wait(&full[s], last_v[s] & 1)) ok = false;
-    } else if (warp == 1) {
-        // ---------------- MMA issuer ----------------
-        if (lane == 0) {
-            bool kind_r[2] = {false, false};  // per group: is its current item remote
-            // 1: issued; 0: an end record; -1: gave up
-            auto mma1 = [&](int i) -> int {
-                const int s = i % NST, v = i / NST, g = i & 1, u = i >> 1;
-                if (!tc::mbar_wait_or_abort(&full[s], v & 1, abort_flag)) return -1;
-                tc::fence_after_sync();
-                const int kind = stage_rec(s)[128];
-                if (kind == 2) return 0;
-                if (u > 0 && !tc::mbar_wait_or_abort(&t_free[g], (u - 1) & 1, abort_flag)) return -1;
-                tc::fence_smem_to_async();
-                tc::fence_after_sync();
-                const bool remote = kind != 0;
-                kind_r[g] = remote;
-                const uint32_t aq = tc::smem_u32(stage_q(s)), bk = aq + QB;
-                if (remote) {
-                    const uint32_t id1 = tc::idesc_bf16(128, BS);
-#pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk)
-                        tc::mma_bf16(tmem + g * 256, tc::desc_kmajor(aq + 256 * kk, D),
-                                     tc::desc_sw128(bk + (kk >> 2) * (BS * 128) + (kk & 3) * 32), id1, kk > 0);
-                } else {
-                    const uint32_t id1 = tc::idesc_bf16(128, NK);
-#pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk)
-                        tc::mma_bf16(tmem + g * 256, tc::desc_sw128(aq + (kk >> 2) * (128 * 128) + (kk & 3) * 32),
-                                     tc::desc_sw128(bk + (kk >> 2) * (NK * 128) + (kk & 3) * 32), id1, kk > 0);
-                }
-                tc::commit(&s_full[g]);
-                return 1;
-            };
-            auto mma2 = [&](int i) -> bool {
-                const int s = i % NST, g = i & 1, u = i >> 1;
-                if (!tc::mbar_wait_or_abort(&p_full[g], u & 1, abort_flag)) return false;
-                tc::fence_after_sync();
-                const uint32_t bv = tc::smem_u32(stage_q(s)) + QB + KVB;
-                const uint32_t id2 = tc::idesc_bf16(128, D, true);
-                if (kind_r[g]) {
-#pragma unroll
-                    for (int kk = 0; kk < BS / 16; ++kk)
-                        tc::mma_bf16_ts(tmem + g * 256 + Lay::O_COL, tmem + g * 256 + 8 * kk,
-                                        tc::desc_sw128_mn(bv + 2048 * kk, BS * 128), id2, kk > 0);
-                } else {
-#pragma unroll
-                    for (int kk = 0; kk < NK / 16; ++kk)
-                        tc::mma_bf16_ts(tmem + g * 256 + Lay::O_COL, tmem + g * 256 + 8 * kk,
-                                        tc::desc_sw128_mn(bv + 2048 * kk, NK * 128), id2, kk > 0);
-                }
-                tc::commit(&o_full[g]);
-                tc::commit(&empty[s]);
-                return true;
-            };
-            int r = mma1(0);
-            if (r < 0) fail();
-            for (int i = 0; r > 0 && ok; ++i) {
-                const int r1 = mma1(i + 1);
-                if (r1 < 0) { fail(); break; }
-                if (!mma2(i)) { fail(); break; }
-                r = r1;
-            }
-            tc::commit(drain);
-            if (!tc::mbar_wait(drain, 0)) ok = false;
-        }
-    } else {
-        // ---------------- softmax groups ----------------
-        const int g = (warp - 2) >> 2, quarter = warp & 3;
-        const int row = quarter * 32 + lane;
-        const uint32_t tS = tmem + g * 256 + ((uint32_t)(quarter * 32) << 16);
-        const uint32_t tO = tS + Lay::O_COL;
-        for (int i = g; ok; i += 2) {
-            const int s = i % NST, v = i / NST, u = i >> 1;
-            if (!__all_sync(0xffffffffu, tc::mbar_wait_or_abort(&full[s], v & 1, abort_flag))) { fail(); break; }
-            const int *rec = stage_rec(s);
-            if (rec[128] == 2) break;  // the end record of this group
-            const bool remote = rec[128] != 0;
-            const int sg = rec[129];
-            const int pr = remote ? rec[row] : -1;
-            const int t0 = remote ? 0 : rec[130];
-            const long long bh = bh0 + sg;
-            __syncwarp();
-            if (lane == 0) tc::mbar_arrive(&empty[s]);
-            float vv[32];
-            if (remote) {
-                if (!__all_sync(0xffffffffu, tc::mbar_wait_or_abort(&s_full[g], u & 1, abort_flag))) { fail(); break; }
-                tc::fence_after_sync();
-                float m = -INFINITY;
-#pragma unroll
-                for (int c0 = 0; c0 < BS; c0 += 32) {
-                    __syncwarp();
-                    tc::tmem_ld32(tS + c0, vv);
-#pragma unroll
-                    for (int k = 0; k < 32; ++k) m = fmaxf(m, vv[k]);
-                }
-                const float m2 = m * scale_log2;
-                float l = 0.f;
-#pragma unroll
-                for (int c0 = 0; c0 < BS; c0 += 32) {
-                    __syncwarp();
-                    tc::tmem_ld32(tS + c0, vv);
-                    uint32_t pk[16];
-#pragma unroll
-                    for (int k = 0; k < 16; ++k) {
-                        const float a = exp2f(fmaf(vv[2 * k], scale_log2, -m2));
-                        const float bb = exp2f(fmaf(vv[2 * k + 1], scale_log2, -m2));
-                        l += a + bb;
-                        pk[k] = pack2(a, bb);
-                    }
-                    __syncwarp();
-                    tc::tmem_st16(tS + (c0 >> 1), pk);
-                }
-                __syncwarp();
-                tc::tmem_st_wait();
-                tc::fence_before_sync();
-                __syncwarp();
-                if (lane == 0) tc::mbar_arrive(&p_full[g]);
-                const float inv = 1.f / l;
-                if (!__all_sync(0xffffffffu, tc::mbar_wait_or_abort(&o_full[g], u & 1, abort_flag))) { fail(); break; }
-                tc::fence_after_sync();
-                const bool live = pr >= 0;
-                const size_t slot = (size_t)bh * S * R + (live ? pr : 0);
-#pragma unroll
-                for (int c0 = 0; c0 < D; c0 += 32) {
-                    __syncwarp();
-                    tc::tmem_ld32(tO + c0, vv);
-                    if (live) {
-                        uint4 *dst = (uint4 *)(part_o + slot * D + c0);
-#pragma unroll
-                        for (int q8 = 0; q8 < 4; ++q8)
-                            dst[q8] = make_uint4(pack2(vv[8 * q8] * inv, vv[8 * q8 + 1] * inv),
-                                                 pack2(vv[8 * q8 + 2] * inv, vv[8 * q8 + 3] * inv),
-                                                 pack2(vv[8 * q8 + 4] * inv, vv[8 * q8 + 5] * inv),
-                                                 pack2(vv[8 * q8 + 6] * inv, vv[8 * q8 + 7] * inv));
-                    }
-                }
-                if (live) part_ml[slot] = make_float2(m2, l);
-                __threadfence();   // this warp's partial rows are visible before its count
-                tc::fence_before_sync();
-                __syncwarp();
-                if (lane == 0) {
-                    atomicAdd(&done[bh], 1);
-                    tc::mbar_arrive(&t_free[g]);
-                }
-                continue;
-            }
-            // ---- a local tile: rows t0 .. t0 + 127 of slice sg ----
-            const int b = (int)(bh / H), h = (int)(bh % H);
-            const int kstart = max(0, t0 / BS - L + 1) * BS;
-            const int t = t0 + row;
-            const bool live = t < S;
-            // this row's remote blocks; their partials once the slice's remote items are all done
-            int jr[RMAX];
-            float2 ml[RMAX];
-            bool waited = true;
-            {
-                const int need = 4 * s_nr[sg];
-                bool got = lane != 0;
-                if (lane == 0)
-                    for (uint32_t it = 0; it < (1u << 22) && !*abort_flag; ++it) {
-                        if (ld_acquire(&done[bh]) >= need) { got = true; break; }
-                        __nanosleep(64);
-                    }
-                waited = __all_sync(0xffffffffu, got);
-            }
-            if (!waited) { fail(); break; }
-            (void)ld_acquire(&done[bh]);  // each lane's own acquire of the partials the count covers
-#pragma unroll
-            for (int r = 0; r < RMAX; ++r) {
-                jr[r] = -1;
-                ml[r] = make_float2(0.f, 0.f);
-                const int j = (r < R && live) ? sel[((size_t)bh * S + t) * R + r] : -1;
-                if (!sel_valid(j, t, BS, L)) continue;
-                jr[r] = j;
-                ml[r] = ld_cg_f2(part_ml + ((size_t)bh * S + t) * R + r);
-            }
-            if (!__all_sync(0xffffffffu, tc::mbar_wait_or_abort(&s_full[g], u & 1, abort_flag))) { fail(); break; }
-            tc::fence_after_sync();
-            const int lo = max(0, t / BS - L + 1) * BS;
-            const int vlo = lo - kstart, vhi = t - kstart;
-            float m = -INFINITY;
-#pragma unroll 1
-            for (int c0 = 0; c0 < NK; c0 += 32) {
-                __syncwarp();
-                tc::tmem_ld32(tS + c0, vv);
-                if (c0 + 31 < vlo || c0 > vhi) continue;
-                if (c0 >= vlo && c0 + 31 <= vhi) {
-#pragma unroll
-                    for (int k = 0; k < 32; ++k) m = fmaxf(m, vv[k]);
-                } else {
-#pragma unroll
-                    for (int k = 0; k < 32; ++k)
-                        if (c0 + k >= vlo && c0 + k <= vhi) m = fmaxf(m, vv[k]);
-                }
-            }
-            const float m2 = (m == -INFINITY) ? 0.f : m * scale_log2;
-            float l = 0.f;
-#pragma unroll 1
-            for (int c0 = 0; c0 < NK; c0 += 32) {
-                __syncwarp();
-                tc::tmem_ld32(tS + c0, vv);
-                uint32_t pk[16];
-                if (c0 + 31 < vlo || c0 > vhi) {
-#pragma unroll
-                    for (int k = 0; k < 16; ++k) pk[k] = 0u;
-                } else {
-                    const bool full_chunk = c0 >= vlo && c0 + 31 <= vhi;
-#pragma unroll
-                    for (int k = 0; k < 16; ++k) {
-                        float a = exp2f(fmaf(vv[2 * k], scale_log2, -m2));
-                        float bb = exp2f(fmaf(vv[2 * k + 1], scale_log2, -m2));
-                        if (!full_chunk) {
-                            a = (c0 + 2 * k >= vlo && c0 + 2 * k <= vhi) ? a : 0.f;
-                            bb = (c0 + 2 * k + 1 >= vlo && c0 + 2 * k + 1 <= vhi) ? bb : 0.f;
-                        }
-                        l += a + bb;
-                        pk[k] = pack2(a, bb);
-                    }
-                }
-                __syncwarp();
-                tc::tmem_st16(tS + (c0 >> 1), pk);
-            }
-            __syncwarp();
-            tc::tmem_st_wait();
-            tc::fence_before_sync();
-            __syncwarp();
-            if (lane == 0) tc::mbar_arrive(&p_full[g]);
-            // merge with the remote partials (max/sum rescaling)
-            float mm = m2;
-#pragma unroll
-            for (int r = 0; r < RMAX; ++r)
-                if (jr[r] >= 0) mm = fmaxf(mm, ml[r].x);
-            const float wl = exp2f(m2 - mm);
-            float den = l * wl;
-            float wr[RMAX];
-#pragma unroll
-            for (int r = 0; r < RMAX; ++r) {
-                wr[r] = 0.f;
-                if (jr[r] >= 0) {
-                    wr[r] = ml[r].y * exp2f(ml[r].x - mm);
-                    den += wr[r];
-                }
-            }
-            const float inv = 1.f / den;
-            if (!__all_sync(0xffffffffu, tc::mbar_wait_or_abort(&o_full[g], u & 1, abort_flag))) { fail(); break; }
-            tc::fence_after_sync();
-            bf16 *orow = O + (((size_t)b * S + t) * H + h) * D;
-#pragma unroll
-            for (int c0 = 0; c0 < D; c0 += 32) {
-                __syncwarp();
-                tc::tmem_ld32(tO + c0, vv);
-                if (live) {
-#pragma unroll
-                    for (int k = 0; k < 32; ++k) vv[k] *= wl;
-#pragma unroll
-                    for (int r = 0; r < RMAX; ++r) {
-                        if (jr[r] < 0) continue;
-                        const uint8_t *src = (const uint8_t *)(part_o + (((size_t)bh * S + t) * R + r) * D + c0);
-#pragma unroll
-                        for (int q8 = 0; q8 < 4; ++q8) {
-                            const uint4 u4 = ld_cg16(src + 16 * q8);
-                            const __nv_bfloat162 *h2 = (const __nv_bfloat162 *)&u4;
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                const float2 fv = __bfloat1622float2(h2[e]);
-                                vv[8 * q8 + 2 * e] = fmaf(wr[r], fv.x, vv[8 * q8 + 2 * e]);
-                                vv[8 * q8 + 2 * e + 1] = fmaf(wr[r], fv.y, vv[8 * q8 + 2 * e + 1]);
-                            }
-                        }
-                    }
-                    uint4 *dst = (uint4 *)(orow + c0);
-#pragma unroll
-                    for (int q8 = 0; q8 < 4; ++q8)
-                        dst[q8] = make_uint4(pack2(vv[8 * q8] * inv, vv[8 * q8 + 1] * inv),
-                                             pack2(vv[8 * q8 + 2] * inv, vv[8 * q8 + 3] * inv),
-                                             pack2(vv[8 * q8 + 4] * inv, vv[8 * q8 + 5] * inv),
-                                             pack2(vv[8 * q8 + 6] * inv, vv[8 * q8 + 7] * inv));
-                }
-            }
-            tc::fence_before_sync();
-            __syncwarp();
-            if (lane == 0) tc::mbar_arrive(&t_free[g]);
-        }
-    }
-    if (!ok) record_error(counters, kDevErrTimeout);
-    tc::fence_before_sync();
-    __syncthreads();
-    tc::fence_after_sync();
-    if (warp == 1) {
-        __syncwarp();
-        tc::tmem_dealloc(tmem, 512);
-    }
-}
-
-// ---------------------------------------------------------------------------
 bool attend_tc_supported(const mono_config &c) {
     if (c.dtype != MONO_BF16 || (c.d != 64 && c.d != 128) || (c.Bs != 64 && c.Bs != 128)) return false;
     const int nk = 128 + (c.L - 1) * c.Bs;
@@ -1993,8 +1149,6 @@ static cudaError_t launch_tc_shape(const Plan &p, const bf16 *Q, const bf16 *K, 
         !make_map_3d(&rmaps.k, K, D, c.S, c.B * c.H, BS) || !make_map_3d(&rmaps.v, V, D, c.S, c.B * c.H, BS))
         return cudaErrorInvalidValue;
     constexpr size_t rsmem = RemoteSmem<D, BS>::BYTES;
-    // the warp-specialised remote kernel where its ring fits, else the two-stage one
-    constexpr bool kRemoteWs = RemoteWs<D, BS>::supported && !MONO_REMOTE_TWO_STAGE;
     if (c.R > 0 && (parts & kAttendPairs)) {
         int32_t *pc = (int32_t *)ws_ptr(p, ws, kRegPairCount);
         int32_t *ps = (int32_t *)ws_ptr(p, ws, kRegPairStart);
@@ -2002,10 +1156,8 @@ static cudaError_t launch_tc_shape(const Plan &p, const bf16 *Q, const bf16 *K, 
         int32_t *pairs = (int32_t *)ws_ptr(p, ws, kRegPairs);
         int4 *work = (int4 *)ws_ptr(p, ws, kRegWork);
         int32_t *nwork = (int32_t *)ws_ptr(p, ws, kRegNWork);
-        int *done = (int *)ws_ptr(p, ws, kRegDone);
         const int nbhh = c.B * c.H;
         const int wcap = p.max_work;  // work items per (b, h)
-        const int grp = std::min(kMaxGroup, nbhh);
         if ((e = cudaMemsetAsync(pc, 0, (size_t)nbh * 4, s)) != cudaSuccess) return e;
         dim3 gq((c.S + kQTile - 1) / kQTile, nbhh);
         const size_t hs = (size_t)p.nb * 4;
@@ -2015,8 +1167,8 @@ static cudaError_t launch_tc_shape(const Plan &p, const bf16 *Q, const bf16 *K, 
                 return e;
         }
         k_pair_count<<<gq, 256, hs, s>>>(sel, pc, c.S, c.R, p.nb, c.Bs, c.L, cnt_err);
-        if ((e = launch_pdl(k_pair_scan, dim3(nbhh), dim3(1024), 0, s, (const int32_t *)pc, ps, pf, work, nwork, done,
-                            done + nbhh, p.nb, wcap, grp)) != cudaSuccess)
+        if ((e = launch_pdl(k_pair_scan, dim3(nbhh), dim3(1024), 0, s, (const int32_t *)pc, ps, pf, work, nwork, p.nb,
+                            wcap)) != cudaSuccess)
             return e;
         if ((e = launch_pdl(k_pair_fill, gq, dim3(256), 2 * hs, s, sel, (const int32_t *)ps, pf, pairs, c.S, c.R, p.nb,
                             c.Bs, c.L)) != cudaSuccess)
@@ -2025,14 +1177,9 @@ static cudaError_t launch_tc_shape(const Plan &p, const bf16 *Q, const bf16 *K, 
         count_launches(2);
     }
     if (c.R > 0 && (parts & kAttendRemote)) {
-        if constexpr (kRemoteWs) {
-            if ((e = cudaFuncSetAttribute(k_remote_ws<D, BS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                          (int)RemoteWs<D, BS>::BYTES)) != cudaSuccess)
-                return e;
-        } else if ((e = cudaFuncSetAttribute(k_remote_tc<D, BS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)rsmem)) != cudaSuccess) {
+        if ((e = cudaFuncSetAttribute(k_remote_tc<D, BS>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rsmem)) !=
+            cudaSuccess)
             return e;
-        }
     }
     // the local part: the warp-specialised kernel where its stages and tensor
     // memory fit, else the single-stage one
@@ -2059,45 +1206,10 @@ static cudaError_t launch_tc_shape(const Plan &p, const bf16 *Q, const bf16 *K, 
     // (attention at S = 32768, 16 heads: 275 us in one group, 327 us in four):
     // fewer launch tails, and the remote kernel balances more work items.
     int remote_ctas = 0;
-    if (c.R > 0) {
-        if constexpr (kRemoteWs) {
-            int dev = 0;
-            if ((e = cudaGetDevice(&dev)) != cudaSuccess ||
-                (e = cudaDeviceGetAttribute(&remote_ctas, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
-                return e;
-        } else if ((e = persistent_grid(k_remote_tc<D, BS>, 256, rsmem, &remote_ctas)) != cudaSuccess) {
-            return e;
-        }
-    }
+    if (c.R > 0 && (e = persistent_grid(k_remote_tc<D, BS>, 256, rsmem, &remote_ctas)) != cudaSuccess)
+        return e;
     const int nbhh = c.B * c.H;
     const int group = c.R > 0 ? std::min(kMaxGroup, nbhh) : nbhh;
-    // all stages at once: the fused kernel per group of slices where it applies and is selected
-    constexpr bool kFused = AttendWs<D, BS, NK>::supported && MONO_ATTEND_FUSED;
-    if constexpr (kFused) {
-        if (c.R > 0 && (parts & kAttendRemote) && (parts & kAttendLocal)) {
-            constexpr size_t fsmem = AttendWs<D, BS, NK>::BYTES;
-            auto kf = k_attend_ws<D, BS, NK, RMAX>;
-            if ((e = cudaFuncSetAttribute(kf, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fsmem)) != cudaSuccess)
-                return e;
-            // [B*H] done counts, then one ticket per launch group: cleared by k_pair_scan
-            int *done = (int *)ws_ptr(p, ws, kRegDone);
-            int dev = 0, sms = 0;
-            if ((e = cudaGetDevice(&dev)) != cudaSuccess ||
-                (e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
-                return e;
-            for (int g0 = 0; g0 < nbhh; g0 += group) {
-                const int ng = std::min(group, nbhh - g0);
-                if ((e = launch_pdl(kf, dim3(sms), dim3(320), fsmem, s, lmaps, rmaps, Q, sel,
-                                    (const int32_t *)ws_ptr(p, ws, kRegPairs), (const int4 *)ws_ptr(p, ws, kRegWork),
-                                    (const int32_t *)ws_ptr(p, ws, kRegNWork), (bf16 *)ws_ptr(p, ws, kRegPartO),
-                                    (float2 *)ws_ptr(p, ws, kRegPartML), done, done + nbhh + g0 / group, O, cnt_err,
-                                    c.S, c.H, c.R, c.L, p.max_work, scale_log2, g0, ng)) != cudaSuccess)
-                    return e;
-                count_launches(1);
-            }
-            return cudaSuccess;
-        }
-    }
     // remote then local per group of slices; one stage at a time: over every group
     const bool both = (parts & kAttendRemote) && (parts & kAttendLocal);
     for (int pass = 0; pass < (both ? 1 : 2); ++pass)
@@ -2106,16 +1218,10 @@ static cudaError_t launch_tc_shape(const Plan &p, const bf16 *Q, const bf16 *K, 
         const bool do_remote = (parts & kAttendRemote) && (both || pass == 0);
         const bool do_local = (parts & kAttendLocal) && (both || pass == 1);
         if (c.R > 0 && do_remote) {
-            if constexpr (kRemoteWs)
-                k_remote_ws<D, BS><<<remote_ctas, RemoteWs<D, BS>::THREADS, RemoteWs<D, BS>::BYTES, s>>>(
-                    rmaps, Q, (const int32_t *)ws_ptr(p, ws, kRegPairs), (const int4 *)ws_ptr(p, ws, kRegWork),
-                    (const int32_t *)ws_ptr(p, ws, kRegNWork), (bf16 *)ws_ptr(p, ws, kRegPartO),
-                    (float2 *)ws_ptr(p, ws, kRegPartML), cnt_err, c.S, c.R, p.max_work, scale_log2, g0, ng);
-            else
-                k_remote_tc<D, BS><<<remote_ctas, 256, rsmem, s>>>(
-                    rmaps, Q, (const int32_t *)ws_ptr(p, ws, kRegPairs), (const int4 *)ws_ptr(p, ws, kRegWork),
-                    (const int32_t *)ws_ptr(p, ws, kRegNWork), (bf16 *)ws_ptr(p, ws, kRegPartO),
-                    (float2 *)ws_ptr(p, ws, kRegPartML), cnt_err, c.S, c.R, p.max_work, scale_log2, g0, ng);
+            k_remote_tc<D, BS><<<remote_ctas, 256, rsmem, s>>>(
+                rmaps, Q, (const int32_t *)ws_ptr(p, ws, kRegPairs), (const int4 *)ws_ptr(p, ws, kRegWork),
+                (const int32_t *)ws_ptr(p, ws, kRegNWork), (bf16 *)ws_ptr(p, ws, kRegPartO),
+                (float2 *)ws_ptr(p, ws, kRegPartML), cnt_err, c.S, c.R, p.max_work, scale_log2, g0, ng);
             count_launches(1);
         }
         if (!do_local) continue;

@@ -197,14 +197,15 @@ __global__ void __launch_bounds__(192, 2) k_gemm_tc(const __grid_constant__ TmaM
 // that concurrent CTAs share A in L2).  The producer runs ahead across tile
 // boundaries through a 4-stage ring of 48 KB stages; the MMA issuer
 // alternates two 128 x 256 fp32 accumulators in TMEM (all 512 columns), so
-// the epilogue of tile i (four warps, TMEM -> registers -> RoPE -> bf16
-// stores) overlaps the MMAs of tile i+1.
+// the epilogue of tile i (eight warps, two per TMEM lane quarter, each half of
+// the columns: TMEM -> registers -> RoPE -> bf16 stores) overlaps the MMAs of
+// tile i+1.
 // ---------------------------------------------------------------------------
 constexpr int PBN = 256, PSTAGES = 4;
 constexpr int PB_BYTES = PBN * BK * 2;
 constexpr int PSMEM_BYTES = PSTAGES * (A_BYTES + PB_BYTES) + 1024;
 
-__global__ void __launch_bounds__(192, 1) k_gemm_tcp(const __grid_constant__ TmaMaps maps, const Epi epi, int K,
+__global__ void __launch_bounds__(320, 1) k_gemm_tcp(const __grid_constant__ TmaMaps maps, const Epi epi, int K,
                                                      int tiles_n, int tiles_m, int nz) {
     extern __shared__ uint8_t smem_raw[];
     __shared__ uint64_t full[PSTAGES], empty[PSTAGES], accf[2], accfree[2], drain;
@@ -229,7 +230,7 @@ __global__ void __launch_bounds__(192, 1) k_gemm_tcp(const __grid_constant__ Tma
         }
         for (int a = 0; a < 2; ++a) {
             tc::mbar_init(&accf[a], 1);
-            tc::mbar_init(&accfree[a], 4);
+            tc::mbar_init(&accfree[a], 8);
         }
         tc::mbar_init(&drain, 1);
         tc::fence_mbar_init();
@@ -294,8 +295,9 @@ __global__ void __launch_bounds__(192, 1) k_gemm_tcp(const __grid_constant__ Tma
         tc::commit(&drain);
         if (!tc::mbar_wait(&drain, 0, 1u << 20)) fail = 1;
     } else if (warp >= 2) {
-        // epilogue: warp w reads TMEM lanes 32*(w%4) .. +31 = tile rows
-        const int q = warp & 3;
+        // epilogue, eight warps: warp w reads TMEM lanes 32*(w%4) .. +31 = tile rows, columns
+        // [128 c, 128 c + 128) with c = (w - 2) / 4
+        const int q = warp & 3, ch = (warp - 2) >> 2;
         const int half = epi.d / 2;
         int lt = 0;
         for (int t = blockIdx.x; t < total; t += G, ++lt) {
@@ -309,7 +311,7 @@ __global__ void __launch_bounds__(192, 1) k_gemm_tcp(const __grid_constant__ Tma
             const int m = m0 + q * 32 + lane;
             const int mode = epi.mode[z];
             bf16 *out = epi.out[z];
-            for (int c0 = 0; c0 < PBN; c0 += 32) {
+            for (int c0 = ch * (PBN / 2); c0 < (ch + 1) * (PBN / 2); c0 += 32) {
                 float v[32];
                 __syncwarp();
                 tc::tmem_ld32(trow + c0, v);
@@ -382,7 +384,7 @@ cudaError_t launch_persistent(const TmaMaps &maps, const Epi &epi, int nz, int K
         return e;
     const int tn = epi.N / PBN, tm = (epi.M + BM - 1) / BM;
     const int total = tn * tm * nz;
-    k_gemm_tcp<<<std::min(total, sms), 192, PSMEM_BYTES, s>>>(maps, epi, K, tn, tm, nz);
+    k_gemm_tcp<<<std::min(total, sms), 320, PSMEM_BYTES, s>>>(maps, epi, K, tn, tm, nz);
     count_launches(1);
     return cudaGetLastError();
 }

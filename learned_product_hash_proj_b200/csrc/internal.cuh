@@ -61,7 +61,6 @@ enum Region {
     kRegPartML,      // [B*H*S*R] float2 (max, sum) of remote partials
     kRegWork,        // [B*H, max_work] int4 (block, first pair, pair count, 0) work items of the remote kernel
     kRegNWork,       // [B*H] int32 number of work items
-    kRegDone,        // [B*H] int32 remote items finished (x4 warps), read by the fused kernel's local tiles
     kRegN
 };
 
