@@ -283,7 +283,7 @@ def run_ours(args):
     single_kernel_stages = {"summaries": "k_summary_assign_w",
                             "lists": "k_posting_dense" if cfg.A <= 4096 else "k_posting_build",
                             "queries": "k_probe_m2" if cfg.M == 2 else "k_probe_rerank",
-                            "remote": "k_remote_ws", "local": "k_local_ws" if cfg.dtype == "bf16" else "k_attend_simt"}
+                            "remote": "k_remote_tc", "local": "k_local_ws" if cfg.dtype == "bf16" else "k_attend_simt"}
     dom = max(single_kernel_stages, key=lambda n: stage[n])
     achieved = ab[dom] / (stage[dom] / 1e3) / 1e9
     window_gbs = ab["route_attend"] / (ra / 1e3) / 1e9

@@ -118,10 +118,10 @@ __device__ __forceinline__ void store_grad16(const GradOut &go, void *out, bool 
     }
     if (rotate) {
         const float2 *hi = go.rope_hi + (size_t)(t / kRopeLo) * (DD / 2) + e0 / 2;
-        const float2 *lo = go.rope_lo + (size_t)(t % kRopeLo) * (DD / 2) + e0 / 2;
+        const float2 *lo = go.rope_lo + (size_t)(e0 / 2) * kRopeLo + t % kRopeLo;  // frequency-major
 #pragma unroll
         for (int pr = 0; pr < 8; ++pr) {
-            const float2 a = __ldg(hi + pr), bb = __ldg(lo + pr);
+            const float2 a = __ldg(hi + pr), bb = __ldg(lo + pr * kRopeLo);
             const float c = a.x * bb.x - a.y * bb.y, sn = a.y * bb.x + a.x * bb.y;
             const float x0 = v[2 * pr], x1 = v[2 * pr + 1];
             v[2 * pr] = x0 * c + x1 * sn;

@@ -90,10 +90,10 @@ __device__ __forceinline__ void epi_store(const Epi &epi, int mode, bf16 *out, i
         const int h = n / epi.d, i0 = n % epi.d;
         if (mode == kEpiRope) {
             const float2 *hi = epi.rope_hi + (size_t)(t / kRopeLo) * half + i0 / 2;
-            const float2 *lo = epi.rope_lo + (size_t)(t % kRopeLo) * half + i0 / 2;
+            const float2 *lo = epi.rope_lo + (size_t)(i0 / 2) * kRopeLo + t % kRopeLo;  // frequency-major
 #pragma unroll
             for (int pr = 0; pr < 16; ++pr) {
-                const float2 a = __ldg(hi + pr), bb = __ldg(lo + pr);
+                const float2 a = __ldg(hi + pr), bb = __ldg(lo + pr * kRopeLo);
                 const float c = a.x * bb.x - a.y * bb.y, sn = a.y * bb.x + a.x * bb.y;
                 const float x0 = v[2 * pr], x1 = v[2 * pr + 1];
                 v[2 * pr] = x0 * c - x1 * sn;

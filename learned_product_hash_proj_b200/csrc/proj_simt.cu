@@ -13,7 +13,8 @@ namespace mono {
 // epilogue combines them with the angle-addition identity in fp32.  This keeps
 // the rotation accurate to a few fp32 ulps at any position without an fp64
 // sincos per element.
-// hi: [nhi][d/2] float2 of (th*64) * w_i ; lo: [64][d/2] float2 of tl * w_i.
+// hi: [nhi][d/2] float2 of (th*64) * w_i ; lo: [d/2][64] float2 of tl * w_i,
+// frequency-major, so that 32 consecutive positions read 256 contiguous bytes.
 // ---------------------------------------------------------------------------
 __global__ void k_rope_tables(float2 *hi, float2 *lo, int nhi, int half, int d, double theta) {
     int idx = blockIdx.x * blockDim.x + threadIdx.x;
@@ -26,7 +27,7 @@ __global__ void k_rope_tables(float2 *hi, float2 *lo, int nhi, int half, int d, 
     sincos(pos * w, &s, &c);
     float2 v = make_float2((float)c, (float)s);
     if (row < nhi) hi[(size_t)row * half + i] = v;
-    else lo[(size_t)(row - nhi) * half + i] = v;
+    else lo[(size_t)i * kRopeLo + (row - nhi)] = v;
 }
 
 cudaError_t launch_rope_tables(const Plan &p, void *ws, cudaStream_t s) {
@@ -42,7 +43,7 @@ cudaError_t launch_rope_tables(const Plan &p, void *ws, cudaStream_t s) {
 
 __device__ __forceinline__ float2 rope_cs(const float2 *hi, const float2 *lo, int t, int i, int half) {
     float2 a = hi[(size_t)(t / kRopeLo) * half + i];
-    float2 b = lo[(size_t)(t % kRopeLo) * half + i];
+    float2 b = lo[(size_t)i * kRopeLo + t % kRopeLo];
     // cos(x+y) = cos x cos y - sin x sin y ; sin(x+y) = sin x cos y + cos x sin y
     return make_float2(a.x * b.x - a.y * b.y, a.y * b.x + a.x * b.y);
 }

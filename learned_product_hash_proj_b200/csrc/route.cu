@@ -935,14 +935,15 @@ constexpr size_t probe_m2_smem(int nb) {
            (size_t)nb * 8;
 }
 
-// The probe, union, causal filter and E cap of one query-head t from its
-// subspace scores (see k_probe_m2): the candidates cid[0 .. nc) in probe
-// order.  Their kbar rows are prefetched to L1 for the rerank.
-template <typename T, int D, int C, int TP, int E>
-__device__ __forceinline__ int select_m2(const float (&s0)[C], const float (&s1)[C], const int2 *s_rng,
-                                         const int32_t *s_ids, const float *kb, int (&cid)[E], int t, size_t bh,
-                                         int S, int Bs, int L, int cap, unsigned long long *counters,
-                                         int32_t *walk_log) {
+// The probe, union, causal filter, E cap and rerank of one query-head t from
+// its subspace scores (see k_probe_m2).  Writes sel; returns the number of
+// remote blocks selected and sets *ign when a forced id was not eligible.
+template <typename T, int D, int C, int TP, int E, int R>
+__device__ __forceinline__ int route_query_m2(const float (&s0)[C], const float (&s1)[C], const T *qp,
+                                              const int2 *s_rng, const int32_t *s_ids, const float *kb,
+                                              const int32_t *forced, int32_t *out, int t, size_t bh, int S,
+                                              int Bs, int L, int cap, unsigned long long *counters,
+                                              int32_t *walk_log, int *ign) {
     constexpr int A = C * C;
     float mx0 = 0.f, mx1 = 0.f;
 #pragma unroll
@@ -1017,9 +1018,10 @@ __device__ __forceinline__ int select_m2(const float (&s0)[C], const float (&s1)
         }
     }
 
-    // union of the probed lists in probe order, causal filter, E cap
+    // union of the probed lists in probe order, causal filter, E cap ...
     const int bq = t / Bs;
     const int lim = bq - L;
+    int cid[E];
 #pragma unroll
     for (int e = 0; e < E; ++e) cid[e] = 0;
     int nc = 0;
@@ -1041,24 +1043,8 @@ __device__ __forceinline__ int select_m2(const float (&s0)[C], const float (&s1)
             ++nc;
         }
     }
-#pragma unroll
-    for (int e = 0; e < E; ++e)
-        if (e < nc)
-#pragma unroll
-            for (int ln = 0; ln < D * 4; ln += 128) tc::prefetch_l1(kb + (size_t)cid[e] * D + ln / 4);
-    return nc;
-}
-
-// The rerank q . kbar_j of the (at most E) candidates of query-head t, their
-// fma chains advancing together in ascending element order; top R (score
-// desc, id asc); the forced block; sel in ascending order.  Returns the number
-// of remote blocks selected and adds 1 to *ign when a forced id was not
-// eligible.
-template <typename T, int D, int E, int R>
-__device__ __forceinline__ int rerank_m2(const T *qp, const float *kb, const int (&cid)[E], int nc,
-                                         const int32_t *forced, int32_t *out, int t, size_t bh, int S, int Bs, int L,
-                                         int *ign) {
-    const int lim = t / Bs - L;
+    // ... and the rerank q . kbar_j of the (at most E) candidates, their
+    // fma chains advancing together in ascending element order
     float acc[E];
 #pragma unroll
     for (int e = 0; e < E; ++e) acc[e] = 0.0f;
@@ -1220,25 +1206,13 @@ __global__ void __launch_bounds__(128, C <= 16 ? 4 : 3) k_probe_m2(const T *__re
     __syncthreads();
     int n_sel = 0, lt_r = 0, ign = 0;
     const float *kb = kbar + bh * nb * D;
-    // every query's candidates first (their kbar rows prefetched), then every rerank: the rows of one query
-    // travel from L2 while the next query is probed
-    int cid[NQ][E], nc[NQ];
-#pragma unroll
-    for (int q = 0; q < NQ; ++q) {
-        const int t = t_lo + tid + 128 * q;
-        nc[q] = 0;
-#pragma unroll
-        for (int e = 0; e < E; ++e) cid[q][e] = 0;
-        if (t < S)
-            nc[q] = select_m2<T, D, C, TP, E>(s0[q], s1[q], s_rng, s_ids, kb, cid[q], t, bh, S, Bs, L, cap, counters,
-                                              walk_log);
-    }
 #pragma unroll
     for (int q = 0; q < NQ; ++q) {
         const int t = t_lo + tid + 128 * q;
         if (t < S) {
-            const int nr = rerank_m2<T, D, E, R>((const T *)(s_q + (tid + 128 * q) * QP), kb, cid[q], nc[q], forced,
-                                                 sel + (bh * S + t) * R, t, bh, S, Bs, L, &ign);
+            const int nr = route_query_m2<T, D, C, TP, E, R>(s0[q], s1[q], (const T *)(s_q + (tid + 128 * q) * QP),
+                                                             s_rng, s_ids, kb, forced, sel + (bh * S + t) * R, t, bh,
+                                                             S, Bs, L, cap, counters, walk_log, &ign);
             n_sel += nr;
             lt_r += nr < R;
         }
