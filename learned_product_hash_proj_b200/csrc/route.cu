@@ -935,6 +935,83 @@ constexpr size_t probe_m2_smem(int nb) {
            (size_t)nb * 8;
 }
 
+// The rerank q . kbar_j of the (at most E) candidates cid[0 .. nc) of
+// query-head t, their fma chains advancing together in ascending element
+// order; top R (score desc, id asc); the forced block; sel in ascending order
+// with -1 padding.  Returns the number of remote blocks selected and adds 1
+// to *ign when a forced id was not eligible.
+template <typename T, int D, int E, int R>
+__device__ __forceinline__ int rerank_m2(const T *qp, const float *kb, const int (&cid)[E], int nc,
+                                         const int32_t *forced, int32_t *out, int t, size_t bh, int S, int Bs, int L,
+                                         int *ign) {
+    const int lim = t / Bs - L;
+    float acc[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) acc[e] = 0.0f;
+#pragma unroll 2
+    for (int i8 = 0; i8 < D / 8; ++i8) {
+        float qv[8];
+        q8<T>(qp + 8 * i8, qv);
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+            if (e < nc) {
+                const float4 *kr = (const float4 *)(kb + (size_t)cid[e] * D + 8 * i8);
+                const float4 x = __ldg(kr), y = __ldg(kr + 1);
+                float a = acc[e];
+                a = __fmaf_rn(qv[0], x.x, a);
+                a = __fmaf_rn(qv[1], x.y, a);
+                a = __fmaf_rn(qv[2], x.z, a);
+                a = __fmaf_rn(qv[3], x.w, a);
+                a = __fmaf_rn(qv[4], y.x, a);
+                a = __fmaf_rn(qv[5], y.y, a);
+                a = __fmaf_rn(qv[6], y.z, a);
+                a = __fmaf_rn(qv[7], y.w, a);
+                acc[e] = a;
+            }
+        }
+    }
+    RegTop<R> rk;
+    rk.init();
+#pragma unroll
+    for (int e = 0; e < E; ++e)
+        if (e < nc) rk.push(acc[e], cid[e]);
+    int ra[R];
+    int nr = nc < R ? nc : R;
+#pragma unroll
+    for (int k = 0; k < R; ++k) ra[k] = rk.a[k];
+    if (forced) {
+        const int f = forced[bh * S + t];
+        if (f >= 0) {
+            if (f <= lim) {
+                bool present = false;
+#pragma unroll
+                for (int k = 0; k < R; ++k) present |= (k < nr) && ra[k] == f;
+                if (!present) {
+                    const int slot = nr < R ? nr : R - 1;
+#pragma unroll
+                    for (int k = 0; k < R; ++k)
+                        if (k == slot) ra[k] = f;
+                    if (nr < R) ++nr;
+                }
+            } else {
+                *ign += 1;
+            }
+        }
+    }
+    // ascending ids, -1 padding
+#pragma unroll
+    for (int k = 0; k < R; ++k)
+        if (k >= nr) ra[k] = 0x7fffffff;
+#pragma unroll
+    for (int x = 0; x < R; ++x)
+#pragma unroll
+        for (int y = 0; y + 1 < R - x; ++y)
+            if (ra[y] > ra[y + 1]) { int tmp = ra[y]; ra[y] = ra[y + 1]; ra[y + 1] = tmp; }
+#pragma unroll
+    for (int k = 0; k < R; ++k) out[k] = k < nr ? ra[k] : -1;
+    return nr;
+}
+
 // The probe, union, causal filter, E cap and rerank of one query-head t from
 // its subspace scores (see k_probe_m2).  Writes sel; returns the number of
 // remote blocks selected and sets *ign when a forced id was not eligible.
@@ -1043,73 +1120,8 @@ __device__ __forceinline__ int route_query_m2(const float (&s0)[C], const float 
             ++nc;
         }
     }
-    // ... and the rerank q . kbar_j of the (at most E) candidates, their
-    // fma chains advancing together in ascending element order
-    float acc[E];
-#pragma unroll
-    for (int e = 0; e < E; ++e) acc[e] = 0.0f;
-#pragma unroll 2
-    for (int i8 = 0; i8 < D / 8; ++i8) {
-        float qv[8];
-        q8<T>(qp + 8 * i8, qv);
-#pragma unroll
-        for (int e = 0; e < E; ++e) {
-            if (e < nc) {
-                const float4 *kr = (const float4 *)(kb + (size_t)cid[e] * D + 8 * i8);
-                const float4 x = __ldg(kr), y = __ldg(kr + 1);
-                float a = acc[e];
-                a = __fmaf_rn(qv[0], x.x, a);
-                a = __fmaf_rn(qv[1], x.y, a);
-                a = __fmaf_rn(qv[2], x.z, a);
-                a = __fmaf_rn(qv[3], x.w, a);
-                a = __fmaf_rn(qv[4], y.x, a);
-                a = __fmaf_rn(qv[5], y.y, a);
-                a = __fmaf_rn(qv[6], y.z, a);
-                a = __fmaf_rn(qv[7], y.w, a);
-                acc[e] = a;
-            }
-        }
-    }
-    RegTop<R> rk;
-    rk.init();
-#pragma unroll
-    for (int e = 0; e < E; ++e)
-        if (e < nc) rk.push(acc[e], cid[e]);
-    int ra[R];
-    int nr = nc < R ? nc : R;
-#pragma unroll
-    for (int k = 0; k < R; ++k) ra[k] = rk.a[k];
-    if (forced) {
-        const int f = forced[bh * S + t];
-        if (f >= 0) {
-            if (f <= lim) {
-                bool present = false;
-#pragma unroll
-                for (int k = 0; k < R; ++k) present |= (k < nr) && ra[k] == f;
-                if (!present) {
-                    const int slot = nr < R ? nr : R - 1;
-#pragma unroll
-                    for (int k = 0; k < R; ++k)
-                        if (k == slot) ra[k] = f;
-                    if (nr < R) ++nr;
-                }
-            } else {
-                *ign += 1;
-            }
-        }
-    }
-    // ascending ids, -1 padding
-#pragma unroll
-    for (int k = 0; k < R; ++k)
-        if (k >= nr) ra[k] = 0x7fffffff;
-#pragma unroll
-    for (int x = 0; x < R; ++x)
-#pragma unroll
-        for (int y = 0; y + 1 < R - x; ++y)
-            if (ra[y] > ra[y + 1]) { int tmp = ra[y]; ra[y] = ra[y + 1]; ra[y + 1] = tmp; }
-#pragma unroll
-    for (int k = 0; k < R; ++k) out[k] = k < nr ? ra[k] : -1;
-    return nr;
+    // ... and the rerank
+    return rerank_m2<T, D, E, R>(qp, kb, cid, nc, forced, out, t, bh, S, Bs, L, ign);
 }
 
 // M = 2 with every size fixed at compile time, so all per-query state stays
@@ -1216,6 +1228,320 @@ __global__ void __launch_bounds__(128, C <= 16 ? 4 : 3) k_probe_m2(const T *__re
             n_sel += nr;
             lt_r += nr < R;
         }
+    }
+    for (int o = 16; o > 0; o >>= 1) {
+        n_sel += __shfl_xor_sync(0xffffffffu, n_sel, o);
+        lt_r += __shfl_xor_sync(0xffffffffu, lt_r, o);
+        ign += __shfl_xor_sync(0xffffffffu, ign, o);
+    }
+    if ((threadIdx.x & 31) == 0) {
+        if (lt_r) atomicAdd(&counters[kCntQueriesLtR], (unsigned long long)lt_r);
+        if (n_sel) atomicAdd(&counters[kCntRemoteSel], (unsigned long long)n_sel);
+        if (ign) atomicAdd(&counters[kCntForcedIgnored], (unsigned long long)ign);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// (A5-A7) the probe for M >= 2 subspaces as a best-first walk of the product
+// grid, every size fixed at compile time.  Same result, arithmetic order and
+// rerank as k_probe_rerank.
+//
+// Each subspace's codes are ranked by (score desc, code asc) lazily: the next
+// rank is an argmax over the codes not yet ranked, taken only when the walk
+// first reaches it.  A tuple of ranks r = (r_0, .., r_{M-1}) scores
+// g(r) = fl(..fl(v_0[r_0] + v_1[r_1]) .. + v_{M-1}[r_{M-1}]), which does not
+// increase when any r_m grows (fp32 addition is monotone in each operand).
+// The tuples form a tree in which the parent of r lowers its last nonzero
+// rank by one.  A heap pops the frontier's first tuple under the probe order
+// (g desc, address asc); the first T pops are the probes provided that no
+// tuple precedes its parent in that order.  A child with a lower g follows
+// its parent; one with an equal g follows it when the raised rank's code is
+// higher, which a tie of the two scores guarantees (ranks order tied codes
+// ascending).  An equal g from unequal scores (the smaller one absorbed by
+// rounding) needs the two scores within delta = (M+1) ulp(2G) of each other.
+// So the walk falls back to scoring the whole grid when
+//  * a child it pushes precedes its parent, or
+//  * after T pops the frontier's best g equals the T-th probe's (the tie
+//    runs past the probes, through tuples not yet visited) and some two
+//    neighbouring ranks of a subspace differ by more than 0 and at most delta;
+//  * or a score is not finite.
+// Exact ties (a zero query, duplicated codewords) thus stay on the walk.
+// ---------------------------------------------------------------------------
+template <int C>
+constexpr int rank_bits() {
+    return C <= 2 ? 1 : C <= 4 ? 2 : C <= 8 ? 3 : C <= 16 ? 4 : 5;
+}
+template <int M, int TP>
+constexpr int bf_heap() {  // each pop removes one tuple and pushes at most M children
+    return 1 + TP * (M - 1);
+}
+template <typename T, int D, int M, int C>
+constexpr size_t probe_bf_smem(int nb) {
+    return (size_t)C * D * 4 + (size_t)128 * probe_q_pitch<T, D>() + (size_t)nb * 8;
+}
+
+template <typename T, int D, int M, int C, int TP, int E, int R>
+__global__ void __launch_bounds__(128) k_probe_bf(const T *__restrict__ Q, const float *__restrict__ kbar,
+                                                  const float *__restrict__ cb, const int32_t *__restrict__ post_ids,
+                                                  const int32_t *__restrict__ post_addr,
+                                                  const int32_t *__restrict__ forced, int32_t *__restrict__ sel,
+                                                  unsigned long long *__restrict__ counters,
+                                                  int32_t *__restrict__ walk_log, int S, int H, int Bs, int L,
+                                                  int cap) {
+    constexpr int DM = D / M, QP = probe_q_pitch<T, D>(), RB = rank_bits<C>();
+    constexpr unsigned RMASK = (1u << RB) - 1u;
+    constexpr int NHEAP = bf_heap<M, TP>();
+    static_assert(M >= 2 && M * RB <= 32 && C <= 32 && C % 4 == 0 && DM % 8 == 0 && TP >= 1 && R >= 1, "shape");
+    extern __shared__ __align__(16) float smem[];
+    pdl_launch_dependents();
+    const int nb = S / Bs;
+    float *s_cbT = smem;                                 // [M][DM][C]: element i of codeword (m, c) at (m DM + i) C + c
+    uint8_t *s_q = (uint8_t *)(s_cbT + C * D);           // [128] query rows, pitch QP
+    int32_t *s_addr = (int32_t *)(s_q + 128 * QP);       // [nb]
+    int32_t *s_ids = s_addr + nb;                        // [nb]
+    const int h = blockIdx.y, b = blockIdx.z;
+    const size_t bh = (size_t)b * H + h;
+    const int tid = threadIdx.x;
+    const int t_lo = blockIdx.x * 128;
+    {
+        constexpr int CH = D * (int)sizeof(T) / 16;
+        const uint8_t *src = (const uint8_t *)(Q + (bh * S + t_lo) * D);
+        for (int i = tid; i < 128 * CH; i += blockDim.x) {
+            const int r = i / CH, c = i % CH;
+            const bool ok = t_lo + r < S;
+            tc::cp_async16(s_q + r * QP + 16 * c, ok ? (const void *)(src + (size_t)r * (D * sizeof(T)) + 16 * c) : Q, ok);
+        }
+    }
+    {
+        const float4 *src = (const float4 *)(cb + (size_t)h * C * D);
+        for (int i4 = tid; i4 < C * D / 4; i4 += blockDim.x) {
+            const float4 f = __ldg(src + i4);
+            const int mc = (4 * i4) / DM, i = (4 * i4) % DM;
+            float *dst = s_cbT + ((mc / C) * DM + i) * C + mc % C;
+            dst[0] = f.x;
+            dst[C] = f.y;
+            dst[2 * C] = f.z;
+            dst[3 * C] = f.w;
+        }
+    }
+    tc::cp_async_wait_all();
+    __syncthreads();
+
+    const int t = t_lo + tid;
+    const T *qrow = (const T *)(s_q + tid * QP);
+    float s[M][C];
+#pragma unroll
+    for (int m = 0; m < M; ++m) {
+        const T *qm[1] = {qrow + m * DM};
+        float sm[1][C];
+        sub_scores_x2<T, DM, C, 1>(qm, s_cbT + m * DM * C, sm);
+#pragma unroll
+        for (int c = 0; c < C; ++c) s[m][c] = sm[0][c];
+    }
+
+    pdl_wait_primary();
+    for (int i = tid; i < nb; i += blockDim.x) {
+        s_addr[i] = post_addr[bh * nb + i];
+        s_ids[i] = post_ids[bh * nb + i];
+    }
+    __syncthreads();
+
+    int n_sel = 0, lt_r = 0, ign = 0;
+    if (t < S) {
+        bool finite = true;
+#pragma unroll
+        for (int m = 0; m < M; ++m)
+#pragma unroll
+            for (int c = 0; c < C; ++c) finite = finite && fabsf(s[m][c]) <= 3.0e38f;
+
+        // lazily ranked codes of each subspace
+        float ov[M][C];
+        int oc[M][C];
+        unsigned taken[M];
+        int ne[M];
+        auto extract = [&](int m) {
+#pragma unroll
+            for (int mm = 0; mm < M; ++mm) {
+                if (mm != m) continue;
+                float best = -INFINITY;
+                int bc = -1;
+#pragma unroll
+                for (int c = 0; c < C; ++c) {
+                    const bool better = !((taken[mm] >> c) & 1u) && (bc < 0 || s[mm][c] > best);
+                    best = better ? s[mm][c] : best;
+                    bc = better ? c : bc;
+                }
+                taken[mm] |= 1u << bc;
+                ov[mm][ne[mm]] = best;
+                oc[mm][ne[mm]] = bc;
+                ++ne[mm];
+            }
+        };
+        auto gscore = [&](unsigned r) {
+            float g = ov[0][r & RMASK];
+#pragma unroll
+            for (int m = 1; m < M; ++m) g = __fadd_rn(g, ov[m][(r >> (RB * m)) & RMASK]);
+            return g;
+        };
+        auto address = [&](unsigned r) {
+            int a = 0;
+#pragma unroll
+            for (int m = 0; m < M; ++m) a = a * C + oc[m][(r >> (RB * m)) & RMASK];
+            return a;
+        };
+
+        int top_a[TP];
+        bool walk = !finite;
+        if (finite) {
+            float G = 0.f;
+#pragma unroll
+            for (int m = 0; m < M; ++m) {
+                float mx = 0.f;
+#pragma unroll
+                for (int c = 0; c < C; ++c) mx = fmaxf(mx, fabsf(s[m][c]));
+                G += mx;
+            }
+            int e2;
+            frexpf(2.f * G + 1e-30f, &e2);
+            const float delta = (float)(M + 1) * ldexpf(1.f, e2 - 24);
+#pragma unroll
+            for (int m = 0; m < M; ++m) {
+                taken[m] = 0u;
+                ne[m] = 0;
+                extract(m);
+            }
+            // heap on the probe order: entry x precedes y when g_x > g_y, or g_x == g_y and a_x < a_y
+            float hv[NHEAP];
+            int ha[NHEAP];
+            unsigned hr[NHEAP];
+            auto first = [](float g1, int a1, float g2, int a2) { return g1 > g2 || (g1 == g2 && a1 < a2); };
+            int hn = 1;
+            hv[0] = gscore(0u);
+            ha[0] = address(0u);
+            hr[0] = 0u;
+            float gT = 0.f;
+            for (int np = 0; np < TP && !walk; ++np) {
+                const float g = hv[0];
+                const int a = ha[0];
+                const unsigned r = hr[0];
+                top_a[np] = a;
+                gT = g;
+                // pop: sift the last entry down from the root
+                --hn;
+                if (hn > 0) {
+                    const float xv = hv[hn];
+                    const int xa = ha[hn];
+                    const unsigned xr = hr[hn];
+                    int i = 0;
+                    while (true) {
+                        int c = 2 * i + 1;
+                        if (c >= hn) break;
+                        if (c + 1 < hn && first(hv[c + 1], ha[c + 1], hv[c], ha[c])) ++c;
+                        if (!first(hv[c], ha[c], xv, xa)) break;
+                        hv[i] = hv[c];
+                        ha[i] = ha[c];
+                        hr[i] = hr[c];
+                        i = c;
+                    }
+                    hv[i] = xv;
+                    ha[i] = xa;
+                    hr[i] = xr;
+                }
+                // children: raise one rank at or after the last nonzero one
+                const int k0 = r == 0u ? 0 : (31 - __clz((int)r)) / RB;
+#pragma unroll
+                for (int k = 0; k < M; ++k) {
+                    if (k < k0) continue;
+                    const int rk = (int)((r >> (RB * k)) & RMASK);
+                    if (rk + 1 >= C) continue;
+                    if (ne[k] == rk + 1) extract(k);
+                    const unsigned cr = r + (1u << (RB * k));
+                    const float cv = gscore(cr);
+                    const int ca = address(cr);
+                    if (cv == g && ca < a) walk = true;  // the child would precede its parent
+                    int i = hn++;
+                    while (i > 0) {
+                        const int pnt = (i - 1) >> 1;
+                        if (!first(cv, ca, hv[pnt], ha[pnt])) break;
+                        hv[i] = hv[pnt];
+                        ha[i] = ha[pnt];
+                        hr[i] = hr[pnt];
+                        i = pnt;
+                    }
+                    hv[i] = cv;
+                    ha[i] = ca;
+                    hr[i] = cr;
+                }
+            }
+            if (!walk && hn > 0 && hv[0] == gT) {
+                // the tie at the T-th probe runs on into unvisited tuples: exact only without absorbed scores
+#pragma unroll
+                for (int m = 0; m < M; ++m)
+                    while (ne[m] < C) extract(m);
+#pragma unroll
+                for (int m = 0; m < M; ++m)
+                    for (int k = 0; k + 1 < C; ++k) {
+                        const float gap = ov[m][k] - ov[m][k + 1];
+                        if (gap > 0.f && gap <= delta) walk = true;
+                    }
+            }
+        }
+        if (walk) {
+            // every address of the grid, in address order
+            log_walk(counters, walk_log, (long long)bh * S + t);
+            float sl[M * C];  // indexable copy of the scores
+#pragma unroll
+            for (int m = 0; m < M; ++m)
+#pragma unroll
+                for (int c = 0; c < C; ++c) sl[m * C + c] = s[m][c];
+            TopT top;
+            top.init(TP);
+            int A = 1;
+#pragma unroll
+            for (int m = 0; m < M; ++m) A *= C;
+            for (int a = 0; a < A; ++a) {
+                int rem = a, code[M];
+#pragma unroll
+                for (int m = M - 1; m >= 0; --m) {
+                    code[m] = rem % C;
+                    rem /= C;
+                }
+                float g = sl[code[0]];
+#pragma unroll
+                for (int m = 1; m < M; ++m) g = __fadd_rn(g, sl[m * C + code[m]]);
+                top.push(g, a);
+            }
+#pragma unroll
+            for (int k = 0; k < TP; ++k) top_a[k] = top.a[k];
+        }
+
+        // union of the probed lists in probe order, causal filter, E cap
+        const int lim = t / Bs - L;
+        int cid[E];
+#pragma unroll
+        for (int e = 0; e < E; ++e) cid[e] = 0;
+        int nc = 0;
+        for (int r = 0; r < TP && nc < E; ++r) {
+            const int a = top_a[r];
+            int lo = 0, hi = nb;  // first entry of address a
+            while (lo < hi) {
+                const int mid = (lo + hi) >> 1;
+                if (s_addr[mid] < a) lo = mid + 1;
+                else hi = mid;
+            }
+            for (int k = lo; k < nb && s_addr[k] == a && k - lo < cap && nc < E; ++k) {
+                const int j = s_ids[k];
+                if (j > lim) break;
+#pragma unroll
+                for (int e = 0; e < E; ++e)
+                    if (e == nc) cid[e] = j;
+                ++nc;
+            }
+        }
+        const int nr = rerank_m2<T, D, E, R>(qrow, kbar + bh * nb * D, cid, nc, forced, sel + (bh * S + t) * R, t,
+                                             bh, S, Bs, L, &ign);
+        n_sel = nr;
+        lt_r = nr < R;
     }
     for (int o = 16; o > 0; o >>= 1) {
         n_sel += __shfl_xor_sync(0xffffffffu, n_sel, o);
@@ -1366,6 +1692,27 @@ cudaError_t launch_queries(const Plan &p, const void *Q, const float *cb, const 
         MONO_M2(float, 64, 8, 4, 5, 2)
     }
 #undef MONO_M2
+#define MONO_BF(TT, DD, MM, CC, TPP, EE, RR)                                                                      \
+    if (c.M == MM && c.d == DD && c.C == CC && c.T == TPP && c.E == EE && c.R == RR) {                          \
+        const size_t smb = probe_bf_smem<TT, DD, MM, CC>(p.nb);                                                  \
+        auto kern = k_probe_bf<TT, DD, MM, CC, TPP, EE, RR>;                                                     \
+        if (smb > 48 * 1024 &&                                                                                   \
+            (e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smb)) != cudaSuccess) \
+            return e;                                                                                            \
+        if ((e = launch_after_lists(kern, g3, smb, s, (const TT *)Q, kbar, cb, ids, saddr, forced, sel, cnt,         \
+                                    walk_log, c.S, c.H, c.Bs, c.L, c.cap)) != cudaSuccess)                          \
+            return e;                                                                                            \
+        count_launches(1);                                                                                       \
+        return cudaGetLastError();                                                                               \
+    }
+    if (bf) {
+        MONO_BF(__nv_bfloat16, 128, 4, 16, 16, 8, 4)
+        MONO_BF(__nv_bfloat16, 64, 4, 16, 16, 5, 2)
+        MONO_BF(__nv_bfloat16, 64, 4, 4, 8, 8, 4)
+    } else {
+        MONO_BF(float, 64, 4, 4, 8, 8, 4)
+    }
+#undef MONO_BF
     const size_t smem = (size_t)c.C * c.d * 4 + (size_t)p.nb * 8;
 #define MONO_LAUNCH_PR(TT, DD)                                                                                     \
     do {                                                                                                           \
