@@ -186,10 +186,14 @@ __device__ __forceinline__ bool timed_out(const unsigned long long *counters) {
 // two-stage pipeline: while item k is computed, the tiles of item k+1 are in
 // flight and the descriptor and pair ids of item k+2 are being loaded.  K_j
 // and V_j arrive by TMA (128-byte swizzle, one thread issues them); the
-// gathered query rows by cp.async.  Per item: S = Q_sel K_j^T and O = P V_j on
-// tcgen05 (TMEM, 64 or 128 columns reused by every item), softmax in fp32,
-// one partial per pair.  As in the local kernel, warps q and q+4 share TMEM
-// lane quarter q and split the columns.
+// gathered query rows by cp.async, eight threads per 128-byte row segment, in
+// the same 128-byte swizzled layout (a ring of the items' pair ids in shared
+// memory tells each thread its rows).  Per item: S = Q_sel K_j^T and
+// O = P V_j on tcgen05 (TMEM, 64 or 128 columns reused by every item),
+// softmax in fp32, one partial per pair: the rows go through shared memory
+// (swizzled) so that every store writes whole 128-byte lines.  As in the
+// local kernel, warps q and q+4 share TMEM lane quarter q and split the
+// columns.
 // ---------------------------------------------------------------------------
 struct RemoteItem {
     long long bh;
@@ -210,7 +214,8 @@ struct RemoteSmem {
     static constexpr int P_OFF = PB <= QB ? -1 : 2 * STAGE;       // -1: P over the stage's Q
     static constexpr int RED_OFF = 2 * STAGE + (PB <= QB ? 0 : PB);  // float [2][128]
     static constexpr int PREF_OFF = RED_OFF + 1024;                // int [kMaxGroup + 1]
-    static constexpr int BAR_OFF = PREF_OFF + ((kMaxGroup + 1) * 4 + 15) / 16 * 16;  // 3 mbarriers + TMEM base
+    static constexpr int PR_OFF = PREF_OFF + ((kMaxGroup + 1) * 4 + 15) / 16 * 16;  // int [3][128] pair-id ring
+    static constexpr int BAR_OFF = PR_OFF + 3 * 128 * 4;           // 3 mbarriers + TMEM base
     static constexpr int BYTES = BAR_OFF + 32;
 };
 
@@ -230,6 +235,7 @@ __global__ void __launch_bounds__(256) k_remote_tc(const __grid_constant__ AttnM
     extern __shared__ __align__(1024) uint8_t smem[];
     float(*s_red)[128] = (float(*)[128])(smem + L::RED_OFF);
     int *s_pref = (int *)(smem + L::PREF_OFF);
+    int(*s_pr)[128] = (int(*)[128])(smem + L::PR_OFF);  // pair ids of item k at s_pr[k % 3]
     uint64_t *bar_kv = (uint64_t *)(smem + L::BAR_OFF);  // [2]: K/V of each stage landed
     uint64_t *mbar = bar_kv + 2;                          // MMA completion
     uint32_t *tmem_base = (uint32_t *)(mbar + 1);
@@ -279,7 +285,11 @@ __global__ void __launch_bounds__(256) k_remote_tc(const __grid_constant__ AttnM
     auto pair_of = [&](const RemoteItem &it) { return row < it.n ? pairs[it.bh * S * R + it.p0 + row] : 0; };
     // the stage's tiles: K_j and V_j by TMA onto bar_kv[stage] (thread 0), the
     // selected query rows by cp.async (every thread, one group)
-    auto issue = [&](int stage, const RemoteItem &it, int pr) {
+    // 16-byte chunk c of row r of a [128, D] bf16 tile in 64-column slabs of
+    // 128-byte rows, chunks swizzled by (r mod 8): the layout of a TMA tile
+    // with 128-byte swizzle
+    auto sw_off = [](int r, int c) { return (uint32_t)((c >> 3) * (128 * 128) + r * 128 + (((c & 7) ^ (r & 7)) << 4)); };
+    auto issue = [&](int stage, const RemoteItem &it, const int *prs) {
         uint8_t *sQ = smem + stage * STAGE, *sK = sQ + QB, *sV = sK + KB;
         if (tid == 0) {
             tc::mbar_expect_tx(&bar_kv[stage], 2 * KB);
@@ -289,10 +299,14 @@ __global__ void __launch_bounds__(256) k_remote_tc(const __grid_constant__ AttnM
                 tc::tma_load_3d(sV + a * (BS * 128), &maps.v, 64 * a, it.j * BS, (int)it.bh, &bar_kv[stage]);
             }
         }
-        const bf16 *qrow = Q + ((size_t)it.bh * S + pr / R) * D;
+        constexpr int CPR = D / 8;  // chunks per row
 #pragma unroll
-        for (int c = half * (D / 16); c < (half + 1) * (D / 16); ++c)
-            tc::cp_async16(sQ + tc::kmajor_chunk(row, c, D), qrow + 8 * c, row < it.n);
+        for (int k = 0; k < 128 * CPR / 256; ++k) {
+            const int idx = tid + 256 * k, r = idx / CPR, c = idx % CPR;
+            const bool live = r < it.n;
+            const bf16 *src = live ? Q + ((size_t)it.bh * S + prs[r] / R) * D + 8 * c : Q;
+            tc::cp_async16(sQ + sw_off(r, c), src, live);
+        }
         asm volatile("cp.async.commit_group;" ::: "memory");
     };
 
@@ -304,18 +318,23 @@ __global__ void __launch_bounds__(256) k_remote_tc(const __grid_constant__ AttnM
     if (f < total) {
         RemoteItem it0 = descr(f);
         int pr0 = pair_of(it0);
-        issue(0, it0, pr0);
-        pend[0] = 0;
         int f1 = f + G;
         bool have1 = f1 < total;
         RemoteItem it1{};
         int pr1 = 0;
         if (have1) { it1 = descr(f1); pr1 = pair_of(it1); }
+        if (half == 0) {
+            s_pr[0][row] = pr0;
+            s_pr[1][row] = pr1;
+        }
+        __syncthreads();
+        issue(0, it0, s_pr[0]);
+        pend[0] = 0;
         for (int k = 0; ok; ++k) {
             const int stage = k & 1;
             const uint32_t kv_parity = (k >> 1) & 1;  // completions of bar_kv[stage] so far, mod 2
             if (have1) {
-                issue(stage ^ 1, it1, pr1);
+                issue(stage ^ 1, it1, s_pr[(k + 1) % 3]);
                 if (stage) pend[0] = ((k + 1) >> 1) & 1;
                 else pend[1] = ((k + 1) >> 1) & 1;
             }
@@ -343,7 +362,7 @@ __global__ void __launch_bounds__(256) k_remote_tc(const __grid_constant__ AttnM
                 const uint32_t aq = tc::smem_u32(sQ), bk = tc::smem_u32(sK);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk)
-                    tc::mma_bf16(tmem, tc::desc_kmajor(aq + 256 * kk, D),
+                    tc::mma_bf16(tmem, tc::desc_sw128(aq + (kk >> 2) * (128 * 128) + (kk & 3) * 32),
                                  tc::desc_sw128(bk + (kk >> 2) * (BS * 128) + (kk & 3) * 32), id, kk > 0);
                 tc::commit(mbar);
             }
@@ -387,6 +406,7 @@ __global__ void __launch_bounds__(256) k_remote_tc(const __grid_constant__ AttnM
             l = s_red[0][row] + s_red[1][row];
             // pair ids of item k+2 (its descriptor load has landed by now), consumed next iteration
             const int pr2 = have2 ? pair_of(it2) : 0;
+            if (half == 0) s_pr[(k + 2) % 3][row] = pr2;
             if (tid == 0 && ok) {
                 const uint32_t id = tc::idesc_bf16(128, D, true);
                 const uint32_t ap = tc::smem_u32(sP), bv = tc::smem_u32(sV);
@@ -399,22 +419,33 @@ __global__ void __launch_bounds__(256) k_remote_tc(const __grid_constant__ AttnM
             ok = __syncthreads_and(ok && tc::mbar_wait(mbar, 1));
             tc::fence_after_sync();
             const bool live = row < it0.n;
-            const size_t slot = (size_t)it0.bh * S * R + pr0;
+            const size_t base = (size_t)it0.bh * S * R;
             const float inv = 1.f / l;
+            // this row's partial, bf16, into shared memory over P (free once the P V MMA has completed)
 #pragma unroll
             for (int c0 = half * DH; c0 < half * DH + DH; c0 += 32) {
                 tc::tmem_ld32(trow + c0, v);
-                if (live && ok) {
-                    uint4 *dst = (uint4 *)(part_o + slot * D + c0);
 #pragma unroll
-                    for (int q8 = 0; q8 < 4; ++q8)
-                        dst[q8] = make_uint4(pack2(v[8 * q8] * inv, v[8 * q8 + 1] * inv),
-                                             pack2(v[8 * q8 + 2] * inv, v[8 * q8 + 3] * inv),
-                                             pack2(v[8 * q8 + 4] * inv, v[8 * q8 + 5] * inv),
-                                             pack2(v[8 * q8 + 6] * inv, v[8 * q8 + 7] * inv));
+                for (int q8 = 0; q8 < 4; ++q8)
+                    *(uint4 *)(sP + sw_off(row, (c0 >> 3) + q8)) =
+                        make_uint4(pack2(v[8 * q8] * inv, v[8 * q8 + 1] * inv),
+                                   pack2(v[8 * q8 + 2] * inv, v[8 * q8 + 3] * inv),
+                                   pack2(v[8 * q8 + 4] * inv, v[8 * q8 + 5] * inv),
+                                   pack2(v[8 * q8 + 6] * inv, v[8 * q8 + 7] * inv));
+            }
+            if (live && ok && half == 0) part_ml[base + pr0] = make_float2(m2, l);
+            __syncthreads();
+            // the rows out, eight threads per 128-byte line of a row
+            if (ok) {
+                constexpr int CPR = D / 8;
+                const int *prs = s_pr[k % 3];
+#pragma unroll
+                for (int kq = 0; kq < 128 * CPR / 256; ++kq) {
+                    const int idx = tid + 256 * kq, r = idx / CPR, c = idx % CPR;
+                    if (r < it0.n)
+                        *(uint4 *)(part_o + (base + prs[r]) * D + 8 * c) = *(const uint4 *)(sP + sw_off(r, c));
                 }
             }
-            if (live && ok && half == 0) part_ml[slot] = make_float2(m2, l);
             tc::fence_before_sync();
             __syncthreads();  // the stage's tiles and TMEM are free again
             tc::fence_after_sync();
