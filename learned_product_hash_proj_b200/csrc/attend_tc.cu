@@ -971,8 +971,8 @@ __global__ void __launch_bounds__(320, 1) k_local_ws(const __grid_constant__ Att
                 ml[r] = part_ml[pq];
                 if (r < kPre) {
 #pragma unroll
-                    for (int q8 = 0; q8 < D / 8; ++q8)
-                        pre[r < kPre ? r : 0][q8] = __ldg((const uint4 *)(part_o + pq * D) + q8);
+                    for (int q8 = 0; q8 < D / 8; q8 += 2)  // 32-byte loads (the rows are 128-byte aligned)
+                        tc::ldg_v8(part_o + pq * D + 8 * q8, pre[r < kPre ? r : 0][q8], pre[r < kPre ? r : 0][q8 + 1]);
                 } else {
                     tc::prefetch_l2(part_o + pq * D);
                 }

@@ -955,17 +955,11 @@ __device__ __forceinline__ int rerank_m2(const T *qp, const float *kb, const int
 #pragma unroll
         for (int e = 0; e < E; ++e) {
             if (e < nc) {
-                const float4 *kr = (const float4 *)(kb + (size_t)cid[e] * D + 8 * i8);
-                const float4 x = __ldg(kr), y = __ldg(kr + 1);
+                float kv[8];  // one 32-byte load (the rows are 32-byte aligned)
+                tc::ldg_v8(kb + (size_t)cid[e] * D + 8 * i8, kv);
                 float a = acc[e];
-                a = __fmaf_rn(qv[0], x.x, a);
-                a = __fmaf_rn(qv[1], x.y, a);
-                a = __fmaf_rn(qv[2], x.z, a);
-                a = __fmaf_rn(qv[3], x.w, a);
-                a = __fmaf_rn(qv[4], y.x, a);
-                a = __fmaf_rn(qv[5], y.y, a);
-                a = __fmaf_rn(qv[6], y.z, a);
-                a = __fmaf_rn(qv[7], y.w, a);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) a = __fmaf_rn(qv[i], kv[i], a);
                 acc[e] = a;
             }
         }
