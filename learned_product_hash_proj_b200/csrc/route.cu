@@ -78,49 +78,80 @@ __global__ void __launch_bounds__(128) k_summary_assign(const T *__restrict__ K,
 // ---------------------------------------------------------------------------
 // (A2, A3) the same summaries with one warp per block: each lane owns D/32
 // adjacent columns and walks the block's rows in ascending t, reading its
-// columns of a row as one 32- or 64-bit word.  A CTA takes 4 x bpw
-// consecutive blocks of one (b, h), each warp bpw of them through a two-deep
-// ring: block q+1's rows stream in (cp.async) while block q is summed.  The
-// head's codebook sits in shared memory, transposed so that lane mc reads
-// codeword mc without bank conflicts.
+// columns of a row as one 32- or 64-bit word straight from global memory (a
+// row per warp load; 16 registers of rows per batch, the next batch in
+// flight while one is summed).  A CTA takes 4 x bpw
+// consecutive blocks of one (b, h), each warp bpw of them; the grid is sized
+// to about one wave of 6 CTAs per SM.  The head's codebook sits in shared
+// memory, transposed so that lane mc reads codeword mc without bank conflicts.
 // grid (ceil(nb / (4 bpw)), H, B), 128 threads.
 // ---------------------------------------------------------------------------
-constexpr int kSumRing = 2;  // staged blocks per warp
-
 inline size_t summary_smem(int M, int C, int Bs, int D, int es) {
-    return ((size_t)M * C * (D / M) + 4 * (size_t)D + 4 * (size_t)M * C) * 4 + 16 +
-           (size_t)4 * kSumRing * Bs * D * es;
+    (void)Bs;
+    (void)es;
+    return ((size_t)M * C * (D / M) + 4 * (size_t)D + 4 * (size_t)M * C) * 4;
 }
 
+template <typename T, int PER>
+struct RowWord;  // this lane's PER columns of one row
+template <>
+struct RowWord<__nv_bfloat16, 2> {
+    using W = uint32_t;
+    static __device__ __forceinline__ void cvt(W w, float (&v)[2]) {
+        const float2 f = __bfloat1622float2(*(const __nv_bfloat162 *)&w);
+        v[0] = f.x; v[1] = f.y;
+    }
+};
+template <>
+struct RowWord<__nv_bfloat16, 4> {
+    using W = uint2;
+    static __device__ __forceinline__ void cvt(W w, float (&v)[4]) {
+        const float2 f0 = __bfloat1622float2(*(const __nv_bfloat162 *)&w.x);
+        const float2 f1 = __bfloat1622float2(*(const __nv_bfloat162 *)&w.y);
+        v[0] = f0.x; v[1] = f0.y; v[2] = f1.x; v[3] = f1.y;
+    }
+};
+template <>
+struct RowWord<float, 2> {
+    using W = float2;
+    static __device__ __forceinline__ void cvt(W w, float (&v)[2]) { v[0] = w.x; v[1] = w.y; }
+};
+template <>
+struct RowWord<float, 4> {
+    using W = float4;
+    static __device__ __forceinline__ void cvt(W w, float (&v)[4]) { v[0] = w.x; v[1] = w.y; v[2] = w.z; v[3] = w.w; }
+};
+
 template <typename T, int D>
-__global__ void __launch_bounds__(128) k_summary_assign_w(const T *__restrict__ K, const float *__restrict__ cb,
+__global__ void __launch_bounds__(128, 6) k_summary_assign_w(const T *__restrict__ K, const float *__restrict__ cb,
                                                           float *__restrict__ kbar, int32_t *__restrict__ addr, int S,
                                                           int Bs, int M, int C, int H, int bpw) {
     constexpr int PER = D / 32;  // columns per lane
     static_assert(PER == 2 || PER == 4, "D = 64 or 128");
+    using RW = RowWord<T, PER>;
+    using W = typename RW::W;
+    constexpr int U = 16 / ((int)sizeof(W) / 4);  // rows per batch: 16 registers of words
     extern __shared__ __align__(16) float sm[];
     const int MC = M * C, dm = D / M;
     float *s_cbT = sm;                              // [dm][M*C]: element i of codeword mc at i * MC + mc
     float *s_kb = s_cbT + MC * dm;                  // [4][D]
     float *s_sc = s_kb + 4 * D;                     // [4][M*C]
-    T *s_rows = (T *)(((uintptr_t)(s_sc + 4 * MC) + 15) & ~(uintptr_t)15);  // [4][kSumRing][Bs*D] staged rows
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int h = blockIdx.y, b = blockIdx.z;
     const int nb = S / Bs;
     const size_t bh = (size_t)b * H + h;
     const int j0 = (blockIdx.x * 4 + warp) * bpw;
-    // block q's rows into ring slot q % 2; one commit group per block (empty past the warp's last block)
-    const int chunks = Bs * D * (int)sizeof(T) / 16;
-    T *rows = s_rows + (size_t)warp * kSumRing * Bs * D;
-    auto prefetch = [&](int q) {
-        if (q < bpw && j0 + q < nb) {
-            const uint8_t *src = (const uint8_t *)(K + (bh * S + (size_t)(j0 + q) * Bs) * D);
-            uint8_t *dst = (uint8_t *)(rows + (size_t)(q % kSumRing) * Bs * D);
-            for (int c = lane; c < chunks; c += 32) tc::cp_async16(dst + 16 * c, src + 16 * c, true);
-        }
-        asm volatile("cp.async.commit_group;" ::: "memory");
+    const int nq = max(0, min(bpw, nb - j0));  // this warp's blocks
+    const int nbt = Bs / U;                     // whole batches per block; Bs % U rows follow them
+    const int total = nq * nbt;
+    auto row_ptr = [&](int q) { return (const W *)(K + (bh * S + (size_t)(j0 + q) * Bs) * D) + lane; };
+    auto load = [&](int k, W (&buf)[U]) {
+        const W *rq = row_ptr(k / nbt) + (size_t)(k % nbt) * U * 32;
+#pragma unroll
+        for (int u = 0; u < U; ++u) buf[u] = __ldg(rq + (size_t)u * 32);
     };
-    prefetch(0);
+    W b0[U], b1[U];
+    if (total > 0) load(0, b0);  // the first rows are in flight while the codebook is staged
     // the head's codebook (C*D floats, [M][C][dm]), transposed, with independent 16-byte loads
     {
         const float4 *src = (const float4 *)(cb + (size_t)h * C * D);
@@ -133,57 +164,38 @@ __global__ void __launch_bounds__(128) k_summary_assign_w(const T *__restrict__ 
             s_cbT[(i + 3) * MC + mc] = f.w;
         }
     }
-    __syncthreads();  // the codebook; block 0 may still be in flight
-    for (int q = 0; q < bpw; ++q) {
+    __syncthreads();
+    float acc[PER];
+#pragma unroll
+    for (int e = 0; e < PER; ++e) acc[e] = 0.0f;
+    // block q after its whole batches: the tail rows, kbar, scores and address; acc is reset for the next block
+    auto finish = [&](int q) {
         const int j = j0 + q;
-        prefetch(q + 1);  // into the slot block q - 1 used (released by the warp barrier ending that step)
-        asm volatile("cp.async.wait_group 1;" ::: "memory");  // block q has landed (this lane's copies)
-        __syncwarp();                                         // ... and every lane's
-        if (j < nb) {
-            const T *rq = rows + (size_t)(q % kSumRing) * Bs * D;
-            float acc[PER];
+        const W *rq = row_ptr(q);
+        for (int t = nbt * U; t < Bs; ++t) {
+            float v[PER];
+            RW::cvt(__ldg(rq + (size_t)t * 32), v);
 #pragma unroll
-            for (int e = 0; e < PER; ++e) acc[e] = 0.0f;
-            for (int t = 0; t < Bs; ++t) {
-                float v[PER];
-                if constexpr (sizeof(T) == 2) {
-                    if constexpr (PER == 2) {
-                        const float2 f = __bfloat1622float2(*(const __nv_bfloat162 *)(rq + (size_t)t * D + 2 * lane));
-                        v[0] = f.x; v[1] = f.y;
-                    } else {
-                        const uint2 u = *(const uint2 *)(rq + (size_t)t * D + 4 * lane);
-                        const float2 f0 = __bfloat1622float2(*(const __nv_bfloat162 *)&u.x);
-                        const float2 f1 = __bfloat1622float2(*(const __nv_bfloat162 *)&u.y);
-                        v[0] = f0.x; v[1] = f0.y; v[2] = f1.x; v[3] = f1.y;
-                    }
-                } else {
+            for (int e = 0; e < PER; ++e) acc[e] = __fadd_rn(acc[e], v[e]);
+        }
 #pragma unroll
-                    for (int e = 0; e < PER; ++e) v[e] = rq[(size_t)t * D + lane * PER + e];
-                }
-#pragma unroll
-                for (int e = 0; e < PER; ++e) acc[e] = __fadd_rn(acc[e], v[e]);
-            }
-#pragma unroll
-            for (int e = 0; e < PER; ++e) {
-                const float v = __fdiv_rn(acc[e], (float)Bs);
-                s_kb[warp * D + lane * PER + e] = v;
-                kbar[(bh * nb + j) * D + lane * PER + e] = v;
-            }
+        for (int e = 0; e < PER; ++e) {
+            const float v = __fdiv_rn(acc[e], (float)Bs);
+            s_kb[warp * D + lane * PER + e] = v;
+            kbar[(bh * nb + j) * D + lane * PER + e] = v;
         }
         __syncwarp();
-        if (j < nb) {
-            for (int mc = lane; mc < MC; mc += 32) {
-                const int m = mc / C;
-                const float *kv = s_kb + warp * D + m * dm;
-                float a = 0.0f;
-                for (int i = 0; i < dm; ++i) a = __fmaf_rn(kv[i], s_cbT[i * MC + mc], a);
-                s_sc[warp * MC + mc] = a;
-            }
+        for (int mc = lane; mc < MC; mc += 32) {
+            const int m = mc / C;
+            const float *kv = s_kb + warp * D + m * dm;
+            float a = 0.0f;
+            for (int i = 0; i < dm; ++i) a = __fmaf_rn(kv[i], s_cbT[i * MC + mc], a);
+            s_sc[warp * MC + mc] = a;
         }
         __syncwarp();
         // one lane per subspace: the first maximum wins (ascending c); lane 0 combines
         int bc = 0;
-        if (j < nb && lane < M) {
+        if (lane < M) {
             const float *sc = s_sc + warp * MC + lane * C;
             float best = sc[0];
             for (int c = 1; c < C; ++c)
@@ -191,8 +203,31 @@ __global__ void __launch_bounds__(128) k_summary_assign_w(const T *__restrict__ 
         }
         long long ad = 0;
         for (int m = 0; m < M; ++m) ad = ad * C + __shfl_sync(0xffffffffu, bc, m);
-        if (j < nb && lane == 0) addr[bh * nb + j] = (int32_t)ad;
+        if (lane == 0) addr[bh * nb + j] = (int32_t)ad;
         __syncwarp();
+#pragma unroll
+        for (int e = 0; e < PER; ++e) acc[e] = 0.0f;
+    };
+    auto consume = [&](int k, const W (&buf)[U]) {
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            float v[PER];
+            RW::cvt(buf[u], v);
+#pragma unroll
+            for (int e = 0; e < PER; ++e) acc[e] = __fadd_rn(acc[e], v[e]);
+        }
+        if (k % nbt == nbt - 1) finish(k / nbt);
+    };
+    if (nbt == 0)  // blocks shorter than one batch
+        for (int q = 0; q < nq; ++q) finish(q);
+    // batches in two register buffers: batch k+1 is in flight while batch k is summed
+    for (int k = 0; k < total; k += 2) {
+        if (k + 1 < total) load(k + 1, b1);
+        consume(k, b0);
+        if (k + 1 < total) {
+            if (k + 2 < total) load(k + 2, b0);
+            consume(k + 1, b1);
+        }
     }
 }
 
@@ -1556,12 +1591,12 @@ cudaError_t launch_summaries(const Plan &p, const void *K, const float *cb, void
     unsigned long long *cnt = (unsigned long long *)ws_ptr(p, ws, kRegCounters);
     cudaError_t e = cudaMemsetAsync(cnt, 0, kCntN * 8, s);
     if (e != cudaSuccess) return e;
-    // blocks per warp: about one wave of 3 CTAs per SM over all blocks; blocks
-    // too large to stage twice per warp take the plain kernel (one CTA per block)
+    // blocks per warp: about one wave of 6 CTAs (24 warps) per SM over all blocks; a codebook too large for
+    // shared memory takes the plain kernel (one CTA per block)
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const long long blocks = (long long)c.B * c.H * p.nb;
-    const int bpw = (int)std::min<long long>(16, std::max<long long>(1, (blocks + 12ll * sms - 1) / (12ll * sms)));
+    const int bpw = (int)std::min<long long>(16, std::max<long long>(1, (blocks + 24ll * sms - 1) / (24ll * sms)));
     const size_t smem = summary_smem(c.M, c.C, c.Bs, c.d, (int)p.es);
     if (smem > 160 * 1024) {
         dim3 g0(p.nb, c.H, c.B);
