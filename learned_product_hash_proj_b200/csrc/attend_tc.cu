@@ -814,6 +814,7 @@ template <int D, int BS, int NK, int RMAX>
 __global__ void __launch_bounds__(320, 1) k_local_ws(const __grid_constant__ AttnMaps maps,
                                                      const int32_t *__restrict__ sel, const bf16 *__restrict__ part_o,
                                                      const float2 *__restrict__ part_ml, bf16 *__restrict__ O,
+                                                     float *__restrict__ o32, float *__restrict__ lse_out,
                                                      unsigned long long *__restrict__ counters, int S, int H, int R,
                                                      int L, float scale_log2, int bh0, int ng) {
     using Lay = LocalWs<D, NK>;
@@ -1053,6 +1054,7 @@ __global__ void __launch_bounds__(320, 1) k_local_ws(const __grid_constant__ Att
                 }
             }
             const float inv = 1.f / den;
+            if (lse_out && live) lse_out[(size_t)bh * S + t] = (mm + log2f(den)) * 0.69314718055994531f;  // ln 2
             if (!__all_sync(0xffffffffu, tc::mbar_wait_or_abort(&o_full[g], u & 1, abort_flag))) { fail(); break; }
             tc::fence_after_sync();
             bf16 *orow = O + (((size_t)b * S + t) * H + h) * D;
@@ -1088,6 +1090,13 @@ __global__ void __launch_bounds__(320, 1) k_local_ws(const __grid_constant__ Att
                                              pack2(v[8 * q8 + 2] * inv, v[8 * q8 + 3] * inv),
                                              pack2(v[8 * q8 + 4] * inv, v[8 * q8 + 5] * inv),
                                              pack2(v[8 * q8 + 6] * inv, v[8 * q8 + 7] * inv));
+                    if (o32) {
+                        float4 *d32 = (float4 *)(o32 + (((size_t)b * S + t) * H + h) * D + c0);
+#pragma unroll
+                        for (int q4 = 0; q4 < 8; ++q4)
+                            d32[q4] = make_float4(v[4 * q4] * inv, v[4 * q4 + 1] * inv, v[4 * q4 + 2] * inv,
+                                                  v[4 * q4 + 3] * inv);
+                    }
                 }
             }
             tc::fence_before_sync();
@@ -1168,7 +1177,7 @@ static cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, siz
 
 template <int D, int BS, int NK, int RMAX>
 static cudaError_t launch_tc_shape(const Plan &p, const bf16 *Q, const bf16 *K, const bf16 *V, const int32_t *sel,
-                                   bf16 *O, void *ws, cudaStream_t s, int parts) {
+                                   bf16 *O, void *ws, cudaStream_t s, int parts, float *o32, float *lse, bool *stats) {
     const mono_config &c = p.cfg;
     unsigned long long *cnt_err = (unsigned long long *)ws_ptr(p, ws, kRegCounters);
     const float scale_log2 = (float)(1.4426950408889634 / sqrt((double)c.d));
@@ -1231,6 +1240,8 @@ static cudaError_t launch_tc_shape(const Plan &p, const bf16 *Q, const bf16 *K, 
             return e;
         if ((e = persistent_grid(kl, 256, smem, &local_ctas)) != cudaSuccess) return e;
     }
+    if (stats) *stats = ws_local && o32 && lse;
+    if (!ws_local) o32 = lse = nullptr;
     // Remote then local, over as many (b, h) slices per launch as the remote
     // kernel's per-group table holds (kMaxGroup).  One launch pair over all
     // slices measured faster than groups sized to keep their partials in L2
@@ -1260,7 +1271,7 @@ static cudaError_t launch_tc_shape(const Plan &p, const bf16 *Q, const bf16 *K, 
             const int tiles = ng * ((c.S + 127) / 128);
             k_local_ws<D, BS, NK, RMAX><<<std::min(local_ctas, tiles), 320, smem, s>>>(
                 lmaps, sel, (const bf16 *)ws_ptr(p, ws, kRegPartO), (const float2 *)ws_ptr(p, ws, kRegPartML), O,
-                cnt_err, c.S, c.H, c.R, c.L, scale_log2, g0, ng);
+                o32, lse, cnt_err, c.S, c.H, c.R, c.L, scale_log2, g0, ng);
         } else {
             kl<<<local_ctas, 256, smem, s>>>(lmaps, sel, (const bf16 *)ws_ptr(p, ws, kRegPartO),
                                              (const float2 *)ws_ptr(p, ws, kRegPartML), O, cnt_err, c.S, c.H, c.R,
@@ -1273,7 +1284,8 @@ static cudaError_t launch_tc_shape(const Plan &p, const bf16 *Q, const bf16 *K, 
 }
 
 cudaError_t launch_attend_tc(const Plan &p, const void *Q, const void *K, const void *V, const int32_t *sel, void *O,
-                             void *ws, cudaStream_t s, int parts) {
+                             void *ws, cudaStream_t s, int parts, float *o32, float *lse, bool *stats) {
+    if (stats) *stats = false;
     const mono_config &c = p.cfg;
     const bf16 *q = (const bf16 *)Q, *k = (const bf16 *)K, *v = (const bf16 *)V;
     bf16 *o = (bf16 *)O;
@@ -1281,9 +1293,9 @@ cudaError_t launch_attend_tc(const Plan &p, const void *Q, const void *K, const 
     // NK = the local key range rounded up to a multiple of 32 (MMA N <= 256)
 #define MONO_TC(DD, BB, NN)                                                                                     \
     do {                                                                                                        \
-        if (c.R <= 2) return launch_tc_shape<DD, BB, NN, 2>(p, q, k, v, sel, o, ws, s, parts);                  \
-        if (c.R <= 4) return launch_tc_shape<DD, BB, NN, 4>(p, q, k, v, sel, o, ws, s, parts);                  \
-        return launch_tc_shape<DD, BB, NN, kMaxR>(p, q, k, v, sel, o, ws, s, parts);                            \
+        if (c.R <= 2) return launch_tc_shape<DD, BB, NN, 2>(p, q, k, v, sel, o, ws, s, parts, o32, lse, stats);                  \
+        if (c.R <= 4) return launch_tc_shape<DD, BB, NN, 4>(p, q, k, v, sel, o, ws, s, parts, o32, lse, stats);                  \
+        return launch_tc_shape<DD, BB, NN, kMaxR>(p, q, k, v, sel, o, ws, s, parts, o32, lse, stats);                            \
     } while (0)
     if (c.d == 64 && c.Bs == 64) {
         if (nk <= 128) MONO_TC(64, 64, 128);

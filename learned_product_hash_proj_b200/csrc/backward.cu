@@ -183,8 +183,9 @@ template <typename T, int DD>
 __global__ void __launch_bounds__(256) k_bwd_dq(const T *__restrict__ Q, const T *__restrict__ K,
                                                 const T *__restrict__ V, const int32_t *__restrict__ sel,
                                                 const float *__restrict__ dO, const GradOut go,
-                                                float *__restrict__ lse_out, float *__restrict__ dsum_out, int B, int H,
-                                                int S, int Bs, int L, int R, float scale) {
+                                                float *__restrict__ lse_out, float *__restrict__ dsum_out,
+                                                const float *__restrict__ o32, int B, int H, int S, int Bs, int L,
+                                                int R, float scale) {
     constexpr int TPQ = DD / kDqE, E = kDqE, U = 2;
     const long long nq = (long long)B * H * S;
     const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
@@ -238,7 +239,18 @@ __global__ void __launch_bounds__(256) k_bwd_dq(const T *__restrict__ Q, const T
         }
     };
 
-    // pass 1: log-sum-exp and O (the first group holds key lo of every query: m is finite after it)
+    // pass 1: log-sum-exp and O (the first group holds key lo of every query: m is finite after it); with the
+    // forward's statistics (o32: O in fp32, lse_out: its log-sum-exp) only D = dO . O
+    float lse, D;
+    if (o32) {
+        float o[E];
+        load16<float>(o32 + (((size_t)b * S + t) * H + h) * DD + e0, o);
+        float dpart = 0.f;
+#pragma unroll
+        for (int e = 0; e < E; ++e) dpart = fmaf(g[e], o[e], dpart);
+        D = group_sum<TPQ>(dpart);
+        lse = lse_out[w];
+    } else {
     float m = -INFINITY, l = 0.f, o[E];
 #pragma unroll
     for (int e = 0; e < E; ++e) o[e] = 0.f;
@@ -275,11 +287,12 @@ __global__ void __launch_bounds__(256) k_bwd_dq(const T *__restrict__ Q, const T
             for (int e = 0; e < E; ++e) o[e] = fmaf(p, vv[e], o[e]);
         }
     });
-    const float lse = m + logf(l);
+    lse = m + logf(l);
     float dpart = 0.f;
 #pragma unroll
     for (int e = 0; e < E; ++e) dpart = fmaf(g[e], o[e] / l, dpart);
-    const float D = group_sum<TPQ>(dpart);
+    D = group_sum<TPQ>(dpart);
+    }
 
     // pass 2: dS and dQ
     float dq[E];
@@ -320,7 +333,7 @@ __global__ void __launch_bounds__(256) k_bwd_dq(const T *__restrict__ Q, const T
         for (int e = 0; e < E; ++e) dq[e] *= scale;
         store_grad16<DD>(go, go.q, true, dq, b, h, t, e0, B, H, S);
         if (e0 == 0) {
-            lse_out[w] = lse;
+            if (!o32) lse_out[w] = lse;
             dsum_out[w] = D;
         }
     }
@@ -611,9 +624,10 @@ cudaError_t gemm_any(int M, int N, int Kd, const TA *A, long long am, long long 
     return cudaGetLastError();
 }
 
+// o32: the forward's O in fp32 (token-major) with its log-sum-exp already in the lse region, or null
 template <typename T>
 cudaError_t attend_backward(const Plan &p, const T *Q, const T *K, const T *V, const int32_t *sel, const float *dO,
-                            const GradOut &go, char *bws, cudaStream_t s) {
+                            const GradOut &go, char *bws, cudaStream_t s, const float *o32 = nullptr) {
     const mono_config &c = p.cfg;
     const BwdLayout L = bwd_layout(p);
     float *lse = (float *)(bws + L.lse), *dsum = (float *)(bws + L.dsum);
@@ -625,9 +639,11 @@ cudaError_t attend_backward(const Plan &p, const T *Q, const T *K, const T *V, c
     const int tpq = c.d / kDqE;
     const unsigned gq = (unsigned)((nq * tpq + 255) / 256);
     if (c.d == 64)
-        k_bwd_dq<T, 64><<<gq, 256, 0, s>>>(Q, K, V, sel, dO, go, lse, dsum, c.B, c.H, c.S, c.Bs, c.L, c.R, scale);
+        k_bwd_dq<T, 64><<<gq, 256, 0, s>>>(Q, K, V, sel, dO, go, lse, dsum, o32, c.B, c.H, c.S, c.Bs, c.L, c.R,
+                                           scale);
     else
-        k_bwd_dq<T, 128><<<gq, 256, 0, s>>>(Q, K, V, sel, dO, go, lse, dsum, c.B, c.H, c.S, c.Bs, c.L, c.R, scale);
+        k_bwd_dq<T, 128><<<gq, 256, 0, s>>>(Q, K, V, sel, dO, go, lse, dsum, o32, c.B, c.H, c.S, c.Bs, c.L, c.R,
+                                            scale);
     count_launches(1);
     if (c.R > 0) {
         const long long n = nq * c.R;
@@ -665,7 +681,8 @@ bool grads_tc_supported(const mono_config &c) {
 template <typename T>
 cudaError_t backward_t(const Plan &p, const T *x, const T *Wq, const T *Wk, const T *Wv, const T *Wo,
                        const int32_t *sel, const T *ddelta, float *dx, float *dWq, float *dWk, float *dWv, float *dWo,
-                       const T *Q, const T *K, const T *V, const T *O, char *bws, void *ws, cudaStream_t s) {
+                       const T *Q, const T *K, const T *V, const T *O, char *bws, void *ws, cudaStream_t s,
+                       const float *o32 = nullptr) {
     const mono_config &c = p.cfg;
     const BwdLayout L = bwd_layout(p);
     unsigned long long *counters = (unsigned long long *)ws_ptr(p, ws, kRegCounters);
@@ -687,7 +704,7 @@ cudaError_t backward_t(const Plan &p, const T *x, const T *Wq, const T *Wk, cons
         float *c0[1] = {dO}, *c1[1] = {dWo};
         if ((e = gemm_grad_tc(BS, Hd, W, 1, 1, a0, false, b0, true, c0, false, counters, s)) != cudaSuccess) return e;
         if ((e = gemm_grad_tc(W, Hd, BS, 1, 1, a0, true, b1, true, c1, false, counters, s)) != cudaSuccess) return e;
-        if ((e = attend_backward<T>(p, Q, K, V, sel, dO, go, bws, s)) != cudaSuccess) return e;
+        if ((e = attend_backward<T>(p, Q, K, V, sel, dO, go, bws, s, o32)) != cudaSuccess) return e;
         // q = x Wq^T (per head, then RoPE):  dWq = dQp^T x (both MN-major),  dx = dQp Wq + dKp Wk + dVp Wv,
         // each dZp as hi + lo
         using B16 = __nv_bfloat16;
@@ -777,15 +794,26 @@ int mono_backward(const mono_plan_t *plan, const void *x, const void *Wq, const 
     void *Q = (char *)workspace + p.off[kRegQ], *K = (char *)workspace + p.off[kRegK];
     void *V = (char *)workspace + p.off[kRegV], *O = (char *)workspace + p.off[kRegO];
     if ((st = mono_project(plan, x, Wq, Wk, Wv, Q, K, V, workspace, stream))) return st;
-    if ((st = mono_attend(plan, Q, K, V, sel, O, workspace, stream))) return st;
     cudaStream_t s = (cudaStream_t)stream;
     char *bws = (char *)bwd_workspace;
+    // the forward attention; where its local kernel can, it also leaves O in fp32 and the log-sum-exp (in the
+    // dK region, free until the dK/dV kernel, and the lse region), so the dQ kernel skips its forward pass
+    const BwdLayout BL = bwd_layout(p);
+    bool stats = false;
+    if (p.fast) {
+        if (cudaError_t e = launch_attend_tc(p, Q, K, V, sel, O, workspace, s, kAttendAll, (float *)(bws + BL.dKp),
+                                             (float *)(bws + BL.lse), &stats))
+            return bwd_status(e);
+    } else if ((st = mono_attend(plan, Q, K, V, sel, O, workspace, stream))) {
+        return st;
+    }
+    const float *o32 = stats ? (const float *)(bws + BL.dKp) : nullptr;
     if (c.dtype == MONO_BF16) {
         using B16 = __nv_bfloat16;
         return bwd_status(backward_t<B16>(p, (const B16 *)x, (const B16 *)Wq, (const B16 *)Wk, (const B16 *)Wv,
                                           (const B16 *)Wo, sel, (const B16 *)ddelta, dx, dWq, dWk, dWv, dWo,
                                           (const B16 *)Q, (const B16 *)K, (const B16 *)V, (const B16 *)O, bws, workspace,
-                                          s));
+                                          s, o32));
     }
     return bwd_status(backward_t<float>(p, (const float *)x, (const float *)Wq, (const float *)Wk, (const float *)Wv,
                                         (const float *)Wo, sel, (const float *)ddelta, dx, dWq, dWk, dWv, dWo,

@@ -139,8 +139,12 @@ cudaError_t gemm_grad_tc(int M, int N, int K, int nsrc, int ngroups, const void 
 int route_static_tables(const Plan &p, void **base, Plan *rp);
 // the stages of the tensor-core attention: pair buckets, remote partials, local part + merge
 enum AttendParts { kAttendPairs = 1, kAttendRemote = 2, kAttendLocal = 4, kAttendAll = 7 };
+// With o32 and lse (backward recompute): the local kernel also writes each row of O in fp32 (token-major like O)
+// and its natural log-sum-exp over the query's keys (scores scaled by 1/sqrt(d)); *stats tells whether the kernel
+// for this shape did.
 cudaError_t launch_attend_tc(const Plan &p, const void *Q, const void *K, const void *V, const int32_t *sel, void *O,
-                             void *ws, cudaStream_t s, int parts = kAttendAll);
+                             void *ws, cudaStream_t s, int parts = kAttendAll, float *o32 = nullptr,
+                             float *lse = nullptr, bool *stats = nullptr);
 
 }  // namespace mono
 
