@@ -282,7 +282,7 @@ def run_ours(args):
     ab = algorithmic_bytes(cfg, npairs=npairs, blocks=nblk)
     single_kernel_stages = {"summaries": "k_summary_assign_w",
                             "lists": "k_posting_dense" if cfg.A <= 4096 else "k_posting_build",
-                            "queries": "k_probe_m2" if cfg.M == 2 else "k_probe_rerank",
+                            "queries": probe_kernel(cfg),
                             "remote": "k_remote_tc", "local": "k_local_ws" if cfg.dtype == "bf16" else "k_attend_simt"}
     dom = max(single_kernel_stages, key=lambda n: stage[n])
     achieved = ab[dom] / (stage[dom] / 1e3) / 1e9
@@ -518,6 +518,18 @@ def measure_backward(plan, cfg, x, Wq, Wk, Wv, Wo, sel, ws, tdt, dev, stream, st
                                         "fp32 lanes x clock (148 x 128 x 2 x 1.965 GHz) for the rest"}}
 
 
+def probe_kernel(cfg) -> str:
+    """The probe kernel the library launches for this shape (its dispatch in csrc/route.cu)."""
+    shape = (cfg.d, cfg.C, cfg.T, cfg.E, cfg.R)
+    if cfg.M == 2 and ((cfg.dtype == "bf16" and shape in ((64, 16, 4, 5, 2), (128, 32, 8, 8, 4))) or
+                       (cfg.dtype != "bf16" and shape in ((64, 16, 4, 5, 2), (64, 8, 4, 5, 2)))):
+        return "k_probe_m2"
+    if cfg.M == 4 and ((cfg.dtype == "bf16" and shape in ((128, 16, 16, 8, 4), (64, 16, 16, 5, 2), (64, 4, 8, 8, 4)))
+                       or (cfg.dtype != "bf16" and shape == (64, 4, 8, 8, 4))):
+        return "k_probe_bf"
+    return "k_probe_rerank"
+
+
 def projection_roofline(cfg, stage: dict) -> dict:
     """Tensor-pipe fraction of the projection GEMMs (outside the route+attend metric): algorithmic flops
     (2 M N K per GEMM: Q/K/V = 3 GEMMs of B*S x H*d x W, the output projection one of B*S x W x H*d) over the
@@ -528,8 +540,9 @@ def projection_roofline(cfg, stage: dict) -> dict:
     for name, st, fl in (("qkv", "project", 3 * gemm), ("out", "out_project", gemm)):
         tf = fl / (stage[st] / 1e3) / 1e12
         out[name] = {"bound": "tensor", "achieved": tf, "peak": tpeak, "unit": "TFLOP/s", "frac": tf / tpeak,
-                     "algorithmic_flops": fl, "ms": stage[st], "kernel": "k_gemm_tc" if cfg.dtype == "bf16"
-                     else "k_gemm_simt"}
+                     "algorithmic_flops": fl, "ms": stage[st],
+                     "kernel": ("k_gemm_tcp" if (cfg.H * cfg.d if name == "qkv" else cfg.W) % 256 == 0 else "k_gemm_tc")
+                     if cfg.dtype == "bf16" else "k_gemm_simt"}
     out["peak_source"] = f"{tsrc} bf16_tflops_sustained (MEASURED_PEAKS.json)"
     if cfg.dtype != "bf16":
         out["note"] = "fp32 storage runs the SIMT GEMM; the bf16 tensor peak is a reference only"

@@ -30,6 +30,9 @@
 #include "mono.h"
 #include "tc.cuh"
 
+#include <cooperative_groups.h>
+namespace cg = cooperative_groups;
+
 namespace mono {
 namespace {
 
@@ -99,6 +102,7 @@ template <typename T>
 __device__ __forceinline__ float row_dot_part(const T *a, const T *b, int n, int lane) {
     constexpr int V = 16 / sizeof(T);
     float acc = 0.f;
+#pragma unroll 4  // the loads of four steps in flight at once
     for (int k = lane * V; k < n; k += 32 * V) {
         const uint4 ua = *(const uint4 *)(a + k), ub = *(const uint4 *)(b + k);
         const T *ta = (const T *)&ua, *tb = (const T *)&ub;
@@ -143,8 +147,9 @@ __global__ void __launch_bounds__(256) k_dec_project(const T *__restrict__ x, co
     }
     for (int b = 0; b < B; ++b) {
         const T *xb = x + (size_t)b * W;
-        const float a0 = warp_sum(row_dot_part(xb, w0, W, lane));
-        const float a1 = warp_sum(row_dot_part(xb, w1, W, lane));
+        const float p0 = row_dot_part(xb, w0, W, lane), p1 = row_dot_part(xb, w1, W, lane);
+        const float a0 = warp_sum(p0);
+        const float a1 = warp_sum(p1);
         if (lane == 0) {
             float r0 = a0, r1 = a1;
             if (which < 2) {
@@ -271,35 +276,43 @@ __device__ __forceinline__ bool before(float v1, int a1, float v2, int a2) {
 
 // ---------------------------------------------------------------------------
 // routing of the step's query, one warp per (b, h); grid (H, B), 32 threads,
-// dynamic shared memory C * d floats (the head's codebooks)
+// dynamic shared memory M C (d/M + 1) floats (the head's codewords, one
+// padding float per row so that the 32 lanes' chains read 32 banks)
 // ---------------------------------------------------------------------------
 template <typename T>
 __global__ void __launch_bounds__(32) k_dec_route(const T *__restrict__ q, const float *__restrict__ cb,
                                                   const int32_t *__restrict__ forced, DecPtrs P, int t, int Bs, int L,
                                                   int R, int E, int M, int C, int TP, int cap, int H, int d, int nb,
                                                   long long A) {
-    extern __shared__ __align__(16) float s_cb[];  // [M][C][dm] of head h
+    extern __shared__ __align__(16) float s_cb[];  // [M][C][dm + 1] of head h
     __shared__ float s_q[kMaxD];
     __shared__ float s_sc[kMaxM * kMaxC];
     __shared__ int s_top[kMaxT];
     __shared__ int s_head[kMaxT], s_cnt[kMaxT];
     __shared__ int s_cand[kMaxE];
     __shared__ float s_score[kMaxE];
-    __shared__ __align__(16) float s_kb[kMaxE > 8 ? 8 : kMaxE][kMaxD];  // candidate kbar rows, 8 at a time
+    __shared__ __align__(16) float s_kb[kMaxE > 8 ? 8 : kMaxE][kMaxD + 4];  // candidate kbar rows, 8 at a time
     const int lane = threadIdx.x;
     const int h = blockIdx.x, b = blockIdx.y;
     const size_t bh = (size_t)b * H + h;
-    for (int i = lane; i < d; i += 32) s_q[i] = to_f(q[bh * d + i]);
+    const int lim = t / Bs - L;  // the latest block a query at t may select
+    // the codewords by asynchronous copies: no lane waits for one load before issuing the next
+    const int dm = d / M;
     {
-        const float4 *src = (const float4 *)(cb + (size_t)h * C * d);
-        for (int i = lane; i < C * d / 4; i += 32) ((float4 *)s_cb)[i] = __ldg(src + i);
+        const float *src = cb + (size_t)h * C * d;
+        for (int i = lane; i < C * d; i += 32)
+            asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(tc::smem_u32(s_cb + (i / dm) * (dm + 1) +
+                                                                                       i % dm)),
+                         "l"(src + i)
+                         : "memory");
     }
+    for (int i = lane; i < d; i += 32) s_q[i] = to_f(q[bh * d + i]);
+    tc::cp_async_wait_all();
     __syncwarp();
     // subspace scores: fma chains in ascending element order from +0
-    const int dm = d / M;
     for (int mc = lane; mc < M * C; mc += 32) {
         const int m = mc / C;
-        const float *w = s_cb + mc * dm;
+        const float *w = s_cb + mc * (dm + 1);
         float a = 0.0f;
         for (int i = 0; i < dm; ++i) a = __fmaf_rn(s_q[m * dm + i], w[i], a);
         s_sc[mc] = a;
@@ -356,7 +369,6 @@ __global__ void __launch_bounds__(32) k_dec_route(const T *__restrict__ q, const
     }
     __syncwarp();
     // union of the probed lists in probe order, causal filter, E cap
-    const int lim = t / Bs - L;
     int nc = 0;
     if (lane == 0) {
         for (int r = 0; r < TP && nc < E; ++r) {
@@ -377,8 +389,10 @@ __global__ void __launch_bounds__(32) k_dec_route(const T *__restrict__ q, const
         const int ne = min(8, nc - e0);
         for (int i = lane; i < ne * d / 4; i += 32) {
             const int e = i / (d / 4), c4 = i % (d / 4);
-            ((float4 *)s_kb[e])[c4] = __ldg((const float4 *)(P.kbar + (bh * nb + s_cand[e0 + e]) * d) + c4);
+            tc::cp_async16((float4 *)s_kb[e] + c4, (const float4 *)(P.kbar + (bh * nb + s_cand[e0 + e]) * d) + c4,
+                           true);
         }
+        tc::cp_async_wait_all();
         __syncwarp();
         if (lane < ne) {
             float a = 0.0f;
@@ -523,6 +537,133 @@ __global__ void __launch_bounds__(256) k_dec_attend(const T *__restrict__ q, con
     }
 }
 
+// ---------------------------------------------------------------------------
+// the same attention split over a cluster of kDecSplit CTAs per (b, h): CTA z
+// of the cluster takes the z-th share of the key list, reduces it as above
+// (chunks through shared memory, 8 warps with online softmaxes, merged in the
+// CTA) to a partial (max, sum, unnormalised o), and CTA 0 merges the shares
+// exactly, reading the others' partials from their shared memory (distributed
+// shared memory of the cluster).  grid (H * kDecSplit, B), cluster
+// (kDecSplit, 1, 1), 256 threads.
+// ---------------------------------------------------------------------------
+constexpr int kDecSplit = 4;
+
+template <typename T>
+__global__ void __launch_bounds__(256) k_dec_attend_cl(const T *__restrict__ q, const T *__restrict__ Kc,
+                                                       const T *__restrict__ Vc, const int32_t *__restrict__ sel,
+                                                       T *__restrict__ O, int t, int S, int Bs, int L, int R, int H,
+                                                       int d, float scale, int CH) {
+    constexpr int kPer = kMaxD / 32, NW = 8;
+    extern __shared__ __align__(16) uint8_t dsm[];  // two buffers of CH keys' K and V rows
+    __shared__ float s_m[NW], s_l[NW];
+    __shared__ float s_acc[NW][kMaxD];
+    __shared__ float s_part[kMaxD + 2];  // this CTA's share: o (unnormalised) [d], max, sum
+    __shared__ int s_js[kMaxR];
+    __shared__ int s_nr;
+    cg::cluster_group cluster = cg::this_cluster();
+    const int z = (int)cluster.block_rank();
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int h = blockIdx.x / kDecSplit, b = blockIdx.y;
+    const size_t bh = (size_t)b * H + h;
+    const int per = d / 32;
+    const int rowb = d * (int)sizeof(T);
+    T *bufK[2] = {(T *)dsm, (T *)(dsm + 2 * CH * rowb)};
+    T *bufV[2] = {(T *)(dsm + CH * rowb), (T *)(dsm + 3 * CH * rowb)};
+    const int bq = t / Bs, lim = bq - L;
+    if (threadIdx.x == 0) {
+        int nr = 0;
+        for (int r = 0; r < R; ++r) {
+            const int j = sel[bh * R + r];
+            if (j >= 0 && j <= lim) s_js[nr++] = j;
+        }
+        s_nr = nr;
+    }
+    __syncthreads();
+    const int nr = s_nr;
+    const int lo = max(0, bq - L + 1) * Bs;
+    const int nkeys = nr * Bs + (t - lo + 1);
+    const int share = (nkeys + kDecSplit - 1) / kDecSplit;
+    const int k_beg = min(nkeys, z * share), k_end = min(nkeys, k_beg + share);
+    auto key_of = [&](int idx) { return idx < nr * Bs ? s_js[idx / Bs] * Bs + idx % Bs : lo + (idx - nr * Bs); };
+    auto stage = [&](int buf, int c0) {
+        const int n = min(CH, k_end - c0), chunks = rowb / 16;
+        for (int i = threadIdx.x; i < n * chunks; i += blockDim.x) {
+            const int k = i / chunks, c = i % chunks;
+            const size_t row = bh * S + key_of(c0 + k);
+            tc::cp_async16((uint8_t *)bufK[buf] + k * rowb + 16 * c, (const uint8_t *)(Kc + row * d) + 16 * c, true);
+            tc::cp_async16((uint8_t *)bufV[buf] + k * rowb + 16 * c, (const uint8_t *)(Vc + row * d) + 16 * c, true);
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+    float qv[kPer];
+    for (int e = 0; e < per; ++e) qv[e] = to_f(q[bh * d + lane * per + e]);
+    float m = -INFINITY, l = 0.f, acc[kPer];
+    for (int e = 0; e < per; ++e) acc[e] = 0.f;
+    if (k_beg < k_end) stage(0, k_beg);
+    for (int c0 = k_beg, cb = 0; c0 < k_end; c0 += CH, cb ^= 1) {
+        if (c0 + CH < k_end) {
+            stage(cb ^ 1, c0 + CH);
+            asm volatile("cp.async.wait_group 1;" ::: "memory");
+        } else {
+            asm volatile("cp.async.wait_group 0;" ::: "memory");
+        }
+        __syncthreads();
+        const int n = min(CH, k_end - c0);
+        for (int k = warp; k < n; k += NW) {
+            const T *kr = bufK[cb] + k * d + lane * per, *vr = bufV[cb] + k * d + lane * per;
+            float part = 0.f;
+            for (int e = 0; e < per; ++e) part = fmaf(qv[e], to_f(kr[e]), part);
+            const float sc = warp_sum(part) * scale;
+            const float mn = fmaxf(m, sc);
+            const float corr = expf(m - mn), p = expf(sc - mn);
+            l = l * corr + p;
+            for (int e = 0; e < per; ++e) acc[e] = fmaf(p, to_f(vr[e]), acc[e] * corr);
+            m = mn;
+        }
+        __syncthreads();
+    }
+    if (lane == 0) {
+        s_m[warp] = m;
+        s_l[warp] = l;
+    }
+    for (int e = 0; e < per; ++e) s_acc[warp][lane * per + e] = acc[e];
+    __syncthreads();
+    if (warp == 0) {  // this CTA's share
+        float mm = -INFINITY;
+        for (int w = 0; w < NW; ++w) mm = fmaxf(mm, s_m[w]);
+        float den = 0.f, o[kPer];
+        for (int e = 0; e < per; ++e) o[e] = 0.f;
+        if (mm != -INFINITY)
+            for (int w = 0; w < NW; ++w) {
+                if (s_m[w] == -INFINITY) continue;  // a warp without keys
+                const float f = expf(s_m[w] - mm);
+                den += s_l[w] * f;
+                for (int e = 0; e < per; ++e) o[e] += s_acc[w][lane * per + e] * f;
+            }
+        for (int e = 0; e < per; ++e) s_part[lane * per + e] = o[e];
+        if (lane == 0) {
+            s_part[d] = mm;
+            s_part[d + 1] = den;
+        }
+    }
+    cluster.sync();  // every share is in its CTA's shared memory
+    if (z == 0 && warp == 0) {
+        float mm = -INFINITY;
+        for (int r = 0; r < kDecSplit; ++r) mm = fmaxf(mm, cluster.map_shared_rank(s_part, r)[d]);
+        float den = 0.f, o[kPer];
+        for (int e = 0; e < per; ++e) o[e] = 0.f;
+        for (int r = 0; r < kDecSplit; ++r) {
+            const float *pr = cluster.map_shared_rank(s_part, r);
+            if (pr[d] == -INFINITY) continue;  // a share without keys
+            const float f = expf(pr[d] - mm);
+            den += pr[d + 1] * f;
+            for (int e = 0; e < per; ++e) o[e] += pr[lane * per + e] * f;
+        }
+        for (int e = 0; e < per; ++e) O[(size_t)b * H * d + (size_t)h * d + lane * per + e] = from_f<T>(o[e] / den);
+    }
+    cluster.sync();  // the shares stay readable until CTA 0 has merged them
+}
+
 // delta_t [B, W] = o [B, H d] Wo^T (Wo [W, H d]); one warp per output column
 template <typename T>
 __global__ void __launch_bounds__(256) k_dec_out(const T *__restrict__ o, const T *__restrict__ Wo,
@@ -661,7 +802,7 @@ int mono_decode_route(const mono_plan_t *plan, int t, const float *codebooks, co
         count_launches(1);
     }
     if (c.R > 0) {
-        const size_t sm = (size_t)c.C * c.d * 4;
+        const size_t sm = (size_t)c.M * c.C * (c.d / c.M + 1) * 4;
         cudaError_t e;
         if (bf) {
             if (sm > 48 * 1024 && (e = cudaFuncSetAttribute(k_dec_route<__nv_bfloat16>,
@@ -695,13 +836,29 @@ int mono_decode_attend(const mono_plan_t *plan, int t, void *cache, void *stream
     cudaStream_t s = (cudaStream_t)stream;
     cudaError_t e;
     if (c.dtype == MONO_BF16) {
-        const size_t sm = (size_t)4 * dec_chunk<__nv_bfloat16>(c.d) * c.d * 2;
-        if ((e = cudaFuncSetAttribute(k_dec_attend<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      (int)sm)))
+        // a CTA's share of at most R + L blocks of keys, in one chunk where it fits
+        const int share = ((c.R + c.L) * c.Bs + kDecSplit - 1) / kDecSplit;
+        const int ch = std::min(dec_chunk<__nv_bfloat16>(c.d), share);
+        const size_t smc = (size_t)4 * ch * c.d * 2;
+        if (smc > 48 * 1024 && (e = cudaFuncSetAttribute(k_dec_attend_cl<__nv_bfloat16>,
+                                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smc)))
             return dec_status(e);
-        k_dec_attend<__nv_bfloat16><<<g, 256, sm, s>>>((const __nv_bfloat16 *)P.Q, (const __nv_bfloat16 *)P.K,
-                                                       (const __nv_bfloat16 *)P.V, P.sel, (__nv_bfloat16 *)P.O, t, c.S,
-                                                       c.Bs, c.L, c.R, c.H, c.d, scale);
+        cudaLaunchConfig_t lc = {};
+        lc.gridDim = dim3(c.H * kDecSplit, c.B);
+        lc.blockDim = dim3(256);
+        lc.dynamicSmemBytes = smc;
+        lc.stream = s;
+        cudaLaunchAttribute at[1];
+        at[0].id = cudaLaunchAttributeClusterDimension;
+        at[0].val.clusterDim.x = kDecSplit;
+        at[0].val.clusterDim.y = 1;
+        at[0].val.clusterDim.z = 1;
+        lc.attrs = at;
+        lc.numAttrs = 1;
+        if ((e = cudaLaunchKernelEx(&lc, k_dec_attend_cl<__nv_bfloat16>, (const __nv_bfloat16 *)P.Q,
+                                    (const __nv_bfloat16 *)P.K, (const __nv_bfloat16 *)P.V, (const int32_t *)P.sel,
+                                    (__nv_bfloat16 *)P.O, t, c.S, c.Bs, c.L, c.R, c.H, c.d, scale, ch)))
+            return dec_status(e);
     } else {
         const size_t sm = (size_t)4 * dec_chunk<float>(c.d) * c.d * 4;
         if ((e = cudaFuncSetAttribute(k_dec_attend<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm)))
