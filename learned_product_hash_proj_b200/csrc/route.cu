@@ -1264,9 +1264,11 @@ __global__ void __launch_bounds__(128, C <= 16 ? 4 : 3) k_probe_m2(const T *__re
 // g(r) = fl(..fl(v_0[r_0] + v_1[r_1]) .. + v_{M-1}[r_{M-1}]), which does not
 // increase when any r_m grows (fp32 addition is monotone in each operand).
 // The tuples form a tree in which the parent of r lowers its last nonzero
-// rank by one.  A heap pops the frontier's first tuple under the probe order
-// (g desc, address asc); the first T pops are the probes provided that no
-// tuple precedes its parent in that order.  A child with a lower g follows
+// rank by one.  The frontier, kept sorted in registers, gives up its first
+// tuple under the probe order (g desc, address asc) T times; the first T pops
+// are the probes provided that no tuple precedes its parent in that order.
+// Only the first T frontier entries are kept: one that ranks below T others
+// can never be popped.  A child with a lower g follows
 // its parent; one with an equal g follows it when the raised rank's code is
 // higher, which a tie of the two scores guarantees (ranks order tied codes
 // ascending).  An equal g from unequal scores (the smaller one absorbed by
@@ -1283,10 +1285,6 @@ template <int C>
 constexpr int rank_bits() {
     return C <= 2 ? 1 : C <= 4 ? 2 : C <= 8 ? 3 : C <= 16 ? 4 : 5;
 }
-template <int M, int TP>
-constexpr int bf_heap() {  // each pop removes one tuple and pushes at most M children
-    return 1 + TP * (M - 1);
-}
 template <typename T, int D, int M, int C>
 constexpr size_t probe_bf_smem(int nb) {
     return (size_t)C * D * 4 + (size_t)128 * probe_q_pitch<T, D>() + (size_t)nb * 8;
@@ -1302,8 +1300,8 @@ __global__ void __launch_bounds__(128) k_probe_bf(const T *__restrict__ Q, const
                                                   int cap) {
     constexpr int DM = D / M, QP = probe_q_pitch<T, D>(), RB = rank_bits<C>();
     constexpr unsigned RMASK = (1u << RB) - 1u;
-    constexpr int NHEAP = bf_heap<M, TP>();
-    static_assert(M >= 2 && M * RB <= 32 && C <= 32 && C % 4 == 0 && DM % 8 == 0 && TP >= 1 && R >= 1, "shape");
+    static_assert(M >= 2 && M * RB <= 16 && C <= 16 && C % 4 == 0 && DM % 8 == 0 && TP >= 1 && R >= 1, "shape");
+    static_assert(M * rank_bits<C>() <= 16 && (C == 16 ? M <= 4 : true), "ranks and address in 16 bits each");
     extern __shared__ __align__(16) float smem[];
     pdl_launch_dependents();
     const int nb = S / Bs;
@@ -1368,7 +1366,7 @@ __global__ void __launch_bounds__(128) k_probe_bf(const T *__restrict__ Q, const
 
         // lazily ranked codes of each subspace
         float ov[M][C];
-        int oc[M][C];
+        uint8_t oc[M][C];
         unsigned taken[M];
         int ne[M];
         auto extract = [&](int m) {
@@ -1385,7 +1383,7 @@ __global__ void __launch_bounds__(128) k_probe_bf(const T *__restrict__ Q, const
                 }
                 taken[mm] |= 1u << bc;
                 ov[mm][ne[mm]] = best;
-                oc[mm][ne[mm]] = bc;
+                oc[mm][ne[mm]] = (uint8_t)bc;
                 ++ne[mm];
             }
         };
@@ -1422,43 +1420,36 @@ __global__ void __launch_bounds__(128) k_probe_bf(const T *__restrict__ Q, const
                 ne[m] = 0;
                 extract(m);
             }
-            // heap on the probe order: entry x precedes y when g_x > g_y, or g_x == g_y and a_x < a_y
-            float hv[NHEAP];
-            int ha[NHEAP];
-            unsigned hr[NHEAP];
-            auto first = [](float g1, int a1, float g2, int a2) { return g1 > g2 || (g1 == g2 && a1 < a2); };
-            int hn = 1;
-            hv[0] = gscore(0u);
-            ha[0] = address(0u);
-            hr[0] = 0u;
+            // the frontier in registers, sorted in the probe order (entry x precedes y when g_x > g_y, or
+            // g_x == g_y and a_x < a_y), keyed by (a << 16) | r; only TP entries are kept: one that ranks below TP
+            // others can never be among the TP pops
+            float fg[TP];
+            unsigned fk[TP];
+            auto first = [](float g1, unsigned k1, float g2, unsigned k2) {
+                return g1 > g2 || (g1 == g2 && (k1 >> 16) < (k2 >> 16));
+            };
+#pragma unroll
+            for (int i = 0; i < TP; ++i) {
+                fg[i] = -INFINITY;
+                fk[i] = 0xffffffffu;
+            }
+            fg[0] = gscore(0u);
+            fk[0] = ((unsigned)address(0u) << 16);
             float gT = 0.f;
             for (int np = 0; np < TP && !walk; ++np) {
-                const float g = hv[0];
-                const int a = ha[0];
-                const unsigned r = hr[0];
+                const float g = fg[0];
+                const unsigned key = fk[0];
+                const unsigned r = key & 0xffffu;
+                const int a = (int)(key >> 16);
                 top_a[np] = a;
                 gT = g;
-                // pop: sift the last entry down from the root
-                --hn;
-                if (hn > 0) {
-                    const float xv = hv[hn];
-                    const int xa = ha[hn];
-                    const unsigned xr = hr[hn];
-                    int i = 0;
-                    while (true) {
-                        int c = 2 * i + 1;
-                        if (c >= hn) break;
-                        if (c + 1 < hn && first(hv[c + 1], ha[c + 1], hv[c], ha[c])) ++c;
-                        if (!first(hv[c], ha[c], xv, xa)) break;
-                        hv[i] = hv[c];
-                        ha[i] = ha[c];
-                        hr[i] = hr[c];
-                        i = c;
-                    }
-                    hv[i] = xv;
-                    ha[i] = xa;
-                    hr[i] = xr;
+#pragma unroll
+                for (int i = 0; i + 1 < TP; ++i) {
+                    fg[i] = fg[i + 1];
+                    fk[i] = fk[i + 1];
                 }
+                fg[TP - 1] = -INFINITY;
+                fk[TP - 1] = 0xffffffffu;
                 // children: raise one rank at or after the last nonzero one
                 const int k0 = r == 0u ? 0 : (31 - __clz((int)r)) / RB;
 #pragma unroll
@@ -1471,21 +1462,20 @@ __global__ void __launch_bounds__(128) k_probe_bf(const T *__restrict__ Q, const
                     const float cv = gscore(cr);
                     const int ca = address(cr);
                     if (cv == g && ca < a) walk = true;  // the child would precede its parent
-                    int i = hn++;
-                    while (i > 0) {
-                        const int pnt = (i - 1) >> 1;
-                        if (!first(cv, ca, hv[pnt], ha[pnt])) break;
-                        hv[i] = hv[pnt];
-                        ha[i] = ha[pnt];
-                        hr[i] = hr[pnt];
-                        i = pnt;
+                    const unsigned ck = ((unsigned)ca << 16) | cr;
+                    // insert: entries from the first one the child precedes move down by one
+#pragma unroll
+                    for (int i = TP - 1; i >= 0; --i) {
+                        const bool here = first(cv, ck, fg[i], fk[i]);
+                        const bool above = i > 0 && first(cv, ck, fg[i > 0 ? i - 1 : 0], fk[i > 0 ? i - 1 : 0]);
+                        if (here) {
+                            fg[i] = above ? fg[i > 0 ? i - 1 : 0] : cv;
+                            fk[i] = above ? fk[i > 0 ? i - 1 : 0] : ck;
+                        }
                     }
-                    hv[i] = cv;
-                    ha[i] = ca;
-                    hr[i] = cr;
                 }
             }
-            if (!walk && hn > 0 && hv[0] == gT) {
+            if (!walk && fg[0] == gT) {  // (an empty slot holds -inf; every score is finite here)
                 // the tie at the T-th probe runs on into unvisited tuples: exact only without absorbed scores
 #pragma unroll
                 for (int m = 0; m < M; ++m)
