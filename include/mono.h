@@ -186,8 +186,11 @@ int mono_route(const mono_plan_t *plan, const void *Q, const void *K, const floa
  *                          resets the routing statistics.
  *  - mono_route_queries:   probe, union, causal filter, E cap, rerank -> sel
  *                          (needs Q); also resets and fills the statistics.
- * Inside mono_route the probe is launched so that it may start while the
- * lists kernel still runs; it waits for the lists before reading them.
+ * The lists kernel is launched so that it may start while the summaries
+ * kernel before it on the stream still runs, and the probe so that it may
+ * start while the lists kernel runs (programmatic dependent launch): each
+ * waits for its predecessor before reading what that one writes, so the
+ * probe loads its queries and scores the codebooks meanwhile.
  * mono_route_summaries resets the device error word. */
 int mono_route_summaries(const mono_plan_t *plan, const void *K, const float *codebooks, void *workspace,
                          void *stream);

@@ -389,8 +389,8 @@ __global__ void __launch_bounds__(256) k_remote_tc(const __grid_constant__ AttnM
                     uint32_t pk[4];
 #pragma unroll
                     for (int u = 0; u < 4; ++u) {
-                        const float a = exp2f(fmaf(v[8 * q8 + 2 * u], scale_log2, -m2));
-                        const float bb = exp2f(fmaf(v[8 * q8 + 2 * u + 1], scale_log2, -m2));
+                        const float a = tc::ex2_fast(fmaf(v[8 * q8 + 2 * u], scale_log2, -m2));
+                        const float bb = tc::ex2_fast(fmaf(v[8 * q8 + 2 * u + 1], scale_log2, -m2));
                         l += a + bb;
                         pk[u] = pack2(a, bb);
                     }
@@ -675,8 +675,8 @@ __global__ void __launch_bounds__(256) k_local_merge_tc(const __grid_constant__ 
 #pragma unroll
                 for (int u = 0; u < 16; ++u) {
                     const int i = 2 * u;
-                    float a = exp2f(fmaf(v[i], scale_log2, -m2));
-                    float bb = exp2f(fmaf(v[i + 1], scale_log2, -m2));
+                    float a = tc::ex2_fast(fmaf(v[i], scale_log2, -m2));
+                    float bb = tc::ex2_fast(fmaf(v[i + 1], scale_log2, -m2));
                     if (!full) {
                         a = (c0 + i >= vlo && c0 + i <= vhi) ? a : 0.f;
                         bb = (c0 + i + 1 >= vlo && c0 + i + 1 <= vhi) ? bb : 0.f;
@@ -1017,8 +1017,8 @@ __global__ void __launch_bounds__(320, 1) k_local_ws(const __grid_constant__ Att
                     const bool full_chunk = c0 >= vlo && c0 + 31 <= vhi;
 #pragma unroll
                     for (int k = 0; k < 16; ++k) {
-                        float a = exp2f(fmaf(v[2 * k], scale_log2, -m2));
-                        float bb = exp2f(fmaf(v[2 * k + 1], scale_log2, -m2));
+                        float a = tc::ex2_fast(fmaf(v[2 * k], scale_log2, -m2));
+                        float bb = tc::ex2_fast(fmaf(v[2 * k + 1], scale_log2, -m2));
                         if (!full_chunk) {
                             a = (c0 + 2 * k >= vlo && c0 + 2 * k <= vhi) ? a : 0.f;
                             bb = (c0 + 2 * k + 1 >= vlo && c0 + 2 * k + 1 <= vhi) ? bb : 0.f;

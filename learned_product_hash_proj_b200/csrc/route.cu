@@ -128,6 +128,7 @@ __global__ void __launch_bounds__(128, 6) k_summary_assign_w(const T *__restrict
                                                           int Bs, int M, int C, int H, int bpw) {
     constexpr int PER = D / 32;  // columns per lane
     static_assert(PER == 2 || PER == 4, "D = 64 or 128");
+    pdl_launch_dependents();  // the lists kernel may start; it waits for the addresses itself
     using RW = RowWord<T, PER>;
     using W = typename RW::W;
     constexpr int U = 16 / ((int)sizeof(W) / 4);  // rows per batch: 16 registers of words
@@ -244,8 +245,11 @@ constexpr int kDenseA = 4096;
 
 __global__ void __launch_bounds__(1024) k_posting_dense(const int32_t *__restrict__ addr, int32_t *__restrict__ ids,
                                                         int32_t *__restrict__ saddr, int32_t *__restrict__ rank,
-                                                        int32_t *__restrict__ overflow, int nb, int cap, int H, int A) {
+                                                        int32_t *__restrict__ overflow, int nb, int cap, int H, int A,
+                                                        unsigned long long *__restrict__ stats) {
     pdl_launch_dependents();
+    pdl_wait_primary();  // the addresses (summaries kernel) are complete
+    if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x < kCntStats) stats[threadIdx.x] = 0ull;  // the probe's
     __shared__ int s_cnt[kDenseA];
     __shared__ int s_part[32];
     __shared__ int s_ov[32];
@@ -334,8 +338,11 @@ __global__ void __launch_bounds__(1024) k_posting_dense(const int32_t *__restric
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(1024) k_posting_build(const int32_t *__restrict__ addr, int32_t *__restrict__ ids,
                                                         int32_t *__restrict__ saddr, int32_t *__restrict__ rank,
-                                                        int32_t *__restrict__ overflow, int nb, int cap, int H) {
+                                                        int32_t *__restrict__ overflow, int nb, int cap, int H,
+                                                        unsigned long long *__restrict__ stats) {
     pdl_launch_dependents();
+    pdl_wait_primary();  // the addresses (summaries kernel) are complete
+    if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x < kCntStats) stats[threadIdx.x] = 0ull;  // the probe's
     extern __shared__ int32_t s_addr[];
     __shared__ int s_ov[32];
     const size_t bh = (size_t)blockIdx.y * H + blockIdx.x;
@@ -408,8 +415,10 @@ __device__ __forceinline__ int first_free(const uint32_t *s_full, int p0, int p1
 __global__ void __launch_bounds__(1024) k_posting_redirect(const int32_t *__restrict__ addr, int32_t *__restrict__ ids,
                                                            int32_t *__restrict__ saddr, int32_t *__restrict__ rank,
                                                            int32_t *__restrict__ overflow, int nb, int cap, int H,
-                                                           int A) {
+                                                           int A, unsigned long long *__restrict__ stats) {
     pdl_launch_dependents();
+    pdl_wait_primary();  // the addresses (summaries kernel) are complete
+    if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x < kCntStats) stats[threadIdx.x] = 0ull;  // the probe's
     extern __shared__ uint32_t s_red[];
     const int nw = (A + 31) / 32;
     uint32_t *s_full = s_red;                          // [nw]: bit set = list full (and every bit past A)
@@ -1287,7 +1296,7 @@ constexpr int rank_bits() {
 }
 template <typename T, int D, int M, int C>
 constexpr size_t probe_bf_smem(int nb) {
-    return (size_t)C * D * 4 + (size_t)128 * probe_q_pitch<T, D>() + (size_t)nb * 8;
+    return (size_t)C * D * 4 + (size_t)128 * probe_q_pitch<T, D>() + (size_t)nb * 8 + 4 * (M * C + kMaxT) * 4;
 }
 
 template <typename T, int D, int M, int C, int TP, int E, int R>
@@ -1309,9 +1318,11 @@ __global__ void __launch_bounds__(128) k_probe_bf(const T *__restrict__ Q, const
     uint8_t *s_q = (uint8_t *)(s_cbT + C * D);           // [128] query rows, pitch QP
     int32_t *s_addr = (int32_t *)(s_q + 128 * QP);       // [nb]
     int32_t *s_ids = s_addr + nb;                        // [nb]
+    float *s_wsc = (float *)(s_ids + nb);                // [4][M*C] scores of the query a warp walks
+    int *s_wtop = (int *)(s_wsc + 4 * M * C);            // [4][TP] its probes
     const int h = blockIdx.y, b = blockIdx.z;
     const size_t bh = (size_t)b * H + h;
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int t_lo = blockIdx.x * 128;
     {
         constexpr int CH = D * (int)sizeof(T) / 16;
@@ -1357,8 +1368,9 @@ __global__ void __launch_bounds__(128) k_probe_bf(const T *__restrict__ Q, const
     __syncthreads();
 
     int n_sel = 0, lt_r = 0, ign = 0;
+    int top_a[TP];
+    bool walk = false, finite = true;
     if (t < S) {
-        bool finite = true;
 #pragma unroll
         for (int m = 0; m < M; ++m)
 #pragma unroll
@@ -1400,8 +1412,7 @@ __global__ void __launch_bounds__(128) k_probe_bf(const T *__restrict__ Q, const
             return a;
         };
 
-        int top_a[TP];
-        bool walk = !finite;
+        walk = !finite;
         if (finite) {
             float G = 0.f;
 #pragma unroll
@@ -1488,8 +1499,9 @@ __global__ void __launch_bounds__(128) k_probe_bf(const T *__restrict__ Q, const
                     }
             }
         }
-        if (walk) {
-            // every address of the grid, in address order
+        if (walk && !finite) {
+            // every address of the grid, in address order (non-finite scores: the sequential order of pushes
+            // decides, as in the general kernel)
             log_walk(counters, walk_log, (long long)bh * S + t);
             float sl[M * C];  // indexable copy of the scores
 #pragma unroll
@@ -1517,6 +1529,67 @@ __global__ void __launch_bounds__(128) k_probe_bf(const T *__restrict__ Q, const
             for (int k = 0; k < TP; ++k) top_a[k] = top.a[k];
         }
 
+    }
+    // queries whose best-first walk could not certify its probes (finite scores): the whole grid, scored by the
+    // warp together (lane l takes the addresses l, l + 32, ...; each keeps its own top TP; TP rounds of a warp
+    // argmax merge them).  For finite scores the probe order is a strict total order, so this equals the
+    // sequential walk.
+    {
+        unsigned wm = __ballot_sync(0xffffffffu, t < S && walk && finite);
+        float *wsc = s_wsc + warp * M * C;
+        int *wtop = s_wtop + warp * TP;
+        while (wm) {
+            const int src = __ffs(wm) - 1;
+            wm &= wm - 1;
+            if (lane == src) {
+                log_walk(counters, walk_log, (long long)bh * S + t);
+#pragma unroll
+                for (int m = 0; m < M; ++m)
+#pragma unroll
+                    for (int c = 0; c < C; ++c) wsc[m * C + c] = s[m][c];
+            }
+            __syncwarp();
+            TopT top;
+            top.init(TP);
+            int A = 1;
+#pragma unroll
+            for (int m = 0; m < M; ++m) A *= C;
+            for (int a = lane; a < A; a += 32) {
+                int rem = a, code[M];
+#pragma unroll
+                for (int m = M - 1; m >= 0; --m) {
+                    code[m] = rem % C;
+                    rem /= C;
+                }
+                float g = wsc[code[0]];
+#pragma unroll
+                for (int m = 1; m < M; ++m) g = __fadd_rn(g, wsc[m * C + code[m]]);
+                top.push(g, a);
+            }
+            int ptr = 0;
+            for (int r = 0; r < TP; ++r) {
+                float bv = ptr < top.n ? top.v[ptr] : -INFINITY;
+                int ba = ptr < top.n ? top.a[ptr] : 0x7fffffff;
+                int bl = lane;
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) {
+                    const float ov2 = __shfl_xor_sync(0xffffffffu, bv, o);
+                    const int oa = __shfl_xor_sync(0xffffffffu, ba, o);
+                    const int ol = __shfl_xor_sync(0xffffffffu, bl, o);
+                    if (TopT::before(ov2, oa, bv, ba)) { bv = ov2; ba = oa; bl = ol; }
+                }
+                if (lane == 0) wtop[r] = ba;
+                if (lane == bl) ++ptr;
+            }
+            __syncwarp();
+            if (lane == src) {
+#pragma unroll
+                for (int k = 0; k < TP; ++k) top_a[k] = wtop[k];
+            }
+            __syncwarp();
+        }
+    }
+    if (t < S) {
         // union of the probed lists in probe order, causal filter, E cap
         const int lim = t / Bs - L;
         int cid[E];
@@ -1602,10 +1675,29 @@ cudaError_t launch_summaries(const Plan &p, const void *K, const float *cb, void
     return cudaGetLastError();
 }
 
+// a kernel launched so that it may start while the kernel before it on the
+// stream still runs (it waits for that kernel itself: griddepcontrol.wait)
+template <typename... KArgs, typename... Args>
+static cudaError_t launch_pdl_k(void (*kern)(KArgs...), dim3 grid, int block, size_t smem, cudaStream_t s,
+                                Args... args) {
+    cudaLaunchConfig_t lc = {};
+    lc.gridDim = grid;
+    lc.blockDim = dim3(block);
+    lc.dynamicSmemBytes = smem;
+    lc.stream = s;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    lc.attrs = at;
+    lc.numAttrs = 1;
+    return cudaLaunchKernelEx(&lc, kern, (KArgs)args...);
+}
+
 cudaError_t launch_lists(const Plan &p, void *ws, cudaStream_t s) {
     const mono_config &c = p.cfg;
-    // the statistics the probe fills (so that the probe can follow this kernel directly)
-    if (cudaError_t e0 = cudaMemsetAsync(ws_ptr(p, ws, kRegCounters), 0, kCntStats * 8, s)) return e0;
+    // the kernel clears the statistics the probe fills (so that the probe can follow it directly), and is
+    // launched programmatically after the summaries: it may start while they run and waits for them itself
+    unsigned long long *stats = (unsigned long long *)ws_ptr(p, ws, kRegCounters);
     dim3 g2(c.H, c.B);
     const int32_t *addr = (const int32_t *)ws_ptr(p, ws, kRegAddr);
     int32_t *ids = (int32_t *)ws_ptr(p, ws, kRegPostIds), *saddr = (int32_t *)ws_ptr(p, ws, kRegPostAddr);
@@ -1619,22 +1711,25 @@ cudaError_t launch_lists(const Plan &p, void *ws, cudaStream_t s) {
             (e = cudaFuncSetAttribute(k_posting_redirect, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn)) !=
                 cudaSuccess)
             return e;
-        k_posting_redirect<<<g2, 1024, dyn, s>>>(addr, ids, saddr, rank, ov, p.nb, c.cap, c.H, (int)p.A);
+        e = launch_pdl_k(k_posting_redirect, g2, 1024, dyn, s, addr, ids, saddr, rank, ov, p.nb, c.cap, c.H,
+                         (int)p.A, stats);
     } else if (p.A <= kDenseA) {
         const size_t dyn = (size_t)p.nb * 8;
         if (dyn + sizeof(int) * (kDenseA + 64) > 48 * 1024 &&
             (e = cudaFuncSetAttribute(k_posting_dense, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn)) !=
                 cudaSuccess)
             return e;
-        k_posting_dense<<<g2, 1024, dyn, s>>>(addr, ids, saddr, rank, ov, p.nb, c.cap, c.H, (int)p.A);
+        e = launch_pdl_k(k_posting_dense, g2, 1024, dyn, s, addr, ids, saddr, rank, ov, p.nb, c.cap, c.H, (int)p.A,
+                         stats);
     } else {
         const size_t dyn = (size_t)p.nb * sizeof(int32_t);
         if (dyn + sizeof(int) * 32 > 48 * 1024 &&
             (e = cudaFuncSetAttribute(k_posting_build, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn)) !=
                 cudaSuccess)
             return e;
-        k_posting_build<<<g2, 1024, dyn, s>>>(addr, ids, saddr, rank, ov, p.nb, c.cap, c.H);
+        e = launch_pdl_k(k_posting_build, g2, 1024, dyn, s, addr, ids, saddr, rank, ov, p.nb, c.cap, c.H, stats);
     }
+    if (e != cudaSuccess) return e;
     count_launches(1);
     return cudaGetLastError();
 }

@@ -173,6 +173,14 @@ __device__ __forceinline__ void ldg_v8(const void *p, uint4 &a, uint4 &b) {
                  : "=r"(a.x), "=r"(a.y), "=r"(a.z), "=r"(a.w), "=r"(b.x), "=r"(b.y), "=r"(b.z), "=r"(b.w)
                  : "l"(p));
 }
+// 2^x by the special-function unit (PTX ex2.approx.ftz: a few ulp, results
+// below the smallest normal flushed to zero): the softmax exponentials, whose
+// tolerance is that of bf16 storage
+__device__ __forceinline__ float ex2_fast(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
 __device__ __forceinline__ void prefetch_l2(const void *p) { asm volatile("prefetch.global.L2 [%0];" ::"l"(p)); }
 __device__ __forceinline__ void prefetch_l1(const void *p) { asm volatile("prefetch.global.L1 [%0];" ::"l"(p)); }
 
