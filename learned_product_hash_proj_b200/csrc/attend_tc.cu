@@ -239,6 +239,7 @@ __global__ void __launch_bounds__(256) k_remote_tc(const __grid_constant__ AttnM
     uint64_t *bar_kv = (uint64_t *)(smem + L::BAR_OFF);  // [2]: K/V of each stage landed
     uint64_t *mbar = bar_kv + 2;                          // MMA completion
     uint32_t *tmem_base = (uint32_t *)(mbar + 1);
+    pdl_trigger();  // the local kernel may start; it waits for the partials itself
     if (timed_out(counters)) return;
     if (tc::smem_u32(smem) & 1023) {  // uniform; TMA's 128-byte swizzle needs 1024-byte aligned tiles
         if (threadIdx.x == 0) record_error(counters, kDevErrSmemAlign);
@@ -248,6 +249,7 @@ __global__ void __launch_bounds__(256) k_remote_tc(const __grid_constant__ AttnM
     const int quarter = warp & 3, half = warp >> 2;
     const int row = quarter * 32 + lane;
 
+    pdl_wait();  // the work items and pair ids (pair kernels) are complete
     if (tid == 0) {
         int acc = 0;
         for (int g = 0; g < ng; ++g) { s_pref[g] = acc; acc += nwork[bh0 + g]; }
@@ -948,6 +950,7 @@ __global__ void __launch_bounds__(320, 1) k_local_ws(const __grid_constant__ Att
             for (int r = 0; r < RMAX; ++r) selv[r] = (r < R && t < S) ? sel[((size_t)bh * S + t) * R + r] : -1;
         };
         if (g < n) load_sel(g);
+        pdl_wait();  // the remote partials (remote kernel) are complete
         for (int i = g; i < n && ok; i += 2) {
             const int u = i >> 1;
             const int f = tile_of(i);
@@ -1260,18 +1263,22 @@ static cudaError_t launch_tc_shape(const Plan &p, const bf16 *Q, const bf16 *K, 
         const bool do_remote = (parts & kAttendRemote) && (both || pass == 0);
         const bool do_local = (parts & kAttendLocal) && (both || pass == 1);
         if (c.R > 0 && do_remote) {
-            k_remote_tc<D, BS><<<remote_ctas, 256, rsmem, s>>>(
-                rmaps, Q, (const int32_t *)ws_ptr(p, ws, kRegPairs), (const int4 *)ws_ptr(p, ws, kRegWork),
-                (const int32_t *)ws_ptr(p, ws, kRegNWork), (bf16 *)ws_ptr(p, ws, kRegPartO),
-                (float2 *)ws_ptr(p, ws, kRegPartML), cnt_err, c.S, c.R, p.max_work, scale_log2, g0, ng);
+            if ((e = launch_pdl(k_remote_tc<D, BS>, dim3(remote_ctas), dim3(256), rsmem, s, rmaps, Q,
+                                (const int32_t *)ws_ptr(p, ws, kRegPairs), (const int4 *)ws_ptr(p, ws, kRegWork),
+                                (const int32_t *)ws_ptr(p, ws, kRegNWork), (bf16 *)ws_ptr(p, ws, kRegPartO),
+                                (float2 *)ws_ptr(p, ws, kRegPartML), cnt_err, c.S, c.R, p.max_work, scale_log2, g0,
+                                ng)) != cudaSuccess)
+                return e;
             count_launches(1);
         }
         if (!do_local) continue;
         if constexpr (ws_local) {
             const int tiles = ng * ((c.S + 127) / 128);
-            k_local_ws<D, BS, NK, RMAX><<<std::min(local_ctas, tiles), 320, smem, s>>>(
-                lmaps, sel, (const bf16 *)ws_ptr(p, ws, kRegPartO), (const float2 *)ws_ptr(p, ws, kRegPartML), O,
-                o32, lse, cnt_err, c.S, c.H, c.R, c.L, scale_log2, g0, ng);
+            if ((e = launch_pdl(k_local_ws<D, BS, NK, RMAX>, dim3(std::min(local_ctas, tiles)), dim3(320), smem, s,
+                                lmaps, sel, (const bf16 *)ws_ptr(p, ws, kRegPartO),
+                                (const float2 *)ws_ptr(p, ws, kRegPartML), O, o32, lse, cnt_err, c.S, c.H, c.R, c.L,
+                                scale_log2, g0, ng)) != cudaSuccess)
+                return e;
         } else {
             kl<<<local_ctas, 256, smem, s>>>(lmaps, sel, (const bf16 *)ws_ptr(p, ws, kRegPartO),
                                              (const float2 *)ws_ptr(p, ws, kRegPartML), O, cnt_err, c.S, c.H, c.R,
