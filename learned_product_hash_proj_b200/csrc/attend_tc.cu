@@ -1290,6 +1290,237 @@ static cudaError_t launch_tc_shape(const Plan &p, const bf16 *Q, const bf16 *K, 
     return cudaSuccess;
 }
 
+// ---------------------------------------------------------------------------
+// backward, local keys, on the tensor cores: for each 128-query tile and its
+// local key window (the forward local kernel's tile), with the forward's
+// log-sum-exp and D = dO . O of each row given,
+//   S  = Q K^T                      (tcgen05, fp32 in TMEM)
+//   dP = dO V^T                     (dO as two bf16 terms hi + lo, both products accumulated)
+//   P  = exp(S / sqrt(d) - lse),  dS = P (dP - D)   (fp32; causal window mask as in the forward)
+//   dQ_local = dS K                 (dS in bf16 from shared memory, K as the MN-major operand)
+// dQ_local (fp32, without the 1/sqrt(d) factor) goes to dq_loc [B*H, S, d]; the
+// SIMT dQ kernel adds the remote keys' part and applies the factor and RoPE.
+// One persistent CTA of 256 threads per SM walks the tiles; TMEM lane quarter
+// q is read by warps q and q + 4, each taking half of the columns.
+// ---------------------------------------------------------------------------
+struct BwdMaps {
+    CUtensorMap q, k, v, dohi, dolo;
+};
+
+template <int D, int NK>
+struct BwdLocalSmem {
+    static constexpr int QB = 128 * D * 2, KB = NK * D * 2, PB = 128 * NK * 2;
+    static constexpr int Q_OFF = 0, K_OFF = QB, V_OFF = QB + KB, DOH_OFF = QB + 2 * KB, DOL_OFF = 2 * QB + 2 * KB;
+    static constexpr int DS_OFF = 3 * QB + 2 * KB;
+    static constexpr int BAR_OFF = DS_OFF + PB;  // 2 mbarriers + TMEM base
+    static constexpr int BYTES = BAR_OFF + 32;
+    static constexpr bool supported = 2 * NK + D <= 512 && NK % 32 == 0 && D % 64 == 0 && BYTES <= 227 * 1024;
+};
+
+template <int D, int BS, int NK>
+__global__ void __launch_bounds__(256, 1) k_bwd_local_dq_tc(const __grid_constant__ BwdMaps maps,
+                                                            const float *__restrict__ lse,
+                                                            const float *__restrict__ dsum, float *__restrict__ dq_loc,
+                                                            unsigned long long *__restrict__ counters, int S, int L,
+                                                            float scale_log2, int nbh) {
+    using Lay = BwdLocalSmem<D, NK>;
+    static_assert(Lay::supported, "tile shape");
+    constexpr int QB = Lay::QB, KB = Lay::KB, HALF = NK / 2, DH = D / 2;
+    static_assert(HALF % 32 == 0 && DH % 32 == 0, "column halves of 32");
+    extern __shared__ __align__(1024) uint8_t smem[];
+    uint8_t *sQ = smem + Lay::Q_OFF, *sK = smem + Lay::K_OFF, *sV = smem + Lay::V_OFF;
+    uint8_t *sDOH = smem + Lay::DOH_OFF, *sDOL = smem + Lay::DOL_OFF, *sDS = smem + Lay::DS_OFF;
+    uint64_t *bar_ld = (uint64_t *)(smem + Lay::BAR_OFF), *mbar = bar_ld + 1;
+    uint32_t *tmem_base = (uint32_t *)(bar_ld + 2);
+    if (timed_out(counters)) return;
+    if (tc::smem_u32(smem) & 1023) {
+        if (threadIdx.x == 0) record_error(counters, kDevErrSmemAlign);
+        return;
+    }
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quarter = warp & 3, half = warp >> 2;
+    const int row = quarter * 32 + lane;
+    const int ntiles = (S + 127) / 128;
+    const int total = nbh * ntiles;
+    if (warp == 0) {
+        tc::tmem_alloc(tmem_base, 512);
+        tc::tmem_relinquish();
+    }
+    if (tid == 0) {
+        tc::mbar_init(bar_ld, 1);
+        tc::mbar_init(mbar, 1);
+        tc::fence_mbar_init();
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = *tmem_base;
+    const uint32_t trow = tmem + ((uint32_t)(quarter * 32) << 16);
+    const uint32_t tS = trow, tP = trow + NK, tQ = trow + 2 * NK;  // S, dP and dQ columns of this lane quarter
+    bool ok = true;
+    int pend = -1;       // thread 0: the load of tile k issued and not yet seen complete
+    uint32_t mph = 0;    // completions of mbar so far, mod 2
+    int k = 0;
+    for (int f = blockIdx.x; f < total && ok; f += gridDim.x, ++k) {
+        const int bh = f / ntiles, t0 = (f % ntiles) * 128;
+        const int kstart = max(0, t0 / BS - L + 1) * BS;
+        const int nq = min(128, S - t0);
+        const int t = t0 + row;
+        const bool live = row < nq;
+        if (tid == 0) {
+            tc::mbar_expect_tx(bar_ld, 3 * QB + 2 * KB);
+#pragma unroll
+            for (int a = 0; a < D / 64; ++a) {
+                tc::tma_load_3d(sQ + a * (128 * 128), &maps.q, 64 * a, t0, bh, bar_ld);
+                tc::tma_load_3d(sDOH + a * (128 * 128), &maps.dohi, 64 * a, t0, bh, bar_ld);
+                tc::tma_load_3d(sDOL + a * (128 * 128), &maps.dolo, 64 * a, t0, bh, bar_ld);
+                tc::tma_load_3d(sK + a * (NK * 128), &maps.k, 64 * a, kstart, bh, bar_ld);
+                tc::tma_load_3d(sV + a * (NK * 128), &maps.v, 64 * a, kstart, bh, bar_ld);
+            }
+            pend = k;
+        }
+        // this row's log-sum-exp (in the exp2 domain) and D
+        const float lse2 = live ? lse[(size_t)bh * S + t] * 1.4426950408889634f : 0.f;
+        const float Drow = live ? dsum[(size_t)bh * S + t] : 0.f;
+        bool landed = true;
+        if (tid == 0) {
+            landed = tc::mbar_wait(bar_ld, (uint32_t)(k & 1));
+            if (landed) pend = -1;
+        }
+        tc::fence_before_sync();
+        ok = __syncthreads_and(landed);
+        tc::fence_after_sync();
+        if (!ok) break;
+        if (tid == 0) {
+            const uint32_t id = tc::idesc_bf16(128, NK);
+            const uint32_t aq = tc::smem_u32(sQ), ah = tc::smem_u32(sDOH), al = tc::smem_u32(sDOL);
+            const uint32_t bk = tc::smem_u32(sK), bv = tc::smem_u32(sV);
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+                const uint32_t ao = (kk >> 2) * (128 * 128) + (kk & 3) * 32, bo = (kk >> 2) * (NK * 128) + (kk & 3) * 32;
+                tc::mma_bf16(tmem, tc::desc_sw128(aq + ao), tc::desc_sw128(bk + bo), id, kk > 0);
+                tc::mma_bf16(tmem + NK, tc::desc_sw128(ah + ao), tc::desc_sw128(bv + bo), id, kk > 0);
+            }
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+                const uint32_t ao = (kk >> 2) * (128 * 128) + (kk & 3) * 32, bo = (kk >> 2) * (NK * 128) + (kk & 3) * 32;
+                tc::mma_bf16(tmem + NK, tc::desc_sw128(al + ao), tc::desc_sw128(bv + bo), id, 1u);
+            }
+            tc::commit(mbar);
+        }
+        ok = __syncthreads_and(tc::mbar_wait(mbar, mph));
+        mph ^= 1u;
+        tc::fence_after_sync();
+        if (!ok) break;
+        // dS over keys s in [lo(t), t]: columns [vlo, vhi]
+        const int lo = max(0, t / BS - L + 1) * BS;
+        const int vlo = lo - kstart, vhi = t - kstart;
+#pragma unroll 1
+        for (int c0 = half * HALF; c0 < half * HALF + HALF; c0 += 32) {
+            float sv[32], pv[32];
+            tc::tmem_ld32(tS + c0, sv);
+            tc::tmem_ld32(tP + c0, pv);
+            uint32_t pk[16];
+#pragma unroll
+            for (int u = 0; u < 16; ++u) {
+                const int i = 2 * u;
+                const bool in0 = live && c0 + i >= vlo && c0 + i <= vhi;
+                const bool in1 = live && c0 + i + 1 >= vlo && c0 + i + 1 <= vhi;
+                const float p0 = in0 ? tc::ex2_fast(fmaf(sv[i], scale_log2, -lse2)) : 0.f;
+                const float p1 = in1 ? tc::ex2_fast(fmaf(sv[i + 1], scale_log2, -lse2)) : 0.f;
+                pk[u] = pack2(p0 * (pv[i] - Drow), p1 * (pv[i + 1] - Drow));
+            }
+#pragma unroll
+            for (int q8 = 0; q8 < 4; ++q8)
+                *(uint4 *)(sDS + tc::kmajor_chunk(row, (c0 >> 3) + q8, NK)) =
+                    make_uint4(pk[4 * q8], pk[4 * q8 + 1], pk[4 * q8 + 2], pk[4 * q8 + 3]);
+        }
+        tc::fence_smem_to_async();
+        tc::fence_before_sync();
+        __syncthreads();
+        tc::fence_after_sync();
+        if (tid == 0) {
+            const uint32_t id = tc::idesc_bf16(128, D, true);
+            const uint32_t ad = tc::smem_u32(sDS), bk = tc::smem_u32(sK);
+#pragma unroll
+            for (int kk = 0; kk < NK / 16; ++kk)
+                tc::mma_bf16(tmem + 2 * NK, tc::desc_kmajor(ad + 256 * kk, NK), tc::desc_sw128_mn(bk + 2048 * kk, NK * 128),
+                             id, kk > 0);
+            tc::commit(mbar);
+        }
+        ok = __syncthreads_and(tc::mbar_wait(mbar, mph));
+        mph ^= 1u;
+        tc::fence_after_sync();
+        if (!ok) break;
+#pragma unroll 1
+        for (int c0 = half * DH; c0 < half * DH + DH; c0 += 32) {
+            float v[32];
+            tc::tmem_ld32(tQ + c0, v);
+            if (live) {
+                float4 *dst = (float4 *)(dq_loc + ((size_t)bh * S + t) * D + c0);
+#pragma unroll
+                for (int q4 = 0; q4 < 8; ++q4) dst[q4] = make_float4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
+            }
+        }
+        tc::fence_before_sync();
+        __syncthreads();  // shared memory and TMEM are free for the next tile
+        tc::fence_after_sync();
+    }
+    // leave no TMA write in flight into this CTA's shared memory
+    if (tid == 0 && pend >= 0 && !tc::mbar_wait(bar_ld, (uint32_t)(pend & 1))) ok = false;
+    if (!ok && tid == 0) record_error(counters, kDevErrTimeout);
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 0) tc::tmem_dealloc(tmem, 512);
+}
+
+
+template <int D, int BS, int NK>
+static cudaError_t launch_bwd_local_dq_shape(const Plan &p, const void *Q, const void *K, const void *V,
+                                             const void *dohi, const void *dolo, const float *lse, const float *dsum,
+                                             float *dq_loc, unsigned long long *counters, cudaStream_t s) {
+    const mono_config &c = p.cfg;
+    using Lay = BwdLocalSmem<D, NK>;
+    BwdMaps maps;
+    const int BH = c.B * c.H;
+    if (!make_map_3d(&maps.q, Q, D, c.S, BH, 128) || !make_map_3d(&maps.k, K, D, c.S, BH, NK) ||
+        !make_map_3d(&maps.v, V, D, c.S, BH, NK) || !make_map_3d(&maps.dohi, dohi, D, c.S, BH, 128) ||
+        !make_map_3d(&maps.dolo, dolo, D, c.S, BH, 128))
+        return cudaErrorInvalidValue;
+    auto kern = k_bwd_local_dq_tc<D, BS, NK>;
+    cudaError_t e;
+    if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::BYTES)) != cudaSuccess)
+        return e;
+    int dev = 0, sms = 148;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+        return e;
+    const int tiles = BH * ((c.S + 127) / 128);
+    const float scale_log2 = (float)(1.4426950408889634 / sqrt((double)c.d));
+    kern<<<std::min(tiles, sms), 256, Lay::BYTES, s>>>(maps, lse, dsum, dq_loc, counters, c.S, c.L, scale_log2, BH);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+bool bwd_local_dq_tc_supported(const mono_config &c) {
+    if (c.dtype != MONO_BF16 || c.Bs != 64 || c.L < 1) return false;
+    const int nk = 128 + (c.L - 1) * c.Bs;
+    return (c.d == 64 && nk <= 192) || (c.d == 128 && nk <= 128);
+}
+
+cudaError_t launch_bwd_local_dq_tc(const Plan &p, const void *Q, const void *K, const void *V, const void *dohi,
+                                  const void *dolo, const float *lse, const float *dsum, float *dq_loc,
+                                  unsigned long long *counters, cudaStream_t s) {
+    const mono_config &c = p.cfg;
+    if (!bwd_local_dq_tc_supported(c)) return cudaErrorInvalidValue;
+    const int nk = 128 + (c.L - 1) * c.Bs;
+    if (c.d == 64 && nk <= 128)
+        return launch_bwd_local_dq_shape<64, 64, 128>(p, Q, K, V, dohi, dolo, lse, dsum, dq_loc, counters, s);
+    if (c.d == 64)
+        return launch_bwd_local_dq_shape<64, 64, 192>(p, Q, K, V, dohi, dolo, lse, dsum, dq_loc, counters, s);
+    return launch_bwd_local_dq_shape<128, 64, 128>(p, Q, K, V, dohi, dolo, lse, dsum, dq_loc, counters, s);
+}
+
 cudaError_t launch_attend_tc(const Plan &p, const void *Q, const void *K, const void *V, const int32_t *sel, void *O,
                              void *ws, cudaStream_t s, int parts, float *o32, float *lse, bool *stats) {
     if (stats) *stats = false;

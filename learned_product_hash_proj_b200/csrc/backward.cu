@@ -38,7 +38,7 @@ namespace mono {
 namespace {
 
 struct BwdLayout {
-    size_t lse, dsum, cnt, start, cursor, list, dO, dQp, dKp, dVp, total;
+    size_t lse, dsum, cnt, start, cursor, list, dO, dQp, dKp, dVp, dOhi, dOlo, dQloc, total;
 };
 
 BwdLayout bwd_layout(const Plan &p) {
@@ -61,6 +61,10 @@ BwdLayout bwd_layout(const Plan &p) {
     L.dQp = take(B * S * H * d * 4);
     L.dKp = take(B * S * H * d * 4);
     L.dVp = take(B * S * H * d * 4);
+    // the tensor-core local dQ: dO as two bf16 terms and its fp32 result, head-major [B*H, S, d]
+    L.dOhi = take(B * H * S * d * 2);
+    L.dOlo = take(B * H * S * d * 2);
+    L.dQloc = take(B * H * S * d * 4);
     L.total = o;
     return L;
 }
@@ -179,13 +183,42 @@ __device__ __forceinline__ float group_sum(float v) {
     return v;
 }
 
+// dO (token-major fp32) as two bf16 terms hi = bf16(v), lo = bf16(v - hi), head-major for the tensor-core local
+// dQ, and D = dO . O of each row from the forward's fp32 O.  One warp per (b, t, h) row; grid covers B*S*H rows.
+template <int DD>
+__global__ void __launch_bounds__(256) k_bwd_prep(const float *__restrict__ dO, const float *__restrict__ o32,
+                                                  __nv_bfloat16 *__restrict__ dohi, __nv_bfloat16 *__restrict__ dolo,
+                                                  float *__restrict__ dsum, int B, int H, int S) {
+    constexpr int PER = DD / 32;
+    const long long w = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (w >= (long long)B * S * H) return;
+    const int h = (int)(w % H);
+    const long long bt = w / H;
+    const int t = (int)(bt % S), b = (int)(bt / S);
+    const size_t hm = (((size_t)b * H + h) * S + t) * DD;  // head-major row
+    float part = 0.f;
+#pragma unroll
+    for (int e = 0; e < PER; ++e) {
+        const int i = lane + 32 * e;
+        const float v = dO[w * DD + i];
+        const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+        dohi[hm + i] = hi;
+        dolo[hm + i] = __float2bfloat16_rn(v - __bfloat162float(hi));
+        part = fmaf(v, o32[w * DD + i], part);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+    if (lane == 0) dsum[((size_t)b * H + h) * S + t] = part;
+}
+
 template <typename T, int DD>
 __global__ void __launch_bounds__(256) k_bwd_dq(const T *__restrict__ Q, const T *__restrict__ K,
                                                 const T *__restrict__ V, const int32_t *__restrict__ sel,
                                                 const float *__restrict__ dO, const GradOut go,
                                                 float *__restrict__ lse_out, float *__restrict__ dsum_out,
-                                                const float *__restrict__ o32, int B, int H, int S, int Bs, int L,
-                                                int R, float scale) {
+                                                const float *__restrict__ o32, const float *__restrict__ dq_loc,
+                                                int B, int H, int S, int Bs, int L, int R, float scale) {
     constexpr int TPQ = DD / kDqE, E = kDqE, U = 2;
     const long long nq = (long long)B * H * S;
     const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
@@ -206,9 +239,11 @@ __global__ void __launch_bounds__(256) k_bwd_dq(const T *__restrict__ Q, const T
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) nloc_w = max(nloc_w, __shfl_xor_sync(0xffffffffu, nloc_w, o));
 
-    // one sweep over the query's keys; f(k row, v row, valid) per group of U keys
+    // one sweep over the query's keys; f(k row, v row, valid) per group of U keys (the remote blocks only when
+    // the tensor cores did the local keys: dq_loc)
+    const int nloc_sweep = dq_loc ? 0 : nloc_w;
     auto sweep = [&](auto &&f) {
-        for (int i = 0; i < nloc_w; i += U) {
+        for (int i = 0; i < nloc_sweep; i += U) {
             const T *kr[U], *vr[U];
             bool ok[U];
 #pragma unroll
@@ -329,6 +364,12 @@ __global__ void __launch_bounds__(256) k_bwd_dq(const T *__restrict__ Q, const T
         }
     });
     if (live) {
+        if (dq_loc) {
+            float dl[E];
+            load16<float>(dq_loc + w * DD + e0, dl);
+#pragma unroll
+            for (int e = 0; e < E; ++e) dq[e] += dl[e];
+        }
 #pragma unroll
         for (int e = 0; e < E; ++e) dq[e] *= scale;
         store_grad16<DD>(go, go.q, true, dq, b, h, t, e0, B, H, S);
@@ -627,7 +668,8 @@ cudaError_t gemm_any(int M, int N, int Kd, const TA *A, long long am, long long 
 // o32: the forward's O in fp32 (token-major) with its log-sum-exp already in the lse region, or null
 template <typename T>
 cudaError_t attend_backward(const Plan &p, const T *Q, const T *K, const T *V, const int32_t *sel, const float *dO,
-                            const GradOut &go, char *bws, cudaStream_t s, const float *o32 = nullptr) {
+                            const GradOut &go, char *bws, cudaStream_t s, const float *o32 = nullptr,
+                            unsigned long long *counters = nullptr) {
     const mono_config &c = p.cfg;
     const BwdLayout L = bwd_layout(p);
     float *lse = (float *)(bws + L.lse), *dsum = (float *)(bws + L.dsum);
@@ -638,12 +680,28 @@ cudaError_t attend_backward(const Plan &p, const T *Q, const T *K, const T *V, c
     cudaError_t e;
     const int tpq = c.d / kDqE;
     const unsigned gq = (unsigned)((nq * tpq + 255) / 256);
+    // with the forward's statistics, the local keys' part of dQ on the tensor cores where the shape allows
+    float *dq_loc = nullptr;
+    if constexpr (sizeof(T) == 2) {
+        if (o32 && counters && bwd_local_dq_tc_supported(c)) {
+            __nv_bfloat16 *dohi = (__nv_bfloat16 *)(bws + L.dOhi), *dolo = (__nv_bfloat16 *)(bws + L.dOlo);
+            dq_loc = (float *)(bws + L.dQloc);
+            const unsigned gp = (unsigned)((nq + 7) / 8);
+            if (c.d == 64)
+                k_bwd_prep<64><<<gp, 256, 0, s>>>(dO, o32, dohi, dolo, dsum, c.B, c.H, c.S);
+            else
+                k_bwd_prep<128><<<gp, 256, 0, s>>>(dO, o32, dohi, dolo, dsum, c.B, c.H, c.S);
+            count_launches(1);
+            if ((e = launch_bwd_local_dq_tc(p, Q, K, V, dohi, dolo, lse, dsum, dq_loc, counters, s)) != cudaSuccess)
+                return e;
+        }
+    }
     if (c.d == 64)
-        k_bwd_dq<T, 64><<<gq, 256, 0, s>>>(Q, K, V, sel, dO, go, lse, dsum, o32, c.B, c.H, c.S, c.Bs, c.L, c.R,
-                                           scale);
+        k_bwd_dq<T, 64><<<gq, 256, 0, s>>>(Q, K, V, sel, dO, go, lse, dsum, o32, dq_loc, c.B, c.H, c.S, c.Bs, c.L,
+                                           c.R, scale);
     else
-        k_bwd_dq<T, 128><<<gq, 256, 0, s>>>(Q, K, V, sel, dO, go, lse, dsum, o32, c.B, c.H, c.S, c.Bs, c.L, c.R,
-                                            scale);
+        k_bwd_dq<T, 128><<<gq, 256, 0, s>>>(Q, K, V, sel, dO, go, lse, dsum, o32, dq_loc, c.B, c.H, c.S, c.Bs, c.L,
+                                            c.R, scale);
     count_launches(1);
     if (c.R > 0) {
         const long long n = nq * c.R;
@@ -704,7 +762,7 @@ cudaError_t backward_t(const Plan &p, const T *x, const T *Wq, const T *Wk, cons
         float *c0[1] = {dO}, *c1[1] = {dWo};
         if ((e = gemm_grad_tc(BS, Hd, W, 1, 1, a0, false, b0, true, c0, false, counters, s)) != cudaSuccess) return e;
         if ((e = gemm_grad_tc(W, Hd, BS, 1, 1, a0, true, b1, true, c1, false, counters, s)) != cudaSuccess) return e;
-        if ((e = attend_backward<T>(p, Q, K, V, sel, dO, go, bws, s, o32)) != cudaSuccess) return e;
+        if ((e = attend_backward<T>(p, Q, K, V, sel, dO, go, bws, s, o32, counters)) != cudaSuccess) return e;
         // q = x Wq^T (per head, then RoPE):  dWq = dQp^T x (both MN-major),  dx = dQp Wq + dKp Wk + dVp Wv,
         // each dZp as hi + lo
         using B16 = __nv_bfloat16;

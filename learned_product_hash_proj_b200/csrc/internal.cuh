@@ -142,6 +142,13 @@ enum AttendParts { kAttendPairs = 1, kAttendRemote = 2, kAttendLocal = 4, kAtten
 // With o32 and lse (backward recompute): the local kernel also writes each row of O in fp32 (token-major like O)
 // and its natural log-sum-exp over the query's keys (scores scaled by 1/sqrt(d)); *stats tells whether the kernel
 // for this shape did.
+// backward, local keys of each query on the tensor cores: dq_loc [B*H, S, d] fp32 = sum over the local keys of
+// P (dP - D) k (without the 1/sqrt(d) factor), from the forward's log-sum-exp and D per row and dO as two bf16
+// terms [B*H, S, d]; shapes where bwd_local_dq_tc_supported
+bool bwd_local_dq_tc_supported(const mono_config &c);
+cudaError_t launch_bwd_local_dq_tc(const Plan &p, const void *Q, const void *K, const void *V, const void *dohi,
+                                  const void *dolo, const float *lse, const float *dsum, float *dq_loc,
+                                  unsigned long long *counters, cudaStream_t s);
 cudaError_t launch_attend_tc(const Plan &p, const void *Q, const void *K, const void *V, const int32_t *sel, void *O,
                              void *ws, cudaStream_t s, int parts = kAttendAll, float *o32 = nullptr,
                              float *lse = nullptr, bool *stats = nullptr);
