@@ -176,6 +176,14 @@ __device__ __forceinline__ uint32_t pack2(float a, float b) {
     return *(uint32_t *)&h;
 }
 
+// a and b as two bf16 terms each: hi = bf16(v), lo = bf16(v - hi) (16 significant bits together)
+__device__ __forceinline__ void split2(float a, float b, uint32_t &hi, uint32_t &lo) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    const float2 hf = __bfloat1622float2(h);
+    hi = *(const uint32_t *)&h;
+    lo = pack2(a - hf.x, b - hf.y);
+}
+
 __device__ __forceinline__ bool timed_out(const unsigned long long *counters) {
     return *(volatile const unsigned long long *)&counters[kCntErr] == kDevErrTimeout;
 }
@@ -1297,7 +1305,7 @@ static cudaError_t launch_tc_shape(const Plan &p, const bf16 *Q, const bf16 *K, 
 //   S  = Q K^T                      (tcgen05, fp32 in TMEM)
 //   dP = dO V^T                     (dO as two bf16 terms hi + lo, both products accumulated)
 //   P  = exp(S / sqrt(d) - lse),  dS = P (dP - D)   (fp32; causal window mask as in the forward)
-//   dQ_local = dS K                 (dS in bf16 from shared memory, K as the MN-major operand)
+//   dQ_local = dS K                 (dS as two bf16 terms from shared memory, K as the MN-major operand)
 // dQ_local (fp32, without the 1/sqrt(d) factor) goes to dq_loc [B*H, S, d]; the
 // SIMT dQ kernel adds the remote keys' part and applies the factor and RoPE.
 // One persistent CTA of 256 threads per SM walks the tiles; TMEM lane quarter
@@ -1311,8 +1319,8 @@ template <int D, int NK>
 struct BwdLocalSmem {
     static constexpr int QB = 128 * D * 2, KB = NK * D * 2, PB = 128 * NK * 2;
     static constexpr int Q_OFF = 0, K_OFF = QB, V_OFF = QB + KB, DOH_OFF = QB + 2 * KB, DOL_OFF = 2 * QB + 2 * KB;
-    static constexpr int DS_OFF = 3 * QB + 2 * KB;
-    static constexpr int BAR_OFF = DS_OFF + PB;  // 2 mbarriers + TMEM base
+    static constexpr int DS_OFF = 3 * QB + 2 * KB, DSL_OFF = DS_OFF + PB;  // dS hi and lo terms
+    static constexpr int BAR_OFF = DSL_OFF + PB;                          // 2 mbarriers + TMEM base
     static constexpr int BYTES = BAR_OFF + 32;
     static constexpr bool supported = 2 * NK + D <= 512 && NK % 32 == 0 && D % 64 == 0 && BYTES <= 227 * 1024;
 };
@@ -1330,6 +1338,7 @@ __global__ void __launch_bounds__(256, 1) k_bwd_local_dq_tc(const __grid_constan
     extern __shared__ __align__(1024) uint8_t smem[];
     uint8_t *sQ = smem + Lay::Q_OFF, *sK = smem + Lay::K_OFF, *sV = smem + Lay::V_OFF;
     uint8_t *sDOH = smem + Lay::DOH_OFF, *sDOL = smem + Lay::DOL_OFF, *sDS = smem + Lay::DS_OFF;
+    uint8_t *sDSL = smem + Lay::DSL_OFF;
     uint64_t *bar_ld = (uint64_t *)(smem + Lay::BAR_OFF), *mbar = bar_ld + 1;
     uint32_t *tmem_base = (uint32_t *)(bar_ld + 2);
     if (timed_out(counters)) return;
@@ -1420,7 +1429,7 @@ __global__ void __launch_bounds__(256, 1) k_bwd_local_dq_tc(const __grid_constan
             float sv[32], pv[32];
             tc::tmem_ld32(tS + c0, sv);
             tc::tmem_ld32(tP + c0, pv);
-            uint32_t pk[16];
+            uint32_t hk[16], lk[16];
 #pragma unroll
             for (int u = 0; u < 16; ++u) {
                 const int i = 2 * u;
@@ -1428,12 +1437,14 @@ __global__ void __launch_bounds__(256, 1) k_bwd_local_dq_tc(const __grid_constan
                 const bool in1 = live && c0 + i + 1 >= vlo && c0 + i + 1 <= vhi;
                 const float p0 = in0 ? tc::ex2_fast(fmaf(sv[i], scale_log2, -lse2)) : 0.f;
                 const float p1 = in1 ? tc::ex2_fast(fmaf(sv[i + 1], scale_log2, -lse2)) : 0.f;
-                pk[u] = pack2(p0 * (pv[i] - Drow), p1 * (pv[i + 1] - Drow));
+                split2(p0 * (pv[i] - Drow), p1 * (pv[i + 1] - Drow), hk[u], lk[u]);
             }
 #pragma unroll
-            for (int q8 = 0; q8 < 4; ++q8)
-                *(uint4 *)(sDS + tc::kmajor_chunk(row, (c0 >> 3) + q8, NK)) =
-                    make_uint4(pk[4 * q8], pk[4 * q8 + 1], pk[4 * q8 + 2], pk[4 * q8 + 3]);
+            for (int q8 = 0; q8 < 4; ++q8) {
+                const uint32_t off = tc::kmajor_chunk(row, (c0 >> 3) + q8, NK);
+                *(uint4 *)(sDS + off) = make_uint4(hk[4 * q8], hk[4 * q8 + 1], hk[4 * q8 + 2], hk[4 * q8 + 3]);
+                *(uint4 *)(sDSL + off) = make_uint4(lk[4 * q8], lk[4 * q8 + 1], lk[4 * q8 + 2], lk[4 * q8 + 3]);
+            }
         }
         tc::fence_smem_to_async();
         tc::fence_before_sync();
@@ -1441,11 +1452,13 @@ __global__ void __launch_bounds__(256, 1) k_bwd_local_dq_tc(const __grid_constan
         tc::fence_after_sync();
         if (tid == 0) {
             const uint32_t id = tc::idesc_bf16(128, D, true);
-            const uint32_t ad = tc::smem_u32(sDS), bk = tc::smem_u32(sK);
+            const uint32_t ad = tc::smem_u32(sDS), adl = tc::smem_u32(sDSL), bk = tc::smem_u32(sK);
 #pragma unroll
-            for (int kk = 0; kk < NK / 16; ++kk)
-                tc::mma_bf16(tmem + 2 * NK, tc::desc_kmajor(ad + 256 * kk, NK), tc::desc_sw128_mn(bk + 2048 * kk, NK * 128),
-                             id, kk > 0);
+            for (int kk = 0; kk < NK / 16; ++kk) {
+                const uint64_t bd = tc::desc_sw128_mn(bk + 2048 * kk, NK * 128);
+                tc::mma_bf16(tmem + 2 * NK, tc::desc_kmajor(ad + 256 * kk, NK), bd, id, kk > 0);
+                tc::mma_bf16(tmem + 2 * NK, tc::desc_kmajor(adl + 256 * kk, NK), bd, id, 1u);
+            }
             tc::commit(mbar);
         }
         ok = __syncthreads_and(tc::mbar_wait(mbar, mph));
@@ -1460,6 +1473,230 @@ __global__ void __launch_bounds__(256, 1) k_bwd_local_dq_tc(const __grid_constan
                 float4 *dst = (float4 *)(dq_loc + ((size_t)bh * S + t) * D + c0);
 #pragma unroll
                 for (int q4 = 0; q4 < 8; ++q4) dst[q4] = make_float4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
+            }
+        }
+        tc::fence_before_sync();
+        __syncthreads();  // shared memory and TMEM are free for the next tile
+        tc::fence_after_sync();
+    }
+    // leave no TMA write in flight into this CTA's shared memory
+    if (tid == 0 && pend >= 0 && !tc::mbar_wait(bar_ld, (uint32_t)(pend & 1))) ok = false;
+    if (!ok && tid == 0) record_error(counters, kDevErrTimeout);
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 0) tc::tmem_dealloc(tmem, 512);
+}
+
+
+// ---------------------------------------------------------------------------
+// backward, local queries of each key, on the tensor cores (key-major): for
+// each tile of 128 keys [k0, k0 + 128) of one head, the NQ = 128 + (L-1) Bs
+// queries [k0, k0 + NQ) whose local window holds some of them,
+//   S^T  = K Q^T,  dP^T = V dO^T   (dO as two bf16 terms, both products accumulated)
+//   P^T  = exp(S^T / sqrt(d) - lse_t),  dS^T = P^T (dP^T - D_t)   (fp32; the window mask of each query)
+//   dV_local = P^T dO,  dK_local = dS^T Q   (P^T and dS^T as two bf16 terms each: the hi terms in a first
+//                                            round, the lo terms through the same buffers in a second, which
+//                                            drops only lo x lo; dO and Q MN-major)
+// to dv_loc and dk_loc [B*H, S, d] (fp32, dK without the 1/sqrt(d) factor);
+// the SIMT dK/dV kernel adds the selecting queries' part.  Same roles as
+// k_bwd_local_dq_tc: one persistent CTA of 256 threads per SM, one MMA thread,
+// TMEM lane quarter q read by warps q and q + 4.
+// ---------------------------------------------------------------------------
+template <int D, int NQ>
+struct BwdKvSmem {
+    static constexpr int KB = 128 * D * 2, QB = NQ * D * 2, PB = 128 * NQ * 2;
+    static constexpr int K_OFF = 0, V_OFF = KB, Q_OFF = 2 * KB, DOH_OFF = 2 * KB + QB, DOL_OFF = 2 * KB + 2 * QB;
+    static constexpr int P_OFF = 2 * KB + 3 * QB, DS_OFF = P_OFF + PB;
+    static constexpr int LSE_OFF = DS_OFF + PB, DD_OFF = LSE_OFF + NQ * 4;  // per query: lse (exp2 domain), D
+    static constexpr int BAR_OFF = DD_OFF + NQ * 4;                         // 2 mbarriers + TMEM base
+    static constexpr int BYTES = BAR_OFF + 32;
+    static constexpr bool supported =
+        2 * NQ + 2 * D <= 512 && NQ % 32 == 0 && NQ <= 256 && D % 64 == 0 && BYTES <= 227 * 1024;
+};
+
+template <int D, int BS, int NQ>
+__global__ void __launch_bounds__(256, 1) k_bwd_local_dkdv_tc(const __grid_constant__ BwdMaps maps,
+                                                              const float *__restrict__ lse,
+                                                              const float *__restrict__ dsum,
+                                                              float *__restrict__ dk_loc, float *__restrict__ dv_loc,
+                                                              unsigned long long *__restrict__ counters, int S, int L,
+                                                              float scale_log2, int nbh) {
+    using Lay = BwdKvSmem<D, NQ>;
+    static_assert(Lay::supported, "tile shape");
+    constexpr int KB = Lay::KB, QB = Lay::QB, HALF = NQ / 2, DH = D / 2;
+    static_assert(HALF % 32 == 0 && DH % 32 == 0, "column halves of 32");
+    extern __shared__ __align__(1024) uint8_t smem[];
+    uint8_t *sK = smem + Lay::K_OFF, *sV = smem + Lay::V_OFF, *sQ = smem + Lay::Q_OFF;
+    uint8_t *sDOH = smem + Lay::DOH_OFF, *sDOL = smem + Lay::DOL_OFF, *sP = smem + Lay::P_OFF, *sDS = smem + Lay::DS_OFF;
+    float *s_lse = (float *)(smem + Lay::LSE_OFF), *s_D = (float *)(smem + Lay::DD_OFF);
+    uint64_t *bar_ld = (uint64_t *)(smem + Lay::BAR_OFF), *mbar = bar_ld + 1;
+    uint32_t *tmem_base = (uint32_t *)(bar_ld + 2);
+    if (timed_out(counters)) return;
+    if (tc::smem_u32(smem) & 1023) {
+        if (threadIdx.x == 0) record_error(counters, kDevErrSmemAlign);
+        return;
+    }
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quarter = warp & 3, half = warp >> 2;
+    const int row = quarter * 32 + lane;
+    const int ntiles = (S + 127) / 128;
+    const int total = nbh * ntiles;
+    if (warp == 0) {
+        tc::tmem_alloc(tmem_base, 512);
+        tc::tmem_relinquish();
+    }
+    if (tid == 0) {
+        tc::mbar_init(bar_ld, 1);
+        tc::mbar_init(mbar, 1);
+        tc::fence_mbar_init();
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = *tmem_base;
+    const uint32_t trow = tmem + ((uint32_t)(quarter * 32) << 16);
+    // S^T, dP^T, dV and dK columns of this lane quarter
+    const uint32_t tS = trow, tP = trow + NQ, tV = trow + 2 * NQ, tK = trow + 2 * NQ + D;
+    bool ok = true;
+    int pend = -1;     // thread 0: the load of tile k issued and not yet seen complete
+    uint32_t mph = 0;  // completions of mbar so far, mod 2
+    int k = 0;
+    for (int f = blockIdx.x; f < total && ok; f += gridDim.x, ++k) {
+        const int bh = f / ntiles, k0 = (f % ntiles) * 128;
+        const int s = k0 + row;  // this thread's key
+        const bool live = s < S;
+        if (tid == 0) {
+            tc::mbar_expect_tx(bar_ld, 2 * KB + 3 * QB);
+#pragma unroll
+            for (int a = 0; a < D / 64; ++a) {
+                tc::tma_load_3d(sK + a * (128 * 128), &maps.k, 64 * a, k0, bh, bar_ld);
+                tc::tma_load_3d(sV + a * (128 * 128), &maps.v, 64 * a, k0, bh, bar_ld);
+                tc::tma_load_3d(sQ + a * (NQ * 128), &maps.q, 64 * a, k0, bh, bar_ld);
+                tc::tma_load_3d(sDOH + a * (NQ * 128), &maps.dohi, 64 * a, k0, bh, bar_ld);
+                tc::tma_load_3d(sDOL + a * (NQ * 128), &maps.dolo, 64 * a, k0, bh, bar_ld);
+            }
+            pend = k;
+        }
+        // the queries' log-sum-exp (exp2 domain) and D
+        for (int c = tid; c < NQ; c += 256) {
+            const int t = k0 + c;
+            s_lse[c] = t < S ? lse[(size_t)bh * S + t] * 1.4426950408889634f : 0.f;
+            s_D[c] = t < S ? dsum[(size_t)bh * S + t] : 0.f;
+        }
+        bool landed = true;
+        if (tid == 0) {
+            landed = tc::mbar_wait(bar_ld, (uint32_t)(k & 1));
+            if (landed) pend = -1;
+        }
+        tc::fence_before_sync();
+        ok = __syncthreads_and(landed);
+        tc::fence_after_sync();
+        if (!ok) break;
+        if (tid == 0) {
+            const uint32_t id = tc::idesc_bf16(128, NQ);
+            const uint32_t ak = tc::smem_u32(sK), av = tc::smem_u32(sV);
+            const uint32_t bq = tc::smem_u32(sQ), bh_ = tc::smem_u32(sDOH), bl = tc::smem_u32(sDOL);
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+                const uint32_t ao = (kk >> 2) * (128 * 128) + (kk & 3) * 32, bo = (kk >> 2) * (NQ * 128) + (kk & 3) * 32;
+                tc::mma_bf16(tmem, tc::desc_sw128(ak + ao), tc::desc_sw128(bq + bo), id, kk > 0);
+                tc::mma_bf16(tmem + NQ, tc::desc_sw128(av + ao), tc::desc_sw128(bh_ + bo), id, kk > 0);
+            }
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+                const uint32_t ao = (kk >> 2) * (128 * 128) + (kk & 3) * 32, bo = (kk >> 2) * (NQ * 128) + (kk & 3) * 32;
+                tc::mma_bf16(tmem + NQ, tc::desc_sw128(av + ao), tc::desc_sw128(bl + bo), id, 1u);
+            }
+            tc::commit(mbar);
+        }
+        ok = __syncthreads_and(tc::mbar_wait(mbar, mph));
+        mph ^= 1u;
+        tc::fence_after_sync();
+        if (!ok) break;
+        // query column c is t = k0 + c; key s is in its window when s <= t < (s / BS + L) BS
+        const int vlo = row, vhi = min((s / BS + L) * BS, S) - 1 - k0;
+        // the hi (lo_terms false) or lo terms of P^T to sP and of dS^T to sDS
+        auto pass = [&](bool lo_terms) {
+#pragma unroll 1
+            for (int c0 = half * HALF; c0 < half * HALF + HALF; c0 += 32) {
+                float sv[32], pv[32];
+                tc::tmem_ld32(tS + c0, sv);
+                tc::tmem_ld32(tP + c0, pv);
+                uint32_t pk[16], dk[16];
+#pragma unroll
+                for (int u = 0; u < 16; ++u) {
+                    const int i = 2 * u;
+                    const bool in0 = live && c0 + i >= vlo && c0 + i <= vhi;
+                    const bool in1 = live && c0 + i + 1 >= vlo && c0 + i + 1 <= vhi;
+                    const float p0 = in0 ? tc::ex2_fast(fmaf(sv[i], scale_log2, -s_lse[c0 + i])) : 0.f;
+                    const float p1 = in1 ? tc::ex2_fast(fmaf(sv[i + 1], scale_log2, -s_lse[c0 + i + 1])) : 0.f;
+                    uint32_t ph, pl, dh, dl;
+                    split2(p0, p1, ph, pl);
+                    split2(p0 * (pv[i] - s_D[c0 + i]), p1 * (pv[i + 1] - s_D[c0 + i + 1]), dh, dl);
+                    pk[u] = lo_terms ? pl : ph;
+                    dk[u] = lo_terms ? dl : dh;
+                }
+#pragma unroll
+                for (int q8 = 0; q8 < 4; ++q8) {
+                    const uint32_t off = tc::kmajor_chunk(row, (c0 >> 3) + q8, NQ);
+                    *(uint4 *)(sP + off) = make_uint4(pk[4 * q8], pk[4 * q8 + 1], pk[4 * q8 + 2], pk[4 * q8 + 3]);
+                    *(uint4 *)(sDS + off) = make_uint4(dk[4 * q8], dk[4 * q8 + 1], dk[4 * q8 + 2], dk[4 * q8 + 3]);
+                }
+            }
+            tc::fence_smem_to_async();
+            tc::fence_before_sync();
+            __syncthreads();
+            tc::fence_after_sync();
+        };
+        pass(false);
+        if (tid == 0) {
+            const uint32_t id = tc::idesc_bf16(128, D, true);
+            const uint32_t ap = tc::smem_u32(sP), ad = tc::smem_u32(sDS);
+            const uint32_t bq = tc::smem_u32(sQ), bh_ = tc::smem_u32(sDOH), bl = tc::smem_u32(sDOL);
+#pragma unroll
+            for (int kk = 0; kk < NQ / 16; ++kk) {
+                const uint64_t pa = tc::desc_kmajor(ap + 256 * kk, NQ), da = tc::desc_kmajor(ad + 256 * kk, NQ);
+                tc::mma_bf16(tmem + 2 * NQ, pa, tc::desc_sw128_mn(bh_ + 2048 * kk, NQ * 128), id, kk > 0);
+                tc::mma_bf16(tmem + 2 * NQ, pa, tc::desc_sw128_mn(bl + 2048 * kk, NQ * 128), id, 1u);
+                tc::mma_bf16(tmem + 2 * NQ + D, da, tc::desc_sw128_mn(bq + 2048 * kk, NQ * 128), id, kk > 0);
+            }
+            tc::commit(mbar);
+        }
+        ok = __syncthreads_and(tc::mbar_wait(mbar, mph));
+        mph ^= 1u;
+        tc::fence_after_sync();
+        if (!ok) break;
+        pass(true);  // sP and sDS are free: the products above have completed
+        if (tid == 0) {
+            const uint32_t id = tc::idesc_bf16(128, D, true);
+            const uint32_t ap = tc::smem_u32(sP), ad = tc::smem_u32(sDS);
+            const uint32_t bq = tc::smem_u32(sQ), bh_ = tc::smem_u32(sDOH);
+#pragma unroll
+            for (int kk = 0; kk < NQ / 16; ++kk) {
+                tc::mma_bf16(tmem + 2 * NQ, tc::desc_kmajor(ap + 256 * kk, NQ),
+                             tc::desc_sw128_mn(bh_ + 2048 * kk, NQ * 128), id, 1u);
+                tc::mma_bf16(tmem + 2 * NQ + D, tc::desc_kmajor(ad + 256 * kk, NQ),
+                             tc::desc_sw128_mn(bq + 2048 * kk, NQ * 128), id, 1u);
+            }
+            tc::commit(mbar);
+        }
+        ok = __syncthreads_and(tc::mbar_wait(mbar, mph));
+        mph ^= 1u;
+        tc::fence_after_sync();
+        if (!ok) break;
+#pragma unroll 1
+        for (int c0 = half * DH; c0 < half * DH + DH; c0 += 32) {
+            float v[32], g[32];
+            tc::tmem_ld32(tV + c0, v);
+            tc::tmem_ld32(tK + c0, g);
+            if (live) {
+                float4 *dv = (float4 *)(dv_loc + ((size_t)bh * S + s) * D + c0);
+                float4 *dk = (float4 *)(dk_loc + ((size_t)bh * S + s) * D + c0);
+#pragma unroll
+                for (int q4 = 0; q4 < 8; ++q4) {
+                    dv[q4] = make_float4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
+                    dk[q4] = make_float4(g[4 * q4], g[4 * q4 + 1], g[4 * q4 + 2], g[4 * q4 + 3]);
+                }
             }
         }
         tc::fence_before_sync();
@@ -1500,6 +1737,48 @@ static cudaError_t launch_bwd_local_dq_shape(const Plan &p, const void *Q, const
     kern<<<std::min(tiles, sms), 256, Lay::BYTES, s>>>(maps, lse, dsum, dq_loc, counters, c.S, c.L, scale_log2, BH);
     count_launches(1);
     return cudaGetLastError();
+}
+
+template <int D, int BS, int NQ>
+static cudaError_t launch_bwd_local_dkdv_shape(const Plan &p, const void *Q, const void *K, const void *V,
+                                               const void *dohi, const void *dolo, const float *lse,
+                                               const float *dsum, float *dk_loc, float *dv_loc,
+                                               unsigned long long *counters, cudaStream_t s) {
+    const mono_config &c = p.cfg;
+    using Lay = BwdKvSmem<D, NQ>;
+    BwdMaps maps;
+    const int BH = c.B * c.H;
+    if (!make_map_3d(&maps.k, K, D, c.S, BH, 128) || !make_map_3d(&maps.v, V, D, c.S, BH, 128) ||
+        !make_map_3d(&maps.q, Q, D, c.S, BH, NQ) || !make_map_3d(&maps.dohi, dohi, D, c.S, BH, NQ) ||
+        !make_map_3d(&maps.dolo, dolo, D, c.S, BH, NQ))
+        return cudaErrorInvalidValue;
+    auto kern = k_bwd_local_dkdv_tc<D, BS, NQ>;
+    cudaError_t e;
+    if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::BYTES)) != cudaSuccess)
+        return e;
+    int dev = 0, sms = 148;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+        return e;
+    const int tiles = BH * ((c.S + 127) / 128);
+    const float scale_log2 = (float)(1.4426950408889634 / sqrt((double)c.d));
+    kern<<<std::min(tiles, sms), 256, Lay::BYTES, s>>>(maps, lse, dsum, dk_loc, dv_loc, counters, c.S, c.L,
+                                                       scale_log2, BH);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_bwd_local_dkdv_tc(const Plan &p, const void *Q, const void *K, const void *V, const void *dohi,
+                                     const void *dolo, const float *lse, const float *dsum, float *dk_loc,
+                                     float *dv_loc, unsigned long long *counters, cudaStream_t s) {
+    const mono_config &c = p.cfg;
+    if (!bwd_local_dq_tc_supported(c)) return cudaErrorInvalidValue;
+    const int nq = 128 + (c.L - 1) * c.Bs;
+    if (c.d == 64 && nq <= 128)
+        return launch_bwd_local_dkdv_shape<64, 64, 128>(p, Q, K, V, dohi, dolo, lse, dsum, dk_loc, dv_loc, counters, s);
+    if (c.d == 64)
+        return launch_bwd_local_dkdv_shape<64, 64, 192>(p, Q, K, V, dohi, dolo, lse, dsum, dk_loc, dv_loc, counters, s);
+    return launch_bwd_local_dkdv_shape<128, 64, 128>(p, Q, K, V, dohi, dolo, lse, dsum, dk_loc, dv_loc, counters, s);
 }
 
 bool bwd_local_dq_tc_supported(const mono_config &c) {

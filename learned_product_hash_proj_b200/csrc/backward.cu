@@ -11,13 +11,20 @@
 //     D_t = dO_t . O_t,   dS_ts = P_ts (dO_t . v_s - D_t),
 //     dQ_t = scale sum_s dS_ts k_s,   dK_s += scale dS_ts q_t,   dV_s += P_ts dO_t.
 // Kernels (fp32 arithmetic, gradients in fp32):
+//   k_bwd_prep   with the forward recompute's fp32 O and log-sum-exp: D per
+//                row and dO head-major as two bf16 terms, for the tensor-core
+//                kernels of the local keys (k_bwd_local_dq_tc and
+//                k_bwd_local_dkdv_tc, in attend_tc.cu);
 //   k_bwd_dq     d/16 lanes per query-head: log-sum-exp and D from recomputed
-//                scores (the stored O is not needed), then dQ;
+//                scores (the stored O is not needed) or from the recompute,
+//                then dQ over the remote blocks and the local keys (or the
+//                tensor cores' local part);
 //   k_bwd_count / k_bwd_scan / k_bwd_fill: per (b, h) and block j, the
 //                queries that selected j (lists in unspecified order);
 //   k_bwd_dkdv   one CTA per (b, h) and tile of up to 64 keys of one block:
-//                walks the block's local queries and its selecting queries,
-//                accumulating dK and dV of its keys in registers;
+//                walks the block's local queries (or starts from the tensor
+//                cores' local part) and its selecting queries, accumulating
+//                dK and dV of its keys in registers;
 //   (dq, dk and dv leave these kernels either as [B,H,S,d] for the post-RoPE
 //   q and k, or rotated back and token-major for the projection gradients)
 //   k_gemm_any   the projection gradients of fp32 storage (generic strided SIMT
@@ -38,7 +45,7 @@ namespace mono {
 namespace {
 
 struct BwdLayout {
-    size_t lse, dsum, cnt, start, cursor, list, dO, dQp, dKp, dVp, dOhi, dOlo, dQloc, total;
+    size_t lse, dsum, cnt, start, cursor, list, dO, dQp, dKp, dVp, dOhi, dOlo, dQloc, dVloc, total;
 };
 
 BwdLayout bwd_layout(const Plan &p) {
@@ -61,10 +68,12 @@ BwdLayout bwd_layout(const Plan &p) {
     L.dQp = take(B * S * H * d * 4);
     L.dKp = take(B * S * H * d * 4);
     L.dVp = take(B * S * H * d * 4);
-    // the tensor-core local dQ: dO as two bf16 terms and its fp32 result, head-major [B*H, S, d]
+    // the tensor-core local parts: dO as two bf16 terms, the local dQ (then the local dK) and the local dV in
+    // fp32, all head-major [B*H, S, d]
     L.dOhi = take(B * H * S * d * 2);
     L.dOlo = take(B * H * S * d * 2);
     L.dQloc = take(B * H * S * d * 4);
+    L.dVloc = take(B * H * S * d * 4);
     L.total = o;
     return L;
 }
@@ -465,8 +474,9 @@ template <typename T, int DD>
 __global__ void __launch_bounds__(kBwdKT * DD / 16, DD == 64 ? 2 : 1) k_bwd_dkdv(
     const T *__restrict__ Q, const T *__restrict__ K, const T *__restrict__ V, const float *__restrict__ dO,
     const float *__restrict__ lse, const float *__restrict__ dsum, const int32_t *__restrict__ cnt,
-    const int32_t *__restrict__ start, const int32_t *__restrict__ list, const GradOut go, int B, int H, int S,
-    int Bs, int L, int R, int nb, float scale) {
+    const int32_t *__restrict__ start, const int32_t *__restrict__ list, const GradOut go,
+    const float *__restrict__ dk_loc, const float *__restrict__ dv_loc, int B, int H, int S, int Bs, int L, int R,
+    int nb, float scale) {
     constexpr int TPK = DD / 16, NT = kBwdKT * TPK, E = 16;
     constexpr int PER = kBwdQG * DD / NT;  // staged elements per thread and array (one dimension, PER queries)
     constexpr int SEG = 20, ROW = TPK * SEG;  // padded segment and row, in floats
@@ -492,7 +502,18 @@ __global__ void __launch_bounds__(kBwdKT * DD / 16, DD == 64 ? 2 : 1) k_bwd_dkdv
         dk[e] = 0.f;
         dv[e] = 0.f;
     }
-    const int t_loc0 = j * Bs, t_loc1 = min(S, (j + L) * Bs);  // local queries [t_loc0, t_loc1)
+    // the local queries' part from the tensor cores (dk_loc without the 1/sqrt(d) factor), or walked here
+    if (dk_loc && live) {
+        float a[E], g[E];
+        load16<float>(dk_loc + (bh * S + key) * DD + e0, a);
+        load16<float>(dv_loc + (bh * S + key) * DD + e0, g);
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+            dk[e] = a[e] * scale;
+            dv[e] = g[e];
+        }
+    }
+    const int t_loc0 = j * Bs, t_loc1 = dk_loc ? t_loc0 : min(S, (j + L) * Bs);  // local queries [t_loc0, t_loc1)
     const int nloc = t_loc1 - t_loc0;
     const int nrem = R > 0 ? cnt[bh * nb + j] : 0;
     const int rem0 = R > 0 ? start[bh * nb + j] : 0;
@@ -711,14 +732,23 @@ cudaError_t attend_backward(const Plan &p, const T *Q, const T *K, const T *V, c
         k_bwd_fill<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(sel, cursor, list, n, c.S, c.R, p.nb, c.Bs, c.L);
         count_launches(3);
     }
+    // the local queries' part of dK and dV on the tensor cores (dK into the local dQ's region, read by now)
+    float *dk_loc = nullptr, *dv_loc = nullptr;
+    if (dq_loc) {
+        dk_loc = dq_loc;
+        dv_loc = (float *)(bws + L.dVloc);
+        if ((e = launch_bwd_local_dkdv_tc(p, Q, K, V, bws + L.dOhi, bws + L.dOlo, lse, dsum, dk_loc, dv_loc, counters,
+                                          s)) != cudaSuccess)
+            return e;
+    }
     const int tpb = (c.Bs + kBwdKT - 1) / kBwdKT;
     const dim3 gk(tpb * p.nb, c.H, c.B);
     if (c.d == 64)
-        k_bwd_dkdv<T, 64><<<gk, kBwdKT * 4, 0, s>>>(Q, K, V, dO, lse, dsum, cnt, start, list, go, c.B, c.H, c.S,
-                                                     c.Bs, c.L, c.R, p.nb, scale);
+        k_bwd_dkdv<T, 64><<<gk, kBwdKT * 4, 0, s>>>(Q, K, V, dO, lse, dsum, cnt, start, list, go, dk_loc, dv_loc, c.B,
+                                                     c.H, c.S, c.Bs, c.L, c.R, p.nb, scale);
     else
-        k_bwd_dkdv<T, 128><<<gk, kBwdKT * 8, 0, s>>>(Q, K, V, dO, lse, dsum, cnt, start, list, go, c.B, c.H, c.S,
-                                                      c.Bs, c.L, c.R, p.nb, scale);
+        k_bwd_dkdv<T, 128><<<gk, kBwdKT * 8, 0, s>>>(Q, K, V, dO, lse, dsum, cnt, start, list, go, dk_loc, dv_loc,
+                                                      c.B, c.H, c.S, c.Bs, c.L, c.R, p.nb, scale);
     count_launches(1);
     return cudaGetLastError();
 }

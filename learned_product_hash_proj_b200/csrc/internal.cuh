@@ -149,6 +149,11 @@ bool bwd_local_dq_tc_supported(const mono_config &c);
 cudaError_t launch_bwd_local_dq_tc(const Plan &p, const void *Q, const void *K, const void *V, const void *dohi,
                                   const void *dolo, const float *lse, const float *dsum, float *dq_loc,
                                   unsigned long long *counters, cudaStream_t s);
+// the same for dK and dV, key-major: dk_loc, dv_loc [B*H, S, d] fp32 = sum over the queries whose local window
+// holds the key of dS q (without the 1/sqrt(d) factor) and P dO; shapes where bwd_local_dq_tc_supported
+cudaError_t launch_bwd_local_dkdv_tc(const Plan &p, const void *Q, const void *K, const void *V, const void *dohi,
+                                     const void *dolo, const float *lse, const float *dsum, float *dk_loc,
+                                     float *dv_loc, unsigned long long *counters, cudaStream_t s);
 cudaError_t launch_attend_tc(const Plan &p, const void *Q, const void *K, const void *V, const int32_t *sel, void *O,
                              void *ws, cudaStream_t s, int parts = kAttendAll, float *o32 = nullptr,
                              float *lse = nullptr, bool *stats = nullptr);
