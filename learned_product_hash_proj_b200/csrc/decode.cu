@@ -395,9 +395,15 @@ __global__ void __launch_bounds__(32) k_dec_route(const T *__restrict__ q, const
         tc::cp_async_wait_all();
         __syncwarp();
         if (lane < ne) {
-            float a = 0.0f;
-            for (int i = 0; i < d; ++i) a = __fmaf_rn(s_q[i], s_kb[lane][i], a);
-            s_score[e0 + lane] = a;
+            // eight runs of d/8 elements as fma chains, added as a balanced tree (the batch rerank's order)
+            float run[8];
+            for (int l = 0; l < 8; ++l) {
+                float a = 0.0f;
+                for (int i = l * d / 8; i < (l + 1) * d / 8; ++i) a = __fmaf_rn(s_q[i], s_kb[lane][i], a);
+                run[l] = a;
+            }
+            s_score[e0 + lane] = __fadd_rn(__fadd_rn(__fadd_rn(run[0], run[1]), __fadd_rn(run[2], run[3])),
+                                           __fadd_rn(__fadd_rn(run[4], run[5]), __fadd_rn(run[6], run[7])));
         }
         __syncwarp();
     }

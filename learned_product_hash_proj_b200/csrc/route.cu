@@ -671,15 +671,23 @@ __global__ void __launch_bounds__(128) k_probe_rerank(const T *__restrict__ Q, c
         for (int k = 0; k < nc && R > 0; ++k) {
             const int j = cand[k];
             const float4 *kr = (const float4 *)(kbar + (bh * nb + j) * D);
-            float acc = 0.0f;
+            // eight runs of D/8 elements as fma chains, added as a balanced tree
+            float run[8];
 #pragma unroll
-            for (int i4 = 0; i4 < D / 4; ++i4) {
-                float4 v = __ldg(kr + i4);
-                acc = __fmaf_rn(q[4 * i4 + 0], v.x, acc);
-                acc = __fmaf_rn(q[4 * i4 + 1], v.y, acc);
-                acc = __fmaf_rn(q[4 * i4 + 2], v.z, acc);
-                acc = __fmaf_rn(q[4 * i4 + 3], v.w, acc);
+            for (int l = 0; l < 8; ++l) {
+                float acc = 0.0f;
+#pragma unroll
+                for (int i4 = l * (D / 32); i4 < (l + 1) * (D / 32); ++i4) {
+                    const float4 v = __ldg(kr + i4);
+                    acc = __fmaf_rn(q[4 * i4 + 0], v.x, acc);
+                    acc = __fmaf_rn(q[4 * i4 + 1], v.y, acc);
+                    acc = __fmaf_rn(q[4 * i4 + 2], v.z, acc);
+                    acc = __fmaf_rn(q[4 * i4 + 3], v.w, acc);
+                }
+                run[l] = acc;
             }
+            const float acc = __fadd_rn(__fadd_rn(__fadd_rn(run[0], run[1]), __fadd_rn(run[2], run[3])),
+                                        __fadd_rn(__fadd_rn(run[4], run[5]), __fadd_rn(run[6], run[7])));
             if (nr == R && !(acc > rv[R - 1] || (acc == rv[R - 1] && j < ra[R - 1]))) continue;
             int pos = nr < R ? nr : R - 1;
             while (pos > 0 && (acc > rv[pos - 1] || (acc == rv[pos - 1] && j < ra[pos - 1]))) {
@@ -956,41 +964,27 @@ template <int C>
 constexpr int probe_nq() {
     return C <= 16 ? 2 : 1;
 }
-template <typename T, int D, int C>
+// shared memory of the probe's candidates: ids (int16), counts, rerank scores
+template <int E>
+constexpr size_t cand_smem(int nq) {
+    return ((size_t)nq * E * 2 + 15) / 16 * 16 + (size_t)nq * 4 + (size_t)nq * E * 4;
+}
+static_assert(kMaxNb <= 32768, "block ids fit int16");
+
+template <typename T, int D, int C, int E>
 constexpr size_t probe_m2_smem(int nb) {
     return (size_t)C * D * 4 + (size_t)C * C * 8 + (size_t)128 * probe_nq<C>() * probe_q_pitch<T, D>() +
-           (size_t)nb * 8;
+           cand_smem<E>(128 * probe_nq<C>()) + (size_t)nb * 8;
 }
 
-// The rerank q . kbar_j of the (at most E) candidates cid[0 .. nc) of
-// query-head t, their fma chains advancing together in ascending element
-// order; top R (score desc, id asc); the forced block; sel in ascending order
-// with -1 padding.  Returns the number of remote blocks selected and adds 1
-// to *ign when a forced id was not eligible.
-template <typename T, int D, int E, int R>
-__device__ __forceinline__ int rerank_m2(const T *qp, const float *kb, const int (&cid)[E], int nc,
-                                         const int32_t *forced, int32_t *out, int t, size_t bh, int S, int Bs, int L,
-                                         int *ign) {
+// Top R of the candidates' rerank scores acc (score desc, id asc), the forced
+// block, sel in ascending order with -1 padding.  Returns the number of remote
+// blocks selected and adds 1 to *ign when a forced id was not eligible.
+template <int E, int R>
+__device__ __forceinline__ int select_top_r(const float (&acc)[E], const int (&cid)[E], int nc,
+                                            const int32_t *forced, int32_t *out, int t, size_t bh, int S, int Bs,
+                                            int L, int *ign) {
     const int lim = t / Bs - L;
-    float acc[E];
-#pragma unroll
-    for (int e = 0; e < E; ++e) acc[e] = 0.0f;
-#pragma unroll 2
-    for (int i8 = 0; i8 < D / 8; ++i8) {
-        float qv[8];
-        q8<T>(qp + 8 * i8, qv);
-#pragma unroll
-        for (int e = 0; e < E; ++e) {
-            if (e < nc) {
-                float kv[8];  // one 32-byte load (the rows are 32-byte aligned)
-                tc::ldg_v8(kb + (size_t)cid[e] * D + 8 * i8, kv);
-                float a = acc[e];
-#pragma unroll
-                for (int i = 0; i < 8; ++i) a = __fmaf_rn(qv[i], kv[i], a);
-                acc[e] = a;
-            }
-        }
-    }
     RegTop<R> rk;
     rk.init();
 #pragma unroll
@@ -1033,15 +1027,152 @@ __device__ __forceinline__ int rerank_m2(const T *qp, const float *kb, const int
     return nr;
 }
 
-// The probe, union, causal filter, E cap and rerank of one query-head t from
-// its subspace scores (see k_probe_m2).  Writes sel; returns the number of
-// remote blocks selected and sets *ign when a forced id was not eligible.
-template <typename T, int D, int C, int TP, int E, int R>
-__device__ __forceinline__ int route_query_m2(const float (&s0)[C], const float (&s1)[C], const T *qp,
-                                              const int2 *s_rng, const int32_t *s_ids, const float *kb,
-                                              const int32_t *forced, int32_t *out, int t, size_t bh, int S,
-                                              int Bs, int L, int cap, unsigned long long *counters,
-                                              int32_t *walk_log, int *ign) {
+// The rerank scores of the query-heads a warp probed (its threads' rows
+// qi = tid + 128 q, q < NQ, of the CTA's tile; each one's candidates in
+// s_cid[qi][E], their number in s_nc[qi]) into s_score[qi][E], eight lanes
+// per query-head: lane l of a group holds run l (elements [l D/8, (l+1) D/8))
+// of q and reads the same run of each candidate's kbar row, so a group reads
+// whole rows.  Its fma chain is the run's value, and three butterfly additions
+// form the tree ((c0 + c1) + (c2 + c3)) + ((c4 + c5) + (c6 + c7)) in every
+// lane of the group (fp32 addition is commutative, so both partners get the
+// same bits).  Four query-heads per round, two rounds' loads in flight.
+template <typename T, int D, int E, int NQ>
+__device__ __forceinline__ void rerank_scores(const uint8_t *s_q, int qpitch, const int16_t *s_cid,
+                                              const int32_t *s_nc, const float *kb, float *s_score) {
+    constexpr int RUN = D / 8, RPI = 2;
+    static_assert(RUN % 8 == 0 && (8 * NQ) % RPI == 0, "runs of whole 8-element chunks");
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, grp = lane >> 3, run = lane & 7;
+#pragma unroll 1
+    for (int r0 = 0; r0 < 8 * NQ; r0 += RPI) {
+        int qi[RPI], nc[RPI];
+        float qv[RPI][RUN], acc[RPI][E];
+#pragma unroll
+        for (int h = 0; h < RPI; ++h) {
+            const int wq = 4 * (r0 + h) + grp;
+            qi[h] = 32 * warp + (wq & 31) + 128 * (wq >> 5);
+            nc[h] = s_nc[qi[h]];
+#pragma unroll
+            for (int i8 = 0; i8 < RUN / 8; ++i8) {
+                float v8[8];
+                q8<T>((const T *)(s_q + qi[h] * qpitch) + run * RUN + 8 * i8, v8);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) qv[h][8 * i8 + i] = v8[i];
+            }
+        }
+#pragma unroll
+        for (int h = 0; h < RPI; ++h)
+#pragma unroll
+            for (int e = 0; e < E; ++e) {
+                float a = 0.0f;
+                if (e < nc[h]) {
+                    const float *row = kb + (size_t)s_cid[qi[h] * E + e] * D + run * RUN;
+#pragma unroll
+                    for (int i8 = 0; i8 < RUN / 8; ++i8) {
+                        float kv[8];
+                        tc::ldg_v8(row + 8 * i8, kv);
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) a = __fmaf_rn(qv[h][8 * i8 + i], kv[i], a);
+                    }
+                }
+                acc[h][e] = a;
+            }
+#pragma unroll
+        for (int h = 0; h < RPI; ++h)
+#pragma unroll
+            for (int e = 0; e < E; ++e) {
+                float a = acc[h][e];
+                a = __fadd_rn(a, __shfl_xor_sync(0xffffffffu, a, 1));
+                a = __fadd_rn(a, __shfl_xor_sync(0xffffffffu, a, 2));
+                a = __fadd_rn(a, __shfl_xor_sync(0xffffffffu, a, 4));
+                acc[h][e] = a;
+            }
+        if (run == 0) {
+#pragma unroll
+            for (int h = 0; h < RPI; ++h)
+#pragma unroll
+                for (int e = 0; e < E; ++e) s_score[qi[h] * E + e] = acc[h][e];
+        }
+    }
+}
+
+// The rerank q . kbar_j of the (at most E) candidates cid[0 .. nc) of
+// query-head t by one thread, in the order of rerank_scores: the eight runs
+// of D/8 elements each as an fma chain from +0 (the candidates' chains
+// advancing together), the run values added as ((c0 + c1) + (c2 + c3)) +
+// ((c4 + c5) + (c6 + c7)); then select_top_r.
+template <typename T, int D, int E, int R>
+__device__ __forceinline__ int rerank_thread(const T *qp, const float *kb, const int (&cid)[E], int nc,
+                                             const int32_t *forced, int32_t *out, int t, size_t bh, int S, int Bs,
+                                             int L, int *ign) {
+    static_assert(D % 64 == 0, "runs of whole 8-element chunks");
+    constexpr int CPR = D / 64;  // 8-element chunks per run
+    float acc[E], half0[E], pair1[E];
+    // runs 2p and 2p + 1 per step: their loads in flight together
+#pragma unroll 1
+    for (int p = 0; p < 4; ++p) {
+        float c[2][E];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+#pragma unroll
+            for (int e = 0; e < E; ++e) c[h][e] = 0.0f;
+#pragma unroll
+            for (int k = 0; k < CPR; ++k) {
+                const int i8 = (2 * p + h) * CPR + k;
+                float qv[8];
+                q8<T>(qp + 8 * i8, qv);
+#pragma unroll
+                for (int e = 0; e < E; ++e) {
+                    if (e < nc) {
+                        float kv[8];  // one 32-byte load (the rows are 32-byte aligned)
+                        tc::ldg_v8(kb + (size_t)cid[e] * D + 8 * i8, kv);
+                        float a = c[h][e];
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) a = __fmaf_rn(qv[i], kv[i], a);
+                        c[h][e] = a;
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+            const float pr = __fadd_rn(c[0][e], c[1][e]);  // c_2p + c_2p+1
+            if (p == 0 || p == 2) pair1[e] = pr;
+            else if (p == 1) half0[e] = __fadd_rn(pair1[e], pr);
+            else acc[e] = __fadd_rn(half0[e], __fadd_rn(pair1[e], pr));  // p == 3: the score
+        }
+    }
+    return select_top_r<E, R>(acc, cid, nc, forced, out, t, bh, S, Bs, L, ign);
+}
+
+// The top-R selection of this thread's query-heads (rows tid + 128 q) from
+// their candidates and rerank scores in shared memory; adds to the counts.
+template <int E, int R, int NQ>
+__device__ __forceinline__ void select_rows(const int16_t *s_cid, const int32_t *s_nc, const float *s_score,
+                                            const int32_t *forced, int32_t *sel, int t_lo, size_t bh, int S, int Bs,
+                                            int L, int &n_sel, int &lt_r, int &ign) {
+#pragma unroll
+    for (int q = 0; q < NQ; ++q) {
+        const int qi = threadIdx.x + 128 * q, t = t_lo + qi;
+        if (t >= S) continue;
+        int cid[E];
+        float acc[E];
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+            cid[e] = s_cid[qi * E + e];
+            acc[e] = s_score[qi * E + e];
+        }
+        const int nr = select_top_r<E, R>(acc, cid, s_nc[qi], forced, sel + (bh * S + t) * R, t, bh, S, Bs, L, &ign);
+        n_sel += nr;
+        lt_r += nr < R;
+    }
+}
+
+// The probe, union, causal filter and E cap of one query-head t from its
+// subspace scores (see k_probe_m2): the candidates in cid[0 .. nc), nc returned.
+template <int C, int TP, int E>
+__device__ __forceinline__ int probe_m2(const float (&s0)[C], const float (&s1)[C], const int2 *s_rng,
+                                        const int32_t *s_ids, int (&cid)[E], int t, size_t bh, int S, int Bs, int L,
+                                        int cap, unsigned long long *counters, int32_t *walk_log) {
     constexpr int A = C * C;
     float mx0 = 0.f, mx1 = 0.f;
 #pragma unroll
@@ -1116,10 +1247,9 @@ __device__ __forceinline__ int route_query_m2(const float (&s0)[C], const float 
         }
     }
 
-    // union of the probed lists in probe order, causal filter, E cap ...
+    // union of the probed lists in probe order, causal filter, E cap
     const int bq = t / Bs;
     const int lim = bq - L;
-    int cid[E];
 #pragma unroll
     for (int e = 0; e < E; ++e) cid[e] = 0;
     int nc = 0;
@@ -1141,8 +1271,7 @@ __device__ __forceinline__ int route_query_m2(const float (&s0)[C], const float 
             ++nc;
         }
     }
-    // ... and the rerank
-    return rerank_m2<T, D, E, R>(qp, kb, cid, nc, forced, out, t, bh, S, Bs, L, ign);
+    return nc;
 }
 
 // M = 2 with every size fixed at compile time, so all per-query state stays
@@ -1167,7 +1296,10 @@ __global__ void __launch_bounds__(128, C <= 16 ? 4 : 3) k_probe_m2(const T *__re
     float *s_cbT = smem;                                 // [2][DM][C]: element i of codeword (m, c) at (m DM + i) C + c
     int2 *s_rng = (int2 *)(s_cbT + C * D);               // [A] positions [first, end) of each address's entries
     uint8_t *s_q = (uint8_t *)(s_rng + A);               // [QT] query rows, pitch QP
-    int32_t *s_addr = (int32_t *)(s_q + QT * QP);        // [nb]
+    int16_t *s_cid = (int16_t *)(s_q + QT * QP);         // [QT][E] candidates of each query-head
+    int32_t *s_nc = (int32_t *)(s_q + QT * QP + (QT * E * 2 + 15) / 16 * 16);  // [QT] their number
+    float *s_score = (float *)(s_nc + QT);               // [QT][E] their rerank scores
+    int32_t *s_addr = (int32_t *)(s_score + QT * E);     // [nb]
     int32_t *s_ids = s_addr + nb;                        // [nb]
     const int h = blockIdx.y, b = blockIdx.z;
     const size_t bh = (size_t)b * H + h;
@@ -1237,19 +1369,22 @@ __global__ void __launch_bounds__(128, C <= 16 ? 4 : 3) k_probe_m2(const T *__re
         if (i == nb - 1 || s_addr[i + 1] != a) s_rng[a].y = i + 1;
     }
     __syncthreads();
-    int n_sel = 0, lt_r = 0, ign = 0;
-    const float *kb = kbar + bh * nb * D;
 #pragma unroll
     for (int q = 0; q < NQ; ++q) {
-        const int t = t_lo + tid + 128 * q;
-        if (t < S) {
-            const int nr = route_query_m2<T, D, C, TP, E, R>(s0[q], s1[q], (const T *)(s_q + (tid + 128 * q) * QP),
-                                                             s_rng, s_ids, kb, forced, sel + (bh * S + t) * R, t, bh,
-                                                             S, Bs, L, cap, counters, walk_log, &ign);
-            n_sel += nr;
-            lt_r += nr < R;
-        }
+        const int qi = tid + 128 * q, t = t_lo + qi;
+        int cid[E] = {};
+        const int nc = t < S ? probe_m2<C, TP, E>(s0[q], s1[q], s_rng, s_ids, cid, t, bh, S, Bs, L, cap, counters,
+                                                  walk_log)
+                             : 0;
+#pragma unroll
+        for (int e = 0; e < E; ++e) s_cid[qi * E + e] = (int16_t)cid[e];
+        s_nc[qi] = nc;
     }
+    __syncwarp();
+    rerank_scores<T, D, E, NQ>(s_q, QP, s_cid, s_nc, kbar + bh * nb * D, s_score);
+    __syncwarp();
+    int n_sel = 0, lt_r = 0, ign = 0;
+    select_rows<E, R, NQ>(s_cid, s_nc, s_score, forced, sel, t_lo, bh, S, Bs, L, n_sel, lt_r, ign);
     for (int o = 16; o > 0; o >>= 1) {
         n_sel += __shfl_xor_sync(0xffffffffu, n_sel, o);
         lt_r += __shfl_xor_sync(0xffffffffu, lt_r, o);
@@ -1613,8 +1748,8 @@ __global__ void __launch_bounds__(128) k_probe_bf(const T *__restrict__ Q, const
                 ++nc;
             }
         }
-        const int nr = rerank_m2<T, D, E, R>(qrow, kbar + bh * nb * D, cid, nc, forced, sel + (bh * S + t) * R, t,
-                                             bh, S, Bs, L, &ign);
+        const int nr = rerank_thread<T, D, E, R>(qrow, kbar + bh * nb * D, cid, nc, forced, sel + (bh * S + t) * R, t,
+                                                 bh, S, Bs, L, &ign);
         n_sel = nr;
         lt_r = nr < R;
     }
@@ -1769,7 +1904,7 @@ cudaError_t launch_queries(const Plan &p, const void *Q, const float *cb, const 
     // compile-time shapes of the configured workloads; any other shape takes the general kernel
 #define MONO_M2(TT, DD, CC, TPP, EE, RR)                                                                          \
     if (c.M == 2 && c.d == DD && c.C == CC && c.T == TPP && c.E == EE && c.R == RR) {                           \
-        const size_t sm2 = probe_m2_smem<TT, DD, CC>(p.nb);                                                     \
+        const size_t sm2 = probe_m2_smem<TT, DD, CC, EE>(p.nb);                                                 \
         auto kern = k_probe_m2<TT, DD, CC, TPP, EE, RR>;                                                        \
         if (sm2 > 48 * 1024 &&                                                                                   \
             (e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm2)) != cudaSuccess) \

@@ -25,8 +25,10 @@
  *     codeword scores, grid scores, rerank scores) is computed in fp32 in the
  *     plain order this library specifies: sums in ascending index order, dot
  *     products as a chain of fused multiply-adds starting from +0.0f in
- *     ascending element order.  Build with -ffp-contract=off so that no other
- *     contraction happens.
+ *     ascending element order, except the rerank score <q, kbar_j>, which is
+ *     eight such chains over the eight contiguous runs of the vector added as
+ *     a balanced tree (dot_tree8).  Build with -ffp-contract=off so that no
+ *     other contraction happens.
  *   - A second statement of the routing (orc_summary_assign64,
  *     orc_route_queries64) takes the same decisions in fp64 from the stored
  *     Q, K and codebooks: the plain-precision reference against which the
@@ -135,6 +137,19 @@ static float dot_fma(const float *a, const float *b, int n)
     float acc = 0.0f;
     for (int i = 0; i < n; ++i) acc = fmaf(a[i], b[i], acc);
     return acc;
+}
+
+/* The rerank score's order: run l = elements [l*n/8, (l+1)*n/8) (integer     */
+/* division) as an fma chain from +0.0f (dot_fma), then the eight run values */
+/* added as ((c0 + c1) + (c2 + c3)) + ((c4 + c5) + (c6 + c7)) in fp32.      */
+static float dot_tree8(const float *a, const float *b, int n)
+{
+    float c[8];
+    for (int l = 0; l < 8; ++l) {
+        const int lo = (int)((long)l * n / 8), hi = (int)((long)(l + 1) * n / 8);
+        c[l] = dot_fma(a + lo, b + lo, hi - lo);
+    }
+    return ((c[0] + c[1]) + (c[2] + c[3])) + ((c[4] + c[5]) + (c[6] + c[7]));
 }
 
 int orc_summary_assign(const orc_cfg *c, const float *K, const float *cb,
@@ -288,7 +303,7 @@ int orc_posting_redirect(const orc_cfg *c, const int32_t *addr, int32_t *list_ad
 /*     first T are the probes.                                               */
 /*  3. walk the probes in rank order, each kept list in ascending block id;  */
 /*     keep block j iff j <= bq - L (bq = t / Bs); stop after E candidates.  */
-/*  4. rerank score <q, kbar_j> (fp32 fma chain); order (score desc, j asc); */
+/*  4. rerank score <q, kbar_j> (fp32, dot_tree8); order (score desc, j asc);*/
 /*     keep the first R; optional forced block (see below); emit ascending, */
 /*     pad with -1.                                                          */
 /* Forced block ([P1] Key Points, forcing the labelled target under the      */
@@ -405,7 +420,7 @@ int orc_route_queries(const orc_cfg *c, const float *Q, const float *kbar, const
         if (ncand) ncand[qi] = nc;
         /* 4. rerank */
         for (int k = 0; k < nc; ++k) {
-            rr[k].g = dot_fma(q, kbar + (bh * nb + cand[k]) * (long)d, d);
+            rr[k].g = dot_tree8(q, kbar + (bh * nb + cand[k]) * (long)d, d);
             rr[k].a = cand[k];
         }
         qsort(rr, (size_t)nc, sizeof(ga_pair), cmp_ga);

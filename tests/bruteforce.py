@@ -11,7 +11,7 @@ import itertools
 
 import numpy as np
 
-from fp32_exact import add32, div32, dot_chain32
+from fp32_exact import add32, div32, dot_chain32, dot_tree32
 
 
 def summaries(K_bh, Bs):
@@ -62,8 +62,10 @@ def redirect_lists(addr, A, cap):
     return lists, overflow
 
 
-def route_bh(Q_bh, K_bh, cw_h, cfg, forced_bh=None, redirect=False):
-    """Route every query of one (batch, head).  Returns (addr, lists, overflow, sel)."""
+def route_bh(Q_bh, K_bh, cw_h, cfg, forced_bh=None, redirect=False, rerank_margins=None, rerank_dot=dot_tree32):
+    """Route every query of one (batch, head).  Returns (addr, lists, overflow, sel).  With a list given as
+    rerank_margins, appends each query's fp32 rerank margin: score(R-th) - score((R+1)-th) when more than R
+    candidates remain, else +inf (rerank_dot: the fp32 dot product the scores use)."""
     S, d = Q_bh.shape
     Bs, M, C, T, R, E, L, cap = cfg.Bs, cfg.M, cfg.C, cfg.T, cfg.R, cfg.E, cfg.L, cfg.cap
     nb = S // Bs
@@ -99,7 +101,11 @@ def route_bh(Q_bh, K_bh, cw_h, cfg, forced_bh=None, redirect=False):
             for j in lists.get(a, []):
                 if j <= bq - L and len(cands) < E:
                     cands.append(j)
-        ranked = sorted(cands, key=lambda j: (-float(dot_chain32(q, kb[j])), j))
+        score = {j: rerank_dot(q, kb[j]) for j in cands}
+        ranked = sorted(cands, key=lambda j: (-float(score[j]), j))
+        if rerank_margins is not None:
+            rerank_margins.append(add32(score[ranked[R - 1]], -score[ranked[R]]) if 0 < R < len(ranked)
+                                  else np.float32(np.inf))
         chosen = ranked[:R]
         if forced_bh is not None and R > 0:
             f = int(forced_bh[t])

@@ -48,3 +48,11 @@ def dot_chain32(a, b) -> np.float32:
     for x, y in zip(a, b):
         acc = fma32(x, y, acc)
     return acc
+
+
+def dot_tree32(a, b) -> np.float32:
+    """Eight fma chains over the contiguous runs [l n / 8, (l + 1) n / 8) of the vectors, added as the balanced
+    tree ((c0 + c1) + (c2 + c3)) + ((c4 + c5) + (c6 + c7)), every step rounded to fp32."""
+    n = len(a)
+    c = [dot_chain32(a[l * n // 8:(l + 1) * n // 8], b[l * n // 8:(l + 1) * n // 8]) for l in range(8)]
+    return add32(add32(add32(c[0], c[1]), add32(c[2], c[3])), add32(add32(c[4], c[5]), add32(c[6], c[7])))

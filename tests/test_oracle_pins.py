@@ -185,6 +185,31 @@ def test_routing_matches_independent_bruteforce(seed, dup):
             np.testing.assert_array_equal(sel[0, h], np.array(b_sel, np.int32))
 
 
+@pytest.mark.parametrize("d,M", [(8, 2), (20, 2), (64, 2)])
+def test_fp32_rerank_scores_sum_eight_runs_as_a_tree(d, M):
+    # The fp32 rerank score is eight fma chains over the contiguous runs [l d / 8, (l + 1) d / 8) added as a
+    # balanced tree.  The oracle's fp32 rerank margins (a difference of two such scores, rounded once) match an
+    # exact-rational emulation of that order bit for bit; the plain single chain gives other bits on some
+    # queries, so the pin tells the two orders apart (d = 20 has runs of two and three elements).
+    cfg = tiny(S=192, Bs=8, H=2, d=d, M=M, L=1, R=2, E=5, T=4, cap=4)
+    inp = synth.make_inputs(cfg, seed=12)
+    Qs, Ks, Vs = stored_qkv(cfg, inp)
+    kbar, addr, _ = oracle.summary_assign(cfg, Ks, inp["codebooks"])
+    sel, ncand, pm, rm, _ = oracle.route_queries(cfg, Qs, kbar, inp["codebooks"], addr)
+    n_finite, n_chain_diff = 0, 0
+    for h in range(cfg.H):
+        tree, chain = [], []
+        route_bh(Qs[0, h], Ks[0, h], inp["codebooks"][h], cfg, rerank_margins=tree)
+        route_bh(Qs[0, h], Ks[0, h], inp["codebooks"][h], cfg, rerank_margins=chain, rerank_dot=dot_chain32)
+        got = rm[0, h]
+        np.testing.assert_array_equal(got.view(np.uint32), np.array(tree, np.float32).view(np.uint32))
+        fin = np.isfinite(got)
+        n_finite += int(fin.sum())
+        n_chain_diff += int((np.array(chain, np.float32)[fin].view(np.uint32) != got[fin].view(np.uint32)).sum())
+    assert n_finite > 50
+    assert n_chain_diff > 0
+
+
 def _fp64_route(cfg, Qs, Ks, cb, forced=None):
     kbar, addr, am = oracle.summary_assign64(cfg, Ks, cb)
     ids, saddr, rank, ov = oracle.posting(cfg, addr)
