@@ -471,10 +471,12 @@ def measure_backward(plan, cfg, x, Wq, Wk, Wv, Wo, sel, ws, tdt, dev, stream, st
     """mono_backward for the step's selection and a seeded upstream gradient: mean of `steps`
     timed calls after one warm-up.  Algorithmic flops: the forward recompute (projection and
     selected-set attention), the projection gradients (8 GEMMs of B*S x H*d x W) and the
-    attention gradients (per query and selected key: 2 dot products in the log-sum-exp pass,
-    3 in the dQ pass, 4 in the dK/dV pass, of d multiply-adds each).  With bf16 storage the
-    GEMMs and the forward attention run on the tensor cores and the attention gradients on the
-    fp32 lanes, so the roofline's target time is the sum of the two parts at their own peaks."""
+    attention gradients (per query and selected key 5 products of d multiply-adds: the score,
+    dO . v, and the dS k, dS q, P dO terms).  With bf16 storage the GEMMs and the forward
+    attention run on the tensor cores; the attention gradients do too where the library's
+    tensor-core backward takes the shape (Bs = 64, d = 64 with L <= 2 or d = 128 with L = 1),
+    else they run on the fp32 lanes, and the roofline's target time is the sum of the two parts
+    at their own peaks."""
     import torch
 
     from learned_product_hash_proj_b200 import mono
@@ -500,9 +502,11 @@ def measure_backward(plan, cfg, x, Wq, Wk, Wv, Wo, sel, ws, tdt, dev, stream, st
     keys = nsel * cfg.Bs + B * H * S * ((cfg.L - 1) * cfg.Bs + (cfg.Bs + 1) / 2)   # selected keys, all queries
     gemm = 2.0 * B * S * H * d * W
     fwd_attn = 2 * keys * 2 * d
-    bwd_attn = (2 + 3 + 4) * keys * 2 * d
+    bwd_attn = 5 * keys * 2 * d
     flops = 3 * gemm + fwd_attn + 8 * gemm + bwd_attn
-    tensor = 11 * gemm + fwd_attn if cfg.dtype == "bf16" else 0.0
+    nk = 128 + (cfg.L - 1) * cfg.Bs
+    attn_tc = cfg.dtype == "bf16" and cfg.Bs == 64 and ((d == 64 and nk <= 192) or (d == 128 and nk <= 128))
+    tensor = (11 * gemm + fwd_attn + (bwd_attn if attn_tc else 0.0)) if cfg.dtype == "bf16" else 0.0
     alu = flops - tensor
     tpeak, tsrc = bf16_sustained_peak()
     target_s = tensor / (tpeak * 1e12) + alu / (FP32_PEAK_TFLOPS * 1e12)
@@ -510,7 +514,8 @@ def measure_backward(plan, cfg, x, Wq, Wk, Wv, Wo, sel, ws, tdt, dev, stream, st
     eff_peak = flops / target_s / 1e12
     return {"ms": ms, "tokens_per_s": B * S / (ms / 1e3),
             "api": "mono_backward (forward recompute + gradients of x, Wq, Wk, Wv, Wo for a fixed selection)",
-            "roofline": {"bound": "tensor+alu", "achieved": tf, "peak": eff_peak, "unit": "TFLOP/s",
+            "roofline": {"bound": "tensor" if alu == 0 else "tensor+alu", "achieved": tf, "peak": eff_peak,
+                         "unit": "TFLOP/s",
                          "frac": tf / eff_peak, "target_ms": target_s * 1e3, "algorithmic_flops": flops,
                          "tensor_flops": tensor, "alu_flops": alu, "peak_tensor_tflops": tpeak,
                          "peak_alu_tflops": FP32_PEAK_TFLOPS,

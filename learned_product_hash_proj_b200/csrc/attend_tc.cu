@@ -1712,6 +1712,268 @@ __global__ void __launch_bounds__(256, 1) k_bwd_local_dkdv_tc(const __grid_const
 }
 
 
+// ---------------------------------------------------------------------------
+// backward, the remote blocks on the tensor cores: one persistent CTA of 256
+// threads per SM walks the (b, h, block j) of the selection lists; for each
+// block, K_j and V_j arrive by TMA and its selecting queries are taken 128 at a
+// time, their Q, dO hi and dO lo rows gathered by cp.async into the 128-byte
+// swizzled layout (eight threads per row).  Per chunk of queries g:
+//   S = Q_g K_j^T,  dP = dO_g V_j^T           (TMEM columns [0, 64), [64, 128))
+//   P = exp(S / sqrt(d) - lse),  dS = P (dP - D)   (every key of a selected block is visible)
+//   dQ_g = dS K_j        -> added to dq_loc rows with fp32 vector atomics (a query has several blocks)
+//   dV_j += P^T dO_g,  dK_j += dS^T Q_g      (TMEM, over all chunks of the block)
+// P and dS are stored once, row-major by query as two bf16 terms each; the
+// row-major tile is the K-major A operand of dQ and the MN-major A operand
+// (M = the block's 64 keys, padded to 128 rows whose results are not read) of
+// dV and dK.  dV_j and dK_j (without the 1/sqrt(d) factor) are then added to the
+// rows of dv_loc and dk_loc that the local kernel wrote: only this CTA writes
+// block j's rows.
+// ---------------------------------------------------------------------------
+template <int D>
+struct BwdRemoteSmem {
+    static constexpr int KB = 64 * D * 2, QB = 128 * D * 2, PB = 128 * 64 * 2;
+    // P hi, P lo, dS hi, dS lo, then Q: each P/dS tile is followed by 16 KB of other tiles, which the padding half
+    // of its MN-major operand reads
+    static constexpr int K_OFF = 0, V_OFF = KB, PH_OFF = 2 * KB, PL_OFF = PH_OFF + PB, DH_OFF = PL_OFF + PB;
+    static constexpr int DL_OFF = DH_OFF + PB, Q_OFF = DL_OFF + PB, GH_OFF = Q_OFF + QB, GL_OFF = GH_OFF + QB;
+    static constexpr int BAR_OFF = GL_OFF + QB;  // 2 mbarriers + TMEM base
+    static constexpr int BYTES = BAR_OFF + 32;
+    static constexpr int TCOLS = 128 + 3 * D;
+    static constexpr bool supported = TCOLS <= 512 && BYTES <= 227 * 1024 && QB >= PB;
+};
+
+__device__ __forceinline__ uint32_t sw128(int r, int c) {  // 16-byte chunk c of row r, 128-row slabs of 64 columns
+    return (uint32_t)((c >> 3) * (128 * 128) + r * 128 + (((c & 7) ^ (r & 7)) << 4));
+}
+
+template <int D>
+__global__ void __launch_bounds__(256, 1) k_bwd_remote_tc(const __grid_constant__ BwdMaps maps, const bf16 *__restrict__ Q,
+                                                          const bf16 *__restrict__ dohi, const bf16 *__restrict__ dolo,
+                                                          const float *__restrict__ lse, const float *__restrict__ dsum,
+                                                          const int32_t *__restrict__ cnt,
+                                                          const int32_t *__restrict__ start,
+                                                          const int32_t *__restrict__ list, float *__restrict__ dq_loc,
+                                                          float *__restrict__ dk_loc, float *__restrict__ dv_loc,
+                                                          unsigned long long *__restrict__ counters, int S, int R,
+                                                          int nb, float scale_log2, int nbh) {
+    constexpr int BS = 64;
+    using Lay = BwdRemoteSmem<D>;
+    static_assert(Lay::supported, "tile shape");
+    constexpr int KB = Lay::KB, DH = D / 2;
+    extern __shared__ __align__(1024) uint8_t smem[];
+    uint8_t *sK = smem + Lay::K_OFF, *sV = smem + Lay::V_OFF, *sQ = smem + Lay::Q_OFF;
+    uint8_t *sGH = smem + Lay::GH_OFF, *sGL = smem + Lay::GL_OFF;
+    uint8_t *sPH = smem + Lay::PH_OFF, *sPL = smem + Lay::PL_OFF, *sDH = smem + Lay::DH_OFF, *sDL = smem + Lay::DL_OFF;
+    uint64_t *bar_ld = (uint64_t *)(smem + Lay::BAR_OFF), *mbar = bar_ld + 1;
+    uint32_t *tmem_base = (uint32_t *)(bar_ld + 2);
+    if (timed_out(counters)) return;
+    if (tc::smem_u32(smem) & 1023) {
+        if (threadIdx.x == 0) record_error(counters, kDevErrSmemAlign);
+        return;
+    }
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quarter = warp & 3, half = warp >> 2;
+    const int row = quarter * 32 + lane;
+    if (warp == 0) {
+        tc::tmem_alloc(tmem_base, 512);
+        tc::tmem_relinquish();
+    }
+    if (tid == 0) {
+        tc::mbar_init(bar_ld, 1);
+        tc::mbar_init(mbar, 1);
+        tc::fence_mbar_init();
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = *tmem_base;
+    const uint32_t trow = tmem + ((uint32_t)(quarter * 32) << 16);
+    // S, dP, dQ, dV and dK columns of this lane quarter
+    const uint32_t tS = trow, tP = trow + 64, tQ = trow + 128, tV = trow + 128 + D, tK = trow + 128 + 2 * D;
+    const uint32_t idS = tc::idesc_bf16(128, BS), idQ = tc::idesc_bf16(128, D, true),
+                   idKV = tc::idesc_bf16(128, D, true, true);
+    bool ok = true;
+    int pend = -1;         // thread 0: the K/V load of block k issued and not yet seen complete
+    uint32_t mph = 0;      // completions of mbar so far, mod 2
+    int k = 0;             // blocks with K/V loaded so far
+    const int total = nbh * nb;
+    for (int f = blockIdx.x; f < total && ok; f += gridDim.x) {
+        const int bh = f / nb, j = f % nb;
+        const int n = cnt[f];
+        if (n == 0) continue;  // uniform
+        const int32_t *lst = list + (size_t)bh * S * R + start[f];
+        if (tid == 0) {
+            tc::mbar_expect_tx(bar_ld, 2 * KB);
+#pragma unroll
+            for (int a = 0; a < D / 64; ++a) {
+                tc::tma_load_3d(sK + a * (BS * 128), &maps.k, 64 * a, j * BS, bh, bar_ld);
+                tc::tma_load_3d(sV + a * (BS * 128), &maps.v, 64 * a, j * BS, bh, bar_ld);
+            }
+            pend = k;
+        }
+        bool landed = true;
+        for (int g0 = 0; g0 < n && ok; g0 += 128) {
+            const int ng = min(128, n - g0);
+            // the chunk's query rows: Q, dO hi, dO lo (zeros past ng), eight threads per 128-byte segment
+            constexpr int CPR = D / 8;
+#pragma unroll
+            for (int kq = 0; kq < 128 * CPR / 256; ++kq) {
+                const int idx = tid + 256 * kq, r = idx / CPR, c = idx % CPR;
+                const bool live = r < ng;
+                const size_t off = live ? ((size_t)bh * S + lst[g0 + r]) * D + 8 * c : 0;
+                tc::cp_async16(sQ + sw128(r, c), Q + off, live);
+                tc::cp_async16(sGH + sw128(r, c), dohi + off, live);
+                tc::cp_async16(sGL + sw128(r, c), dolo + off, live);
+            }
+            asm volatile("cp.async.commit_group;" ::: "memory");
+            const bool live = row < ng;
+            const int t = live ? lst[g0 + row] : 0;
+            const float lse2 = live ? lse[(size_t)bh * S + t] * 1.4426950408889634f : 0.f;
+            const float Drow = live ? dsum[(size_t)bh * S + t] : 0.f;
+            tc::cp_async_wait_all();
+            if (tid == 0 && g0 == 0) {
+                landed = tc::mbar_wait(bar_ld, (uint32_t)(k & 1));
+                if (landed) pend = -1;
+            }
+            tc::fence_smem_to_async();
+            tc::fence_before_sync();
+            ok = __syncthreads_and(landed);
+            tc::fence_after_sync();
+            if (!ok) break;
+            if (tid == 0) {
+                const uint32_t aq = tc::smem_u32(sQ), ah = tc::smem_u32(sGH), al = tc::smem_u32(sGL);
+                const uint32_t bk = tc::smem_u32(sK), bv = tc::smem_u32(sV);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t ao = (kk >> 2) * (128 * 128) + (kk & 3) * 32, bo = (kk >> 2) * (BS * 128) + (kk & 3) * 32;
+                    tc::mma_bf16(tmem, tc::desc_sw128(aq + ao), tc::desc_sw128(bk + bo), idS, kk > 0);
+                    tc::mma_bf16(tmem + 64, tc::desc_sw128(ah + ao), tc::desc_sw128(bv + bo), idS, kk > 0);
+                }
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t ao = (kk >> 2) * (128 * 128) + (kk & 3) * 32, bo = (kk >> 2) * (BS * 128) + (kk & 3) * 32;
+                    tc::mma_bf16(tmem + 64, tc::desc_sw128(al + ao), tc::desc_sw128(bv + bo), idS, 1u);
+                }
+                tc::commit(mbar);
+            }
+            ok = __syncthreads_and(tc::mbar_wait(mbar, mph));
+            mph ^= 1u;
+            tc::fence_after_sync();
+            if (!ok) break;
+            // P and dS of this row over the block's 64 keys (this warp's 32 of them), hi and lo terms
+            {
+                const int c0 = half * 32;
+                float sv[32], pv[32];
+                tc::tmem_ld32(tS + c0, sv);
+                tc::tmem_ld32(tP + c0, pv);
+                uint32_t ph[16], pl[16], dh[16], dl[16];
+#pragma unroll
+                for (int u = 0; u < 16; ++u) {
+                    const float p0 = live ? tc::ex2_fast(fmaf(sv[2 * u], scale_log2, -lse2)) : 0.f;
+                    const float p1 = live ? tc::ex2_fast(fmaf(sv[2 * u + 1], scale_log2, -lse2)) : 0.f;
+                    split2(p0, p1, ph[u], pl[u]);
+                    split2(p0 * (pv[2 * u] - Drow), p1 * (pv[2 * u + 1] - Drow), dh[u], dl[u]);
+                }
+#pragma unroll
+                for (int q8 = 0; q8 < 4; ++q8) {
+                    const uint32_t off = sw128(row, (c0 >> 3) + q8);
+                    *(uint4 *)(sPH + off) = make_uint4(ph[4 * q8], ph[4 * q8 + 1], ph[4 * q8 + 2], ph[4 * q8 + 3]);
+                    *(uint4 *)(sPL + off) = make_uint4(pl[4 * q8], pl[4 * q8 + 1], pl[4 * q8 + 2], pl[4 * q8 + 3]);
+                    *(uint4 *)(sDH + off) = make_uint4(dh[4 * q8], dh[4 * q8 + 1], dh[4 * q8 + 2], dh[4 * q8 + 3]);
+                    *(uint4 *)(sDL + off) = make_uint4(dl[4 * q8], dl[4 * q8 + 1], dl[4 * q8 + 2], dl[4 * q8 + 3]);
+                }
+            }
+            tc::fence_smem_to_async();
+            tc::fence_before_sync();
+            __syncthreads();
+            tc::fence_after_sync();
+            if (tid == 0) {
+                const uint32_t bk = tc::smem_u32(sK), bq = tc::smem_u32(sQ), gh = tc::smem_u32(sGH),
+                               gl = tc::smem_u32(sGL);
+                const uint32_t a_ph = tc::smem_u32(sPH), a_pl = tc::smem_u32(sPL), a_dh = tc::smem_u32(sDH),
+                               a_dl = tc::smem_u32(sDL);
+                // dQ_g = dS K_j: A = dS (K-major over the 64 keys), B = K_j (MN-major)
+#pragma unroll
+                for (int kk = 0; kk < BS / 16; ++kk) {
+                    const uint64_t bd = tc::desc_sw128_mn(bk + 2048 * kk, BS * 128);
+                    tc::mma_bf16(tmem + 128, tc::desc_sw128(a_dh + 32 * kk), bd, idQ, kk > 0);
+                    tc::mma_bf16(tmem + 128, tc::desc_sw128(a_dl + 32 * kk), bd, idQ, 1u);
+                }
+                // dV_j += P^T dO_g and dK_j += dS^T Q_g: A = P, dS read MN-major (M = keys; the second 64-key
+                // half of the 128-row operand points at another tile and its rows are not read), K = the chunk's
+                // queries, B = dO, Q (MN-major)
+#pragma unroll
+                for (int kk = 0; kk < 128 / 16; ++kk) {
+                    const bool acc = g0 > 0 || kk > 0;
+                    const uint64_t bgh = tc::desc_sw128_mn(gh + 2048 * kk, 128 * 128);
+                    const uint64_t bgl = tc::desc_sw128_mn(gl + 2048 * kk, 128 * 128);
+                    const uint64_t bqd = tc::desc_sw128_mn(bq + 2048 * kk, 128 * 128);
+                    const uint64_t aph = tc::desc_sw128_mn(a_ph + 2048 * kk, Lay::PB);
+                    const uint64_t apl = tc::desc_sw128_mn(a_pl + 2048 * kk, Lay::PB);
+                    const uint64_t adh = tc::desc_sw128_mn(a_dh + 2048 * kk, Lay::PB);
+                    const uint64_t adl = tc::desc_sw128_mn(a_dl + 2048 * kk, Lay::PB);
+                    tc::mma_bf16(tmem + 128 + D, aph, bgh, idKV, acc);
+                    tc::mma_bf16(tmem + 128 + D, aph, bgl, idKV, 1u);
+                    tc::mma_bf16(tmem + 128 + D, apl, bgh, idKV, 1u);
+                    tc::mma_bf16(tmem + 128 + 2 * D, adh, bqd, idKV, acc);
+                    tc::mma_bf16(tmem + 128 + 2 * D, adl, bqd, idKV, 1u);
+                }
+                tc::commit(mbar);
+            }
+            ok = __syncthreads_and(tc::mbar_wait(mbar, mph));
+            mph ^= 1u;
+            tc::fence_after_sync();
+            if (!ok) break;
+            // this row's dQ part, added to the query's fp32 dQ
+#pragma unroll 1
+            for (int c0 = half * DH; c0 < half * DH + DH; c0 += 32) {
+                float v[32];
+                tc::tmem_ld32(tQ + c0, v);
+                if (live) {
+                    float4 *dst = (float4 *)(dq_loc + ((size_t)bh * S + t) * D + c0);
+#pragma unroll
+                    for (int q4 = 0; q4 < 8; ++q4)
+                        atomicAdd(dst + q4, make_float4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]));
+                }
+            }
+            tc::fence_before_sync();
+            __syncthreads();  // shared memory and the S, dP, dQ columns are free for the next chunk
+            tc::fence_after_sync();
+        }
+        if (!ok) break;
+        ++k;
+        // dV_j and dK_j: TMEM rows 0..63 (lane quarters 0 and 1; quarters 2 and 3 hold the padding rows), added to
+        // the local parts of the block's keys
+        if (quarter < 2) {
+            const size_t key = (size_t)bh * S + j * BS + row;
+#pragma unroll 1
+            for (int c0 = half * DH; c0 < half * DH + DH; c0 += 32) {
+                float v[32], g[32];
+                tc::tmem_ld32(tV + c0, v);
+                tc::tmem_ld32(tK + c0, g);
+                float4 *dv = (float4 *)(dv_loc + key * D + c0);
+                float4 *dk = (float4 *)(dk_loc + key * D + c0);
+#pragma unroll
+                for (int q4 = 0; q4 < 8; ++q4) {
+                    const float4 a = dv[q4], b = dk[q4];
+                    dv[q4] = make_float4(a.x + v[4 * q4], a.y + v[4 * q4 + 1], a.z + v[4 * q4 + 2], a.w + v[4 * q4 + 3]);
+                    dk[q4] = make_float4(b.x + g[4 * q4], b.y + g[4 * q4 + 1], b.z + g[4 * q4 + 2], b.w + g[4 * q4 + 3]);
+                }
+            }
+        }
+        tc::fence_before_sync();
+        __syncthreads();  // K/V tiles and the dV/dK columns are free for the next block
+        tc::fence_after_sync();
+    }
+    // leave no TMA write in flight into this CTA's shared memory
+    if (tid == 0 && pend >= 0 && !tc::mbar_wait(bar_ld, (uint32_t)(pend & 1))) ok = false;
+    if (!ok && tid == 0) record_error(counters, kDevErrTimeout);
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 0) tc::tmem_dealloc(tmem, 512);
+}
+
+
 template <int D, int BS, int NK>
 static cudaError_t launch_bwd_local_dq_shape(const Plan &p, const void *Q, const void *K, const void *V,
                                              const void *dohi, const void *dolo, const float *lse, const float *dsum,
@@ -1779,6 +2041,51 @@ cudaError_t launch_bwd_local_dkdv_tc(const Plan &p, const void *Q, const void *K
     if (c.d == 64)
         return launch_bwd_local_dkdv_shape<64, 64, 192>(p, Q, K, V, dohi, dolo, lse, dsum, dk_loc, dv_loc, counters, s);
     return launch_bwd_local_dkdv_shape<128, 64, 128>(p, Q, K, V, dohi, dolo, lse, dsum, dk_loc, dv_loc, counters, s);
+}
+
+template <int D>
+static cudaError_t launch_bwd_remote_shape(const Plan &p, const void *Q, const void *K, const void *V,
+                                           const void *dohi, const void *dolo, const float *lse, const float *dsum,
+                                           const int32_t *cnt, const int32_t *start, const int32_t *list,
+                                           float *dq_loc, float *dk_loc, float *dv_loc, unsigned long long *counters,
+                                           cudaStream_t s) {
+    const mono_config &c = p.cfg;
+    using Lay = BwdRemoteSmem<D>;
+    BwdMaps maps;
+    const int BH = c.B * c.H;
+    if (!make_map_3d(&maps.k, K, D, c.S, BH, 64) || !make_map_3d(&maps.v, V, D, c.S, BH, 64))
+        return cudaErrorInvalidValue;
+    maps.q = maps.k;  // unused
+    maps.dohi = maps.k;
+    maps.dolo = maps.k;
+    auto kern = k_bwd_remote_tc<D>;
+    cudaError_t e;
+    if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::BYTES)) != cudaSuccess)
+        return e;
+    int dev = 0, sms = 148;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+        return e;
+    const float scale_log2 = (float)(1.4426950408889634 / sqrt((double)c.d));
+    const int total = BH * p.nb;
+    kern<<<std::min(total, sms), 256, Lay::BYTES, s>>>(maps, (const bf16 *)Q, (const bf16 *)dohi, (const bf16 *)dolo,
+                                                       lse, dsum, cnt, start, list, dq_loc, dk_loc, dv_loc, counters,
+                                                       c.S, c.R, p.nb, scale_log2, BH);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_bwd_remote_tc(const Plan &p, const void *Q, const void *K, const void *V, const void *dohi,
+                                 const void *dolo, const float *lse, const float *dsum, const int32_t *cnt,
+                                 const int32_t *start, const int32_t *list, float *dq_loc, float *dk_loc,
+                                 float *dv_loc, unsigned long long *counters, cudaStream_t s) {
+    const mono_config &c = p.cfg;
+    if (!bwd_local_dq_tc_supported(c)) return cudaErrorInvalidValue;
+    if (c.d == 64)
+        return launch_bwd_remote_shape<64>(p, Q, K, V, dohi, dolo, lse, dsum, cnt, start, list, dq_loc, dk_loc,
+                                           dv_loc, counters, s);
+    return launch_bwd_remote_shape<128>(p, Q, K, V, dohi, dolo, lse, dsum, cnt, start, list, dq_loc, dk_loc, dv_loc,
+                                        counters, s);
 }
 
 bool bwd_local_dq_tc_supported(const mono_config &c) {

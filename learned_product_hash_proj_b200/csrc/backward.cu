@@ -13,18 +13,19 @@
 // Kernels (fp32 arithmetic, gradients in fp32):
 //   k_bwd_prep   with the forward recompute's fp32 O and log-sum-exp: D per
 //                row and dO head-major as two bf16 terms, for the tensor-core
-//                kernels of the local keys (k_bwd_local_dq_tc and
-//                k_bwd_local_dkdv_tc, in attend_tc.cu);
+//                kernels;
 //   k_bwd_dq     d/16 lanes per query-head: log-sum-exp and D from recomputed
 //                scores (the stored O is not needed) or from the recompute,
-//                then dQ over the remote blocks and the local keys (or the
-//                tensor cores' local part);
+//                then dQ over the local keys and the remote blocks;
 //   k_bwd_count / k_bwd_scan / k_bwd_fill: per (b, h) and block j, the
 //                queries that selected j (lists in unspecified order);
 //   k_bwd_dkdv   one CTA per (b, h) and tile of up to 64 keys of one block:
-//                walks the block's local queries (or starts from the tensor
-//                cores' local part) and its selecting queries, accumulating
-//                dK and dV of its keys in registers;
+//                walks the block's local queries and its selecting queries,
+//                accumulating dK and dV of its keys in registers;
+//   (with bf16 storage, the forward recompute's statistics and Bs = 64 the
+//   attention gradients run instead on the tensor cores: k_bwd_local_dq_tc,
+//   k_bwd_local_dkdv_tc and k_bwd_remote_tc in attend_tc.cu, then
+//   k_bwd_finish for the factor, the inverse rotation and the layout)
 //   (dq, dk and dv leave these kernels either as [B,H,S,d] for the post-RoPE
 //   q and k, or rotated back and token-major for the projection gradients)
 //   k_gemm_any   the projection gradients of fp32 storage (generic strided SIMT
@@ -45,7 +46,7 @@ namespace mono {
 namespace {
 
 struct BwdLayout {
-    size_t lse, dsum, cnt, start, cursor, list, dO, dQp, dKp, dVp, dOhi, dOlo, dQloc, dVloc, total;
+    size_t lse, dsum, cnt, start, cursor, list, dO, dQp, dKp, dVp, dOhi, dOlo, dQloc, dKloc, dVloc, total;
 };
 
 BwdLayout bwd_layout(const Plan &p) {
@@ -68,11 +69,12 @@ BwdLayout bwd_layout(const Plan &p) {
     L.dQp = take(B * S * H * d * 4);
     L.dKp = take(B * S * H * d * 4);
     L.dVp = take(B * S * H * d * 4);
-    // the tensor-core local parts: dO as two bf16 terms, the local dQ (then the local dK) and the local dV in
-    // fp32, all head-major [B*H, S, d]
+    // the tensor-core path: dO as two bf16 terms, and dQ, dK, dV in fp32 (without the 1/sqrt(d) factor, before
+    // the inverse rotation), all head-major [B*H, S, d]
     L.dOhi = take(B * H * S * d * 2);
     L.dOlo = take(B * H * S * d * 2);
     L.dQloc = take(B * H * S * d * 4);
+    L.dKloc = take(B * H * S * d * 4);
     L.dVloc = take(B * H * S * d * 4);
     L.total = o;
     return L;
@@ -221,13 +223,42 @@ __global__ void __launch_bounds__(256) k_bwd_prep(const float *__restrict__ dO, 
     if (lane == 0) dsum[((size_t)b * H + h) * S + t] = part;
 }
 
+// The tensor-core path's last step: dQ and dK (times 1/sqrt(d)) and dV from their head-major fp32 sums to the
+// operands of the projection gradients (store_grad16: rotated back, token-major).  One thread per 16 dimensions
+// of a (b, h, t) row.
+template <int DD>
+__global__ void __launch_bounds__(256) k_bwd_finish(const float *__restrict__ dq, const float *__restrict__ dk,
+                                                    const float *__restrict__ dv, const GradOut go, int B, int H,
+                                                    int S, float scale) {
+    constexpr int TPR = DD / 16;
+    const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (gid >= (long long)B * H * S * TPR) return;
+    const long long w = gid / TPR;
+    const int e0 = (int)(gid % TPR) * 16;
+    const int t = (int)(w % S);
+    const long long bh = w / S;
+    const int b = (int)(bh / H), h = (int)(bh % H);
+    float q[16], k[16], v[16];
+    load16<float>(dq + w * DD + e0, q);
+    load16<float>(dk + w * DD + e0, k);
+    load16<float>(dv + w * DD + e0, v);
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+        q[e] *= scale;
+        k[e] *= scale;
+    }
+    store_grad16<DD>(go, go.q, true, q, b, h, t, e0, B, H, S);
+    store_grad16<DD>(go, go.k, true, k, b, h, t, e0, B, H, S);
+    store_grad16<DD>(go, go.v, false, v, b, h, t, e0, B, H, S);
+}
+
 template <typename T, int DD>
 __global__ void __launch_bounds__(256) k_bwd_dq(const T *__restrict__ Q, const T *__restrict__ K,
                                                 const T *__restrict__ V, const int32_t *__restrict__ sel,
                                                 const float *__restrict__ dO, const GradOut go,
                                                 float *__restrict__ lse_out, float *__restrict__ dsum_out,
-                                                const float *__restrict__ o32, const float *__restrict__ dq_loc,
-                                                int B, int H, int S, int Bs, int L, int R, float scale) {
+                                                const float *__restrict__ o32, int B, int H, int S, int Bs, int L,
+                                                int R, float scale) {
     constexpr int TPQ = DD / kDqE, E = kDqE, U = 2;
     const long long nq = (long long)B * H * S;
     const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
@@ -248,11 +279,9 @@ __global__ void __launch_bounds__(256) k_bwd_dq(const T *__restrict__ Q, const T
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) nloc_w = max(nloc_w, __shfl_xor_sync(0xffffffffu, nloc_w, o));
 
-    // one sweep over the query's keys; f(k row, v row, valid) per group of U keys (the remote blocks only when
-    // the tensor cores did the local keys: dq_loc)
-    const int nloc_sweep = dq_loc ? 0 : nloc_w;
+    // one sweep over the query's keys; f(k row, v row, valid) per group of U keys
     auto sweep = [&](auto &&f) {
-        for (int i = 0; i < nloc_sweep; i += U) {
+        for (int i = 0; i < nloc_w; i += U) {
             const T *kr[U], *vr[U];
             bool ok[U];
 #pragma unroll
@@ -373,12 +402,6 @@ __global__ void __launch_bounds__(256) k_bwd_dq(const T *__restrict__ Q, const T
         }
     });
     if (live) {
-        if (dq_loc) {
-            float dl[E];
-            load16<float>(dq_loc + w * DD + e0, dl);
-#pragma unroll
-            for (int e = 0; e < E; ++e) dq[e] += dl[e];
-        }
 #pragma unroll
         for (int e = 0; e < E; ++e) dq[e] *= scale;
         store_grad16<DD>(go, go.q, true, dq, b, h, t, e0, B, H, S);
@@ -474,9 +497,8 @@ template <typename T, int DD>
 __global__ void __launch_bounds__(kBwdKT * DD / 16, DD == 64 ? 2 : 1) k_bwd_dkdv(
     const T *__restrict__ Q, const T *__restrict__ K, const T *__restrict__ V, const float *__restrict__ dO,
     const float *__restrict__ lse, const float *__restrict__ dsum, const int32_t *__restrict__ cnt,
-    const int32_t *__restrict__ start, const int32_t *__restrict__ list, const GradOut go,
-    const float *__restrict__ dk_loc, const float *__restrict__ dv_loc, int B, int H, int S, int Bs, int L, int R,
-    int nb, float scale) {
+    const int32_t *__restrict__ start, const int32_t *__restrict__ list, const GradOut go, int B, int H, int S,
+    int Bs, int L, int R, int nb, float scale) {
     constexpr int TPK = DD / 16, NT = kBwdKT * TPK, E = 16;
     constexpr int PER = kBwdQG * DD / NT;  // staged elements per thread and array (one dimension, PER queries)
     constexpr int SEG = 20, ROW = TPK * SEG;  // padded segment and row, in floats
@@ -502,18 +524,7 @@ __global__ void __launch_bounds__(kBwdKT * DD / 16, DD == 64 ? 2 : 1) k_bwd_dkdv
         dk[e] = 0.f;
         dv[e] = 0.f;
     }
-    // the local queries' part from the tensor cores (dk_loc without the 1/sqrt(d) factor), or walked here
-    if (dk_loc && live) {
-        float a[E], g[E];
-        load16<float>(dk_loc + (bh * S + key) * DD + e0, a);
-        load16<float>(dv_loc + (bh * S + key) * DD + e0, g);
-#pragma unroll
-        for (int e = 0; e < E; ++e) {
-            dk[e] = a[e] * scale;
-            dv[e] = g[e];
-        }
-    }
-    const int t_loc0 = j * Bs, t_loc1 = dk_loc ? t_loc0 : min(S, (j + L) * Bs);  // local queries [t_loc0, t_loc1)
+    const int t_loc0 = j * Bs, t_loc1 = min(S, (j + L) * Bs);  // local queries [t_loc0, t_loc1)
     const int nloc = t_loc1 - t_loc0;
     const int nrem = R > 0 ? cnt[bh * nb + j] : 0;
     const int rem0 = R > 0 ? start[bh * nb + j] : 0;
@@ -701,12 +712,24 @@ cudaError_t attend_backward(const Plan &p, const T *Q, const T *K, const T *V, c
     cudaError_t e;
     const int tpq = c.d / kDqE;
     const unsigned gq = (unsigned)((nq * tpq + 255) / 256);
-    // with the forward's statistics, the local keys' part of dQ on the tensor cores where the shape allows
-    float *dq_loc = nullptr;
+    auto build_lists = [&]() -> cudaError_t {
+        if (c.R == 0) return cudaSuccess;
+        const long long n = nq * c.R;
+        cudaError_t e2;
+        if ((e2 = cudaMemsetAsync(cnt, 0, (size_t)c.B * c.H * p.nb * 4, s)) != cudaSuccess) return e2;
+        k_bwd_count<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(sel, cnt, n, c.S, c.R, p.nb, c.Bs, c.L);
+        k_bwd_scan<<<c.B * c.H, 1024, 0, s>>>(cnt, start, cursor, p.nb);
+        k_bwd_fill<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(sel, cursor, list, n, c.S, c.R, p.nb, c.Bs, c.L);
+        count_launches(3);
+        return cudaSuccess;
+    };
+    // With the forward's statistics and a shape the kernels take, every attention gradient on the tensor cores:
+    // the local keys query-major (dQ) and key-major (dK, dV), then the remote blocks block by block.
     if constexpr (sizeof(T) == 2) {
         if (o32 && counters && bwd_local_dq_tc_supported(c)) {
             __nv_bfloat16 *dohi = (__nv_bfloat16 *)(bws + L.dOhi), *dolo = (__nv_bfloat16 *)(bws + L.dOlo);
-            dq_loc = (float *)(bws + L.dQloc);
+            float *dq_loc = (float *)(bws + L.dQloc), *dk_loc = (float *)(bws + L.dKloc);
+            float *dv_loc = (float *)(bws + L.dVloc);
             const unsigned gp = (unsigned)((nq + 7) / 8);
             if (c.d == 64)
                 k_bwd_prep<64><<<gp, 256, 0, s>>>(dO, o32, dohi, dolo, dsum, c.B, c.H, c.S);
@@ -715,40 +738,38 @@ cudaError_t attend_backward(const Plan &p, const T *Q, const T *K, const T *V, c
             count_launches(1);
             if ((e = launch_bwd_local_dq_tc(p, Q, K, V, dohi, dolo, lse, dsum, dq_loc, counters, s)) != cudaSuccess)
                 return e;
+            if ((e = launch_bwd_local_dkdv_tc(p, Q, K, V, dohi, dolo, lse, dsum, dk_loc, dv_loc, counters, s)) !=
+                cudaSuccess)
+                return e;
+            if ((e = build_lists()) != cudaSuccess) return e;
+            if (c.R > 0 && (e = launch_bwd_remote_tc(p, Q, K, V, dohi, dolo, lse, dsum, cnt, start, list, dq_loc,
+                                                     dk_loc, dv_loc, counters, s)) != cudaSuccess)
+                return e;
+            const unsigned gf = (unsigned)((nq * (c.d / 16) + 255) / 256);
+            if (c.d == 64)
+                k_bwd_finish<64><<<gf, 256, 0, s>>>(dq_loc, dk_loc, dv_loc, go, c.B, c.H, c.S, scale);
+            else
+                k_bwd_finish<128><<<gf, 256, 0, s>>>(dq_loc, dk_loc, dv_loc, go, c.B, c.H, c.S, scale);
+            count_launches(1);
+            return cudaGetLastError();
         }
     }
     if (c.d == 64)
-        k_bwd_dq<T, 64><<<gq, 256, 0, s>>>(Q, K, V, sel, dO, go, lse, dsum, o32, dq_loc, c.B, c.H, c.S, c.Bs, c.L,
-                                           c.R, scale);
+        k_bwd_dq<T, 64><<<gq, 256, 0, s>>>(Q, K, V, sel, dO, go, lse, dsum, o32, c.B, c.H, c.S, c.Bs, c.L, c.R,
+                                           scale);
     else
-        k_bwd_dq<T, 128><<<gq, 256, 0, s>>>(Q, K, V, sel, dO, go, lse, dsum, o32, dq_loc, c.B, c.H, c.S, c.Bs, c.L,
-                                            c.R, scale);
+        k_bwd_dq<T, 128><<<gq, 256, 0, s>>>(Q, K, V, sel, dO, go, lse, dsum, o32, c.B, c.H, c.S, c.Bs, c.L, c.R,
+                                            scale);
     count_launches(1);
-    if (c.R > 0) {
-        const long long n = nq * c.R;
-        if ((e = cudaMemsetAsync(cnt, 0, (size_t)c.B * c.H * p.nb * 4, s)) != cudaSuccess) return e;
-        k_bwd_count<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(sel, cnt, n, c.S, c.R, p.nb, c.Bs, c.L);
-        k_bwd_scan<<<c.B * c.H, 1024, 0, s>>>(cnt, start, cursor, p.nb);
-        k_bwd_fill<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(sel, cursor, list, n, c.S, c.R, p.nb, c.Bs, c.L);
-        count_launches(3);
-    }
-    // the local queries' part of dK and dV on the tensor cores (dK into the local dQ's region, read by now)
-    float *dk_loc = nullptr, *dv_loc = nullptr;
-    if (dq_loc) {
-        dk_loc = dq_loc;
-        dv_loc = (float *)(bws + L.dVloc);
-        if ((e = launch_bwd_local_dkdv_tc(p, Q, K, V, bws + L.dOhi, bws + L.dOlo, lse, dsum, dk_loc, dv_loc, counters,
-                                          s)) != cudaSuccess)
-            return e;
-    }
+    if ((e = build_lists()) != cudaSuccess) return e;
     const int tpb = (c.Bs + kBwdKT - 1) / kBwdKT;
     const dim3 gk(tpb * p.nb, c.H, c.B);
     if (c.d == 64)
-        k_bwd_dkdv<T, 64><<<gk, kBwdKT * 4, 0, s>>>(Q, K, V, dO, lse, dsum, cnt, start, list, go, dk_loc, dv_loc, c.B,
-                                                     c.H, c.S, c.Bs, c.L, c.R, p.nb, scale);
+        k_bwd_dkdv<T, 64><<<gk, kBwdKT * 4, 0, s>>>(Q, K, V, dO, lse, dsum, cnt, start, list, go, c.B, c.H, c.S,
+                                                     c.Bs, c.L, c.R, p.nb, scale);
     else
-        k_bwd_dkdv<T, 128><<<gk, kBwdKT * 8, 0, s>>>(Q, K, V, dO, lse, dsum, cnt, start, list, go, dk_loc, dv_loc,
-                                                      c.B, c.H, c.S, c.Bs, c.L, c.R, p.nb, scale);
+        k_bwd_dkdv<T, 128><<<gk, kBwdKT * 8, 0, s>>>(Q, K, V, dO, lse, dsum, cnt, start, list, go, c.B, c.H, c.S,
+                                                      c.Bs, c.L, c.R, p.nb, scale);
     count_launches(1);
     return cudaGetLastError();
 }

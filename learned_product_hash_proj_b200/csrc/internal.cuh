@@ -154,6 +154,12 @@ cudaError_t launch_bwd_local_dq_tc(const Plan &p, const void *Q, const void *K, 
 cudaError_t launch_bwd_local_dkdv_tc(const Plan &p, const void *Q, const void *K, const void *V, const void *dohi,
                                      const void *dolo, const float *lse, const float *dsum, float *dk_loc,
                                      float *dv_loc, unsigned long long *counters, cudaStream_t s);
+// the remote blocks' part on the tensor cores, from the per-block lists of selecting queries (cnt, start, list as
+// [B*H, nb] and [B*H, S*R]): dq_loc += (fp32 atomics), dk_loc and dv_loc rows of each block += (one CTA per block)
+cudaError_t launch_bwd_remote_tc(const Plan &p, const void *Q, const void *K, const void *V, const void *dohi,
+                                 const void *dolo, const float *lse, const float *dsum, const int32_t *cnt,
+                                 const int32_t *start, const int32_t *list, float *dq_loc, float *dk_loc,
+                                 float *dv_loc, unsigned long long *counters, cudaStream_t s);
 cudaError_t launch_attend_tc(const Plan &p, const void *Q, const void *K, const void *V, const int32_t *sel, void *O,
                              void *ws, cudaStream_t s, int parts = kAttendAll, float *o32 = nullptr,
                              float *lse = nullptr, bool *stats = nullptr);
