@@ -1731,13 +1731,18 @@ __global__ void __launch_bounds__(256, 1) k_bwd_local_dkdv_tc(const __grid_const
 // ---------------------------------------------------------------------------
 template <int D>
 struct BwdRemoteSmem {
+    // NS stages of the gathered rows and of K/V: two at d = 64 (the next chunk's rows and the next block's K/V
+    // load while a chunk is computed), one at d = 128 (shared memory)
+    static constexpr int NS = D == 64 ? 2 : 1;
     static constexpr int KB = 64 * D * 2, QB = 128 * D * 2, PB = 128 * 64 * 2;
-    // P hi, P lo, dS hi, dS lo, then Q: each P/dS tile is followed by 16 KB of other tiles, which the padding half
-    // of its MN-major operand reads
-    static constexpr int K_OFF = 0, V_OFF = KB, PH_OFF = 2 * KB, PL_OFF = PH_OFF + PB, DH_OFF = PL_OFF + PB;
-    static constexpr int DL_OFF = DH_OFF + PB, Q_OFF = DL_OFF + PB, GH_OFF = Q_OFF + QB, GL_OFF = GH_OFF + QB;
-    static constexpr int BAR_OFF = GL_OFF + QB;  // 2 mbarriers + TMEM base
-    static constexpr int BYTES = BAR_OFF + 32;
+    // K, V per stage; P hi, P lo, dS hi, dS lo; then Q, dO hi, dO lo per stage.  Each P/dS tile is followed by at
+    // least 16 KB of other tiles, which the padding half of its MN-major operand reads
+    static constexpr int K_OFF = 0, V_OFF = NS * KB, PH_OFF = 2 * NS * KB, PL_OFF = PH_OFF + PB;
+    static constexpr int DH_OFF = PL_OFF + PB, DL_OFF = DH_OFF + PB, Q_OFF = DL_OFF + PB;
+    static constexpr int GH_OFF = Q_OFF + NS * QB, GL_OFF = GH_OFF + NS * QB;
+    static constexpr int BAR_OFF = GL_OFF + NS * QB;  // NS K/V mbarriers, the MMA mbarrier, TMEM base
+    static constexpr int WIN_OFF = BAR_OFF + 64;      // int [2][256]: list sizes and starts of a window of blocks
+    static constexpr int BYTES = WIN_OFF + 2 * 256 * 4;
     static constexpr int TCOLS = 128 + 3 * D;
     static constexpr bool supported = TCOLS <= 512 && BYTES <= 227 * 1024 && QB >= PB;
 };
@@ -1745,6 +1750,12 @@ struct BwdRemoteSmem {
 __device__ __forceinline__ uint32_t sw128(int r, int c) {  // 16-byte chunk c of row r, 128-row slabs of 64 columns
     return (uint32_t)((c >> 3) * (128 * 128) + r * 128 + (((c & 7) ^ (r & 7)) << 4));
 }
+
+// one chunk of the remote work: up to 128 selecting queries [g0, g0 + 128) of the CTA's k-th block (list entry
+// f = blockIdx.x + k gridDim.x, n queries from list position st); k < 0: none
+struct BwdChunk {
+    int k, g0, n, st;
+};
 
 template <int D>
 __global__ void __launch_bounds__(256, 1) k_bwd_remote_tc(const __grid_constant__ BwdMaps maps, const bf16 *__restrict__ Q,
@@ -1759,13 +1770,11 @@ __global__ void __launch_bounds__(256, 1) k_bwd_remote_tc(const __grid_constant_
     constexpr int BS = 64;
     using Lay = BwdRemoteSmem<D>;
     static_assert(Lay::supported, "tile shape");
-    constexpr int KB = Lay::KB, DH = D / 2;
+    constexpr int NS = Lay::NS, KB = Lay::KB, QB = Lay::QB, DH = D / 2;
     extern __shared__ __align__(1024) uint8_t smem[];
-    uint8_t *sK = smem + Lay::K_OFF, *sV = smem + Lay::V_OFF, *sQ = smem + Lay::Q_OFF;
-    uint8_t *sGH = smem + Lay::GH_OFF, *sGL = smem + Lay::GL_OFF;
     uint8_t *sPH = smem + Lay::PH_OFF, *sPL = smem + Lay::PL_OFF, *sDH = smem + Lay::DH_OFF, *sDL = smem + Lay::DL_OFF;
-    uint64_t *bar_ld = (uint64_t *)(smem + Lay::BAR_OFF), *mbar = bar_ld + 1;
-    uint32_t *tmem_base = (uint32_t *)(bar_ld + 2);
+    uint64_t *bar_kv = (uint64_t *)(smem + Lay::BAR_OFF), *mbar = bar_kv + NS;
+    uint32_t *tmem_base = (uint32_t *)(mbar + 1);
     if (timed_out(counters)) return;
     if (tc::smem_u32(smem) & 1023) {
         if (threadIdx.x == 0) record_error(counters, kDevErrSmemAlign);
@@ -1779,7 +1788,7 @@ __global__ void __launch_bounds__(256, 1) k_bwd_remote_tc(const __grid_constant_
         tc::tmem_relinquish();
     }
     if (tid == 0) {
-        tc::mbar_init(bar_ld, 1);
+        for (int i = 0; i < NS; ++i) tc::mbar_init(&bar_kv[i], 1);
         tc::mbar_init(mbar, 1);
         tc::fence_mbar_init();
     }
@@ -1792,187 +1801,274 @@ __global__ void __launch_bounds__(256, 1) k_bwd_remote_tc(const __grid_constant_
     const uint32_t tS = trow, tP = trow + 64, tQ = trow + 128, tV = trow + 128 + D, tK = trow + 128 + 2 * D;
     const uint32_t idS = tc::idesc_bf16(128, BS), idQ = tc::idesc_bf16(128, D, true),
                    idKV = tc::idesc_bf16(128, D, true, true);
-    bool ok = true;
-    int pend = -1;         // thread 0: the K/V load of block k issued and not yet seen complete
-    uint32_t mph = 0;      // completions of mbar so far, mod 2
-    int k = 0;             // blocks with K/V loaded so far
     const int total = nbh * nb;
-    for (int f = blockIdx.x; f < total && ok; f += gridDim.x) {
-        const int bh = f / nb, j = f % nb;
-        const int n = cnt[f];
-        if (n == 0) continue;  // uniform
-        const int32_t *lst = list + (size_t)bh * S * R + start[f];
-        if (tid == 0) {
-            tc::mbar_expect_tx(bar_ld, 2 * KB);
-#pragma unroll
-            for (int a = 0; a < D / 64; ++a) {
-                tc::tma_load_3d(sK + a * (BS * 128), &maps.k, 64 * a, j * BS, bh, bar_ld);
-                tc::tma_load_3d(sV + a * (BS * 128), &maps.v, 64 * a, j * BS, bh, bar_ld);
+
+    // This CTA's chunks in order: its blocks f = blockIdx.x + k gridDim.x with a nonempty list, 128 queries at a
+    // time.  The list sizes and starts of 256 of its blocks at a time sit in shared memory, so that finding the
+    // next chunk waits on no global load; the next chunk's list entries are requested at the top of a chunk, its
+    // rows gathered once the first products are issued, its log-sum-exp and D read there too.
+    int *s_bn = (int *)(smem + Lay::WIN_OFF), *s_bs = s_bn + 256;
+    const int G = gridDim.x;
+    int kw = -256;  // first k of the window
+    auto find_block = [&](int k) {  // the first of this CTA's blocks k' >= k with a nonempty list (uniform)
+        for (;; ++k) {
+            if ((long long)blockIdx.x + (long long)k * G >= total) return BwdChunk{-1, 0, 0, 0};
+            if (k >= kw + 256) {
+                __syncthreads();  // every thread is done with the old window
+                const long long f = (long long)blockIdx.x + (long long)(k + tid) * G;
+                s_bn[tid] = f < total ? cnt[f] : 0;
+                s_bs[tid] = f < total ? start[f] : 0;
+                __syncthreads();
+                kw = k;
             }
-            pend = k;
+            const int n = s_bn[k - kw];
+            if (n > 0) return BwdChunk{k, 0, n, s_bs[k - kw]};
         }
+    };
+    auto next_of = [&](const BwdChunk &c) {
+        if (c.g0 + 128 < c.n) return BwdChunk{c.k, c.g0 + 128, c.n, c.st};
+        return find_block(c.k + 1);
+    };
+    auto f_of = [&](const BwdChunk &c) { return blockIdx.x + c.k * G; };
+    constexpr int CPR = D / 8, KQ = 128 * CPR / 256;  // 16-byte segments per row; rows per thread in a gather
+    // the list entries of chunk c this thread gathers (rows tid / CPR + (256 / CPR) kq) and its softmax row's
+    auto req_idx = [&](const BwdChunk &c, int (&ri)[KQ], int &rt) {
+        const int f = f_of(c), bh = f / nb, ng = min(128, c.n - c.g0);
+        const int32_t *lst = list + (size_t)bh * S * R + c.st + c.g0;
+#pragma unroll
+        for (int kq = 0; kq < KQ; ++kq) {
+            const int r = tid / CPR + (256 / CPR) * kq;
+            ri[kq] = r < ng ? lst[r] : -1;
+        }
+        rt = row < ng ? lst[row] : -1;
+    };
+    // stage `st` of the gathered rows of chunk c (zeros past its end) from the requested entries
+    auto gather = [&](const BwdChunk &c, int st, const int (&ri)[KQ]) {
+        const int bh = f_of(c) / nb;
+        uint8_t *sQ = smem + Lay::Q_OFF + st * QB, *sGH = smem + Lay::GH_OFF + st * QB, *sGL = smem + Lay::GL_OFF + st * QB;
+        const int cc = tid % CPR;
+#pragma unroll
+        for (int kq = 0; kq < KQ; ++kq) {
+            const int r = tid / CPR + (256 / CPR) * kq;
+            const bool live = ri[kq] >= 0;
+            const size_t off = live ? ((size_t)bh * S + ri[kq]) * D + 8 * cc : 0;
+            tc::cp_async16(sQ + sw128(r, cc), Q + off, live);
+            tc::cp_async16(sGH + sw128(r, cc), dohi + off, live);
+            tc::cp_async16(sGL + sw128(r, cc), dolo + off, live);
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+    int pend[NS];  // thread 0: per K/V stage, the parity of a load issued and not yet seen complete, or -1
+#pragma unroll
+    for (int i = 0; i < NS; ++i) pend[i] = -1;
+    auto load_kv = [&](const BwdChunk &c, int kb) {  // K_j, V_j of chunk c's block into K/V stage kb % NS
+        if (tid != 0) return;
+        const int f = f_of(c), ks = kb % NS, bh = f / nb, j = f % nb;
+        uint8_t *sK = smem + Lay::K_OFF + ks * KB, *sV = smem + Lay::V_OFF + ks * KB;
+        tc::mbar_expect_tx(&bar_kv[ks], 2 * KB);
+#pragma unroll
+        for (int a = 0; a < D / 64; ++a) {
+            tc::tma_load_3d(sK + a * (BS * 128), &maps.k, 64 * a, j * BS, bh, &bar_kv[ks]);
+            tc::tma_load_3d(sV + a * (BS * 128), &maps.v, 64 * a, j * BS, bh, &bar_kv[ks]);
+        }
+        pend[ks] = (kb / NS) & 1;
+    };
+    // this thread's softmax row of a chunk: query, log-sum-exp (exp2 domain), D
+    auto row_stats = [&](const BwdChunk &c, int rt, int &t, float &l2, float &dd) {
+        const size_t base = (size_t)(f_of(c) / nb) * S;
+        t = rt >= 0 ? rt : 0;
+        l2 = rt >= 0 ? lse[base + rt] * 1.4426950408889634f : 0.f;
+        dd = rt >= 0 ? dsum[base + rt] : 0.f;
+    };
+
+    bool ok = true;
+    uint32_t mph = 0;  // completions of mbar so far, mod 2
+    BwdChunk c = find_block(0);
+    int kb = 0, ck = 0;  // blocks and chunks begun
+    int t_c = 0;
+    float lse_c = 0.f, D_c = 0.f;
+    if (c.k >= 0) {
+        int ri[KQ], rt;
+        req_idx(c, ri, rt);
+        load_kv(c, 0);
+        gather(c, 0, ri);
+        row_stats(c, rt, t_c, lse_c, D_c);
+    }
+    while (c.k >= 0 && ok) {
+        const int f = f_of(c), bh = f / nb, j = f % nb;
+        const int ng = min(128, c.n - c.g0);
+        const int st = ck % NS, ks = kb % NS;
+        const bool live = row < ng;
+        const int t = t_c;
+        const float lse2 = lse_c, Drow = D_c;
+        const BwdChunk nx = next_of(c);
+        const bool nx_new_block = nx.k != c.k;
+        int ri_nx[KQ], rt_nx = -1;
+        if (nx.k >= 0) {
+            req_idx(nx, ri_nx, rt_nx);  // used below (two stages) or after this chunk (one)
+            if (NS == 2 && nx_new_block) load_kv(nx, kb + 1);
+        }
+        tc::cp_async_wait_all();  // this chunk's rows (the only copies in flight)
         bool landed = true;
-        for (int g0 = 0; g0 < n && ok; g0 += 128) {
-            const int ng = min(128, n - g0);
-            // the chunk's query rows: Q, dO hi, dO lo (zeros past ng), eight threads per 128-byte segment
-            constexpr int CPR = D / 8;
-#pragma unroll
-            for (int kq = 0; kq < 128 * CPR / 256; ++kq) {
-                const int idx = tid + 256 * kq, r = idx / CPR, c = idx % CPR;
-                const bool live = r < ng;
-                const size_t off = live ? ((size_t)bh * S + lst[g0 + r]) * D + 8 * c : 0;
-                tc::cp_async16(sQ + sw128(r, c), Q + off, live);
-                tc::cp_async16(sGH + sw128(r, c), dohi + off, live);
-                tc::cp_async16(sGL + sw128(r, c), dolo + off, live);
-            }
-            asm volatile("cp.async.commit_group;" ::: "memory");
-            const bool live = row < ng;
-            const int t = live ? lst[g0 + row] : 0;
-            const float lse2 = live ? lse[(size_t)bh * S + t] * 1.4426950408889634f : 0.f;
-            const float Drow = live ? dsum[(size_t)bh * S + t] : 0.f;
-            tc::cp_async_wait_all();
-            if (tid == 0 && g0 == 0) {
-                landed = tc::mbar_wait(bar_ld, (uint32_t)(k & 1));
-                if (landed) pend = -1;
-            }
-            tc::fence_smem_to_async();
-            tc::fence_before_sync();
-            ok = __syncthreads_and(landed);
-            tc::fence_after_sync();
-            if (!ok) break;
-            if (tid == 0) {
-                const uint32_t aq = tc::smem_u32(sQ), ah = tc::smem_u32(sGH), al = tc::smem_u32(sGL);
-                const uint32_t bk = tc::smem_u32(sK), bv = tc::smem_u32(sV);
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t ao = (kk >> 2) * (128 * 128) + (kk & 3) * 32, bo = (kk >> 2) * (BS * 128) + (kk & 3) * 32;
-                    tc::mma_bf16(tmem, tc::desc_sw128(aq + ao), tc::desc_sw128(bk + bo), idS, kk > 0);
-                    tc::mma_bf16(tmem + 64, tc::desc_sw128(ah + ao), tc::desc_sw128(bv + bo), idS, kk > 0);
-                }
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t ao = (kk >> 2) * (128 * 128) + (kk & 3) * 32, bo = (kk >> 2) * (BS * 128) + (kk & 3) * 32;
-                    tc::mma_bf16(tmem + 64, tc::desc_sw128(al + ao), tc::desc_sw128(bv + bo), idS, 1u);
-                }
-                tc::commit(mbar);
-            }
-            ok = __syncthreads_and(tc::mbar_wait(mbar, mph));
-            mph ^= 1u;
-            tc::fence_after_sync();
-            if (!ok) break;
-            // P and dS of this row over the block's 64 keys (this warp's 32 of them), hi and lo terms
-            {
-                const int c0 = half * 32;
-                float sv[32], pv[32];
-                tc::tmem_ld32(tS + c0, sv);
-                tc::tmem_ld32(tP + c0, pv);
-                uint32_t ph[16], pl[16], dh[16], dl[16];
-#pragma unroll
-                for (int u = 0; u < 16; ++u) {
-                    const float p0 = live ? tc::ex2_fast(fmaf(sv[2 * u], scale_log2, -lse2)) : 0.f;
-                    const float p1 = live ? tc::ex2_fast(fmaf(sv[2 * u + 1], scale_log2, -lse2)) : 0.f;
-                    split2(p0, p1, ph[u], pl[u]);
-                    split2(p0 * (pv[2 * u] - Drow), p1 * (pv[2 * u + 1] - Drow), dh[u], dl[u]);
-                }
-#pragma unroll
-                for (int q8 = 0; q8 < 4; ++q8) {
-                    const uint32_t off = sw128(row, (c0 >> 3) + q8);
-                    *(uint4 *)(sPH + off) = make_uint4(ph[4 * q8], ph[4 * q8 + 1], ph[4 * q8 + 2], ph[4 * q8 + 3]);
-                    *(uint4 *)(sPL + off) = make_uint4(pl[4 * q8], pl[4 * q8 + 1], pl[4 * q8 + 2], pl[4 * q8 + 3]);
-                    *(uint4 *)(sDH + off) = make_uint4(dh[4 * q8], dh[4 * q8 + 1], dh[4 * q8 + 2], dh[4 * q8 + 3]);
-                    *(uint4 *)(sDL + off) = make_uint4(dl[4 * q8], dl[4 * q8 + 1], dl[4 * q8 + 2], dl[4 * q8 + 3]);
-                }
-            }
-            tc::fence_smem_to_async();
-            tc::fence_before_sync();
-            __syncthreads();
-            tc::fence_after_sync();
-            if (tid == 0) {
-                const uint32_t bk = tc::smem_u32(sK), bq = tc::smem_u32(sQ), gh = tc::smem_u32(sGH),
-                               gl = tc::smem_u32(sGL);
-                const uint32_t a_ph = tc::smem_u32(sPH), a_pl = tc::smem_u32(sPL), a_dh = tc::smem_u32(sDH),
-                               a_dl = tc::smem_u32(sDL);
-                // dQ_g = dS K_j: A = dS (K-major over the 64 keys), B = K_j (MN-major)
-#pragma unroll
-                for (int kk = 0; kk < BS / 16; ++kk) {
-                    const uint64_t bd = tc::desc_sw128_mn(bk + 2048 * kk, BS * 128);
-                    tc::mma_bf16(tmem + 128, tc::desc_sw128(a_dh + 32 * kk), bd, idQ, kk > 0);
-                    tc::mma_bf16(tmem + 128, tc::desc_sw128(a_dl + 32 * kk), bd, idQ, 1u);
-                }
-                // dV_j += P^T dO_g and dK_j += dS^T Q_g: A = P, dS read MN-major (M = keys; the second 64-key
-                // half of the 128-row operand points at another tile and its rows are not read), K = the chunk's
-                // queries, B = dO, Q (MN-major)
-#pragma unroll
-                for (int kk = 0; kk < 128 / 16; ++kk) {
-                    const bool acc = g0 > 0 || kk > 0;
-                    const uint64_t bgh = tc::desc_sw128_mn(gh + 2048 * kk, 128 * 128);
-                    const uint64_t bgl = tc::desc_sw128_mn(gl + 2048 * kk, 128 * 128);
-                    const uint64_t bqd = tc::desc_sw128_mn(bq + 2048 * kk, 128 * 128);
-                    const uint64_t aph = tc::desc_sw128_mn(a_ph + 2048 * kk, Lay::PB);
-                    const uint64_t apl = tc::desc_sw128_mn(a_pl + 2048 * kk, Lay::PB);
-                    const uint64_t adh = tc::desc_sw128_mn(a_dh + 2048 * kk, Lay::PB);
-                    const uint64_t adl = tc::desc_sw128_mn(a_dl + 2048 * kk, Lay::PB);
-                    tc::mma_bf16(tmem + 128 + D, aph, bgh, idKV, acc);
-                    tc::mma_bf16(tmem + 128 + D, aph, bgl, idKV, 1u);
-                    tc::mma_bf16(tmem + 128 + D, apl, bgh, idKV, 1u);
-                    tc::mma_bf16(tmem + 128 + 2 * D, adh, bqd, idKV, acc);
-                    tc::mma_bf16(tmem + 128 + 2 * D, adl, bqd, idKV, 1u);
-                }
-                tc::commit(mbar);
-            }
-            ok = __syncthreads_and(tc::mbar_wait(mbar, mph));
-            mph ^= 1u;
-            tc::fence_after_sync();
-            if (!ok) break;
-            // this row's dQ part, added to the query's fp32 dQ
-#pragma unroll 1
-            for (int c0 = half * DH; c0 < half * DH + DH; c0 += 32) {
-                float v[32];
-                tc::tmem_ld32(tQ + c0, v);
-                if (live) {
-                    float4 *dst = (float4 *)(dq_loc + ((size_t)bh * S + t) * D + c0);
-#pragma unroll
-                    for (int q4 = 0; q4 < 8; ++q4)
-                        atomicAdd(dst + q4, make_float4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]));
-                }
-            }
-            tc::fence_before_sync();
-            __syncthreads();  // shared memory and the S, dP, dQ columns are free for the next chunk
-            tc::fence_after_sync();
+        if (tid == 0 && c.g0 == 0) {
+            landed = tc::mbar_wait(&bar_kv[ks], (uint32_t)((kb / NS) & 1));
+            if (landed) pend[ks] = -1;
         }
+        tc::fence_smem_to_async();
+        tc::fence_before_sync();
+        ok = __syncthreads_and(landed);
+        tc::fence_after_sync();
         if (!ok) break;
-        ++k;
-        // dV_j and dK_j: TMEM rows 0..63 (lane quarters 0 and 1; quarters 2 and 3 hold the padding rows), added to
-        // the local parts of the block's keys
-        if (quarter < 2) {
-            const size_t key = (size_t)bh * S + j * BS + row;
-#pragma unroll 1
-            for (int c0 = half * DH; c0 < half * DH + DH; c0 += 32) {
-                float v[32], g[32];
-                tc::tmem_ld32(tV + c0, v);
-                tc::tmem_ld32(tK + c0, g);
-                float4 *dv = (float4 *)(dv_loc + key * D + c0);
-                float4 *dk = (float4 *)(dk_loc + key * D + c0);
+        const uint8_t *sK = smem + Lay::K_OFF + ks * KB, *sV = smem + Lay::V_OFF + ks * KB;
+        const uint8_t *sQ = smem + Lay::Q_OFF + st * QB, *sGH = smem + Lay::GH_OFF + st * QB,
+                      *sGL = smem + Lay::GL_OFF + st * QB;
+        if (tid == 0) {
+            const uint32_t aq = tc::smem_u32(sQ), ah = tc::smem_u32(sGH), al = tc::smem_u32(sGL);
+            const uint32_t bk = tc::smem_u32(sK), bv = tc::smem_u32(sV);
 #pragma unroll
-                for (int q4 = 0; q4 < 8; ++q4) {
-                    const float4 a = dv[q4], b = dk[q4];
-                    dv[q4] = make_float4(a.x + v[4 * q4], a.y + v[4 * q4 + 1], a.z + v[4 * q4 + 2], a.w + v[4 * q4 + 3]);
-                    dk[q4] = make_float4(b.x + g[4 * q4], b.y + g[4 * q4 + 1], b.z + g[4 * q4 + 2], b.w + g[4 * q4 + 3]);
+            for (int kk = 0; kk < D / 16; ++kk) {
+                const uint32_t ao = (kk >> 2) * (128 * 128) + (kk & 3) * 32, bo = (kk >> 2) * (BS * 128) + (kk & 3) * 32;
+                tc::mma_bf16(tmem, tc::desc_sw128(aq + ao), tc::desc_sw128(bk + bo), idS, kk > 0);
+                tc::mma_bf16(tmem + 64, tc::desc_sw128(ah + ao), tc::desc_sw128(bv + bo), idS, kk > 0);
+            }
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+                const uint32_t ao = (kk >> 2) * (128 * 128) + (kk & 3) * 32, bo = (kk >> 2) * (BS * 128) + (kk & 3) * 32;
+                tc::mma_bf16(tmem + 64, tc::desc_sw128(al + ao), tc::desc_sw128(bv + bo), idS, 1u);
+            }
+            tc::commit(mbar);
+        }
+        if (NS == 2 && nx.k >= 0) {  // the next chunk's rows load while this one is computed
+            gather(nx, (ck + 1) % NS, ri_nx);
+            row_stats(nx, rt_nx, t_c, lse_c, D_c);
+        }
+        ok = __syncthreads_and(tc::mbar_wait(mbar, mph));
+        mph ^= 1u;
+        tc::fence_after_sync();
+        if (!ok) break;
+        // P and dS of this row over the block's 64 keys (this warp's 32 of them), hi and lo terms
+        {
+            const int c0 = half * 32;
+            float sv[32], pv[32];
+            tc::tmem_ld32(tS + c0, sv);
+            tc::tmem_ld32(tP + c0, pv);
+            uint32_t ph[16], pl[16], dh[16], dl[16];
+#pragma unroll
+            for (int u = 0; u < 16; ++u) {
+                const float p0 = live ? tc::ex2_fast(fmaf(sv[2 * u], scale_log2, -lse2)) : 0.f;
+                const float p1 = live ? tc::ex2_fast(fmaf(sv[2 * u + 1], scale_log2, -lse2)) : 0.f;
+                split2(p0, p1, ph[u], pl[u]);
+                split2(p0 * (pv[2 * u] - Drow), p1 * (pv[2 * u + 1] - Drow), dh[u], dl[u]);
+            }
+#pragma unroll
+            for (int q8 = 0; q8 < 4; ++q8) {
+                const uint32_t off = sw128(row, (c0 >> 3) + q8);
+                *(uint4 *)(sPH + off) = make_uint4(ph[4 * q8], ph[4 * q8 + 1], ph[4 * q8 + 2], ph[4 * q8 + 3]);
+                *(uint4 *)(sPL + off) = make_uint4(pl[4 * q8], pl[4 * q8 + 1], pl[4 * q8 + 2], pl[4 * q8 + 3]);
+                *(uint4 *)(sDH + off) = make_uint4(dh[4 * q8], dh[4 * q8 + 1], dh[4 * q8 + 2], dh[4 * q8 + 3]);
+                *(uint4 *)(sDL + off) = make_uint4(dl[4 * q8], dl[4 * q8 + 1], dl[4 * q8 + 2], dl[4 * q8 + 3]);
+            }
+        }
+        tc::fence_smem_to_async();
+        tc::fence_before_sync();
+        __syncthreads();
+        tc::fence_after_sync();
+        if (tid == 0) {
+            const uint32_t bk = tc::smem_u32(sK), bq = tc::smem_u32(sQ), gh = tc::smem_u32(sGH),
+                           gl = tc::smem_u32(sGL);
+            const uint32_t a_ph = tc::smem_u32(sPH), a_pl = tc::smem_u32(sPL), a_dh = tc::smem_u32(sDH),
+                           a_dl = tc::smem_u32(sDL);
+            // dQ_g = dS K_j: A = dS (K-major over the 64 keys), B = K_j (MN-major)
+#pragma unroll
+            for (int kk = 0; kk < BS / 16; ++kk) {
+                const uint64_t bd = tc::desc_sw128_mn(bk + 2048 * kk, BS * 128);
+                tc::mma_bf16(tmem + 128, tc::desc_sw128(a_dh + 32 * kk), bd, idQ, kk > 0);
+                tc::mma_bf16(tmem + 128, tc::desc_sw128(a_dl + 32 * kk), bd, idQ, 1u);
+            }
+            // dV_j += P^T dO_g and dK_j += dS^T Q_g: A = P, dS read MN-major (M = keys; the second 64-key
+            // half of the 128-row operand points at another tile and its rows are not read), K = the chunk's
+            // queries, B = dO, Q (MN-major)
+#pragma unroll
+            for (int kk = 0; kk < 128 / 16; ++kk) {
+                const bool acc = c.g0 > 0 || kk > 0;
+                const uint64_t bgh = tc::desc_sw128_mn(gh + 2048 * kk, 128 * 128);
+                const uint64_t bgl = tc::desc_sw128_mn(gl + 2048 * kk, 128 * 128);
+                const uint64_t bqd = tc::desc_sw128_mn(bq + 2048 * kk, 128 * 128);
+                const uint64_t aph = tc::desc_sw128_mn(a_ph + 2048 * kk, Lay::PB);
+                const uint64_t apl = tc::desc_sw128_mn(a_pl + 2048 * kk, Lay::PB);
+                const uint64_t adh = tc::desc_sw128_mn(a_dh + 2048 * kk, Lay::PB);
+                const uint64_t adl = tc::desc_sw128_mn(a_dl + 2048 * kk, Lay::PB);
+                tc::mma_bf16(tmem + 128 + D, aph, bgh, idKV, acc);
+                tc::mma_bf16(tmem + 128 + D, aph, bgl, idKV, 1u);
+                tc::mma_bf16(tmem + 128 + D, apl, bgh, idKV, 1u);
+                tc::mma_bf16(tmem + 128 + 2 * D, adh, bqd, idKV, acc);
+                tc::mma_bf16(tmem + 128 + 2 * D, adl, bqd, idKV, 1u);
+            }
+            tc::commit(mbar);
+        }
+        ok = __syncthreads_and(tc::mbar_wait(mbar, mph));
+        mph ^= 1u;
+        tc::fence_after_sync();
+        if (!ok) break;
+        // this row's dQ part, added to the query's fp32 dQ
+#pragma unroll 1
+        for (int c0 = half * DH; c0 < half * DH + DH; c0 += 32) {
+            float v[32];
+            tc::tmem_ld32(tQ + c0, v);
+            if (live) {
+                float4 *dst = (float4 *)(dq_loc + ((size_t)bh * S + t) * D + c0);
+#pragma unroll
+                for (int q4 = 0; q4 < 8; ++q4)
+                    atomicAdd(dst + q4, make_float4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]));
+            }
+        }
+        if (nx_new_block) {
+            // dV_j and dK_j: TMEM rows 0..63 (lane quarters 0 and 1; quarters 2 and 3 hold the padding rows), added
+            // to the local parts of the block's keys (only this CTA writes them)
+            if (quarter < 2) {
+                const size_t key = (size_t)bh * S + j * BS + row;
+#pragma unroll 1
+                for (int c0 = half * DH; c0 < half * DH + DH; c0 += 32) {
+                    float v[32], g[32];
+                    tc::tmem_ld32(tV + c0, v);
+                    tc::tmem_ld32(tK + c0, g);
+                    float4 *dv = (float4 *)(dv_loc + key * D + c0);
+                    float4 *dk = (float4 *)(dk_loc + key * D + c0);
+#pragma unroll
+                    for (int q4 = 0; q4 < 8; ++q4) {
+                        const float4 a = dv[q4], b = dk[q4];
+                        dv[q4] = make_float4(a.x + v[4 * q4], a.y + v[4 * q4 + 1], a.z + v[4 * q4 + 2],
+                                             a.w + v[4 * q4 + 3]);
+                        dk[q4] = make_float4(b.x + g[4 * q4], b.y + g[4 * q4 + 1], b.z + g[4 * q4 + 2],
+                                             b.w + g[4 * q4 + 3]);
+                    }
                 }
             }
+            ++kb;
         }
         tc::fence_before_sync();
-        __syncthreads();  // K/V tiles and the dV/dK columns are free for the next block
+        __syncthreads();  // this chunk's shared memory and TMEM columns are free
         tc::fence_after_sync();
+        if (NS == 1 && nx.k >= 0) {  // one stage: the next chunk loads only now
+            if (nx_new_block) load_kv(nx, kb);
+            gather(nx, 0, ri_nx);
+            row_stats(nx, rt_nx, t_c, lse_c, D_c);
+        }
+        c = nx;
+        ++ck;
     }
-    // leave no TMA write in flight into this CTA's shared memory
-    if (tid == 0 && pend >= 0 && !tc::mbar_wait(bar_ld, (uint32_t)(pend & 1))) ok = false;
+    // leave no copy in flight into this CTA's shared memory
+    tc::cp_async_wait_all();
+    if (tid == 0) {
+#pragma unroll
+        for (int i = 0; i < NS; ++i)
+            if (pend[i] >= 0 && !tc::mbar_wait(&bar_kv[i], (uint32_t)pend[i])) ok = false;
+    }
     if (!ok && tid == 0) record_error(counters, kDevErrTimeout);
     tc::fence_before_sync();
     __syncthreads();
     if (warp == 0) tc::tmem_dealloc(tmem, 512);
 }
-
 
 template <int D, int BS, int NK>
 static cudaError_t launch_bwd_local_dq_shape(const Plan &p, const void *Q, const void *K, const void *V,
