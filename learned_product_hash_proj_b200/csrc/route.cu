@@ -959,10 +959,20 @@ template <typename T, int D>
 constexpr int probe_q_pitch() {
     return D * (int)sizeof(T) + 16;
 }
-// queries per thread: two where both queries' subspace scores fit in registers
+// queries per thread (one: a thread's scores and probe state fit in 80 registers, so six CTAs of 128 threads
+// share an SM and their warps hide each other's latency; two queries per thread at 128 registers, which share
+// every codebook read, measured 12 % slower), threads per CTA and the CTAs per SM the register budget is sized for
 template <int C>
 constexpr int probe_nq() {
-    return C <= 16 ? 2 : 1;
+    return 1;
+}
+template <int C>
+constexpr int probe_threads() {
+    return 128;
+}
+template <int C>
+constexpr int probe_min_ctas() {
+    return C <= 16 ? 6 : 3;
 }
 // shared memory of the probe's candidates: ids (int16), counts, rerank scores
 template <int E>
@@ -973,8 +983,8 @@ static_assert(kMaxNb <= 32768, "block ids fit int16");
 
 template <typename T, int D, int C, int E>
 constexpr size_t probe_m2_smem(int nb) {
-    return (size_t)C * D * 4 + (size_t)C * C * 8 + (size_t)128 * probe_nq<C>() * probe_q_pitch<T, D>() +
-           cand_smem<E>(128 * probe_nq<C>()) + (size_t)nb * 8;
+    return (size_t)C * D * 4 + (size_t)C * C * 8 + (size_t)probe_threads<C>() * probe_nq<C>() * probe_q_pitch<T, D>() +
+           cand_smem<E>(probe_threads<C>() * probe_nq<C>()) + (size_t)nb * 8;
 }
 
 // Top R of the candidates' rerank scores acc (score desc, id asc), the forced
@@ -1028,7 +1038,7 @@ __device__ __forceinline__ int select_top_r(const float (&acc)[E], const int (&c
 }
 
 // The rerank scores of the query-heads a warp probed (its threads' rows
-// qi = tid + 128 q, q < NQ, of the CTA's tile; each one's candidates in
+// qi = tid + NT q, q < NQ, of the CTA's tile; each one's candidates in
 // s_cid[qi][E], their number in s_nc[qi]) into s_score[qi][E], eight lanes
 // per query-head: lane l of a group holds run l (elements [l D/8, (l+1) D/8))
 // of q and reads the same run of each candidate's kbar row, so a group reads
@@ -1036,7 +1046,7 @@ __device__ __forceinline__ int select_top_r(const float (&acc)[E], const int (&c
 // form the tree ((c0 + c1) + (c2 + c3)) + ((c4 + c5) + (c6 + c7)) in every
 // lane of the group (fp32 addition is commutative, so both partners get the
 // same bits).  Four query-heads per round, two rounds' loads in flight.
-template <typename T, int D, int E, int NQ>
+template <typename T, int D, int E, int NQ, int NT>
 __device__ __forceinline__ void rerank_scores(const uint8_t *s_q, int qpitch, const int16_t *s_cid,
                                               const int32_t *s_nc, const float *kb, float *s_score) {
     constexpr int RUN = D / 8, RPI = 2;
@@ -1049,7 +1059,7 @@ __device__ __forceinline__ void rerank_scores(const uint8_t *s_q, int qpitch, co
 #pragma unroll
         for (int h = 0; h < RPI; ++h) {
             const int wq = 4 * (r0 + h) + grp;
-            qi[h] = 32 * warp + (wq & 31) + 128 * (wq >> 5);
+            qi[h] = 32 * warp + (wq & 31) + NT * (wq >> 5);
             nc[h] = s_nc[qi[h]];
 #pragma unroll
             for (int i8 = 0; i8 < RUN / 8; ++i8) {
@@ -1144,15 +1154,15 @@ __device__ __forceinline__ int rerank_thread(const T *qp, const float *kb, const
     return select_top_r<E, R>(acc, cid, nc, forced, out, t, bh, S, Bs, L, ign);
 }
 
-// The top-R selection of this thread's query-heads (rows tid + 128 q) from
+// The top-R selection of this thread's query-heads (rows tid + NT q) from
 // their candidates and rerank scores in shared memory; adds to the counts.
-template <int E, int R, int NQ>
+template <int E, int R, int NQ, int NT>
 __device__ __forceinline__ void select_rows(const int16_t *s_cid, const int32_t *s_nc, const float *s_score,
                                             const int32_t *forced, int32_t *sel, int t_lo, size_t bh, int S, int Bs,
                                             int L, int &n_sel, int &lt_r, int &ign) {
 #pragma unroll
     for (int q = 0; q < NQ; ++q) {
-        const int qi = threadIdx.x + 128 * q, t = t_lo + qi;
+        const int qi = threadIdx.x + NT * q, t = t_lo + qi;
         if (t >= S) continue;
         int cid[E];
         float acc[E];
@@ -1275,20 +1285,21 @@ __device__ __forceinline__ int probe_m2(const float (&s0)[C], const float (&s1)[
 }
 
 // M = 2 with every size fixed at compile time, so all per-query state stays
-// in registers.  A CTA takes 128 x NQ consecutive queries of one (b, h); its
-// thread tid the queries tid, tid + 128, ...  Everything the CTA reads more
+// in registers.  A CTA takes NT x NQ consecutive queries of one (b, h); its
+// thread tid the queries tid, tid + NT, ...  Everything the CTA reads more
 // than once goes to shared memory in one batch: the query rows, the head's
 // codebooks (transposed for the paired chains) and the (b, h) posting arrays.
 // Same pruning rule and arithmetic order as k_probe_rerank.
 template <typename T, int D, int C, int TP, int E, int R>
-__global__ void __launch_bounds__(128, C <= 16 ? 4 : 3) k_probe_m2(const T *__restrict__ Q, const float *__restrict__ kbar,
+__global__ void __launch_bounds__(probe_threads<C>(), probe_min_ctas<C>()) k_probe_m2(const T *__restrict__ Q, const float *__restrict__ kbar,
                                                      const float *__restrict__ cb, const int32_t *__restrict__ post_ids,
                                                      const int32_t *__restrict__ post_addr,
                                                      const int32_t *__restrict__ forced, int32_t *__restrict__ sel,
                                                      unsigned long long *__restrict__ counters,
                                                      int32_t *__restrict__ walk_log, int S, int H, int Bs,
                                                      int L, int cap) {
-    constexpr int DM = D / 2, A = C * C, QP = probe_q_pitch<T, D>(), NQ = probe_nq<C>(), QT = 128 * NQ;
+    constexpr int DM = D / 2, A = C * C, QP = probe_q_pitch<T, D>(), NQ = probe_nq<C>(), NT = probe_threads<C>();
+    constexpr int QT = NT * NQ;
     static_assert(C <= 32 && TP <= C * C && R >= 1 && E >= 1 && QP % 16 == 0 && DM % 8 == 0, "shape");
     extern __shared__ __align__(16) float smem[];
     pdl_launch_dependents();  // the attention's first kernel may start; it waits for sel itself
@@ -1337,7 +1348,7 @@ __global__ void __launch_bounds__(128, C <= 16 ? 4 : 3) k_probe_m2(const T *__re
         const T *qm0[NQ], *qm1[NQ];
 #pragma unroll
         for (int q = 0; q < NQ; ++q) {
-            qm0[q] = (const T *)(s_q + (tid + 128 * q) * QP);
+            qm0[q] = (const T *)(s_q + (tid + NT * q) * QP);
             qm1[q] = qm0[q] + DM;
         }
         sub_scores_x2<T, DM, C, NQ>(qm0, s_cbT, s0);
@@ -1371,7 +1382,7 @@ __global__ void __launch_bounds__(128, C <= 16 ? 4 : 3) k_probe_m2(const T *__re
     __syncthreads();
 #pragma unroll
     for (int q = 0; q < NQ; ++q) {
-        const int qi = tid + 128 * q, t = t_lo + qi;
+        const int qi = tid + NT * q, t = t_lo + qi;
         int cid[E] = {};
         const int nc = t < S ? probe_m2<C, TP, E>(s0[q], s1[q], s_rng, s_ids, cid, t, bh, S, Bs, L, cap, counters,
                                                   walk_log)
@@ -1381,10 +1392,10 @@ __global__ void __launch_bounds__(128, C <= 16 ? 4 : 3) k_probe_m2(const T *__re
         s_nc[qi] = nc;
     }
     __syncwarp();
-    rerank_scores<T, D, E, NQ>(s_q, QP, s_cid, s_nc, kbar + bh * nb * D, s_score);
+    rerank_scores<T, D, E, NQ, NT>(s_q, QP, s_cid, s_nc, kbar + bh * nb * D, s_score);
     __syncwarp();
     int n_sel = 0, lt_r = 0, ign = 0;
-    select_rows<E, R, NQ>(s_cid, s_nc, s_score, forced, sel, t_lo, bh, S, Bs, L, n_sel, lt_r, ign);
+    select_rows<E, R, NQ, NT>(s_cid, s_nc, s_score, forced, sel, t_lo, bh, S, Bs, L, n_sel, lt_r, ign);
     for (int o = 16; o > 0; o >>= 1) {
         n_sel += __shfl_xor_sync(0xffffffffu, n_sel, o);
         lt_r += __shfl_xor_sync(0xffffffffu, lt_r, o);
@@ -1872,11 +1883,11 @@ cudaError_t launch_lists(const Plan &p, void *ws, cudaStream_t s) {
 // a probe kernel, launched so that it may start while the lists kernel before
 // it on the stream still runs (it waits for the lists itself: pdl_wait_primary)
 template <typename... KArgs, typename... Args>
-static cudaError_t launch_after_lists(void (*kern)(KArgs...), dim3 grid, size_t smem, cudaStream_t s,
+static cudaError_t launch_after_lists(void (*kern)(KArgs...), dim3 grid, int threads, size_t smem, cudaStream_t s,
                                       Args... args) {
     cudaLaunchConfig_t lc = {};
     lc.gridDim = grid;
-    lc.blockDim = dim3(128);
+    lc.blockDim = dim3(threads);
     lc.dynamicSmemBytes = smem;
     lc.stream = s;
     cudaLaunchAttribute at[1];
@@ -1909,8 +1920,9 @@ cudaError_t launch_queries(const Plan &p, const void *Q, const float *cb, const 
         if (sm2 > 48 * 1024 &&                                                                                   \
             (e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm2)) != cudaSuccess) \
             return e;                                                                                            \
-        const dim3 gm2((c.S + 128 * probe_nq<CC>() - 1) / (128 * probe_nq<CC>()), c.H, c.B);                  \
-        if ((e = launch_after_lists(kern, gm2, sm2, s, (const TT *)Q, kbar, cb, ids, saddr, forced, sel, cnt,        \
+        const dim3 gm2((c.S + probe_threads<CC>() * probe_nq<CC>() - 1) / (probe_threads<CC>() * probe_nq<CC>()), c.H, \
+                       c.B);                  \
+        if ((e = launch_after_lists(kern, gm2, probe_threads<CC>(), sm2, s, (const TT *)Q, kbar, cb, ids, saddr, forced, sel, cnt,        \
                                     walk_log, c.S, c.H, c.Bs, c.L, c.cap)) != cudaSuccess)                          \
             return e;                                                                                            \
         count_launches(1);                                                                                       \
@@ -1931,7 +1943,7 @@ cudaError_t launch_queries(const Plan &p, const void *Q, const float *cb, const 
         if (smb > 48 * 1024 &&                                                                                   \
             (e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smb)) != cudaSuccess) \
             return e;                                                                                            \
-        if ((e = launch_after_lists(kern, g3, smb, s, (const TT *)Q, kbar, cb, ids, saddr, forced, sel, cnt,         \
+        if ((e = launch_after_lists(kern, g3, 128, smb, s, (const TT *)Q, kbar, cb, ids, saddr, forced, sel, cnt,         \
                                     walk_log, c.S, c.H, c.Bs, c.L, c.cap)) != cudaSuccess)                          \
             return e;                                                                                            \
         count_launches(1);                                                                                       \
@@ -1953,7 +1965,7 @@ cudaError_t launch_queries(const Plan &p, const void *Q, const float *cb, const 
             e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);                \
             if (e != cudaSuccess) return e;                                                                        \
         }                                                                                                          \
-        if ((e = launch_after_lists(kern, g3, smem, s, (const TT *)Q, kbar, cb, ids, saddr, forced, sel, cnt,        \
+        if ((e = launch_after_lists(kern, g3, 128, smem, s, (const TT *)Q, kbar, cb, ids, saddr, forced, sel, cnt,        \
                                     walk_log, c.S, c.H, c.Bs, c.L, c.R, c.E, c.M, c.C, c.T, c.cap)) != cudaSuccess)  \
             return e;                                                                                              \
     } while (0)
