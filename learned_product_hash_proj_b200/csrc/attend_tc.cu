@@ -1720,7 +1720,7 @@ __global__ void __launch_bounds__(256, 1) k_bwd_local_dkdv_tc(const __grid_const
 // swizzled layout (eight threads per row).  Per chunk of queries g:
 //   S = Q_g K_j^T,  dP = dO_g V_j^T           (TMEM columns [0, 64), [64, 128))
 //   P = exp(S / sqrt(d) - lse),  dS = P (dP - D)   (every key of a selected block is visible)
-//   dQ_g = dS K_j        -> added to dq_loc rows with fp32 vector atomics (a query has several blocks)
+//   dQ_g = dS K_j        -> one fp32 row per (query, slot) in dq_pair, summed in slot order later
 //   dV_j += P^T dO_g,  dK_j += dS^T Q_g      (TMEM, over all chunks of the block)
 // P and dS are stored once, row-major by query as two bf16 terms each; the
 // row-major tile is the K-major A operand of dQ and the MN-major A operand
@@ -1763,7 +1763,7 @@ __global__ void __launch_bounds__(256, 1) k_bwd_remote_tc(const __grid_constant_
                                                           const float *__restrict__ lse, const float *__restrict__ dsum,
                                                           const int32_t *__restrict__ cnt,
                                                           const int32_t *__restrict__ start,
-                                                          const int32_t *__restrict__ list, float *__restrict__ dq_loc,
+                                                          const int32_t *__restrict__ list, float *__restrict__ dq_pair,
                                                           float *__restrict__ dk_loc, float *__restrict__ dv_loc,
                                                           unsigned long long *__restrict__ counters, int S, int R,
                                                           int nb, float scale_log2, int nbh) {
@@ -1838,9 +1838,9 @@ __global__ void __launch_bounds__(256, 1) k_bwd_remote_tc(const __grid_constant_
 #pragma unroll
         for (int kq = 0; kq < KQ; ++kq) {
             const int r = tid / CPR + (256 / CPR) * kq;
-            ri[kq] = r < ng ? lst[r] : -1;
+            ri[kq] = r < ng ? lst[r] / R : -1;
         }
-        rt = row < ng ? lst[row] : -1;
+        rt = row < ng ? lst[row] : -1;  // the pair t * R + r
     };
     // stage `st` of the gathered rows of chunk c (zeros past its end) from the requested entries
     auto gather = [&](const BwdChunk &c, int st, const int (&ri)[KQ]) {
@@ -1873,12 +1873,12 @@ __global__ void __launch_bounds__(256, 1) k_bwd_remote_tc(const __grid_constant_
         }
         pend[ks] = (kb / NS) & 1;
     };
-    // this thread's softmax row of a chunk: query, log-sum-exp (exp2 domain), D
+    // this thread's softmax row of a chunk: pair, log-sum-exp of its query (exp2 domain), D
     auto row_stats = [&](const BwdChunk &c, int rt, int &t, float &l2, float &dd) {
         const size_t base = (size_t)(f_of(c) / nb) * S;
         t = rt >= 0 ? rt : 0;
-        l2 = rt >= 0 ? lse[base + rt] * 1.4426950408889634f : 0.f;
-        dd = rt >= 0 ? dsum[base + rt] : 0.f;
+        l2 = rt >= 0 ? lse[base + rt / R] * 1.4426950408889634f : 0.f;
+        dd = rt >= 0 ? dsum[base + rt / R] : 0.f;
     };
 
     bool ok = true;
@@ -2010,16 +2010,15 @@ __global__ void __launch_bounds__(256, 1) k_bwd_remote_tc(const __grid_constant_
         mph ^= 1u;
         tc::fence_after_sync();
         if (!ok) break;
-        // this row's dQ part, added to the query's fp32 dQ
+        // this row's dQ part, to its (query, slot) row (t holds the pair)
 #pragma unroll 1
         for (int c0 = half * DH; c0 < half * DH + DH; c0 += 32) {
             float v[32];
             tc::tmem_ld32(tQ + c0, v);
             if (live) {
-                float4 *dst = (float4 *)(dq_loc + ((size_t)bh * S + t) * D + c0);
+                float4 *dst = (float4 *)(dq_pair + ((size_t)bh * S * R + t) * D + c0);
 #pragma unroll
-                for (int q4 = 0; q4 < 8; ++q4)
-                    atomicAdd(dst + q4, make_float4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]));
+                for (int q4 = 0; q4 < 8; ++q4) dst[q4] = make_float4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
             }
         }
         if (nx_new_block) {
@@ -2143,7 +2142,7 @@ template <int D>
 static cudaError_t launch_bwd_remote_shape(const Plan &p, const void *Q, const void *K, const void *V,
                                            const void *dohi, const void *dolo, const float *lse, const float *dsum,
                                            const int32_t *cnt, const int32_t *start, const int32_t *list,
-                                           float *dq_loc, float *dk_loc, float *dv_loc, unsigned long long *counters,
+                                           float *dq_pair, float *dk_loc, float *dv_loc, unsigned long long *counters,
                                            cudaStream_t s) {
     const mono_config &c = p.cfg;
     using Lay = BwdRemoteSmem<D>;
@@ -2165,7 +2164,7 @@ static cudaError_t launch_bwd_remote_shape(const Plan &p, const void *Q, const v
     const float scale_log2 = (float)(1.4426950408889634 / sqrt((double)c.d));
     const int total = BH * p.nb;
     kern<<<std::min(total, sms), 256, Lay::BYTES, s>>>(maps, (const bf16 *)Q, (const bf16 *)dohi, (const bf16 *)dolo,
-                                                       lse, dsum, cnt, start, list, dq_loc, dk_loc, dv_loc, counters,
+                                                       lse, dsum, cnt, start, list, dq_pair, dk_loc, dv_loc, counters,
                                                        c.S, c.R, p.nb, scale_log2, BH);
     count_launches(1);
     return cudaGetLastError();
@@ -2173,14 +2172,14 @@ static cudaError_t launch_bwd_remote_shape(const Plan &p, const void *Q, const v
 
 cudaError_t launch_bwd_remote_tc(const Plan &p, const void *Q, const void *K, const void *V, const void *dohi,
                                  const void *dolo, const float *lse, const float *dsum, const int32_t *cnt,
-                                 const int32_t *start, const int32_t *list, float *dq_loc, float *dk_loc,
+                                 const int32_t *start, const int32_t *list, float *dq_pair, float *dk_loc,
                                  float *dv_loc, unsigned long long *counters, cudaStream_t s) {
     const mono_config &c = p.cfg;
     if (!bwd_local_dq_tc_supported(c)) return cudaErrorInvalidValue;
     if (c.d == 64)
-        return launch_bwd_remote_shape<64>(p, Q, K, V, dohi, dolo, lse, dsum, cnt, start, list, dq_loc, dk_loc,
+        return launch_bwd_remote_shape<64>(p, Q, K, V, dohi, dolo, lse, dsum, cnt, start, list, dq_pair, dk_loc,
                                            dv_loc, counters, s);
-    return launch_bwd_remote_shape<128>(p, Q, K, V, dohi, dolo, lse, dsum, cnt, start, list, dq_loc, dk_loc, dv_loc,
+    return launch_bwd_remote_shape<128>(p, Q, K, V, dohi, dolo, lse, dsum, cnt, start, list, dq_pair, dk_loc, dv_loc,
                                         counters, s);
 }
 

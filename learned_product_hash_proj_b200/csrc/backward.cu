@@ -46,7 +46,9 @@ namespace mono {
 namespace {
 
 struct BwdLayout {
-    size_t lse, dsum, cnt, start, cursor, list, dO, dQp, dKp, dVp, dOhi, dOlo, dQloc, dKloc, dVloc, total;
+    size_t lse, dsum, cnt, start, cursor, list, sortbuf, slab, dO, dQp, dKp, dVp, dOhi, dOlo, dQloc, dKloc, dVloc,
+        dQpair, total;
+    size_t slab_bytes;
 };
 
 BwdLayout bwd_layout(const Plan &p) {
@@ -65,6 +67,10 @@ BwdLayout bwd_layout(const Plan &p) {
     L.start = take(B * H * nb * 4);
     L.cursor = take(B * H * nb * 4);
     L.list = take(B * H * S * R * 4);
+    L.sortbuf = take(2 * B * H * S * R * 4);  // a list segment too long for shared memory, padded to a power of two
+    // split-K partial tiles of the weight gradients: four ranges of the three-output dWq, dWk, dWv product
+    L.slab_bytes = 4 * 3 * (size_t)H * d * c.W * 4;
+    L.slab = take(L.slab_bytes);
     L.dO = take(B * S * H * d * 4);
     L.dQp = take(B * S * H * d * 4);
     L.dKp = take(B * S * H * d * 4);
@@ -76,6 +82,7 @@ BwdLayout bwd_layout(const Plan &p) {
     L.dQloc = take(B * H * S * d * 4);
     L.dKloc = take(B * H * S * d * 4);
     L.dVloc = take(B * H * S * d * 4);
+    L.dQpair = take(B * H * S * R * d * 4);  // the remote blocks' dQ parts, one row per (query, slot)
     L.total = o;
     return L;
 }
@@ -223,13 +230,15 @@ __global__ void __launch_bounds__(256) k_bwd_prep(const float *__restrict__ dO, 
     if (lane == 0) dsum[((size_t)b * H + h) * S + t] = part;
 }
 
-// The tensor-core path's last step: dQ and dK (times 1/sqrt(d)) and dV from their head-major fp32 sums to the
-// operands of the projection gradients (store_grad16: rotated back, token-major).  One thread per 16 dimensions
-// of a (b, h, t) row.
+// The tensor-core path's last step: dQ (the local part plus the remote blocks' parts of the query's valid
+// slots, in slot order) and dK (times 1/sqrt(d)) and dV from their head-major fp32 sums to the operands of the
+// projection gradients (store_grad16: rotated back, token-major).  One thread per 16 dimensions of a (b, h, t)
+// row.
 template <int DD>
 __global__ void __launch_bounds__(256) k_bwd_finish(const float *__restrict__ dq, const float *__restrict__ dk,
-                                                    const float *__restrict__ dv, const GradOut go, int B, int H,
-                                                    int S, float scale) {
+                                                    const float *__restrict__ dv, const float *__restrict__ dq_pair,
+                                                    const int32_t *__restrict__ sel, const GradOut go, int B, int H,
+                                                    int S, int Bs, int L, int R, float scale) {
     constexpr int TPR = DD / 16;
     const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     if (gid >= (long long)B * H * S * TPR) return;
@@ -242,6 +251,14 @@ __global__ void __launch_bounds__(256) k_bwd_finish(const float *__restrict__ dq
     load16<float>(dq + w * DD + e0, q);
     load16<float>(dk + w * DD + e0, k);
     load16<float>(dv + w * DD + e0, v);
+    // the remote blocks' parts in slot order
+    for (int r = 0; r < R; ++r) {
+        if (!bwd_sel_valid(sel[w * R + r], t, Bs, L)) continue;
+        float pq[16];
+        load16<float>(dq_pair + (w * R + r) * DD + e0, pq);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) q[e] += pq[e];
+    }
 #pragma unroll
     for (int e = 0; e < 16; ++e) {
         q[e] *= scale;
@@ -473,7 +490,42 @@ __global__ void __launch_bounds__(256) k_bwd_fill(const int32_t *__restrict__ se
     const int j = sel[i];
     if (!bwd_sel_valid(j, t, Bs, L)) return;
     const int pos = atomicAdd(&cursor[bh * nb + j], 1);
-    list[bh * S * R + pos] = t;
+    list[bh * S * R + pos] = (int)(i - bh * S * R);  // the pair t * R + r; k_bwd_sort orders each block's list
+}
+
+// Each block's list of pairs (from k_bwd_fill, in atomic order) sorted ascending, so that every sum over a
+// block's queries runs in one order on every call.  One CTA per (b, h, block): a bitonic network over the
+// list padded with INT_MAX to a power of two P, in shared memory when P <= 8192, else in sortbuf (the
+// segment's own 2 n ints at twice its list offset).  grid B*H*nb, 256 threads.
+__global__ void __launch_bounds__(256) k_bwd_sort(int32_t *__restrict__ list, int32_t *__restrict__ sortbuf,
+                                                  const int32_t *__restrict__ cnt, const int32_t *__restrict__ start,
+                                                  int S, int R, int nb) {
+    __shared__ int32_t sh[8192];
+    const int seg = blockIdx.x, tid = threadIdx.x;
+    const int n = cnt[seg];
+    if (n <= 1) return;
+    const size_t base = (size_t)(seg / nb) * S * R;
+    int32_t *a = list + base + start[seg];
+    int P = 1;
+    while (P < n) P <<= 1;
+    int32_t *w = P <= 8192 ? sh : sortbuf + 2 * base + 2 * (size_t)start[seg];
+    for (int i = tid; i < P; i += blockDim.x) w[i] = i < n ? a[i] : 0x7fffffff;
+    __syncthreads();
+    for (int k = 2; k <= P; k <<= 1)
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            for (int i = tid; i < P; i += blockDim.x) {
+                const int l = i ^ j;
+                if (l > i) {
+                    const int x = w[i], y = w[l];
+                    if ((x > y) == ((i & k) == 0)) {
+                        w[i] = y;
+                        w[l] = x;
+                    }
+                }
+            }
+            __syncthreads();
+        }
+    for (int i = tid; i < n; i += blockDim.x) a[i] = w[i];
 }
 
 // ---------------------------------------------------------------------------
@@ -538,7 +590,7 @@ __global__ void __launch_bounds__(kBwdKT * DD / 16, DD == 64 ? 2 : 1) k_bwd_dkdv
         for (int k = 0; k < PER; ++k) {
             const int n = g0 + fq0 + k * (NT / DD);
             const bool in = n < nq;
-            const int t = !in ? 0 : n < nloc ? t_loc0 + n : list[bh * S * R + rem0 + (n - nloc)];
+            const int t = !in ? 0 : n < nloc ? t_loc0 + n : list[bh * S * R + rem0 + (n - nloc)] / R;
             rt[k] = t;
             rq[k] = in ? to_f(Q[(bh * S + t) * DD + fe]) : 0.f;
             rg[k] = in ? dO[(((size_t)b * S + t) * H + h) * DD + fe] : 0.f;
@@ -627,7 +679,9 @@ __global__ void __launch_bounds__(kBwdKT * DD / 16, DD == 64 ? 2 : 1) k_bwd_dkdv
 template <typename TA, typename TB>
 __global__ void __launch_bounds__(256) k_gemm_any(int M, int N, int Kd, const TA *__restrict__ A, long long am,
                                                   long long ak, const TB *__restrict__ Bm, long long bk, long long bn,
-                                                  float *__restrict__ C, long long ldc, int kchunk, bool atomic) {
+                                                  float *__restrict__ C, long long ldc, int kchunk, bool atomic,
+                                                  long long zstride) {
+    C += blockIdx.z * zstride;  // split k ranges into their own slabs
     __shared__ __align__(16) float sA[8][128 + 4];
     __shared__ __align__(16) float sB[8][128 + 4];
     const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
@@ -677,23 +731,48 @@ __global__ void __launch_bounds__(256) k_gemm_any(int M, int N, int Kd, const TA
 }
 
 // beta 0: C = A B; beta 1: C += A B.  Output tiles fewer than twice the SMs split K.
+// C (+)= sum of the split slabs in ascending order (n4 float4s each)
+__global__ void __launch_bounds__(256) k_slab_sum(const float4 *__restrict__ slab, float4 *__restrict__ C, long long n4,
+                                                  int split, bool accumulate) {
+    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (long long)gridDim.x * blockDim.x) {
+        float4 a = __ldg(slab + i);
+        for (int p = 1; p < split; ++p) {
+            const float4 b = __ldg(slab + (size_t)p * n4 + i);
+            a = make_float4(__fadd_rn(a.x, b.x), __fadd_rn(a.y, b.y), __fadd_rn(a.z, b.z), __fadd_rn(a.w, b.w));
+        }
+        if (accumulate) {
+            const float4 o = C[i];
+            a = make_float4(__fadd_rn(o.x, a.x), __fadd_rn(o.y, a.y), __fadd_rn(o.z, a.z), __fadd_rn(o.w, a.w));
+        }
+        C[i] = a;
+    }
+}
+
 template <typename TA, typename TB>
 cudaError_t gemm_any(int M, int N, int Kd, const TA *A, long long am, long long ak, const TB *Bm, long long bk,
-                     long long bn, float *C, long long ldc, float beta, cudaStream_t s) {
+                     long long bn, float *C, long long ldc, float beta, float *slab, size_t slab_bytes,
+                     cudaStream_t s) {
     if (M == 0 || N == 0) return cudaSuccess;
     const int tiles = ((N + 127) / 128) * ((M + 127) / 128);
     int split = 1;
     while (split < 32 && tiles * split < 2 * 148 && Kd / (split * 2) >= 256) split *= 2;
+    // the k ranges' partial products go to slabs summed in range order (the same bits on every run)
+    const size_t out_bytes = (size_t)M * N * sizeof(float);
+    while (split > 1 && (!slab || ldc != N || split * out_bytes > slab_bytes)) split /= 2;
     const int kchunk = ((Kd + split - 1) / split + 7) / 8 * 8;
-    const bool atomic = split > 1 || beta != 0.f;
-    cudaError_t e;
-    if (atomic && beta == 0.f) {
-        if (ldc != N) return cudaErrorInvalidValue;  // callers pass dense C
-        if ((e = cudaMemsetAsync(C, 0, (size_t)M * N * sizeof(float), s)) != cudaSuccess) return e;
-    }
     dim3 g((N + 127) / 128, (M + 127) / 128, split);
-    k_gemm_any<TA, TB><<<g, 256, 0, s>>>(M, N, Kd, A, am, ak, Bm, bk, bn, C, ldc, kchunk, atomic);
-    count_launches(1);
+    if (split == 1) {
+        // one CTA per output element: C = product, or C += product with beta = 1
+        k_gemm_any<TA, TB><<<g, 256, 0, s>>>(M, N, Kd, A, am, ak, Bm, bk, bn, C, ldc, kchunk, beta != 0.f, 0ll);
+        count_launches(1);
+        return cudaGetLastError();
+    }
+    k_gemm_any<TA, TB><<<g, 256, 0, s>>>(M, N, Kd, A, am, ak, Bm, bk, bn, slab, N, kchunk, false,
+                                         (long long)M * N);
+    const long long n4 = (long long)M * N / 4;
+    k_slab_sum<<<(unsigned)std::min<long long>((n4 + 255) / 256, 8 * 148), 256, 0, s>>>(
+        (const float4 *)slab, (float4 *)C, n4, split, beta != 0.f);
+    count_launches(2);
     return cudaGetLastError();
 }
 
@@ -720,7 +799,9 @@ cudaError_t attend_backward(const Plan &p, const T *Q, const T *K, const T *V, c
         k_bwd_count<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(sel, cnt, n, c.S, c.R, p.nb, c.Bs, c.L);
         k_bwd_scan<<<c.B * c.H, 1024, 0, s>>>(cnt, start, cursor, p.nb);
         k_bwd_fill<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(sel, cursor, list, n, c.S, c.R, p.nb, c.Bs, c.L);
-        count_launches(3);
+        k_bwd_sort<<<(unsigned)(c.B * c.H * p.nb), 256, 0, s>>>(list, (int32_t *)(bws + L.sortbuf), cnt, start, c.S,
+                                                               c.R, p.nb);
+        count_launches(4);
         return cudaSuccess;
     };
     // With the forward's statistics and a shape the kernels take, every attention gradient on the tensor cores:
@@ -742,14 +823,17 @@ cudaError_t attend_backward(const Plan &p, const T *Q, const T *K, const T *V, c
                 cudaSuccess)
                 return e;
             if ((e = build_lists()) != cudaSuccess) return e;
-            if (c.R > 0 && (e = launch_bwd_remote_tc(p, Q, K, V, dohi, dolo, lse, dsum, cnt, start, list, dq_loc,
+            float *dq_pair = (float *)(bws + L.dQpair);
+            if (c.R > 0 && (e = launch_bwd_remote_tc(p, Q, K, V, dohi, dolo, lse, dsum, cnt, start, list, dq_pair,
                                                      dk_loc, dv_loc, counters, s)) != cudaSuccess)
                 return e;
             const unsigned gf = (unsigned)((nq * (c.d / 16) + 255) / 256);
             if (c.d == 64)
-                k_bwd_finish<64><<<gf, 256, 0, s>>>(dq_loc, dk_loc, dv_loc, go, c.B, c.H, c.S, scale);
+                k_bwd_finish<64><<<gf, 256, 0, s>>>(dq_loc, dk_loc, dv_loc, dq_pair, sel, go, c.B, c.H, c.S, c.Bs,
+                                                    c.L, c.R, scale);
             else
-                k_bwd_finish<128><<<gf, 256, 0, s>>>(dq_loc, dk_loc, dv_loc, go, c.B, c.H, c.S, scale);
+                k_bwd_finish<128><<<gf, 256, 0, s>>>(dq_loc, dk_loc, dv_loc, dq_pair, sel, go, c.B, c.H, c.S, c.Bs,
+                                                     c.L, c.R, scale);
             count_launches(1);
             return cudaGetLastError();
         }
@@ -796,6 +880,7 @@ cudaError_t backward_t(const Plan &p, const T *x, const T *Wq, const T *Wk, cons
     const BwdLayout L = bwd_layout(p);
     unsigned long long *counters = (unsigned long long *)ws_ptr(p, ws, kRegCounters);
     float *dO = (float *)(bws + L.dO);
+    float *slab = (float *)(bws + L.slab);
     const int BS = c.B * c.S, Hd = c.H * c.d, W = c.W;
     const bool tc = grads_tc_supported(c);
     // dQp, dKp, dVp: the attention gradients before RoPE, token-major, written by the attention kernels
@@ -811,8 +896,12 @@ cudaError_t backward_t(const Plan &p, const T *x, const T *Wq, const T *Wk, cons
         // delta = O Wo^T:  dO = ddelta Wo (Wo MN-major),  dWo = ddelta^T O (both MN-major)
         const void *a0[1] = {ddelta}, *b0[1] = {Wo}, *b1[1] = {O};
         float *c0[1] = {dO}, *c1[1] = {dWo};
-        if ((e = gemm_grad_tc(BS, Hd, W, 1, 1, a0, false, b0, true, c0, false, counters, s)) != cudaSuccess) return e;
-        if ((e = gemm_grad_tc(W, Hd, BS, 1, 1, a0, true, b1, true, c1, false, counters, s)) != cudaSuccess) return e;
+        if ((e = gemm_grad_tc(BS, Hd, W, 1, 1, a0, false, b0, true, c0, false, slab, L.slab_bytes, counters, s)) !=
+            cudaSuccess)
+            return e;
+        if ((e = gemm_grad_tc(W, Hd, BS, 1, 1, a0, true, b1, true, c1, false, slab, L.slab_bytes, counters, s)) !=
+            cudaSuccess)
+            return e;
         if ((e = attend_backward<T>(p, Q, K, V, sel, dO, go, bws, s, o32, counters)) != cudaSuccess) return e;
         // q = x Wq^T (per head, then RoPE):  dWq = dQp^T x (both MN-major),  dx = dQp Wq + dKp Wk + dVp Wv,
         // each dZp as hi + lo
@@ -822,21 +911,37 @@ cudaError_t backward_t(const Plan &p, const T *x, const T *Wq, const T *Wk, cons
         const void *ah[6] = {hq, hq + n, hk, hk + n, hv, hv + n};
         const void *xs[6] = {x, x, x, x, x, x}, *wz[6] = {Wq, Wq, Wk, Wk, Wv, Wv};
         float *cw[3] = {dWq, dWk, dWv}, *cx[1] = {dx};
-        if ((e = gemm_grad_tc(Hd, W, BS, 2, 3, ah, true, xs, true, cw, false, counters, s)) != cudaSuccess) return e;
-        return gemm_grad_tc(BS, W, Hd, 6, 1, ah, false, wz, true, cx, false, counters, s);
+        if ((e = gemm_grad_tc(Hd, W, BS, 2, 3, ah, true, xs, true, cw, false, slab, L.slab_bytes, counters, s)) !=
+            cudaSuccess)
+            return e;
+        return gemm_grad_tc(BS, W, Hd, 6, 1, ah, false, wz, true, cx, false, slab, L.slab_bytes, counters, s);
     }
     const float *dQp = (const float *)go.q, *dKp = (const float *)go.k, *dVp = (const float *)go.v;
     // delta = O Wo^T:  dO = ddelta Wo,  dWo = ddelta^T O
-    if ((e = gemm_any<T, T>(BS, Hd, W, ddelta, W, 1, Wo, Hd, 1, dO, Hd, 0.f, s)) != cudaSuccess) return e;
-    if ((e = gemm_any<T, T>(W, Hd, BS, ddelta, 1, W, O, Hd, 1, dWo, Hd, 0.f, s)) != cudaSuccess) return e;
+    if ((e = gemm_any<T, T>(BS, Hd, W, ddelta, W, 1, Wo, Hd, 1, dO, Hd, 0.f, slab, L.slab_bytes, s)) !=
+        cudaSuccess)
+        return e;
+    if ((e = gemm_any<T, T>(W, Hd, BS, ddelta, 1, W, O, Hd, 1, dWo, Hd, 0.f, slab, L.slab_bytes, s)) !=
+        cudaSuccess)
+        return e;
     if ((e = attend_backward<T>(p, Q, K, V, sel, dO, go, bws, s)) != cudaSuccess) return e;
     // q = x Wq^T (per head, then RoPE):  dWq = dQp^T x,  dx = dQp Wq + dKp Wk + dVp Wv
-    if ((e = gemm_any<float, T>(Hd, W, BS, dQp, 1, Hd, x, W, 1, dWq, W, 0.f, s)) != cudaSuccess) return e;
-    if ((e = gemm_any<float, T>(Hd, W, BS, dKp, 1, Hd, x, W, 1, dWk, W, 0.f, s)) != cudaSuccess) return e;
-    if ((e = gemm_any<float, T>(Hd, W, BS, dVp, 1, Hd, x, W, 1, dWv, W, 0.f, s)) != cudaSuccess) return e;
-    if ((e = gemm_any<float, T>(BS, W, Hd, dQp, Hd, 1, Wq, W, 1, dx, W, 0.f, s)) != cudaSuccess) return e;
-    if ((e = gemm_any<float, T>(BS, W, Hd, dKp, Hd, 1, Wk, W, 1, dx, W, 1.f, s)) != cudaSuccess) return e;
-    return gemm_any<float, T>(BS, W, Hd, dVp, Hd, 1, Wv, W, 1, dx, W, 1.f, s);
+    if ((e = gemm_any<float, T>(Hd, W, BS, dQp, 1, Hd, x, W, 1, dWq, W, 0.f, slab, L.slab_bytes, s)) !=
+        cudaSuccess)
+        return e;
+    if ((e = gemm_any<float, T>(Hd, W, BS, dKp, 1, Hd, x, W, 1, dWk, W, 0.f, slab, L.slab_bytes, s)) !=
+        cudaSuccess)
+        return e;
+    if ((e = gemm_any<float, T>(Hd, W, BS, dVp, 1, Hd, x, W, 1, dWv, W, 0.f, slab, L.slab_bytes, s)) !=
+        cudaSuccess)
+        return e;
+    if ((e = gemm_any<float, T>(BS, W, Hd, dQp, Hd, 1, Wq, W, 1, dx, W, 0.f, slab, L.slab_bytes, s)) !=
+        cudaSuccess)
+        return e;
+    if ((e = gemm_any<float, T>(BS, W, Hd, dKp, Hd, 1, Wk, W, 1, dx, W, 1.f, slab, L.slab_bytes, s)) !=
+        cudaSuccess)
+        return e;
+    return gemm_any<float, T>(BS, W, Hd, dVp, Hd, 1, Wv, W, 1, dx, W, 1.f, slab, L.slab_bytes, s);
 }
 
 int bwd_check(std::initializer_list<const void *> ptrs) {

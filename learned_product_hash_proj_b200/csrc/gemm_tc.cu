@@ -453,7 +453,9 @@ cudaError_t launch_out_project_tc(const Plan &p, const void *O, const void *Wo, 
 // row contiguous in m or n).  ngroups independent outputs (dWq, dWk, dWv),
 // each the sum of nsrc products over the same K (dx = dQp Wq + dKp Wk + dVp Wv;
 // an fp32 operand given as the two bf16 terms of its hi + lo split); the k
-// slices are split over blockIdx.z, partial sums added with fp32 atomics.  Same roles as k_gemm_tc; an MN-major tile is two 64-wide column
+// slices are split over blockIdx.z, each range's partial tile stored in its
+// own slab and the slabs summed in range order by k_split_sum (the same bits
+// on every run).  Same roles as k_gemm_tc; an MN-major tile is two 64-wide column
 // blocks of 64 K-rows each (128-byte swizzle), 8 KB apart.
 // ---------------------------------------------------------------------------
 namespace {
@@ -473,6 +475,7 @@ struct GradArgs {
     int split;       // k-slice ranges per output tile (blockIdx.z % split)
     int a_mn, b_mn;  // operand major-ness
     int atomic;      // add into C instead of storing
+    float *slab;     // split > 1: range part of output g goes to slab + (g * split + part) * M * N
     unsigned long long *counters;
 };
 
@@ -560,7 +563,7 @@ __global__ void __launch_bounds__(192, 2) k_gemm_grad_tc(const __grid_constant__
         const bool ok = nk > 0 && tc::mbar_wait(&accf, 0, 1u << 20);
         tc::fence_after_sync();
         const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16);
-        float *out = g.out[grp];
+        float *out = g.slab ? g.slab + ((size_t)grp * g.split + part) * g.M * g.N : g.out[grp];
         for (int c0 = 0; c0 < BN; c0 += 32) {
             float v[32];
             tc::tmem_ld32(trow + c0, v);
@@ -591,6 +594,33 @@ __global__ void __launch_bounds__(192, 2) k_gemm_grad_tc(const __grid_constant__
     if (warp == 1) tc::tmem_dealloc(tmem, BN);
 }
 
+// C_g (+)= sum over parts of slab[g][part] in ascending part order; n4 float4s per output
+__global__ void __launch_bounds__(256) k_split_sum(const float4 *__restrict__ slab, float4 *__restrict__ c0,
+                                                   float4 *__restrict__ c1, float4 *__restrict__ c2, long long n4,
+                                                   int split, int ngroups, int accumulate) {
+    const long long total = n4 * ngroups;
+    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+         i += (long long)gridDim.x * blockDim.x) {
+        const int g = (int)(i / n4);
+        const long long e = i % n4;
+        const float4 *src = slab + (size_t)g * split * n4 + e;
+        float4 a = __ldg(src);
+        for (int p = 1; p < split; ++p) {
+            const float4 b = __ldg(src + (size_t)p * n4);
+            a.x = __fadd_rn(a.x, b.x);
+            a.y = __fadd_rn(a.y, b.y);
+            a.z = __fadd_rn(a.z, b.z);
+            a.w = __fadd_rn(a.w, b.w);
+        }
+        float4 *dst = (g == 0 ? c0 : g == 1 ? c1 : c2) + e;
+        if (accumulate) {
+            const float4 o = *dst;
+            a = make_float4(__fadd_rn(o.x, a.x), __fadd_rn(o.y, a.y), __fadd_rn(o.z, a.z), __fadd_rn(o.w, a.w));
+        }
+        *dst = a;
+    }
+}
+
 }  // namespace
 
 bool gemm_grad_tc_supported(int M, int N, int K, bool a_mn, bool b_mn) {
@@ -600,8 +630,8 @@ bool gemm_grad_tc_supported(int M, int N, int K, bool a_mn, bool b_mn) {
 }
 
 cudaError_t gemm_grad_tc(int M, int N, int K, int nsrc, int ngroups, const void *const *A, bool a_mn,
-                         const void *const *B, bool b_mn, float *const *C, bool accumulate,
-                         unsigned long long *counters, cudaStream_t s) {
+                         const void *const *B, bool b_mn, float *const *C, bool accumulate, float *slab,
+                         size_t slab_bytes, unsigned long long *counters, cudaStream_t s) {
     if (M == 0 || N == 0) return cudaSuccess;
     if (nsrc < 1 || ngroups < 1 || ngroups > 3 || nsrc * ngroups > kGradMaxOps) return cudaErrorInvalidValue;
     if (!gemm_grad_tc_supported(M, N, K, a_mn, b_mn) || !get_encode()) return cudaErrorNotSupported;
@@ -632,23 +662,30 @@ cudaError_t gemm_grad_tc(int M, int N, int K, int nsrc, int ngroups, const void 
             }
         }
     }
+    // as many slabs as the scratch holds
+    const size_t out_bytes = (size_t)M * N * sizeof(float);
+    while (split > 1 && (!slab || (size_t)ngroups * split * out_bytes > slab_bytes)) --split;
     const int per = (total + split - 1) / split;
     split = (total + per - 1) / per;  // every k range non-empty
     GradArgs g{};
     for (int i = 0; i < 3; ++i) g.out[i] = C[i < ngroups ? i : 0];
     g.M = M; g.N = N; g.K = K; g.nsrc = nsrc; g.ngroups = ngroups; g.split = split;
     g.a_mn = a_mn; g.b_mn = b_mn;
-    g.atomic = split > 1 || accumulate;
+    g.atomic = split == 1 && accumulate;  // one CTA per output element: a deterministic add
+    g.slab = split > 1 ? slab : nullptr;
     g.counters = counters;
     cudaError_t e;
-    if (split > 1 && !accumulate)
-        for (int i = 0; i < ngroups; ++i)
-            if ((e = cudaMemsetAsync(C[i], 0, (size_t)M * N * sizeof(float), s)) != cudaSuccess) return e;
     if ((e = cudaFuncSetAttribute(k_gemm_grad_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES)) !=
         cudaSuccess)
         return e;
     dim3 grid((N + BN - 1) / BN, (M + BM - 1) / BM, ngroups * split);
     k_gemm_grad_tc<<<grid, 192, SMEM_BYTES, s>>>(maps, g);
+    count_launches(1);
+    if ((e = cudaGetLastError()) != cudaSuccess || split == 1) return e;
+    const long long n4 = (long long)M * N / 4;
+    const int grid2 = (int)std::min<long long>((n4 * ngroups + 255) / 256, 8ll * sms);
+    k_split_sum<<<grid2, 256, 0, s>>>((const float4 *)slab, (float4 *)C[0], (float4 *)C[ngroups > 1 ? 1 : 0],
+                                      (float4 *)C[ngroups > 2 ? 2 : 0], n4, split, ngroups, accumulate ? 1 : 0);
     count_launches(1);
     return cudaGetLastError();
 }

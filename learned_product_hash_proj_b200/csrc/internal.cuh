@@ -129,10 +129,12 @@ cudaError_t launch_stage_reduce(const Plan &p, const float *stage, int nranks, v
 // C_g[M,N] (fp32) (+)= sum_{src < nsrc} A_{g,src}(m,k) B_{g,src}(n,k) for g < ngroups (<= 3, nsrc * ngroups
 // <= 6; A and B hold the operands group-major), bf16 operands on the tensor cores; an operand is K-major
 // ([M|N rows][K]) or MN-major ([K rows][M|N]).  Pointers 16-byte aligned; row lengths multiples of 8 (supported() checks).
+// K is split over several CTAs where the output tiles alone leave the SMs idle and slab (slab_bytes of fp32
+// scratch) holds the partial tiles; they are summed in a fixed order, so the result is the same on every run.
 bool gemm_grad_tc_supported(int M, int N, int K, bool a_mn, bool b_mn);
 cudaError_t gemm_grad_tc(int M, int N, int K, int nsrc, int ngroups, const void *const *A, bool a_mn,
-                         const void *const *B, bool b_mn, float *const *C, bool accumulate,
-                         unsigned long long *counters, cudaStream_t s);
+                         const void *const *B, bool b_mn, float *const *C, bool accumulate, float *slab,
+                         size_t slab_bytes, unsigned long long *counters, cudaStream_t s);
 // The routing regions that mono_route_static uses for plan `p` (offsets in
 // rp->off relative to *base, the device address of its fixed array on the
 // current device); MONO_ERR_SCRATCH if they do not fit.
@@ -154,11 +156,12 @@ cudaError_t launch_bwd_local_dq_tc(const Plan &p, const void *Q, const void *K, 
 cudaError_t launch_bwd_local_dkdv_tc(const Plan &p, const void *Q, const void *K, const void *V, const void *dohi,
                                      const void *dolo, const float *lse, const float *dsum, float *dk_loc,
                                      float *dv_loc, unsigned long long *counters, cudaStream_t s);
-// the remote blocks' part on the tensor cores, from the per-block lists of selecting queries (cnt, start, list as
-// [B*H, nb] and [B*H, S*R]): dq_loc += (fp32 atomics), dk_loc and dv_loc rows of each block += (one CTA per block)
+// the remote blocks' part on the tensor cores, from the per-block lists of selecting pairs t * R + r (cnt,
+// start, list as [B*H, nb] and [B*H, S*R], each list ascending): dq_pair [B*H, S*R, d] = each pair's dQ part,
+// dk_loc and dv_loc rows of each block += (one CTA per block)
 cudaError_t launch_bwd_remote_tc(const Plan &p, const void *Q, const void *K, const void *V, const void *dohi,
                                  const void *dolo, const float *lse, const float *dsum, const int32_t *cnt,
-                                 const int32_t *start, const int32_t *list, float *dq_loc, float *dk_loc,
+                                 const int32_t *start, const int32_t *list, float *dq_pair, float *dk_loc,
                                  float *dv_loc, unsigned long long *counters, cudaStream_t s);
 cudaError_t launch_attend_tc(const Plan &p, const void *Q, const void *K, const void *V, const int32_t *sel, void *O,
                              void *ws, cudaStream_t s, int parts = kAttendAll, float *o32 = nullptr,

@@ -109,3 +109,32 @@ def test_backward_matches_oracle(name):
     rel = 1e-4 if dtype == "f32" else 2e-2
     for nm, got in (("x", dx), ("Wq", dWq), ("Wk", dWk), ("Wv", dWv), ("Wo", dWo)):
         close(to_np(got), ref[nm], rel, f"d{nm}")
+
+
+@pytest.mark.parametrize("name", ["f32", "bf16_S4096"])
+def test_backward_is_bit_reproducible(name):
+    # Every sum of the backward runs in a fixed order (block lists sorted, the remote blocks' dQ parts summed in
+    # slot order, split-K partial tiles summed in range order): two calls give the same bits.  bf16_S4096 takes
+    # the tensor-core attention gradients, f32 the SIMT ones; both split K in the weight gradients.
+    cfg = small(**FULL_CASES[name])
+    run = Run(cfg, seed=8).run_stages()
+    plan, d = run.plan, run.dev
+    rng = np.random.default_rng(9)
+    dd = rng.standard_normal((cfg.B, cfg.S, cfg.W)).astype(np.float32)
+    if cfg.dtype == "bf16":
+        dd = synth.round_bf16(dd)
+    ddelta = torch.from_numpy(np.asarray(dd, np.float32)).to(plan.dtype).cuda().contiguous()
+    hd = cfg.H * cfg.d
+    f32 = dict(dtype=torch.float32, device="cuda")
+    outs = []
+    for _ in range(2):
+        dx = torch.empty((cfg.B, cfg.S, cfg.W), **f32)
+        dWq, dWk, dWv = (torch.empty((hd, cfg.W), **f32) for _ in range(3))
+        dWo = torch.empty((cfg.W, hd), **f32)
+        ws, bws = plan.workspace(), mono.backward_workspace(plan)
+        mono.backward(plan, d["x"], d["Wq"], d["Wk"], d["Wv"], d["Wo"], run.sel, ddelta, dx, dWq, dWk, dWv, dWo, ws,
+                      bws)
+        torch.cuda.synchronize()
+        outs.append((dx, dWq, dWk, dWv, dWo))
+    for a, b in zip(*outs):
+        assert torch.equal(a, b)
