@@ -27,6 +27,7 @@ from __future__ import annotations
 import argparse
 import json
 import os
+import math
 import statistics
 import sys
 import threading
@@ -265,6 +266,9 @@ def run_ours(args):
             stage_ms[n].append(ev[i].elapsed_time(ev[i + 1]))
     mean = lambda v: sum(v) / len(v)
     # max over ranks of the per-rank means
+    srt = sorted(ra_ms)
+    pct = lambda q: srt[min(len(srt) - 1, int(math.ceil(q * len(srt))) - 1)]  # nearest-rank percentile
+    lat = dist.reduce_max([statistics.median(ra_ms), pct(0.99), srt[-1]], device=dev)
     agg = dist.reduce_max([mean(ra_ms), mean(fwd_ms), t_wall] + [mean(stage_ms[n]) for n in names], device=dev)
     ra, fwd, wall = agg[0], agg[1], agg[2]
     stage = dict(zip(names, agg[3:]))
@@ -363,6 +367,9 @@ def run_ours(args):
                        "l2": "flushed before every step (256 MiB write, outside the stage events)",
                        "replicas": "one independent replica per GPU (no data-path collective)"},
             "route_attend_ms": ra, "forward_tokens_per_s": tokens / (fwd / 1e3),
+            "route_attend_latency": {"median_ms": lat[0], "p99_ms": lat[1], "max_ms": lat[2], "steps": args.steps,
+                                     "note": "per timed step; p99 is the nearest-rank percentile (with few steps, the "
+                                             "largest); max over ranks"},
             "stage_ms": stage,
             "stage_note": "stage_ms from separately timed steps, each stage through its own entry point; "
                           f"their window sum ({stage_sum:.4f} ms) exceeds route_attend_ms where mono_route "

@@ -139,12 +139,19 @@ __global__ void __launch_bounds__(256) k_dec_project(const T *__restrict__ x, co
     const int n0 = h * d + 2 * i;
     const T *Wm = which == 0 ? Wq : (which == 1 ? Wk : Wv);
     const T *w0 = Wm + (size_t)n0 * W, *w1 = w0 + W;
+    // before the previous kernel of the stream completes: the weight rows into L2 and the rotation angle
+    for (int o = lane * 64; o < W * (int)sizeof(T); o += 32 * 64) {
+        tc::prefetch_l2((const char *)w0 + o);
+        tc::prefetch_l2((const char *)w1 + o);
+    }
     double c = 1.0, s = 0.0;
     if (which < 2) {
         const double ang = (double)t * pow(theta, -2.0 * (double)i / (double)d);
         c = cos(ang);
         s = sin(ang);
     }
+    tc::grid_dep_wait();  // x may come from it, and the previous step's kernels read q and the caches
+    tc::grid_dep_launch();
     for (int b = 0; b < B; ++b) {
         const T *xb = x + (size_t)b * W;
         const float p0 = row_dot_part(xb, w0, W, lane), p1 = row_dot_part(xb, w1, W, lane);
@@ -236,6 +243,8 @@ __global__ void __launch_bounds__(32) k_dec_block(const T *__restrict__ Kc, cons
     const int h = blockIdx.x, b = blockIdx.y;
     const size_t bh = (size_t)b * H + h;
     const int j = t / Bs;
+    tc::grid_dep_wait();  // the block's last key (projection)
+    tc::grid_dep_launch();
     const int a = dec_summary<T>(Kc, cb, P.kbar, P.addr, bh, h, j, S, Bs, d, M, C, nb, s_kb, s_sc);
     if (threadIdx.x == 0) dec_append(P.count, P.head, P.tail, P.next, P.overflow, bh, A, nb, a, j, cap);
 }
@@ -306,6 +315,8 @@ __global__ void __launch_bounds__(32) k_dec_route(const T *__restrict__ q, const
                          "l"(src + i)
                          : "memory");
     }
+    tc::grid_dep_wait();  // q (projection) and the lists (block update) are complete
+    tc::grid_dep_launch();
     for (int i = lane; i < d; i += 32) s_q[i] = to_f(q[bh * d + i]);
     tc::cp_async_wait_all();
     __syncwarp();
@@ -472,6 +483,8 @@ __global__ void __launch_bounds__(256) k_dec_attend(const T *__restrict__ q, con
     T *bufK[2] = {(T *)dsm, (T *)(dsm + 2 * CH * rowb)};
     T *bufV[2] = {(T *)(dsm + CH * rowb), (T *)(dsm + 3 * CH * rowb)};
     const int bq = t / Bs, lim = bq - L;
+    tc::grid_dep_wait();  // sel (route), q and the newest key and value (projection)
+    tc::grid_dep_launch();
     if (threadIdx.x == 0) {  // the selected remote blocks; ids outside [0, t/Bs - L] are skipped
         int nr = 0;
         for (int r = 0; r < R; ++r) {
@@ -576,6 +589,8 @@ __global__ void __launch_bounds__(256) k_dec_attend_cl(const T *__restrict__ q, 
     T *bufK[2] = {(T *)dsm, (T *)(dsm + 2 * CH * rowb)};
     T *bufV[2] = {(T *)(dsm + CH * rowb), (T *)(dsm + 3 * CH * rowb)};
     const int bq = t / Bs, lim = bq - L;
+    tc::grid_dep_wait();  // sel (route), q and the newest key and value (projection)
+    tc::grid_dep_launch();
     if (threadIdx.x == 0) {
         int nr = 0;
         for (int r = 0; r < R; ++r) {
@@ -678,11 +693,42 @@ __global__ void __launch_bounds__(256) k_dec_out(const T *__restrict__ o, const 
     const int w = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     if (w >= W) return;
     const T *wr = Wo + (size_t)w * N;
+    for (int off = lane * 64; off < N * (int)sizeof(T); off += 32 * 64) tc::prefetch_l2((const char *)wr + off);
+    tc::grid_dep_wait();  // o (attention)
+    tc::grid_dep_launch();
     for (int b = 0; b < B; ++b) {
         const T *ob = o + (size_t)b * N;
         const float a = warp_sum(row_dot_part(ob, wr, N, lane));
         if (lane == 0) delta[(size_t)b * W + w] = from_f<T>(a);
     }
+}
+
+// The kernels of a decode step are launched with programmatic dependent launch: each one's blocks may start while
+// the kernel before it in the stream runs, and wait (grid_dep_wait) before they touch anything that kernel writes
+// or reads; the launch gaps between the step's small kernels overlap.  cluster > 1 adds a cluster dimension.
+template <typename... KArgs, typename... Args>
+cudaError_t dec_launch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, int cluster,
+                       Args... args) {
+    cudaLaunchConfig_t lc = {};
+    lc.gridDim = grid;
+    lc.blockDim = block;
+    lc.dynamicSmemBytes = smem;
+    lc.stream = s;
+    cudaLaunchAttribute at[2];
+    int na = 0;
+    at[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+    if (cluster > 1) {
+        at[na].id = cudaLaunchAttributeClusterDimension;
+        at[na].val.clusterDim.x = cluster;
+        at[na].val.clusterDim.y = 1;
+        at[na].val.clusterDim.z = 1;
+        ++na;
+    }
+    lc.attrs = at;
+    lc.numAttrs = na;
+    return cudaLaunchKernelEx(&lc, kern, (KArgs)args...);
 }
 
 int dec_check(const mono_plan_t *plan, const void *cache) {
@@ -771,17 +817,18 @@ int mono_decode_project(const mono_plan_t *plan, int t, const void *x_t, const v
     const int warps = 3 * c.H * c.d / 2;
     const int grid = (warps + 7) / 8;
     cudaStream_t s = (cudaStream_t)stream;
+    cudaError_t e;
     if (c.dtype == MONO_BF16)
-        k_dec_project<__nv_bfloat16><<<grid, 256, 0, s>>>(
-            (const __nv_bfloat16 *)x_t, (const __nv_bfloat16 *)Wq, (const __nv_bfloat16 *)Wk,
-            (const __nv_bfloat16 *)Wv, (__nv_bfloat16 *)P.Q, (__nv_bfloat16 *)P.K, (__nv_bfloat16 *)P.V, t, c.B, c.W,
-            c.H, c.d, c.S, c.rope_theta);
+        e = dec_launch(k_dec_project<__nv_bfloat16>, dim3(grid), dim3(256), 0, s, 1, (const __nv_bfloat16 *)x_t,
+                       (const __nv_bfloat16 *)Wq, (const __nv_bfloat16 *)Wk, (const __nv_bfloat16 *)Wv,
+                       (__nv_bfloat16 *)P.Q, (__nv_bfloat16 *)P.K, (__nv_bfloat16 *)P.V, t, c.B, c.W, c.H, c.d, c.S,
+                       c.rope_theta);
     else
-        k_dec_project<float><<<grid, 256, 0, s>>>((const float *)x_t, (const float *)Wq, (const float *)Wk,
-                                                  (const float *)Wv, (float *)P.Q, (float *)P.K, (float *)P.V, t, c.B,
-                                                  c.W, c.H, c.d, c.S, c.rope_theta);
+        e = dec_launch(k_dec_project<float>, dim3(grid), dim3(256), 0, s, 1, (const float *)x_t, (const float *)Wq,
+                       (const float *)Wk, (const float *)Wv, (float *)P.Q, (float *)P.K, (float *)P.V, t, c.B, c.W,
+                       c.H, c.d, c.S, c.rope_theta);
     count_launches(1);
-    return dec_status(cudaGetLastError());
+    return dec_status(e != cudaSuccess ? e : cudaGetLastError());
 }
 
 int mono_decode_route(const mono_plan_t *plan, int t, const float *codebooks, const int32_t *forced_t, void *cache,
@@ -798,33 +845,34 @@ int mono_decode_route(const mono_plan_t *plan, int t, const float *codebooks, co
     cudaStream_t s = (cudaStream_t)stream;
     const dim3 g(c.H, c.B);
     const bool bf = c.dtype == MONO_BF16;
+    cudaError_t e;
     if (t % c.Bs == c.Bs - 1) {  // position t completes block t / Bs
         if (bf)
-            k_dec_block<__nv_bfloat16><<<g, 32, 0, s>>>((const __nv_bfloat16 *)P.K, codebooks, P, t, c.S, c.Bs, c.d,
-                                                        c.M, c.C, c.H, p.nb, p.A, c.cap);
+            e = dec_launch(k_dec_block<__nv_bfloat16>, g, dim3(32), 0, s, 1, (const __nv_bfloat16 *)P.K, codebooks, P,
+                           t, c.S, c.Bs, c.d, c.M, c.C, c.H, p.nb, p.A, c.cap);
         else
-            k_dec_block<float><<<g, 32, 0, s>>>((const float *)P.K, codebooks, P, t, c.S, c.Bs, c.d, c.M, c.C, c.H,
-                                                p.nb, p.A, c.cap);
+            e = dec_launch(k_dec_block<float>, g, dim3(32), 0, s, 1, (const float *)P.K, codebooks, P, t, c.S, c.Bs,
+                           c.d, c.M, c.C, c.H, p.nb, p.A, c.cap);
         count_launches(1);
+        if (e != cudaSuccess) return dec_status(e);
     }
     if (c.R > 0) {
         const size_t sm = (size_t)c.M * c.C * (c.d / c.M + 1) * 4;
-        cudaError_t e;
         if (bf) {
             if (sm > 48 * 1024 && (e = cudaFuncSetAttribute(k_dec_route<__nv_bfloat16>,
                                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm)))
                 return dec_status(e);
-            k_dec_route<__nv_bfloat16><<<g, 32, sm, s>>>((const __nv_bfloat16 *)P.Q, codebooks, forced_t, P, t,
-                                                         c.Bs, c.L, c.R, c.E, c.M, c.C, c.T, c.cap, c.H, c.d, p.nb,
-                                                         p.A);
+            e = dec_launch(k_dec_route<__nv_bfloat16>, g, dim3(32), sm, s, 1, (const __nv_bfloat16 *)P.Q, codebooks,
+                           forced_t, P, t, c.Bs, c.L, c.R, c.E, c.M, c.C, c.T, c.cap, c.H, c.d, p.nb, p.A);
         } else {
             if (sm > 48 * 1024 &&
                 (e = cudaFuncSetAttribute(k_dec_route<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm)))
                 return dec_status(e);
-            k_dec_route<float><<<g, 32, sm, s>>>((const float *)P.Q, codebooks, forced_t, P, t, c.Bs, c.L, c.R, c.E,
-                                                 c.M, c.C, c.T, c.cap, c.H, c.d, p.nb, p.A);
+            e = dec_launch(k_dec_route<float>, g, dim3(32), sm, s, 1, (const float *)P.Q, codebooks, forced_t, P, t,
+                           c.Bs, c.L, c.R, c.E, c.M, c.C, c.T, c.cap, c.H, c.d, p.nb, p.A);
         }
         count_launches(1);
+        if (e != cudaSuccess) return dec_status(e);
     }
     return dec_status(cudaGetLastError());
 }
@@ -849,28 +897,19 @@ int mono_decode_attend(const mono_plan_t *plan, int t, void *cache, void *stream
         if (smc > 48 * 1024 && (e = cudaFuncSetAttribute(k_dec_attend_cl<__nv_bfloat16>,
                                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smc)))
             return dec_status(e);
-        cudaLaunchConfig_t lc = {};
-        lc.gridDim = dim3(c.H * kDecSplit, c.B);
-        lc.blockDim = dim3(256);
-        lc.dynamicSmemBytes = smc;
-        lc.stream = s;
-        cudaLaunchAttribute at[1];
-        at[0].id = cudaLaunchAttributeClusterDimension;
-        at[0].val.clusterDim.x = kDecSplit;
-        at[0].val.clusterDim.y = 1;
-        at[0].val.clusterDim.z = 1;
-        lc.attrs = at;
-        lc.numAttrs = 1;
-        if ((e = cudaLaunchKernelEx(&lc, k_dec_attend_cl<__nv_bfloat16>, (const __nv_bfloat16 *)P.Q,
-                                    (const __nv_bfloat16 *)P.K, (const __nv_bfloat16 *)P.V, (const int32_t *)P.sel,
-                                    (__nv_bfloat16 *)P.O, t, c.S, c.Bs, c.L, c.R, c.H, c.d, scale, ch)))
+        if ((e = dec_launch(k_dec_attend_cl<__nv_bfloat16>, dim3(c.H * kDecSplit, c.B), dim3(256), smc, s, kDecSplit,
+                            (const __nv_bfloat16 *)P.Q, (const __nv_bfloat16 *)P.K, (const __nv_bfloat16 *)P.V,
+                            (const int32_t *)P.sel, (__nv_bfloat16 *)P.O, t, c.S, c.Bs, c.L, c.R, c.H, c.d, scale,
+                            ch)))
             return dec_status(e);
     } else {
         const size_t sm = (size_t)4 * dec_chunk<float>(c.d) * c.d * 4;
         if ((e = cudaFuncSetAttribute(k_dec_attend<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm)))
             return dec_status(e);
-        k_dec_attend<float><<<g, 256, sm, s>>>((const float *)P.Q, (const float *)P.K, (const float *)P.V, P.sel,
-                                               (float *)P.O, t, c.S, c.Bs, c.L, c.R, c.H, c.d, scale);
+        if ((e = dec_launch(k_dec_attend<float>, g, dim3(256), sm, s, 1, (const float *)P.Q, (const float *)P.K,
+                            (const float *)P.V, (const int32_t *)P.sel, (float *)P.O, t, c.S, c.Bs, c.L, c.R, c.H,
+                            c.d, scale)))
+            return dec_status(e);
     }
     count_launches(1);
     return dec_status(cudaGetLastError());
@@ -892,14 +931,15 @@ int mono_decode_step(const mono_plan_t *plan, int t, const void *x_t, const void
     const DecPtrs P = dec_ptrs(dec_layout(p), cache);
     cudaStream_t s = (cudaStream_t)stream;
     const int grid = (c.W + 7) / 8;
+    cudaError_t e;
     if (c.dtype == MONO_BF16)
-        k_dec_out<__nv_bfloat16><<<grid, 256, 0, s>>>((const __nv_bfloat16 *)P.O, (const __nv_bfloat16 *)Wo,
-                                                      (__nv_bfloat16 *)delta_t, c.B, c.W, c.H * c.d);
+        e = dec_launch(k_dec_out<__nv_bfloat16>, dim3(grid), dim3(256), 0, s, 1, (const __nv_bfloat16 *)P.O,
+                       (const __nv_bfloat16 *)Wo, (__nv_bfloat16 *)delta_t, c.B, c.W, c.H * c.d);
     else
-        k_dec_out<float><<<grid, 256, 0, s>>>((const float *)P.O, (const float *)Wo, (float *)delta_t, c.B, c.W,
-                                              c.H * c.d);
+        e = dec_launch(k_dec_out<float>, dim3(grid), dim3(256), 0, s, 1, (const float *)P.O, (const float *)Wo,
+                       (float *)delta_t, c.B, c.W, c.H * c.d);
     count_launches(1);
-    return dec_status(cudaGetLastError());
+    return dec_status(e != cudaSuccess ? e : cudaGetLastError());
 }
 
 }  // extern "C"

@@ -184,6 +184,16 @@ __device__ __forceinline__ float ex2_fast(float x) {
 __device__ __forceinline__ void prefetch_l2(const void *p) { asm volatile("prefetch.global.L2 [%0];" ::"l"(p)); }
 __device__ __forceinline__ void prefetch_l1(const void *p) { asm volatile("prefetch.global.L1 [%0];" ::"l"(p)); }
 
+// --- programmatic dependent launch --------------------------------------------
+// grid_dep_wait: wait until the kernel this one was launched after (with the
+// programmatic-serialisation attribute) has completed and its writes are
+// visible; a no-op for a kernel launched without a programmatic predecessor.
+// grid_dep_launch: let the kernel launched after this one start its own
+// prologue (its blocks are scheduled once every block of this one has issued
+// it or exited).
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // --- TMA tile loads (no cluster multicast) --------------------------------
 // `map` is the address of a CUtensorMap in parameter, constant or global memory.
 __device__ __forceinline__ void tma_load_3d(void *dst, const void *map, int x, int y, int z, uint64_t *mbar) {
