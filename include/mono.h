@@ -378,8 +378,13 @@ int mono_decode_step(const mono_plan_t *plan, int t, const void *x_t, const void
  * differentiated: projection, RoPE, exact softmax over the selected token set
  * of each query (the blocks of sel that lie in [0, t/Bs - L] plus the local
  * tokens [max(0, t/Bs - L + 1) * Bs, t]), output projection.  Gradients are
- * fp32 and accumulated in fp32; dK and dV of a block sum the queries that
- * selected it in an unspecified order.  The backward workspace is a separate
+ * fp32 and accumulated in fp32, every sum in a fixed order (the queries that
+ * selected a block in ascending order, a query's remote blocks in slot order,
+ * split-K partial products in range order), so two calls on the same inputs
+ * give the same bits.  With bf16 storage, Bs = 64 and d = 64 with L <= 2 or
+ * d = 128 with L = 1, mono_backward runs the attention gradients on the tensor
+ * cores with every operand given to 16 significant bits (bf16 hi + lo terms).
+ * The backward workspace is a separate
  * caller-allocated buffer of mono_backward_workspace_bytes bytes (256-byte
  * aligned).
  * ------------------------------------------------------------------------ */

@@ -299,6 +299,7 @@ __global__ void __launch_bounds__(32) k_dec_route(const T *__restrict__ q, const
     __shared__ int s_top[kMaxT];
     __shared__ int s_head[kMaxT], s_cnt[kMaxT];
     __shared__ int s_cand[kMaxE];
+    __shared__ int s_walk[kMaxT][kMaxE];  // the first eligible entries of each probed list
     __shared__ float s_score[kMaxE];
     __shared__ __align__(16) float s_kb[kMaxE > 8 ? 8 : kMaxE][kMaxD + 4];  // candidate kbar rows, 8 at a time
     const int lane = threadIdx.x;
@@ -379,21 +380,28 @@ __global__ void __launch_bounds__(32) k_dec_route(const T *__restrict__ q, const
         s_head[lane] = ok ? P.head[bh * A + a] : -1;
     }
     __syncwarp();
-    // union of the probed lists in probe order, causal filter, E cap
-    int nc = 0;
-    if (lane == 0) {
-        for (int r = 0; r < TP && nc < E; ++r) {
-            if (s_cnt[r] <= 0) continue;
-            // at most cap kept entries; an id outside [0, nb) ends the walk
-            int steps = 0;
-            for (int j = s_head[r]; (unsigned)j < (unsigned)nb && nc < E && steps < cap;
-                 j = P.next[bh * nb + j], ++steps) {
-                if (j > lim) break;  // ascending ids: the rest are later still
-                s_cand[nc++] = j;
-            }
+    // union of the probed lists in probe order, causal filter, E cap: lane r walks list r (its first E eligible
+    // entries at most; at most cap kept entries; an id outside [0, nb) ends a walk), so the T chains of dependent
+    // loads run side by side; then the lists are concatenated in probe order up to E
+    int mine = 0;
+    if (lane < TP && s_cnt[lane] > 0) {
+        int steps = 0;
+        for (int j = s_head[lane]; (unsigned)j < (unsigned)nb && mine < E && steps < cap;
+             j = P.next[bh * nb + j], ++steps) {
+            if (j > lim) break;  // ascending ids: the rest are later still
+            s_walk[lane][mine++] = j;
         }
     }
-    nc = __shfl_sync(0xffffffffu, nc, 0);
+    int before_me = mine;  // inclusive prefix of the walked counts over the lanes in probe order
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, before_me, o);
+        if (lane >= o) before_me += y;
+    }
+    before_me -= mine;
+    for (int k = 0; k < mine && before_me + k < E; ++k) s_cand[before_me + k] = s_walk[lane][k];
+    int nc = __shfl_sync(0xffffffffu, before_me + mine, 31);
+    nc = nc < E ? nc : E;
     __syncwarp();
     // rerank: q . kbar_j, one candidate per lane, from rows staged 8 at a time
     for (int e0 = 0; e0 < nc; e0 += 8) {
