@@ -822,18 +822,18 @@ __device__ __forceinline__ unsigned survivors(const float (&s)[C], float delta) 
 // Taken codes are masked with -inf; the scores are finite for finite inputs.
 template <int C, int T0>
 __device__ __forceinline__ void top_codes(const float (&s)[C], float (&uv)[T0], int (&ui)[T0]) {
-    static_assert((C & (C - 1)) == 0 && C >= 2, "C a power of two");
-    float w[C];
-#pragma unroll
-    for (int c = 0; c < C; ++c) w[c] = s[c];
+    static_assert((C & (C - 1)) == 0 && C >= 2 && C <= 32, "C a power of two");
+    unsigned taken = 0;  // codes already ranked read as -inf (no copy of the scores: fewer registers)
 #pragma unroll
     for (int k = 0; k < T0; ++k) {
         float tv[C / 2];
         int ti[C / 2];
 #pragma unroll
         for (int p = 0; p < C / 2; ++p) {
-            const bool r = w[2 * p + 1] > w[2 * p];
-            tv[p] = r ? w[2 * p + 1] : w[2 * p];
+            const float a = (taken >> (2 * p)) & 1u ? -INFINITY : s[2 * p];
+            const float b = (taken >> (2 * p + 1)) & 1u ? -INFINITY : s[2 * p + 1];
+            const bool r = b > a;
+            tv[p] = r ? b : a;
             ti[p] = r ? 2 * p + 1 : 2 * p;
         }
 #pragma unroll
@@ -847,10 +847,7 @@ __device__ __forceinline__ void top_codes(const float (&s)[C], float (&uv)[T0], 
         }
         uv[k] = tv[0];
         ui[k] = ti[0];
-        if (k + 1 < T0) {
-#pragma unroll
-            for (int c = 0; c < C; ++c) w[c] = (c == ti[0]) ? -INFINITY : w[c];
-        }
+        taken |= 1u << ti[0];
     }
 }
 

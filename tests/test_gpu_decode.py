@@ -178,3 +178,47 @@ def test_decode_full_steps(dtype):
     assert_close(to_np(O).reshape(cfg.B, cfg.S, cfg.H, cfg.d).transpose(0, 2, 1, 3), ref_o, dtype, "decode attention")
     ref_delta = oracle.out_project(cfg, to_np(O).astype(np.float64), inp["Wo"])
     assert_close(to_np(torch.stack(deltas, dim=1)), ref_delta, dtype, "decode output projection")
+
+
+def test_decode_steps_in_a_cuda_graph_equal_eager_steps():
+    # The step's kernels start early under programmatic dependent launch and wait for their predecessor; captured
+    # into one CUDA graph and replayed, the steps give the same bits as eager calls: deltas, selections and the
+    # cache's tables.
+    cfg = small(dtype="bf16", B=2, S=192)
+    run = Run(cfg, seed=6)
+    plan, d = run.plan, run.dev
+    xs = [d["x"][:, t, :].contiguous() for t in range(cfg.S)]
+
+    def steps(graph):
+        cache = mono.decode_cache(plan)
+        mono.decode_prefill(plan, 0, d["codebooks"], cache)
+        sreg = mono.decode_region(plan, cache, "sel")
+        deltas = [torch.empty((cfg.B, cfg.W), dtype=plan.dtype, device="cuda") for _ in range(cfg.S)]
+        sels = [torch.empty_like(sreg) for _ in range(cfg.S)]
+
+        def body():
+            for t in range(cfg.S):
+                mono.decode_step(plan, t, xs[t], d["Wq"], d["Wk"], d["Wv"], d["Wo"], d["codebooks"], deltas[t],
+                                 cache)
+                sels[t].copy_(sreg)
+
+        torch.cuda.synchronize()
+        if graph:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                body()
+            g.replay()
+        else:
+            body()
+        torch.cuda.synchronize()
+        tables = [mono.decode_region(plan, cache, k).clone() for k in ("kbar", "addr", "count", "head", "next")]
+        return deltas, sels, tables
+
+    eager, captured = steps(False), steps(True)
+    for a, b in zip(eager[0], captured[0]):
+        assert torch.equal(a, b)
+    for a, b in zip(eager[1], captured[1]):
+        assert torch.equal(a, b)
+    for a, b in zip(eager[2], captured[2]):
+        assert torch.equal(a.view(torch.int32) if a.dtype == torch.float32 else a,
+                           b.view(torch.int32) if b.dtype == torch.float32 else b)
