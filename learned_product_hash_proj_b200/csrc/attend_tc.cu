@@ -44,11 +44,9 @@ constexpr int kMaxGroup = 256;               // (b, h) slices per launch group
 constexpr int kQTile = 1024;  // queries per CTA of the count and fill kernels
 
 // Programmatic dependent launch along the attention's kernels: each kernel
-// lets its successor's CTAs start at once, and each waits for its
-// predecessor's results only before reading them (without a programmatic
-// launch the wait returns at once).
-__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
-__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// lets its successor's CTAs start at once (tc::grid_dep_launch), and each
+// waits for its predecessor's results only before reading them
+// (tc::grid_dep_wait; without a programmatic launch the wait returns at once).
 
 // grid (ceil(S/kQTile), B*H), 256 threads, smem nb ints
 __global__ void __launch_bounds__(256) k_pair_count(const int32_t *__restrict__ sel, int32_t *__restrict__ cnt,
@@ -80,13 +78,13 @@ __global__ void __launch_bounds__(1024) k_pair_scan(const int32_t *__restrict__ 
                                                     int32_t *__restrict__ nwork, int nb, int wcap) {
     __shared__ int s_w[32], s_c[32];
     __shared__ int carry_p, carry_c;
-    pdl_trigger();
+    tc::grid_dep_launch();
     const long long bh = blockIdx.x;
     if (threadIdx.x == 0) {
         carry_p = 0;
         carry_c = 0;
     }
-    pdl_wait();  // the counts are complete
+    tc::grid_dep_wait();  // the counts are complete
     __syncthreads();
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int nw = blockDim.x >> 5;
@@ -137,10 +135,10 @@ __global__ void __launch_bounds__(256) k_pair_fill(const int32_t *__restrict__ s
                                                    int R, int nb, int Bs, int L) {
     extern __shared__ int s_h[];
     int *s_base = s_h + nb;
-    pdl_trigger();
+    tc::grid_dep_launch();
     const long long bh = blockIdx.y;
     for (int j = threadIdx.x; j < nb; j += blockDim.x) s_h[j] = 0;
-    pdl_wait();  // the bucket starts and cleared cursors
+    tc::grid_dep_wait();  // the bucket starts and cleared cursors
     __syncthreads();
     const int t0 = blockIdx.x * kQTile, t1 = min(S, t0 + kQTile);
     constexpr int kPer = (kQTile / 256) * kMaxR;   // pairs one thread can hold
@@ -247,7 +245,7 @@ __global__ void __launch_bounds__(256) k_remote_tc(const __grid_constant__ AttnM
     uint64_t *bar_kv = (uint64_t *)(smem + L::BAR_OFF);  // [2]: K/V of each stage landed
     uint64_t *mbar = bar_kv + 2;                          // MMA completion
     uint32_t *tmem_base = (uint32_t *)(mbar + 1);
-    pdl_trigger();  // the local kernel may start; it waits for the partials itself
+    tc::grid_dep_launch();  // the local kernel may start; it waits for the partials itself
     if (timed_out(counters)) return;
     if (tc::smem_u32(smem) & 1023) {  // uniform; TMA's 128-byte swizzle needs 1024-byte aligned tiles
         if (threadIdx.x == 0) record_error(counters, kDevErrSmemAlign);
@@ -257,7 +255,7 @@ __global__ void __launch_bounds__(256) k_remote_tc(const __grid_constant__ AttnM
     const int quarter = warp & 3, half = warp >> 2;
     const int row = quarter * 32 + lane;
 
-    pdl_wait();  // the work items and pair ids (pair kernels) are complete
+    tc::grid_dep_wait();  // the work items and pair ids (pair kernels) are complete
     if (tid == 0) {
         int acc = 0;
         for (int g = 0; g < ng; ++g) { s_pref[g] = acc; acc += nwork[bh0 + g]; }
@@ -958,7 +956,7 @@ __global__ void __launch_bounds__(320, 1) k_local_ws(const __grid_constant__ Att
             for (int r = 0; r < RMAX; ++r) selv[r] = (r < R && t < S) ? sel[((size_t)bh * S + t) * R + r] : -1;
         };
         if (g < n) load_sel(g);
-        pdl_wait();  // the remote partials (remote kernel) are complete
+        tc::grid_dep_wait();  // the remote partials (remote kernel) are complete
         for (int i = g; i < n && ok; i += 2) {
             const int u = i >> 1;
             const int f = tile_of(i);
@@ -1169,7 +1167,7 @@ static bool make_map_3d(CUtensorMap *map, const void *ptr, int D, int S, int BH,
 }
 
 // a kernel launched so that it may start while the kernel before it on the
-// stream still runs (it waits for its predecessor itself: pdl_wait)
+// stream still runs (it waits for its predecessor itself: tc::grid_dep_wait)
 template <typename... KArgs, typename... Args>
 static cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
                               Args... args) {

@@ -26,8 +26,6 @@ namespace mono {
 // and score the codebooks meanwhile), and the probe waits for the lists to be
 // complete and visible only before it reads them.  Without a programmatic
 // launch the wait returns at once.
-__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
-__device__ __forceinline__ void pdl_wait_primary() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 // ---------------------------------------------------------------------------
 // (A2, A3) block summary kbar = mean of the Bs post-RoPE keys, and the product
@@ -128,7 +126,7 @@ __global__ void __launch_bounds__(128, 6) k_summary_assign_w(const T *__restrict
                                                           int Bs, int M, int C, int H, int bpw) {
     constexpr int PER = D / 32;  // columns per lane
     static_assert(PER == 2 || PER == 4, "D = 64 or 128");
-    pdl_launch_dependents();  // the lists kernel may start; it waits for the addresses itself
+    tc::grid_dep_launch();  // the lists kernel may start; it waits for the addresses itself
     using RW = RowWord<T, PER>;
     using W = typename RW::W;
     constexpr int U = 16 / ((int)sizeof(W) / 4);  // rows per batch: 16 registers of words
@@ -247,8 +245,8 @@ __global__ void __launch_bounds__(1024) k_posting_dense(const int32_t *__restric
                                                         int32_t *__restrict__ saddr, int32_t *__restrict__ rank,
                                                         int32_t *__restrict__ overflow, int nb, int cap, int H, int A,
                                                         unsigned long long *__restrict__ stats) {
-    pdl_launch_dependents();
-    pdl_wait_primary();  // the addresses (summaries kernel) are complete
+    tc::grid_dep_launch();
+    tc::grid_dep_wait();  // the addresses (summaries kernel) are complete
     if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x < kCntStats) stats[threadIdx.x] = 0ull;  // the probe's
     __shared__ int s_cnt[kDenseA];
     __shared__ int s_part[32];
@@ -340,8 +338,8 @@ __global__ void __launch_bounds__(1024) k_posting_build(const int32_t *__restric
                                                         int32_t *__restrict__ saddr, int32_t *__restrict__ rank,
                                                         int32_t *__restrict__ overflow, int nb, int cap, int H,
                                                         unsigned long long *__restrict__ stats) {
-    pdl_launch_dependents();
-    pdl_wait_primary();  // the addresses (summaries kernel) are complete
+    tc::grid_dep_launch();
+    tc::grid_dep_wait();  // the addresses (summaries kernel) are complete
     if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x < kCntStats) stats[threadIdx.x] = 0ull;  // the probe's
     extern __shared__ int32_t s_addr[];
     __shared__ int s_ov[32];
@@ -416,8 +414,8 @@ __global__ void __launch_bounds__(1024) k_posting_redirect(const int32_t *__rest
                                                            int32_t *__restrict__ saddr, int32_t *__restrict__ rank,
                                                            int32_t *__restrict__ overflow, int nb, int cap, int H,
                                                            int A, unsigned long long *__restrict__ stats) {
-    pdl_launch_dependents();
-    pdl_wait_primary();  // the addresses (summaries kernel) are complete
+    tc::grid_dep_launch();
+    tc::grid_dep_wait();  // the addresses (summaries kernel) are complete
     if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x < kCntStats) stats[threadIdx.x] = 0ull;  // the probe's
     extern __shared__ uint32_t s_red[];
     const int nw = (A + 31) / 32;
@@ -546,8 +544,8 @@ __global__ void __launch_bounds__(128) k_probe_rerank(const T *__restrict__ Q, c
                                                       unsigned long long *__restrict__ counters,
                                                       int32_t *__restrict__ walk_log, int S, int H, int Bs,
                                                       int L, int R, int E, int M, int C, int Tp, int cap) {
-    pdl_wait_primary();  // the posting lists are complete
-    pdl_launch_dependents();
+    tc::grid_dep_wait();  // the posting lists are complete
+    tc::grid_dep_launch();
     extern __shared__ float smem[];
     const int nb = S / Bs;
     float *s_cb = smem;                                     // [M*C*dm] = C*D floats
@@ -1299,7 +1297,7 @@ __global__ void __launch_bounds__(probe_threads<C>(), probe_min_ctas<C>()) k_pro
     constexpr int QT = NT * NQ;
     static_assert(C <= 32 && TP <= C * C && R >= 1 && E >= 1 && QP % 16 == 0 && DM % 8 == 0, "shape");
     extern __shared__ __align__(16) float smem[];
-    pdl_launch_dependents();  // the attention's first kernel may start; it waits for sel itself
+    tc::grid_dep_launch();  // the attention's first kernel may start; it waits for sel itself
     const int nb = S / Bs;
     float *s_cbT = smem;                                 // [2][DM][C]: element i of codeword (m, c) at (m DM + i) C + c
     int2 *s_rng = (int2 *)(s_cbT + C * D);               // [A] positions [first, end) of each address's entries
@@ -1353,7 +1351,7 @@ __global__ void __launch_bounds__(probe_threads<C>(), probe_min_ctas<C>()) k_pro
     }
 
     // the posting lists: complete once the lists kernel is (programmatic launch)
-    pdl_wait_primary();
+    tc::grid_dep_wait();
     if ((nb & 3) == 0) {  // 16-byte aligned rows of the posting arrays
         for (int i = tid; i < nb / 4; i += blockDim.x) {
             tc::cp_async16(s_addr + 4 * i, post_addr + bh * nb + 4 * i, true);
@@ -1455,7 +1453,7 @@ __global__ void __launch_bounds__(128) k_probe_bf(const T *__restrict__ Q, const
     static_assert(M >= 2 && M * RB <= 16 && C <= 16 && C % 4 == 0 && DM % 8 == 0 && TP >= 1 && R >= 1, "shape");
     static_assert(M * rank_bits<C>() <= 16 && (C == 16 ? M <= 4 : true), "ranks and address in 16 bits each");
     extern __shared__ __align__(16) float smem[];
-    pdl_launch_dependents();
+    tc::grid_dep_launch();
     const int nb = S / Bs;
     float *s_cbT = smem;                                 // [M][DM][C]: element i of codeword (m, c) at (m DM + i) C + c
     uint8_t *s_q = (uint8_t *)(s_cbT + C * D);           // [128] query rows, pitch QP
@@ -1503,7 +1501,7 @@ __global__ void __launch_bounds__(128) k_probe_bf(const T *__restrict__ Q, const
         for (int c = 0; c < C; ++c) s[m][c] = sm[0][c];
     }
 
-    pdl_wait_primary();
+    tc::grid_dep_wait();
     for (int i = tid; i < nb; i += blockDim.x) {
         s_addr[i] = post_addr[bh * nb + i];
         s_ids[i] = post_ids[bh * nb + i];
@@ -1878,7 +1876,7 @@ cudaError_t launch_lists(const Plan &p, void *ws, cudaStream_t s) {
 }
 
 // a probe kernel, launched so that it may start while the lists kernel before
-// it on the stream still runs (it waits for the lists itself: pdl_wait_primary)
+// it on the stream still runs (it waits for the lists itself: tc::grid_dep_wait)
 template <typename... KArgs, typename... Args>
 static cudaError_t launch_after_lists(void (*kern)(KArgs...), dim3 grid, int threads, size_t smem, cudaStream_t s,
                                       Args... args) {
