@@ -141,27 +141,26 @@ __global__ void __launch_bounds__(256) k_pair_fill(const int32_t *__restrict__ s
     tc::grid_dep_wait();  // the bucket starts and cleared cursors
     __syncthreads();
     const int t0 = blockIdx.x * kQTile, t1 = min(S, t0 + kQTile);
-    constexpr int kPer = (kQTile / 256) * kMaxR;   // pairs one thread can hold
-    int my_j[kPer], my_rank[kPer], my_val[kPer];
-    int n = 0;
+    // two passes over the tile's selections: count per block, then place each pair at its block's global
+    // offset plus a shared cursor (no per-thread pair arrays, which would sit in local memory)
     for (int t = t0 + threadIdx.x; t < t1; t += blockDim.x)
         for (int r = 0; r < R; ++r) {
             const int j = sel[((size_t)bh * S + t) * R + r];
-            if (!sel_valid(j, t, Bs, L)) continue;
-            my_j[n] = j;
-            my_rank[n] = atomicAdd(&s_h[j], 1);
-            my_val[n] = t * R + r;
-            ++n;
+            if (sel_valid(j, t, Bs, L)) atomicAdd(&s_h[j], 1);
         }
     __syncthreads();
-    for (int j = threadIdx.x; j < nb; j += blockDim.x)
-        if (s_h[j]) s_base[j] = atomicAdd(&fill[bh * nb + j], s_h[j]);
+    for (int j = threadIdx.x; j < nb; j += blockDim.x) {
+        const int c = s_h[j];
+        if (c) s_base[j] = start[bh * nb + j] + atomicAdd(&fill[bh * nb + j], c);
+        s_h[j] = 0;
+    }
     __syncthreads();
     int32_t *seg = pairs + (size_t)bh * S * R;
-    for (int k = 0; k < n; ++k) {
-        const int j = my_j[k];
-        seg[start[bh * nb + j] + s_base[j] + my_rank[k]] = my_val[k];
-    }
+    for (int t = t0 + threadIdx.x; t < t1; t += blockDim.x)
+        for (int r = 0; r < R; ++r) {
+            const int j = sel[((size_t)bh * S + t) * R + r];
+            if (sel_valid(j, t, Bs, L)) seg[s_base[j] + atomicAdd(&s_h[j], 1)] = t * R + r;
+        }
 }
 
 // ---------------------------------------------------------------------------
