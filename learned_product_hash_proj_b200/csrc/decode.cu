@@ -286,9 +286,12 @@ __device__ __forceinline__ bool before(float v1, int a1, float v2, int a2) {
 // ---------------------------------------------------------------------------
 // routing of the step's query, one warp per (b, h); grid (H, B), 32 threads,
 // dynamic shared memory M C (d/M + 1) floats (the head's codewords, one
-// padding float per row so that the 32 lanes' chains read 32 banks)
+// padding float per row so that the 32 lanes' chains read 32 banks).  TPM >=
+// T is the length of each lane's sorted list of its best addresses, fixed at
+// compile time so that the list stays in registers (a lane's first T entries
+// are its top T; the entries after them are never reached by the merge).
 // ---------------------------------------------------------------------------
-template <typename T>
+template <typename T, int TPM>
 __global__ void __launch_bounds__(32) k_dec_route(const T *__restrict__ q, const float *__restrict__ cb,
                                                   const int32_t *__restrict__ forced, DecPtrs P, int t, int Bs, int L,
                                                   int R, int E, int M, int C, int TP, int cap, int H, int d, int nb,
@@ -331,10 +334,11 @@ __global__ void __launch_bounds__(32) k_dec_route(const T *__restrict__ q, const
     }
     __syncwarp();
     // every address scored (subspace 0 most significant, summed in ascending
-    // subspace order); each lane keeps its top TP by (score desc, address asc)
-    float lv[kMaxT];
-    int la[kMaxT];
-    for (int k = 0; k < TP; ++k) { lv[k] = -INFINITY; la[k] = 0x7fffffff; }
+    // subspace order); each lane keeps its top TPM by (score desc, address asc)
+    float lv[TPM];
+    int la[TPM];
+#pragma unroll
+    for (int k = 0; k < TPM; ++k) { lv[k] = -INFINITY; la[k] = 0x7fffffff; }
     const int A32 = (int)A;  // <= 4096 on this path
     for (int a32 = lane; a32 < A32; a32 += 32) {
         int rest = a32, radix = A32 / C;
@@ -345,21 +349,26 @@ __global__ void __launch_bounds__(32) k_dec_route(const T *__restrict__ q, const
             radix /= C;
             v = m == 0 ? s_sc[cm] : __fadd_rn(v, s_sc[m * C + cm]);
         }
-        if (!before(v, a32, lv[TP - 1], la[TP - 1])) continue;
-        int k = TP - 1;
-        while (k > 0 && before(v, a32, lv[k - 1], la[k - 1])) {
-            lv[k] = lv[k - 1];
-            la[k] = la[k - 1];
-            --k;
+        if (!before(v, a32, lv[TPM - 1], la[TPM - 1])) continue;
+        // insertion: the new entry moves down past every entry it precedes
+        float cv = v;
+        int ca = a32;
+#pragma unroll
+        for (int k = 0; k < TPM; ++k) {
+            if (before(cv, ca, lv[k], la[k])) {
+                const float tv = lv[k];
+                const int ta = la[k];
+                lv[k] = cv;
+                la[k] = ca;
+                cv = tv;
+                ca = ta;
+            }
         }
-        lv[k] = v;
-        la[k] = a32;
     }
-    // merge: TP rounds of a warp argmax over the lanes' heads
-    int ptr = 0;
+    // merge: TP rounds of a warp argmax over the lanes' heads; the winning lane drops its head
     for (int r = 0; r < TP; ++r) {
-        float bv = ptr < TP ? lv[ptr] : -INFINITY;
-        int ba = ptr < TP ? la[ptr] : 0x7fffffff;
+        float bv = lv[0];
+        int ba = la[0];
         int bl = lane;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
@@ -369,7 +378,15 @@ __global__ void __launch_bounds__(32) k_dec_route(const T *__restrict__ q, const
             if (before(ov, oa, bv, ba)) { bv = ov; ba = oa; bl = ol; }
         }
         if (lane == 0) s_top[r] = ba;
-        if (lane == bl) ++ptr;
+        if (lane == bl) {
+#pragma unroll
+            for (int k = 0; k + 1 < TPM; ++k) {
+                lv[k] = lv[k + 1];
+                la[k] = la[k + 1];
+            }
+            lv[TPM - 1] = -INFINITY;
+            la[TPM - 1] = 0x7fffffff;
+        }
     }
     __syncwarp();
     // the probed lists' heads and counts, fetched at once
@@ -416,6 +433,7 @@ __global__ void __launch_bounds__(32) k_dec_route(const T *__restrict__ q, const
         if (lane < ne) {
             // eight runs of d/8 elements as fma chains, added as a balanced tree (the batch rerank's order)
             float run[8];
+#pragma unroll
             for (int l = 0; l < 8; ++l) {
                 float a = 0.0f;
                 for (int i = l * d / 8; i < (l + 1) * d / 8; ++i) a = __fmaf_rn(s_q[i], s_kb[lane][i], a);
@@ -430,12 +448,12 @@ __global__ void __launch_bounds__(32) k_dec_route(const T *__restrict__ q, const
         // top R by (score desc, id asc), in rank order
         int ra[kMaxR];
         int nr = 0;
-        bool used[kMaxE] = {};
+        unsigned used = 0;  // candidates taken (E <= 32)
         for (; nr < R && nr < nc; ++nr) {
             int bi = -1;
             for (int e = 0; e < nc; ++e)
-                if (!used[e] && (bi < 0 || before(s_score[e], s_cand[e], s_score[bi], s_cand[bi]))) bi = e;
-            used[bi] = true;
+                if (!((used >> e) & 1u) && (bi < 0 || before(s_score[e], s_cand[e], s_score[bi], s_cand[bi]))) bi = e;
+            used |= 1u << bi;
             ra[nr] = s_cand[bi];
         }
         if (forced) {
@@ -866,19 +884,22 @@ int mono_decode_route(const mono_plan_t *plan, int t, const float *codebooks, co
     }
     if (c.R > 0) {
         const size_t sm = (size_t)c.M * c.C * (c.d / c.M + 1) * 4;
-        if (bf) {
-            if (sm > 48 * 1024 && (e = cudaFuncSetAttribute(k_dec_route<__nv_bfloat16>,
-                                                            cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm)))
-                return dec_status(e);
-            e = dec_launch(k_dec_route<__nv_bfloat16>, g, dim3(32), sm, s, 1, (const __nv_bfloat16 *)P.Q, codebooks,
-                           forced_t, P, t, c.Bs, c.L, c.R, c.E, c.M, c.C, c.T, c.cap, c.H, c.d, p.nb, p.A);
-        } else {
+        static_assert(kMaxT <= 32, "per-lane address lists of at most 32 entries");
+        auto route = [&](auto kern, const auto *q) -> cudaError_t {
+            cudaError_t err;
             if (sm > 48 * 1024 &&
-                (e = cudaFuncSetAttribute(k_dec_route<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm)))
-                return dec_status(e);
-            e = dec_launch(k_dec_route<float>, g, dim3(32), sm, s, 1, (const float *)P.Q, codebooks, forced_t, P, t,
-                           c.Bs, c.L, c.R, c.E, c.M, c.C, c.T, c.cap, c.H, c.d, p.nb, p.A);
-        }
+                (err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm)) != cudaSuccess)
+                return err;
+            return dec_launch(kern, g, dim3(32), sm, s, 1, q, codebooks, forced_t, P, t, c.Bs, c.L, c.R, c.E, c.M,
+                              c.C, c.T, c.cap, c.H, c.d, p.nb, p.A);
+        };
+#define MONO_DEC_ROUTE(TT)                                                                                       \
+    (c.T <= 4 ? route(k_dec_route<TT, 4>, (const TT *)P.Q)                                                       \
+              : c.T <= 8 ? route(k_dec_route<TT, 8>, (const TT *)P.Q)                                            \
+                         : c.T <= 16 ? route(k_dec_route<TT, 16>, (const TT *)P.Q)                               \
+                                     : route(k_dec_route<TT, 32>, (const TT *)P.Q))
+        e = bf ? MONO_DEC_ROUTE(__nv_bfloat16) : MONO_DEC_ROUTE(float);
+#undef MONO_DEC_ROUTE
         count_launches(1);
         if (e != cudaSuccess) return dec_status(e);
     }
