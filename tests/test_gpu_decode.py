@@ -43,6 +43,9 @@ CASES = {
     "bf16": dict(dtype="bf16"),
     "d128_bf16": dict(d=128, H=2, S=256, Bs=64, C=16, cap=4, dtype="bf16"),
     "M4_L1_R4": dict(M=4, C=4, T=8, E=8, R=4, L=1, cap=2),
+    # the route's per-lane address lists at their two longest compile-time lengths (16 and 32)
+    "T16": dict(T=16, E=8, R=4),
+    "M4_C8_T32": dict(M=4, C=8, T=32, E=16, R=4, cap=2),
     "local_only": dict(R=0),
     "zero_ties": dict(x="zeros"),
 }
