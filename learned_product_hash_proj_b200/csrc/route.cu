@@ -1307,10 +1307,14 @@ __global__ void __launch_bounds__(probe_threads<C>(), probe_min_ctas<C>()) k_pro
     float *s_score = (float *)(s_nc + QT);               // [QT][E] their rerank scores
     int32_t *s_addr = (int32_t *)(s_score + QT * E);     // [nb]
     int32_t *s_ids = s_addr + nb;                        // [nb]
-    const int h = blockIdx.y, b = blockIdx.z;
+    // CTAs in dispatch order take the query tiles latest first, every (b, h) of a tile in turn: later queries have
+    // more causal candidates to rerank, so the launch ends on its lightest tiles
+    const int nbh = gridDim.y * gridDim.z;
+    const int lin = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z);
+    const int h = (lin % nbh) % gridDim.y, b = (lin % nbh) / gridDim.y;
     const size_t bh = (size_t)b * H + h;
     const int tid = threadIdx.x;
-    const int t_lo = blockIdx.x * QT;
+    const int t_lo = (gridDim.x - 1 - lin / nbh) * QT;
     {
         constexpr int CH = D * (int)sizeof(T) / 16;  // 16-byte chunks per query row
         const uint8_t *src = (const uint8_t *)(Q + (bh * S + t_lo) * D);
